@@ -1,0 +1,529 @@
+"""HQMQ KV-cache encode/decode throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl hqmq|reference]
+
+One step = one pass of the whole hot path over the whole synthetic KV cache of
+the workload, layer by layer: codebooks for every (layer, role, head), then
+per (layer, role) call Med3x (median + ordered outlier list, when the workload
+has it), encode, and decode back to bf16.  Inputs are resident in HBM before
+the timed region (the default workload's cache is 42.95 GB, far above L2).
+
+Prints one JSON line.  `value` = bf16 KV bytes taken through encode and
+decode per second, summed over ranks (every rank codes its own cache: weak
+scaling, no collective on the data path).  `e2e` is the same metric through
+the C ABI from pinned host buffers (input H2D and compressed cache D2H inside
+the timed region).  `--impl reference` times the CPU oracle (the plain
+reference implementation of the method) on a bounded sample of the same
+workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "HQMQ encode/decode GB/s (bf16 KV) and % of B200 HBM roofline, S=8/32"
+DEFAULT_WORKLOAD = "llama3_70b_128k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
+ALU_LANES = 148 * 128          # FP32 lanes of a B200 (148 SMs x 128)
+KERNELS_MED3 = 9               # 3 histogram + 3 select + count + scan + write
+OUTLIER_CAP_FRAC = 0.15        # list capacity: 15% of the chunks of a call
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    import torch
+    if n_gpus <= 1 or "RANK" not in os.environ:
+        return 0, 1, None
+    import torch.distributed as dist
+    import datetime
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                            device_id=torch.device("cuda", local))
+    return dist.get_rank(), dist.get_world_size(), dist
+
+
+def max_over_ranks(v, dist, device):
+    """Max of a float over ranks (identity without a process group)."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = "/tmp/hqmq_clocks_%d.csv" % os.getpid()
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the path
+class Cache:
+    """Device-resident synthetic cache of one workload and its code buffers."""
+
+    def __init__(self, w, rank, device):
+        import torch
+        from kv_cache_quantization_hqmq_b200 import hqmq
+        from kv_cache_quantization_hqmq_b200 import workloads as W
+        self.w = w
+        B, H, T, D = w.call_shape
+        self.shape = (B, H, T, D)
+        self.n_chunks = B * H * T * D // 4
+        self.n_words = hqmq.hqmq_index_words(B, H, T, D, w.S)
+        # each rank codes its own cache (different input seed)
+        wr = w.with_(input_seed=w.input_seed + 1000 * rank)
+        self.x = torch.empty((w.layers, 2) + self.shape, dtype=w.torch_dtype, device=device)
+        for l in range(w.layers):
+            for r in range(2):
+                self.x[l, r].copy_(W.make_call_input(wr, l, r, device=device))
+        self.codebook = torch.empty(w.n_groups * w.S * 4, dtype=torch.float32, device=device)
+        self.words = torch.empty((w.layers, 2, self.n_words), dtype=torch.int32, device=device)
+        self.radius = torch.empty((w.layers, 2, self.n_chunks), dtype=torch.int16, device=device)
+        self.y = torch.empty(self.shape, dtype=torch.bfloat16, device=device)
+        self.status = hqmq.new_status(device)
+        self.gran = hqmq.HQMQ_GRAN_CHUNK
+        if w.med3:
+            self.cap = int(OUTLIER_CAP_FRAC * self.n_chunks)
+            self.rmed = torch.empty((w.layers, 2, H), dtype=torch.float32, device=device)
+            self.thr = torch.empty((w.layers, 2, H), dtype=torch.float32, device=device)
+            self.out_idx = torch.empty((w.layers, 2, self.cap), dtype=torch.int32, device=device)
+            self.out_val = torch.empty((w.layers, 2, self.cap * 4), dtype=torch.int16, device=device)
+            self.slab_off = torch.empty((w.layers, 2, B * H + 1), dtype=torch.int32, device=device)
+            self.ws = torch.empty(hqmq.hqmq_outlier_workspace_size(B, H, T, D, self.gran),
+                                  dtype=torch.uint8, device=device)
+
+    def kernels_per_step(self):
+        per_call = 2 + (KERNELS_MED3 if self.w.med3 else 0)
+        return 1 + self.w.n_calls * per_call
+
+    def step(self, timers=None, x_override=None):
+        """One pass over the cache.  timers: dict name -> list of (start, end)
+        CUDA events recorded around the launches of that kernel family."""
+        import torch
+        from kv_cache_quantization_hqmq_b200 import hqmq
+        w = self.w
+        H = w.heads
+        stream = torch.cuda.current_stream()
+
+        def ev():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            return e
+
+        hqmq.hqmq_make_codebook(w.codebook_seed, w.S, w.n_groups, 0, self.codebook, stream)
+        for l in range(w.layers):
+            for r in range(2):
+                x = self.x[l, r] if x_override is None else x_override(l, r)
+                g0 = (l * 2 + r) * H
+                cb = self.codebook[g0 * w.S * 4:(g0 + H) * w.S * 4]
+                thr = None
+                if w.med3:
+                    t0 = ev() if timers is not None else None
+                    hqmq.hqmq_outlier_extract(x, w.C, self.gran, self.rmed[l, r], self.thr[l, r],
+                                              self.out_idx[l, r], self.out_val[l, r],
+                                              self.slab_off[l, r], self.cap, self.ws, self.status,
+                                              stream)
+                    if timers is not None:
+                        timers["med3"].append((t0, ev()))
+                    thr = self.thr[l, r]
+                t0 = ev() if timers is not None else None
+                hqmq.hqmq_encode(x, cb, w.S, thr, self.gran, self.words[l, r], self.radius[l, r],
+                                 self.status, stream)
+                t1 = ev() if timers is not None else None
+                if w.med3:
+                    hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S,
+                                     self.out_idx[l, r], self.out_val[l, r], self.slab_off[l, r],
+                                     self.cap, self.gran, self.y, self.status, stream)
+                else:
+                    hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S, None, None,
+                                     None, 0, self.gran, self.y, self.status, stream)
+                if timers is not None:
+                    t2 = ev()
+                    timers["encode"].append((t0, t1))
+                    timers["decode"].append((t1, t2))
+
+
+def algorithmic_bytes(w, n_outliers_per_call):
+    """Bytes the method must move per call (Measurement)."""
+    B, H, T, D = w.call_shape
+    n_chunks = B * H * T * D // 4
+    x_bytes = B * H * T * D * w.elem_bytes
+    b = math.ceil(math.log2(24 * w.S))
+    code_bytes = n_chunks * (b / 8.0 + 2.0)
+    out_bytes = n_outliers_per_call * 12.0 if w.med3 else 0.0
+    return {
+        # Med3x: read the input once for the median and once for the list
+        "med3": 2 * x_bytes + out_bytes if w.med3 else 0.0,
+        "encode": x_bytes + code_bytes,
+        "decode": code_bytes + out_bytes + B * H * T * D * 2,
+    }
+
+
+def alu_ops_per_chunk(S):
+    """Lane operations of the S-codeword search per chunk:
+    per secondary codeword one quaternion product (16 FMA), the 2T score
+    (3 max + 3 add + 1 add + 1 max) and the argmax update (1 compare +
+    2 select) = 27; per chunk ~60 more (load, norm, closed-form p, radius,
+    packing)."""
+    return 27 * S + 60
+
+
+def elapsed_ms(pairs):
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def run_hqmq(args):
+    import torch
+    rank, world, dist = dist_setup(args.gpus)
+    device = torch.device("cuda", torch.cuda.current_device())
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    from kv_cache_quantization_hqmq_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    peaks = load_peaks()
+
+    # CPU baseline first, in spawned processes (no fork after CUDA init)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    cache = Cache(w, rank, device)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        cache.step()
+    torch.cuda.synchronize()
+    st = hqmq.read_status(cache.status)
+
+    timers = {"med3": [], "encode": [], "decode": []}
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(dist)
+    torch.cuda.synchronize()
+    clocks.start()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(args.steps):
+        cache.step(timers)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(dist)
+    clk = clocks.stop()
+    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_total, dist, device)
+    ms_step = ms_total / args.steps
+
+    n_out = st["n_outliers"] / max(1, args.warmup) / w.n_calls if w.med3 else 0.0
+    ab = algorithmic_bytes(w, n_out)
+    kern = {}
+    for name in ("med3", "encode", "decode"):
+        if not timers[name]:
+            continue
+        t = statistics.mean(elapsed_ms(timers[name]))
+        gbs = ab[name] / (t * 1e-3) / 1e9
+        kern[name] = {"ms_per_call": round(t, 4), "calls_per_step": w.n_calls,
+                      "algorithmic_bytes_per_call": int(ab[name]),
+                      "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+                      "bf16_gbs": round(w.call_elems * w.elem_bytes / (t * 1e-3) / 1e9, 1)}
+    B, H, T, D = w.call_shape
+    n_chunks = B * H * T * D // 4
+    t_enc = kern["encode"]["ms_per_call"] * 1e-3
+    alu_peak = ALU_LANES * peaks["sm_max_mhz"] * 1e6
+    alu_achieved = alu_ops_per_chunk(w.S) * n_chunks / t_enc
+    kern["encode"]["alu_ops_per_chunk"] = alu_ops_per_chunk(w.S)
+    kern["encode"]["alu_frac"] = round(alu_achieved / alu_peak, 4)
+
+    enc_alu_bound = kern["encode"]["alu_frac"] > kern["encode"]["hbm_frac"]
+    if enc_alu_bound:
+        roof = {"kernel": "k_encode", "bound": "alu", "achieved": round(alu_achieved / 1e12, 3),
+                "peak": round(alu_peak / 1e12, 3), "unit": "T lane-ops/s",
+                "frac": round(alu_achieved / alu_peak, 4), "traffic": None,
+                "peak_source": "148 SMs x 128 FP32 lanes x %s max SM MHz" % peaks["sm_max_mhz"]}
+    else:
+        roof = {"kernel": "k_encode", "bound": "hbm", "achieved": kern["encode"]["hbm_gbs"],
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kern["encode"]["hbm_frac"],
+                "traffic": None, "peak_source": peaks["source"]}
+
+    cache_bytes = w.cache_bytes
+    value = world * cache_bytes / (ms_step * 1e-3) / 1e9
+    b = math.ceil(math.log2(24 * w.S))
+    bits = (b + 16) / 4.0
+    n_elems_call = w.call_elems
+    out_bits = (n_out * (64 + 32) / n_elems_call) if w.med3 else 0.0
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(cache, args, dist, device)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.layers, "kv_heads": H, "head_dim": D,
+                   "batch": B, "tokens": T, "S": w.S, "med3": ("chunk, C=%g" % w.C) if w.med3 else "off",
+                   "input": w.dtype, "cache_gb": round(cache_bytes / 1e9, 2),
+                   "l2": "inputs larger than L2 (%.0f MB per call, %.1f GB per step)"
+                         % (w.call_elems * w.elem_bytes / 1e6, cache_bytes / 1e9),
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "value_is": "bf16 KV bytes through Med3x+encode+decode per second"},
+        "kernels": kern,
+        "roofline": roof,
+        "bits_per_element": {"ours_codes": bits, "ours_outliers": round(out_bits, 4),
+                             "pages_S8": 3.79, "pages_S32": 5},
+        "outlier_fraction": round(n_out / n_chunks, 5) if w.med3 else 0.0,
+        "status_flags": st["flags"],
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": cache.kernels_per_step() * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_e2e(cache, args, dist, device):
+    """Same step through the C ABI with the input in pinned host memory: every
+    call's input is copied H2D, and the compressed cache (index words, radii,
+    outlier list) D2H, inside the timed region."""
+    import torch
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    w = cache.w
+    call_bytes = w.call_elems * w.elem_bytes
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = 16 << 30
+    # distinct pinned host inputs (up to all calls, within half the free RAM)
+    n_host = int(max(2, min(w.n_calls, (avail // 2) // (call_bytes + 1))))
+    host_x = [torch.empty(cache.shape, dtype=w.torch_dtype, pin_memory=True) for _ in range(n_host)]
+    for i, hx in enumerate(host_x):
+        hx.copy_(cache.x[i // 2 % w.layers, i % 2])
+    host_words = torch.empty(cache.n_words, dtype=torch.int32, pin_memory=True)
+    host_rad = torch.empty(cache.n_chunks, dtype=torch.int16, pin_memory=True)
+    host_oi = host_ov = None
+    if w.med3:
+        host_oi = torch.empty(cache.cap, dtype=torch.int32, pin_memory=True)
+        host_ov = torch.empty(cache.cap * 4, dtype=torch.int16, pin_memory=True)
+    xbuf = torch.empty(cache.shape, dtype=w.torch_dtype, device=device)
+    h2d = d2h = 0
+
+    def x_of(l, r):
+        nonlocal h2d
+        xbuf.copy_(host_x[(l * 2 + r) % n_host], non_blocking=True)
+        h2d += call_bytes
+        return xbuf
+
+    def one_step():
+        nonlocal d2h
+        cache.step(x_override=x_of)
+        # compressed cache back to the host (per call, last call's buffers
+        # stand for all: same sizes)
+        for l in range(w.layers):
+            for r in range(2):
+                host_words.copy_(cache.words[l, r], non_blocking=True)
+                host_rad.copy_(cache.radius[l, r], non_blocking=True)
+                d2h += cache.n_words * 4 + cache.n_chunks * 2
+                if w.med3:
+                    host_oi.copy_(cache.out_idx[l, r], non_blocking=True)
+                    host_ov.copy_(cache.out_val[l, r], non_blocking=True)
+                    d2h += cache.cap * 4 + cache.cap * 8
+
+    steps = max(1, min(args.steps, 3))
+    one_step()
+    torch.cuda.synchronize()
+    h2d = d2h = 0
+    barrier(dist)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        one_step()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(dist)
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, device) / steps
+    world = 1 if dist is None else dist.get_world_size()
+    return {"value": round(world * w.cache_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 2), "steps": steps,
+            "h2d_bytes_per_step": h2d // steps, "d2h_bytes_per_step": d2h // steps,
+            "host_inputs": "%d distinct pinned call inputs reused round-robin" % n_host}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def _oracle_sample_job(args):
+    """Runs in a spawned process: the oracle's Med3x + encode + decode of one
+    (head) slab sample of one call."""
+    name, layer, role, tokens, head = args
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    from kv_cache_quantization_hqmq_b200 import workloads as W
+    from oracle import hqmq_oracle as oracle
+    w = W.WORKLOADS[name]
+    x = W.as_numpy_bits(W.make_call_input(w, layer, role, tokens=tokens))
+    x = np.ascontiguousarray(x[:, head:head + 1])
+    B, H, T, D = x.shape
+    g0 = W.group0(layer, role, w.heads) + head
+    t0 = time.perf_counter()
+    cb = oracle.make_codebook(w.codebook_seed, w.S, 1, g0)
+    thr = None
+    oi = ov = None
+    if w.med3:
+        rmed, thr = oracle.med3_threshold(x, w.C, 0)
+        oi, ov, so, n, _ = oracle.extract(x, thr)
+    words, rad, best, second, _ = oracle.encode(x, cb, w.S, thr=thr)
+    oracle.decode(words, rad, cb, w.S, B, H, T, D, out_idx=oi, out_val=ov)
+    return time.perf_counter() - t0, x.size * w.elem_bytes
+
+
+def cpu_baseline(w, seconds_target=20.0):
+    """The oracle, as it stands, on a bounded sample: the first `tokens`
+    tokens of single-head slabs of layer 0, K and V, in parallel over the host
+    cores (one spawned process per slab)."""
+    import multiprocessing as mp
+    cores = os.cpu_count() or 1
+    # calibrate: brute force costs ~24 S codewords per chunk
+    probe_tokens = 256
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(1) as pool:
+        t, nbytes = pool.map(_oracle_sample_job, [(w.name, 0, 0, probe_tokens, 0)])[0]
+    per_token = t / probe_tokens
+    n_jobs = min(cores, 2 * w.heads)
+    tokens = int(max(probe_tokens, min(w.tokens, seconds_target / max(per_token, 1e-9))))
+    tokens = max(32, (tokens // 32) * 32)
+    jobs = [(w.name, 0, j % 2, tokens, (j // 2) % w.heads) for j in range(n_jobs)]
+    t0 = time.perf_counter()
+    with ctx.Pool(n_jobs) as pool:
+        res = pool.map(_oracle_sample_job, jobs)
+    wall = time.perf_counter() - t0
+    total_bytes = sum(r[1] for r in res)
+    busy = max(r[0] for r in res)
+    return {"value": round(total_bytes / busy / 1e9, 6), "unit": "GB/s", "cores": n_jobs,
+            "kind": "oracle",
+            "sample": "%d single-head slabs (layer 0, K and V) x %d tokens x batch %d of %s; "
+                      "Med3x + encode + decode by the plain C oracle, one process per slab; "
+                      "wall %.1f s" % (n_jobs, tokens, w.batch, w.name, wall)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from kv_cache_quantization_hqmq_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    times = []
+    cpu = None
+    per_step = max(3.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        cpu = cpu_baseline(w, per_step)
+        if i >= args.warmup:
+            times.append(cpu["value"])
+    value = statistics.mean(times)
+    cpu["value"] = round(value, 6)
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "GB/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "S": w.S,
+                       "med3": ("chunk, C=%g" % w.C) if w.med3 else "off"},
+            "impl": "reference", "cpu_baseline": cpu,
+            "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="hqmq", choices=["hqmq", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_hqmq(args)
+
+
+if __name__ == "__main__":
+    main()

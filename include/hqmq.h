@@ -1,0 +1,186 @@
+/*
+ * hqmq.h -- C ABI of libhqmq, the B200 (sm_100a) implementation of the
+ * HQMQ (Hurwitz Quaternion Multiplicative Quantization) KV-cache codec.
+ *
+ * What is computed (sources named by page and section):
+ *   - every 4 consecutive elements of a K or V head vector form a quaternion
+ *     x = (w, i, j, k) (arXiv 2605.27646 abstract, paperdance.org/p/2605.27646;
+ *     gist.science/nl/paper/2605.27646, Technische Samenvatting, Methodologie);
+ *   - x is split into its norm r = |x| and direction u = x / r (same section);
+ *   - u is snapped to the codeword q_p q_s maximising <u, q_p q_s>, where q_p
+ *     runs over the 24-element Hurwitz group 2T and q_s over S seeded random
+ *     unit quaternions of this (layer, head, role): 24 S codewords from S
+ *     stored quaternions (gist.science/nl, Technische Samenvatting, section 1
+ *     "Multiplicatieve Samenstelling van Codeboeken"; abstract);
+ *   - optionally first, Med3x: the median chunk norm r_med of the current
+ *     batch is taken per head; chunks with r > C r_med (C = 3) are kept in
+ *     fp16 in a side list and the rest is quantised (gist.science/nl,
+ *     Technische Samenvatting, section 3 "Mediane-Multiplier
+ *     Uitbijterextractie"; gist.science/pt, Resumo Tecnico, section 3);
+ *   - decode rebuilds r * (q_p q_s) and restores the outliers (the fused
+ *     decoder of gist.science/nl, Technische Samenvatting, "Memory en
+ *     Latentie", reads the same stored pair).
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - one call = one (layer, role) tensor x[B][H][T][D], row-major, D % 4 == 0
+ *     and (T*D/4) % 32 == 0.  Chunk j covers elements 4j .. 4j+3; its head is
+ *     (j / (T*D/4)) % H; a "slab" is one (b, h) pair, slab index b*H + h.
+ *   - 2T enumeration p in [0,24): p = 2a + sg for the units +-1,+-i,+-j,+-k
+ *     (a = axis w,i,j,k; sg = 1 for the minus sign); p = 8 + m for
+ *     1/2((-1)^m0, (-1)^m1, (-1)^m2, (-1)^m3), m_c = bit c of m.
+ *   - codeword index s*24 + p; among equal fp32 scores the lowest index wins.
+ *   - index width b = ceil(log2(24 S)) bits; per group of 32 consecutive
+ *     chunks, b uint32 words; bit i of chunk k's index is bit k*b+i of the
+ *     group's b-word stream (LSB first).
+ *   - radius: fp16, round-to-nearest-even, saturated at 65504.
+ *   - codebook group numbering g = (layer*2 + role)*H + head (role 0 = K,
+ *     1 = V); a call's H codebooks are therefore contiguous.
+ *
+ * Ownership and execution: the caller allocates every buffer; all pointers
+ * are device pointers unless stated; nothing is allocated, freed or kept
+ * between calls.  Every compute entry point only enqueues work on `stream`
+ * (a cudaStream_t passed as void*; NULL = the legacy default stream) and
+ * returns without synchronising.  Argument errors are returned synchronously
+ * and nothing is enqueued.  Data-dependent conditions (outlier capacity
+ * overflow, fp16 saturation, non-finite input, corrupt indices) never trap:
+ * they are recorded in the device-resident hqmq_status (if non-NULL), whose
+ * counters the calls add to; the caller zeroes it.
+ */
+#ifndef HQMQ_H
+#define HQMQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HQMQ_API __attribute__((visibility("default")))
+#else
+#define HQMQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define HQMQ_OK 0
+#define HQMQ_ERR_ARG 1        /* a size, enum or pointer argument is invalid   */
+#define HQMQ_ERR_ALIGN 2      /* a pointer misses its stated alignment         */
+#define HQMQ_ERR_CUDA 3       /* a CUDA launch or runtime call failed          */
+#define HQMQ_ERR_WORKSPACE 4  /* workspace smaller than hqmq_outlier_workspace_size */
+
+/* Element types of x / y. */
+#define HQMQ_BF16 0
+#define HQMQ_F32 1
+
+/* Med3x granularity: chunk norms (the pages' rule) or single |x| elements. */
+#define HQMQ_GRAN_CHUNK 0
+#define HQMQ_GRAN_ELEMENT 1
+
+/* hqmq_status.flags bits. */
+#define HQMQ_FLAG_OUTLIER_OVERFLOW 1u /* more outliers than cap; n_outliers = needed */
+#define HQMQ_FLAG_SATURATED 2u        /* an fp16 radius or outlier value saturated   */
+#define HQMQ_FLAG_NONFINITE 4u        /* a chunk norm was NaN or inf                 */
+#define HQMQ_FLAG_BAD_INDEX 8u        /* decode met an index >= 24 S                 */
+
+/* Device-resident status record (caller-allocated, 32 bytes, 8-byte aligned).
+ * Calls OR flags in and add to the counters. */
+typedef struct {
+    uint32_t flags;
+    uint32_t reserved;
+    uint64_t n_outliers;   /* outliers found by hqmq_outlier_extract          */
+    uint64_t n_saturated;  /* fp16 values clamped to +-65504                  */
+    uint64_t n_nonfinite;  /* chunks encoded with a NaN/inf norm              */
+} hqmq_status;
+
+/* Library version string, e.g. "hqmq-b200 1.0". */
+HQMQ_API const char *hqmq_version(void);
+
+/* Static text for a return code. */
+HQMQ_API const char *hqmq_error_string(int err);
+
+/* Index width b = ceil(log2(24 S)) for S in [1, 65535]; 0 if S is out of range. */
+HQMQ_API uint32_t hqmq_index_bits(uint32_t S);
+
+/* Number of uint32 index words of one call: (B*H*T*D/128) * b; 0 on bad shape. */
+HQMQ_API uint64_t hqmq_index_words(int B, int H, int T, int D, uint32_t S);
+
+/* Secondary codebooks (gist.science/nl, Technische Samenvatting, section 1:
+ * S random unit quaternions per (layer, head, role), no calibration;
+ * abstract: seeded).  Writes d_codebook[n_groups][S][4] fp32 for groups
+ * group0 .. group0 + n_groups - 1.  Quaternion (g, s): Philox4x32-10 with
+ * counter (s, g, 0, 0) and key (seed low 32 bits, seed high 32 bits) gives
+ * four uint32 v; u = (v + 1/2) 2^-32; two Box-Muller pairs in fp64 give four
+ * N(0,1) deviates z; q = z / |z| rounded to fp32.
+ * S in [1, 65535]; n_groups >= 1; group0 + n_groups <= 2^32;
+ * d_codebook 16-byte aligned. */
+HQMQ_API int hqmq_make_codebook(uint64_t seed, uint32_t S, uint32_t n_groups, uint32_t group0,
+                       float *d_codebook, void *stream);
+
+/* Bytes of device workspace hqmq_outlier_extract needs for this shape. */
+HQMQ_API uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gran);
+
+/* Med3x (gist.science/nl, Technische Samenvatting, section 3; the pages
+ * use chunk norms, HQMQ_GRAN_CHUNK; HQMQ_GRAN_ELEMENT applies the same rule
+ * to single-element magnitudes |x|).
+ * Per head h, over all B batches and T tokens of this call:
+ *   r_med[h] = lower median (rank N/2 - 1 of N ascending) of the fp32 chunk
+ *              norms r = sqrt(fma(x3,x3, fma(x2,x2, fma(x1,x1, x0*x0))))
+ *              (or of |x| per element); a NaN sorts above +inf;
+ *   thr[h]   = fl32(C * r_med[h]).
+ * A chunk (element) is an outlier iff r > thr[h] (|x| > thr[h]).  The outlier
+ * list is written in ascending flat index order:
+ *   chunk mode:   d_out_idx[n] = chunk index j, d_out_val[n*4 + i] = fp16 bits
+ *                 of element 4j+i;
+ *   element mode: d_out_idx[n] = element index, d_out_val[n] = fp16 bits;
+ *   fp16 = round-to-nearest-even, finite values beyond +-65504 saturate.
+ * d_slab_off[B*H+1]: entries of slab (b,h) are [slab_off[b*H+h], slab_off[b*H+h+1]).
+ * Entries at positions >= cap are not written (d_slab_off still holds the
+ * full offsets); the status then gets HQMQ_FLAG_OUTLIER_OVERFLOW and
+ * n_outliers the required total, so the caller can retry with a larger cap.
+ * d_x: bf16 or fp32 [B][H][T][D], 16-byte aligned.  d_rmed, d_thr: fp32 [H].
+ * d_out_idx: uint32[cap]; d_out_val: uint16[cap*4] (chunk) or [cap] (element),
+ * 4-byte aligned.  d_ws: at least hqmq_outlier_workspace_size bytes,
+ * 256-byte aligned, contents on entry ignored.  C > 0 and finite.
+ * B*H*T*D must be < 2^32. */
+HQMQ_API int hqmq_outlier_extract(const void *d_x, int dtype, int B, int H, int T, int D, float C,
+                         int gran, float *d_rmed, float *d_thr, uint32_t *d_out_idx,
+                         uint16_t *d_out_val, uint32_t *d_slab_off, uint64_t cap, void *d_ws,
+                         uint64_t ws_bytes, hqmq_status *d_status, void *stream);
+
+/* Encode (gist.science/nl, Technische Samenvatting, Methodologie and
+ * section 1): per chunk j
+ *   - if d_thr != NULL: chunk mode zeroes a chunk with r > thr[h]; element
+ *     mode zeroes each element with |x| > thr[h] (Med3x, the outliers live in
+ *     the list of hqmq_outlier_extract);
+ *   - r = fp32 norm as above; radius[j] = fp16(r) (saturating);
+ *   - index = argmax over s, p of <x, q_p q_s> evaluated as
+ *     <x conj(q_s), q_p> with the nearest 2T element in closed form; ties to
+ *     the lowest s*24+p; r == 0 gives index 0;
+ *   - a NaN/inf norm gives index 0 and radius 0x7E00 and is counted.
+ * d_codebook: fp32 [H][S][4] (this call's heads), 16-byte aligned.
+ * d_idx_words: uint32[hqmq_index_words(B,H,T,D,S)], fully overwritten.
+ * d_radius: uint16 fp16 bits [B*H*T*D/4], 4-byte aligned. */
+HQMQ_API int hqmq_encode(const void *d_x, int dtype, int B, int H, int T, int D, const float *d_codebook,
+                uint32_t S, const float *d_thr, int gran, uint32_t *d_idx_words,
+                uint16_t *d_radius, hqmq_status *d_status, void *stream);
+
+/* Decode: y = round(fl32(r * c_i)) with r the fp16 radius, c = q_p q_s in
+ * fp32 (each component the left-to-right sum of its four Hamilton terms; the
+ * terms are exact because q_p's entries are 0, +-1, +-1/2), round = RN-even to
+ * bf16 (out_dtype HQMQ_BF16) or none (HQMQ_F32).  Outliers, if d_out_idx is
+ * non-NULL (list, offsets and granularity as written by hqmq_outlier_extract,
+ * entries below cap only): chunk mode replaces the chunk by round(fp16
+ * value); element mode gives round(fl32(fl32(r * c_i) + value)).  An index
+ * >= 24 S decodes to 0 and sets HQMQ_FLAG_BAD_INDEX.
+ * d_y: [B][H][T][D] of out_dtype, 16-byte aligned. */
+HQMQ_API int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, const float *d_codebook,
+                uint32_t S, const uint32_t *d_out_idx, const uint16_t *d_out_val,
+                const uint32_t *d_slab_off, uint64_t cap, int gran, int B, int H, int T, int D,
+                void *d_y, int out_dtype, hqmq_status *d_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQMQ_H */

@@ -1,0 +1,163 @@
+// api.cu -- the extern "C" entry points of libhqmq declared in include/hqmq.h:
+// argument validation (synchronous, before anything is enqueued) and the
+// dispatch to the kernels of codebook.cu, med3.cu, encode.cu and decode.cu.
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "../../include/hqmq.h"
+
+extern "C" int hqmq_launch_codebook(uint64_t seed, uint32_t S, uint32_t n_groups, uint32_t group0,
+                                    float *d_codebook, cudaStream_t stream);
+extern "C" int hqmq_launch_encode(const void *x, int dtype, int B, int H, int T, int D,
+                                  const float *cb, uint32_t S, uint32_t b, const float *thr,
+                                  int gran, uint32_t *words, uint16_t *radius, hqmq_status *st,
+                                  int sm_count, cudaStream_t stream);
+extern "C" int hqmq_launch_decode(const uint32_t *words, const uint16_t *radius, const float *cb,
+                                  uint32_t S, uint32_t b, const uint32_t *out_idx,
+                                  const uint16_t *out_val, const uint32_t *slab_off, uint64_t cap,
+                                  int gran, int B, int H, int T, int D, void *y, int out_dtype,
+                                  hqmq_status *st, int sm_count, cudaStream_t stream);
+extern "C" uint64_t hqmq_med3_workspace_bytes(int B, int H, int T, int D);
+extern "C" int hqmq_launch_outlier_extract(const void *x, int dtype, int B, int H, int T, int D,
+                                           float C, int gran, float *rmed, float *thr,
+                                           uint32_t *out_idx, uint16_t *out_val,
+                                           uint32_t *slab_off, uint64_t cap, void *ws,
+                                           hqmq_status *st, int sm_count, cudaStream_t stream);
+
+namespace {
+
+constexpr uint32_t S_MAX = 65535;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape rules shared by every call: positive sizes, D % 4 == 0, whole packing
+// groups per slab ((T*D/4) % 32 == 0), at most 65535 slabs (grid y), and
+// fewer than 2^32 elements (32-bit flat element indices).
+bool shape_ok(int B, int H, int T, int D) {
+    if (B <= 0 || H <= 0 || T <= 0 || D <= 0) return false;
+    if (D % 4 != 0) return false;
+    uint64_t cps = (uint64_t)T * D / 4;
+    if (cps % 32 != 0) return false;
+    if ((uint64_t)B * H > 65535) return false;
+    if ((uint64_t)B * H * T * D >= (1ull << 32)) return false;
+    return true;
+}
+
+bool dtype_ok(int d) { return d == HQMQ_BF16 || d == HQMQ_F32; }
+bool gran_ok(int g) { return g == HQMQ_GRAN_CHUNK || g == HQMQ_GRAN_ELEMENT; }
+
+// SM count of the current device, cached per device id.
+int sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < 64) {
+        int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *hqmq_version(void) { return "hqmq-b200 1.0"; }
+
+const char *hqmq_error_string(int err) {
+    switch (err) {
+        case HQMQ_OK: return "ok";
+        case HQMQ_ERR_ARG: return "invalid argument";
+        case HQMQ_ERR_ALIGN: return "misaligned pointer";
+        case HQMQ_ERR_CUDA: return "CUDA error";
+        case HQMQ_ERR_WORKSPACE: return "workspace too small";
+        default: return "unknown error";
+    }
+}
+
+uint32_t hqmq_index_bits(uint32_t S) {
+    if (S < 1 || S > S_MAX) return 0;
+    uint64_t n = 24ull * S;
+    uint32_t b = 0;
+    while ((1ull << b) < n) ++b;
+    return b;
+}
+
+uint64_t hqmq_index_words(int B, int H, int T, int D, uint32_t S) {
+    uint32_t b = hqmq_index_bits(S);
+    if (!b || !shape_ok(B, H, T, D)) return 0;
+    return ((uint64_t)B * H * T * D / 128) * b;
+}
+
+int hqmq_make_codebook(uint64_t seed, uint32_t S, uint32_t n_groups, uint32_t group0,
+                       float *d_codebook, void *stream) {
+    if (S < 1 || S > S_MAX || n_groups < 1 || !d_codebook) return HQMQ_ERR_ARG;
+    if ((uint64_t)group0 + n_groups > (1ull << 32)) return HQMQ_ERR_ARG;
+    if (!aligned(d_codebook, 16)) return HQMQ_ERR_ALIGN;
+    return hqmq_launch_codebook(seed, S, n_groups, group0, d_codebook, (cudaStream_t)stream);
+}
+
+uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gran) {
+    if (!shape_ok(B, H, T, D) || !gran_ok(gran)) return 0;
+    return hqmq_med3_workspace_bytes(B, H, T, D);
+}
+
+int hqmq_outlier_extract(const void *d_x, int dtype, int B, int H, int T, int D, float C,
+                         int gran, float *d_rmed, float *d_thr, uint32_t *d_out_idx,
+                         uint16_t *d_out_val, uint32_t *d_slab_off, uint64_t cap, void *d_ws,
+                         uint64_t ws_bytes, hqmq_status *d_status, void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
+    if (!(C > 0.0f) || !(C < 3.0e38f)) return HQMQ_ERR_ARG;
+    if (!d_x || !d_rmed || !d_thr || !d_slab_off || !d_ws) return HQMQ_ERR_ARG;
+    if (cap > 0 && (!d_out_idx || !d_out_val)) return HQMQ_ERR_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_rmed, 4) || !aligned(d_thr, 4) ||
+        !aligned(d_slab_off, 4) || !aligned(d_ws, 256) || !aligned(d_out_idx, 4) ||
+        !aligned(d_out_val, 4) || !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    if (ws_bytes < hqmq_med3_workspace_bytes(B, H, T, D)) return HQMQ_ERR_WORKSPACE;
+    int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_outlier_extract(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_out_idx,
+                                       d_out_val, d_slab_off, cap, d_ws, d_status, sm,
+                                       (cudaStream_t)stream);
+}
+
+int hqmq_encode(const void *d_x, int dtype, int B, int H, int T, int D, const float *d_codebook,
+                uint32_t S, const float *d_thr, int gran, uint32_t *d_idx_words,
+                uint16_t *d_radius, hqmq_status *d_status, void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
+    if (S < 1 || S > S_MAX) return HQMQ_ERR_ARG;
+    if (!d_x || !d_codebook || !d_idx_words || !d_radius) return HQMQ_ERR_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_codebook, 16) || !aligned(d_idx_words, 4) ||
+        !aligned(d_radius, 4) || !aligned(d_thr, 4) || !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_encode(d_x, dtype, B, H, T, D, d_codebook, S, hqmq_index_bits(S), d_thr,
+                              gran, d_idx_words, d_radius, d_status, sm, (cudaStream_t)stream);
+}
+
+int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, const float *d_codebook,
+                uint32_t S, const uint32_t *d_out_idx, const uint16_t *d_out_val,
+                const uint32_t *d_slab_off, uint64_t cap, int gran, int B, int H, int T, int D,
+                void *d_y, int out_dtype, hqmq_status *d_status, void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(out_dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
+    if (S < 1 || S > S_MAX) return HQMQ_ERR_ARG;
+    if (!d_idx_words || !d_radius || !d_codebook || !d_y) return HQMQ_ERR_ARG;
+    if (d_out_idx && (!d_out_val || !d_slab_off)) return HQMQ_ERR_ARG;
+    if (!aligned(d_idx_words, 4) || !aligned(d_radius, 4) || !aligned(d_codebook, 16) ||
+        !aligned(d_y, 16) || !aligned(d_out_idx, 4) || !aligned(d_out_val, 4) ||
+        !aligned(d_slab_off, 4) || !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_decode(d_idx_words, d_radius, d_codebook, S, hqmq_index_bits(S), d_out_idx,
+                              d_out_val, d_slab_off, cap, gran, B, H, T, D, d_y, out_dtype,
+                              d_status, sm, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,139 @@
+// hqmq_device.cuh -- device helpers shared by the libhqmq kernels (sm_100a).
+//
+// Every fp32 step that decides a stored bit pattern (chunk norm, radius,
+// codeword, decoded value) is written with explicit IEEE round-to-nearest
+// intrinsics so that no FMA contraction or reassociation can change it.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/hqmq.h"
+
+namespace hqmq {
+
+constexpr unsigned FULL = 0xFFFFFFFFu;
+
+struct DevStatus {  // same layout as hqmq_status
+    unsigned int flags;
+    unsigned int reserved;
+    unsigned long long n_outliers;
+    unsigned long long n_saturated;
+    unsigned long long n_nonfinite;
+};
+static_assert(sizeof(DevStatus) == sizeof(hqmq_status), "status layout");
+
+// Norm of a chunk (w, i, j, k): r2 = fma(x3,x3, fma(x2,x2, fma(x1,x1, x0*x0))),
+// r = sqrt(r2), every step IEEE round-to-nearest.
+__device__ __forceinline__ float chunk_norm(float x0, float x1, float x2, float x3) {
+    float r2 = __fmul_rn(x0, x0);
+    r2 = __fmaf_rn(x1, x1, r2);
+    r2 = __fmaf_rn(x2, x2, r2);
+    r2 = __fmaf_rn(x3, x3, r2);
+    return __fsqrt_rn(r2);
+}
+
+// Order key of a non-negative magnitude: its bits; every NaN -> 0x7FFFFFFF.
+__device__ __forceinline__ uint32_t mag_key(float v) {
+    return (v != v) ? 0x7FFFFFFFu : __float_as_uint(v);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h16) {
+    return __uint_as_float(h16 << 16);
+}
+
+// fp32 -> fp16 bits, round-to-nearest-even; finite values that would round to
+// inf saturate to +-65504 (*sat = 1); NaN -> sign | 0x7E00.
+__device__ __forceinline__ uint16_t f32_to_f16_sat(float v, int &sat) {
+    uint16_t sign = (uint16_t)((__float_as_uint(v) >> 16) & 0x8000u);
+    if (v != v) return (uint16_t)(sign | 0x7E00u);
+    uint16_t h = __half_as_ushort(__float2half_rn(v));
+    if ((h & 0x7FFFu) == 0x7C00u && fabsf(v) != __int_as_float(0x7F800000)) {
+        sat = 1;
+        return (uint16_t)(sign | 0x7BFFu);
+    }
+    return h;
+}
+
+__device__ __forceinline__ float f16_bits_to_f32(uint32_t h) {
+    return __half2float(__ushort_as_half((unsigned short)h));
+}
+
+// Element e of the input (bf16 bits or fp32).
+template <int DT>
+__device__ __forceinline__ void load_chunk(const void *x, size_t j, float &x0, float &x1,
+                                           float &x2, float &x3) {
+    if (DT == HQMQ_BF16) {
+        uint2 v = __ldg(reinterpret_cast<const uint2 *>(x) + j);
+        x0 = __uint_as_float(v.x << 16);
+        x1 = __uint_as_float(v.x & 0xFFFF0000u);
+        x2 = __uint_as_float(v.y << 16);
+        x3 = __uint_as_float(v.y & 0xFFFF0000u);
+    } else {
+        float4 v = __ldg(reinterpret_cast<const float4 *>(x) + j);
+        x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
+    }
+}
+
+// Streaming (read-once) variant: evict-first hint for data not reused soon.
+template <int DT>
+__device__ __forceinline__ void load_chunk_stream(const void *x, size_t j, float &x0, float &x1,
+                                                  float &x2, float &x3) {
+    if (DT == HQMQ_BF16) {
+        uint2 v = __ldcs(reinterpret_cast<const uint2 *>(x) + j);
+        x0 = __uint_as_float(v.x << 16);
+        x1 = __uint_as_float(v.x & 0xFFFF0000u);
+        x2 = __uint_as_float(v.y << 16);
+        x3 = __uint_as_float(v.y & 0xFFFF0000u);
+    } else {
+        float4 v = __ldcs(reinterpret_cast<const float4 *>(x) + j);
+        x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
+    }
+}
+
+// 2T element p as fp32 (w, i, j, k).
+__device__ __forceinline__ void element_2t(int p, float &a0, float &a1, float &a2, float &a3) {
+    if (p < 8) {
+        float sg = (p & 1) ? -1.0f : 1.0f;
+        int ax = p >> 1;
+        a0 = ax == 0 ? sg : 0.0f;
+        a1 = ax == 1 ? sg : 0.0f;
+        a2 = ax == 2 ? sg : 0.0f;
+        a3 = ax == 3 ? sg : 0.0f;
+    } else {
+        int m = p - 8;
+        a0 = (m & 1) ? -0.5f : 0.5f;
+        a1 = (m & 2) ? -0.5f : 0.5f;
+        a2 = (m & 4) ? -0.5f : 0.5f;
+        a3 = (m & 8) ? -0.5f : 0.5f;
+    }
+}
+
+// Codeword q_p q_s in fp32: each component the left-to-right sum of its four
+// Hamilton terms (ij = k), each term one fp32 product.
+__device__ __forceinline__ float4 codeword(int p, float4 q) {
+    float a0, a1, a2, a3;
+    element_2t(p, a0, a1, a2, a3);
+    float4 c;
+    float t;
+    t = __fmul_rn(a0, q.x); t = __fsub_rn(t, __fmul_rn(a1, q.y));
+    t = __fsub_rn(t, __fmul_rn(a2, q.z)); t = __fsub_rn(t, __fmul_rn(a3, q.w)); c.x = t;
+    t = __fmul_rn(a0, q.y); t = __fadd_rn(t, __fmul_rn(a1, q.x));
+    t = __fadd_rn(t, __fmul_rn(a2, q.w)); t = __fsub_rn(t, __fmul_rn(a3, q.z)); c.y = t;
+    t = __fmul_rn(a0, q.z); t = __fsub_rn(t, __fmul_rn(a1, q.w));
+    t = __fadd_rn(t, __fmul_rn(a2, q.x)); t = __fadd_rn(t, __fmul_rn(a3, q.y)); c.z = t;
+    t = __fmul_rn(a0, q.w); t = __fadd_rn(t, __fmul_rn(a1, q.z));
+    t = __fsub_rn(t, __fmul_rn(a2, q.y)); t = __fadd_rn(t, __fmul_rn(a3, q.x)); c.w = t;
+    return c;
+}
+
+__device__ __forceinline__ void status_add(DevStatus *st, unsigned flag,
+                                           unsigned long long *ctr, unsigned long long n) {
+    if (st && n) {
+        atomicOr(&st->flags, flag);
+        atomicAdd(ctr, n);
+    }
+}
+
+}  // namespace hqmq

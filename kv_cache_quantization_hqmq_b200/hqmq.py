@@ -1,0 +1,180 @@
+"""Thin Python binding of libhqmq (include/hqmq.h).
+
+Argument marshalling only: every step of the HQMQ path runs in the CUDA
+kernels of libhqmq.so.  torch provides device memory and streams.  There is no
+fallback: if the library is missing or fails to load, importing this module
+raises.
+
+Entry points keep the C names.  Tensors are passed where the C ABI takes
+device pointers; shapes and dtypes are read from them; `stream` defaults to
+torch's current stream.  Non-zero return codes raise HQMQError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhqmq.so")
+
+HQMQ_OK, HQMQ_ERR_ARG, HQMQ_ERR_ALIGN, HQMQ_ERR_CUDA, HQMQ_ERR_WORKSPACE = 0, 1, 2, 3, 4
+HQMQ_BF16, HQMQ_F32 = 0, 1
+HQMQ_GRAN_CHUNK, HQMQ_GRAN_ELEMENT = 0, 1
+FLAG_OUTLIER_OVERFLOW, FLAG_SATURATED, FLAG_NONFINITE, FLAG_BAD_INDEX = 1, 2, 4, 8
+
+
+class HQMQError(RuntimeError):
+    def __init__(self, fn, rc):
+        super().__init__("%s failed: %s (%d)" % (fn, _lib.hqmq_error_string(rc).decode(), rc))
+        self.rc = rc
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libhqmq.so is not built (%s); run "
+                      "`python -m kv_cache_quantization_hqmq_b200.build`" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P, _I, _U32, _U64, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_float
+_SIGS = {
+    "hqmq_version": (ctypes.c_char_p, []),
+    "hqmq_error_string": (ctypes.c_char_p, [_I]),
+    "hqmq_index_bits": (_U32, [_U32]),
+    "hqmq_index_words": (_U64, [_I, _I, _I, _I, _U32]),
+    "hqmq_make_codebook": (_I, [_U64, _U32, _U32, _U32, _P, _P]),
+    "hqmq_outlier_workspace_size": (_U64, [_I, _I, _I, _I, _I]),
+    "hqmq_outlier_extract": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P, _U64, _P,
+                                  _U64, _P, _P]),
+    "hqmq_encode": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _I, _P, _P, _P, _P]),
+    "hqmq_decode": (_I, [_P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P, _I, _P, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def lib():
+    return _lib
+
+
+def _check(name, rc):
+    if rc != HQMQ_OK:
+        raise HQMQError(name, rc)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return HQMQ_BF16
+    if t.dtype == torch.float32:
+        return HQMQ_F32
+    raise TypeError("HQMQ tensors are bf16 or fp32, got %s" % t.dtype)
+
+
+def _shape4(x):
+    if x.dim() != 4:
+        raise ValueError("expected a [B, H, T, D] tensor, got shape %s" % (tuple(x.shape),))
+    if not x.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return tuple(int(v) for v in x.shape)
+
+
+# ---------------------------------------------------------------- queries
+def hqmq_version():
+    return _lib.hqmq_version().decode()
+
+
+def hqmq_index_bits(S):
+    return int(_lib.hqmq_index_bits(S))
+
+
+def hqmq_index_words(B, H, T, D, S):
+    return int(_lib.hqmq_index_words(B, H, T, D, S))
+
+
+def hqmq_outlier_workspace_size(B, H, T, D, gran=HQMQ_GRAN_CHUNK):
+    return int(_lib.hqmq_outlier_workspace_size(B, H, T, D, gran))
+
+
+# ---------------------------------------------------------------- calls
+def hqmq_make_codebook(seed, S, n_groups, group0, codebook, stream=None):
+    """codebook: fp32 device tensor of n_groups * S * 4 elements."""
+    assert codebook.dtype == torch.float32 and codebook.numel() == n_groups * S * 4
+    _check("hqmq_make_codebook", _lib.hqmq_make_codebook(seed, S, n_groups, group0,
+                                                         _ptr(codebook), _stream(stream)))
+    return codebook
+
+
+def hqmq_outlier_extract(x, C, gran, rmed, thr, out_idx, out_val, slab_off, cap, ws,
+                         status=None, stream=None):
+    B, H, T, D = _shape4(x)
+    _check("hqmq_outlier_extract", _lib.hqmq_outlier_extract(
+        _ptr(x), _dtype_code(x), B, H, T, D, float(C), gran, _ptr(rmed), _ptr(thr),
+        _ptr(out_idx), _ptr(out_val), _ptr(slab_off), int(cap), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(status), _stream(stream)))
+
+
+def hqmq_encode(x, codebook, S, thr, gran, idx_words, radius, status=None, stream=None):
+    B, H, T, D = _shape4(x)
+    _check("hqmq_encode", _lib.hqmq_encode(
+        _ptr(x), _dtype_code(x), B, H, T, D, _ptr(codebook), S, _ptr(thr), gran,
+        _ptr(idx_words), _ptr(radius), _ptr(status), _stream(stream)))
+
+
+def hqmq_decode(idx_words, radius, codebook, S, out_idx, out_val, slab_off, cap, gran, y,
+                status=None, stream=None):
+    B, H, T, D = _shape4(y)
+    _check("hqmq_decode", _lib.hqmq_decode(
+        _ptr(idx_words), _ptr(radius), _ptr(codebook), S, _ptr(out_idx), _ptr(out_val),
+        _ptr(slab_off), int(cap), gran, B, H, T, D, _ptr(y), _dtype_code(y), _ptr(status),
+        _stream(stream)))
+
+
+# ---------------------------------------------------------------- buffers
+def new_status(device="cuda"):
+    """A zeroed device hqmq_status (4 x 64-bit words)."""
+    return torch.zeros(4, dtype=torch.int64, device=device)
+
+
+def read_status(status):
+    v = status.cpu().numpy().view("uint64")
+    return {"flags": int(v[0] & 0xFFFFFFFF), "n_outliers": int(v[1]),
+            "n_saturated": int(v[2]), "n_nonfinite": int(v[3])}
+
+
+def alloc_codes(B, H, T, D, S, device="cuda"):
+    """(idx_words uint32 as int32, radius fp16 bits as int16) for one call."""
+    nw = hqmq_index_words(B, H, T, D, S)
+    if nw == 0:
+        raise ValueError("bad shape/S")
+    words = torch.empty(nw, dtype=torch.int32, device=device)
+    radius = torch.empty(B * H * T * D // 4, dtype=torch.int16, device=device)
+    return words, radius
+
+
+def alloc_outliers(B, H, T, D, cap, gran=HQMQ_GRAN_CHUNK, device="cuda"):
+    """(rmed, thr, out_idx, out_val, slab_off, ws) for one call's Med3x step."""
+    rmed = torch.empty(H, dtype=torch.float32, device=device)
+    thr = torch.empty(H, dtype=torch.float32, device=device)
+    out_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=device)
+    out_val = torch.empty(max(cap, 1) * (4 if gran == HQMQ_GRAN_CHUNK else 1), dtype=torch.int16,
+                          device=device)
+    slab_off = torch.empty(B * H + 1, dtype=torch.int32, device=device)
+    ws = torch.empty(hqmq_outlier_workspace_size(B, H, T, D, gran), dtype=torch.uint8,
+                     device=device)
+    return rmed, thr, out_idx, out_val, slab_off, ws

@@ -1,0 +1,87 @@
+"""The C ABI library loads here (no GPU needed), exports every entry point
+include/hqmq.h declares, and rejects bad arguments synchronously before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hqmq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kv_cache_quantization_hqmq_b200 import build
+    build.build()
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    return hqmq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"HQMQ_API\s+[\w\s\*]*?\b(hqmq_\w+)\s*\(", text)
+
+
+def test_header_declares_the_four_calls_of_the_path():
+    names = declared_functions()
+    for n in ("hqmq_make_codebook", "hqmq_outlier_extract", "hqmq_encode", "hqmq_decode"):
+        assert n in names
+    assert len(names) == len(set(names)) >= 9
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_only_declared_symbols_are_exported():
+    import subprocess
+    from kv_cache_quantization_hqmq_b200 import build
+    out = subprocess.check_output(["nm", "-D", "--defined-only", build.LIB], text=True)
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and "hqmq" in l}
+    assert exported == set(declared_functions())
+
+
+def test_host_queries(lib):
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    assert hqmq.hqmq_version().startswith("hqmq-b200")
+    assert hqmq.hqmq_index_bits(8) == 8 and hqmq.hqmq_index_bits(32) == 10
+    assert hqmq.hqmq_index_bits(0) == 0 and hqmq.hqmq_index_bits(65536) == 0
+    # 70B call: 1 x 8 x 131072 x 128 -> 1,048,576 groups x 10 words
+    assert hqmq.hqmq_index_words(1, 8, 131072, 128, 32) == 1048576 * 10
+    assert hqmq.hqmq_index_words(1, 1, 3, 128, 8) == 24       # 3 groups x 8 words
+    assert hqmq.hqmq_index_words(1, 1, 3, 12, 8) == 0         # 9 chunks: not whole groups
+    assert hqmq.hqmq_index_words(1, 1, 8, 6, 8) == 0          # D % 4 != 0
+    assert hqmq.hqmq_outlier_workspace_size(1, 8, 131072, 128) > 8 * 2048 * 4
+    assert hqmq.hqmq_outlier_workspace_size(1, 8, 131072, 128, 2) == 0
+
+
+def test_bad_arguments_rejected_without_cuda(lib):
+    P = ctypes.c_void_p
+    good = P(1 << 20)                   # never dereferenced: validation fails first
+    st = None
+    # S out of range / bad shapes / unknown enums -> HQMQ_ERR_ARG (1)
+    assert lib.hqmq_make_codebook(1, 0, 4, 0, good, None) == 1
+    assert lib.hqmq_make_codebook(1, 8, 0, 0, good, None) == 1
+    assert lib.hqmq_make_codebook(1, 8, 2, 0xFFFFFFFF, good, None) == 1
+    assert lib.hqmq_encode(good, 0, 1, 1, 8, 6, good, 8, None, 0, good, good, st, None) == 1
+    assert lib.hqmq_encode(good, 0, 1, 1, 3, 12, good, 8, None, 0, good, good, st, None) == 1
+    assert lib.hqmq_encode(good, 2, 1, 1, 8, 128, good, 8, None, 0, good, good, st, None) == 1
+    assert lib.hqmq_encode(good, 0, 1, 1, 8, 128, good, 70000, None, 0, good, good, st, None) == 1
+    assert lib.hqmq_encode(good, 0, 1, 1, 8, 128, good, 8, None, 5, good, good, st, None) == 1
+    assert lib.hqmq_encode(None, 0, 1, 1, 8, 128, good, 8, None, 0, good, good, st, None) == 1
+    assert lib.hqmq_encode(good, 0, 300, 300, 8, 128, good, 8, None, 0, good, good, st, None) == 1
+    # misaligned pointers -> HQMQ_ERR_ALIGN (2)
+    assert lib.hqmq_encode(P((1 << 20) + 8), 0, 1, 1, 8, 128, good, 8, None, 0, good, good, st,
+                           None) == 2
+    assert lib.hqmq_decode(good, P((1 << 20) + 2), good, 8, None, None, None, 0, 0, 1, 1, 8, 128,
+                           good, 0, st, None) == 2
+    # outlier extract: C must be positive and finite; workspace must be large enough
+    assert lib.hqmq_outlier_extract(good, 0, 1, 1, 8, 128, ctypes.c_float(0.0), 0, good, good,
+                                    good, good, good, 16, good, 1 << 20, st, None) == 1
+    assert lib.hqmq_outlier_extract(good, 0, 1, 1, 8, 128, ctypes.c_float(float("inf")), 0, good,
+                                    good, good, good, good, 16, good, 1 << 20, st, None) == 1
+    assert lib.hqmq_outlier_extract(good, 0, 1, 1, 8, 128, ctypes.c_float(3.0), 0, good, good,
+                                    good, good, good, 16, good, 16, st, None) == 4
