@@ -116,6 +116,12 @@ WORKLOADS = {
                                 "normal_channels", channel_frac=0.01, channel_scale=30.0,
                                 note="Llama-3-70B GQA cache, 131072 tokens (42.95 GB K+V bf16), "
                                      "1% channels x30, Med3x C=3, S=32, layer by layer"),
+    # one layer (K and V) of the Llama-3-70B 128k cache: the same calls and
+    # kernels at 537 MB, small enough for a full ncu capture
+    "llama3_70b_128k_1layer": Workload("llama3_70b_128k_1layer", 1, 8, 128, 1, 131072, "bf16", 32,
+                                       True, "normal_channels", channel_frac=0.01,
+                                       channel_scale=30.0,
+                                       note="one layer of the Llama-3-70B 128k cache (profiling)"),
 }
 
 

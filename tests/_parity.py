@@ -112,8 +112,9 @@ def check_codes(oracle, x_np, cb_np, S, gpu_idx, gpu_radius, thr=None, gran=0, c
         bad = gap > NEAR_TIE_REL * np.abs(best[mm].astype(np.float64))
         assert not bad.any(), "non-tie index mismatch at chunks %s (gap %s)" % (
             chunks[mm][bad][:10], gap[bad][:10])
-    near = int(np.sum(best.astype(np.float64) - second.astype(np.float64)
-                      <= NEAR_TIE_REL * np.abs(best.astype(np.float64))))
+    nz = best > 0          # zero (or zeroed outlier) chunks have no search
+    near = int(np.sum(nz & (best.astype(np.float64) - second.astype(np.float64)
+                            <= NEAR_TIE_REL * np.abs(best.astype(np.float64)))))
     return chunks.size, int(mm.size), near
 
 
