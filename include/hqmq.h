@@ -179,6 +179,33 @@ HQMQ_API int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, 
                 const uint32_t *d_slab_off, uint64_t cap, int gran, int B, int H, int T, int D,
                 void *d_y, int out_dtype, hqmq_status *d_status, void *stream);
 
+/* Size of the fixed device scratch array of hqmq_outlier_extract_noalloc. */
+#define HQMQ_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* hqmq_outlier_extract without a workspace argument.  The paper has no
+ * counterpart of this entry point; it exists for callers that cannot
+ * allocate device memory: a serving engine that has reserved all of the
+ * GPU's memory for its own pool, or a hook running where cudaMalloc/cudaFree
+ * (which may synchronise the device) are not allowed.  The caller still
+ * passes every input and output.
+ *
+ * The scratch lives in one file-scope device array of
+ * HQMQ_NOALLOC_SCRATCH_BYTES (1 MiB) that every GPU which loads libhqmq holds
+ * until the process exits.  Shapes whose hqmq_outlier_workspace_size exceeds
+ * it are rejected with HQMQ_ERR_WORKSPACE (a 1 x 8 x 131072 x 128 call needs
+ * about 130 KB).  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current) and caches it;
+ * make that first call before any stream capture.  All calls on a device
+ * share the one array: calls whose execution overlaps on the GPU (different
+ * streams without ordering between them) race and give wrong results.  Each
+ * call clears what must start at zero.  Nothing is allocated or freed.
+ * Arguments, results and errors are otherwise those of hqmq_outlier_extract. */
+HQMQ_API int hqmq_outlier_extract_noalloc(const void *d_x, int dtype, int B, int H, int T, int D,
+                                          float C, int gran, float *d_rmed, float *d_thr,
+                                          uint32_t *d_out_idx, uint16_t *d_out_val,
+                                          uint32_t *d_slab_off, uint64_t cap,
+                                          hqmq_status *d_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

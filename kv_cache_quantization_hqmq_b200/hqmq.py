@@ -48,6 +48,8 @@ _SIGS = {
                                   _U64, _P, _P]),
     "hqmq_encode": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _I, _P, _P, _P, _P]),
     "hqmq_decode": (_I, [_P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P, _I, _P, _P]),
+    "hqmq_outlier_extract_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P,
+                                          _U64, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -127,6 +129,17 @@ def hqmq_outlier_extract(x, C, gran, rmed, thr, out_idx, out_val, slab_off, cap,
         _ptr(x), _dtype_code(x), B, H, T, D, float(C), gran, _ptr(rmed), _ptr(thr),
         _ptr(out_idx), _ptr(out_val), _ptr(slab_off), int(cap), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(status), _stream(stream)))
+
+
+def hqmq_outlier_extract_noalloc(x, C, gran, rmed, thr, out_idx, out_val, slab_off, cap,
+                                 status=None, stream=None):
+    """Med3x with the library's fixed 1 MiB device scratch instead of a
+    caller workspace, for callers that cannot allocate device memory.  Calls
+    on one device share that scratch: do not let two of them overlap."""
+    B, H, T, D = _shape4(x)
+    _check("hqmq_outlier_extract_noalloc", _lib.hqmq_outlier_extract_noalloc(
+        _ptr(x), _dtype_code(x), B, H, T, D, float(C), gran, _ptr(rmed), _ptr(thr),
+        _ptr(out_idx), _ptr(out_val), _ptr(slab_off), int(cap), _ptr(status), _stream(stream)))
 
 
 def hqmq_encode(x, codebook, S, thr, gran, idx_words, radius, status=None, stream=None):
