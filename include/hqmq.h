@@ -173,7 +173,9 @@ HQMQ_API int hqmq_encode(const void *d_x, int dtype, int B, int H, int T, int D,
  * entries below cap only): chunk mode replaces the chunk by round(fp16
  * value); element mode gives round(fl32(fl32(r * c_i) + value)).  An index
  * >= 24 S decodes to 0 and sets HQMQ_FLAG_BAD_INDEX.
- * d_y: [B][H][T][D] of out_dtype, 16-byte aligned. */
+ * d_idx_words and d_radius as written by hqmq_encode; d_y: [B][H][T][D]
+ * of out_dtype, 16-byte aligned.  With a list, a second kernel applies the
+ * outliers after the main pass on the same stream. */
 HQMQ_API int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, const float *d_codebook,
                 uint32_t S, const uint32_t *d_out_idx, const uint16_t *d_out_val,
                 const uint32_t *d_slab_off, uint64_t cap, int gran, int B, int H, int T, int D,

@@ -6,21 +6,22 @@
 // inside their attention kernel ("Memory en Latentie"); here it is a
 // standalone streaming kernel that writes the dense bf16 (or fp32) tensor.
 //
-// Each CTA owns one slab (b, h) and builds that head's 24 S codeword table in
-// shared memory once (for S <= 170; larger S recomputes the codeword per
-// chunk).  Threads decode 2 consecutive chunks per step, so every output
-// store is one aligned 16-byte vector (8 bf16).  The slab is cut into
-// ranges of RANGE chunks; after a range's main pass the CTA applies that
-// range's outliers (chunk mode: overwrite after a barrier; element mode: an
-// add-back buffer in shared memory, pre-filled with -0.0, the exact additive
-// identity).
+// Two launches on the caller's stream:
+//  * k_decode: each CTA owns one slab (b, h), builds that head's 24 S
+//    codeword table in shared memory once (S <= 170; larger S recomputes the
+//    codeword per chunk) and streams its chunks: per chunk pair one 4-byte
+//    radius load, the index bits, 8 products and one 16-byte store; no
+//    barriers after the table build;
+//  * k_decode_outliers (only with an outlier list): one thread per list
+//    entry overwrites the chunk (chunk mode) or adds the fp16 value to the
+//    recomputed fl32(r * c) of its element (element mode).
 #include "hqmq_device.cuh"
 
 namespace hqmq {
 
 constexpr int DEC_THREADS = 256;
-constexpr int RANGE = 2048;          // chunks per range (8 per thread)
-constexpr int MODE_NONE = 0, MODE_CHUNK = 1, MODE_ELEM = 2;
+constexpr int PAIRS = 4;             // chunk pairs per thread per step (8 chunks in flight)
+constexpr int OUT_THREADS = 256;
 
 __device__ __forceinline__ uint32_t get_index(const uint32_t *__restrict__ words, uint64_t grp,
                                               uint32_t k, uint32_t b) {
@@ -32,28 +33,16 @@ __device__ __forceinline__ uint32_t get_index(const uint32_t *__restrict__ words
     return (uint32_t)(v >> o) & ((1u << b) - 1u);
 }
 
-// First position in [lo, hi) with key >= v (keys ascending).
-__device__ __forceinline__ uint32_t lower_bound(const uint32_t *__restrict__ keys, uint32_t lo,
-                                                uint32_t hi, uint32_t v) {
-    while (lo < hi) {
-        uint32_t mid = lo + ((hi - lo) >> 1);
-        if (__ldg(keys + mid) < v) lo = mid + 1; else hi = mid;
-    }
-    return lo;
-}
-
-template <int OUT_DT, int MODE, bool TABLE>
+// Main pass: every chunk -> round(fl32(r * c_i)).  Thread t of a warp handles
+// the chunk pairs w*PAIRS*32 + u*32 + t (u < PAIRS): each load and each
+// 16-byte store instruction of the warp is contiguous, and PAIRS pairs of
+// loads are in flight per thread.
+template <int OUT_DT, bool TABLE>
 __global__ void __launch_bounds__(DEC_THREADS)
 k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius,
-         const float4 *__restrict__ cb_all, uint32_t S, uint32_t b,
-         const uint32_t *__restrict__ out_idx, const uint16_t *__restrict__ out_val,
-         const uint32_t *__restrict__ slab_off, uint64_t cap, int H, uint32_t chunks_per_slab,
-         void *__restrict__ y, DevStatus *st) {
-    extern __shared__ float4 smem[];
-    float4 *s_tab = smem;                                            // [24 S] if TABLE
-    float *s_add = reinterpret_cast<float *>(smem + (TABLE ? 24 * S : 0));  // [RANGE*4]
-    __shared__ uint32_t s_rng[2];
-
+         const float4 *__restrict__ cb_all, uint32_t S, uint32_t b, int H,
+         uint32_t chunks_per_slab, void *__restrict__ y, DevStatus *st) {
+    extern __shared__ float4 s_tab[];              // [24 S] if TABLE
     const int slab = blockIdx.y;
     const int h = slab % H;
     const float4 *cb = cb_all + (size_t)h * S;
@@ -63,121 +52,133 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
             s_tab[i] = codeword((int)(i % 24u), __ldg(cb + i / 24u));
         __syncthreads();
     }
-    const uint64_t chunk0 = (uint64_t)slab * chunks_per_slab;     // first chunk of the slab
-    uint32_t o_lo = 0, o_hi = 0;                                     // this slab's list entries
-    if (MODE != MODE_NONE) {
-        uint64_t a = slab_off[slab], e = slab_off[slab + 1];
-        o_lo = (uint32_t)(a < cap ? a : cap);
-        o_hi = (uint32_t)(e < cap ? e : cap);
-    }
+    const uint64_t chunk0 = (uint64_t)slab * chunks_per_slab;
+    const uint32_t pairs_per_slab = chunks_per_slab / 2;
+    const int lane = threadIdx.x & 31;
+    const uint32_t warp_g = blockIdx.x * (DEC_THREADS / 32) + (threadIdx.x >> 5);
+    const uint32_t n_warps = gridDim.x * (DEC_THREADS / 32);
     unsigned n_bad = 0;
-    const uint32_t n_ranges = (chunks_per_slab + RANGE - 1) / RANGE;
-    for (uint32_t rg = blockIdx.x; rg < n_ranges; rg += gridDim.x) {
-        const uint32_t c0 = rg * RANGE;
-        const uint32_t c1 = min(c0 + RANGE, chunks_per_slab);
-        if (MODE != MODE_NONE) {
-            if (threadIdx.x == 0) {
-                uint32_t base = (uint32_t)(MODE == MODE_ELEM ? 4 : 1);
-                uint32_t lo_key = (uint32_t)((chunk0 + c0) * base);
-                uint32_t hi_key = (uint32_t)((chunk0 + c1) * base);
-                uint32_t lo = lower_bound(out_idx, o_lo, o_hi, lo_key);
-                s_rng[0] = lo;
-                s_rng[1] = lower_bound(out_idx, lo, o_hi, hi_key);
-            }
-            if (MODE == MODE_ELEM)
-                for (int i = threadIdx.x; i < RANGE * 4; i += DEC_THREADS) s_add[i] = -0.0f;
-            __syncthreads();
-            if (MODE == MODE_ELEM) {
-                const uint32_t e0 = (uint32_t)((chunk0 + c0) * 4);
-                const uint32_t n_e = (c1 - c0) * 4;
-                for (uint32_t q = s_rng[0] + threadIdx.x; q < s_rng[1]; q += DEC_THREADS) {
-                    const uint32_t e = __ldg(out_idx + q) - e0;
-                    if (e < n_e) s_add[e] = f16_bits_to_f32(__ldg(out_val + q));   // unsorted list guard
-                }
-                __syncthreads();
+    for (uint32_t p0 = warp_g * PAIRS * 32; p0 < pairs_per_slab; p0 += n_warps * PAIRS * 32) {
+        uint32_t rr[PAIRS], idx[PAIRS][2];
+#pragma unroll
+        for (int u = 0; u < PAIRS; ++u) {              // all loads first
+            const uint32_t pr = p0 + u * 32 + lane;
+            rr[u] = 0; idx[u][0] = idx[u][1] = 0;
+            if (pr < pairs_per_slab) {
+                const uint64_t j = chunk0 + 2 * (uint64_t)pr;
+                rr[u] = __ldcs(reinterpret_cast<const uint32_t *>(radius) + (j >> 1));
+                idx[u][0] = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
+                idx[u][1] = get_index(words, j >> 5, (uint32_t)(j & 31u) + 1, b);
             }
         }
-        for (uint32_t c = c0 + 2 * threadIdx.x; c < c1; c += 2 * DEC_THREADS) {
-            const uint64_t j = chunk0 + c;                 // even: (T*D/4) % 32 == 0
-            const uint32_t rr2 = __ldg(reinterpret_cast<const uint32_t *>(radius) + (j >> 1));
-            const uint64_t grp = j >> 5;
-            const uint32_t k = (uint32_t)(j & 31u);
+#pragma unroll
+        for (int u = 0; u < PAIRS; ++u) {
+            const uint32_t pr = p0 + u * 32 + lane;
+            if (pr >= pairs_per_slab) break;
+            const uint64_t j = chunk0 + 2 * (uint64_t)pr;
             float out[8];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                uint32_t idx = get_index(words, grp, k + u, b);
-                float r = f16_bits_to_f32(u ? (rr2 >> 16) : (rr2 & 0xFFFFu));
+            for (int v = 0; v < 2; ++v) {
+                float r = f16_bits_to_f32(v ? (rr[u] >> 16) : (rr[u] & 0xFFFFu));
+                const uint32_t ix = idx[u][v];
                 float4 cw;
-                if (idx < n_words) {
-                    cw = TABLE ? s_tab[idx] : codeword((int)(idx % 24u), __ldg(cb + idx / 24u));
+                if (ix < n_words) {
+                    cw = TABLE ? s_tab[ix] : codeword((int)(ix % 24u), __ldg(cb + ix / 24u));
                 } else {
                     cw = make_float4(0.f, 0.f, 0.f, 0.f);
                     r = 0.0f;
                     ++n_bad;
                 }
-                out[4 * u + 0] = __fmul_rn(r, cw.x);
-                out[4 * u + 1] = __fmul_rn(r, cw.y);
-                out[4 * u + 2] = __fmul_rn(r, cw.z);
-                out[4 * u + 3] = __fmul_rn(r, cw.w);
-            }
-            if (MODE == MODE_ELEM) {
-                const float *ad = s_add + (c - c0) * 4;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) out[i] = __fadd_rn(out[i], ad[i]);
+                out[4 * v + 0] = __fmul_rn(r, cw.x);
+                out[4 * v + 1] = __fmul_rn(r, cw.y);
+                out[4 * v + 2] = __fmul_rn(r, cw.z);
+                out[4 * v + 3] = __fmul_rn(r, cw.w);
             }
             if (OUT_DT == HQMQ_BF16) {
-                uint4 v;
-                __nv_bfloat162 p0 = __floats2bfloat162_rn(out[0], out[1]);
-                __nv_bfloat162 p1 = __floats2bfloat162_rn(out[2], out[3]);
-                __nv_bfloat162 p2 = __floats2bfloat162_rn(out[4], out[5]);
-                __nv_bfloat162 p3 = __floats2bfloat162_rn(out[6], out[7]);
-                v.x = *reinterpret_cast<uint32_t *>(&p0);
-                v.y = *reinterpret_cast<uint32_t *>(&p1);
-                v.z = *reinterpret_cast<uint32_t *>(&p2);
-                v.w = *reinterpret_cast<uint32_t *>(&p3);
-                __stcs(reinterpret_cast<uint4 *>(y) + (j >> 1), v);
+                uint4 q;
+                __nv_bfloat162 a0 = __floats2bfloat162_rn(out[0], out[1]);
+                __nv_bfloat162 a1 = __floats2bfloat162_rn(out[2], out[3]);
+                __nv_bfloat162 a2 = __floats2bfloat162_rn(out[4], out[5]);
+                __nv_bfloat162 a3 = __floats2bfloat162_rn(out[6], out[7]);
+                q.x = *reinterpret_cast<uint32_t *>(&a0);
+                q.y = *reinterpret_cast<uint32_t *>(&a1);
+                q.z = *reinterpret_cast<uint32_t *>(&a2);
+                q.w = *reinterpret_cast<uint32_t *>(&a3);
+                __stcs(reinterpret_cast<uint4 *>(y) + (j >> 1), q);
             } else {
                 float4 *yp = reinterpret_cast<float4 *>(y) + j;
                 __stcs(yp, make_float4(out[0], out[1], out[2], out[3]));
                 __stcs(yp + 1, make_float4(out[4], out[5], out[6], out[7]));
             }
         }
-        if (MODE == MODE_CHUNK) {
-            __syncthreads();   // main-pass stores of this range precede the overwrite
-            for (uint32_t q = s_rng[0] + threadIdx.x; q < s_rng[1]; q += DEC_THREADS) {
-                const uint64_t j = __ldg(out_idx + q);
-                if (j < chunk0 + c0 || j >= chunk0 + c1) continue;   // unsorted list guard
-                const uint32_t *vv = reinterpret_cast<const uint32_t *>(out_val + (size_t)q * 4);
-                uint32_t v01 = __ldg(vv), v23 = __ldg(vv + 1);
-                float f0 = f16_bits_to_f32(v01 & 0xFFFFu), f1 = f16_bits_to_f32(v01 >> 16);
-                float f2 = f16_bits_to_f32(v23 & 0xFFFFu), f3 = f16_bits_to_f32(v23 >> 16);
-                if (OUT_DT == HQMQ_BF16) {
-                    __nv_bfloat162 p0 = __floats2bfloat162_rn(f0, f1);
-                    __nv_bfloat162 p1 = __floats2bfloat162_rn(f2, f3);
-                    uint2 v;
-                    v.x = *reinterpret_cast<uint32_t *>(&p0);
-                    v.y = *reinterpret_cast<uint32_t *>(&p1);
-                    reinterpret_cast<uint2 *>(y)[j] = v;
-                } else {
-                    reinterpret_cast<float4 *>(y)[j] = make_float4(f0, f1, f2, f3);
-                }
-            }
-        }
-        if (MODE != MODE_NONE) __syncthreads();   // s_rng / s_add reuse by the next range
     }
     unsigned nb = __reduce_add_sync(FULL, n_bad);
-    if ((threadIdx.x & 31) == 0 && nb && st) atomicOr(&st->flags, HQMQ_FLAG_BAD_INDEX);
+    if (lane == 0 && nb && st) atomicOr(&st->flags, HQMQ_FLAG_BAD_INDEX);
 }
 
-template <int OUT_DT, int MODE, bool TABLE>
-static int launch_t(const uint32_t *words, const uint16_t *radius, const float *cb, uint32_t S,
-                    uint32_t b, const uint32_t *out_idx, const uint16_t *out_val,
-                    const uint32_t *slab_off, uint64_t cap, int B, int H,
-                    uint32_t chunks_per_slab, void *y, hqmq_status *st, int sm_count,
-                    cudaStream_t stream) {
-    auto kern = k_decode<OUT_DT, MODE, TABLE>;
-    size_t smem = (TABLE ? (size_t)24 * S * sizeof(float4) : 0) +
-                  (MODE == MODE_ELEM ? (size_t)RANGE * 4 * sizeof(float) : 0);
+// Outlier pass, one thread per list entry below cap (after the main pass, on
+// the same stream).  Chunk mode: the chunk becomes round(fp16 values).
+// Element mode: the element becomes round(fl32(fl32(r * c_e) + v)), with
+// r * c_e recomputed from the chunk's code exactly as the main pass does.
+// Entries whose index lies outside the tensor are skipped.
+template <int OUT_DT, int GRAN>
+__global__ void __launch_bounds__(OUT_THREADS)
+k_decode_outliers(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius,
+                  const float4 *__restrict__ cb_all, uint32_t S, uint32_t b, int H,
+                  uint32_t chunks_per_slab, uint64_t n_chunks,
+                  const uint32_t *__restrict__ out_idx, const uint16_t *__restrict__ out_val,
+                  const uint32_t *__restrict__ slab_off, uint64_t n_slabs, uint64_t cap,
+                  void *__restrict__ y) {
+    uint64_t n = slab_off[n_slabs];
+    if (n > cap) n = cap;
+    for (uint64_t q = (uint64_t)blockIdx.x * OUT_THREADS + threadIdx.x; q < n;
+         q += (uint64_t)gridDim.x * OUT_THREADS) {
+        const uint64_t e = __ldg(out_idx + q);
+        if (GRAN == HQMQ_GRAN_CHUNK) {
+            if (e >= n_chunks) continue;
+            const uint32_t *vv = reinterpret_cast<const uint32_t *>(out_val + q * 4);
+            const uint32_t v01 = __ldg(vv), v23 = __ldg(vv + 1);
+            const float f0 = f16_bits_to_f32(v01 & 0xFFFFu), f1 = f16_bits_to_f32(v01 >> 16);
+            const float f2 = f16_bits_to_f32(v23 & 0xFFFFu), f3 = f16_bits_to_f32(v23 >> 16);
+            if (OUT_DT == HQMQ_BF16) {
+                __nv_bfloat162 a0 = __floats2bfloat162_rn(f0, f1);
+                __nv_bfloat162 a1 = __floats2bfloat162_rn(f2, f3);
+                uint2 o;
+                o.x = *reinterpret_cast<uint32_t *>(&a0);
+                o.y = *reinterpret_cast<uint32_t *>(&a1);
+                reinterpret_cast<uint2 *>(y)[e] = o;
+            } else {
+                reinterpret_cast<float4 *>(y)[e] = make_float4(f0, f1, f2, f3);
+            }
+        } else {
+            if (e >= 4 * n_chunks) continue;
+            const uint64_t j = e >> 2;
+            const int i = (int)(e & 3u);
+            const int h = (int)((j / chunks_per_slab) % (uint64_t)H);
+            const uint32_t ix = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
+            float r = f16_bits_to_f32(__ldg(radius + j));
+            float c = 0.0f;
+            if (ix < 24u * S) {
+                const float4 cw = codeword((int)(ix % 24u), __ldg(cb_all + (size_t)h * S + ix / 24u));
+                c = i == 0 ? cw.x : i == 1 ? cw.y : i == 2 ? cw.z : cw.w;
+            } else {
+                r = 0.0f;
+            }
+            const float val = __fadd_rn(__fmul_rn(r, c), f16_bits_to_f32(__ldg(out_val + q)));
+            if (OUT_DT == HQMQ_BF16)
+                reinterpret_cast<__nv_bfloat16 *>(y)[e] = __float2bfloat16_rn(val);
+            else
+                reinterpret_cast<float *>(y)[e] = val;
+        }
+    }
+}
+
+template <int OUT_DT, bool TABLE>
+static int launch_main(const uint32_t *words, const uint16_t *radius, const float *cb, uint32_t S,
+                       uint32_t b, int B, int H, uint32_t cps, void *y, hqmq_status *st,
+                       int sm_count, cudaStream_t stream) {
+    auto kern = k_decode<OUT_DT, TABLE>;
+    size_t smem = TABLE ? (size_t)24 * S * sizeof(float4) : 0;
     if (smem > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
@@ -187,43 +188,54 @@ static int launch_t(const uint32_t *words, const uint16_t *radius, const float *
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, DEC_THREADS, smem) !=
             cudaSuccess || occ < 1)
         occ = 1;
-    int n_slabs = B * H;
-    uint64_t ranges = (chunks_per_slab + RANGE - 1) / RANGE;
-    uint64_t fill = ((uint64_t)sm_count * occ + n_slabs - 1) / n_slabs;
-    uint64_t gx = ranges < fill ? ranges : fill;
+    const int n_slabs = B * H;
+    const uint64_t per_cta = (uint64_t)DEC_THREADS * PAIRS * 2;     // chunks per CTA step
+    const uint64_t want = (cps + per_cta - 1) / per_cta;
+    const uint64_t fill = ((uint64_t)sm_count * occ + n_slabs - 1) / n_slabs;
+    uint64_t gx = want < fill ? want : fill;
     if (gx < 1) gx = 1;
     dim3 grid((unsigned)gx, (unsigned)n_slabs);
     kern<<<grid, DEC_THREADS, smem, stream>>>(words, radius, reinterpret_cast<const float4 *>(cb),
-                                              S, b, out_idx, out_val, slab_off, cap, H,
-                                              chunks_per_slab, y,
-                                              reinterpret_cast<DevStatus *>(st));
+                                              S, b, H, cps, y, reinterpret_cast<DevStatus *>(st));
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
-template <int OUT_DT, int MODE>
-static int launch_m(bool table, const uint32_t *words, const uint16_t *radius, const float *cb,
-                    uint32_t S, uint32_t b, const uint32_t *out_idx, const uint16_t *out_val,
-                    const uint32_t *slab_off, uint64_t cap, int B, int H, uint32_t cps, void *y,
-                    hqmq_status *st, int sm, cudaStream_t stream) {
-    return table ? launch_t<OUT_DT, MODE, true>(words, radius, cb, S, b, out_idx, out_val, slab_off,
-                                                cap, B, H, cps, y, st, sm, stream)
-                 : launch_t<OUT_DT, MODE, false>(words, radius, cb, S, b, out_idx, out_val,
-                                                 slab_off, cap, B, H, cps, y, st, sm, stream);
+template <int OUT_DT>
+static int launch_out(int gran, const uint32_t *words, const uint16_t *radius, const float *cb,
+                      uint32_t S, uint32_t b, int B, int H, uint32_t cps,
+                      const uint32_t *out_idx, const uint16_t *out_val, const uint32_t *slab_off,
+                      uint64_t cap, void *y, int sm_count, cudaStream_t stream) {
+    const uint64_t n_slabs = (uint64_t)B * H;
+    const uint64_t n_chunks = n_slabs * cps;
+    // the list length is only known on the device: size the grid for cap
+    uint64_t blocks = (cap + OUT_THREADS - 1) / OUT_THREADS;
+    const uint64_t max_blocks = (uint64_t)sm_count * 8;
+    if (blocks > max_blocks) blocks = max_blocks;
+    if (blocks < 1) blocks = 1;
+    const float4 *cb4 = reinterpret_cast<const float4 *>(cb);
+    if (gran == HQMQ_GRAN_CHUNK)
+        k_decode_outliers<OUT_DT, HQMQ_GRAN_CHUNK><<<(unsigned)blocks, OUT_THREADS, 0, stream>>>(
+            words, radius, cb4, S, b, H, cps, n_chunks, out_idx, out_val, slab_off, n_slabs, cap,
+            y);
+    else
+        k_decode_outliers<OUT_DT, HQMQ_GRAN_ELEMENT><<<(unsigned)blocks, OUT_THREADS, 0, stream>>>(
+            words, radius, cb4, S, b, H, cps, n_chunks, out_idx, out_val, slab_off, n_slabs, cap,
+            y);
+    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
 template <int OUT_DT>
-static int launch_o(int mode, bool table, const uint32_t *words, const uint16_t *radius,
-                    const float *cb, uint32_t S, uint32_t b, const uint32_t *out_idx,
-                    const uint16_t *out_val, const uint32_t *slab_off, uint64_t cap, int B, int H,
-                    uint32_t cps, void *y, hqmq_status *st, int sm, cudaStream_t stream) {
-    if (mode == MODE_CHUNK)
-        return launch_m<OUT_DT, MODE_CHUNK>(table, words, radius, cb, S, b, out_idx, out_val,
-                                            slab_off, cap, B, H, cps, y, st, sm, stream);
-    if (mode == MODE_ELEM)
-        return launch_m<OUT_DT, MODE_ELEM>(table, words, radius, cb, S, b, out_idx, out_val,
-                                           slab_off, cap, B, H, cps, y, st, sm, stream);
-    return launch_m<OUT_DT, MODE_NONE>(table, words, radius, cb, S, b, out_idx, out_val, slab_off,
-                                       cap, B, H, cps, y, st, sm, stream);
+static int launch_all(bool table, int gran, const uint32_t *words, const uint16_t *radius,
+                      const float *cb, uint32_t S, uint32_t b, const uint32_t *out_idx,
+                      const uint16_t *out_val, const uint32_t *slab_off, uint64_t cap, int B,
+                      int H, uint32_t cps, void *y, hqmq_status *st, int sm,
+                      cudaStream_t stream) {
+    int rc = table ? launch_main<OUT_DT, true>(words, radius, cb, S, b, B, H, cps, y, st, sm, stream)
+                   : launch_main<OUT_DT, false>(words, radius, cb, S, b, B, H, cps, y, st, sm,
+                                                stream);
+    if (rc != HQMQ_OK || out_idx == nullptr || cap == 0) return rc;
+    return launch_out<OUT_DT>(gran, words, radius, cb, S, b, B, H, cps, out_idx, out_val, slab_off,
+                              cap, y, sm, stream);
 }
 
 }  // namespace hqmq
@@ -234,12 +246,11 @@ extern "C" int hqmq_launch_decode(const uint32_t *words, const uint16_t *radius,
                                   int gran, int B, int H, int T, int D, void *y, int out_dtype,
                                   hqmq_status *st, int sm_count, cudaStream_t stream) {
     using namespace hqmq;
-    uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
-    int mode = out_idx == nullptr ? MODE_NONE : (gran == HQMQ_GRAN_CHUNK ? MODE_CHUNK : MODE_ELEM);
-    bool table = S <= 170;
+    const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
+    const bool table = S <= 170;
     if (out_dtype == HQMQ_BF16)
-        return launch_o<HQMQ_BF16>(mode, table, words, radius, cb, S, b, out_idx, out_val, slab_off,
-                                   cap, B, H, cps, y, st, sm_count, stream);
-    return launch_o<HQMQ_F32>(mode, table, words, radius, cb, S, b, out_idx, out_val, slab_off,
-                              cap, B, H, cps, y, st, sm_count, stream);
+        return launch_all<HQMQ_BF16>(table, gran, words, radius, cb, S, b, out_idx, out_val,
+                                     slab_off, cap, B, H, cps, y, st, sm_count, stream);
+    return launch_all<HQMQ_F32>(table, gran, words, radius, cb, S, b, out_idx, out_val, slab_off,
+                                cap, B, H, cps, y, st, sm_count, stream);
 }

@@ -92,6 +92,31 @@ __device__ __forceinline__ void load_chunk_stream(const void *x, size_t j, float
     }
 }
 
+// Raw chunk storage (8 bytes for bf16, 16 for fp32) to keep several chunks
+// in flight per thread at a low register cost.
+template <int DT> struct RawChunk;
+template <> struct RawChunk<HQMQ_BF16> {
+    uint2 v;
+    __device__ __forceinline__ void load(const void *x, size_t j) {
+        v = __ldcs(reinterpret_cast<const uint2 *>(x) + j);
+    }
+    __device__ __forceinline__ void zero() { v = make_uint2(0u, 0u); }
+    __device__ __forceinline__ float e(int i) const {
+        uint32_t w = (i < 2) ? v.x : v.y;
+        return (i & 1) ? __uint_as_float(w & 0xFFFF0000u) : __uint_as_float(w << 16);
+    }
+};
+template <> struct RawChunk<HQMQ_F32> {
+    float4 v;
+    __device__ __forceinline__ void load(const void *x, size_t j) {
+        v = __ldcs(reinterpret_cast<const float4 *>(x) + j);
+    }
+    __device__ __forceinline__ void zero() { v = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ float e(int i) const {
+        return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+    }
+};
+
 // 2T element p as fp32 (w, i, j, k).
 __device__ __forceinline__ void element_2t(int p, float &a0, float &a1, float &a2, float &a3) {
     if (p < 8) {

@@ -23,8 +23,11 @@ namespace hqmq {
 
 constexpr int HIST_BINS = 2048;
 constexpr int MED_THREADS = 256;
+constexpr int MED_UNROLL = 4;        // chunks in flight per thread
 constexpr int TILE = 4096;           // chunks per extraction tile
 constexpr int EXT_THREADS = 256;
+constexpr int EXT_ROWS = 8;          // rows of EXT_THREADS chunks loaded at once (count)
+constexpr int WR_ROWS = 4;           // the same for the ordered write
 
 struct SelState {
     uint32_t prefix;   // key bits fixed so far
@@ -49,20 +52,36 @@ k_med_hist(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
     constexpr int hi_shift = shift + pass_width(P);      // bits above the digit
     const uint32_t want = P == 0 ? 0u : (state[h].prefix >> hi_shift);
     const uint64_t base = (uint64_t)slab * chunks_per_slab;
-    for (uint32_t c = blockIdx.x * MED_THREADS + threadIdx.x; c < chunks_per_slab;
-         c += gridDim.x * MED_THREADS) {
-        float x0, x1, x2, x3;
-        load_chunk_stream<DT>(x, base + c, x0, x1, x2, x3);
-        if (GRAN == HQMQ_GRAN_CHUNK) {
-            uint32_t key = mag_key(chunk_norm(x0, x1, x2, x3));
-            if (P == 0 || (key >> hi_shift) == want) atomicAdd(&s_hist[(key >> shift) & mask], 1u);
-        } else {
-            uint32_t k4[4] = {mag_key(fabsf(x0)), mag_key(fabsf(x1)), mag_key(fabsf(x2)),
-                              mag_key(fabsf(x3))};
+    const uint32_t stride = gridDim.x * MED_THREADS;
+    for (uint32_t c0 = blockIdx.x * MED_THREADS + threadIdx.x; c0 < chunks_per_slab;
+         c0 += MED_UNROLL * stride) {
+        RawChunk<DT> raw[MED_UNROLL];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                if (P == 0 || (k4[i] >> hi_shift) == want)
-                    atomicAdd(&s_hist[(k4[i] >> shift) & mask], 1u);
+        for (int u = 0; u < MED_UNROLL; ++u) {       // all loads first
+            const uint32_t c = c0 + u * stride;
+            raw[u].zero();
+            if (c < chunks_per_slab) raw[u].load(x, base + c);
+        }
+        float v[MED_UNROLL][4];
+#pragma unroll
+        for (int u = 0; u < MED_UNROLL; ++u)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[u][i] = raw[u].e(i);
+#pragma unroll
+        for (int u = 0; u < MED_UNROLL; ++u) {
+            if (c0 + u * stride >= chunks_per_slab) break;
+            if (GRAN == HQMQ_GRAN_CHUNK) {
+                uint32_t key = mag_key(chunk_norm(v[u][0], v[u][1], v[u][2], v[u][3]));
+                if (P == 0 || (key >> hi_shift) == want)
+                    atomicAdd(&s_hist[(key >> shift) & mask], 1u);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint32_t key = mag_key(fabsf(v[u][i]));
+                    if (P == 0 || (key >> hi_shift) == want)
+                        atomicAdd(&s_hist[(key >> shift) & mask], 1u);
+                }
+            }
         }
     }
     __syncthreads();
@@ -148,10 +167,18 @@ k_extract_count(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
     const uint32_t c1 = min(c0 + TILE, chunks_per_slab);
     const uint64_t base = (uint64_t)slab * chunks_per_slab;
     uint32_t cnt = 0;
-    for (uint32_t c = c0 + threadIdx.x; c < c1; c += EXT_THREADS) {
-        float x0, x1, x2, x3;
-        load_chunk<DT>(x, base + c, x0, x1, x2, x3);
-        cnt += __popc(outlier_mask<GRAN>(x0, x1, x2, x3, th));
+    for (uint32_t cb = c0 + threadIdx.x; cb < c1; cb += EXT_ROWS * EXT_THREADS) {
+        RawChunk<DT> v[EXT_ROWS];
+#pragma unroll
+        for (int u = 0; u < EXT_ROWS; ++u) {
+            const uint32_t c = cb + u * EXT_THREADS;
+            v[u].zero();
+            if (c < c1) v[u].load(x, base + c);
+        }
+#pragma unroll
+        for (int u = 0; u < EXT_ROWS; ++u)
+            if (cb + u * EXT_THREADS < c1)
+                cnt += __popc(outlier_mask<GRAN>(v[u].e(0), v[u].e(1), v[u].e(2), v[u].e(3), th));
     }
     cnt = __reduce_add_sync(FULL, cnt);
     if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = cnt;
@@ -221,7 +248,8 @@ k_extract_write(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
                 uint32_t tiles_per_slab, const float *__restrict__ thr,
                 const uint32_t *__restrict__ tile_off, uint64_t cap,
                 uint32_t *__restrict__ out_idx, uint16_t *__restrict__ out_val, DevStatus *st) {
-    __shared__ uint32_t s_warp[EXT_THREADS / 32];
+    constexpr int NW = EXT_THREADS / 32;
+    __shared__ uint32_t s_tot[WR_ROWS][NW];
     const int slab = blockIdx.y;
     const float th = thr[slab % H];
     const uint32_t c0 = blockIdx.x * TILE;
@@ -230,62 +258,79 @@ k_extract_write(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     uint64_t pos = tile_off[(uint64_t)slab * tiles_per_slab + blockIdx.x];
     unsigned n_sat = 0;
-    for (uint32_t cb = c0; cb < c1; cb += EXT_THREADS) {
-        const uint32_t c = cb + threadIdx.x;
-        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-        uint32_t m = 0;
-        if (c < c1) {
-            load_chunk<DT>(x, base + c, x0, x1, x2, x3);
-            m = outlier_mask<GRAN>(x0, x1, x2, x3, th);
-        }
-        const uint32_t n = __popc(m);
-        uint32_t inc = n;
+    // WR_ROWS rows of EXT_THREADS chunks per batch: row u, thread t holds
+    // chunk cb + u*EXT_THREADS + t, so list order = (row, warp, lane) order
+    for (uint32_t cb = c0; cb < c1; cb += WR_ROWS * EXT_THREADS) {
+        RawChunk<DT> v[WR_ROWS];
+        uint32_t m[WR_ROWS], incl[WR_ROWS];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            uint32_t u = __shfl_up_sync(FULL, inc, o);
-            if (lane >= o) inc += u;
+        for (int u = 0; u < WR_ROWS; ++u) {
+            const uint32_t c = cb + u * EXT_THREADS + threadIdx.x;
+            v[u].zero();
+            if (c < c1) v[u].load(x, base + c);
         }
-        if (lane == 31) s_warp[wid] = inc;
+#pragma unroll
+        for (int u = 0; u < WR_ROWS; ++u) {
+            const uint32_t c = cb + u * EXT_THREADS + threadIdx.x;
+            m[u] = c < c1 ? outlier_mask<GRAN>(v[u].e(0), v[u].e(1), v[u].e(2), v[u].e(3), th)
+                          : 0u;
+            uint32_t inc = __popc(m[u]);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                uint32_t t = __shfl_up_sync(FULL, inc, o);
+                if (lane >= o) inc += t;
+            }
+            incl[u] = inc;
+            if (lane == 31) s_tot[u][wid] = inc;
+        }
         __syncthreads();
-        uint32_t wbase = 0, total = 0;
+        uint32_t run = 0;          // outliers of this batch before (row u, warp wid)
+        uint32_t batch_total = 0;
 #pragma unroll
-        for (int w = 0; w < EXT_THREADS / 32; ++w) {
-            uint32_t sw = s_warp[w];
-            wbase += w < wid ? sw : 0u;
-            total += sw;
-        }
-        uint64_t p = pos + wbase + inc - n;
-        if (m) {
-            const uint64_t j = base + c;
-            if (GRAN == HQMQ_GRAN_CHUNK) {
-                if (p < cap) {
-                    int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-                    uint32_t h0 = f32_to_f16_sat(x0, s0), h1 = f32_to_f16_sat(x1, s1);
-                    uint32_t h2 = f32_to_f16_sat(x2, s2), h3 = f32_to_f16_sat(x3, s3);
-                    n_sat += s0 + s1 + s2 + s3;
-                    out_idx[p] = (uint32_t)j;
-                    uint32_t *vv = reinterpret_cast<uint32_t *>(out_val + p * 4);
-                    vv[0] = h0 | (h1 << 16);
-                    vv[1] = h2 | (h3 << 16);
-                }
-            } else {
-                const float xs[4] = {x0, x1, x2, x3};
+        for (int u = 0; u < WR_ROWS; ++u)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if (m & (1u << i)) {
-                        if (p < cap) {
-                            int s = 0;
-                            out_val[p] = f32_to_f16_sat(xs[i], s);
-                            n_sat += s;
-                            out_idx[p] = (uint32_t)(j * 4 + i);
+            for (int w = 0; w < NW; ++w) batch_total += s_tot[u][w];
+#pragma unroll
+        for (int u = 0; u < WR_ROWS; ++u) {
+            uint32_t before = run;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                uint32_t t = s_tot[u][w];
+                before += w < wid ? t : 0u;
+                run += t;
+            }
+            if (m[u]) {
+                uint64_t p = pos + before + incl[u] - __popc(m[u]);
+                const uint64_t j = base + cb + u * EXT_THREADS + threadIdx.x;
+                if (GRAN == HQMQ_GRAN_CHUNK) {
+                    if (p < cap) {
+                        int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+                        uint32_t h0 = f32_to_f16_sat(v[u].e(0), s0), h1 = f32_to_f16_sat(v[u].e(1), s1);
+                        uint32_t h2 = f32_to_f16_sat(v[u].e(2), s2), h3 = f32_to_f16_sat(v[u].e(3), s3);
+                        n_sat += s0 + s1 + s2 + s3;
+                        out_idx[p] = (uint32_t)j;
+                        uint32_t *vv = reinterpret_cast<uint32_t *>(out_val + p * 4);
+                        vv[0] = h0 | (h1 << 16);
+                        vv[1] = h2 | (h3 << 16);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (m[u] & (1u << i)) {
+                            if (p < cap) {
+                                int sv = 0;
+                                out_val[p] = f32_to_f16_sat(v[u].e(i), sv);
+                                n_sat += sv;
+                                out_idx[p] = (uint32_t)(j * 4 + i);
+                            }
+                            ++p;
                         }
-                        ++p;
                     }
                 }
             }
         }
-        pos += total;
-        __syncthreads();   // s_warp reuse
+        pos += batch_total;
+        __syncthreads();   // s_tot reuse
     }
     unsigned ns = __reduce_add_sync(FULL, n_sat);
     if (lane == 0 && ns && st) status_add(st, HQMQ_FLAG_SATURATED, &st->n_saturated, ns);
