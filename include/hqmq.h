@@ -181,6 +181,39 @@ HQMQ_API int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, 
                 const uint32_t *d_slab_off, uint64_t cap, int gran, int B, int H, int T, int D,
                 void *d_y, int out_dtype, hqmq_status *d_status, void *stream);
 
+/* Exact table-driven search (same results as hqmq_encode).  The best codeword
+ * for x is u times the best codeword for x' = conj(u) x, where u = sign(x_a)
+ * e_a is the unit of 2T along x's largest coordinate; this holds because the
+ * effective codebook {q_p q_s} is closed under left multiplication by 2T, a
+ * group (gist.science/nl, Technische Samenvatting, section 1).  x' lies in
+ * the cube face x'_0 >= |x'_k|; its gnomonic coordinates t = x'_k / x'_0 are
+ * mapped by u = t (A + B t^2) (A = 4/pi in fp32, B = 1 - A) and u is cut into
+ * 32^3 cells; per cell the table lists (up to 8) codewords that can be the
+ * argmax somewhere in the cell, widened by 1e-5 in t to cover rounding: a
+ * codeword is dropped only if it is farther from the cell centre than the best
+ * one by more than twice the cell's angular radius, or if another codeword
+ * beats it at all 8 corners (the score difference is linear in the gnomonic
+ * coordinates).  Cells with more than 8 candidates fall back to the
+ * S-codeword loop.  Supports S in [1, 48]. */
+
+/* Bytes of search table per codebook group (524288), or 0 if S is unsupported. */
+HQMQ_API uint64_t hqmq_search_table_bytes(uint32_t S);
+
+/* Builds the tables of n_groups codebooks: d_codebook[n_groups][S][4] fp32 as
+ * written by hqmq_make_codebook, d_table n_groups * hqmq_search_table_bytes(S)
+ * bytes, both 16-byte aligned.  n_groups <= 65535 per call. */
+HQMQ_API int hqmq_make_search_table(const float *d_codebook, uint32_t S, uint32_t n_groups,
+                                    void *d_table, void *stream);
+
+/* hqmq_encode using the search tables of this call's H heads (d_table = the
+ * tables of the same groups as d_codebook, [H] x hqmq_search_table_bytes(S)).
+ * Arguments, outputs and results as hqmq_encode: indices equal hqmq_encode's
+ * except where two codewords' fp32 scores are within rounding of each other. */
+HQMQ_API int hqmq_encode_lut(const void *d_x, int dtype, int B, int H, int T, int D,
+                             const float *d_codebook, uint32_t S, const void *d_table,
+                             const float *d_thr, int gran, uint32_t *d_idx_words,
+                             uint16_t *d_radius, hqmq_status *d_status, void *stream);
+
 /* Size of the fixed device scratch array of hqmq_outlier_extract_noalloc. */
 #define HQMQ_NOALLOC_SCRATCH_BYTES (1u << 20)
 

@@ -25,6 +25,15 @@ extern "C" int hqmq_launch_outlier_extract(const void *x, int dtype, int B, int 
                                            uint32_t *slab_off, uint64_t cap, void *ws,
                                            hqmq_status *st, int sm_count, cudaStream_t stream);
 
+extern "C" uint64_t hqmq_lut_bytes_per_group(uint32_t S);
+extern "C" int hqmq_launch_build_search_table(const float *cb, uint32_t S, uint32_t n_groups,
+                                              void *table, cudaStream_t stream);
+extern "C" int hqmq_launch_encode_lut(const void *x, int dtype, int B, int H, int T, int D,
+                                      const float *cb, uint32_t S, uint32_t b, const void *table,
+                                      const float *thr, int gran, uint32_t *words,
+                                      uint16_t *radius, hqmq_status *st, int sm_count,
+                                      cudaStream_t stream);
+
 namespace {
 
 constexpr uint32_t S_MAX = 65535;
@@ -158,6 +167,34 @@ int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, const flo
     return hqmq_launch_decode(d_idx_words, d_radius, d_codebook, S, hqmq_index_bits(S), d_out_idx,
                               d_out_val, d_slab_off, cap, gran, B, H, T, D, d_y, out_dtype,
                               d_status, sm, (cudaStream_t)stream);
+}
+
+uint64_t hqmq_search_table_bytes(uint32_t S) { return hqmq_lut_bytes_per_group(S); }
+
+int hqmq_make_search_table(const float *d_codebook, uint32_t S, uint32_t n_groups,
+                           void *d_table, void *stream) {
+    if (hqmq_lut_bytes_per_group(S) == 0 || n_groups < 1 || n_groups > 65535) return HQMQ_ERR_ARG;
+    if (!d_codebook || !d_table) return HQMQ_ERR_ARG;
+    if (!aligned(d_codebook, 16) || !aligned(d_table, 16)) return HQMQ_ERR_ALIGN;
+    return hqmq_launch_build_search_table(d_codebook, S, n_groups, d_table, (cudaStream_t)stream);
+}
+
+int hqmq_encode_lut(const void *d_x, int dtype, int B, int H, int T, int D,
+                    const float *d_codebook, uint32_t S, const void *d_table, const float *d_thr,
+                    int gran, uint32_t *d_idx_words, uint16_t *d_radius, hqmq_status *d_status,
+                    void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
+    if (hqmq_lut_bytes_per_group(S) == 0) return HQMQ_ERR_ARG;
+    if (!d_x || !d_codebook || !d_table || !d_idx_words || !d_radius) return HQMQ_ERR_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_codebook, 16) || !aligned(d_table, 16) ||
+        !aligned(d_idx_words, 4) || !aligned(d_radius, 4) || !aligned(d_thr, 4) ||
+        !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_encode_lut(d_x, dtype, B, H, T, D, d_codebook, S, hqmq_index_bits(S),
+                                  d_table, d_thr, gran, d_idx_words, d_radius, d_status, sm,
+                                  (cudaStream_t)stream);
 }
 
 }  // extern "C"

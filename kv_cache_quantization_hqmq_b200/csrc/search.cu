@@ -1,0 +1,454 @@
+// search.cu -- exact local search for the HQMQ encode (table-driven).
+//
+// The encode snaps a chunk x to the codeword c = q_p q_s of the 24 S-word
+// effective codebook with the largest <x, c> (gist.science/nl, Technische
+// Samenvatting, section 1).  The S-codeword loop of encode.cu costs one
+// quaternion product per secondary codeword.  This file replaces it by a
+// lookup of the few codewords that can win in the neighbourhood of x:
+//
+// 1. Folding.  Let a be the coordinate of largest |x_a| and u = sign(x_a) e_a
+//    one of the 8 units +-1, +-i, +-j, +-k of 2T.  x' = conj(u) x (a signed
+//    permutation of x, exact) has x'_0 = |x_a| >= |x'_k|.  Because the
+//    codebook C = {q_p q_s} is closed under left multiplication by 2T (2T is
+//    a group, same section), <x, c> = <x', conj(u) c> and conj(u) c runs over
+//    C as c does: the best codeword for x is u times the best for x'.
+// 2. Cells.  x' lies in the cube face x'_0 >= |x'_k|; its gnomonic
+//    coordinates t_k = x'_k / x'_0 lie in [-1, 1]^3.  They are mapped by the
+//    monotone u(t) = t (A + B t^2) (A = 4/pi, B = 1 - A, so u(+-1) = +-1), which
+//    roughly equalises the angular size of the cells, and u is cut into G^3
+//    cells.
+// 3. Candidates.  For each cell (grown by DELTA on every side to absorb fp32
+//    rounding of t), a codeword c is kept unless (i) its angle from the cell
+//    centre exceeds the best angle there by more than twice the cell's angular
+//    radius, or (ii) another codeword c* beats it at all 8 corners of the cell:
+//    <(1, t), c* - c> is linear in t, so c* beats c on the whole cell iff it
+//    does at the corners.  Both tests only drop codewords that cannot be the
+//    argmax anywhere in the cell, so the list is a superset of the possible
+//    winners.  Up to SLOTS survivors are stored; a cell with more is marked
+//    OVERFLOW and its chunks use the S-codeword loop.
+// 4. Encode.  Score the cell's candidates with fp32 <x', c'>, keep the best
+//    (equal scores: the lowest index after mapping back), map back
+//    p = index(u q_p').  The tables stay in global memory (L2-resident: 512 KB
+//    per head); candidate codewords come from a shared-memory copy of the 24 S
+//    codewords replicated 8 times so that the 8 lanes of each quarter-warp
+//    read 8 different bank groups (no conflicts).
+#include "hqmq_device.cuh"
+
+namespace hqmq {
+
+constexpr int LUT_G = 32;
+constexpr int LUT_CELLS = LUT_G * LUT_G * LUT_G;   // 32768 cells, 512 KB per group
+constexpr float MAP_A = 1.27323954f;               // 4 / pi (fp32)
+constexpr float MAP_B = 1.0f - MAP_A;              // exact (Sterbenz)
+constexpr int LUT_SLOTS = 8;
+constexpr uint32_t LUT_EMPTY = 0xFFFFu;
+constexpr uint32_t LUT_OVERFLOW = 0xFFFEu;
+constexpr uint32_t LUT_MAX_S = 48;                // 24 S codeword ids fit in 16 bits;
+                                                  // shared memory fits 8 copies (144 KB)
+constexpr double LUT_DELTA = 1e-5;                // cell growth in t (fp32 error ~1e-7)
+constexpr int BUILD_THREADS = 128;
+constexpr int BUILD_MAXC = 64;                     // candidates kept before pruning
+constexpr int ENC_THREADS = 1024;
+
+// Inverse of u(t) = t (A + B t^2) on [-1, 1] (monotone: u' >= A + 3B > 0), by
+// bisection in fp64.
+__device__ double t_of_u(double u) {
+    if (u <= -1.0) return -1.0;
+    if (u >= 1.0) return 1.0;
+    double lo = -1.0, hi = 1.0;
+    const double a = (double)MAP_A, b = (double)MAP_B;
+    for (int it = 0; it < 64; ++it) {
+        const double m = 0.5 * (lo + hi);
+        if (m * (a + b * m * m) < u) lo = m; else hi = m;
+    }
+    return 0.5 * (lo + hi);
+}
+
+// ---------------------------------------------------------------------------
+// table build: one thread per (cell, group)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(BUILD_THREADS)
+k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__restrict__ tables) {
+    extern __shared__ double4 s_cw[];                 // [24 S] codewords in fp64 (exact copies)
+    const uint32_t g = blockIdx.y;
+    const uint32_t n_words = 24u * S;
+    for (uint32_t i = threadIdx.x; i < n_words; i += BUILD_THREADS) {
+        float4 c = codeword((int)(i % 24u), cb_all[(size_t)g * S + i / 24u]);
+        s_cw[i] = make_double4(c.x, c.y, c.z, c.w);
+    }
+    __syncthreads();
+    const uint32_t cell = blockIdx.x * BUILD_THREADS + threadIdx.x;
+    if (cell >= (uint32_t)LUT_CELLS) return;
+    const int ic[3] = {(int)(cell / (LUT_G * LUT_G)), (int)((cell / LUT_G) % LUT_G),
+                       (int)(cell % LUT_G)};
+    double lo[3], hi[3], mid[3];
+    for (int k = 0; k < 3; ++k) {
+        lo[k] = t_of_u(-1.0 + 2.0 * ic[k] / LUT_G) - LUT_DELTA;
+        hi[k] = t_of_u(-1.0 + 2.0 * (ic[k] + 1) / LUT_G) + LUT_DELTA;
+        mid[k] = 0.5 * (lo[k] + hi[k]);
+    }
+    // corners (unnormalised (1, t)) and the centre direction
+    double cor[8][4];
+    for (int q = 0; q < 8; ++q) {
+        cor[q][0] = 1.0;
+        for (int k = 0; k < 3; ++k) cor[q][k + 1] = ((q >> k) & 1) ? hi[k] : lo[k];
+    }
+    double cn = sqrt(1.0 + mid[0] * mid[0] + mid[1] * mid[1] + mid[2] * mid[2]);
+    const double uc[4] = {1.0 / cn, mid[0] / cn, mid[1] / cn, mid[2] / cn};
+    double cos_rho = 1.0;                              // angular radius of the cell
+    for (int q = 0; q < 8; ++q) {
+        double n = sqrt(cor[q][0] * cor[q][0] + cor[q][1] * cor[q][1] + cor[q][2] * cor[q][2] +
+                        cor[q][3] * cor[q][3]);
+        double d = (uc[0] * cor[q][0] + uc[1] * cor[q][1] + uc[2] * cor[q][2] +
+                    uc[3] * cor[q][3]) / n;
+        cos_rho = fmin(cos_rho, d);
+    }
+    double best = -2.0;
+    for (uint32_t i = 0; i < n_words; ++i) {
+        double4 c = s_cw[i];
+        best = fmax(best, uc[0] * c.x + uc[1] * c.y + uc[2] * c.z + uc[3] * c.w);
+    }
+    const double rho = acos(fmin(1.0, cos_rho));
+    const double lim = acos(fmax(-1.0, fmin(1.0, best))) + 2.0 * rho + 1e-9;
+    const double cos_lim = lim >= 3.141592653589793 ? -2.0 : cos(lim) - 1e-12;
+    // (i) angle prefilter
+    uint32_t cand[BUILD_MAXC];
+    double cdot[BUILD_MAXC];
+    int nc = 0;
+    bool overflow = false;
+    for (uint32_t i = 0; i < n_words; ++i) {
+        double4 c = s_cw[i];
+        double d = uc[0] * c.x + uc[1] * c.y + uc[2] * c.z + uc[3] * c.w;
+        if (d >= cos_lim) {
+            if (nc == BUILD_MAXC) { overflow = true; break; }
+            cand[nc] = i;
+            cdot[nc] = d;
+            ++nc;
+        }
+    }
+    uint32_t keep[LUT_SLOTS];
+    double kdot[LUT_SLOTS];
+    int nk = 0;
+    if (!overflow) {
+        // (ii) dominance on the corners
+        for (int j = 0; j < nc && !overflow; ++j) {
+            const double4 cj = s_cw[cand[j]];
+            bool dominated = false;
+            for (int k = 0; k < nc && !dominated; ++k) {
+                if (k == j) continue;
+                const double4 ck = s_cw[cand[k]];
+                const double d0 = ck.x - cj.x, d1 = ck.y - cj.y, d2 = ck.z - cj.z,
+                             d3 = ck.w - cj.w;
+                bool all = true;
+                for (int q = 0; q < 8 && all; ++q) {
+                    double v = cor[q][0] * d0 + cor[q][1] * d1 + cor[q][2] * d2 + cor[q][3] * d3;
+                    all = v > 1e-12;
+                }
+                dominated = all;
+            }
+            if (!dominated) {
+                if (nk == LUT_SLOTS) { overflow = true; break; }
+                // insertion by descending centre score: the likely winner first
+                int pos = nk++;
+                while (pos > 0 && kdot[pos - 1] < cdot[j]) {
+                    keep[pos] = keep[pos - 1];
+                    kdot[pos] = kdot[pos - 1];
+                    --pos;
+                }
+                keep[pos] = cand[j];
+                kdot[pos] = cdot[j];
+            }
+        }
+    }
+    uint32_t slot[LUT_SLOTS];
+    for (int q = 0; q < LUT_SLOTS; ++q) slot[q] = q < nk ? keep[q] : LUT_EMPTY;
+    if (overflow) slot[0] = LUT_OVERFLOW;
+    tables[(size_t)g * LUT_CELLS + cell] =
+        make_uint4(slot[0] | (slot[1] << 16), slot[2] | (slot[3] << 16),
+                   slot[4] | (slot[5] << 16), slot[6] | (slot[7] << 16));
+}
+
+// ---------------------------------------------------------------------------
+// encode with the table
+// ---------------------------------------------------------------------------
+
+// Index (0..23) of the 2T element a*b for a, b given by index (exact: the
+// entries are 0, +-1, +-1/2 and every product of two of them is exact).
+__device__ int mul_2t(int pa, int pb) {
+    float a0, a1, a2, a3, b0, b1, b2, b3;
+    element_2t(pa, a0, a1, a2, a3);
+    element_2t(pb, b0, b1, b2, b3);
+    const float w = a0 * b0 - a1 * b1 - a2 * b2 - a3 * b3;
+    const float x = a0 * b1 + a1 * b0 + a2 * b3 - a3 * b2;
+    const float y = a0 * b2 - a1 * b3 + a2 * b0 + a3 * b1;
+    const float z = a0 * b3 + a1 * b2 - a2 * b1 + a3 * b0;
+    for (int p = 0; p < 24; ++p) {
+        float c0, c1, c2, c3;
+        element_2t(p, c0, c1, c2, c3);
+        if (c0 == w && c1 == x && c2 == y && c3 == z) return p;
+    }
+    return 0;
+}
+
+// Face of x: the unit u = sign(x_a) e_a (2T index 2a + sign) and x' = conj(u) x.
+__device__ __forceinline__ int fold(float x0, float x1, float x2, float x3, float &y0, float &y1,
+                                    float &y2, float &y3) {
+    const float a0 = fabsf(x0), a1 = fabsf(x1), a2 = fabsf(x2), a3 = fabsf(x3);
+    const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+    const int a = (a0 == m) ? 0 : (a1 == m) ? 1 : (a2 == m) ? 2 : 3;
+    // conj(e_a) x for a = 0..3: x, (x1,-x0,x3,-x2), (x2,-x3,-x0,x1), (x3,x2,-x1,-x0)
+    if (a == 0) { y0 = x0; y1 = x1; y2 = x2; y3 = x3; }
+    else if (a == 1) { y0 = x1; y1 = -x0; y2 = x3; y3 = -x2; }
+    else if (a == 2) { y0 = x2; y1 = -x3; y2 = -x0; y3 = x1; }
+    else { y0 = x3; y1 = x2; y2 = -x1; y3 = -x0; }
+    const bool neg = y0 < 0.0f;
+    if (neg) { y0 = -y0; y1 = -y1; y2 = -y2; y3 = -y3; }
+    return 2 * a + (neg ? 1 : 0);
+}
+
+__device__ __forceinline__ int cell_coord(float t) {
+    const float u = t * __fmaf_rn(MAP_B, t * t, MAP_A);
+    int i = (int)((u + 1.0f) * (0.5f * LUT_G));
+    return i < 0 ? 0 : (i > LUT_G - 1 ? LUT_G - 1 : i);
+}
+
+// S-codeword loop for one chunk (used for OVERFLOW cells); same result rules
+// as encode.cu: ties to the lowest s, then the closed-form 2T choice.
+__device__ __forceinline__ float dot_conj_score2(float x0, float x1, float x2, float x3, float4 q,
+                                                 float &y0, float &y1, float &y2, float &y3) {
+    y0 = __fmaf_rn(x3, q.w, __fmaf_rn(x2, q.z, __fmaf_rn(x1, q.y, __fmul_rn(x0, q.x))));
+    y1 = __fmaf_rn(x3, q.z, __fmaf_rn(-x2, q.w, __fmaf_rn(x1, q.x, __fmul_rn(-x0, q.y))));
+    y2 = __fmaf_rn(-x3, q.y, __fmaf_rn(x2, q.x, __fmaf_rn(x1, q.w, __fmul_rn(-x0, q.z))));
+    y3 = __fmaf_rn(x3, q.x, __fmaf_rn(x2, q.y, __fmaf_rn(-x1, q.z, __fmul_rn(-x0, q.w))));
+    const float a0 = fabsf(y0), a1 = fabsf(y1), a2 = fabsf(y2), a3 = fabsf(y3);
+    const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+    const float sum = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
+    return fmaxf(__fadd_rn(m, m), sum);
+}
+
+__device__ __forceinline__ int closest_2t_of(float y0, float y1, float y2, float y3) {
+    const float a0 = fabsf(y0), a1 = fabsf(y1), a2 = fabsf(y2), a3 = fabsf(y3);
+    const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+    const float sum = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
+    if (__fadd_rn(m, m) >= sum) {
+        const int ax = (a0 == m) ? 0 : (a1 == m) ? 1 : (a2 == m) ? 2 : 3;
+        const float ya = ax == 0 ? y0 : ax == 1 ? y1 : ax == 2 ? y2 : y3;
+        return 2 * ax + (ya < 0.0f ? 1 : 0);
+    }
+    return 8 + (y0 < 0.0f ? 1 : 0) + (y1 < 0.0f ? 2 : 0) + (y2 < 0.0f ? 4 : 0) +
+           (y3 < 0.0f ? 8 : 0);
+}
+
+__device__ uint32_t sloop_index(float x0, float x1, float x2, float x3,
+                                const float4 *__restrict__ cb, uint32_t S) {
+    float best = -1.0f;
+    uint32_t bs = 0;
+    float y0, y1, y2, y3;
+    for (uint32_t s = 0; s < S; ++s) {
+        const float sc = dot_conj_score2(x0, x1, x2, x3, __ldg(cb + s), y0, y1, y2, y3);
+        if (sc > best) { best = sc; bs = s; }
+    }
+    dot_conj_score2(x0, x1, x2, x3, __ldg(cb + bs), y0, y1, y2, y3);
+    return bs * 24u + (uint32_t)closest_2t_of(y0, y1, y2, y3);
+}
+
+__device__ __forceinline__ uint64_t shfl64(uint64_t v, int src) {
+    const uint32_t lo = __shfl_sync(FULL, (uint32_t)v, src);
+    const uint32_t hi = __shfl_sync(FULL, (uint32_t)(v >> 32), src);
+    return ((uint64_t)hi << 32) | lo;
+}
+
+__device__ __forceinline__ uint64_t shfl64_down(uint64_t v, int d) {
+    const uint32_t lo = __shfl_down_sync(FULL, (uint32_t)v, d);
+    const uint32_t hi = __shfl_down_sync(FULL, (uint32_t)(v >> 32), d);
+    return ((uint64_t)hi << 32) | lo;
+}
+
+// Packs the warp's 32 b-bit indices (lane k = chunk k) LSB-first into b words.
+// Each lane first gathers the 64-bit stream window starting at its own chunk
+// (k, k+1, ..., by doubling), then lane w < b takes word w from the window of
+// the chunk where that word starts.  Needs b in [5, 21].
+__device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b, int lane,
+                                             uint32_t *__restrict__ dst) {
+    uint64_t v = idx;
+    const uint32_t n1 = __shfl_down_sync(FULL, idx, 1);
+    if (lane + 1 < 32) v |= (uint64_t)n1 << b;
+    const uint64_t v2 = shfl64_down(v, 2);
+    if (lane + 2 < 32) v |= v2 << (2 * b);                 // 2b <= 42
+    const uint64_t v4 = shfl64_down(v, 4);
+    if (lane + 4 < 32 && 4 * b < 64) v |= v4 << (4 * b);
+    const int k0 = (32 * lane) / (int)b;
+    const int o = 32 * lane - k0 * (int)b;                   // < b, and o + 32 <= 64
+    const uint64_t vk = shfl64(v, k0 & 31);
+    if (lane < (int)b) dst[lane] = (uint32_t)(vk >> o);
+}
+
+template <int DT>
+__global__ void __launch_bounds__(ENC_THREADS, 1)
+k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint64_t n_groups,
+             const float4 *__restrict__ cb_all, uint32_t S, uint32_t b,
+             const uint4 *__restrict__ tables, const float *__restrict__ thr, int gran,
+             uint32_t *__restrict__ words, uint16_t *__restrict__ radius, DevStatus *st) {
+    extern __shared__ float4 s_tab[];                              // [24 S][8] replicated
+    __shared__ uint8_t s_mul[8][24];                               // u * q_p' for the 8 units
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n_warps = ENC_THREADS / 32;
+    const uint32_t n_words = 24u * S;
+    const uint32_t lane7 = (uint32_t)(lane & 7);
+    for (int i = threadIdx.x; i < 8 * 24; i += ENC_THREADS)
+        s_mul[i / 24][i % 24] = (uint8_t)mul_2t(i / 24, i % 24);
+
+    // this CTA's contiguous range of packing groups (32 chunks each)
+    const uint64_t g_begin = n_groups * blockIdx.x / gridDim.x;
+    const uint64_t g_end = n_groups * (blockIdx.x + 1) / gridDim.x;
+    int cur_head = -1;
+    unsigned n_nf = 0, n_sat = 0;
+    for (uint64_t seg = g_begin; seg < g_end;) {
+        const uint64_t slab = seg / groups_per_slab;
+        const uint64_t seg_end = min(g_end, (slab + 1) * groups_per_slab);
+        const int h = (int)(slab % (uint64_t)H);
+        const float4 *cb = cb_all + (size_t)h * S;
+        const uint4 *tb = tables + (size_t)h * LUT_CELLS;
+        if (h != cur_head) {                        // (block-uniform)
+            __syncthreads();
+            for (uint32_t i = threadIdx.x; i < n_words * 8; i += ENC_THREADS) {
+                const uint32_t id = i >> 3;
+                s_tab[i] = codeword((int)(id % 24u), __ldg(cb + id / 24u));
+            }
+            __syncthreads();
+            cur_head = h;
+        }
+        const float th = thr ? __ldg(thr + h) : 0.0f;
+        uint64_t G = seg + warp;
+        RawChunk<DT> nxt;                           // x of the next group, loaded early
+        if (G < seg_end) nxt.load(x, G * 32 + lane);
+        for (; G < seg_end; G += n_warps) {
+            const RawChunk<DT> cur = nxt;
+            if (G + n_warps < seg_end) nxt.load(x, (G + n_warps) * 32 + lane);
+            float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
+            float r = chunk_norm(x0, x1, x2, x3);
+            if (thr) {
+                if (gran == HQMQ_GRAN_CHUNK) {
+                    if (r > th) { x0 = x1 = x2 = x3 = 0.0f; r = 0.0f; }
+                } else {
+                    if (fabsf(x0) > th) x0 = 0.0f;
+                    if (fabsf(x1) > th) x1 = 0.0f;
+                    if (fabsf(x2) > th) x2 = 0.0f;
+                    if (fabsf(x3) > th) x3 = 0.0f;
+                    r = chunk_norm(x0, x1, x2, x3);
+                }
+            }
+            const bool finite = r == r && r != __int_as_float(0x7F800000);
+            const bool search = finite && r > 0.0f;
+            // every lane takes part in the candidate loop (it votes); lanes
+            // without a search carry an all-empty record
+            float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+            int pu = 0;
+            uint4 rec = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+            if (search) {
+                pu = fold(x0, x1, x2, x3, y0, y1, y2, y3);
+                float inv;
+                asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(y0));   // cells are widened
+                const int cell = (cell_coord(y1 * inv) * LUT_G + cell_coord(y2 * inv)) * LUT_G +
+                                 cell_coord(y3 * inv);
+                rec = __ldg(tb + cell);
+            }
+            const bool fallback = (rec.x & 0xFFFFu) == LUT_OVERFLOW;
+            if (fallback) rec = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+            const uint32_t sl[4] = {rec.x, rec.y, rec.z, rec.w};
+            const uint32_t id0 = rec.x & 0xFFFFu;
+            float best = __int_as_float(0xFF800000);     // -inf
+            uint32_t bid = 0;
+            uint32_t bmap = 0xFFFFFFFFu;
+#pragma unroll
+            for (int k = 0; k < LUT_SLOTS; ++k) {
+                const uint32_t idk = (sl[k >> 1] >> ((k & 1) * 16)) & 0xFFFFu;
+                if (!__any_sync(FULL, idk != LUT_EMPTY)) break;
+                // a lane whose list is shorter re-scores its first candidate
+                const uint32_t id = idk != LUT_EMPTY ? idk : id0;
+                if (id0 != LUT_EMPTY) {
+                    const float4 c = s_tab[(id << 3) | lane7];
+                    const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z,
+                                     __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
+                    if (sc > best) {
+                        best = sc; bid = id; bmap = 0xFFFFFFFFu;
+                    } else if (sc == best && id != bid) {   // exact tie: lowest original index
+                        if (bmap == 0xFFFFFFFFu)
+                            bmap = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
+                        const uint32_t m = (id / 24u) * 24u + s_mul[pu][id % 24u];
+                        if (m < bmap) { bid = id; bmap = m; }
+                    }
+                }
+            }
+            uint32_t idx = 0;
+            if (search && !fallback) idx = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
+            if (fallback) idx = sloop_index(x0, x1, x2, x3, cb, S);
+            uint16_t rh;
+            if (!finite) {
+                rh = 0x7E00u;
+                ++n_nf;
+            } else {
+                int sat = 0;
+                rh = f32_to_f16_sat(r, sat);
+                n_sat += sat;
+            }
+            radius[G * 32 + lane] = rh;
+            pack_group32(idx, b, lane, words + G * b);
+        }
+        seg = seg_end;
+    }
+    const unsigned nf = __reduce_add_sync(FULL, n_nf);
+    const unsigned ns = __reduce_add_sync(FULL, n_sat);
+    if (lane == 0 && st) {
+        if (nf) status_add(st, HQMQ_FLAG_NONFINITE, &st->n_nonfinite, nf);
+        if (ns) status_add(st, HQMQ_FLAG_SATURATED, &st->n_saturated, ns);
+    }
+}
+
+static size_t enc_smem_bytes(uint32_t S) { return (size_t)24 * S * 8 * sizeof(float4); }
+
+}  // namespace hqmq
+
+extern "C" uint64_t hqmq_lut_bytes_per_group(uint32_t S) {
+    if (S < 1 || S > hqmq::LUT_MAX_S) return 0;
+    return (uint64_t)hqmq::LUT_CELLS * sizeof(uint4);
+}
+
+extern "C" int hqmq_launch_build_search_table(const float *cb, uint32_t S, uint32_t n_groups,
+                                              void *table, cudaStream_t stream) {
+    using namespace hqmq;
+    const size_t smem = (size_t)24 * S * sizeof(double4);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(k_build_search_table, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return HQMQ_ERR_CUDA;
+    dim3 grid(LUT_CELLS / BUILD_THREADS, n_groups);
+    k_build_search_table<<<grid, BUILD_THREADS, smem, stream>>>(
+        reinterpret_cast<const float4 *>(cb), S, reinterpret_cast<uint4 *>(table));
+    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}
+
+extern "C" int hqmq_launch_encode_lut(const void *x, int dtype, int B, int H, int T, int D,
+                                      const float *cb, uint32_t S, uint32_t b, const void *table,
+                                      const float *thr, int gran, uint32_t *words,
+                                      uint16_t *radius, hqmq_status *st, int sm_count,
+                                      cudaStream_t stream) {
+    using namespace hqmq;
+    const uint32_t gps = (uint32_t)(((uint64_t)T * D / 4) / 32);
+    const uint64_t n_groups = (uint64_t)B * H * gps;
+    const size_t smem = enc_smem_bytes(S);
+    auto kern = dtype == HQMQ_BF16 ? k_encode_lut<HQMQ_BF16> : k_encode_lut<HQMQ_F32>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return HQMQ_ERR_CUDA;
+    // one CTA per SM, each a contiguous share of the call's groups
+    uint64_t ctas = (uint64_t)sm_count;
+    const uint64_t want = (n_groups + 31) / 32;
+    if (ctas > want) ctas = want;
+    if (ctas < 1) ctas = 1;
+    kern<<<(unsigned)ctas, ENC_THREADS, smem, stream>>>(
+        x, H, gps, n_groups, reinterpret_cast<const float4 *>(cb), S, b,
+        reinterpret_cast<const uint4 *>(table), thr, gran, words, radius,
+        reinterpret_cast<DevStatus *>(st));
+    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}

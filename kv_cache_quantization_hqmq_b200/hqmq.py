@@ -50,6 +50,9 @@ _SIGS = {
     "hqmq_decode": (_I, [_P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P, _I, _P, _P]),
     "hqmq_outlier_extract_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P,
                                           _U64, _P, _P]),
+    "hqmq_search_table_bytes": (_U64, [_U32]),
+    "hqmq_make_search_table": (_I, [_P, _U32, _U32, _P, _P]),
+    "hqmq_encode_lut": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _P, _I, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -146,6 +149,26 @@ def hqmq_encode(x, codebook, S, thr, gran, idx_words, radius, status=None, strea
     B, H, T, D = _shape4(x)
     _check("hqmq_encode", _lib.hqmq_encode(
         _ptr(x), _dtype_code(x), B, H, T, D, _ptr(codebook), S, _ptr(thr), gran,
+        _ptr(idx_words), _ptr(radius), _ptr(status), _stream(stream)))
+
+
+def hqmq_search_table_bytes(S):
+    return int(_lib.hqmq_search_table_bytes(S))
+
+
+def hqmq_make_search_table(codebook, S, n_groups, table, stream=None):
+    """table: uint8 device tensor of n_groups * hqmq_search_table_bytes(S) bytes."""
+    assert table.numel() * table.element_size() >= n_groups * hqmq_search_table_bytes(S)
+    _check("hqmq_make_search_table", _lib.hqmq_make_search_table(
+        _ptr(codebook), S, n_groups, _ptr(table), _stream(stream)))
+    return table
+
+
+def hqmq_encode_lut(x, codebook, S, table, thr, gran, idx_words, radius, status=None,
+                    stream=None):
+    B, H, T, D = _shape4(x)
+    _check("hqmq_encode_lut", _lib.hqmq_encode_lut(
+        _ptr(x), _dtype_code(x), B, H, T, D, _ptr(codebook), S, _ptr(table), _ptr(thr), gran,
         _ptr(idx_words), _ptr(radius), _ptr(status), _stream(stream)))
 
 

@@ -69,11 +69,23 @@ def gpu_med3(x_dev, C=3.0, gran=0, cap=None):
                 status=hqmq.read_status(st))
 
 
-def gpu_encode(x_dev, cb_dev, S, thr_dev=None, gran=0):
+def gpu_search_table(cb_dev, S, n_groups):
+    t = torch.empty(n_groups * hqmq.hqmq_search_table_bytes(S), dtype=torch.uint8, device="cuda")
+    hqmq.hqmq_make_search_table(cb_dev, S, n_groups, t)
+    return t
+
+
+def gpu_encode(x_dev, cb_dev, S, thr_dev=None, gran=0, encoder="sloop"):
+    """encoder: "sloop" (hqmq_encode) or "lut" (hqmq_encode_lut with tables
+    built here from the same codebook)."""
     B, H, T, D = x_dev.shape
     words, radius = hqmq.alloc_codes(B, H, T, D, S)
     st = hqmq.new_status()
-    hqmq.hqmq_encode(x_dev, cb_dev, S, thr_dev, gran, words, radius, st)
+    if encoder == "lut":
+        table = gpu_search_table(cb_dev, S, H)
+        hqmq.hqmq_encode_lut(x_dev, cb_dev, S, table, thr_dev, gran, words, radius, st)
+    else:
+        hqmq.hqmq_encode(x_dev, cb_dev, S, thr_dev, gran, words, radius, st)
     torch.cuda.synchronize()
     return words, radius, hqmq.read_status(st)
 

@@ -39,8 +39,12 @@ def x_to_dev(x_np):
     return bf16_dev(x_np) if x_np.dtype == np.uint16 else dev(x_np)
 
 
-def full_call(oracle, x_np, S, cb_np, med3=False, C=3.0, gran=0, name="", check_e2e=True):
-    """Whole-call parity: Med3x (optional), encode, decode."""
+ENCODERS = ["sloop", "lut"]
+
+
+def full_call(oracle, x_np, S, cb_np, med3=False, C=3.0, gran=0, name="", check_e2e=True,
+              encoder="sloop"):
+    """Whole-call parity: Med3x (optional), encode (S-loop or table search), decode."""
     B, H, T, D = x_np.shape
     xd = x_to_dev(x_np)
     cbd = dev(cb_np.reshape(-1))
@@ -48,11 +52,11 @@ def full_call(oracle, x_np, S, cb_np, med3=False, C=3.0, gran=0, name="", check_
     if med3:
         med = gpu_med3(xd, C, gran)
         thr_o, oi_o, ov_o, so_o, n_o = check_med3(oracle, x_np, med, C, gran)
-    words, radius, st = gpu_encode(xd, cbd, S, med["thr"] if med3 else None, gran)
+    words, radius, st = gpu_encode(xd, cbd, S, med["thr"] if med3 else None, gran, encoder)
     n_chunks = B * H * T * D // 4
     gi = unpack_indices(to_host(words), S, n_chunks)
     n, mm, near = check_codes(oracle, x_np, cb_np, S, gi, to_host(radius), thr=thr_o, gran=gran)
-    report(name, n, mm, near)
+    report("%s [%s]" % (name, encoder), n, mm, near)
     # decode parity on the ORACLE's codes: bit-exact, bf16 and fp32 outputs
     ow, orad, _, _, _ = oracle.encode(x_np, cb_np, S, thr=thr_o, gran=gran)
     owd, orad_d = dev(ow.view(np.int32)), dev(orad.view(np.int16))
@@ -100,38 +104,44 @@ def test_codebook_matches_oracle(oracle, S, G):
 
 
 # ------------------------------------------------------------------ whole calls
-def test_tiny_config(oracle):
+@pytest.mark.parametrize("encoder", ENCODERS)
+def test_tiny_config(oracle, encoder):
     w = W.WORKLOADS["tiny"]
     cb = oracle.make_codebook(w.codebook_seed, w.S, w.n_groups)
     for role in (0, 1):
         x = W.as_numpy_bits(W.make_call_input(w, 0, role))
         g0 = W.group0(0, role, w.heads)
-        full_call(oracle, x, w.S, cb[g0:g0 + w.heads], name="tiny role %d" % role)
+        full_call(oracle, x, w.S, cb[g0:g0 + w.heads], name="tiny role %d" % role,
+                  encoder=encoder)
 
 
+@pytest.mark.parametrize("encoder", ENCODERS)
 @pytest.mark.parametrize("layer", [0, 31])
-def test_llama8b_short(oracle, layer):
+def test_llama8b_short(oracle, layer, encoder):
     w = W.WORKLOADS["llama3_8b"]
     x = W.as_numpy_bits(W.make_call_input(w, layer, 1, tokens=256))
     cb = oracle.make_codebook(w.codebook_seed, w.S, w.heads, W.group0(layer, 1, w.heads))
-    full_call(oracle, x, w.S, cb, name="llama8b L%d T256" % layer)
+    full_call(oracle, x, w.S, cb, name="llama8b L%d T256" % layer, encoder=encoder)
 
 
+@pytest.mark.parametrize("encoder", ENCODERS)
 @pytest.mark.parametrize("gran", [0, 1])
-def test_qwen_med3_short(oracle, gran):
+def test_qwen_med3_short(oracle, gran, encoder):
     w = W.WORKLOADS["qwen_outlier"]
     x = W.as_numpy_bits(W.make_call_input(w, 3, 0, tokens=512))
     cb = oracle.make_codebook(w.codebook_seed, w.S, w.heads, W.group0(3, 0, w.heads))
-    r = full_call(oracle, x, w.S, cb, med3=True, gran=gran, name="qwen T512 gran %d" % gran)
+    r = full_call(oracle, x, w.S, cb, med3=True, gran=gran, name="qwen T512 gran %d" % gran,
+                  encoder=encoder)
     assert r["med"]["status"]["n_outliers"] > 0
 
 
+@pytest.mark.parametrize("encoder", ENCODERS)
 @pytest.mark.parametrize("S", [8, 32])
-def test_mha_batched_med3_short(oracle, S):
+def test_mha_batched_med3_short(oracle, S, encoder):
     w = W.WORKLOADS["mha7b_s8"]
     x = W.as_numpy_bits(W.make_call_input(w, 5, 1, tokens=64, batch=3))
     cb = oracle.make_codebook(w.codebook_seed, S, w.heads, W.group0(5, 1, w.heads))
-    full_call(oracle, x, S, cb, med3=True, name="mha B3 T64 S%d" % S)
+    full_call(oracle, x, S, cb, med3=True, name="mha B3 T64 S%d" % S, encoder=encoder)
 
 
 # ------------------------------------------------------------------ edge cases
@@ -145,19 +155,34 @@ def test_codebook_sizes(oracle, S):
     full_call(oracle, x, S, cb, name="S=%d" % S, check_e2e=S < 1000)
 
 
+@pytest.mark.parametrize("S", [1, 2, 3, 8, 17, 32, 48])
+def test_search_table_codebook_sizes(oracle, S):
+    rng = np.random.default_rng(100 + S)
+    x = rng.standard_normal((1, 2, 64, 128)).astype(np.float32)
+    cb = oracle.make_codebook(11, S, 2)
+    full_call(oracle, x, S, cb, name="S=%d" % S, encoder="lut")
+
+
+def test_search_table_rejects_large_S():
+    assert hqmq.hqmq_search_table_bytes(49) == 0
+    assert hqmq.hqmq_search_table_bytes(48) == 32 ** 3 * 16
+
+
+@pytest.mark.parametrize("encoder", ENCODERS)
 @pytest.mark.parametrize("shape", [(1, 1, 32, 4), (2, 3, 8, 64), (1, 2, 40, 256), (3, 1, 200, 128),
                                    (1, 1, 4100, 128)])
-def test_shapes_and_ragged_tails(oracle, shape):
+def test_shapes_and_ragged_tails(oracle, shape, encoder):
     # ragged: 4100 tokens -> 131200 chunks per slab, not a multiple of the
     # 2048-chunk decode range nor of the 4096-chunk extraction tile
     rng = np.random.default_rng(sum(shape))
     x = (rng.standard_t(3, shape) * 2).astype(np.float32)
     x = W.as_numpy_bits(torch.from_numpy(x).to(torch.bfloat16))
     cb = oracle.make_codebook(2, 8, shape[1])
-    full_call(oracle, x, 8, cb, med3=True, name="shape %s" % (shape,))
+    full_call(oracle, x, 8, cb, med3=True, name="shape %s" % (shape,), encoder=encoder)
 
 
-def test_zero_nonfinite_and_saturating_chunks(oracle):
+@pytest.mark.parametrize("encoder", ENCODERS)
+def test_zero_nonfinite_and_saturating_chunks(oracle, encoder):
     x = np.random.default_rng(1).standard_normal((1, 1, 32, 128)).astype(np.float32)
     c = x.reshape(-1, 4)
     c[0] = 0.0
@@ -168,13 +193,14 @@ def test_zero_nonfinite_and_saturating_chunks(oracle):
     c[5] = [-0.0, 0.0, -0.0, 0.0]
     cb = oracle.make_codebook(1, 8, 1)
     xd, cbd = dev(x), dev(cb.reshape(-1))
-    words, radius, st = gpu_encode(xd, cbd, 8)
+    words, radius, st = gpu_encode(xd, cbd, 8, encoder=encoder)
     gi = unpack_indices(to_host(words), 8, 1024)
     check_codes(oracle, x, cb, 8, gi, to_host(radius))
     assert st["n_nonfinite"] == 3 and st["n_saturated"] == 1 and st["flags"] == 6
 
 
-def test_exact_ties_go_to_lowest_index(oracle):
+@pytest.mark.parametrize("encoder", ENCODERS)
+def test_exact_ties_go_to_lowest_index(oracle, encoder):
     cb = np.array([[[1.0, 0.0, 0.0, 0.0], [0.0, 1.0, 0.0, 0.0], [0.5, 0.5, 0.5, 0.5]]],
                   np.float32)
     x = np.zeros((1, 1, 1, 128), np.float32)
@@ -185,7 +211,7 @@ def test_exact_ties_go_to_lowest_index(oracle):
     c[3] = [-1, 0, 0, 0]
     c[4] = [1, -1, 1, -1]
     xd, cbd = dev(x), dev(cb.reshape(-1))
-    words, radius, st = gpu_encode(xd, cbd, 3)
+    words, radius, st = gpu_encode(xd, cbd, 3, encoder=encoder)
     gi = unpack_indices(to_host(words), 3, 32)
     words_o, rad_o, *_ = oracle.encode(x, cb, 3)
     assert np.array_equal(gi, unpack_indices(words_o, 3, 32))
@@ -218,7 +244,7 @@ def test_arguments_rejected(oracle):
 
 
 # ------------------------------------------------------------------ full sizes
-def _full_size_call(oracle, name, layer, role, n_sample=20000, gran=0):
+def _full_size_call(oracle, name, layer, role, n_sample=20000, gran=0, encoder="sloop"):
     w = W.WORKLOADS[name]
     B, H, T, D = w.call_shape
     xd = W.make_call_input(w, layer, role, device="cuda")
@@ -236,7 +262,7 @@ def _full_size_call(oracle, name, layer, role, n_sample=20000, gran=0):
         thr_o, oi_o, ov_o, so_o, n_o = check_med3(oracle, x, med, w.C, gran)
         print("[parity] %s L%d role %d: %d outliers (%.3f%%)" % (
             name, layer, role, n_o, 100.0 * n_o / (B * H * T * D / (4 if gran == 0 else 1))))
-    words, radius, st = gpu_encode(xd, cbd, w.S, med["thr"] if med else None, gran)
+    words, radius, st = gpu_encode(xd, cbd, w.S, med["thr"] if med else None, gran, encoder)
     n_chunks = B * H * T * D // 4
     gi = unpack_indices(to_host(words), w.S, n_chunks)
     rng = np.random.default_rng(layer * 2 + role)
@@ -248,7 +274,7 @@ def _full_size_call(oracle, name, layer, role, n_sample=20000, gran=0):
     chunks = np.unique(np.concatenate([chunks, np.array(extra, np.int64)]))
     n, mm, near = check_codes(oracle, x, cb, w.S, gi, to_host(radius), thr=thr_o, gran=gran,
                               chunks=chunks)
-    report("%s L%d role %d (sampled)" % (name, layer, role), n, mm, near)
+    report("%s L%d role %d (sampled) [%s]" % (name, layer, role, encoder), n, mm, near)
     # decode at full size: seeded random codes + the oracle's outlier list
     rs = np.random.default_rng(99)
     b = hqmq.hqmq_index_bits(w.S)
@@ -273,20 +299,24 @@ def _full_size_call(oracle, name, layer, role, n_sample=20000, gran=0):
     assert ok.all(), np.argwhere(~ok.reshape(-1))[:5]
 
 
-def test_full_size_llama8b_call(oracle):
-    _full_size_call(oracle, "llama3_8b", 7, 0)
+@pytest.mark.parametrize("encoder", ENCODERS)
+def test_full_size_llama8b_call(oracle, encoder):
+    _full_size_call(oracle, "llama3_8b", 7, 0, encoder=encoder)
 
 
-def test_full_size_qwen_call(oracle):
-    _full_size_call(oracle, "qwen_outlier", 27, 1)
+@pytest.mark.parametrize("encoder", ENCODERS)
+def test_full_size_qwen_call(oracle, encoder):
+    _full_size_call(oracle, "qwen_outlier", 27, 1, encoder=encoder)
 
 
-def test_full_size_mha_call(oracle):
-    _full_size_call(oracle, "mha7b_s32", 0, 0, n_sample=5000)
+@pytest.mark.parametrize("encoder", ENCODERS)
+def test_full_size_mha_call(oracle, encoder):
+    _full_size_call(oracle, "mha7b_s32", 0, 0, n_sample=5000, encoder=encoder)
 
 
-def test_full_size_llama70b_call(oracle):
-    _full_size_call(oracle, "llama3_70b_128k", 40, 1, n_sample=10000)
+@pytest.mark.parametrize("encoder", ENCODERS)
+def test_full_size_llama70b_call(oracle, encoder):
+    _full_size_call(oracle, "llama3_70b_128k", 40, 1, n_sample=10000, encoder=encoder)
 
 
 def test_full_size_llama70b_call_element_mode(oracle):

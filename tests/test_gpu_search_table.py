@@ -1,0 +1,101 @@
+"""The search tables built on the GPU list, for every cell, a superset of the
+codewords that can win there: for many directions x (random, on cell
+boundaries, on Voronoi boundaries between codewords) the exact fp64 argmax of
+<x, c> over all 24 S codewords is in the list of x's cell, computed here
+independently in numpy from the table's documented layout (fold by the unit of
+the largest coordinate, gnomonic coordinates t, u = t (A + B t^2) with
+A = fp32(4/pi), B = 1 - A, 32^3 cells in u, 8 uint16 slots, 0xFFFF empty,
+0xFFFE overflow).  A point within 1e-6 of a cell face is checked against the
+cells on both sides (the kernel's fp32 arithmetic may pick either)."""
+import itertools
+import numpy as np
+import pytest
+import torch
+
+from _parity import gpu_search_table, to_host
+
+pytestmark = pytest.mark.gpu
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+G = 32
+A = float(np.float32(4.0 / np.pi))
+B = float(np.float32(1.0 - np.float32(A)))
+
+
+def fold(x):
+    """x' = conj(u) x for u = sign(x_a) e_a, a = first index of max |x_i|."""
+    a = np.argmax(np.abs(x), axis=1)
+    y = np.empty_like(x)
+    x0, x1, x2, x3 = x.T
+    cases = [np.stack([x0, x1, x2, x3], 1), np.stack([x1, -x0, x3, -x2], 1),
+             np.stack([x2, -x3, -x0, x1], 1), np.stack([x3, x2, -x1, -x0], 1)]
+    for k in range(4):
+        y[a == k] = cases[k][a == k]
+    y *= np.where(y[:, :1] < 0, -1.0, 1.0)
+    return y, a
+
+
+def u_of_t(t):
+    return t * (A + B * t * t)
+
+
+def t_of_u(u):
+    lo, hi = -np.ones_like(u), np.ones_like(u)
+    for _ in range(60):
+        m = 0.5 * (lo + hi)
+        below = u_of_t(m) < u
+        lo, hi = np.where(below, m, lo), np.where(below, hi, m)
+    return 0.5 * (lo + hi)
+
+
+def cell_candidates(y, eps=1e-6):
+    """All cells the point may land in: per axis floor of (u +- eps)."""
+    t = y[:, 1:] / y[:, :1]
+    u = u_of_t(t)
+    lo = np.clip(np.floor((u - eps + 1.0) * (G / 2)).astype(int), 0, G - 1)
+    hi = np.clip(np.floor((u + eps + 1.0) * (G / 2)).astype(int), 0, G - 1)
+    out = []
+    for pick in itertools.product((0, 1), repeat=3):
+        i = np.where(np.array(pick) == 1, hi, lo)
+        out.append((i[:, 0] * G + i[:, 1]) * G + i[:, 2])
+    return out
+
+
+@pytest.mark.parametrize("S", [8, 32, 48])
+def test_table_lists_contain_the_exact_argmax(oracle, S):
+    cb = oracle.make_codebook(5, S, 1)
+    tab = to_host(gpu_search_table(torch.from_numpy(cb.reshape(-1)).cuda(), S, 1))
+    rec = tab.view(np.uint16).reshape(G ** 3, 8).astype(np.int64)
+    overflow = rec[:, 0] == 0xFFFE
+    assert not np.any((rec[:, 0] == 0xFFFF))          # every cell lists something
+    assert overflow.mean() < 0.01
+    cw = np.array([oracle.codeword(i % 24, cb[0, i // 24]) for i in range(24 * S)], np.float64)
+    rng = np.random.default_rng(S)
+    xs = [rng.standard_normal((200000, 4))]
+    # points whose coordinates sit on cell boundaries
+    b = rng.integers(0, G + 1, (20000, 3))
+    t = t_of_u(-1.0 + 2.0 * b / G)
+    xs.append(np.concatenate([np.ones((20000, 1)), t], 1) * rng.choice([-1, 1], (20000, 1)))
+    # points on the bisector of two neighbouring codewords (exact ties)
+    i, j = rng.integers(0, 24 * S, (2, 20000))
+    xs.append(cw[i] + cw[j])
+    x = np.concatenate(xs).astype(np.float32).astype(np.float64)
+    x = x[np.linalg.norm(x, axis=1) > 1e-3]
+    y, _ = fold(x)
+    sc = y @ cw.T
+    best = sc.max(1, keepdims=True)
+    winners = sc >= best - 1e-12 * np.abs(best)       # every (near-)exact argmax
+    n_checked = 0
+    rows = np.arange(len(y))
+    for cell in cell_candidates(y):
+        lists = rec[cell]
+        ok = overflow[cell].copy()
+        for k in range(8):
+            lk = lists[:, k]
+            ok |= (lk < 24 * S) & winners[rows, np.minimum(lk, 24 * S - 1)]
+        assert ok.all(), "argmax missing from %d cell lists" % (~ok).sum()
+        n_checked += len(cell)
+    print("[table] S=%d: %d lookups, overflow cells %.3f%%, mean list %.2f"
+          % (S, n_checked, 100 * overflow.mean(),
+             (rec[~overflow] != 0xFFFF).sum(1).mean()))
