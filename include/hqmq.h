@@ -82,6 +82,8 @@ extern "C" {
 #define HQMQ_FLAG_SATURATED 2u        /* an fp16 radius or outlier value saturated   */
 #define HQMQ_FLAG_NONFINITE 4u        /* a chunk norm was NaN or inf                 */
 #define HQMQ_FLAG_BAD_INDEX 8u        /* decode met an index >= 24 S                 */
+#define HQMQ_FLAG_MED3_FALLBACK 16u   /* a head's sampled median window missed; its
+                                         median came from the exact (slow) path    */
 
 /* Device-resident status record (caller-allocated, 32 bytes, 8-byte aligned).
  * Calls OR flags in and add to the counters. */
@@ -117,7 +119,10 @@ HQMQ_API uint64_t hqmq_index_words(int B, int H, int T, int D, uint32_t S);
 HQMQ_API int hqmq_make_codebook(uint64_t seed, uint32_t S, uint32_t n_groups, uint32_t group0,
                        float *d_codebook, void *stream);
 
-/* Bytes of device workspace hqmq_outlier_extract needs for this shape. */
+/* Bytes of device workspace hqmq_outlier_extract (and hqmq_encode_med3) needs
+ * for this shape: two 64 Ki-bin histograms per head, the keys of the median
+ * window, the uncertain-threshold list and per-tile counts (about 10 MB for
+ * a 1 x 8 x 131072 x 128 call). */
 HQMQ_API uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gran);
 
 /* Med3x (gist.science/nl, Technische Samenvatting, section 3; the pages
@@ -138,6 +143,14 @@ HQMQ_API uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gr
  * Entries at positions >= cap are not written (d_slab_off still holds the
  * full offsets); the status then gets HQMQ_FLAG_OUTLIER_OVERFLOW and
  * n_outliers the required total, so the caller can retry with a larger cap.
+ * Data flow (two reads of x): a 1/32 sample fixes per head a key window that
+ * holds the median rank with overwhelming probability; one full read counts
+ * the keys below the window, keeps the keys inside it and counts per
+ * 1024-chunk tile the chunks above the threshold's range; the exact median is
+ * selected from the window keys (a head whose window misses the median, or
+ * whose buffers overflow, is decided by an exact three-pass selection over x
+ * instead, so the result never depends on the sample); the second read
+ * writes the ordered list.
  * d_x: bf16 or fp32 [B][H][T][D], 16-byte aligned.  d_rmed, d_thr: fp32 [H].
  * d_out_idx: uint32[cap]; d_out_val: uint16[cap*4] (chunk) or [cap] (element),
  * 4-byte aligned.  d_ws: at least hqmq_outlier_workspace_size bytes,
@@ -214,6 +227,20 @@ HQMQ_API int hqmq_encode_lut(const void *d_x, int dtype, int B, int H, int T, in
                              const float *d_thr, int gran, uint32_t *d_idx_words,
                              uint16_t *d_radius, hqmq_status *d_status, void *stream);
 
+/* Med3x and encode in two reads of x: hqmq_outlier_extract's median and tile
+ * counts (first read), then one pass that writes the ordered outlier list and
+ * encodes the zeroed chunks with the search tables (second read).  Outputs
+ * equal hqmq_outlier_extract followed by hqmq_encode_lut (or hqmq_encode when
+ * d_table is NULL, which costs a third read).  Workspace as
+ * hqmq_outlier_workspace_size; other arguments as in those calls. */
+HQMQ_API uint64_t hqmq_encode_med3_workspace_size(int B, int H, int T, int D, int gran);
+HQMQ_API int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, float C,
+                              int gran, const float *d_codebook, uint32_t S, const void *d_table,
+                              uint32_t *d_idx_words, uint16_t *d_radius, float *d_rmed,
+                              float *d_thr, uint32_t *d_out_idx, uint16_t *d_out_val,
+                              uint32_t *d_slab_off, uint64_t cap, void *d_ws, uint64_t ws_bytes,
+                              hqmq_status *d_status, void *stream);
+
 /* Size of the fixed device scratch array of hqmq_outlier_extract_noalloc. */
 #define HQMQ_NOALLOC_SCRATCH_BYTES (1u << 20)
 
@@ -224,11 +251,12 @@ HQMQ_API int hqmq_encode_lut(const void *d_x, int dtype, int B, int H, int T, in
  * (which may synchronise the device) are not allowed.  The caller still
  * passes every input and output.
  *
- * The scratch lives in one file-scope device array of
- * HQMQ_NOALLOC_SCRATCH_BYTES (1 MiB) that every GPU which loads libhqmq holds
- * until the process exits.  Shapes whose hqmq_outlier_workspace_size exceeds
- * it are rejected with HQMQ_ERR_WORKSPACE (a 1 x 8 x 131072 x 128 call needs
- * about 130 KB).  The first call on a device looks up the array's device
+ * It runs the compact three-pass radix selection (three reads of x for the
+ * median, two for the list), whose scratch is 8 KB per head plus 8 bytes per
+ * 4096 chunks, in one file-scope device array of HQMQ_NOALLOC_SCRATCH_BYTES
+ * (1 MiB) that every GPU which loads libhqmq holds until the process exits.
+ * Shapes that need more are rejected with HQMQ_ERR_WORKSPACE (a
+ * 1 x 8 x 131072 x 128 call needs about 130 KB).  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress, with that device current) and caches it;
  * make that first call before any stream capture.  All calls on a device
  * share the one array: calls whose execution overlaps on the GPU (different

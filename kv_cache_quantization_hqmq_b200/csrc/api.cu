@@ -25,6 +25,18 @@ extern "C" int hqmq_launch_outlier_extract(const void *x, int dtype, int B, int 
                                            uint32_t *slab_off, uint64_t cap, void *ws,
                                            hqmq_status *st, int sm_count, cudaStream_t stream);
 
+extern "C" uint64_t hqmq_window_workspace_bytes(int B, int H, int T, int D, int gran);
+extern "C" int hqmq_launch_med3_window(const void *x, int dtype, int B, int H, int T, int D,
+                                       float C, int gran, float *rmed, float *thr,
+                                       uint32_t *slab_off, uint64_t cap, void *ws,
+                                       hqmq_status *st, int sm_count, cudaStream_t stream,
+                                       const uint32_t **tile_off, uint32_t *tiles_per_slab);
+extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int T, int D,
+                                     const float *cb, uint32_t S, uint32_t b, const void *table,
+                                     const float *thr, int gran, uint32_t *words,
+                                     uint16_t *radius, const uint32_t *tile_off, uint64_t cap,
+                                     uint32_t *out_idx, uint16_t *out_val, hqmq_status *st,
+                                     int sm_count, cudaStream_t stream);
 extern "C" uint64_t hqmq_lut_bytes_per_group(uint32_t S);
 extern "C" int hqmq_launch_build_search_table(const float *cb, uint32_t S, uint32_t n_groups,
                                               void *table, cudaStream_t stream);
@@ -112,7 +124,7 @@ int hqmq_make_codebook(uint64_t seed, uint32_t S, uint32_t n_groups, uint32_t gr
 
 uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gran) {
     if (!shape_ok(B, H, T, D) || !gran_ok(gran)) return 0;
-    return hqmq_med3_workspace_bytes(B, H, T, D);
+    return hqmq_window_workspace_bytes(B, H, T, D, gran);
 }
 
 int hqmq_outlier_extract(const void *d_x, int dtype, int B, int H, int T, int D, float C,
@@ -127,12 +139,62 @@ int hqmq_outlier_extract(const void *d_x, int dtype, int B, int H, int T, int D,
         !aligned(d_slab_off, 4) || !aligned(d_ws, 256) || !aligned(d_out_idx, 4) ||
         !aligned(d_out_val, 4) || !aligned(d_status, 8))
         return HQMQ_ERR_ALIGN;
-    if (ws_bytes < hqmq_med3_workspace_bytes(B, H, T, D)) return HQMQ_ERR_WORKSPACE;
+    if (ws_bytes < hqmq_window_workspace_bytes(B, H, T, D, gran)) return HQMQ_ERR_WORKSPACE;
     int sm = sm_count();
     if (sm <= 0) return HQMQ_ERR_CUDA;
-    return hqmq_launch_outlier_extract(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_out_idx,
-                                       d_out_val, d_slab_off, cap, d_ws, d_status, sm,
-                                       (cudaStream_t)stream);
+    const uint32_t *tile_off = nullptr;
+    uint32_t tps = 0;
+    int rc = hqmq_launch_med3_window(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_slab_off,
+                                     cap, d_ws, d_status, sm, (cudaStream_t)stream, &tile_off,
+                                     &tps);
+    if (rc != HQMQ_OK) return rc;
+    return hqmq_launch_list_pass(d_x, dtype, B, H, T, D, nullptr, 1, 5, nullptr, d_thr, gran,
+                                 nullptr, nullptr, tile_off, cap, d_out_idx, d_out_val, d_status,
+                                 sm, (cudaStream_t)stream);
+}
+
+uint64_t hqmq_encode_med3_workspace_size(int B, int H, int T, int D, int gran) {
+    return hqmq_outlier_workspace_size(B, H, T, D, gran);
+}
+
+int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, float C, int gran,
+                     const float *d_codebook, uint32_t S, const void *d_table,
+                     uint32_t *d_idx_words, uint16_t *d_radius, float *d_rmed, float *d_thr,
+                     uint32_t *d_out_idx, uint16_t *d_out_val, uint32_t *d_slab_off, uint64_t cap,
+                     void *d_ws, uint64_t ws_bytes, hqmq_status *d_status, void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
+    if (!(C > 0.0f) || !(C < 3.0e38f)) return HQMQ_ERR_ARG;
+    if (S < 1 || S > S_MAX) return HQMQ_ERR_ARG;
+    if (d_table && hqmq_lut_bytes_per_group(S) == 0) return HQMQ_ERR_ARG;
+    if (!d_x || !d_codebook || !d_idx_words || !d_radius || !d_rmed || !d_thr || !d_slab_off ||
+        !d_ws)
+        return HQMQ_ERR_ARG;
+    if (cap > 0 && (!d_out_idx || !d_out_val)) return HQMQ_ERR_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_codebook, 16) || !aligned(d_table, 16) ||
+        !aligned(d_idx_words, 4) || !aligned(d_radius, 4) || !aligned(d_rmed, 4) ||
+        !aligned(d_thr, 4) || !aligned(d_slab_off, 4) || !aligned(d_ws, 256) ||
+        !aligned(d_out_idx, 4) || !aligned(d_out_val, 4) || !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    if (ws_bytes < hqmq_window_workspace_bytes(B, H, T, D, gran)) return HQMQ_ERR_WORKSPACE;
+    int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    const uint32_t *tile_off = nullptr;
+    uint32_t tps = 0;
+    int rc = hqmq_launch_med3_window(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_slab_off,
+                                     cap, d_ws, d_status, sm, (cudaStream_t)stream, &tile_off,
+                                     &tps);
+    if (rc != HQMQ_OK) return rc;
+    const uint32_t b = hqmq_index_bits(S);
+    if (d_table)   // list and encode in the same (second) read of x
+        return hqmq_launch_list_pass(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table, d_thr,
+                                     gran, d_idx_words, d_radius, tile_off, cap, d_out_idx,
+                                     d_out_val, d_status, sm, (cudaStream_t)stream);
+    rc = hqmq_launch_list_pass(d_x, dtype, B, H, T, D, nullptr, 1, 5, nullptr, d_thr, gran,
+                               nullptr, nullptr, tile_off, cap, d_out_idx, d_out_val, d_status,
+                               sm, (cudaStream_t)stream);
+    if (rc != HQMQ_OK) return rc;
+    return hqmq_launch_encode(d_x, dtype, B, H, T, D, d_codebook, S, b, d_thr, gran, d_idx_words,
+                              d_radius, d_status, sm, (cudaStream_t)stream);
 }
 
 int hqmq_encode(const void *d_x, int dtype, int B, int H, int T, int D, const float *d_codebook,

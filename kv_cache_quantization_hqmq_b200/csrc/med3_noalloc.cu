@@ -65,9 +65,10 @@ extern "C" HQMQ_API int hqmq_outlier_extract_noalloc(const void *d_x, int dtype,
                                                     uint32_t *d_out_idx, uint16_t *d_out_val,
                                                     uint32_t *d_slab_off, uint64_t cap,
                                                     hqmq_status *d_status, void *stream) {
-    // same argument rules as hqmq_outlier_extract
-    uint64_t need = hqmq_outlier_workspace_size(B, H, T, D, gran);
-    if (need == 0) return HQMQ_ERR_ARG;
+    // same argument rules as hqmq_outlier_extract; the scratch need is that of
+    // the compact three-pass radix selection this entry point runs
+    if (hqmq_outlier_workspace_size(B, H, T, D, gran) == 0) return HQMQ_ERR_ARG;
+    const uint64_t need = hqmq_med3_workspace_bytes(B, H, T, D);
     if (dtype != HQMQ_BF16 && dtype != HQMQ_F32) return HQMQ_ERR_ARG;
     if (!(C > 0.0f) || !(C < 3.0e38f)) return HQMQ_ERR_ARG;
     if (!d_x || !d_rmed || !d_thr || !d_slab_off) return HQMQ_ERR_ARG;

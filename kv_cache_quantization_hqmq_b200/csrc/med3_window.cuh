@@ -1,0 +1,69 @@
+// med3_window.cuh -- shared layout of the two-read Med3x pipeline
+// (med3_window.cu: sample, window, full pass, selection, tile offsets;
+// search.cu: the encode pass that also writes the ordered outlier list).
+#pragma once
+
+#include <math.h>
+
+#include "hqmq_device.cuh"
+
+namespace hqmq {
+
+constexpr int TILE_GROUPS = 32;                  // packing groups per warp tile
+constexpr int TILE_CHUNKS = TILE_GROUPS * 32;    // 1024 chunks
+constexpr int SAMPLE_PERIOD = 128;               // sample chunks 4k..4k+3 of every 128
+constexpr int KEY_BINS = 65536;                  // sample and fine histograms
+constexpr int WINDOW_SIGMAS = 8;                 // half-width of the rank window
+
+// Per-head state of the rank window.
+struct WinState {
+    uint32_t lo_key, hi_key;   // candidate keys: lo_key <= key < hi_key
+    uint32_t shift;            // fine bin = (key - lo_key) >> shift
+    uint32_t miss;             // 1: exact fallback decides this head
+    float t_lo, t_hi;          // thr is known to lie in [t_lo, t_hi]
+    uint32_t pad[2];
+};
+
+struct FusedLayout {
+    uint64_t sample_hist, fine_hist, win, below, cand_n, cand, amb_n, amb, tile_cnt, tile_off,
+        total;
+    uint64_t cand_cap;         // keys per head
+    uint64_t amb_cap;          // (tile, key) pairs per call
+    uint64_t n_per_head;       // keys per head (chunks or elements)
+    uint32_t tiles_per_slab;
+    uint64_t n_tiles;
+};
+
+inline uint64_t align256_(uint64_t v) { return (v + 255) & ~(uint64_t)255; }
+
+inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
+    FusedLayout L;
+    const uint64_t cps = (uint64_t)T * D / 4;
+    const uint64_t gps = cps / 32;
+    L.tiles_per_slab = (uint32_t)((gps + TILE_GROUPS - 1) / TILE_GROUPS);
+    L.n_tiles = (uint64_t)B * H * L.tiles_per_slab;
+    L.n_per_head = (uint64_t)B * cps * (gran == HQMQ_GRAN_CHUNK ? 1 : 4);
+    // expected window: +-WINDOW_SIGMAS sample standard deviations of the median
+    // rank, plus the two 2^15-key edge bins; the buffer holds twice that
+    const double ns = (double)L.n_per_head / 32.0 + 1.0;
+    const double frac = (2.0 * WINDOW_SIGMAS * 0.5 * sqrt(ns) + 8.0) / ns + 0.02;
+    uint64_t cap = (uint64_t)(2.0 * frac * (double)L.n_per_head) + 4096;
+    L.cand_cap = cap < L.n_per_head ? cap : L.n_per_head;
+    const uint64_t n_keys = L.n_per_head * H;
+    L.amb_cap = n_keys / 25 + 4096;              // 4% of the keys may sit in thr's band
+    uint64_t off = 0;
+    L.sample_hist = off; off = align256_(off + (uint64_t)H * KEY_BINS * 4);
+    L.fine_hist = off;   off = align256_(off + (uint64_t)H * KEY_BINS * 4);
+    L.win = off;         off = align256_(off + (uint64_t)H * sizeof(WinState));
+    L.below = off;       off = align256_(off + (uint64_t)H * 8);
+    L.cand_n = off;      off = align256_(off + (uint64_t)H * 8);
+    L.amb_n = off;       off = align256_(off + 8);
+    L.cand = off;        off = align256_(off + (uint64_t)H * L.cand_cap * 4);
+    L.amb = off;         off = align256_(off + L.amb_cap * 8);
+    L.tile_cnt = off;    off = align256_(off + L.n_tiles * 4);
+    L.tile_off = off;    off = align256_(off + L.n_tiles * 4);
+    L.total = off;
+    return L;
+}
+
+}  // namespace hqmq

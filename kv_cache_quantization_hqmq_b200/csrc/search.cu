@@ -32,7 +32,7 @@
 //    per head); candidate codewords come from a shared-memory copy of the 24 S
 //    codewords replicated 8 times so that the 8 lanes of each quarter-warp
 //    read 8 different bank groups (no conflicts).
-#include "hqmq_device.cuh"
+#include "med3_window.cuh"
 
 namespace hqmq {
 
@@ -283,33 +283,41 @@ __device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b, int lane,
     if (lane < (int)b) dst[lane] = (uint32_t)(vk >> o);
 }
 
-template <int DT>
+// LIST: 0 = no list; HQMQ_GRAN_CHUNK + 1 / HQMQ_GRAN_ELEMENT + 1 = write the
+// ordered outlier list of that granularity (thr exact, tile_off from the
+// Med3x window pipeline).  ENC: encode (else write the list only).
+// Work: warp tiles of TILE_GROUPS consecutive packing groups; a CTA owns a
+// contiguous range of tiles and walks it slab by slab (one head at a time).
+template <int DT, int LIST, bool ENC>
 __global__ void __launch_bounds__(ENC_THREADS, 1)
-k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint64_t n_groups,
-             const float4 *__restrict__ cb_all, uint32_t S, uint32_t b,
+k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32_t tiles_per_slab,
+             uint64_t n_tiles, const float4 *__restrict__ cb_all, uint32_t S, uint32_t b,
              const uint4 *__restrict__ tables, const float *__restrict__ thr, int gran,
-             uint32_t *__restrict__ words, uint16_t *__restrict__ radius, DevStatus *st) {
+             uint32_t *__restrict__ words, uint16_t *__restrict__ radius,
+             const uint32_t *__restrict__ tile_off, uint64_t cap, uint32_t *__restrict__ out_idx,
+             uint16_t *__restrict__ out_val, DevStatus *st) {
     extern __shared__ float4 s_tab[];                              // [24 S][8] replicated
     __shared__ uint8_t s_mul[8][24];                               // u * q_p' for the 8 units
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
     const int n_warps = ENC_THREADS / 32;
     const uint32_t n_words = 24u * S;
     const uint32_t lane7 = (uint32_t)(lane & 7);
-    for (int i = threadIdx.x; i < 8 * 24; i += ENC_THREADS)
-        s_mul[i / 24][i % 24] = (uint8_t)mul_2t(i / 24, i % 24);
+    if (ENC)
+        for (int i = threadIdx.x; i < 8 * 24; i += ENC_THREADS)
+            s_mul[i / 24][i % 24] = (uint8_t)mul_2t(i / 24, i % 24);
 
-    // this CTA's contiguous range of packing groups (32 chunks each)
-    const uint64_t g_begin = n_groups * blockIdx.x / gridDim.x;
-    const uint64_t g_end = n_groups * (blockIdx.x + 1) / gridDim.x;
+    const uint64_t t_begin = n_tiles * blockIdx.x / gridDim.x;
+    const uint64_t t_end = n_tiles * (blockIdx.x + 1) / gridDim.x;
     int cur_head = -1;
     unsigned n_nf = 0, n_sat = 0;
-    for (uint64_t seg = g_begin; seg < g_end;) {
-        const uint64_t slab = seg / groups_per_slab;
-        const uint64_t seg_end = min(g_end, (slab + 1) * groups_per_slab);
+    for (uint64_t seg = t_begin; seg < t_end;) {
+        const uint64_t slab = seg / tiles_per_slab;
+        const uint64_t seg_end = min(t_end, (slab + 1) * tiles_per_slab);
         const int h = (int)(slab % (uint64_t)H);
         const float4 *cb = cb_all + (size_t)h * S;
         const uint4 *tb = tables + (size_t)h * LUT_CELLS;
-        if (h != cur_head) {                        // (block-uniform)
+        if (ENC && h != cur_head) {                  // (block-uniform)
             __syncthreads();
             for (uint32_t i = threadIdx.x; i < n_words * 8; i += ENC_THREADS) {
                 const uint32_t id = i >> 3;
@@ -318,82 +326,134 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint64
             __syncthreads();
             cur_head = h;
         }
-        const float th = thr ? __ldg(thr + h) : 0.0f;
-        uint64_t G = seg + warp;
-        RawChunk<DT> nxt;                           // x of the next group, loaded early
-        if (G < seg_end) nxt.load(x, G * 32 + lane);
-        for (; G < seg_end; G += n_warps) {
-            const RawChunk<DT> cur = nxt;
-            if (G + n_warps < seg_end) nxt.load(x, (G + n_warps) * 32 + lane);
-            float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
-            float r = chunk_norm(x0, x1, x2, x3);
-            if (thr) {
-                if (gran == HQMQ_GRAN_CHUNK) {
-                    if (r > th) { x0 = x1 = x2 = x3 = 0.0f; r = 0.0f; }
-                } else {
-                    if (fabsf(x0) > th) x0 = 0.0f;
-                    if (fabsf(x1) > th) x1 = 0.0f;
-                    if (fabsf(x2) > th) x2 = 0.0f;
-                    if (fabsf(x3) > th) x3 = 0.0f;
-                    r = chunk_norm(x0, x1, x2, x3);
-                }
-            }
-            const bool finite = r == r && r != __int_as_float(0x7F800000);
-            const bool search = finite && r > 0.0f;
-            // every lane takes part in the candidate loop (it votes); lanes
-            // without a search carry an all-empty record
-            float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-            int pu = 0;
-            uint4 rec = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-            if (search) {
-                pu = fold(x0, x1, x2, x3, y0, y1, y2, y3);
-                float inv;
-                asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(y0));   // cells are widened
-                const int cell = (cell_coord(y1 * inv) * LUT_G + cell_coord(y2 * inv)) * LUT_G +
-                                 cell_coord(y3 * inv);
-                rec = __ldg(tb + cell);
-            }
-            const bool fallback = (rec.x & 0xFFFFu) == LUT_OVERFLOW;
-            if (fallback) rec = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-            const uint32_t sl[4] = {rec.x, rec.y, rec.z, rec.w};
-            const uint32_t id0 = rec.x & 0xFFFFu;
-            float best = __int_as_float(0xFF800000);     // -inf
-            uint32_t bid = 0;
-            uint32_t bmap = 0xFFFFFFFFu;
+        const bool med3 = thr != nullptr;
+        const float th = med3 ? __ldg(thr + h) : 0.0f;
+        for (uint64_t t = seg + warp; t < seg_end; t += n_warps) {
+            const uint32_t g0 = (uint32_t)(t % tiles_per_slab) * TILE_GROUPS;
+            const uint32_t g1 = min(g0 + TILE_GROUPS, groups_per_slab);
+            const uint64_t gbase = slab * groups_per_slab;
+            uint64_t lpos = LIST ? (uint64_t)__ldg(tile_off + t) : 0;   // list position
+            RawChunk<DT> nxt;
+            nxt.load(x, (gbase + g0) * 32 + lane);
+            for (uint32_t g = g0; g < g1; ++g) {
+                const uint64_t G = gbase + g;
+                const RawChunk<DT> cur = nxt;
+                if (g + 1 < g1) nxt.load(x, (G + 1) * 32 + lane);
+                float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
+                float r = chunk_norm(x0, x1, x2, x3);
+                if (LIST == HQMQ_GRAN_CHUNK + 1) {           // ordered chunk list
+                    const bool o = r > th;
+                    const uint32_t m = __ballot_sync(FULL, o);
+                    if (o) {
+                        const uint64_t p = lpos + __popc(m & lt);
+                        if (p < cap) {
+                            int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+                            const uint32_t h0 = f32_to_f16_sat(x0, s0), h1 = f32_to_f16_sat(x1, s1);
+                            const uint32_t h2 = f32_to_f16_sat(x2, s2), h3 = f32_to_f16_sat(x3, s3);
+                            n_sat += s0 + s1 + s2 + s3;
+                            out_idx[p] = (uint32_t)(G * 32 + lane);
+                            uint32_t *vv = reinterpret_cast<uint32_t *>(out_val + p * 4);
+                            vv[0] = h0 | (h1 << 16);
+                            vv[1] = h2 | (h3 << 16);
+                        }
+                    }
+                    lpos += __popc(m);
+                } else if (LIST == HQMQ_GRAN_ELEMENT + 1) {  // ordered element list
+                    const float xs[4] = {x0, x1, x2, x3};
+                    uint32_t mk = 0;
 #pragma unroll
-            for (int k = 0; k < LUT_SLOTS; ++k) {
-                const uint32_t idk = (sl[k >> 1] >> ((k & 1) * 16)) & 0xFFFFu;
-                if (!__any_sync(FULL, idk != LUT_EMPTY)) break;
-                // a lane whose list is shorter re-scores its first candidate
-                const uint32_t id = idk != LUT_EMPTY ? idk : id0;
-                if (id0 != LUT_EMPTY) {
-                    const float4 c = s_tab[(id << 3) | lane7];
-                    const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z,
-                                     __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
-                    if (sc > best) {
-                        best = sc; bid = id; bmap = 0xFFFFFFFFu;
-                    } else if (sc == best && id != bid) {   // exact tie: lowest original index
-                        if (bmap == 0xFFFFFFFFu)
-                            bmap = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
-                        const uint32_t m = (id / 24u) * 24u + s_mul[pu][id % 24u];
-                        if (m < bmap) { bid = id; bmap = m; }
+                    for (int i = 0; i < 4; ++i) mk |= (fabsf(xs[i]) > th ? 1u : 0u) << i;
+                    const uint32_t n = __popc(mk);
+                    uint32_t inc = n;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t v = __shfl_up_sync(FULL, inc, o);
+                        if (lane >= o) inc += v;
+                    }
+                    uint64_t p = lpos + inc - n;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (mk & (1u << i)) {
+                            if (p < cap) {
+                                int sv = 0;
+                                out_val[p] = f32_to_f16_sat(xs[i], sv);
+                                n_sat += sv;
+                                out_idx[p] = (uint32_t)((G * 32 + lane) * 4 + i);
+                            }
+                            ++p;
+                        }
+                    }
+                    lpos += __shfl_sync(FULL, inc, 31);
+                }
+                if (!ENC) continue;
+                if (med3) {
+                    if (gran == HQMQ_GRAN_CHUNK) {
+                        if (r > th) { x0 = x1 = x2 = x3 = 0.0f; r = 0.0f; }
+                    } else {
+                        if (fabsf(x0) > th) x0 = 0.0f;
+                        if (fabsf(x1) > th) x1 = 0.0f;
+                        if (fabsf(x2) > th) x2 = 0.0f;
+                        if (fabsf(x3) > th) x3 = 0.0f;
+                        r = chunk_norm(x0, x1, x2, x3);
                     }
                 }
+                const bool finite = r == r && r != __int_as_float(0x7F800000);
+                const bool search = finite && r > 0.0f;
+                // every lane takes part in the candidate loop (it votes); lanes
+                // without a search carry an all-empty record
+                float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+                int pu = 0;
+                uint4 rec = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+                if (search) {
+                    pu = fold(x0, x1, x2, x3, y0, y1, y2, y3);
+                    float inv;
+                    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(y0));   // cells are widened
+                    const int cell = (cell_coord(y1 * inv) * LUT_G + cell_coord(y2 * inv)) * LUT_G +
+                                     cell_coord(y3 * inv);
+                    rec = __ldg(tb + cell);
+                }
+                const bool fallback = (rec.x & 0xFFFFu) == LUT_OVERFLOW;
+                if (fallback) rec = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+                const uint32_t sl[4] = {rec.x, rec.y, rec.z, rec.w};
+                const uint32_t id0 = rec.x & 0xFFFFu;
+                float best = __int_as_float(0xFF800000);     // -inf
+                uint32_t bid = 0;
+                uint32_t bmap = 0xFFFFFFFFu;
+#pragma unroll
+                for (int k = 0; k < LUT_SLOTS; ++k) {
+                    const uint32_t idk = (sl[k >> 1] >> ((k & 1) * 16)) & 0xFFFFu;
+                    if (!__any_sync(FULL, idk != LUT_EMPTY)) break;
+                    // a lane whose list is shorter re-scores its first candidate
+                    const uint32_t id = idk != LUT_EMPTY ? idk : id0;
+                    if (id0 != LUT_EMPTY) {
+                        const float4 c = s_tab[(id << 3) | lane7];
+                        const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z,
+                                         __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
+                        if (sc > best) {
+                            best = sc; bid = id; bmap = 0xFFFFFFFFu;
+                        } else if (sc == best && id != bid) {   // exact tie: lowest original index
+                            if (bmap == 0xFFFFFFFFu)
+                                bmap = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
+                            const uint32_t m = (id / 24u) * 24u + s_mul[pu][id % 24u];
+                            if (m < bmap) { bid = id; bmap = m; }
+                        }
+                    }
+                }
+                uint32_t idx = 0;
+                if (search && !fallback) idx = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
+                if (fallback) idx = sloop_index(x0, x1, x2, x3, cb, S);
+                uint16_t rh;
+                if (!finite) {
+                    rh = 0x7E00u;
+                    ++n_nf;
+                } else {
+                    int sat = 0;
+                    rh = f32_to_f16_sat(r, sat);
+                    n_sat += sat;
+                }
+                radius[G * 32 + lane] = rh;
+                pack_group32(idx, b, lane, words + G * b);
             }
-            uint32_t idx = 0;
-            if (search && !fallback) idx = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
-            if (fallback) idx = sloop_index(x0, x1, x2, x3, cb, S);
-            uint16_t rh;
-            if (!finite) {
-                rh = 0x7E00u;
-                ++n_nf;
-            } else {
-                int sat = 0;
-                rh = f32_to_f16_sat(r, sat);
-                n_sat += sat;
-            }
-            radius[G * 32 + lane] = rh;
-            pack_group32(idx, b, lane, words + G * b);
         }
         seg = seg_end;
     }
@@ -428,27 +488,83 @@ extern "C" int hqmq_launch_build_search_table(const float *cb, uint32_t S, uint3
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
+namespace hqmq {
+
+template <int DT, int LIST, bool ENC>
+static int launch_lut(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
+                      uint32_t b, const void *table, const float *thr, int gran, uint32_t *words,
+                      uint16_t *radius, const uint32_t *tile_off, uint64_t cap, uint32_t *out_idx,
+                      uint16_t *out_val, hqmq_status *st, int sm_count, cudaStream_t stream) {
+    const uint32_t gps = (uint32_t)(((uint64_t)T * D / 4) / 32);
+    const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
+    const uint64_t n_tiles = (uint64_t)B * H * tps;
+    const size_t smem = ENC ? enc_smem_bytes(S) : 0;
+    auto kern = k_encode_lut<DT, LIST, ENC>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return HQMQ_ERR_CUDA;
+    // one CTA per SM, each a contiguous share of the call's tiles
+    uint64_t ctas = (uint64_t)sm_count;
+    const uint64_t want = (n_tiles + 7) / 8;
+    if (ctas > want) ctas = want;
+    if (ctas < 1) ctas = 1;
+    kern<<<(unsigned)ctas, ENC_THREADS, smem, stream>>>(
+        x, H, gps, tps, n_tiles, reinterpret_cast<const float4 *>(cb), S, b,
+        reinterpret_cast<const uint4 *>(table), thr, gran, words, radius, tile_off, cap, out_idx,
+        out_val, reinterpret_cast<DevStatus *>(st));
+    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}
+
+template <int LIST, bool ENC>
+static int launch_lut_dt(int dtype, int B, int H, int T, int D, const void *x, const float *cb,
+                         uint32_t S, uint32_t b, const void *table, const float *thr, int gran,
+                         uint32_t *words, uint16_t *radius, const uint32_t *tile_off, uint64_t cap,
+                         uint32_t *out_idx, uint16_t *out_val, hqmq_status *st, int sm,
+                         cudaStream_t stream) {
+    if (dtype == HQMQ_BF16)
+        return launch_lut<HQMQ_BF16, LIST, ENC>(B, H, T, D, x, cb, S, b, table, thr, gran, words,
+                                                radius, tile_off, cap, out_idx, out_val, st, sm,
+                                                stream);
+    return launch_lut<HQMQ_F32, LIST, ENC>(B, H, T, D, x, cb, S, b, table, thr, gran, words, radius,
+                                           tile_off, cap, out_idx, out_val, st, sm, stream);
+}
+
+}  // namespace hqmq
+
 extern "C" int hqmq_launch_encode_lut(const void *x, int dtype, int B, int H, int T, int D,
                                       const float *cb, uint32_t S, uint32_t b, const void *table,
                                       const float *thr, int gran, uint32_t *words,
                                       uint16_t *radius, hqmq_status *st, int sm_count,
                                       cudaStream_t stream) {
+    return hqmq::launch_lut_dt<0, true>(dtype, B, H, T, D, x, cb, S, b, table, thr, gran, words,
+                                        radius, nullptr, 0, nullptr, nullptr, st, sm_count, stream);
+}
+
+// Pass C of the two-read Med3x: the ordered list (from exact thr and tile
+// offsets) and, if table != NULL, the encode in the same read.
+extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int T, int D,
+                                     const float *cb, uint32_t S, uint32_t b, const void *table,
+                                     const float *thr, int gran, uint32_t *words,
+                                     uint16_t *radius, const uint32_t *tile_off, uint64_t cap,
+                                     uint32_t *out_idx, uint16_t *out_val, hqmq_status *st,
+                                     int sm_count, cudaStream_t stream) {
     using namespace hqmq;
-    const uint32_t gps = (uint32_t)(((uint64_t)T * D / 4) / 32);
-    const uint64_t n_groups = (uint64_t)B * H * gps;
-    const size_t smem = enc_smem_bytes(S);
-    auto kern = dtype == HQMQ_BF16 ? k_encode_lut<HQMQ_BF16> : k_encode_lut<HQMQ_F32>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return HQMQ_ERR_CUDA;
-    // one CTA per SM, each a contiguous share of the call's groups
-    uint64_t ctas = (uint64_t)sm_count;
-    const uint64_t want = (n_groups + 31) / 32;
-    if (ctas > want) ctas = want;
-    if (ctas < 1) ctas = 1;
-    kern<<<(unsigned)ctas, ENC_THREADS, smem, stream>>>(
-        x, H, gps, n_groups, reinterpret_cast<const float4 *>(cb), S, b,
-        reinterpret_cast<const uint4 *>(table), thr, gran, words, radius,
-        reinterpret_cast<DevStatus *>(st));
-    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+    const bool enc = table != nullptr;
+    if (gran == HQMQ_GRAN_CHUNK) {
+        return enc ? launch_lut_dt<HQMQ_GRAN_CHUNK + 1, true>(dtype, B, H, T, D, x, cb, S, b, table,
+                                                             thr, gran, words, radius, tile_off,
+                                                             cap, out_idx, out_val, st, sm_count,
+                                                             stream)
+                   : launch_lut_dt<HQMQ_GRAN_CHUNK + 1, false>(dtype, B, H, T, D, x, cb, S, b,
+                                                              table, thr, gran, words, radius,
+                                                              tile_off, cap, out_idx, out_val, st,
+                                                              sm_count, stream);
+    }
+    return enc ? launch_lut_dt<HQMQ_GRAN_ELEMENT + 1, true>(dtype, B, H, T, D, x, cb, S, b, table,
+                                                           thr, gran, words, radius, tile_off, cap,
+                                                           out_idx, out_val, st, sm_count, stream)
+               : launch_lut_dt<HQMQ_GRAN_ELEMENT + 1, false>(dtype, B, H, T, D, x, cb, S, b, table,
+                                                            thr, gran, words, radius, tile_off,
+                                                            cap, out_idx, out_val, st, sm_count,
+                                                            stream);
 }

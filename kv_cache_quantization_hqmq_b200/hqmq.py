@@ -23,6 +23,7 @@ HQMQ_OK, HQMQ_ERR_ARG, HQMQ_ERR_ALIGN, HQMQ_ERR_CUDA, HQMQ_ERR_WORKSPACE = 0, 1,
 HQMQ_BF16, HQMQ_F32 = 0, 1
 HQMQ_GRAN_CHUNK, HQMQ_GRAN_ELEMENT = 0, 1
 FLAG_OUTLIER_OVERFLOW, FLAG_SATURATED, FLAG_NONFINITE, FLAG_BAD_INDEX = 1, 2, 4, 8
+FLAG_MED3_FALLBACK = 16
 
 
 class HQMQError(RuntimeError):
@@ -50,6 +51,9 @@ _SIGS = {
     "hqmq_decode": (_I, [_P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P, _I, _P, _P]),
     "hqmq_outlier_extract_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P,
                                           _U64, _P, _P]),
+    "hqmq_encode_med3_workspace_size": (_U64, [_I, _I, _I, _I, _I]),
+    "hqmq_encode_med3": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _U32, _P, _P, _P, _P, _P, _P,
+                              _P, _P, _U64, _P, _U64, _P, _P]),
     "hqmq_search_table_bytes": (_U64, [_U32]),
     "hqmq_make_search_table": (_I, [_P, _U32, _U32, _P, _P]),
     "hqmq_encode_lut": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _P, _I, _P, _P, _P, _P]),
@@ -116,6 +120,10 @@ def hqmq_outlier_workspace_size(B, H, T, D, gran=HQMQ_GRAN_CHUNK):
     return int(_lib.hqmq_outlier_workspace_size(B, H, T, D, gran))
 
 
+def hqmq_encode_med3_workspace_size(B, H, T, D, gran=HQMQ_GRAN_CHUNK):
+    return int(_lib.hqmq_encode_med3_workspace_size(B, H, T, D, gran))
+
+
 # ---------------------------------------------------------------- calls
 def hqmq_make_codebook(seed, S, n_groups, group0, codebook, stream=None):
     """codebook: fp32 device tensor of n_groups * S * 4 elements."""
@@ -170,6 +178,17 @@ def hqmq_encode_lut(x, codebook, S, table, thr, gran, idx_words, radius, status=
     _check("hqmq_encode_lut", _lib.hqmq_encode_lut(
         _ptr(x), _dtype_code(x), B, H, T, D, _ptr(codebook), S, _ptr(table), _ptr(thr), gran,
         _ptr(idx_words), _ptr(radius), _ptr(status), _stream(stream)))
+
+
+def hqmq_encode_med3(x, C, gran, codebook, S, table, idx_words, radius, rmed, thr, out_idx,
+                     out_val, slab_off, cap, ws, status=None, stream=None):
+    """Med3x + encode in two reads of x (table may be None: S-codeword loop)."""
+    B, H, T, D = _shape4(x)
+    _check("hqmq_encode_med3", _lib.hqmq_encode_med3(
+        _ptr(x), _dtype_code(x), B, H, T, D, float(C), gran, _ptr(codebook), S, _ptr(table),
+        _ptr(idx_words), _ptr(radius), _ptr(rmed), _ptr(thr), _ptr(out_idx), _ptr(out_val),
+        _ptr(slab_off), int(cap), _ptr(ws), ws.numel() * ws.element_size(), _ptr(status),
+        _stream(stream)))
 
 
 def hqmq_decode(idx_words, radius, codebook, S, out_idx, out_val, slab_off, cap, gran, y,

@@ -1,0 +1,151 @@
+"""Med3x in two reads (hqmq_outlier_extract's window pipeline and the fused
+hqmq_encode_med3) against the oracle, including inputs built to defeat the
+sample window (so the exact fallback decides) and to overflow its buffers."""
+import numpy as np
+import pytest
+import torch
+
+from _parity import (check_codes, check_med3, gpu_search_table, same_f16_or_bf16_bits, same_f32,
+                     to_host, unpack_indices)
+
+pytestmark = pytest.mark.gpu
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+from kv_cache_quantization_hqmq_b200 import hqmq  # noqa: E402
+from kv_cache_quantization_hqmq_b200 import workloads as W  # noqa: E402
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def x_dev(x):
+    return dev(x.view(np.int16)).view(torch.bfloat16) if x.dtype == np.uint16 else dev(x)
+
+
+def fused(x_np, cb_np, S, gran, use_table, C=3.0, cap=None):
+    B, H, T, D = x_np.shape
+    xd = x_dev(x_np)
+    cbd = dev(cb_np.reshape(-1))
+    n = B * H * T * D // 4 if gran == 0 else B * H * T * D
+    cap = n if cap is None else cap
+    table = gpu_search_table(cbd, S, H) if use_table else None
+    words, radius = hqmq.alloc_codes(B, H, T, D, S)
+    rmed, thr, oi, ov, so, _ = hqmq.alloc_outliers(B, H, T, D, cap, gran)
+    ws = torch.empty(hqmq.hqmq_encode_med3_workspace_size(B, H, T, D, gran), dtype=torch.uint8,
+                     device="cuda")
+    st = hqmq.new_status()
+    hqmq.hqmq_encode_med3(xd, C, gran, cbd, S, table, words, radius, rmed, thr, oi, ov, so, cap,
+                          ws, st)
+    torch.cuda.synchronize()
+    return dict(words=words, radius=radius, rmed=rmed, thr=thr, out_idx=oi, out_val=ov,
+                slab_off=so, cap=cap, status=hqmq.read_status(st))
+
+
+def check_fused(oracle, x_np, S, gran, use_table, seed=1, cap=None):
+    B, H, T, D = x_np.shape
+    cb = oracle.make_codebook(seed, S, H)
+    g = fused(x_np, cb, S, gran, use_table, cap=cap)
+    thr_o, *_ = check_med3(oracle, x_np, g, 3.0, gran)
+    gi = unpack_indices(to_host(g["words"]), S, B * H * T * D // 4)
+    n, mm, near = check_codes(oracle, x_np, cb, S, gi, to_host(g["radius"]), thr=thr_o, gran=gran)
+    print("[fused] %s gran %d table %d: %d chunks, %d near-tie mismatches, %d outliers"
+          % (x_np.shape, gran, use_table, n, mm, g["status"]["n_outliers"]))
+    return g
+
+
+@pytest.mark.parametrize("use_table", [True, False])
+@pytest.mark.parametrize("gran", [0, 1])
+def test_fused_qwen(oracle, gran, use_table):
+    w = W.WORKLOADS["qwen_outlier"]
+    x = W.as_numpy_bits(W.make_call_input(w, 4, 1, tokens=1024))
+    g = check_fused(oracle, x, w.S, gran, use_table)
+    if gran == 0:   # chunk norms: the sample window holds (element mode may fall back here)
+        assert not g["status"]["flags"] & hqmq.FLAG_MED3_FALLBACK
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 32, 4), (2, 3, 8, 64), (3, 2, 200, 128),
+                                   (1, 1, 4100, 128), (8, 2, 96, 128)])
+def test_fused_shapes(oracle, shape):
+    rng = np.random.default_rng(sum(shape) + 7)
+    x = (rng.standard_t(3, shape) * 1.5).astype(np.float32)
+    x = W.as_numpy_bits(torch.from_numpy(x).to(torch.bfloat16))
+    check_fused(oracle, x, 8, 0, True)
+    check_fused(oracle, x, 8, 1, True)
+
+
+def test_fused_fp32_input(oracle):
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((2, 2, 64, 128)).astype(np.float32)
+    x.reshape(-1, 4)[::37] *= 20.0
+    check_fused(oracle, x, 32, 0, True)
+
+
+def test_window_miss_takes_the_exact_fallback(oracle):
+    # the sample reads, in the q-th period of 128 chunks of a slab, the quad of
+    # chunks in slot (37 q) mod 32: make exactly those huge, so that the
+    # sampled median is far above the true one
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((1, 2, 512, 128)).astype(np.float32)
+    c = x.reshape(1, 2, -1, 4)
+    pos = np.arange(c.shape[2])
+    sampled = (pos % 128) // 4 == (37 * (pos // 128)) % 32
+    c[:, :, sampled] *= 1000.0
+    x = W.as_numpy_bits(torch.from_numpy(x).to(torch.bfloat16))
+    g = check_fused(oracle, x, 8, 0, True)
+    assert g["status"]["flags"] & hqmq.FLAG_MED3_FALLBACK
+    check_fused(oracle, x, 8, 1, False)
+
+
+def test_uncertain_band_overflow_takes_the_exact_fallback(oracle):
+    # half of the chunks at norm 1, half just around 3: every chunk of the
+    # second half sits in the threshold's uncertainty band
+    rng = np.random.default_rng(5)
+    n = 1 * 1 * 2048 * 32
+    u = rng.standard_normal((n, 4))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    r = np.where(np.arange(n) % 2 == 0, 1.0, 3.0 * (1 + 1e-3 * rng.standard_normal(n)))
+    x = (u * r[:, None]).astype(np.float32).reshape(1, 1, 2048, 128)
+    g = check_fused(oracle, x, 8, 0, True)
+    assert g["status"]["flags"] & hqmq.FLAG_MED3_FALLBACK
+
+
+def test_fused_capacity_overflow(oracle):
+    w = W.WORKLOADS["qwen_outlier"]
+    x = W.as_numpy_bits(W.make_call_input(w, 0, 0, tokens=256))
+    g = check_fused(oracle, x, w.S, 0, True, cap=50)
+    assert g["status"]["flags"] & hqmq.FLAG_OUTLIER_OVERFLOW
+
+
+def test_fused_equals_separate_calls_full_size_70b(oracle):
+    # one full 70B call: fused (two reads) vs hqmq_outlier_extract +
+    # hqmq_encode_lut (the same kernels' results by definition): bit-identical
+    w = W.WORKLOADS["llama3_70b_128k"]
+    B, H, T, D = w.call_shape
+    xd = W.make_call_input(w, 11, 0, device="cuda")
+    cb = torch.empty(H * w.S * 4, dtype=torch.float32, device="cuda")
+    hqmq.hqmq_make_codebook(w.codebook_seed, w.S, H, W.group0(11, 0, H), cb)
+    table = gpu_search_table(cb, w.S, H)
+    cap = B * H * T * D // 4 // 10
+    words, radius = hqmq.alloc_codes(B, H, T, D, w.S)
+    rmed, thr, oi, ov, so, ws = hqmq.alloc_outliers(B, H, T, D, cap)
+    st = hqmq.new_status()
+    hqmq.hqmq_encode_med3(xd, w.C, 0, cb, w.S, table, words, radius, rmed, thr, oi, ov, so, cap,
+                          ws, st)
+    words2, radius2 = hqmq.alloc_codes(B, H, T, D, w.S)
+    rmed2, thr2, oi2, ov2, so2, ws2 = hqmq.alloc_outliers(B, H, T, D, cap)
+    st2 = hqmq.new_status()
+    hqmq.hqmq_outlier_extract(xd, w.C, 0, rmed2, thr2, oi2, ov2, so2, cap, ws2, st2)
+    hqmq.hqmq_encode_lut(xd, cb, w.S, table, thr2, 0, words2, radius2, st2)
+    torch.cuda.synchronize()
+    for a, b in ((words, words2), (radius, radius2), (thr, thr2), (so, so2)):
+        assert torch.equal(a, b)
+    n = int(so[-1])
+    assert torch.equal(oi[:n], oi2[:n]) and torch.equal(ov[:4 * n], ov2[:4 * n])
+    assert hqmq.read_status(st) == hqmq.read_status(st2)
+    assert not hqmq.read_status(st)["flags"] & hqmq.FLAG_MED3_FALLBACK
+    # and the median / threshold equal the oracle's
+    x = W.as_numpy_bits(xd)
+    rmed_o, thr_o = oracle.med3_threshold(x, w.C, 0)
+    assert same_f32(to_host(thr), thr_o).all()

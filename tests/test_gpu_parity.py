@@ -260,8 +260,11 @@ def _full_size_call(oracle, name, layer, role, n_sample=20000, gran=0, encoder="
     if w.med3:
         med = gpu_med3(xd, w.C, gran)
         thr_o, oi_o, ov_o, so_o, n_o = check_med3(oracle, x, med, w.C, gran)
-        print("[parity] %s L%d role %d: %d outliers (%.3f%%)" % (
-            name, layer, role, n_o, 100.0 * n_o / (B * H * T * D / (4 if gran == 0 else 1))))
+        print("[parity] %s L%d role %d: %d outliers (%.3f%%), status flags %d" % (
+            name, layer, role, n_o, 100.0 * n_o / (B * H * T * D / (4 if gran == 0 else 1)),
+            med["status"]["flags"]))
+        if gran == 0:
+            assert not med["status"]["flags"] & hqmq.FLAG_MED3_FALLBACK
     words, radius, st = gpu_encode(xd, cbd, w.S, med["thr"] if med else None, gran, encoder)
     n_chunks = B * H * T * D // 4
     gi = unpack_indices(to_host(words), w.S, n_chunks)

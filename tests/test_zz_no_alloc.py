@@ -49,6 +49,9 @@ def test_noalloc_matches_workspace_entry_point_twice(gran):
         b, sb = _run(x, gran, cap, noalloc=False)
         for u, v in zip(a, b):
             assert np.array_equal(u.view(np.uint8), v.view(np.uint8))
+        # the workspace entry point may report that its sampled median window
+        # fell back to the exact path (a diagnostic bit this one never sets)
+        sb["flags"] &= ~hqmq.FLAG_MED3_FALLBACK
         assert sa == sb and sa["n_outliers"] > 0
 
 
