@@ -33,7 +33,7 @@ namespace hqmq {
 
 constexpr int WIN_THREADS = 1024;
 constexpr int PB_THREADS = 256;
-constexpr int FINAL_KEYS = 4096;   // keys of one fine bin held in shared memory
+constexpr int FINAL_KEYS = 8192;   // per-key counters of one fine bin (bin width <= 2^13)
 
 __device__ __forceinline__ float key_to_float(uint32_t k) {
     return k >= 0x7F800001u ? __int_as_float(0x7FC00000) : __uint_as_float(k);
@@ -60,9 +60,17 @@ __device__ __forceinline__ void chunk_keys(float x0, float x1, float x2, float x
 // ---------------------------------------------------------------------------
 // A: sample histogram
 // ---------------------------------------------------------------------------
+constexpr int SAMPLE_THREADS = 1024;
+
 template <int DT, int GRAN>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(SAMPLE_THREADS)
 k_sample_hist(const void *__restrict__ x, int H, uint32_t cps, uint32_t *__restrict__ hist) {
+    // per-CTA histogram in shared memory: 65536 16-bit counters packed in
+    // pairs (a CTA sees far fewer than 65536 samples), then one global add
+    // per non-empty bin
+    extern __shared__ uint32_t s_pair[];                       // [KEY_BINS / 2]
+    for (int i = threadIdx.x; i < KEY_BINS / 2; i += blockDim.x) s_pair[i] = 0;
+    __syncthreads();
     const int slab = blockIdx.y;
     uint32_t *hh = hist + (size_t)(slab % H) * KEY_BINS;
     const uint64_t base = (uint64_t)slab * cps;
@@ -75,51 +83,99 @@ k_sample_hist(const void *__restrict__ x, int H, uint32_t cps, uint32_t *__restr
         const uint32_t slot = (37u * q) & 31u;
         uint64_t j0 = base + (uint64_t)q * SAMPLE_PERIOD + 4u * slot;
         if (j0 + 4 > base + cps) j0 = base + (uint64_t)q * SAMPLE_PERIOD;   // short last period
+        RawChunk<DT> v[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c].load(x, j0 + c);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            RawChunk<DT> v;
-            v.load(x, j0 + c);
             constexpr int NK = GRAN == HQMQ_GRAN_CHUNK ? 1 : 4;
             uint32_t k[4];
-            chunk_keys<GRAN>(v.e(0), v.e(1), v.e(2), v.e(3), k);
+            chunk_keys<GRAN>(v[c].e(0), v[c].e(1), v[c].e(2), v[c].e(3), k);
 #pragma unroll
-            for (int i = 0; i < NK; ++i) atomicAdd(hh + (k[i] >> 15), 1u);
+            for (int i = 0; i < NK; ++i) {
+                const uint32_t bin = k[i] >> 15;
+                atomicAdd(&s_pair[bin >> 1], 1u << ((bin & 1) * 16));
+            }
         }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < KEY_BINS / 2; i += blockDim.x) {
+        const uint32_t v = s_pair[i];
+        if (v & 0xFFFFu) atomicAdd(hh + 2 * i, v & 0xFFFFu);
+        if (v >> 16) atomicAdd(hh + 2 * i + 1, v >> 16);
     }
 }
 
-// Block-wide: the bin whose cumulative count first exceeds `rank` (bins of
-// 64 consecutive entries per thread, 1024 threads).
-__device__ void find_rank_bin(const uint32_t *__restrict__ hist, uint64_t rank, uint32_t *s_warp,
-                              uint32_t *s_out, int which) {
-    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
-    uint32_t local = 0;
-    for (int i = 0; i < 64; ++i) local += hist[t * 64 + i];
-    uint32_t inc = local;
+// Block-wide (1024 threads = 32 warps) search of a histogram of NB bins, warp
+// w owning the contiguous bins [w NB/32, (w+1) NB/32), read coalesced:
+// rank_bin_totals() stores the warp totals and the totals of every block of
+// 32 bins; rank_bin_find() then locates the warp, the block (from the block
+// totals) and the bin (one 32-bin read), and returns in s_out[which] the bin
+// whose cumulative count first exceeds `rank` and in s_out[which + 2] the
+// rank inside that bin.
+template <int NB>
+__device__ void rank_bin_totals(const uint32_t *hist, uint32_t *s_wtot, uint32_t *s_blk) {
+    constexpr int PER = NB / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint32_t acc = 0;
+    for (int i = 0; i < PER; i += 32) {
+        const uint32_t bt = __reduce_add_sync(FULL, hist[w * PER + i + lane]);
+        if (lane == 0) s_blk[(w * PER + i) / 32] = bt;
+        acc += bt;
+    }
+    if (lane == 0) s_wtot[w] = acc;
+    __syncthreads();
+}
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        uint32_t v = __shfl_up_sync(FULL, inc, o);
-        if (lane >= o) inc += v;
+        const uint32_t u = __shfl_up_sync(FULL, v, o);
+        if (lane >= o) v += u;
     }
-    if (lane == 31) s_warp[wid] = inc;
-    __syncthreads();
-    if (wid == 0) {
-        uint32_t w = s_warp[lane], wi = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            uint32_t v = __shfl_up_sync(FULL, wi, o);
-            if (lane >= o) wi += v;
+    return v;
+}
+
+template <int NB>
+__device__ void rank_bin_find(const uint32_t *hist, const uint32_t *s_wtot,
+                              const uint32_t *s_blk, uint64_t rank, uint32_t *s_out, int which) {
+    constexpr int PER = NB / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint64_t cum = 0;
+    int ww = 31;
+    for (int k = 0; k < 32; ++k) {
+        const uint32_t t = s_wtot[k];
+        if (rank < cum + t) { ww = k; break; }
+        cum += t;
+    }
+    if (w == ww) {
+        uint64_t c = cum;
+        int blk = -1;
+        for (int i = 0; i < PER / 32; i += 32) {             // block totals of this warp
+            const uint32_t v = (i + lane < PER / 32) ? s_blk[ww * (PER / 32) + i + lane] : 0u;
+            const uint32_t inc = warp_incl_scan(v, lane);
+            const uint32_t tot = __shfl_sync(FULL, inc, 31);
+            if (rank < c + tot) {
+                const uint32_t bal = __ballot_sync(FULL, rank < c + inc);
+                const int src = __ffs(bal) - 1;
+                blk = i + src;
+                c += __shfl_sync(FULL, inc - v, src);
+                break;
+            }
+            c += tot;
         }
-        s_warp[lane] = wi - w;
-    }
-    __syncthreads();
-    const uint64_t excl = (uint64_t)s_warp[wid] + inc - local;
-    if (rank >= excl && rank < excl + local) {
-        uint64_t c = excl;
-        for (int i = 0; i < 64; ++i) {
-            const uint32_t n = hist[t * 64 + i];
-            if (rank < c + n) { s_out[which] = t * 64 + i; s_out[which + 2] = (uint32_t)(rank - c); break; }
-            c += n;
+        if (blk >= 0) {                   // (rank below the total, as the callers ensure)
+            const uint32_t v = hist[ww * PER + blk * 32 + lane];
+            const uint32_t inc = warp_incl_scan(v, lane);
+            const bool mine = rank >= c + inc - v && rank < c + inc;
+            const uint32_t bal = __ballot_sync(FULL, mine);
+            if (lane == __ffs(bal) - 1) {
+                s_out[which] = (uint32_t)(ww * PER + blk * 32 + lane);
+                s_out[which + 2] = (uint32_t)(rank - (c + inc - v));
+            }
+        } else if (lane == 0) {
+            s_out[which] = NB - 1;
+            s_out[which + 2] = 0;
         }
     }
     __syncthreads();
@@ -132,28 +188,24 @@ __global__ void __launch_bounds__(WIN_THREADS)
 k_window_select(uint64_t n_per_head, float C, const uint32_t *__restrict__ sample_hist,
                 uint32_t *__restrict__ fine_hist, WinState *__restrict__ win,
                 unsigned long long *__restrict__ below, unsigned long long *__restrict__ cand_n) {
-    __shared__ uint32_t s_warp[32];
+    __shared__ uint32_t s_wtot[32];
+    __shared__ uint32_t s_blk[KEY_BINS / 32];
     __shared__ uint32_t s_out[4];
-    __shared__ unsigned long long s_tot;
     const int h = blockIdx.x;
     const uint32_t *hist = sample_hist + (size_t)h * KEY_BINS;
     uint32_t *fh = fine_hist + (size_t)h * KEY_BINS;
     for (int i = threadIdx.x; i < KEY_BINS; i += WIN_THREADS) fh[i] = 0;
-    if (threadIdx.x == 0) s_tot = 0;
-    __syncthreads();
-    uint32_t local = 0;
-    for (int i = threadIdx.x; i < KEY_BINS; i += WIN_THREADS) local += hist[i];
-    local = __reduce_add_sync(FULL, local);
-    if ((threadIdx.x & 31) == 0) atomicAdd(&s_tot, (unsigned long long)local);
-    __syncthreads();
-    const double ns = (double)s_tot;
+    rank_bin_totals<KEY_BINS>(hist, s_wtot, s_blk);
+    uint64_t tot = 0;
+    for (int k = 0; k < 32; ++k) tot += s_wtot[k];
+    const double ns = (double)tot;
     const double q = ((double)(n_per_head / 2 - 1) + 0.5) / (double)n_per_head;
     const double half = WINDOW_SIGMAS * 0.5 * sqrt(ns) + 4.0;
     double rlo = floor(q * ns - half), rhi = ceil(q * ns + half);
     if (rlo < 0) rlo = 0;
     if (rhi > ns - 1) rhi = ns - 1;
-    find_rank_bin(hist, (uint64_t)rlo, s_warp, s_out, 0);
-    find_rank_bin(hist, (uint64_t)rhi, s_warp, s_out, 1);
+    rank_bin_find<KEY_BINS>(hist, s_wtot, s_blk, (uint64_t)rlo, s_out, 0);
+    rank_bin_find<KEY_BINS>(hist, s_wtot, s_blk, (uint64_t)rhi, s_out, 1);
     if (threadIdx.x == 0) {
         WinState w;
         const uint64_t lo = (uint64_t)s_out[0] << 15;
@@ -296,50 +348,42 @@ k_med_final(uint64_t n_per_head, float C, WinState *__restrict__ win,
             uint64_t cand_cap, const uint32_t *__restrict__ fine_hist,
             const unsigned long long *__restrict__ amb_n, uint64_t amb_cap,
             float *__restrict__ rmed, float *__restrict__ thr) {
-    __shared__ uint32_t s_warp[32];
+    __shared__ uint32_t s_wtot[32];
+    __shared__ uint32_t s_blk[KEY_BINS / 32];
     __shared__ uint32_t s_out[4];
-    __shared__ uint32_t s_keys[FINAL_KEYS];
-    __shared__ unsigned int s_n;
+    __shared__ uint32_t s_cnt[FINAL_KEYS];             // one counter per key of the bin
     const int h = blockIdx.x;
     const WinState w = win[h];
     const long long k = (long long)(n_per_head / 2 - 1) - (long long)below[h];
     const unsigned long long nc = cand_n[h];
-    const bool miss = (*amb_n > amb_cap) || k < 0 || (unsigned long long)k >= nc || nc > cand_cap;
-    if (miss) {                                            // block-uniform
+    const bool miss = (*amb_n > amb_cap) || k < 0 || (unsigned long long)k >= nc ||
+                      nc > cand_cap || (1u << w.shift) > (uint32_t)FINAL_KEYS;
+    if (miss) {                                        // block-uniform
         if (threadIdx.x == 0) win[h].miss = 1;
         return;
     }
-    if (threadIdx.x == 0) s_n = 0;
-    find_rank_bin(fine_hist + (size_t)h * KEY_BINS, (uint64_t)k, s_warp, s_out, 0);
-    const uint32_t bin = s_out[0];
-    const uint32_t kk = s_out[2];                          // rank inside the bin
+    const uint32_t *fh = fine_hist + (size_t)h * KEY_BINS;
+    rank_bin_totals<KEY_BINS>(fh, s_wtot, s_blk);
+    rank_bin_find<KEY_BINS>(fh, s_wtot, s_blk, (uint64_t)k, s_out, 0);
+    const uint32_t bin_lo = w.lo_key + (s_out[0] << w.shift);
+    const uint32_t kk = s_out[2];                      // rank inside the fine bin
+    const uint32_t width = 1u << w.shift;
+    for (uint32_t i = threadIdx.x; i < (uint32_t)FINAL_KEYS; i += WIN_THREADS) s_cnt[i] = 0;
+    __syncthreads();
+    // count every candidate key of the bin by its exact value (bf16 inputs
+    // repeat values, so a bin may hold many equal keys)
     const uint32_t *ch = cand + (uint64_t)h * cand_cap;
     for (uint64_t i = threadIdx.x; i < nc; i += WIN_THREADS) {
-        const uint32_t key = ch[i];
-        if (((key - w.lo_key) >> w.shift) == bin) {
-            const unsigned int p = atomicAdd(&s_n, 1u);
-            if (p < FINAL_KEYS) s_keys[p] = key;
-        }
+        const uint32_t d = ch[i] - bin_lo;
+        if (d < width) atomicAdd(&s_cnt[d], 1u);
     }
     __syncthreads();
-    const unsigned int n = s_n;
-    if (n > FINAL_KEYS) {
-        if (threadIdx.x == 0) win[h].miss = 1;
-        return;
-    }
-    // rank of each collected key among the bin's keys (ties by position)
-    for (unsigned int i = threadIdx.x; i < n; i += WIN_THREADS) {
-        const uint32_t ki = s_keys[i];
-        unsigned int r = 0;
-        for (unsigned int u = 0; u < n; ++u) {
-            const uint32_t ku = s_keys[u];
-            r += (ku < ki || (ku == ki && u < i)) ? 1u : 0u;
-        }
-        if (r == kk) {
-            const float m = key_to_float(ki);
-            rmed[h] = m;
-            thr[h] = __fmul_rn(C, m);
-        }
+    rank_bin_totals<FINAL_KEYS>(s_cnt, s_wtot, s_blk);
+    rank_bin_find<FINAL_KEYS>(s_cnt, s_wtot, s_blk, kk, s_out, 1);
+    if (threadIdx.x == 0) {
+        const float m = key_to_float(bin_lo + s_out[1]);
+        rmed[h] = m;
+        thr[h] = __fmul_rn(C, m);
     }
 }
 
@@ -466,41 +510,68 @@ k_tile_scan(const uint32_t *__restrict__ tile_cnt, uint64_t n_tiles, uint32_t ti
             uint32_t n_slabs, uint64_t cap, uint32_t *__restrict__ tile_off,
             uint32_t *__restrict__ slab_off, DevStatus *st) {
     __shared__ unsigned long long s_warp[32];
+    __shared__ unsigned long long s_carry;
     const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
-    const uint64_t per = (n_tiles + 1023) / 1024;
-    const uint64_t i0 = (uint64_t)t * per;
-    const uint64_t i1 = min(n_tiles, i0 + per);
-    unsigned long long local = 0;
-    for (uint64_t i = i0; i < i1; ++i) local += tile_cnt[i];
-    unsigned long long inc = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        unsigned long long v = __shfl_up_sync(FULL, inc, o);
-        if (lane >= o) inc += v;
-    }
-    if (lane == 31) s_warp[wid] = inc;
+    if (t == 0) s_carry = 0;
     __syncthreads();
-    if (wid == 0) {
-        unsigned long long wv = s_warp[lane], wi = wv;
+    // blocks of 16384 tiles: thread t scans tiles 16t .. 16t+15 of the block
+    constexpr int PT = 16;
+    for (uint64_t b0 = 0; b0 < n_tiles; b0 += 1024 * PT) {
+        uint32_t v[PT];
+        const uint64_t first = b0 + (uint64_t)PT * t;
+        if (first + PT <= n_tiles) {
+            const uint4 *p4 = reinterpret_cast<const uint4 *>(tile_cnt + first);
+#pragma unroll
+            for (int q = 0; q < PT / 4; ++q) {
+                const uint4 u = p4[q];
+                v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < PT; ++k) v[k] = first + k < n_tiles ? tile_cnt[first + k] : 0u;
+        }
+        unsigned long long local = 0;
+#pragma unroll
+        for (int k = 0; k < PT; ++k) local += v[k];
+        unsigned long long inc = local;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            unsigned long long v = __shfl_up_sync(FULL, wi, o);
-            if (lane >= o) wi += v;
+            const unsigned long long u = __shfl_up_sync(FULL, inc, o);
+            if (lane >= o) inc += u;
         }
-        s_warp[lane] = wi - wv;
+        if (lane == 31) s_warp[wid] = inc;
+        __syncthreads();
+        if (wid == 0) {
+            const unsigned long long wv = s_warp[lane];
+            unsigned long long wi = wv;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long u = __shfl_up_sync(FULL, wi, o);
+                if (lane >= o) wi += u;
+            }
+            s_warp[lane] = wi - wv;
+        }
+        __syncthreads();
+        unsigned long long run = s_carry + s_warp[wid] + inc - local;
+#pragma unroll
+        for (int k = 0; k < PT; ++k) {
+            const uint64_t i = first + k;
+            if (i < n_tiles) {
+                tile_off[i] = (uint32_t)run;
+                if (i % tiles_per_slab == 0) slab_off[i / tiles_per_slab] = (uint32_t)run;
+            }
+            run += v[k];
+        }
+        __syncthreads();
+        if (t == 1023) s_carry = run;
+        __syncthreads();
     }
-    __syncthreads();
-    unsigned long long run = s_warp[wid] + inc - local;
-    for (uint64_t i = i0; i < i1; ++i) {
-        tile_off[i] = (uint32_t)run;
-        if (i % tiles_per_slab == 0) slab_off[i / tiles_per_slab] = (uint32_t)run;
-        run += tile_cnt[i];
-    }
-    if (t == 1023) {
-        slab_off[n_slabs] = (uint32_t)run;   // thread 1023 ends at n_tiles
+    if (t == 0) {
+        const unsigned long long total = s_carry;
+        slab_off[n_slabs] = (uint32_t)total;
         if (st) {
-            atomicAdd(&st->n_outliers, run);
-            if (run > cap) atomicOr(&st->flags, HQMQ_FLAG_OUTLIER_OVERFLOW);
+            atomicAdd(&st->n_outliers, total);
+            if (total > cap) atomicOr(&st->flags, HQMQ_FLAG_OUTLIER_OVERFLOW);
         }
     }
 }
@@ -531,11 +602,20 @@ static int run_window(const void *x, int B, int H, int T, int D, float C, float 
         cudaMemsetAsync(amb_n, 0, 8, stream) != cudaSuccess)
         return HQMQ_ERR_CUDA;
     const uint32_t n_quads = (cps + SAMPLE_PERIOD - 1) / SAMPLE_PERIOD;
-    uint64_t ax = (n_quads + 255) / 256;
-    const uint64_t afill = ((uint64_t)sm_count * 4 + n_slabs - 1) / n_slabs;
+    uint64_t ax = (n_quads + SAMPLE_THREADS - 1) / SAMPLE_THREADS;
+    const uint64_t afill = ((uint64_t)sm_count + n_slabs - 1) / n_slabs;
     if (ax > afill) ax = afill;
+    // 16-bit shared counters: at most 60000 samples per CTA
+    const uint64_t keys_per_quad = 4 * (GRAN == HQMQ_GRAN_CHUNK ? 1 : 4);
+    const uint64_t ax_min = ((uint64_t)n_quads * keys_per_quad + 59999) / 60000;
+    if (ax < ax_min) ax = ax_min;
     if (ax < 1) ax = 1;
-    k_sample_hist<DT, GRAN><<<dim3((unsigned)ax, (unsigned)n_slabs), 256, 0, stream>>>(
+    const size_t sample_smem = (size_t)KEY_BINS / 2 * sizeof(uint32_t);
+    if (cudaFuncSetAttribute(k_sample_hist<DT, GRAN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sample_smem) != cudaSuccess)
+        return HQMQ_ERR_CUDA;
+    k_sample_hist<DT, GRAN><<<dim3((unsigned)ax, (unsigned)n_slabs), SAMPLE_THREADS, sample_smem,
+                              stream>>>(
         x, H, cps, sample_hist);
     k_window_select<<<H, WIN_THREADS, 0, stream>>>(L.n_per_head, C, sample_hist, fine_hist, win,
                                                    below, cand_n);

@@ -41,8 +41,10 @@ constexpr int LUT_CELLS = LUT_G * LUT_G * LUT_G;   // 32768 cells, 512 KB per gr
 constexpr float MAP_A = 1.27323954f;               // 4 / pi (fp32)
 constexpr float MAP_B = 1.0f - MAP_A;              // exact (Sterbenz)
 constexpr int LUT_SLOTS = 8;
-constexpr uint32_t LUT_EMPTY = 0xFFFFu;
-constexpr uint32_t LUT_OVERFLOW = 0xFFFEu;
+// Record: 8 slots of 16 bits; slot k holds candidate id k in its low 12 bits
+// (24 S <= 4096); the top 4 bits of slot 0 hold the count (1..8), 0 marks an
+// overflowing cell; slots past the count repeat candidate 0.
+constexpr uint32_t LUT_ID_MASK = 0x0FFFu;
 constexpr uint32_t LUT_MAX_S = 48;                // 24 S codeword ids fit in 16 bits;
                                                   // shared memory fits 8 copies (144 KB)
 constexpr double LUT_DELTA = 1e-5;                // cell growth in t (fp32 error ~1e-7)
@@ -161,8 +163,9 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
         }
     }
     uint32_t slot[LUT_SLOTS];
-    for (int q = 0; q < LUT_SLOTS; ++q) slot[q] = q < nk ? keep[q] : LUT_EMPTY;
-    if (overflow) slot[0] = LUT_OVERFLOW;
+    if (overflow) nk = 0;
+    for (int q = 0; q < LUT_SLOTS; ++q) slot[q] = nk > 0 ? keep[q < nk ? q : 0] : 0u;
+    slot[0] |= (uint32_t)nk << 12;
     tables[(size_t)g * LUT_CELLS + cell] =
         make_uint4(slot[0] | (slot[1] << 16), slot[2] | (slot[3] << 16),
                    slot[4] | (slot[5] << 16), slot[6] | (slot[7] << 16));
@@ -267,8 +270,21 @@ __device__ __forceinline__ uint64_t shfl64_down(uint64_t v, int d) {
 // Packs the warp's 32 b-bit indices (lane k = chunk k) LSB-first into b words.
 // Each lane first gathers the 64-bit stream window starting at its own chunk
 // (k, k+1, ..., by doubling), then lane w < b takes word w from the window of
-// the chunk where that word starts.  Needs b in [5, 21].
-__device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b, int lane,
+// the chunk where that word starts (k0 = 32 w / b at bit offset o, both
+// computed once per thread).  Needs b in [5, 21].
+struct PackConst {
+    int k0, o;
+};
+
+__device__ __forceinline__ PackConst pack_const(uint32_t b, int lane) {
+    PackConst c;
+    c.k0 = (32 * lane) / (int)b;
+    c.o = 32 * lane - c.k0 * (int)b;               // < b, and o + 32 <= 64
+    c.k0 &= 31;
+    return c;
+}
+
+__device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b, int lane, PackConst pc,
                                              uint32_t *__restrict__ dst) {
     uint64_t v = idx;
     const uint32_t n1 = __shfl_down_sync(FULL, idx, 1);
@@ -277,10 +293,27 @@ __device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b, int lane,
     if (lane + 2 < 32) v |= v2 << (2 * b);                 // 2b <= 42
     const uint64_t v4 = shfl64_down(v, 4);
     if (lane + 4 < 32 && 4 * b < 64) v |= v4 << (4 * b);
-    const int k0 = (32 * lane) / (int)b;
-    const int o = 32 * lane - k0 * (int)b;                   // < b, and o + 32 <= 64
-    const uint64_t vk = shfl64(v, k0 & 31);
-    if (lane < (int)b) dst[lane] = (uint32_t)(vk >> o);
+    const uint64_t vk = shfl64(v, pc.k0);
+    if (lane < (int)b) dst[lane] = (uint32_t)(vk >> pc.o);
+}
+
+// Best candidate among the first `cnt` of a record with exact ties broken by
+// the lowest original index (the rare path, taken only when two candidates
+// score exactly the same).
+__device__ __noinline__ uint32_t best_with_ties(uint4 rec, uint32_t cnt, float y0, float y1,
+                                                float y2, float y3, const float4 *s_tab,
+                                                uint32_t lane7, const uint8_t *mul_row) {
+    float best = __int_as_float(0xFF800000);
+    uint32_t bmap = 0xFFFFFFFFu;
+    for (uint32_t k = 0; k < cnt; ++k) {
+        const uint32_t word = k < 2 ? rec.x : k < 4 ? rec.y : k < 6 ? rec.z : rec.w;
+        const uint32_t id = (word >> ((k & 1) * 16)) & LUT_ID_MASK;
+        const float4 c = s_tab[(id << 3) | lane7];
+        const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z, __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
+        const uint32_t m = (id / 24u) * 24u + mul_row[id % 24u];
+        if (sc > best || (sc == best && m < bmap)) { best = sc; bmap = m; }
+    }
+    return bmap;
 }
 
 // LIST: 0 = no list; HQMQ_GRAN_CHUNK + 1 / HQMQ_GRAN_ELEMENT + 1 = write the
@@ -303,6 +336,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
     const int n_warps = ENC_THREADS / 32;
     const uint32_t n_words = 24u * S;
     const uint32_t lane7 = (uint32_t)(lane & 7);
+    const PackConst pc = pack_const(b, lane);
     if (ENC)
         for (int i = threadIdx.x; i < 8 * 24; i += ENC_THREADS)
             s_mul[i / 24][i % 24] = (uint8_t)mul_2t(i / 24, i % 24);
@@ -399,11 +433,11 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 }
                 const bool finite = r == r && r != __int_as_float(0x7F800000);
                 const bool search = finite && r > 0.0f;
-                // every lane takes part in the candidate loop (it votes); lanes
-                // without a search carry an all-empty record
+                // every lane runs the candidate loop up to the warp's longest
+                // list (lanes without a search score candidate 0 of cell 0)
                 float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
                 int pu = 0;
-                uint4 rec = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+                uint4 rec = make_uint4(1u << 12, 0u, 0u, 0u);
                 if (search) {
                     pu = fold(x0, x1, x2, x3, y0, y1, y2, y3);
                     float inv;
@@ -412,36 +446,29 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                                      cell_coord(y3 * inv);
                     rec = __ldg(tb + cell);
                 }
-                const bool fallback = (rec.x & 0xFFFFu) == LUT_OVERFLOW;
-                if (fallback) rec = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+                const uint32_t cnt = (rec.x >> 12) & 0xFu;
+                const bool fallback = cnt == 0;                    // overflowing cell
                 const uint32_t sl[4] = {rec.x, rec.y, rec.z, rec.w};
-                const uint32_t id0 = rec.x & 0xFFFFu;
-                float best = __int_as_float(0xFF800000);     // -inf
-                uint32_t bid = 0;
-                uint32_t bmap = 0xFFFFFFFFu;
+                const uint32_t kmax = __reduce_max_sync(FULL, cnt);
+                float best = __int_as_float(0xFF800000);           // -inf
+                uint32_t bid = rec.x & LUT_ID_MASK;
+                bool tie = false;
 #pragma unroll
                 for (int k = 0; k < LUT_SLOTS; ++k) {
-                    const uint32_t idk = (sl[k >> 1] >> ((k & 1) * 16)) & 0xFFFFu;
-                    if (!__any_sync(FULL, idk != LUT_EMPTY)) break;
-                    // a lane whose list is shorter re-scores its first candidate
-                    const uint32_t id = idk != LUT_EMPTY ? idk : id0;
-                    if (id0 != LUT_EMPTY) {
-                        const float4 c = s_tab[(id << 3) | lane7];
-                        const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z,
-                                         __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
-                        if (sc > best) {
-                            best = sc; bid = id; bmap = 0xFFFFFFFFu;
-                        } else if (sc == best && id != bid) {   // exact tie: lowest original index
-                            if (bmap == 0xFFFFFFFFu)
-                                bmap = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
-                            const uint32_t m = (id / 24u) * 24u + s_mul[pu][id % 24u];
-                            if (m < bmap) { bid = id; bmap = m; }
-                        }
-                    }
+                    if ((uint32_t)k >= kmax) break;                // warp-uniform
+                    const uint32_t id = (sl[k >> 1] >> ((k & 1) * 16)) & LUT_ID_MASK;
+                    const float4 c = s_tab[(id << 3) | lane7];
+                    const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z,
+                                     __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
+                    tie |= (sc == best) & (id != bid);
+                    if (sc > best) { best = sc; bid = id; }
                 }
                 uint32_t idx = 0;
                 if (search && !fallback) idx = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
-                if (fallback) idx = sloop_index(x0, x1, x2, x3, cb, S);
+                if (__any_sync(FULL, search && tie && !fallback))  // exact ties: rare
+                    if (search && tie && !fallback)
+                        idx = best_with_ties(rec, cnt, y0, y1, y2, y3, s_tab, lane7, s_mul[pu]);
+                if (search && fallback) idx = sloop_index(x0, x1, x2, x3, cb, S);
                 uint16_t rh;
                 if (!finite) {
                     rh = 0x7E00u;
@@ -452,7 +479,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                     n_sat += sat;
                 }
                 radius[G * 32 + lane] = rh;
-                pack_group32(idx, b, lane, words + G * b);
+                pack_group32(idx, b, lane, pc, words + G * b);
             }
         }
         seg = seg_end;

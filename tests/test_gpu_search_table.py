@@ -4,8 +4,8 @@ boundaries, on Voronoi boundaries between codewords) the exact fp64 argmax of
 <x, c> over all 24 S codewords is in the list of x's cell, computed here
 independently in numpy from the table's documented layout (fold by the unit of
 the largest coordinate, gnomonic coordinates t, u = t (A + B t^2) with
-A = fp32(4/pi), B = 1 - A, 32^3 cells in u, 8 uint16 slots, 0xFFFF empty,
-0xFFFE overflow).  A point within 1e-6 of a cell face is checked against the
+A = fp32(4/pi), B = 1 - A, 32^3 cells in u, 8 uint16 slots holding 12-bit
+candidate ids, the top 4 bits of slot 0 holding the count, 0 = overflow).  A point within 1e-6 of a cell face is checked against the
 cells on both sides (the kernel's fp32 arithmetic may pick either)."""
 import itertools
 import numpy as np
@@ -66,9 +66,12 @@ def cell_candidates(y, eps=1e-6):
 def test_table_lists_contain_the_exact_argmax(oracle, S):
     cb = oracle.make_codebook(5, S, 1)
     tab = to_host(gpu_search_table(torch.from_numpy(cb.reshape(-1)).cuda(), S, 1))
-    rec = tab.view(np.uint16).reshape(G ** 3, 8).astype(np.int64)
-    overflow = rec[:, 0] == 0xFFFE
-    assert not np.any((rec[:, 0] == 0xFFFF))          # every cell lists something
+    raw = tab.view(np.uint16).reshape(G ** 3, 8).astype(np.int64)
+    count = raw[:, 0] >> 12
+    overflow = count == 0
+    rec = raw & 0xFFF
+    rec[np.arange(8)[None, :] >= count[:, None]] = 0xFFFF    # past the count: not listed
+    assert np.all(count <= 8) and np.all(rec[:, 0] < 24 * S)
     assert overflow.mean() < 0.01
     cw = np.array([oracle.codeword(i % 24, cb[0, i // 24]) for i in range(24 * S)], np.float64)
     rng = np.random.default_rng(S)
