@@ -131,44 +131,56 @@ k_decode_outliers(const uint32_t *__restrict__ words, const uint16_t *__restrict
                   void *__restrict__ y) {
     uint64_t n = slab_off[n_slabs];
     if (n > cap) n = cap;
-    for (uint64_t q = (uint64_t)blockIdx.x * OUT_THREADS + threadIdx.x; q < n;
-         q += (uint64_t)gridDim.x * OUT_THREADS) {
-        const uint64_t e = __ldg(out_idx + q);
-        if (GRAN == HQMQ_GRAN_CHUNK) {
-            if (e >= n_chunks) continue;
-            const uint32_t *vv = reinterpret_cast<const uint32_t *>(out_val + q * 4);
-            const uint32_t v01 = __ldg(vv), v23 = __ldg(vv + 1);
-            const float f0 = f16_bits_to_f32(v01 & 0xFFFFu), f1 = f16_bits_to_f32(v01 >> 16);
-            const float f2 = f16_bits_to_f32(v23 & 0xFFFFu), f3 = f16_bits_to_f32(v23 >> 16);
-            if (OUT_DT == HQMQ_BF16) {
-                __nv_bfloat162 a0 = __floats2bfloat162_rn(f0, f1);
-                __nv_bfloat162 a1 = __floats2bfloat162_rn(f2, f3);
-                uint2 o;
-                o.x = *reinterpret_cast<uint32_t *>(&a0);
-                o.y = *reinterpret_cast<uint32_t *>(&a1);
-                reinterpret_cast<uint2 *>(y)[e] = o;
+    const uint64_t stride = (uint64_t)gridDim.x * OUT_THREADS;
+    for (uint64_t q0 = (uint64_t)blockIdx.x * OUT_THREADS + threadIdx.x; q0 < n;
+         q0 += 4 * stride) {
+        uint32_t ev[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {                 // four independent entries in flight
+            const uint64_t q = q0 + u * stride;
+            ev[u] = q < n ? __ldg(out_idx + q) : 0xFFFFFFFFu;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint64_t q = q0 + u * stride;
+            if (q >= n) break;
+            const uint64_t e = ev[u];
+            if (GRAN == HQMQ_GRAN_CHUNK) {
+                if (e >= n_chunks) continue;
+                const uint32_t *vv = reinterpret_cast<const uint32_t *>(out_val + q * 4);
+                const uint32_t v01 = __ldg(vv), v23 = __ldg(vv + 1);
+                const float f0 = f16_bits_to_f32(v01 & 0xFFFFu), f1 = f16_bits_to_f32(v01 >> 16);
+                const float f2 = f16_bits_to_f32(v23 & 0xFFFFu), f3 = f16_bits_to_f32(v23 >> 16);
+                if (OUT_DT == HQMQ_BF16) {
+                    __nv_bfloat162 a0 = __floats2bfloat162_rn(f0, f1);
+                    __nv_bfloat162 a1 = __floats2bfloat162_rn(f2, f3);
+                    uint2 o;
+                    o.x = *reinterpret_cast<uint32_t *>(&a0);
+                    o.y = *reinterpret_cast<uint32_t *>(&a1);
+                    reinterpret_cast<uint2 *>(y)[e] = o;
+                } else {
+                    reinterpret_cast<float4 *>(y)[e] = make_float4(f0, f1, f2, f3);
+                }
             } else {
-                reinterpret_cast<float4 *>(y)[e] = make_float4(f0, f1, f2, f3);
+                if (e >= 4 * n_chunks) continue;
+                const uint64_t j = e >> 2;
+                const int i = (int)(e & 3u);
+                const int h = (int)((j / chunks_per_slab) % (uint64_t)H);
+                const uint32_t ix = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
+                float r = f16_bits_to_f32(__ldg(radius + j));
+                float c = 0.0f;
+                if (ix < 24u * S) {
+                    const float4 cw = codeword((int)(ix % 24u), __ldg(cb_all + (size_t)h * S + ix / 24u));
+                    c = i == 0 ? cw.x : i == 1 ? cw.y : i == 2 ? cw.z : cw.w;
+                } else {
+                    r = 0.0f;
+                }
+                const float val = __fadd_rn(__fmul_rn(r, c), f16_bits_to_f32(__ldg(out_val + q)));
+                if (OUT_DT == HQMQ_BF16)
+                    reinterpret_cast<__nv_bfloat16 *>(y)[e] = __float2bfloat16_rn(val);
+                else
+                    reinterpret_cast<float *>(y)[e] = val;
             }
-        } else {
-            if (e >= 4 * n_chunks) continue;
-            const uint64_t j = e >> 2;
-            const int i = (int)(e & 3u);
-            const int h = (int)((j / chunks_per_slab) % (uint64_t)H);
-            const uint32_t ix = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
-            float r = f16_bits_to_f32(__ldg(radius + j));
-            float c = 0.0f;
-            if (ix < 24u * S) {
-                const float4 cw = codeword((int)(ix % 24u), __ldg(cb_all + (size_t)h * S + ix / 24u));
-                c = i == 0 ? cw.x : i == 1 ? cw.y : i == 2 ? cw.z : cw.w;
-            } else {
-                r = 0.0f;
-            }
-            const float val = __fadd_rn(__fmul_rn(r, c), f16_bits_to_f32(__ldg(out_val + q)));
-            if (OUT_DT == HQMQ_BF16)
-                reinterpret_cast<__nv_bfloat16 *>(y)[e] = __float2bfloat16_rn(val);
-            else
-                reinterpret_cast<float *>(y)[e] = val;
         }
     }
 }

@@ -56,6 +56,29 @@ __device__ __forceinline__ uint16_t f32_to_f16_sat(float v, int &sat) {
     return h;
 }
 
+// Two values to packed fp16 bits (a in the low half), same rules as
+// f32_to_f16_sat; the common in-range case is one packed conversion.
+__device__ __forceinline__ uint32_t f32x2_to_f16x2_sat(float a, float b, int &sat) {
+    if (fabsf(a) < 65504.0f && fabsf(b) < 65504.0f) {      // (false for NaN)
+        const __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<const uint32_t *>(&h);
+    }
+    int s0 = 0, s1 = 0;
+    const uint32_t lo = f32_to_f16_sat(a, s0), hi = f32_to_f16_sat(b, s1);
+    sat += s0 + s1;
+    return lo | (hi << 16);
+}
+
+// A finite, non-negative radius to fp16 bits: round to nearest even,
+// saturating at 65504 (values from 65520 up would round to inf).
+__device__ __forceinline__ uint16_t radius_to_f16(float r, int &sat) {
+    if (r >= 65520.0f) {
+        sat = 1;
+        return 0x7BFFu;
+    }
+    return __half_as_ushort(__float2half_rn(r));
+}
+
 __device__ __forceinline__ float f16_bits_to_f32(uint32_t h) {
     return __half2float(__ushort_as_half((unsigned short)h));
 }

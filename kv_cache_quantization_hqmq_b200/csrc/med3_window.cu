@@ -252,7 +252,7 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
          uint32_t *__restrict__ fine_hist, unsigned long long *__restrict__ amb_n,
          uint2 *__restrict__ amb, uint64_t amb_cap, uint32_t *__restrict__ tile_cnt) {
     constexpr int NK = GRAN == HQMQ_GRAN_CHUNK ? 1 : 4;
-    constexpr int U = 4;                              // groups in flight per lane
+    constexpr int U = 8;                              // groups in flight per lane
     const int lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
     const uint32_t gps = cps / 32;

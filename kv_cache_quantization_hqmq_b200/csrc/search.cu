@@ -42,8 +42,9 @@ constexpr float MAP_A = 1.27323954f;               // 4 / pi (fp32)
 constexpr float MAP_B = 1.0f - MAP_A;              // exact (Sterbenz)
 constexpr int LUT_SLOTS = 8;
 // Record: 8 slots of 16 bits; slot k holds candidate id k in its low 12 bits
-// (24 S <= 4096); the top 4 bits of slot 0 hold the count (1..8), 0 marks an
-// overflowing cell; slots past the count repeat candidate 0.
+// (24 S < 4096); the top 4 bits of slot 0 hold the count (1..8), 0 marks an
+// overflowing cell; slots past the count hold the dummy id 24 S, whose
+// shared-memory codeword is zero (score 0, below every real best score).
 constexpr uint32_t LUT_ID_MASK = 0x0FFFu;
 constexpr uint32_t LUT_MAX_S = 48;                // 24 S codeword ids fit in 16 bits;
                                                   // shared memory fits 8 copies (144 KB)
@@ -164,7 +165,7 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
     }
     uint32_t slot[LUT_SLOTS];
     if (overflow) nk = 0;
-    for (int q = 0; q < LUT_SLOTS; ++q) slot[q] = nk > 0 ? keep[q < nk ? q : 0] : 0u;
+    for (int q = 0; q < LUT_SLOTS; ++q) slot[q] = nk > 0 ? (q < nk ? keep[q] : n_words) : 0u;
     slot[0] |= (uint32_t)nk << 12;
     tables[(size_t)g * LUT_CELLS + cell] =
         make_uint4(slot[0] | (slot[1] << 16), slot[2] | (slot[3] << 16),
@@ -284,15 +285,21 @@ __device__ __forceinline__ PackConst pack_const(uint32_t b, int lane) {
     return c;
 }
 
-__device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b, int lane, PackConst pc,
+// BB = the index width when known at compile time (then every shift is a
+// constant), 0 = use b.
+template <int BB>
+__device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b_rt, int lane, PackConst pc,
                                              uint32_t *__restrict__ dst) {
+    const uint32_t b = BB ? (uint32_t)BB : b_rt;
     uint64_t v = idx;
     const uint32_t n1 = __shfl_down_sync(FULL, idx, 1);
     if (lane + 1 < 32) v |= (uint64_t)n1 << b;
     const uint64_t v2 = shfl64_down(v, 2);
     if (lane + 2 < 32) v |= v2 << (2 * b);                 // 2b <= 42
-    const uint64_t v4 = shfl64_down(v, 4);
-    if (lane + 4 < 32 && 4 * b < 64) v |= v4 << (4 * b);
+    if (BB == 0 || 4 * BB < 64) {
+        const uint64_t v4 = shfl64_down(v, 4);
+        if (lane + 4 < 32 && 4 * b < 64) v |= v4 << (4 * b);
+    }
     const uint64_t vk = shfl64(v, pc.k0);
     if (lane < (int)b) dst[lane] = (uint32_t)(vk >> pc.o);
 }
@@ -321,16 +328,17 @@ __device__ __noinline__ uint32_t best_with_ties(uint4 rec, uint32_t cnt, float y
 // Med3x window pipeline).  ENC: encode (else write the list only).
 // Work: warp tiles of TILE_GROUPS consecutive packing groups; a CTA owns a
 // contiguous range of tiles and walks it slab by slab (one head at a time).
-template <int DT, int LIST, bool ENC>
+template <int DT, int LIST, bool ENC, int BB>
 __global__ void __launch_bounds__(ENC_THREADS, 1)
 k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32_t tiles_per_slab,
-             uint64_t n_tiles, const float4 *__restrict__ cb_all, uint32_t S, uint32_t b,
+             uint32_t n_tiles, const float4 *__restrict__ cb_all, uint32_t S, uint32_t b_rt,
              const uint4 *__restrict__ tables, const float *__restrict__ thr, int gran,
              uint32_t *__restrict__ words, uint16_t *__restrict__ radius,
              const uint32_t *__restrict__ tile_off, uint64_t cap, uint32_t *__restrict__ out_idx,
              uint16_t *__restrict__ out_val, DevStatus *st) {
-    extern __shared__ float4 s_tab[];                              // [24 S][8] replicated
-    __shared__ uint8_t s_mul[8][24];                               // u * q_p' for the 8 units
+    extern __shared__ float4 s_tab[];                    // [24 S + 1][8]: codewords, then zero
+    __shared__ uint8_t s_mul[8][24];                     // u * q_p' for the 8 units
+    const uint32_t b = BB ? (uint32_t)BB : b_rt;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = (1u << lane) - 1u;
     const int n_warps = ENC_THREADS / 32;
@@ -341,54 +349,56 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
         for (int i = threadIdx.x; i < 8 * 24; i += ENC_THREADS)
             s_mul[i / 24][i % 24] = (uint8_t)mul_2t(i / 24, i % 24);
 
-    const uint64_t t_begin = n_tiles * blockIdx.x / gridDim.x;
-    const uint64_t t_end = n_tiles * (blockIdx.x + 1) / gridDim.x;
+    // (chunk and list indices fit 32 bits: a call has fewer than 2^32 elements)
+    const uint32_t t_begin = (uint32_t)((uint64_t)n_tiles * blockIdx.x / gridDim.x);
+    const uint32_t t_end = (uint32_t)((uint64_t)n_tiles * (blockIdx.x + 1) / gridDim.x);
+    const uint32_t cap32 = cap < 0xFFFFFFFFull ? (uint32_t)cap : 0xFFFFFFFFu;
     int cur_head = -1;
     unsigned n_nf = 0, n_sat = 0;
-    for (uint64_t seg = t_begin; seg < t_end;) {
-        const uint64_t slab = seg / tiles_per_slab;
-        const uint64_t seg_end = min(t_end, (slab + 1) * tiles_per_slab);
-        const int h = (int)(slab % (uint64_t)H);
+    for (uint32_t seg = t_begin; seg < t_end;) {
+        const uint32_t slab = seg / tiles_per_slab;
+        const uint32_t seg_end = min(t_end, (slab + 1) * tiles_per_slab);
+        const int h = (int)(slab % (uint32_t)H);
         const float4 *cb = cb_all + (size_t)h * S;
         const uint4 *tb = tables + (size_t)h * LUT_CELLS;
-        if (ENC && h != cur_head) {                  // (block-uniform)
+        if (ENC && h != cur_head) {                      // (block-uniform)
             __syncthreads();
-            for (uint32_t i = threadIdx.x; i < n_words * 8; i += ENC_THREADS) {
+            for (uint32_t i = threadIdx.x; i < (n_words + 1) * 8; i += ENC_THREADS) {
                 const uint32_t id = i >> 3;
-                s_tab[i] = codeword((int)(id % 24u), __ldg(cb + id / 24u));
+                s_tab[i] = id < n_words ? codeword((int)(id % 24u), __ldg(cb + id / 24u))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
             }
             __syncthreads();
             cur_head = h;
         }
         const bool med3 = thr != nullptr;
         const float th = med3 ? __ldg(thr + h) : 0.0f;
-        for (uint64_t t = seg + warp; t < seg_end; t += n_warps) {
-            const uint32_t g0 = (uint32_t)(t % tiles_per_slab) * TILE_GROUPS;
+        for (uint32_t t = seg + warp; t < seg_end; t += n_warps) {
+            const uint32_t g0 = (t % tiles_per_slab) * TILE_GROUPS;
             const uint32_t g1 = min(g0 + TILE_GROUPS, groups_per_slab);
-            const uint64_t gbase = slab * groups_per_slab;
-            uint64_t lpos = LIST ? (uint64_t)__ldg(tile_off + t) : 0;   // list position
+            const uint32_t gbase = slab * groups_per_slab;
+            uint32_t lpos = LIST ? __ldg(tile_off + t) : 0u;   // list position
             RawChunk<DT> nxt;
-            nxt.load(x, (gbase + g0) * 32 + lane);
+            nxt.load(x, (size_t)(gbase + g0) * 32 + lane);
             for (uint32_t g = g0; g < g1; ++g) {
-                const uint64_t G = gbase + g;
+                const uint32_t G = gbase + g;
+                const uint32_t j = G * 32 + (uint32_t)lane;   // chunk index
                 const RawChunk<DT> cur = nxt;
-                if (g + 1 < g1) nxt.load(x, (G + 1) * 32 + lane);
+                if (g + 1 < g1) nxt.load(x, (size_t)j + 32);
                 float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
                 float r = chunk_norm(x0, x1, x2, x3);
                 if (LIST == HQMQ_GRAN_CHUNK + 1) {           // ordered chunk list
                     const bool o = r > th;
                     const uint32_t m = __ballot_sync(FULL, o);
                     if (o) {
-                        const uint64_t p = lpos + __popc(m & lt);
-                        if (p < cap) {
-                            int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-                            const uint32_t h0 = f32_to_f16_sat(x0, s0), h1 = f32_to_f16_sat(x1, s1);
-                            const uint32_t h2 = f32_to_f16_sat(x2, s2), h3 = f32_to_f16_sat(x3, s3);
-                            n_sat += s0 + s1 + s2 + s3;
-                            out_idx[p] = (uint32_t)(G * 32 + lane);
-                            uint32_t *vv = reinterpret_cast<uint32_t *>(out_val + p * 4);
-                            vv[0] = h0 | (h1 << 16);
-                            vv[1] = h2 | (h3 << 16);
+                        const uint32_t p = lpos + __popc(m & lt);
+                        if (p < cap32) {
+                            int sv = 0;
+                            const uint32_t h01 = f32x2_to_f16x2_sat(x0, x1, sv);
+                            const uint32_t h23 = f32x2_to_f16x2_sat(x2, x3, sv);
+                            n_sat += sv;
+                            out_idx[p] = j;
+                            reinterpret_cast<uint2 *>(out_val)[p] = make_uint2(h01, h23);
                         }
                     }
                     lpos += __popc(m);
@@ -404,15 +414,15 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                         const uint32_t v = __shfl_up_sync(FULL, inc, o);
                         if (lane >= o) inc += v;
                     }
-                    uint64_t p = lpos + inc - n;
+                    uint32_t p = lpos + inc - n;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         if (mk & (1u << i)) {
-                            if (p < cap) {
+                            if (p < cap32) {
                                 int sv = 0;
                                 out_val[p] = f32_to_f16_sat(xs[i], sv);
                                 n_sat += sv;
-                                out_idx[p] = (uint32_t)((G * 32 + lane) * 4 + i);
+                                out_idx[p] = j * 4 + i;
                             }
                             ++p;
                         }
@@ -451,7 +461,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 const uint32_t sl[4] = {rec.x, rec.y, rec.z, rec.w};
                 const uint32_t kmax = __reduce_max_sync(FULL, cnt);
                 float best = __int_as_float(0xFF800000);           // -inf
-                uint32_t bid = rec.x & LUT_ID_MASK;
+                uint32_t bid = 0;
                 bool tie = false;
 #pragma unroll
                 for (int k = 0; k < LUT_SLOTS; ++k) {
@@ -460,7 +470,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                     const float4 c = s_tab[(id << 3) | lane7];
                     const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z,
                                      __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
-                    tie |= (sc == best) & (id != bid);
+                    tie |= sc == best;               // (the zero dummy never ties a best > 0)
                     if (sc > best) { best = sc; bid = id; }
                 }
                 uint32_t idx = 0;
@@ -475,11 +485,11 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                     ++n_nf;
                 } else {
                     int sat = 0;
-                    rh = f32_to_f16_sat(r, sat);
+                    rh = radius_to_f16(r, sat);
                     n_sat += sat;
                 }
-                radius[G * 32 + lane] = rh;
-                pack_group32(idx, b, lane, pc, words + G * b);
+                radius[j] = rh;
+                pack_group32<BB>(idx, b, lane, pc, words + (size_t)G * b);
             }
         }
         seg = seg_end;
@@ -492,7 +502,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
     }
 }
 
-static size_t enc_smem_bytes(uint32_t S) { return (size_t)24 * S * 8 * sizeof(float4); }
+static size_t enc_smem_bytes(uint32_t S) { return ((size_t)24 * S + 1) * 8 * sizeof(float4); }
 
 }  // namespace hqmq
 
@@ -517,22 +527,23 @@ extern "C" int hqmq_launch_build_search_table(const float *cb, uint32_t S, uint3
 
 namespace hqmq {
 
-template <int DT, int LIST, bool ENC>
-static int launch_lut(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
-                      uint32_t b, const void *table, const float *thr, int gran, uint32_t *words,
-                      uint16_t *radius, const uint32_t *tile_off, uint64_t cap, uint32_t *out_idx,
-                      uint16_t *out_val, hqmq_status *st, int sm_count, cudaStream_t stream) {
+template <int DT, int LIST, bool ENC, int BB>
+static int launch_lut_bb(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
+                         uint32_t b, const void *table, const float *thr, int gran,
+                         uint32_t *words, uint16_t *radius, const uint32_t *tile_off, uint64_t cap,
+                         uint32_t *out_idx, uint16_t *out_val, hqmq_status *st, int sm_count,
+                         cudaStream_t stream) {
     const uint32_t gps = (uint32_t)(((uint64_t)T * D / 4) / 32);
     const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
-    const uint64_t n_tiles = (uint64_t)B * H * tps;
+    const uint32_t n_tiles = (uint32_t)((uint64_t)B * H * tps);
     const size_t smem = ENC ? enc_smem_bytes(S) : 0;
-    auto kern = k_encode_lut<DT, LIST, ENC>;
+    auto kern = k_encode_lut<DT, LIST, ENC, BB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return HQMQ_ERR_CUDA;
     // one CTA per SM, each a contiguous share of the call's tiles
     uint64_t ctas = (uint64_t)sm_count;
-    const uint64_t want = (n_tiles + 7) / 8;
+    const uint64_t want = ((uint64_t)n_tiles + 7) / 8;
     if (ctas > want) ctas = want;
     if (ctas < 1) ctas = 1;
     kern<<<(unsigned)ctas, ENC_THREADS, smem, stream>>>(
@@ -540,6 +551,26 @@ static int launch_lut(int B, int H, int T, int D, const void *x, const float *cb
         reinterpret_cast<const uint4 *>(table), thr, gran, words, radius, tile_off, cap, out_idx,
         out_val, reinterpret_cast<DevStatus *>(st));
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}
+
+// Index widths 8 (S = 8..10) and 10 (S = 22..42) get kernels with constant
+// shifts; others use the runtime width.
+template <int DT, int LIST, bool ENC>
+static int launch_lut(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
+                      uint32_t b, const void *table, const float *thr, int gran, uint32_t *words,
+                      uint16_t *radius, const uint32_t *tile_off, uint64_t cap, uint32_t *out_idx,
+                      uint16_t *out_val, hqmq_status *st, int sm_count, cudaStream_t stream) {
+    if (ENC && b == 8)
+        return launch_lut_bb<DT, LIST, ENC, 8>(B, H, T, D, x, cb, S, b, table, thr, gran, words,
+                                               radius, tile_off, cap, out_idx, out_val, st,
+                                               sm_count, stream);
+    if (ENC && b == 10)
+        return launch_lut_bb<DT, LIST, ENC, 10>(B, H, T, D, x, cb, S, b, table, thr, gran, words,
+                                                radius, tile_off, cap, out_idx, out_val, st,
+                                                sm_count, stream);
+    return launch_lut_bb<DT, LIST, ENC, 0>(B, H, T, D, x, cb, S, b, table, thr, gran, words,
+                                           radius, tile_off, cap, out_idx, out_val, st, sm_count,
+                                           stream);
 }
 
 template <int LIST, bool ENC>
