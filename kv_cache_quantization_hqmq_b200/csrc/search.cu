@@ -269,10 +269,37 @@ __device__ __forceinline__ uint64_t shfl64_down(uint64_t v, int d) {
 }
 
 // Packs the warp's 32 b-bit indices (lane k = chunk k) LSB-first into b words.
-// Each lane first gathers the 64-bit stream window starting at its own chunk
-// (k, k+1, ..., by doubling), then lane w < b takes word w from the window of
-// the chunk where that word starts (k0 = 32 w / b at bit offset o, both
-// computed once per thread).  Needs b in [5, 21].
+//
+// Index width known at compile time (BB = 8 or 10): word w (lane w < BB) is
+// the OR of PACK_TERMS consecutive indices, starting with chunk
+// k0 = floor(32 w / BB) at bit offset o = 32 w - BB k0:
+//   (idx[k0] >> o) | (idx[k0+1] << (BB - o)) | (idx[k0+2] << (2 BB - o)) | ...
+// each fetched with one shuffle.  The checks below show that every shift is
+// below 32 and every source lane exists.
+//
+// Width at run time (BB = 0, b in [5, 21]): each lane first gathers the 64-bit
+// stream window starting at its own chunk (k, k+1, ..., by doubling), then
+// lane w < b takes word w from the window of the chunk where that word starts.
+template <int BB>
+__host__ __device__ constexpr int pack_terms() {
+    int n = 0;
+    for (int w = 0; w < BB; ++w) {
+        const int o = (32 * w) % BB;
+        const int m = (31 + o) / BB + 1;
+        n = m > n ? m : n;
+    }
+    return n;
+}
+
+template <int BB>
+__host__ __device__ constexpr bool pack_plan_ok() {
+    constexpr int nt = pack_terms<BB>();
+    if (BB * (nt - 1) >= 32) return false;                  // a shift of 32 or more
+    for (int w = 0; w < BB; ++w)
+        if ((32 * w) / BB + nt - 1 > 31) return false;      // a source lane past 31
+    return true;
+}
+
 struct PackConst {
     int k0, o;
 };
@@ -285,23 +312,29 @@ __device__ __forceinline__ PackConst pack_const(uint32_t b, int lane) {
     return c;
 }
 
-// BB = the index width when known at compile time (then every shift is a
-// constant), 0 = use b.
 template <int BB>
 __device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b_rt, int lane, PackConst pc,
                                              uint32_t *__restrict__ dst) {
-    const uint32_t b = BB ? (uint32_t)BB : b_rt;
-    uint64_t v = idx;
-    const uint32_t n1 = __shfl_down_sync(FULL, idx, 1);
-    if (lane + 1 < 32) v |= (uint64_t)n1 << b;
-    const uint64_t v2 = shfl64_down(v, 2);
-    if (lane + 2 < 32) v |= v2 << (2 * b);                 // 2b <= 42
-    if (BB == 0 || 4 * BB < 64) {
+    if constexpr (BB != 0) {
+        constexpr int NT = pack_terms<BB>();
+        static_assert(pack_plan_ok<BB>(), "packing plan out of range");
+        uint32_t wv = __shfl_sync(FULL, idx, pc.k0) >> pc.o;
+#pragma unroll
+        for (int m = 1; m < NT; ++m)
+            wv |= __shfl_sync(FULL, idx, (pc.k0 + m) & 31) << (uint32_t)(BB * m - pc.o);
+        if (lane < BB) dst[lane] = wv;
+    } else {
+        const uint32_t b = b_rt;
+        uint64_t v = idx;
+        const uint32_t n1 = __shfl_down_sync(FULL, idx, 1);
+        if (lane + 1 < 32) v |= (uint64_t)n1 << b;
+        const uint64_t v2 = shfl64_down(v, 2);
+        if (lane + 2 < 32) v |= v2 << (2 * b);                 // 2b <= 42
         const uint64_t v4 = shfl64_down(v, 4);
         if (lane + 4 < 32 && 4 * b < 64) v |= v4 << (4 * b);
+        const uint64_t vk = shfl64(v, pc.k0);
+        if (lane < (int)b) dst[lane] = (uint32_t)(vk >> pc.o);
     }
-    const uint64_t vk = shfl64(v, pc.k0);
-    if (lane < (int)b) dst[lane] = (uint32_t)(vk >> pc.o);
 }
 
 // Best candidate among the first `cnt` of a record with exact ties broken by
@@ -432,7 +465,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 if (!ENC) continue;
                 if (med3) {
                     if (gran == HQMQ_GRAN_CHUNK) {
-                        if (r > th) { x0 = x1 = x2 = x3 = 0.0f; r = 0.0f; }
+                        if (r > th) r = 0.0f;        // outlier chunk: no search, radius 0
                     } else {
                         if (fabsf(x0) > th) x0 = 0.0f;
                         if (fabsf(x1) > th) x1 = 0.0f;
