@@ -194,22 +194,27 @@ HQMQ_API int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, 
                 const uint32_t *d_slab_off, uint64_t cap, int gran, int B, int H, int T, int D,
                 void *d_y, int out_dtype, hqmq_status *d_status, void *stream);
 
-/* Exact table-driven search (same results as hqmq_encode).  The best codeword
- * for x is u times the best codeword for x' = conj(u) x, where u = sign(x_a)
- * e_a is the unit of 2T along x's largest coordinate; this holds because the
- * effective codebook {q_p q_s} is closed under left multiplication by 2T, a
- * group (gist.science/nl, Technische Samenvatting, section 1).  x' lies in
- * the cube face x'_0 >= |x'_k|; its gnomonic coordinates t = x'_k / x'_0 are
- * mapped by u = t (A + B t^2) (A = 4/pi in fp32, B = 1 - A) and u is cut into
- * 32^3 cells; per cell the table lists (up to 8) codewords that can be the
- * argmax somewhere in the cell, widened by 1e-5 in t to cover rounding: a
- * codeword is dropped only if it is farther from the cell centre than the best
- * one by more than twice the cell's angular radius, or if another codeword
- * beats it at all 8 corners (the score difference is linear in the gnomonic
- * coordinates).  Cells with more than 8 candidates fall back to the
- * S-codeword loop.  Supports S in [1, 48]. */
+/* Exact table-driven search (same results as hqmq_encode; the argmax of
+ * <x, c> over the 24 S codewords c = q_p q_s, ties to the lowest index:
+ * gist.science/nl, Technische Samenvatting, section 1).  A chunk x lies on one
+ * of 8 cube faces: a = the first coordinate of largest |x_a|, and the sign of
+ * x_a.  Its gnomonic coordinates t (the other three coordinates in index
+ * order, divided by |x_a|, in [-1, 1]) are mapped by u = t (A + B t^2)
+ * (A = 4/pi in fp32, B = 1 - A) and u is cut into 32^3 cells per face.  Per
+ * cell the table lists, in increasing index order, up to 8 codewords that can
+ * be the argmax somewhere in the cell, widened by 1e-5 in t to cover
+ * rounding: a codeword is dropped only if it is farther from the cell centre
+ * than the best one by more than twice the cell's angular radius, or if
+ * another codeword beats it at all 8 corners (the score difference is linear
+ * in x).  Cells with more than 8 candidates fall back to the S-codeword loop.
+ * Supports S in [1, 48].
+ *
+ * Layout per group: uint4 [8 faces: 2 a + (x_a < 0)][32][32][32]; slot k of
+ * a record is the 16-bit half k of the uint4 (low half first); its low 12 bits
+ * hold a codeword id s 24 + p; the top 4 bits of slot 0 hold the count (0 =
+ * overflow); slots past the count hold 24 S. */
 
-/* Bytes of search table per codebook group (524288), or 0 if S is unsupported. */
+/* Bytes of search table per codebook group (4194304), or 0 if S is unsupported. */
 HQMQ_API uint64_t hqmq_search_table_bytes(uint32_t S);
 
 /* Builds the tables of n_groups codebooks: d_codebook[n_groups][S][4] fp32 as

@@ -1,50 +1,54 @@
 // search.cu -- exact local search for the HQMQ encode (table-driven).
 //
 // The encode snaps a chunk x to the codeword c = q_p q_s of the 24 S-word
-// effective codebook with the largest <x, c> (gist.science/nl, Technische
-// Samenvatting, section 1).  The S-codeword loop of encode.cu costs one
-// quaternion product per secondary codeword.  This file replaces it by a
-// lookup of the few codewords that can win in the neighbourhood of x:
+// effective codebook with the largest <x, c>, ties to the lowest index
+// s 24 + p (gist.science/nl, Technische Samenvatting, section 1).  The
+// S-codeword loop of encode.cu costs one quaternion product per secondary
+// codeword.  This file replaces it by a lookup of the few codewords that can
+// win in the neighbourhood of x:
 //
-// 1. Folding.  Let a be the coordinate of largest |x_a| and u = sign(x_a) e_a
-//    one of the 8 units +-1, +-i, +-j, +-k of 2T.  x' = conj(u) x (a signed
-//    permutation of x, exact) has x'_0 = |x_a| >= |x'_k|.  Because the
-//    codebook C = {q_p q_s} is closed under left multiplication by 2T (2T is
-//    a group, same section), <x, c> = <x', conj(u) c> and conj(u) c runs over
-//    C as c does: the best codeword for x is u times the best for x'.
-// 2. Cells.  x' lies in the cube face x'_0 >= |x'_k|; its gnomonic
-//    coordinates t_k = x'_k / x'_0 lie in [-1, 1]^3.  They are mapped by the
-//    monotone u(t) = t (A + B t^2) (A = 4/pi, B = 1 - A, so u(+-1) = +-1), which
-//    roughly equalises the angular size of the cells, and u is cut into G^3
-//    cells.
+// 1. Faces.  Let a be the first coordinate of largest |x_a| and sg = (x_a < 0).
+//    x lies on face f = 2 a + sg of the cube: the directions with
+//    |x_a| >= |x_k| and that sign of x_a.  Its gnomonic coordinates are the
+//    other three coordinates, in index order, divided by |x_a|:
+//    t in [-1, 1]^3.
+// 2. Cells.  t is mapped by the monotone u(t) = t (A + B t^2) (A = 4/pi,
+//    B = 1 - A, so u(+-1) = +-1), which roughly equalises the angular size of
+//    the cells, and u is cut into G^3 cells per face.
 // 3. Candidates.  For each cell (grown by DELTA on every side to absorb fp32
 //    rounding of t), a codeword c is kept unless (i) its angle from the cell
 //    centre exceeds the best angle there by more than twice the cell's angular
 //    radius, or (ii) another codeword c* beats it at all 8 corners of the cell:
-//    <(1, t), c* - c> is linear in t, so c* beats c on the whole cell iff it
-//    does at the corners.  Both tests only drop codewords that cannot be the
-//    argmax anywhere in the cell, so the list is a superset of the possible
-//    winners.  Up to SLOTS survivors are stored; a cell with more is marked
-//    OVERFLOW and its chunks use the S-codeword loop.
-// 4. Encode.  Score the cell's candidates with fp32 <x', c'>, keep the best
-//    (equal scores: the lowest index after mapping back), map back
-//    p = index(u q_p').  The tables stay in global memory (L2-resident: 512 KB
-//    per head); candidate codewords come from a shared-memory copy of the 24 S
-//    codewords replicated 8 times so that the 8 lanes of each quarter-warp
-//    read 8 different bank groups (no conflicts).
+//    <x, c* - c> is linear in x, and the cell's directions are positive
+//    multiples of the points of a box with those corners, so c* beats c on the
+//    whole cell iff it does at the corners.  Both tests only drop codewords
+//    that cannot be the argmax anywhere in the cell, so the list is a superset
+//    of the possible winners.  Up to SLOTS survivors are stored in increasing
+//    index order; a cell with more is marked OVERFLOW and its chunks use the
+//    S-codeword loop.
+// 4. Encode.  Score the cell's candidates in slot order with fp32 <x, c> and
+//    keep a candidate only if it scores strictly higher: among equal scores
+//    the lowest index wins, as the rule asks.  The tables stay in global memory
+//    (L2-resident: 4 MB per head, 8 faces x 32^3 cells x 16 B); candidate
+//    codewords come from a shared-memory copy of the 24 S codewords replicated
+//    8 times so that the 8 lanes of each quarter-warp read 8 different bank
+//    groups (no conflicts).
 #include "med3_window.cuh"
 
 namespace hqmq {
 
 constexpr int LUT_G = 32;
-constexpr int LUT_CELLS = LUT_G * LUT_G * LUT_G;   // 32768 cells, 512 KB per group
+constexpr int LUT_CELLS = LUT_G * LUT_G * LUT_G;   // 32768 cells per face
+constexpr int LUT_FACES = 8;
+constexpr int LUT_ENTRIES = LUT_FACES * LUT_CELLS;  // 4 MB per group
 constexpr float MAP_A = 1.27323954f;               // 4 / pi (fp32)
 constexpr float MAP_B = 1.0f - MAP_A;              // exact (Sterbenz)
 constexpr int LUT_SLOTS = 8;
 // Record: 8 slots of 16 bits; slot k holds candidate id k in its low 12 bits
-// (24 S < 4096); the top 4 bits of slot 0 hold the count (1..8), 0 marks an
-// overflowing cell; slots past the count hold the dummy id 24 S, whose
-// shared-memory codeword is zero (score 0, below every real best score).
+// (24 S < 4096), in increasing order; the top 4 bits of slot 0 hold the count
+// (1..8), 0 marks an overflowing cell; slots past the count hold the dummy id
+// 24 S, whose shared-memory codeword is zero (score 0, below every real best
+// score, and last in slot order).
 constexpr uint32_t LUT_ID_MASK = 0x0FFFu;
 constexpr uint32_t LUT_MAX_S = 48;                // 24 S codeword ids fit in 16 bits;
                                                   // shared memory fits 8 copies (144 KB)
@@ -80,24 +84,33 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
         s_cw[i] = make_double4(c.x, c.y, c.z, c.w);
     }
     __syncthreads();
-    const uint32_t cell = blockIdx.x * BUILD_THREADS + threadIdx.x;
-    if (cell >= (uint32_t)LUT_CELLS) return;
-    const int ic[3] = {(int)(cell / (LUT_G * LUT_G)), (int)((cell / LUT_G) % LUT_G),
-                       (int)(cell % LUT_G)};
+    const uint32_t entry = blockIdx.x * BUILD_THREADS + threadIdx.x;   // face * cells + cell
+    if (entry >= (uint32_t)LUT_ENTRIES) return;
+    const int face = (int)(entry / LUT_CELLS), cell = (int)(entry % LUT_CELLS);
+    const int ax = face >> 1;                          // coordinate of largest |x|
+    const double sgn = (face & 1) ? -1.0 : 1.0;        // its sign
+    int other[3];                                      // the other coordinates, in order
+    for (int k = 0, n = 0; k < 4; ++k)
+        if (k != ax) other[n++] = k;
+    const int ic[3] = {cell / (LUT_G * LUT_G), (cell / LUT_G) % LUT_G, cell % LUT_G};
     double lo[3], hi[3], mid[3];
     for (int k = 0; k < 3; ++k) {
         lo[k] = t_of_u(-1.0 + 2.0 * ic[k] / LUT_G) - LUT_DELTA;
         hi[k] = t_of_u(-1.0 + 2.0 * (ic[k] + 1) / LUT_G) + LUT_DELTA;
         mid[k] = 0.5 * (lo[k] + hi[k]);
     }
-    // corners (unnormalised (1, t)) and the centre direction
+    // corners (x_a = +-1, the others = t) and the centre direction
     double cor[8][4];
     for (int q = 0; q < 8; ++q) {
-        cor[q][0] = 1.0;
-        for (int k = 0; k < 3; ++k) cor[q][k + 1] = ((q >> k) & 1) ? hi[k] : lo[k];
+        cor[q][ax] = sgn;
+        for (int k = 0; k < 3; ++k) cor[q][other[k]] = ((q >> k) & 1) ? hi[k] : lo[k];
     }
-    double cn = sqrt(1.0 + mid[0] * mid[0] + mid[1] * mid[1] + mid[2] * mid[2]);
-    const double uc[4] = {1.0 / cn, mid[0] / cn, mid[1] / cn, mid[2] / cn};
+    double uc[4];
+    {
+        const double cn = sqrt(1.0 + mid[0] * mid[0] + mid[1] * mid[1] + mid[2] * mid[2]);
+        uc[ax] = sgn / cn;
+        for (int k = 0; k < 3; ++k) uc[other[k]] = mid[k] / cn;
+    }
     double cos_rho = 1.0;                              // angular radius of the cell
     for (int q = 0; q < 8; ++q) {
         double n = sqrt(cor[q][0] * cor[q][0] + cor[q][1] * cor[q][1] + cor[q][2] * cor[q][2] +
@@ -116,7 +129,6 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
     const double cos_lim = lim >= 3.141592653589793 ? -2.0 : cos(lim) - 1e-12;
     // (i) angle prefilter
     uint32_t cand[BUILD_MAXC];
-    double cdot[BUILD_MAXC];
     int nc = 0;
     bool overflow = false;
     for (uint32_t i = 0; i < n_words; ++i) {
@@ -124,13 +136,10 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
         double d = uc[0] * c.x + uc[1] * c.y + uc[2] * c.z + uc[3] * c.w;
         if (d >= cos_lim) {
             if (nc == BUILD_MAXC) { overflow = true; break; }
-            cand[nc] = i;
-            cdot[nc] = d;
-            ++nc;
+            cand[nc++] = i;
         }
     }
     uint32_t keep[LUT_SLOTS];
-    double kdot[LUT_SLOTS];
     int nk = 0;
     if (!overflow) {
         // (ii) dominance on the corners
@@ -151,15 +160,7 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
             }
             if (!dominated) {
                 if (nk == LUT_SLOTS) { overflow = true; break; }
-                // insertion by descending centre score: the likely winner first
-                int pos = nk++;
-                while (pos > 0 && kdot[pos - 1] < cdot[j]) {
-                    keep[pos] = keep[pos - 1];
-                    kdot[pos] = kdot[pos - 1];
-                    --pos;
-                }
-                keep[pos] = cand[j];
-                kdot[pos] = cdot[j];
+                keep[nk++] = cand[j];                  // (cand is in increasing id order)
             }
         }
     }
@@ -167,7 +168,7 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
     if (overflow) nk = 0;
     for (int q = 0; q < LUT_SLOTS; ++q) slot[q] = nk > 0 ? (q < nk ? keep[q] : n_words) : 0u;
     slot[0] |= (uint32_t)nk << 12;
-    tables[(size_t)g * LUT_CELLS + cell] =
+    tables[(size_t)g * LUT_ENTRIES + entry] =
         make_uint4(slot[0] | (slot[1] << 16), slot[2] | (slot[3] << 16),
                    slot[4] | (slot[5] << 16), slot[6] | (slot[7] << 16));
 }
@@ -175,40 +176,6 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
 // ---------------------------------------------------------------------------
 // encode with the table
 // ---------------------------------------------------------------------------
-
-// Index (0..23) of the 2T element a*b for a, b given by index (exact: the
-// entries are 0, +-1, +-1/2 and every product of two of them is exact).
-__device__ int mul_2t(int pa, int pb) {
-    float a0, a1, a2, a3, b0, b1, b2, b3;
-    element_2t(pa, a0, a1, a2, a3);
-    element_2t(pb, b0, b1, b2, b3);
-    const float w = a0 * b0 - a1 * b1 - a2 * b2 - a3 * b3;
-    const float x = a0 * b1 + a1 * b0 + a2 * b3 - a3 * b2;
-    const float y = a0 * b2 - a1 * b3 + a2 * b0 + a3 * b1;
-    const float z = a0 * b3 + a1 * b2 - a2 * b1 + a3 * b0;
-    for (int p = 0; p < 24; ++p) {
-        float c0, c1, c2, c3;
-        element_2t(p, c0, c1, c2, c3);
-        if (c0 == w && c1 == x && c2 == y && c3 == z) return p;
-    }
-    return 0;
-}
-
-// Face of x: the unit u = sign(x_a) e_a (2T index 2a + sign) and x' = conj(u) x.
-__device__ __forceinline__ int fold(float x0, float x1, float x2, float x3, float &y0, float &y1,
-                                    float &y2, float &y3) {
-    const float a0 = fabsf(x0), a1 = fabsf(x1), a2 = fabsf(x2), a3 = fabsf(x3);
-    const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-    const int a = (a0 == m) ? 0 : (a1 == m) ? 1 : (a2 == m) ? 2 : 3;
-    // conj(e_a) x for a = 0..3: x, (x1,-x0,x3,-x2), (x2,-x3,-x0,x1), (x3,x2,-x1,-x0)
-    if (a == 0) { y0 = x0; y1 = x1; y2 = x2; y3 = x3; }
-    else if (a == 1) { y0 = x1; y1 = -x0; y2 = x3; y3 = -x2; }
-    else if (a == 2) { y0 = x2; y1 = -x3; y2 = -x0; y3 = x1; }
-    else { y0 = x3; y1 = x2; y2 = -x1; y3 = -x0; }
-    const bool neg = y0 < 0.0f;
-    if (neg) { y0 = -y0; y1 = -y1; y2 = -y2; y3 = -y3; }
-    return 2 * a + (neg ? 1 : 0);
-}
 
 __device__ __forceinline__ int cell_coord(float t) {
     const float u = t * __fmaf_rn(MAP_B, t * t, MAP_A);
@@ -337,25 +304,6 @@ __device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b_rt, int la
     }
 }
 
-// Best candidate among the first `cnt` of a record with exact ties broken by
-// the lowest original index (the rare path, taken only when two candidates
-// score exactly the same).
-__device__ __noinline__ uint32_t best_with_ties(uint4 rec, uint32_t cnt, float y0, float y1,
-                                                float y2, float y3, const float4 *s_tab,
-                                                uint32_t lane7, const uint8_t *mul_row) {
-    float best = __int_as_float(0xFF800000);
-    uint32_t bmap = 0xFFFFFFFFu;
-    for (uint32_t k = 0; k < cnt; ++k) {
-        const uint32_t word = k < 2 ? rec.x : k < 4 ? rec.y : k < 6 ? rec.z : rec.w;
-        const uint32_t id = (word >> ((k & 1) * 16)) & LUT_ID_MASK;
-        const float4 c = s_tab[(id << 3) | lane7];
-        const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z, __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
-        const uint32_t m = (id / 24u) * 24u + mul_row[id % 24u];
-        if (sc > best || (sc == best && m < bmap)) { best = sc; bmap = m; }
-    }
-    return bmap;
-}
-
 // LIST: 0 = no list; HQMQ_GRAN_CHUNK + 1 / HQMQ_GRAN_ELEMENT + 1 = write the
 // ordered outlier list of that granularity (thr exact, tile_off from the
 // Med3x window pipeline).  ENC: encode (else write the list only).
@@ -370,7 +318,6 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
              const uint32_t *__restrict__ tile_off, uint64_t cap, uint32_t *__restrict__ out_idx,
              uint16_t *__restrict__ out_val, DevStatus *st) {
     extern __shared__ float4 s_tab[];                    // [24 S + 1][8]: codewords, then zero
-    __shared__ uint8_t s_mul[8][24];                     // u * q_p' for the 8 units
     const uint32_t b = BB ? (uint32_t)BB : b_rt;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = (1u << lane) - 1u;
@@ -378,9 +325,6 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
     const uint32_t n_words = 24u * S;
     const uint32_t lane7 = (uint32_t)(lane & 7);
     const PackConst pc = pack_const(b, lane);
-    if (ENC)
-        for (int i = threadIdx.x; i < 8 * 24; i += ENC_THREADS)
-            s_mul[i / 24][i % 24] = (uint8_t)mul_2t(i / 24, i % 24);
 
     // (chunk and list indices fit 32 bits: a call has fewer than 2^32 elements)
     const uint32_t t_begin = (uint32_t)((uint64_t)n_tiles * blockIdx.x / gridDim.x);
@@ -393,7 +337,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
         const uint32_t seg_end = min(t_end, (slab + 1) * tiles_per_slab);
         const int h = (int)(slab % (uint32_t)H);
         const float4 *cb = cb_all + (size_t)h * S;
-        const uint4 *tb = tables + (size_t)h * LUT_CELLS;
+        const uint4 *tb = tables + (size_t)h * LUT_ENTRIES;
         if (ENC && h != cur_head) {                      // (block-uniform)
             __syncthreads();
             for (uint32_t i = threadIdx.x; i < (n_words + 1) * 8; i += ENC_THREADS) {
@@ -478,39 +422,44 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 const bool search = finite && r > 0.0f;
                 // every lane runs the candidate loop up to the warp's longest
                 // list (lanes without a search score candidate 0 of cell 0)
-                float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-                int pu = 0;
                 uint4 rec = make_uint4(1u << 12, 0u, 0u, 0u);
                 if (search) {
-                    pu = fold(x0, x1, x2, x3, y0, y1, y2, y3);
+                    const float a0 = fabsf(x0), a1 = fabsf(x1), a2 = fabsf(x2), a3 = fabsf(x3);
+                    const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+                    const bool e0 = a0 == m, e01 = e0 || a1 == m, e012 = e01 || a2 == m;
+                    // face: first coordinate a of largest |x_a| and the sign of
+                    // x_a; cell: the other three coordinates in index order / m
+                    const int a = e0 ? 0 : e01 ? 1 : e012 ? 2 : 3;
+                    const float xa = e0 ? x0 : e01 ? x1 : e012 ? x2 : x3;
+                    const float c1 = e0 ? x1 : x0;
+                    const float c2 = e01 ? x2 : x1;
+                    const float c3 = e012 ? x3 : x2;
                     float inv;
-                    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(y0));   // cells are widened
-                    const int cell = (cell_coord(y1 * inv) * LUT_G + cell_coord(y2 * inv)) * LUT_G +
-                                     cell_coord(y3 * inv);
-                    rec = __ldg(tb + cell);
+                    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(m));   // cells are widened
+                    const int cell = (cell_coord(c1 * inv) * LUT_G + cell_coord(c2 * inv)) * LUT_G +
+                                     cell_coord(c3 * inv);
+                    const int face = 2 * a + (xa < 0.0f ? 1 : 0);
+                    rec = __ldg(tb + face * LUT_CELLS + cell);
                 }
                 const uint32_t cnt = (rec.x >> 12) & 0xFu;
                 const bool fallback = cnt == 0;                    // overflowing cell
                 const uint32_t sl[4] = {rec.x, rec.y, rec.z, rec.w};
                 const uint32_t kmax = __reduce_max_sync(FULL, cnt);
+                // slots hold increasing ids: a strictly higher score replaces
+                // the best, so equal scores keep the lowest index
                 float best = __int_as_float(0xFF800000);           // -inf
                 uint32_t bid = 0;
-                bool tie = false;
 #pragma unroll
                 for (int k = 0; k < LUT_SLOTS; ++k) {
                     if ((uint32_t)k >= kmax) break;                // warp-uniform
                     const uint32_t id = (sl[k >> 1] >> ((k & 1) * 16)) & LUT_ID_MASK;
                     const float4 c = s_tab[(id << 3) | lane7];
-                    const float sc = __fmaf_rn(y3, c.w, __fmaf_rn(y2, c.z,
-                                     __fmaf_rn(y1, c.y, __fmul_rn(y0, c.x))));
-                    tie |= sc == best;               // (the zero dummy never ties a best > 0)
+                    const float sc = __fmaf_rn(x3, c.w, __fmaf_rn(x2, c.z,
+                                     __fmaf_rn(x1, c.y, __fmul_rn(x0, c.x))));
                     if (sc > best) { best = sc; bid = id; }
                 }
                 uint32_t idx = 0;
-                if (search && !fallback) idx = (bid / 24u) * 24u + s_mul[pu][bid % 24u];
-                if (__any_sync(FULL, search && tie && !fallback))  // exact ties: rare
-                    if (search && tie && !fallback)
-                        idx = best_with_ties(rec, cnt, y0, y1, y2, y3, s_tab, lane7, s_mul[pu]);
+                if (search && !fallback) idx = bid;
                 if (search && fallback) idx = sloop_index(x0, x1, x2, x3, cb, S);
                 uint16_t rh;
                 if (!finite) {
@@ -541,7 +490,7 @@ static size_t enc_smem_bytes(uint32_t S) { return ((size_t)24 * S + 1) * 8 * siz
 
 extern "C" uint64_t hqmq_lut_bytes_per_group(uint32_t S) {
     if (S < 1 || S > hqmq::LUT_MAX_S) return 0;
-    return (uint64_t)hqmq::LUT_CELLS * sizeof(uint4);
+    return (uint64_t)hqmq::LUT_ENTRIES * sizeof(uint4);
 }
 
 extern "C" int hqmq_launch_build_search_table(const float *cb, uint32_t S, uint32_t n_groups,
@@ -552,7 +501,7 @@ extern "C" int hqmq_launch_build_search_table(const float *cb, uint32_t S, uint3
         cudaFuncSetAttribute(k_build_search_table, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return HQMQ_ERR_CUDA;
-    dim3 grid(LUT_CELLS / BUILD_THREADS, n_groups);
+    dim3 grid(LUT_ENTRIES / BUILD_THREADS, n_groups);
     k_build_search_table<<<grid, BUILD_THREADS, smem, stream>>>(
         reinterpret_cast<const float4 *>(cb), S, reinterpret_cast<uint4 *>(table));
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;

@@ -165,7 +165,7 @@ def test_search_table_codebook_sizes(oracle, S):
 
 def test_search_table_rejects_large_S():
     assert hqmq.hqmq_search_table_bytes(49) == 0
-    assert hqmq.hqmq_search_table_bytes(48) == 32 ** 3 * 16
+    assert hqmq.hqmq_search_table_bytes(48) == 8 * 32 ** 3 * 16
 
 
 @pytest.mark.parametrize("encoder", ENCODERS)
