@@ -39,7 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 ALU_LANES = 148 * 128          # FP32 lanes of a B200 (148 SMs x 128)
 # kernels per call: fused Med3x+encode = sample, window, full pass, final
 # select, fallback check, uncertain fix-up, tile scan, list+encode pass
-KERNELS_MED3_ENCODE = 8
+KERNELS_MED3_ENCODE = 4          # k_sample_window, k_pass_b, k_finalize, k_encode_lut
 OUTLIER_CAP_FRAC = 0.15        # list capacity: 15% of the chunks of a call
 
 
@@ -200,7 +200,7 @@ class Cache:
 
     def kernels_per_step(self):
         if self.w.med3:
-            enc = KERNELS_MED3_ENCODE + (0 if self.table is not None else 2)
+            enc = KERNELS_MED3_ENCODE + (0 if self.table is not None else 1)
             dec = 2                        # main pass + outlier pass
         else:
             enc, dec = 1, 1

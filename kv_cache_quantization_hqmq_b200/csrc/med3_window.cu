@@ -6,27 +6,29 @@
 // iff r > fl32(C r_med).  The results are exactly those of the three-pass radix
 // select of med3.cu; only the data flow differs:
 //
-//  A  k_sample_hist    reads a 1/32 sample (4 consecutive chunks of every 128,
+//  A+W k_sample_window reads a 1/32 sample (4 consecutive chunks of every 128,
 //                      the quad's slot rotating through all 32 slots) into a
-//                      per-head histogram of the top 16 key bits.
-//  W  k_window_select  picks per head a key window [lo, hi) that holds the
-//                      sample ranks within +-8 standard deviations of the median
-//                      rank; the exact threshold then lies in [t_lo, t_hi].
-//  B  k_pass_b         one full read: per head the count of keys below the
+//                      per-head histogram of the top 16 key bits; the last
+//                      CTA of each head then picks a key window [lo, hi) that
+//                      holds the sample ranks within +-8 standard deviations of
+//                      the median rank; the exact threshold then lies in
+//                      [t_lo, t_hi].
+//  B   k_pass_b        one full read: per head the count of keys below the
 //                      window and the keys inside it (list + fine histogram);
 //                      per 1024-chunk tile the count of certain outliers
 //                      (r > t_hi) and a list of uncertain ones (t_lo < r <= t_hi).
-//  F  k_med_final      per head: the exact median from the window keys.
-//  X  k_fallback_exact per head whose window missed the median (or whose buffers
-//                      overflowed): exact three-pass select over x and exact
-//                      tile counts.  Never taken on the bench workloads; it keeps
-//                      the result exact for any input.
-//  U  k_amb_fixup      adds the uncertain keys that exceed the exact threshold.
-//  S  k_tile_scan      tile offsets, per-slab offsets, total, overflow status.
-//  C  (search.cu)      the second read writes the ordered list (and encodes).
+//  F   k_finalize      per head: the exact median from the window keys, or,
+//                      if the window missed the median (or a buffer
+//                      overflowed), the exact three-pass select over x and
+//                      exact tile counts (never taken on the bench workloads;
+//                      it keeps the result exact for any input); then the
+//                      uncertain keys above the exact threshold; the last CTA
+//                      scans the tile counts into tile and slab offsets.
+//  C   (search.cu)     the second read writes the ordered list (and encodes).
 //
-// No kernel waits on another CTA; every step is a separate launch on the
-// caller's stream.
+// A memset clears the histograms and counters first.  No CTA waits for
+// another: where a step needs the results of all CTAs of the previous one,
+// the last CTA to finish (an atomic ticket after a fence) does it.
 #include "med3_window.cuh"
 
 namespace hqmq {
@@ -58,21 +60,155 @@ __device__ __forceinline__ void chunk_keys(float x0, float x1, float x2, float x
 }
 
 // ---------------------------------------------------------------------------
-// A: sample histogram
+// Histogram search helpers
+// ---------------------------------------------------------------------------
+// Histogram reads: GLOBAL = bins written by other CTAs (read through L2).
+template <bool GLOBAL>
+__device__ __forceinline__ uint32_t hist_ld(const uint32_t *p) {
+    if constexpr (GLOBAL) return __ldcg(p);
+    else return *p;
+}
+
+// Block-wide (1024 threads = 32 warps) search of a histogram of NB bins, warp
+// w owning the contiguous bins [w NB/32, (w+1) NB/32), read coalesced:
+// rank_bin_totals() stores the warp totals and the totals of every block of
+// 32 bins; rank_bin_find() then locates the warp, the block (from the block
+// totals) and the bin (one 32-bin read), and returns in s_out[which] the bin
+// whose cumulative count first exceeds `rank` and in s_out[which + 2] the
+// rank inside that bin.
+template <int NB, bool GLOBAL>
+__device__ void rank_bin_totals(const uint32_t *hist, uint32_t *s_wtot, uint32_t *s_blk) {
+    constexpr int PER = NB / 32;
+    constexpr int UNR = PER / 32 < 8 ? PER / 32 : 8;       // loads in flight per lane
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint32_t acc = 0;
+    for (int i = 0; i < PER; i += 32 * UNR) {
+        uint32_t v[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) v[u] = hist_ld<GLOBAL>(hist + w * PER + i + 32 * u + lane);
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const uint32_t bt = __reduce_add_sync(FULL, v[u]);
+            if (lane == 0) s_blk[(w * PER + i) / 32 + u] = bt;
+            acc += bt;
+        }
+    }
+    if (lane == 0) s_wtot[w] = acc;
+    __syncthreads();
+}
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(FULL, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+template <int NB, bool GLOBAL>
+__device__ void rank_bin_find(const uint32_t *hist, const uint32_t *s_wtot,
+                              const uint32_t *s_blk, uint64_t rank, uint32_t *s_out, int which) {
+    constexpr int PER = NB / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint64_t cum = 0;
+    int ww = 31;
+    for (int k = 0; k < 32; ++k) {
+        const uint32_t t = s_wtot[k];
+        if (rank < cum + t) { ww = k; break; }
+        cum += t;
+    }
+    if (w == ww) {
+        uint64_t c = cum;
+        int blk = -1;
+        for (int i = 0; i < PER / 32; i += 32) {             // block totals of this warp
+            const uint32_t v = (i + lane < PER / 32) ? s_blk[ww * (PER / 32) + i + lane] : 0u;
+            const uint32_t inc = warp_incl_scan(v, lane);
+            const uint32_t tot = __shfl_sync(FULL, inc, 31);
+            if (rank < c + tot) {
+                const uint32_t bal = __ballot_sync(FULL, rank < c + inc);
+                const int src = __ffs(bal) - 1;
+                blk = i + src;
+                c += __shfl_sync(FULL, inc - v, src);
+                break;
+            }
+            c += tot;
+        }
+        if (blk >= 0) {                   // (rank below the total, as the callers ensure)
+            const uint32_t v = hist_ld<GLOBAL>(hist + ww * PER + blk * 32 + lane);
+            const uint32_t inc = warp_incl_scan(v, lane);
+            const bool mine = rank >= c + inc - v && rank < c + inc;
+            const uint32_t bal = __ballot_sync(FULL, mine);
+            if (lane == __ffs(bal) - 1) {
+                s_out[which] = (uint32_t)(ww * PER + blk * 32 + lane);
+                s_out[which + 2] = (uint32_t)(rank - (c + inc - v));
+            }
+        } else if (lane == 0) {
+            s_out[which] = NB - 1;
+            s_out[which + 2] = 0;
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// A + W: sample histogram; the last sample CTA of each head picks its window
 // ---------------------------------------------------------------------------
 constexpr int SAMPLE_THREADS = 1024;
 
+// Window of head h from its complete sample histogram (one CTA).
+__device__ void select_window(int h, uint64_t n_per_head, float C, const uint32_t *hist,
+                              WinState *win, unsigned long long *below,
+                              unsigned long long *cand_n, uint32_t *s_wtot, uint32_t *s_blk,
+                              uint32_t *s_out) {
+    rank_bin_totals<KEY_BINS, true>(hist, s_wtot, s_blk);
+    uint64_t tot = 0;
+    for (int k = 0; k < 32; ++k) tot += s_wtot[k];
+    const double ns = (double)tot;
+    const double q = ((double)(n_per_head / 2 - 1) + 0.5) / (double)n_per_head;
+    const double half = WINDOW_SIGMAS * 0.5 * sqrt(ns) + 4.0;
+    double rlo = floor(q * ns - half), rhi = ceil(q * ns + half);
+    if (rlo < 0) rlo = 0;
+    if (rhi > ns - 1) rhi = ns - 1;
+    rank_bin_find<KEY_BINS, true>(hist, s_wtot, s_blk, (uint64_t)rlo, s_out, 0);
+    rank_bin_find<KEY_BINS, true>(hist, s_wtot, s_blk, (uint64_t)rhi, s_out, 1);
+    if (threadIdx.x == 0) {
+        WinState w;
+        const uint64_t lo = (uint64_t)s_out[0] << 15;
+        uint64_t hi = ((uint64_t)s_out[1] + 1) << 15;
+        if (hi > 0x80000000ull) hi = 0x80000000ull;
+        const uint64_t span = hi - lo;
+        uint32_t sh = 0;
+        while (((span - 1) >> sh) >= (uint64_t)KEY_BINS) ++sh;
+        w.lo_key = (uint32_t)lo;
+        w.hi_key = (uint32_t)(hi - 1) + 1u;          // (hi <= 2^31)
+        w.shift = sh;
+        w.miss = 0;
+        w.t_lo = thr_of_key(C, (uint32_t)lo);
+        w.t_hi = thr_of_key(C, (uint32_t)(hi - 1));
+        w.pad[0] = w.pad[1] = 0;
+        win[h] = w;
+        below[h] = 0;
+        cand_n[h] = 0;
+    }
+}
+
 template <int DT, int GRAN>
 __global__ void __launch_bounds__(SAMPLE_THREADS)
-k_sample_hist(const void *__restrict__ x, int H, uint32_t cps, uint32_t *__restrict__ hist) {
+k_sample_window(const void *__restrict__ x, int H, uint32_t cps, uint32_t ctas_per_head,
+                uint64_t n_per_head, float C, uint32_t *__restrict__ hist,
+                uint32_t *__restrict__ sample_done, WinState *__restrict__ win,
+                unsigned long long *__restrict__ below, unsigned long long *__restrict__ cand_n) {
     // per-CTA histogram in shared memory: 65536 16-bit counters packed in
     // pairs (a CTA sees far fewer than 65536 samples), then one global add
     // per non-empty bin
     extern __shared__ uint32_t s_pair[];                       // [KEY_BINS / 2]
+    __shared__ uint32_t s_wtot[32], s_blk[KEY_BINS / 32], s_out[4], s_last;
     for (int i = threadIdx.x; i < KEY_BINS / 2; i += blockDim.x) s_pair[i] = 0;
     __syncthreads();
     const int slab = blockIdx.y;
-    uint32_t *hh = hist + (size_t)(slab % H) * KEY_BINS;
+    const int h = slab % H;
+    uint32_t *hh = hist + (size_t)h * KEY_BINS;
     const uint64_t base = (uint64_t)slab * cps;
     const uint32_t n_quads = (cps + SAMPLE_PERIOD - 1) / SAMPLE_PERIOD;
     for (uint32_t q = blockIdx.x * blockDim.x + threadIdx.x; q < n_quads;
@@ -104,127 +240,15 @@ k_sample_hist(const void *__restrict__ x, int H, uint32_t cps, uint32_t *__restr
         if (v & 0xFFFFu) atomicAdd(hh + 2 * i, v & 0xFFFFu);
         if (v >> 16) atomicAdd(hh + 2 * i + 1, v >> 16);
     }
-}
-
-// Block-wide (1024 threads = 32 warps) search of a histogram of NB bins, warp
-// w owning the contiguous bins [w NB/32, (w+1) NB/32), read coalesced:
-// rank_bin_totals() stores the warp totals and the totals of every block of
-// 32 bins; rank_bin_find() then locates the warp, the block (from the block
-// totals) and the bin (one 32-bin read), and returns in s_out[which] the bin
-// whose cumulative count first exceeds `rank` and in s_out[which + 2] the
-// rank inside that bin.
-template <int NB>
-__device__ void rank_bin_totals(const uint32_t *hist, uint32_t *s_wtot, uint32_t *s_blk) {
-    constexpr int PER = NB / 32;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    uint32_t acc = 0;
-    for (int i = 0; i < PER; i += 32) {
-        const uint32_t bt = __reduce_add_sync(FULL, hist[w * PER + i + lane]);
-        if (lane == 0) s_blk[(w * PER + i) / 32] = bt;
-        acc += bt;
-    }
-    if (lane == 0) s_wtot[w] = acc;
+    // the last of the head's CTAs (no CTA waits for another) reads the
+    // complete histogram: every CTA's adds are ordered before its ticket
+    __threadfence();
     __syncthreads();
-}
-
-__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t u = __shfl_up_sync(FULL, v, o);
-        if (lane >= o) v += u;
-    }
-    return v;
-}
-
-template <int NB>
-__device__ void rank_bin_find(const uint32_t *hist, const uint32_t *s_wtot,
-                              const uint32_t *s_blk, uint64_t rank, uint32_t *s_out, int which) {
-    constexpr int PER = NB / 32;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    uint64_t cum = 0;
-    int ww = 31;
-    for (int k = 0; k < 32; ++k) {
-        const uint32_t t = s_wtot[k];
-        if (rank < cum + t) { ww = k; break; }
-        cum += t;
-    }
-    if (w == ww) {
-        uint64_t c = cum;
-        int blk = -1;
-        for (int i = 0; i < PER / 32; i += 32) {             // block totals of this warp
-            const uint32_t v = (i + lane < PER / 32) ? s_blk[ww * (PER / 32) + i + lane] : 0u;
-            const uint32_t inc = warp_incl_scan(v, lane);
-            const uint32_t tot = __shfl_sync(FULL, inc, 31);
-            if (rank < c + tot) {
-                const uint32_t bal = __ballot_sync(FULL, rank < c + inc);
-                const int src = __ffs(bal) - 1;
-                blk = i + src;
-                c += __shfl_sync(FULL, inc - v, src);
-                break;
-            }
-            c += tot;
-        }
-        if (blk >= 0) {                   // (rank below the total, as the callers ensure)
-            const uint32_t v = hist[ww * PER + blk * 32 + lane];
-            const uint32_t inc = warp_incl_scan(v, lane);
-            const bool mine = rank >= c + inc - v && rank < c + inc;
-            const uint32_t bal = __ballot_sync(FULL, mine);
-            if (lane == __ffs(bal) - 1) {
-                s_out[which] = (uint32_t)(ww * PER + blk * 32 + lane);
-                s_out[which + 2] = (uint32_t)(rank - (c + inc - v));
-            }
-        } else if (lane == 0) {
-            s_out[which] = NB - 1;
-            s_out[which + 2] = 0;
-        }
-    }
+    if (threadIdx.x == 0) s_last = atomicAdd(sample_done + h, 1u) == ctas_per_head - 1 ? 1u : 0u;
     __syncthreads();
-}
-
-// ---------------------------------------------------------------------------
-// W: window per head
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(WIN_THREADS)
-k_window_select(uint64_t n_per_head, float C, const uint32_t *__restrict__ sample_hist,
-                uint32_t *__restrict__ fine_hist, WinState *__restrict__ win,
-                unsigned long long *__restrict__ below, unsigned long long *__restrict__ cand_n) {
-    __shared__ uint32_t s_wtot[32];
-    __shared__ uint32_t s_blk[KEY_BINS / 32];
-    __shared__ uint32_t s_out[4];
-    const int h = blockIdx.x;
-    const uint32_t *hist = sample_hist + (size_t)h * KEY_BINS;
-    uint32_t *fh = fine_hist + (size_t)h * KEY_BINS;
-    for (int i = threadIdx.x; i < KEY_BINS; i += WIN_THREADS) fh[i] = 0;
-    rank_bin_totals<KEY_BINS>(hist, s_wtot, s_blk);
-    uint64_t tot = 0;
-    for (int k = 0; k < 32; ++k) tot += s_wtot[k];
-    const double ns = (double)tot;
-    const double q = ((double)(n_per_head / 2 - 1) + 0.5) / (double)n_per_head;
-    const double half = WINDOW_SIGMAS * 0.5 * sqrt(ns) + 4.0;
-    double rlo = floor(q * ns - half), rhi = ceil(q * ns + half);
-    if (rlo < 0) rlo = 0;
-    if (rhi > ns - 1) rhi = ns - 1;
-    rank_bin_find<KEY_BINS>(hist, s_wtot, s_blk, (uint64_t)rlo, s_out, 0);
-    rank_bin_find<KEY_BINS>(hist, s_wtot, s_blk, (uint64_t)rhi, s_out, 1);
-    if (threadIdx.x == 0) {
-        WinState w;
-        const uint64_t lo = (uint64_t)s_out[0] << 15;
-        uint64_t hi = ((uint64_t)s_out[1] + 1) << 15;
-        if (hi > 0x80000000ull) hi = 0x80000000ull;
-        const uint64_t span = hi - lo;
-        uint32_t sh = 0;
-        while (((span - 1) >> sh) >= (uint64_t)KEY_BINS) ++sh;
-        w.lo_key = (uint32_t)lo;
-        w.hi_key = (uint32_t)(hi - 1) + 1u;          // (hi <= 2^31)
-        w.shift = sh;
-        w.miss = 0;
-        w.t_lo = thr_of_key(C, (uint32_t)lo);
-        w.t_hi = thr_of_key(C, (uint32_t)(hi - 1));
-        w.pad[0] = w.pad[1] = 0;
-        win[h] = w;
-        below[h] = 0;
-        cand_n[h] = 0;
-    }
+    if (!s_last) return;
+    __threadfence();
+    select_window(h, n_per_head, C, hh, win, below, cand_n, s_wtot, s_blk, s_out);
 }
 
 // ---------------------------------------------------------------------------
@@ -339,74 +363,80 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
 }
 
 // ---------------------------------------------------------------------------
-// F: exact median from the window keys
+// F + X + U + S: per head the exact median (or the exact fallback), the
+// uncertain keys above it; the last CTA then scans the tile counts
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(WIN_THREADS)
-k_med_final(uint64_t n_per_head, float C, WinState *__restrict__ win,
-            const unsigned long long *__restrict__ below,
-            const unsigned long long *__restrict__ cand_n, const uint32_t *__restrict__ cand,
-            uint64_t cand_cap, const uint32_t *__restrict__ fine_hist,
-            const unsigned long long *__restrict__ amb_n, uint64_t amb_cap,
-            float *__restrict__ rmed, float *__restrict__ thr) {
-    __shared__ uint32_t s_wtot[32];
-    __shared__ uint32_t s_blk[KEY_BINS / 32];
-    __shared__ uint32_t s_out[4];
-    __shared__ uint32_t s_cnt[FINAL_KEYS];             // one counter per key of the bin
-    const int h = blockIdx.x;
-    const WinState w = win[h];
+struct FinalSmem {
+    uint32_t buf[FINAL_KEYS];          // per-key counters (median) or 2048 bins (fallback)
+    uint32_t blk[KEY_BINS / 32];
+    uint32_t wtot[32];
+    uint32_t out[4];
+    float thr;
+    uint32_t miss, last;
+};
+
+// Exact median of head h from the window keys.  False if the window missed.
+__device__ bool window_median(int h, uint64_t n_per_head, float C, const WinState &w,
+                              const unsigned long long *below, const unsigned long long *cand_n,
+                              const uint32_t *cand, uint64_t cand_cap, const uint32_t *fine_hist,
+                              bool amb_overflow, float *rmed, float *thr, FinalSmem &sm) {
     const long long k = (long long)(n_per_head / 2 - 1) - (long long)below[h];
     const unsigned long long nc = cand_n[h];
-    const bool miss = (*amb_n > amb_cap) || k < 0 || (unsigned long long)k >= nc ||
-                      nc > cand_cap || (1u << w.shift) > (uint32_t)FINAL_KEYS;
-    if (miss) {                                        // block-uniform
-        if (threadIdx.x == 0) win[h].miss = 1;
-        return;
-    }
+    if (amb_overflow || k < 0 || (unsigned long long)k >= nc || nc > cand_cap ||
+        (1u << w.shift) > (uint32_t)FINAL_KEYS)
+        return false;                                  // (block-uniform)
     const uint32_t *fh = fine_hist + (size_t)h * KEY_BINS;
-    rank_bin_totals<KEY_BINS>(fh, s_wtot, s_blk);
-    rank_bin_find<KEY_BINS>(fh, s_wtot, s_blk, (uint64_t)k, s_out, 0);
-    const uint32_t bin_lo = w.lo_key + (s_out[0] << w.shift);
-    const uint32_t kk = s_out[2];                      // rank inside the fine bin
+    rank_bin_totals<KEY_BINS, false>(fh, sm.wtot, sm.blk);
+    rank_bin_find<KEY_BINS, false>(fh, sm.wtot, sm.blk, (uint64_t)k, sm.out, 0);
+    const uint32_t bin_lo = w.lo_key + (sm.out[0] << w.shift);
+    const uint32_t kk = sm.out[2];                     // rank inside the fine bin
     const uint32_t width = 1u << w.shift;
-    for (uint32_t i = threadIdx.x; i < (uint32_t)FINAL_KEYS; i += WIN_THREADS) s_cnt[i] = 0;
+    for (uint32_t i = threadIdx.x; i < (uint32_t)FINAL_KEYS; i += WIN_THREADS) sm.buf[i] = 0;
     __syncthreads();
     // count every candidate key of the bin by its exact value (bf16 inputs
     // repeat values, so a bin may hold many equal keys)
     const uint32_t *ch = cand + (uint64_t)h * cand_cap;
-    for (uint64_t i = threadIdx.x; i < nc; i += WIN_THREADS) {
-        const uint32_t d = ch[i] - bin_lo;
-        if (d < width) atomicAdd(&s_cnt[d], 1u);
+    constexpr int U = 4;
+    for (uint64_t i0 = threadIdx.x; i0 < nc; i0 += (uint64_t)U * WIN_THREADS) {
+        uint32_t d[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint64_t i = i0 + (uint64_t)u * WIN_THREADS;
+            d[u] = i < nc ? ch[i] - bin_lo : 0xFFFFFFFFu;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (d[u] < width) atomicAdd(&sm.buf[d[u]], 1u);
     }
     __syncthreads();
-    rank_bin_totals<FINAL_KEYS>(s_cnt, s_wtot, s_blk);
-    rank_bin_find<FINAL_KEYS>(s_cnt, s_wtot, s_blk, kk, s_out, 1);
+    rank_bin_totals<FINAL_KEYS, false>(sm.buf, sm.wtot, sm.blk);
+    rank_bin_find<FINAL_KEYS, false>(sm.buf, sm.wtot, sm.blk, kk, sm.out, 1);
     if (threadIdx.x == 0) {
-        const float m = key_to_float(bin_lo + s_out[1]);
+        const float m = key_to_float(bin_lo + sm.out[1]);
+        const float t = __fmul_rn(C, m);
         rmed[h] = m;
-        thr[h] = __fmul_rn(C, m);
+        thr[h] = t;
+        sm.thr = t;
     }
+    __syncthreads();
+    return true;
 }
 
-// ---------------------------------------------------------------------------
-// X: exact fallback for heads whose window missed (one CTA per head)
-// ---------------------------------------------------------------------------
+// Exact three-pass radix select over x for head h, then its exact tile
+// counts (the path when the sample window missed the median).
 template <int DT, int GRAN>
-__global__ void __launch_bounds__(WIN_THREADS)
-k_fallback_exact(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tiles_per_slab,
-                 uint64_t n_per_head, float C, const WinState *__restrict__ win,
-                 float *__restrict__ rmed, float *__restrict__ thr, uint32_t *__restrict__ tile_cnt,
-                 DevStatus *st) {
+__device__ void exact_fallback(const void *x, int B, int H, int h, uint32_t cps,
+                               uint32_t tiles_per_slab, uint64_t n_per_head, float C, float *rmed,
+                               float *thr, uint32_t *tile_cnt, DevStatus *st, FinalSmem &sm) {
     constexpr int NK = GRAN == HQMQ_GRAN_CHUNK ? 1 : 4;
-    __shared__ uint32_t s_hist[2048];
-    __shared__ uint32_t s_warp[32];
-    __shared__ uint32_t s_out[4];
-    const int h = blockIdx.x;
-    if (!win[h].miss) return;                              // the common case
+    uint32_t *s_hist = sm.buf;                         // 2048 bins
+    uint32_t *s_warp = sm.wtot;
     if (threadIdx.x == 0 && st) atomicOr(&st->flags, HQMQ_FLAG_MED3_FALLBACK);
     uint32_t prefix = 0;
     uint64_t krem = n_per_head / 2 - 1;
     const int shifts[3] = {20, 9, 0};
     const int widths[3] = {11, 11, 9};
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     for (int P = 0; P < 3; ++P) {
         for (int i = threadIdx.x; i < 2048; i += WIN_THREADS) s_hist[i] = 0;
         __syncthreads();
@@ -426,44 +456,32 @@ k_fallback_exact(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_
             }
         }
         __syncthreads();
-        // 2048 bins: threads 0..1023 own 2 bins each; reuse the 64-bin finder
-        // through a padded copy is unnecessary: scan directly
-        uint32_t b0 = s_hist[2 * threadIdx.x], b1 = s_hist[2 * threadIdx.x + 1];
-        uint32_t local = b0 + b1, inc = local;
-        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            uint32_t v = __shfl_up_sync(FULL, inc, o);
-            if (lane >= o) inc += v;
-        }
+        // 2048 bins: thread t owns bins 2t and 2t+1
+        const uint32_t b0 = s_hist[2 * threadIdx.x], b1 = s_hist[2 * threadIdx.x + 1];
+        const uint32_t local = b0 + b1;
+        const uint32_t inc = warp_incl_scan(local, lane);
         if (lane == 31) s_warp[wid] = inc;
         __syncthreads();
         if (wid == 0) {
-            uint32_t wv = s_warp[lane], wi = wv;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                uint32_t v = __shfl_up_sync(FULL, wi, o);
-                if (lane >= o) wi += v;
-            }
-            s_warp[lane] = wi - wv;
+            const uint32_t wv = s_warp[lane];
+            s_warp[lane] = warp_incl_scan(wv, lane) - wv;
         }
         __syncthreads();
         const uint64_t excl = (uint64_t)s_warp[wid] + inc - local;
         if (krem >= excl && krem < excl + local) {
             const uint32_t digit = krem < excl + b0 ? 2 * threadIdx.x : 2 * threadIdx.x + 1;
-            s_out[0] = digit;
-            s_out[1] = (uint32_t)(krem - (krem < excl + b0 ? excl : excl + b0));
+            sm.out[0] = digit;
+            sm.out[1] = (uint32_t)(krem - (krem < excl + b0 ? excl : excl + b0));
         }
         __syncthreads();
-        prefix |= s_out[0] << sh;
-        krem = s_out[1];
+        prefix |= sm.out[0] << sh;
+        krem = sm.out[1];
         __syncthreads();
     }
     const float m = key_to_float(prefix);
     const float th = __fmul_rn(C, m);
     if (threadIdx.x == 0) { rmed[h] = m; thr[h] = th; }
     // exact tile counts of this head's slabs
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const uint32_t gps = cps / 32;
     for (int b = 0; b < B; ++b) {
         const uint64_t slab = (uint64_t)b * H + h;
@@ -484,96 +502,102 @@ k_fallback_exact(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_
     }
 }
 
-// ---------------------------------------------------------------------------
-// U: uncertain keys above the exact threshold
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
-k_amb_fixup(int H, uint32_t tiles_per_slab, const WinState *__restrict__ win,
-            const float *__restrict__ thr, const unsigned long long *__restrict__ amb_n,
-            const uint2 *__restrict__ amb, uint64_t amb_cap, uint32_t *__restrict__ tile_cnt) {
-    uint64_t n = *amb_n;
-    if (n > amb_cap) return;                 // every head then took the fallback
-    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (uint64_t)gridDim.x * blockDim.x) {
-        const uint2 e = amb[i];
-        const int h = (int)((e.x / tiles_per_slab) % (uint32_t)H);
-        if (win[h].miss) continue;           // recounted exactly by the fallback
-        if (__uint_as_float(e.y) > thr[h]) atomicAdd(tile_cnt + e.x, 1u);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// S: tile offsets (one CTA; each thread scans a contiguous run of tiles)
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024)
-k_tile_scan(const uint32_t *__restrict__ tile_cnt, uint64_t n_tiles, uint32_t tiles_per_slab,
-            uint32_t n_slabs, uint64_t cap, uint32_t *__restrict__ tile_off,
-            uint32_t *__restrict__ slab_off, DevStatus *st) {
-    __shared__ unsigned long long s_warp[32];
-    __shared__ unsigned long long s_carry;
+// Exclusive scan of the tile counts into tile offsets and slab offsets (one
+// CTA: 4096 tiles per step, 4 per thread, loaded and stored as uint4).
+__device__ void scan_tiles(const uint32_t *tile_cnt, uint64_t n_tiles, uint32_t tiles_per_slab,
+                           uint32_t n_slabs, uint64_t cap, uint32_t *tile_off, uint32_t *slab_off,
+                           DevStatus *st, FinalSmem &sm) {
     const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
-    if (t == 0) s_carry = 0;
-    __syncthreads();
-    // blocks of 16384 tiles: thread t scans tiles 16t .. 16t+15 of the block
-    constexpr int PT = 16;
-    for (uint64_t b0 = 0; b0 < n_tiles; b0 += 1024 * PT) {
-        uint32_t v[PT];
-        const uint64_t first = b0 + (uint64_t)PT * t;
-        if (first + PT <= n_tiles) {
-            const uint4 *p4 = reinterpret_cast<const uint4 *>(tile_cnt + first);
-#pragma unroll
-            for (int q = 0; q < PT / 4; ++q) {
-                const uint4 u = p4[q];
-                v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
-            }
+    uint32_t *s_warp = sm.wtot;
+    unsigned long long carry = 0;                      // (the same in every thread)
+    for (uint64_t b0 = 0; b0 < n_tiles; b0 += 4 * WIN_THREADS) {
+        const uint64_t i0 = b0 + 4 * (uint64_t)t;
+        uint32_t v[4] = {0u, 0u, 0u, 0u};
+        const bool full = i0 + 4 <= n_tiles;
+        if (full) {
+            const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(tile_cnt + i0));
+            v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
         } else {
 #pragma unroll
-            for (int k = 0; k < PT; ++k) v[k] = first + k < n_tiles ? tile_cnt[first + k] : 0u;
+            for (int k = 0; k < 4; ++k) v[k] = i0 + k < n_tiles ? __ldcg(tile_cnt + i0 + k) : 0u;
         }
-        unsigned long long local = 0;
-#pragma unroll
-        for (int k = 0; k < PT; ++k) local += v[k];
-        unsigned long long inc = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long u = __shfl_up_sync(FULL, inc, o);
-            if (lane >= o) inc += u;
-        }
+        // (a tile holds at most 4096 keys: every partial sum below fits 32 bits)
+        const uint32_t local = v[0] + v[1] + v[2] + v[3];
+        const uint32_t inc = warp_incl_scan(local, lane);
         if (lane == 31) s_warp[wid] = inc;
         __syncthreads();
         if (wid == 0) {
-            const unsigned long long wv = s_warp[lane];
-            unsigned long long wi = wv;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned long long u = __shfl_up_sync(FULL, wi, o);
-                if (lane >= o) wi += u;
-            }
+            const uint32_t wv = s_warp[lane];
+            const uint32_t wi = warp_incl_scan(wv, lane);
             s_warp[lane] = wi - wv;
+            if (lane == 31) sm.out[0] = wi;                // this step's total
         }
         __syncthreads();
-        unsigned long long run = s_carry + s_warp[wid] + inc - local;
+        const uint32_t o0 = (uint32_t)(carry + s_warp[wid] + inc - local);
+        const uint32_t o1 = o0 + v[0], o2 = o1 + v[1], o3 = o2 + v[2];
+        if (full) {
+            *reinterpret_cast<uint4 *>(tile_off + i0) = make_uint4(o0, o1, o2, o3);
+        } else {
+            const uint32_t o[4] = {o0, o1, o2, o3};
 #pragma unroll
-        for (int k = 0; k < PT; ++k) {
-            const uint64_t i = first + k;
-            if (i < n_tiles) {
-                tile_off[i] = (uint32_t)run;
-                if (i % tiles_per_slab == 0) slab_off[i / tiles_per_slab] = (uint32_t)run;
-            }
-            run += v[k];
+            for (int k = 0; k < 4; ++k)
+                if (i0 + k < n_tiles) tile_off[i0 + k] = o[k];
         }
-        __syncthreads();
-        if (t == 1023) s_carry = run;
-        __syncthreads();
+        carry += sm.out[0];
+        __syncthreads();                               // (s_warp and out reused)
     }
+    // tile_off was written by this CTA: visible to it after the barrier
+    for (uint32_t sl = t; sl < n_slabs; sl += WIN_THREADS)
+        slab_off[sl] = tile_off[(uint64_t)sl * tiles_per_slab];
     if (t == 0) {
-        const unsigned long long total = s_carry;
-        slab_off[n_slabs] = (uint32_t)total;
+        slab_off[n_slabs] = (uint32_t)carry;
         if (st) {
-            atomicAdd(&st->n_outliers, total);
-            if (total > cap) atomicOr(&st->flags, HQMQ_FLAG_OUTLIER_OVERFLOW);
+            atomicAdd(&st->n_outliers, carry);
+            if (carry > cap) atomicOr(&st->flags, HQMQ_FLAG_OUTLIER_OVERFLOW);
         }
     }
+}
+
+template <int DT, int GRAN>
+__global__ void __launch_bounds__(WIN_THREADS)
+k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tiles_per_slab,
+           uint64_t n_tiles, uint64_t n_per_head, float C, WinState *__restrict__ win,
+           const unsigned long long *__restrict__ below,
+           const unsigned long long *__restrict__ cand_n, const uint32_t *__restrict__ cand,
+           uint64_t cand_cap, const uint32_t *__restrict__ fine_hist,
+           const unsigned long long *__restrict__ amb_n, const uint2 *__restrict__ amb,
+           uint64_t amb_cap, float *__restrict__ rmed, float *__restrict__ thr,
+           uint32_t *__restrict__ tile_cnt, uint32_t *__restrict__ tile_off,
+           uint32_t *__restrict__ slab_off, uint32_t n_slabs, uint64_t cap,
+           uint32_t *__restrict__ fin_done, DevStatus *st) {
+    __shared__ FinalSmem sm;
+    const int h = blockIdx.x;
+    const WinState w = win[h];
+    const unsigned long long n_amb = *amb_n;
+    const bool amb_overflow = n_amb > amb_cap;
+    const bool ok = window_median(h, n_per_head, C, w, below, cand_n, cand, cand_cap, fine_hist,
+                                  amb_overflow, rmed, thr, sm);
+    if (!ok) {
+        if (threadIdx.x == 0) win[h].miss = 1;
+        exact_fallback<DT, GRAN>(x, B, H, h, cps, tiles_per_slab, n_per_head, C, rmed, thr,
+                                 tile_cnt, st, sm);
+    } else {
+        // uncertain keys of this head above its exact threshold
+        const float th = sm.thr;
+        for (uint64_t i = threadIdx.x; i < n_amb; i += WIN_THREADS) {
+            const uint2 e = amb[i];
+            if ((int)((e.x / tiles_per_slab) % (uint32_t)H) != h) continue;
+            if (__uint_as_float(e.y) > th) atomicAdd(tile_cnt + e.x, 1u);
+        }
+    }
+    // the last CTA to finish (no CTA waits for another) scans the tiles
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) sm.last = atomicAdd(fin_done, 1u) == gridDim.x - 1 ? 1u : 0u;
+    __syncthreads();
+    if (!sm.last) return;
+    __threadfence();
+    scan_tiles(tile_cnt, n_tiles, tiles_per_slab, n_slabs, cap, tile_off, slab_off, st, sm);
 }
 
 // ---------------------------------------------------------------------------
@@ -587,10 +611,11 @@ static int run_window(const void *x, int B, int H, int T, int D, float C, float 
     const FusedLayout L = fused_layout(B, H, T, D, GRAN);
     uint32_t *sample_hist = reinterpret_cast<uint32_t *>(ws + L.sample_hist);
     uint32_t *fine_hist = reinterpret_cast<uint32_t *>(ws + L.fine_hist);
+    Counters *ctr = reinterpret_cast<Counters *>(ws + L.counters);
+    uint32_t *sample_done = reinterpret_cast<uint32_t *>(ws + L.counters + sizeof(Counters));
     WinState *win = reinterpret_cast<WinState *>(ws + L.win);
     unsigned long long *below = reinterpret_cast<unsigned long long *>(ws + L.below);
     unsigned long long *cand_n = reinterpret_cast<unsigned long long *>(ws + L.cand_n);
-    unsigned long long *amb_n = reinterpret_cast<unsigned long long *>(ws + L.amb_n);
     uint32_t *cand = reinterpret_cast<uint32_t *>(ws + L.cand);
     uint2 *amb = reinterpret_cast<uint2 *>(ws + L.amb);
     uint32_t *tile_cnt = reinterpret_cast<uint32_t *>(ws + L.tile_cnt);
@@ -598,12 +623,12 @@ static int run_window(const void *x, int B, int H, int T, int D, float C, float 
     const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
     const int n_slabs = B * H;
 
-    if (cudaMemsetAsync(sample_hist, 0, (size_t)H * KEY_BINS * 4, stream) != cudaSuccess ||
-        cudaMemsetAsync(amb_n, 0, 8, stream) != cudaSuccess)
-        return HQMQ_ERR_CUDA;
+    // histograms and counters
+    if (cudaMemsetAsync(ws, 0, L.zero_bytes, stream) != cudaSuccess) return HQMQ_ERR_CUDA;
+    // A + W: one wave of CTAs (one per SM: 128 KB of shared counters each)
     const uint32_t n_quads = (cps + SAMPLE_PERIOD - 1) / SAMPLE_PERIOD;
     uint64_t ax = (n_quads + SAMPLE_THREADS - 1) / SAMPLE_THREADS;
-    const uint64_t afill = ((uint64_t)sm_count + n_slabs - 1) / n_slabs;
+    const uint64_t afill = (uint64_t)sm_count / (uint64_t)n_slabs;
     if (ax > afill) ax = afill;
     // 16-bit shared counters: at most 60000 samples per CTA
     const uint64_t keys_per_quad = 4 * (GRAN == HQMQ_GRAN_CHUNK ? 1 : 4);
@@ -611,29 +636,26 @@ static int run_window(const void *x, int B, int H, int T, int D, float C, float 
     if (ax < ax_min) ax = ax_min;
     if (ax < 1) ax = 1;
     const size_t sample_smem = (size_t)KEY_BINS / 2 * sizeof(uint32_t);
-    if (cudaFuncSetAttribute(k_sample_hist<DT, GRAN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(k_sample_window<DT, GRAN>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sample_smem) != cudaSuccess)
         return HQMQ_ERR_CUDA;
-    k_sample_hist<DT, GRAN><<<dim3((unsigned)ax, (unsigned)n_slabs), SAMPLE_THREADS, sample_smem,
-                              stream>>>(
-        x, H, cps, sample_hist);
-    k_window_select<<<H, WIN_THREADS, 0, stream>>>(L.n_per_head, C, sample_hist, fine_hist, win,
-                                                   below, cand_n);
+    k_sample_window<DT, GRAN><<<dim3((unsigned)ax, (unsigned)n_slabs), SAMPLE_THREADS,
+                                sample_smem, stream>>>(x, H, cps, (uint32_t)(ax * B), L.n_per_head,
+                                                       C, sample_hist, sample_done, win, below,
+                                                       cand_n);
+    // B
     uint64_t bx = (L.n_tiles + PB_THREADS / 32 - 1) / (PB_THREADS / 32);
     const uint64_t bmax = (uint64_t)sm_count * 8;
     if (bx > bmax) bx = bmax;
     k_pass_b<DT, GRAN><<<(unsigned)bx, PB_THREADS, 0, stream>>>(
         x, H, cps, L.tiles_per_slab, L.n_tiles, win, below, cand_n, cand, L.cand_cap, fine_hist,
-        amb_n, amb, L.amb_cap, tile_cnt);
-    k_med_final<<<H, WIN_THREADS, 0, stream>>>(L.n_per_head, C, win, below, cand_n, cand,
-                                               L.cand_cap, fine_hist, amb_n, L.amb_cap, rmed, thr);
-    k_fallback_exact<DT, GRAN><<<H, WIN_THREADS, 0, stream>>>(
-        x, B, H, cps, L.tiles_per_slab, L.n_per_head, C, win, rmed, thr, tile_cnt, st);
-    const uint64_t ux = (uint64_t)sm_count * 2;
-    k_amb_fixup<<<(unsigned)ux, 256, 0, stream>>>(H, L.tiles_per_slab, win, thr, amb_n, amb,
-                                                  L.amb_cap, tile_cnt);
-    k_tile_scan<<<1, 1024, 0, stream>>>(tile_cnt, L.n_tiles, L.tiles_per_slab, (uint32_t)n_slabs,
-                                        cap, tile_off, slab_off, st);
+        &ctr->amb_n, amb, L.amb_cap, tile_cnt);
+    // F + X + U + S
+    k_finalize<DT, GRAN><<<H, WIN_THREADS, 0, stream>>>(
+        x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, below, cand_n, cand,
+        L.cand_cap, fine_hist, &ctr->amb_n, amb, L.amb_cap, rmed, thr, tile_cnt, tile_off,
+        slab_off, (uint32_t)n_slabs, cap, &ctr->fin_done, st);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 

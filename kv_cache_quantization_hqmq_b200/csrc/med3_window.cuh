@@ -24,9 +24,18 @@ struct WinState {
     uint32_t pad[2];
 };
 
+// Counters, cleared with the histograms at the start of every call.
+struct Counters {
+    unsigned long long amb_n;  // uncertain (tile, key) pairs appended
+    uint32_t fin_done;         // CTAs of the finalize step that are done
+    uint32_t pad;
+    // followed by uint32_t sample_done[H]: sample CTAs of head h that are done
+};
+
 struct FusedLayout {
-    uint64_t sample_hist, fine_hist, win, below, cand_n, cand, amb_n, amb, tile_cnt, tile_off,
+    uint64_t sample_hist, fine_hist, counters, win, below, cand_n, cand, amb, tile_cnt, tile_off,
         total;
+    uint64_t zero_bytes;       // [0, zero_bytes) is cleared per call
     uint64_t cand_cap;         // keys per head
     uint64_t amb_cap;          // (tile, key) pairs per call
     uint64_t n_per_head;       // keys per head (chunks or elements)
@@ -54,10 +63,11 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     uint64_t off = 0;
     L.sample_hist = off; off = align256_(off + (uint64_t)H * KEY_BINS * 4);
     L.fine_hist = off;   off = align256_(off + (uint64_t)H * KEY_BINS * 4);
+    L.counters = off;    off = align256_(off + sizeof(Counters) + (uint64_t)H * 4);
+    L.zero_bytes = off;
     L.win = off;         off = align256_(off + (uint64_t)H * sizeof(WinState));
     L.below = off;       off = align256_(off + (uint64_t)H * 8);
     L.cand_n = off;      off = align256_(off + (uint64_t)H * 8);
-    L.amb_n = off;       off = align256_(off + 8);
     L.cand = off;        off = align256_(off + (uint64_t)H * L.cand_cap * 4);
     L.amb = off;         off = align256_(off + L.amb_cap * 8);
     L.tile_cnt = off;    off = align256_(off + L.n_tiles * 4);
