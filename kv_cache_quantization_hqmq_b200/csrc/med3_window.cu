@@ -62,41 +62,6 @@ __device__ __forceinline__ void chunk_keys(float x0, float x1, float x2, float x
 // ---------------------------------------------------------------------------
 // Histogram search helpers
 // ---------------------------------------------------------------------------
-// Histogram reads: GLOBAL = bins written by other CTAs (read through L2).
-template <bool GLOBAL>
-__device__ __forceinline__ uint32_t hist_ld(const uint32_t *p) {
-    if constexpr (GLOBAL) return __ldcg(p);
-    else return *p;
-}
-
-// Block-wide (1024 threads = 32 warps) search of a histogram of NB bins, warp
-// w owning the contiguous bins [w NB/32, (w+1) NB/32), read coalesced:
-// rank_bin_totals() stores the warp totals and the totals of every block of
-// 32 bins; rank_bin_find() then locates the warp, the block (from the block
-// totals) and the bin (one 32-bin read), and returns in s_out[which] the bin
-// whose cumulative count first exceeds `rank` and in s_out[which + 2] the
-// rank inside that bin.
-template <int NB, bool GLOBAL>
-__device__ void rank_bin_totals(const uint32_t *hist, uint32_t *s_wtot, uint32_t *s_blk) {
-    constexpr int PER = NB / 32;
-    constexpr int UNR = PER / 32 < 8 ? PER / 32 : 8;       // loads in flight per lane
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    uint32_t acc = 0;
-    for (int i = 0; i < PER; i += 32 * UNR) {
-        uint32_t v[UNR];
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) v[u] = hist_ld<GLOBAL>(hist + w * PER + i + 32 * u + lane);
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const uint32_t bt = __reduce_add_sync(FULL, v[u]);
-            if (lane == 0) s_blk[(w * PER + i) / 32 + u] = bt;
-            acc += bt;
-        }
-    }
-    if (lane == 0) s_wtot[w] = acc;
-    __syncthreads();
-}
-
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -106,46 +71,74 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
     return v;
 }
 
+// Block-wide (1024 threads) select of two ranks in a histogram of NB bins.
+// Warp w owns the contiguous bins [w NB/32, (w+1) NB/32), read as 128-bin
+// pieces (lane l: bins 4l..4l+3 of each piece, one 16-byte load; all pieces
+// in flight).  One block scan of the 32 warp totals finds the warp holding
+// each rank; that warp finds the piece from its piece totals, re-reads that
+// piece and scans it.  Returns in s_out[k] the bin whose cumulative count
+// first exceeds rank k (k = 0, 1) and in s_out[k + 2] the rank inside that bin
+// (NB - 1 and 0 if the rank is not below the total).
+template <bool GLOBAL>
+__device__ __forceinline__ uint4 hist_ld4(const uint32_t *p) {
+    // GLOBAL: bins written by other CTAs of this kernel (read through L2)
+    if constexpr (GLOBAL) return __ldcg(reinterpret_cast<const uint4 *>(p));
+    else return *reinterpret_cast<const uint4 *>(p);
+}
+
 template <int NB, bool GLOBAL>
-__device__ void rank_bin_find(const uint32_t *hist, const uint32_t *s_wtot,
-                              const uint32_t *s_blk, uint64_t rank, uint32_t *s_out, int which) {
-    constexpr int PER = NB / 32;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    uint64_t cum = 0;
-    int ww = 31;
-    for (int k = 0; k < 32; ++k) {
-        const uint32_t t = s_wtot[k];
-        if (rank < cum + t) { ww = k; break; }
-        cum += t;
+__device__ void block_select2(const uint32_t *hist, uint64_t r0, uint64_t r1, uint32_t *s_warp,
+                              uint32_t *s_out) {
+    constexpr int PW = NB / 32;                         // bins per warp
+    constexpr int NP = PW / 128;                        // 128-bin pieces per warp
+    static_assert(PW % 128 == 0 && NP <= 16, "histogram size");
+    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+    if (t == 0) {
+        s_out[0] = s_out[1] = NB - 1;
+        s_out[2] = s_out[3] = 0;
     }
-    if (w == ww) {
-        uint64_t c = cum;
-        int blk = -1;
-        for (int i = 0; i < PER / 32; i += 32) {             // block totals of this warp
-            const uint32_t v = (i + lane < PER / 32) ? s_blk[ww * (PER / 32) + i + lane] : 0u;
-            const uint32_t inc = warp_incl_scan(v, lane);
-            const uint32_t tot = __shfl_sync(FULL, inc, 31);
-            if (rank < c + tot) {
-                const uint32_t bal = __ballot_sync(FULL, rank < c + inc);
-                const int src = __ffs(bal) - 1;
-                blk = i + src;
-                c += __shfl_sync(FULL, inc - v, src);
-                break;
-            }
-            c += tot;
+    const uint32_t *wh = hist + wid * PW;
+    uint32_t ps[NP];
+#pragma unroll
+    for (int c = 0; c < NP; ++c) {
+        const uint4 u = hist_ld4<GLOBAL>(wh + c * 128 + 4 * lane);
+        ps[c] = u.x + u.y + u.z + u.w;
+    }
+    uint32_t wtot = 0;
+#pragma unroll
+    for (int c = 0; c < NP; ++c) {
+        ps[c] = __reduce_add_sync(FULL, ps[c]);
+        wtot += ps[c];
+    }
+    if (lane == 0) s_warp[wid] = wtot;
+    __syncthreads();
+    if (wid == 0) {
+        const uint32_t wv = s_warp[lane];
+        s_warp[lane] = warp_incl_scan(wv, lane) - wv;
+    }
+    __syncthreads();
+    const uint64_t wex = s_warp[wid];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const uint64_t r = k ? r1 : r0;
+        if (r < wex || r >= wex + wtot) continue;       // (warp-uniform)
+        uint64_t c0 = wex;
+        int pc = NP - 1;
+#pragma unroll
+        for (int c = 0; c < NP; ++c) {
+            if (r < c0 + ps[c]) { pc = c; break; }
+            c0 += ps[c];
         }
-        if (blk >= 0) {                   // (rank below the total, as the callers ensure)
-            const uint32_t v = hist_ld<GLOBAL>(hist + ww * PER + blk * 32 + lane);
-            const uint32_t inc = warp_incl_scan(v, lane);
-            const bool mine = rank >= c + inc - v && rank < c + inc;
-            const uint32_t bal = __ballot_sync(FULL, mine);
-            if (lane == __ffs(bal) - 1) {
-                s_out[which] = (uint32_t)(ww * PER + blk * 32 + lane);
-                s_out[which + 2] = (uint32_t)(rank - (c + inc - v));
-            }
-        } else if (lane == 0) {
-            s_out[which] = NB - 1;
-            s_out[which + 2] = 0;
+        const uint4 u = hist_ld4<GLOBAL>(wh + pc * 128 + 4 * lane);
+        const uint32_t ls = u.x + u.y + u.z + u.w;
+        const uint32_t inc = warp_incl_scan(ls, lane);
+        const uint64_t before = c0 + inc - ls;
+        if (r >= before && r < before + ls) {
+            const uint32_t rr = (uint32_t)(r - before);
+            const uint32_t e = rr < u.x ? 0 : rr < u.x + u.y ? 1 : rr < u.x + u.y + u.z ? 2 : 3;
+            const uint32_t eb = e == 0 ? 0 : e == 1 ? u.x : e == 2 ? u.x + u.y : u.x + u.y + u.z;
+            s_out[k] = (uint32_t)(wid * PW + pc * 128 + 4 * lane) + e;
+            s_out[k + 2] = rr - eb;
         }
     }
     __syncthreads();
@@ -156,22 +149,18 @@ __device__ void rank_bin_find(const uint32_t *hist, const uint32_t *s_wtot,
 // ---------------------------------------------------------------------------
 constexpr int SAMPLE_THREADS = 1024;
 
-// Window of head h from its complete sample histogram (one CTA).
-__device__ void select_window(int h, uint64_t n_per_head, float C, const uint32_t *hist,
-                              WinState *win, unsigned long long *below,
-                              unsigned long long *cand_n, uint32_t *s_wtot, uint32_t *s_blk,
-                              uint32_t *s_out) {
-    rank_bin_totals<KEY_BINS, true>(hist, s_wtot, s_blk);
-    uint64_t tot = 0;
-    for (int k = 0; k < 32; ++k) tot += s_wtot[k];
-    const double ns = (double)tot;
+// Window of head h from its complete sample histogram (one CTA).  n_samples:
+// the head's sample count (every sampled quad adds 4 chunks' keys).
+__device__ void select_window(int h, uint64_t n_per_head, uint64_t n_samples, float C,
+                              const uint32_t *hist, WinState *win, unsigned long long *below,
+                              unsigned long long *cand_n, uint32_t *s_warp, uint32_t *s_out) {
+    const double ns = (double)n_samples;
     const double q = ((double)(n_per_head / 2 - 1) + 0.5) / (double)n_per_head;
     const double half = WINDOW_SIGMAS * 0.5 * sqrt(ns) + 4.0;
     double rlo = floor(q * ns - half), rhi = ceil(q * ns + half);
     if (rlo < 0) rlo = 0;
     if (rhi > ns - 1) rhi = ns - 1;
-    rank_bin_find<KEY_BINS, true>(hist, s_wtot, s_blk, (uint64_t)rlo, s_out, 0);
-    rank_bin_find<KEY_BINS, true>(hist, s_wtot, s_blk, (uint64_t)rhi, s_out, 1);
+    block_select2<KEY_BINS, true>(hist, (uint64_t)rlo, (uint64_t)rhi, s_warp, s_out);
     if (threadIdx.x == 0) {
         WinState w;
         const uint64_t lo = (uint64_t)s_out[0] << 15;
@@ -194,16 +183,16 @@ __device__ void select_window(int h, uint64_t n_per_head, float C, const uint32_
 }
 
 template <int DT, int GRAN>
-__global__ void __launch_bounds__(SAMPLE_THREADS)
+__global__ void __launch_bounds__(SAMPLE_THREADS, 1)
 k_sample_window(const void *__restrict__ x, int H, uint32_t cps, uint32_t ctas_per_head,
-                uint64_t n_per_head, float C, uint32_t *__restrict__ hist,
+                uint64_t n_per_head, uint64_t n_samples, float C, uint32_t *__restrict__ hist,
                 uint32_t *__restrict__ sample_done, WinState *__restrict__ win,
                 unsigned long long *__restrict__ below, unsigned long long *__restrict__ cand_n) {
     // per-CTA histogram in shared memory: 65536 16-bit counters packed in
     // pairs (a CTA sees far fewer than 65536 samples), then one global add
     // per non-empty bin
     extern __shared__ uint32_t s_pair[];                       // [KEY_BINS / 2]
-    __shared__ uint32_t s_wtot[32], s_blk[KEY_BINS / 32], s_out[4], s_last;
+    __shared__ uint32_t s_warp[32], s_out[4], s_last;
     for (int i = threadIdx.x; i < KEY_BINS / 2; i += blockDim.x) s_pair[i] = 0;
     __syncthreads();
     const int slab = blockIdx.y;
@@ -248,7 +237,7 @@ k_sample_window(const void *__restrict__ x, int H, uint32_t cps, uint32_t ctas_p
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    select_window(h, n_per_head, C, hh, win, below, cand_n, s_wtot, s_blk, s_out);
+    select_window(h, n_per_head, n_samples, C, hh, win, below, cand_n, s_warp, s_out);
 }
 
 // ---------------------------------------------------------------------------
@@ -366,9 +355,8 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
 // F + X + U + S: per head the exact median (or the exact fallback), the
 // uncertain keys above it; the last CTA then scans the tile counts
 // ---------------------------------------------------------------------------
-struct FinalSmem {
+struct __align__(16) FinalSmem {
     uint32_t buf[FINAL_KEYS];          // per-key counters (median) or 2048 bins (fallback)
-    uint32_t blk[KEY_BINS / 32];
     uint32_t wtot[32];
     uint32_t out[4];
     float thr;
@@ -386,33 +374,45 @@ __device__ bool window_median(int h, uint64_t n_per_head, float C, const WinStat
         (1u << w.shift) > (uint32_t)FINAL_KEYS)
         return false;                                  // (block-uniform)
     const uint32_t *fh = fine_hist + (size_t)h * KEY_BINS;
-    rank_bin_totals<KEY_BINS, false>(fh, sm.wtot, sm.blk);
-    rank_bin_find<KEY_BINS, false>(fh, sm.wtot, sm.blk, (uint64_t)k, sm.out, 0);
+    block_select2<KEY_BINS, false>(fh, (uint64_t)k, (uint64_t)k, sm.wtot, sm.out);
     const uint32_t bin_lo = w.lo_key + (sm.out[0] << w.shift);
     const uint32_t kk = sm.out[2];                     // rank inside the fine bin
     const uint32_t width = 1u << w.shift;
+    __syncthreads();                                   // (everyone has read out[])
     for (uint32_t i = threadIdx.x; i < (uint32_t)FINAL_KEYS; i += WIN_THREADS) sm.buf[i] = 0;
     __syncthreads();
     // count every candidate key of the bin by its exact value (bf16 inputs
-    // repeat values, so a bin may hold many equal keys)
+    // repeat values, so a bin may hold many equal keys); 16-byte loads, U in
+    // flight per thread
     const uint32_t *ch = cand + (uint64_t)h * cand_cap;
-    constexpr int U = 4;
-    for (uint64_t i0 = threadIdx.x; i0 < nc; i0 += (uint64_t)U * WIN_THREADS) {
-        uint32_t d[U];
+    const uint4 *ch4 = reinterpret_cast<const uint4 *>(ch);
+    const uint64_t n4 = nc / 4;
+    constexpr int U = 8;
+    for (uint64_t i0 = threadIdx.x; i0 < n4; i0 += (uint64_t)U * WIN_THREADS) {
+        uint4 q[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const uint64_t i = i0 + (uint64_t)u * WIN_THREADS;
-            d[u] = i < nc ? ch[i] - bin_lo : 0xFFFFFFFFu;
+            q[u] = i < n4 ? ch4[i] : make_uint4(bin_lo - 1u, bin_lo - 1u, bin_lo - 1u, bin_lo - 1u);
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u)
-            if (d[u] < width) atomicAdd(&sm.buf[d[u]], 1u);
+        for (int u = 0; u < U; ++u) {
+            const uint32_t d0 = q[u].x - bin_lo, d1 = q[u].y - bin_lo;
+            const uint32_t d2 = q[u].z - bin_lo, d3 = q[u].w - bin_lo;
+            if (d0 < width) atomicAdd(&sm.buf[d0], 1u);
+            if (d1 < width) atomicAdd(&sm.buf[d1], 1u);
+            if (d2 < width) atomicAdd(&sm.buf[d2], 1u);
+            if (d3 < width) atomicAdd(&sm.buf[d3], 1u);
+        }
+    }
+    for (uint64_t i = 4 * n4 + threadIdx.x; i < nc; i += WIN_THREADS) {
+        const uint32_t d = ch[i] - bin_lo;
+        if (d < width) atomicAdd(&sm.buf[d], 1u);
     }
     __syncthreads();
-    rank_bin_totals<FINAL_KEYS, false>(sm.buf, sm.wtot, sm.blk);
-    rank_bin_find<FINAL_KEYS, false>(sm.buf, sm.wtot, sm.blk, kk, sm.out, 1);
+    block_select2<FINAL_KEYS, false>(sm.buf, kk, kk, sm.wtot, sm.out);
     if (threadIdx.x == 0) {
-        const float m = key_to_float(bin_lo + sm.out[1]);
+        const float m = key_to_float(bin_lo + sm.out[0]);
         const float t = __fmul_rn(C, m);
         rmed[h] = m;
         thr[h] = t;
@@ -503,28 +503,42 @@ __device__ void exact_fallback(const void *x, int B, int H, int h, uint32_t cps,
 }
 
 // Exclusive scan of the tile counts into tile offsets and slab offsets (one
-// CTA: 4096 tiles per step, 4 per thread, loaded and stored as uint4).
+// CTA).  Per step, warp w owns SCAN_WARP consecutive tiles, read and written as
+// 128-tile pieces (lane l: tiles 4l..4l+3 of each piece, one 16-byte access;
+// all pieces in flight); each piece is scanned by the warp, the block scans
+// the 32 warp totals.
+constexpr int SCAN_PIECES = 8;
+constexpr int SCAN_WARP = SCAN_PIECES * 128;
 __device__ void scan_tiles(const uint32_t *tile_cnt, uint64_t n_tiles, uint32_t tiles_per_slab,
                            uint32_t n_slabs, uint64_t cap, uint32_t *tile_off, uint32_t *slab_off,
                            DevStatus *st, FinalSmem &sm) {
     const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
     uint32_t *s_warp = sm.wtot;
     unsigned long long carry = 0;                      // (the same in every thread)
-    for (uint64_t b0 = 0; b0 < n_tiles; b0 += 4 * WIN_THREADS) {
-        const uint64_t i0 = b0 + 4 * (uint64_t)t;
-        uint32_t v[4] = {0u, 0u, 0u, 0u};
-        const bool full = i0 + 4 <= n_tiles;
-        if (full) {
-            const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(tile_cnt + i0));
-            v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
-        } else {
+    for (uint64_t b0 = 0; b0 < n_tiles; b0 += (uint64_t)SCAN_WARP * 32) {
+        const uint64_t wb = b0 + (uint64_t)wid * SCAN_WARP;
+        uint4 v[SCAN_PIECES];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) v[k] = i0 + k < n_tiles ? __ldcg(tile_cnt + i0 + k) : 0u;
+        for (int c = 0; c < SCAN_PIECES; ++c) {
+            const uint64_t i0 = wb + c * 128 + 4 * lane;
+            if (i0 + 4 <= n_tiles) {
+                v[c] = __ldcg(reinterpret_cast<const uint4 *>(tile_cnt + i0));
+            } else {
+                v[c].x = i0 < n_tiles ? __ldcg(tile_cnt + i0) : 0u;
+                v[c].y = i0 + 1 < n_tiles ? __ldcg(tile_cnt + i0 + 1) : 0u;
+                v[c].z = i0 + 2 < n_tiles ? __ldcg(tile_cnt + i0 + 2) : 0u;
+                v[c].w = 0u;                           // (i0 + 3 >= n_tiles here)
+            }
         }
         // (a tile holds at most 4096 keys: every partial sum below fits 32 bits)
-        const uint32_t local = v[0] + v[1] + v[2] + v[3];
-        const uint32_t inc = warp_incl_scan(local, lane);
-        if (lane == 31) s_warp[wid] = inc;
+        uint32_t inc[SCAN_PIECES], ls[SCAN_PIECES], wtot = 0;
+#pragma unroll
+        for (int c = 0; c < SCAN_PIECES; ++c) {
+            ls[c] = v[c].x + v[c].y + v[c].z + v[c].w;
+            inc[c] = warp_incl_scan(ls[c], lane);
+            wtot += __shfl_sync(FULL, inc[c], 31);
+        }
+        if (lane == 0) s_warp[wid] = wtot;
         __syncthreads();
         if (wid == 0) {
             const uint32_t wv = s_warp[lane];
@@ -533,15 +547,23 @@ __device__ void scan_tiles(const uint32_t *tile_cnt, uint64_t n_tiles, uint32_t 
             if (lane == 31) sm.out[0] = wi;                // this step's total
         }
         __syncthreads();
-        const uint32_t o0 = (uint32_t)(carry + s_warp[wid] + inc - local);
-        const uint32_t o1 = o0 + v[0], o2 = o1 + v[1], o3 = o2 + v[2];
-        if (full) {
-            *reinterpret_cast<uint4 *>(tile_off + i0) = make_uint4(o0, o1, o2, o3);
-        } else {
-            const uint32_t o[4] = {o0, o1, o2, o3};
+        uint32_t base = (uint32_t)(carry + s_warp[wid]);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                if (i0 + k < n_tiles) tile_off[i0 + k] = o[k];
+        for (int c = 0; c < SCAN_PIECES; ++c) {
+            const uint64_t i0 = wb + c * 128 + 4 * lane;
+            uint4 o;
+            o.x = base + inc[c] - ls[c];
+            o.y = o.x + v[c].x;
+            o.z = o.y + v[c].y;
+            o.w = o.z + v[c].z;
+            if (i0 + 4 <= n_tiles) {
+                *reinterpret_cast<uint4 *>(tile_off + i0) = o;
+            } else {
+                if (i0 < n_tiles) tile_off[i0] = o.x;
+                if (i0 + 1 < n_tiles) tile_off[i0 + 1] = o.y;
+                if (i0 + 2 < n_tiles) tile_off[i0 + 2] = o.z;
+            }
+            base += __shfl_sync(FULL, inc[c], 31);
         }
         carry += sm.out[0];
         __syncthreads();                               // (s_warp and out reused)
@@ -642,7 +664,8 @@ static int run_window(const void *x, int B, int H, int T, int D, float C, float 
         return HQMQ_ERR_CUDA;
     k_sample_window<DT, GRAN><<<dim3((unsigned)ax, (unsigned)n_slabs), SAMPLE_THREADS,
                                 sample_smem, stream>>>(x, H, cps, (uint32_t)(ax * B), L.n_per_head,
-                                                       C, sample_hist, sample_done, win, below,
+                                                       (uint64_t)B * n_quads * keys_per_quad, C,
+                                                       sample_hist, sample_done, win, below,
                                                        cand_n);
     // B
     uint64_t bx = (L.n_tiles + PB_THREADS / 32 - 1) / (PB_THREADS / 32);

@@ -58,6 +58,7 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     const double frac = (2.0 * WINDOW_SIGMAS * 0.5 * sqrt(ns) + 8.0) / ns + 0.02;
     uint64_t cap = (uint64_t)(2.0 * frac * (double)L.n_per_head) + 4096;
     L.cand_cap = cap < L.n_per_head ? cap : L.n_per_head;
+    L.cand_cap = (L.cand_cap + 3) & ~(uint64_t)3;   // each head's keys start 16-byte aligned
     const uint64_t n_keys = L.n_per_head * H;
     L.amb_cap = n_keys / 25 + 4096;              // 4% of the keys may sit in thr's band
     uint64_t off = 0;
