@@ -31,6 +31,24 @@ extern "C" int hqmq_launch_med3_window(const void *x, int dtype, int B, int H, i
                                        uint32_t *slab_off, uint64_t cap, void *ws,
                                        hqmq_status *st, int sm_count, cudaStream_t stream,
                                        const uint32_t **tile_off, uint32_t *tiles_per_slab);
+extern "C" int hqmq_launch_med3_front(const void *x, int dtype, int B, int H, int T, int D,
+                                      float C, int gran, void *ws, int pass_b, int sm_count,
+                                      cudaStream_t stream);
+extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, int T, int D,
+                                       float C, int gran, float *rmed, float *thr,
+                                       uint32_t *slab_off, uint64_t cap, void *ws,
+                                       hqmq_status *st, cudaStream_t stream,
+                                       const uint32_t **tile_off, uint32_t *tiles_per_slab);
+extern "C" int hqmq_launch_spec_encode(const void *x, int dtype, int B, int H, int T, int D,
+                                       const float *cb, uint32_t S, uint32_t b, const void *table,
+                                       uint32_t *words, uint16_t *radius, void *ws, int sm_count,
+                                       cudaStream_t stream);
+extern "C" int hqmq_launch_fix_pass(const void *x, int dtype, int B, int H, int T, int D,
+                                    const float *cb, uint32_t S, uint32_t b, const void *table,
+                                    const float *thr, uint32_t *words, uint16_t *radius,
+                                    const uint32_t *tile_off, uint64_t cap, uint32_t *out_idx,
+                                    uint16_t *out_val, void *ws, hqmq_status *st, int sm_count,
+                                    cudaStream_t stream);
 extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int T, int D,
                                      const float *cb, uint32_t S, uint32_t b, const void *table,
                                      const float *thr, int gran, uint32_t *words,
@@ -180,11 +198,28 @@ int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, flo
     if (sm <= 0) return HQMQ_ERR_CUDA;
     const uint32_t *tile_off = nullptr;
     uint32_t tps = 0;
-    int rc = hqmq_launch_med3_window(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_slab_off,
-                                     cap, d_ws, d_status, sm, (cudaStream_t)stream, &tile_off,
-                                     &tps);
-    if (rc != HQMQ_OK) return rc;
     const uint32_t b = hqmq_index_bits(S);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (d_table && gran == HQMQ_GRAN_CHUNK) {
+        // one read of x: the encode pass also does pass B's work and encodes
+        // speculatively; the fix-up pass then reads only the chunks that may
+        // be outliers
+        int rc = hqmq_launch_med3_front(d_x, dtype, B, H, T, D, C, gran, d_ws, 0, sm, s);
+        if (rc == HQMQ_OK)
+            rc = hqmq_launch_spec_encode(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table,
+                                         d_idx_words, d_radius, d_ws, sm, s);
+        if (rc == HQMQ_OK)
+            rc = hqmq_launch_med3_finish(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr,
+                                         d_slab_off, cap, d_ws, d_status, s, &tile_off, &tps);
+        if (rc == HQMQ_OK)
+            rc = hqmq_launch_fix_pass(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table, d_thr,
+                                      d_idx_words, d_radius, tile_off, cap, d_out_idx, d_out_val,
+                                      d_ws, d_status, sm, s);
+        return rc;
+    }
+    int rc = hqmq_launch_med3_window(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_slab_off,
+                                     cap, d_ws, d_status, sm, s, &tile_off, &tps);
+    if (rc != HQMQ_OK) return rc;
     if (d_table)   // list and encode in the same (second) read of x
         return hqmq_launch_list_pass(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table, d_thr,
                                      gran, d_idx_words, d_radius, tile_off, cap, d_out_idx,

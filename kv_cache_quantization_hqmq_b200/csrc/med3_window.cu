@@ -243,20 +243,6 @@ k_sample_window(const void *__restrict__ x, int H, uint32_t cps, uint32_t ctas_p
 // ---------------------------------------------------------------------------
 // B: one full read
 // ---------------------------------------------------------------------------
-constexpr int STAGE = 256;          // window keys staged per warp before one global append
-
-// Appends the warp's staged window keys to the head's buffer (one atomic).
-__device__ __forceinline__ void flush_stage(uint32_t *stage, uint32_t n, int lane,
-                                            unsigned long long *cand_n_h, uint32_t *cand_h,
-                                            uint64_t cand_cap) {
-    unsigned long long base = 0;
-    if (lane == 0) base = atomicAdd(cand_n_h, (unsigned long long)n);
-    base = __shfl_sync(FULL, base, 0);
-    for (uint32_t i = lane; i < n; i += 32)
-        if (base + i < cand_cap) cand_h[base + i] = stage[i];
-    __syncwarp();
-}
-
 template <int DT, int GRAN>
 __global__ void __launch_bounds__(PB_THREADS)
 k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_slab, uint64_t n_tiles,
@@ -625,27 +611,19 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
 // ---------------------------------------------------------------------------
 // host: steps A..S (the caller then launches pass C)
 // ---------------------------------------------------------------------------
+// Memset, A + W and (unless the caller's encode pass does its work) B.
 template <int DT, int GRAN>
-static int run_window(const void *x, int B, int H, int T, int D, float C, float *rmed, float *thr,
-                      uint32_t *slab_off, uint64_t cap, char *ws, hqmq_status *st_,
-                      int sm_count, cudaStream_t stream) {
-    DevStatus *st = reinterpret_cast<DevStatus *>(st_);
+static int run_front(const void *x, int B, int H, int T, int D, float C, char *ws, bool pass_b,
+                     int sm_count, cudaStream_t stream) {
     const FusedLayout L = fused_layout(B, H, T, D, GRAN);
+    const SpecArgs a = spec_args(ws, L);
     uint32_t *sample_hist = reinterpret_cast<uint32_t *>(ws + L.sample_hist);
-    uint32_t *fine_hist = reinterpret_cast<uint32_t *>(ws + L.fine_hist);
-    Counters *ctr = reinterpret_cast<Counters *>(ws + L.counters);
     uint32_t *sample_done = reinterpret_cast<uint32_t *>(ws + L.counters + sizeof(Counters));
     WinState *win = reinterpret_cast<WinState *>(ws + L.win);
-    unsigned long long *below = reinterpret_cast<unsigned long long *>(ws + L.below);
-    unsigned long long *cand_n = reinterpret_cast<unsigned long long *>(ws + L.cand_n);
-    uint32_t *cand = reinterpret_cast<uint32_t *>(ws + L.cand);
-    uint2 *amb = reinterpret_cast<uint2 *>(ws + L.amb);
-    uint32_t *tile_cnt = reinterpret_cast<uint32_t *>(ws + L.tile_cnt);
-    uint32_t *tile_off = reinterpret_cast<uint32_t *>(ws + L.tile_off);
     const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
     const int n_slabs = B * H;
 
-    // histograms and counters
+    // histograms, counters and per-head status counts
     if (cudaMemsetAsync(ws, 0, L.zero_bytes, stream) != cudaSuccess) return HQMQ_ERR_CUDA;
     // A + W: one wave of CTAs (one per SM: 128 KB of shared counters each)
     const uint32_t n_quads = (cps + SAMPLE_PERIOD - 1) / SAMPLE_PERIOD;
@@ -665,20 +643,35 @@ static int run_window(const void *x, int B, int H, int T, int D, float C, float 
     k_sample_window<DT, GRAN><<<dim3((unsigned)ax, (unsigned)n_slabs), SAMPLE_THREADS,
                                 sample_smem, stream>>>(x, H, cps, (uint32_t)(ax * B), L.n_per_head,
                                                        (uint64_t)B * n_quads * keys_per_quad, C,
-                                                       sample_hist, sample_done, win, below,
-                                                       cand_n);
-    // B
-    uint64_t bx = (L.n_tiles + PB_THREADS / 32 - 1) / (PB_THREADS / 32);
-    const uint64_t bmax = (uint64_t)sm_count * 8;
-    if (bx > bmax) bx = bmax;
-    k_pass_b<DT, GRAN><<<(unsigned)bx, PB_THREADS, 0, stream>>>(
-        x, H, cps, L.tiles_per_slab, L.n_tiles, win, below, cand_n, cand, L.cand_cap, fine_hist,
-        &ctr->amb_n, amb, L.amb_cap, tile_cnt);
-    // F + X + U + S
+                                                       sample_hist, sample_done, win, a.below,
+                                                       a.cand_n);
+    if (pass_b) {
+        uint64_t bx = (L.n_tiles + PB_THREADS / 32 - 1) / (PB_THREADS / 32);
+        const uint64_t bmax = (uint64_t)sm_count * 8;
+        if (bx > bmax) bx = bmax;
+        k_pass_b<DT, GRAN><<<(unsigned)bx, PB_THREADS, 0, stream>>>(
+            x, H, cps, L.tiles_per_slab, L.n_tiles, win, a.below, a.cand_n, a.cand, a.cand_cap,
+            a.fine_hist, a.amb_n, a.amb, a.amb_cap, a.tile_cnt);
+    }
+    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}
+
+// F + X + U + S.
+template <int DT, int GRAN>
+static int run_finish(const void *x, int B, int H, int T, int D, float C, float *rmed, float *thr,
+                      uint32_t *slab_off, uint64_t cap, char *ws, hqmq_status *st_,
+                      cudaStream_t stream) {
+    DevStatus *st = reinterpret_cast<DevStatus *>(st_);
+    const FusedLayout L = fused_layout(B, H, T, D, GRAN);
+    const SpecArgs a = spec_args(ws, L);
+    Counters *ctr = reinterpret_cast<Counters *>(ws + L.counters);
+    WinState *win = reinterpret_cast<WinState *>(ws + L.win);
+    uint32_t *tile_off = reinterpret_cast<uint32_t *>(ws + L.tile_off);
+    const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
     k_finalize<DT, GRAN><<<H, WIN_THREADS, 0, stream>>>(
-        x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, below, cand_n, cand,
-        L.cand_cap, fine_hist, &ctr->amb_n, amb, L.amb_cap, rmed, thr, tile_cnt, tile_off,
-        slab_off, (uint32_t)n_slabs, cap, &ctr->fin_done, st);
+        x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, a.below, a.cand_n,
+        a.cand, a.cand_cap, a.fine_hist, a.amb_n, a.amb, a.amb_cap, rmed, thr, a.tile_cnt,
+        tile_off, slab_off, (uint32_t)(B * H), cap, &ctr->fin_done, st);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
@@ -688,27 +681,55 @@ extern "C" uint64_t hqmq_window_workspace_bytes(int B, int H, int T, int D, int 
     return hqmq::fused_layout(B, H, T, D, gran).total;
 }
 
-// Steps A..S; returns the tile offsets (inside ws) for pass C.
-extern "C" int hqmq_launch_med3_window(const void *x, int dtype, int B, int H, int T, int D,
+// Steps memset, A + W and (if pass_b) B.
+extern "C" int hqmq_launch_med3_front(const void *x, int dtype, int B, int H, int T, int D,
+                                      float C, int gran, void *ws, int pass_b, int sm_count,
+                                      cudaStream_t stream) {
+    using namespace hqmq;
+    char *w = reinterpret_cast<char *>(ws);
+    const bool pb = pass_b != 0;
+    if (dtype == HQMQ_BF16)
+        return gran == HQMQ_GRAN_CHUNK
+                   ? run_front<HQMQ_BF16, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, w, pb, sm_count, stream)
+                   : run_front<HQMQ_BF16, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, w, pb, sm_count,
+                                                             stream);
+    return gran == HQMQ_GRAN_CHUNK
+               ? run_front<HQMQ_F32, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, w, pb, sm_count, stream)
+               : run_front<HQMQ_F32, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, w, pb, sm_count, stream);
+}
+
+// Steps F + X + U + S; returns the tile offsets (inside ws) for the list pass.
+extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, int T, int D,
                                        float C, int gran, float *rmed, float *thr,
                                        uint32_t *slab_off, uint64_t cap, void *ws,
-                                       hqmq_status *st, int sm_count, cudaStream_t stream,
+                                       hqmq_status *st, cudaStream_t stream,
                                        const uint32_t **tile_off, uint32_t *tiles_per_slab) {
     using namespace hqmq;
     const FusedLayout L = fused_layout(B, H, T, D, gran);
     char *w = reinterpret_cast<char *>(ws);
     *tile_off = reinterpret_cast<const uint32_t *>(w + L.tile_off);
     *tiles_per_slab = L.tiles_per_slab;
-    if (dtype == HQMQ_BF16) {
-        if (gran == HQMQ_GRAN_CHUNK)
-            return run_window<HQMQ_BF16, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off,
-                                                          cap, w, st, sm_count, stream);
-        return run_window<HQMQ_BF16, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr, slab_off, cap,
-                                                        w, st, sm_count, stream);
-    }
-    if (gran == HQMQ_GRAN_CHUNK)
-        return run_window<HQMQ_F32, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off, cap, w,
-                                                     st, sm_count, stream);
-    return run_window<HQMQ_F32, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr, slab_off, cap, w,
-                                                   st, sm_count, stream);
+    if (dtype == HQMQ_BF16)
+        return gran == HQMQ_GRAN_CHUNK
+                   ? run_finish<HQMQ_BF16, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off,
+                                                            cap, w, st, stream)
+                   : run_finish<HQMQ_BF16, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr,
+                                                              slab_off, cap, w, st, stream);
+    return gran == HQMQ_GRAN_CHUNK
+               ? run_finish<HQMQ_F32, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off, cap,
+                                                       w, st, stream)
+               : run_finish<HQMQ_F32, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr, slab_off, cap,
+                                                         w, st, stream);
+}
+
+// All steps A..S (two-read path); returns the tile offsets for pass C.
+extern "C" int hqmq_launch_med3_window(const void *x, int dtype, int B, int H, int T, int D,
+                                       float C, int gran, float *rmed, float *thr,
+                                       uint32_t *slab_off, uint64_t cap, void *ws,
+                                       hqmq_status *st, int sm_count, cudaStream_t stream,
+                                       const uint32_t **tile_off, uint32_t *tiles_per_slab) {
+    const int rc = hqmq_launch_med3_front(x, dtype, B, H, T, D, C, gran, ws, 1, sm_count, stream);
+    if (rc != HQMQ_OK) return rc;
+    return hqmq_launch_med3_finish(x, dtype, B, H, T, D, C, gran, rmed, thr, slab_off, cap, ws, st,
+                                   stream, tile_off, tiles_per_slab);
 }

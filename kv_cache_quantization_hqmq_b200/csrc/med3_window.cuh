@@ -34,7 +34,7 @@ struct Counters {
 
 struct FusedLayout {
     uint64_t sample_hist, fine_hist, counters, win, below, cand_n, cand, amb, tile_cnt, tile_off,
-        total;
+        cbits, head_stat, total;
     uint64_t zero_bytes;       // [0, zero_bytes) is cleared per call
     uint64_t cand_cap;         // keys per head
     uint64_t amb_cap;          // (tile, key) pairs per call
@@ -65,6 +65,7 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     L.sample_hist = off; off = align256_(off + (uint64_t)H * KEY_BINS * 4);
     L.fine_hist = off;   off = align256_(off + (uint64_t)H * KEY_BINS * 4);
     L.counters = off;    off = align256_(off + sizeof(Counters) + (uint64_t)H * 4);
+    L.head_stat = off;   off = align256_(off + (uint64_t)H * 16);   // per head: non-finite, saturated
     L.zero_bytes = off;
     L.win = off;         off = align256_(off + (uint64_t)H * sizeof(WinState));
     L.below = off;       off = align256_(off + (uint64_t)H * 8);
@@ -73,8 +74,54 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     L.amb = off;         off = align256_(off + L.amb_cap * 8);
     L.tile_cnt = off;    off = align256_(off + L.n_tiles * 4);
     L.tile_off = off;    off = align256_(off + L.n_tiles * 4);
+    L.cbits = off;       off = align256_(off + (uint64_t)B * H * gps * 4);
     L.total = off;
     return L;
+}
+
+constexpr int STAGE = 256;          // window keys staged per warp before one global append
+
+// Appends the warp's staged window keys to the head's buffer (one atomic).
+__device__ __forceinline__ void flush_stage(uint32_t *stage, uint32_t n, int lane,
+                                            unsigned long long *cand_n_h, uint32_t *cand_h,
+                                            uint64_t cand_cap) {
+    unsigned long long base = 0;
+    if (lane == 0) base = atomicAdd(cand_n_h, (unsigned long long)n);
+    base = __shfl_sync(FULL, base, 0);
+    for (uint32_t i = lane; i < n; i += 32)
+        if (base + i < cand_cap) cand_h[base + i] = stage[i];
+    __syncwarp();
+}
+
+// Workspace pointers of the one-read chunk-mode path: the encode pass also
+// does pass B's work and encodes speculatively (a chunk above the largest
+// possible threshold t_hi as an outlier, every other chunk as a bulk chunk);
+// the fix-up pass after the exact threshold writes the list.
+struct SpecArgs {
+    const WinState *win;
+    unsigned long long *below, *cand_n, *amb_n;
+    uint32_t *cand, *fine_hist, *tile_cnt;
+    uint2 *amb;
+    uint64_t cand_cap, amb_cap;
+    uint32_t *cbits;                 // per packing group: chunks with r > t_lo
+    unsigned long long *head_stat;   // per head: [non-finite, saturated] of the encode pass
+};
+
+inline SpecArgs spec_args(char *ws, const FusedLayout &L) {
+    SpecArgs a;
+    a.win = reinterpret_cast<const WinState *>(ws + L.win);
+    a.below = reinterpret_cast<unsigned long long *>(ws + L.below);
+    a.cand_n = reinterpret_cast<unsigned long long *>(ws + L.cand_n);
+    a.amb_n = reinterpret_cast<unsigned long long *>(ws + L.counters);   // Counters::amb_n
+    a.cand = reinterpret_cast<uint32_t *>(ws + L.cand);
+    a.fine_hist = reinterpret_cast<uint32_t *>(ws + L.fine_hist);
+    a.tile_cnt = reinterpret_cast<uint32_t *>(ws + L.tile_cnt);
+    a.amb = reinterpret_cast<uint2 *>(ws + L.amb);
+    a.cand_cap = L.cand_cap;
+    a.amb_cap = L.amb_cap;
+    a.cbits = reinterpret_cast<uint32_t *>(ws + L.cbits);
+    a.head_stat = reinterpret_cast<unsigned long long *>(ws + L.head_stat);
+    return a;
 }
 
 }  // namespace hqmq

@@ -307,8 +307,28 @@ __device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b_rt, int la
 // LIST: 0 = no list; HQMQ_GRAN_CHUNK + 1 / HQMQ_GRAN_ELEMENT + 1 = write the
 // ordered outlier list of that granularity (thr exact, tile_off from the
 // Med3x window pipeline).  ENC: encode (else write the list only).
+// LIST_SPEC (chunk mode, the one-read path, before the exact threshold is
+// known): also does pass B's work for the Med3x window (keys below and inside
+// the window, certain outliers per tile, uncertain keys) and encodes
+// speculatively: a chunk with r > t_hi (above every possible threshold) as an
+// outlier (index 0, radius 0), every other chunk as a bulk chunk; records per
+// packing group the chunks with r > t_lo.
+// LIST_FIX (after the exact threshold): for each recorded chunk, decides
+// r > thr, writes the ordered list and zeroes the codes of the outliers with
+// r <= t_hi; a head whose window missed gets the full list + encode pass.
 // Work: warp tiles of TILE_GROUPS consecutive packing groups; a CTA owns a
 // contiguous range of tiles and walks it slab by slab (one head at a time).
+constexpr int LIST_SPEC = 3;
+constexpr int LIST_FIX = 4;
+
+// Clears the b-bit index of lane `lane` in its packing group's words.
+__device__ __forceinline__ void clear_index(uint32_t *gw, uint32_t b, int lane) {
+    const uint32_t bit = b * (uint32_t)lane, w0 = bit >> 5, o = bit & 31u;
+    const uint32_t mask = (1u << b) - 1u;                // (b <= 21)
+    atomicAnd(gw + w0, ~(mask << o));
+    if (o + b > 32u) atomicAnd(gw + w0 + 1, ~(mask >> (32u - o)));
+}
+
 template <int DT, int LIST, bool ENC, int BB>
 __global__ void __launch_bounds__(ENC_THREADS, 1)
 k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32_t tiles_per_slab,
@@ -316,8 +336,9 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
              const uint4 *__restrict__ tables, const float *__restrict__ thr, int gran,
              uint32_t *__restrict__ words, uint16_t *__restrict__ radius,
              const uint32_t *__restrict__ tile_off, uint64_t cap, uint32_t *__restrict__ out_idx,
-             uint16_t *__restrict__ out_val, DevStatus *st) {
+             uint16_t *__restrict__ out_val, DevStatus *st, SpecArgs sa) {
     extern __shared__ float4 s_tab[];                    // [24 S + 1][8]: codewords, then zero
+                                                         // (LIST_SPEC: then the key stages)
     const uint32_t b = BB ? (uint32_t)BB : b_rt;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = (1u << lane) - 1u;
@@ -332,13 +353,27 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
     const uint32_t cap32 = cap < 0xFFFFFFFFull ? (uint32_t)cap : 0xFFFFFFFFu;
     int cur_head = -1;
     unsigned n_nf = 0, n_sat = 0;
+    // LIST_SPEC: this warp's stage of window keys (of head stage_h)
+    uint32_t *stage = reinterpret_cast<uint32_t *>(s_tab + (size_t)(n_words + 1) * 8) + warp * STAGE;
+    uint32_t n_stage = 0;
+    int stage_h = -1;
     for (uint32_t seg = t_begin; seg < t_end;) {
         const uint32_t slab = seg / tiles_per_slab;
         const uint32_t seg_end = min(t_end, (slab + 1) * tiles_per_slab);
         const int h = (int)(slab % (uint32_t)H);
         const float4 *cb = cb_all + (size_t)h * S;
         const uint4 *tb = tables + (size_t)h * LUT_ENTRIES;
-        if (ENC && h != cur_head) {                      // (block-uniform)
+        WinState w{};
+        if (LIST == LIST_SPEC || LIST == LIST_FIX) w = sa.win[h];
+        const bool miss = LIST == LIST_FIX && w.miss != 0;    // (block-uniform)
+        if (LIST == LIST_SPEC && h != stage_h) {
+            if (n_stage)
+                flush_stage(stage, n_stage, lane, sa.cand_n + stage_h,
+                            sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap);
+            n_stage = 0;
+            stage_h = h;
+        }
+        if (ENC && h != cur_head && (LIST != LIST_FIX || miss)) {   // (block-uniform)
             __syncthreads();
             for (uint32_t i = threadIdx.x; i < (n_words + 1) * 8; i += ENC_THREADS) {
                 const uint32_t id = i >> 3;
@@ -354,7 +389,68 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
             const uint32_t g0 = (t % tiles_per_slab) * TILE_GROUPS;
             const uint32_t g1 = min(g0 + TILE_GROUPS, groups_per_slab);
             const uint32_t gbase = slab * groups_per_slab;
-            uint32_t lpos = LIST ? __ldg(tile_off + t) : 0u;   // list position
+            uint32_t lpos = (LIST && LIST != LIST_SPEC) ? __ldg(tile_off + t) : 0u;   // list position
+            if (LIST == LIST_FIX && !miss) {
+                // the recorded chunks (r > t_lo) of this tile, in order: lane i
+                // reads group i's bits; candidate k (in tile order) goes to lane
+                // k mod 32, which finds its group by a search over the
+                // inclusive counts and its chunk as the group's n-th set bit
+                const uint32_t ng = g1 - g0;
+                const uint32_t gw = (uint32_t)lane < ng ? __ldg(sa.cbits + gbase + g0 + lane) : 0u;
+                const uint32_t pcount = __popc(gw);
+                uint32_t incl = pcount;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t v = __shfl_up_sync(FULL, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                const uint32_t total = __shfl_sync(FULL, incl, 31);
+                for (uint32_t k0 = 0; k0 < total; k0 += 32) {        // (warp-uniform)
+                    const uint32_t k = k0 + (uint32_t)lane;
+                    const bool c = k < total;
+                    uint32_t gl = 0;                                // first group with incl > k
+#pragma unroll
+                    for (int step = 16; step >= 1; step >>= 1) {
+                        const uint32_t v = __shfl_sync(FULL, incl, (int)(gl + step - 1));
+                        if (v <= k) gl += step;
+                    }
+                    gl &= 31u;
+                    const uint32_t ex = __shfl_sync(FULL, incl - pcount, (int)gl);
+                    const uint32_t word = __shfl_sync(FULL, gw, (int)gl);
+                    const uint32_t bit = c ? __fns(word, 0u, (int)(k - ex + 1)) : 0u;
+                    const uint32_t G = gbase + g0 + gl;
+                    const uint32_t j = G * 32 + bit;
+                    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f, r = 0.f;
+                    if (c) {
+                        RawChunk<DT> v;
+                        v.load(x, j);
+                        x0 = v.e(0); x1 = v.e(1); x2 = v.e(2); x3 = v.e(3);
+                        r = chunk_norm(x0, x1, x2, x3);
+                    }
+                    const bool o = c && r > th;
+                    const uint32_t mo = __ballot_sync(FULL, o);
+                    if (o) {
+                        const uint32_t p = lpos + __popc(mo & lt);
+                        if (p < cap32) {
+                            int sv = 0;
+                            const uint32_t h01 = f32x2_to_f16x2_sat(x0, x1, sv);
+                            const uint32_t h23 = f32x2_to_f16x2_sat(x2, x3, sv);
+                            n_sat += sv;
+                            out_idx[p] = j;
+                            reinterpret_cast<uint2 *>(out_val)[p] = make_uint2(h01, h23);
+                        }
+                        if (!(r > w.t_hi)) {                // encoded as a bulk chunk: zero it
+                            radius[j] = 0;
+                            clear_index(words + (size_t)G * b, b, (int)bit);
+                        }
+                    } else if (c && !(r > w.t_hi) && r >= 65520.0f) {
+                        ++n_sat;                             // bulk radius saturated (uncounted)
+                    }
+                    lpos += __popc(mo);
+                }
+                continue;
+            }
+            uint32_t t_def = 0, t_below = 0;                  // LIST_SPEC
             RawChunk<DT> nxt;
             nxt.load(x, (size_t)(gbase + g0) * 32 + lane);
             for (uint32_t g = g0; g < g1; ++g) {
@@ -364,7 +460,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 if (g + 1 < g1) nxt.load(x, (size_t)j + 32);
                 float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
                 float r = chunk_norm(x0, x1, x2, x3);
-                if (LIST == HQMQ_GRAN_CHUNK + 1) {           // ordered chunk list
+                if (LIST == HQMQ_GRAN_CHUNK + 1 || LIST == LIST_FIX) {   // ordered chunk list
                     const bool o = r > th;
                     const uint32_t m = __ballot_sync(FULL, o);
                     if (o) {
@@ -406,8 +502,46 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                     }
                     lpos += __shfl_sync(FULL, inc, 31);
                 }
+                bool spec_cand = false;                      // LIST_SPEC: r > t_lo
+                if (LIST == LIST_SPEC) {
+                    const uint32_t key = mag_key(r);
+                    t_below += key < w.lo_key ? 1u : 0u;
+                    const bool in = key >= w.lo_key && key < w.hi_key;
+                    const uint32_t mi = __ballot_sync(FULL, in);
+                    if (mi) {
+                        if (n_stage + 32 > STAGE) {
+                            flush_stage(stage, n_stage, lane, sa.cand_n + h,
+                                        sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap);
+                            n_stage = 0;
+                        }
+                        if (in) {
+                            stage[n_stage + __popc(mi & lt)] = key;
+                            atomicAdd(sa.fine_hist + (size_t)h * KEY_BINS +
+                                          ((key - w.lo_key) >> w.shift), 1u);
+                        }
+                        n_stage += __popc(mi);
+                        __syncwarp();
+                    }
+                    const bool dfn = r > w.t_hi;             // (NaN: false)
+                    spec_cand = r > w.t_lo;
+                    t_def += dfn ? 1u : 0u;
+                    const uint32_t mc = __ballot_sync(FULL, spec_cand);
+                    if (lane == 0) sa.cbits[G] = mc;
+                    const bool unc = spec_cand && !dfn;
+                    const uint32_t mu = __ballot_sync(FULL, unc);
+                    if (mu) {
+                        unsigned long long base = 0;
+                        if (lane == 0) base = atomicAdd(sa.amb_n, (unsigned long long)__popc(mu));
+                        base = __shfl_sync(FULL, base, 0);
+                        if (unc) {
+                            const unsigned long long pos = base + __popc(mu & lt);
+                            if (pos < sa.amb_cap) sa.amb[pos] = make_uint2(t, key);
+                        }
+                    }
+                    if (dfn) r = 0.0f;                       // certain outlier: radius 0, index 0
+                }
                 if (!ENC) continue;
-                if (med3) {
+                if (med3 && LIST != LIST_SPEC) {
                     if (gran == HQMQ_GRAN_CHUNK) {
                         if (r > th) r = 0.0f;        // outlier chunk: no search, radius 0
                     } else {
@@ -468,13 +602,45 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 } else {
                     int sat = 0;
                     rh = radius_to_f16(r, sat);
-                    n_sat += sat;
+                    if (!spec_cand) n_sat += sat;            // (LIST_FIX decides the others)
                 }
                 radius[j] = rh;
                 pack_group32<BB>(idx, b, lane, pc, words + (size_t)G * b);
             }
+            if (LIST == LIST_SPEC) {
+                t_def = __reduce_add_sync(FULL, t_def);
+                t_below = __reduce_add_sync(FULL, t_below);
+                if (lane == 0) {
+                    sa.tile_cnt[t] = t_def;
+                    if (t_below) atomicAdd(sa.below + h, (unsigned long long)t_below);
+                }
+            }
+        }
+        if (LIST == LIST_SPEC) {                             // status counts per head
+            const unsigned nf = __reduce_add_sync(FULL, n_nf);
+            const unsigned ns = __reduce_add_sync(FULL, n_sat);
+            if (lane == 0 && (nf | ns)) {
+                atomicAdd(sa.head_stat + 2 * h, (unsigned long long)nf);
+                atomicAdd(sa.head_stat + 2 * h + 1, (unsigned long long)ns);
+            }
+            n_nf = n_sat = 0;
         }
         seg = seg_end;
+    }
+    if (LIST == LIST_SPEC) {
+        if (n_stage)
+            flush_stage(stage, n_stage, lane, sa.cand_n + stage_h,
+                        sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap);
+        return;
+    }
+    if (LIST == LIST_FIX && blockIdx.x == 0 && st) {
+        // the encode pass's status counts of the heads whose result stands
+        for (int hh = threadIdx.x; hh < H; hh += ENC_THREADS)
+            if (!sa.win[hh].miss) {
+                const unsigned long long nf = sa.head_stat[2 * hh], ns = sa.head_stat[2 * hh + 1];
+                status_add(st, HQMQ_FLAG_NONFINITE, &st->n_nonfinite, nf);
+                status_add(st, HQMQ_FLAG_SATURATED, &st->n_saturated, ns);
+            }
     }
     const unsigned nf = __reduce_add_sync(FULL, n_nf);
     const unsigned ns = __reduce_add_sync(FULL, n_sat);
@@ -514,11 +680,12 @@ static int launch_lut_bb(int B, int H, int T, int D, const void *x, const float 
                          uint32_t b, const void *table, const float *thr, int gran,
                          uint32_t *words, uint16_t *radius, const uint32_t *tile_off, uint64_t cap,
                          uint32_t *out_idx, uint16_t *out_val, hqmq_status *st, int sm_count,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const SpecArgs &sa) {
     const uint32_t gps = (uint32_t)(((uint64_t)T * D / 4) / 32);
     const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
     const uint32_t n_tiles = (uint32_t)((uint64_t)B * H * tps);
-    const size_t smem = ENC ? enc_smem_bytes(S) : 0;
+    const size_t smem = (ENC ? enc_smem_bytes(S) : 0) +
+                        (LIST == LIST_SPEC ? (size_t)(ENC_THREADS / 32) * STAGE * 4 : 0);
     auto kern = k_encode_lut<DT, LIST, ENC, BB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
@@ -531,7 +698,7 @@ static int launch_lut_bb(int B, int H, int T, int D, const void *x, const float 
     kern<<<(unsigned)ctas, ENC_THREADS, smem, stream>>>(
         x, H, gps, tps, n_tiles, reinterpret_cast<const float4 *>(cb), S, b,
         reinterpret_cast<const uint4 *>(table), thr, gran, words, radius, tile_off, cap, out_idx,
-        out_val, reinterpret_cast<DevStatus *>(st));
+        out_val, reinterpret_cast<DevStatus *>(st), sa);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
@@ -541,18 +708,19 @@ template <int DT, int LIST, bool ENC>
 static int launch_lut(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
                       uint32_t b, const void *table, const float *thr, int gran, uint32_t *words,
                       uint16_t *radius, const uint32_t *tile_off, uint64_t cap, uint32_t *out_idx,
-                      uint16_t *out_val, hqmq_status *st, int sm_count, cudaStream_t stream) {
+                      uint16_t *out_val, hqmq_status *st, int sm_count, cudaStream_t stream,
+                      const SpecArgs &sa) {
     if (ENC && b == 8)
         return launch_lut_bb<DT, LIST, ENC, 8>(B, H, T, D, x, cb, S, b, table, thr, gran, words,
                                                radius, tile_off, cap, out_idx, out_val, st,
-                                               sm_count, stream);
+                                               sm_count, stream, sa);
     if (ENC && b == 10)
         return launch_lut_bb<DT, LIST, ENC, 10>(B, H, T, D, x, cb, S, b, table, thr, gran, words,
                                                 radius, tile_off, cap, out_idx, out_val, st,
-                                                sm_count, stream);
+                                                sm_count, stream, sa);
     return launch_lut_bb<DT, LIST, ENC, 0>(B, H, T, D, x, cb, S, b, table, thr, gran, words,
                                            radius, tile_off, cap, out_idx, out_val, st, sm_count,
-                                           stream);
+                                           stream, sa);
 }
 
 template <int LIST, bool ENC>
@@ -560,13 +728,13 @@ static int launch_lut_dt(int dtype, int B, int H, int T, int D, const void *x, c
                          uint32_t S, uint32_t b, const void *table, const float *thr, int gran,
                          uint32_t *words, uint16_t *radius, const uint32_t *tile_off, uint64_t cap,
                          uint32_t *out_idx, uint16_t *out_val, hqmq_status *st, int sm,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const SpecArgs &sa = SpecArgs{}) {
     if (dtype == HQMQ_BF16)
         return launch_lut<HQMQ_BF16, LIST, ENC>(B, H, T, D, x, cb, S, b, table, thr, gran, words,
                                                 radius, tile_off, cap, out_idx, out_val, st, sm,
-                                                stream);
+                                                stream, sa);
     return launch_lut<HQMQ_F32, LIST, ENC>(B, H, T, D, x, cb, S, b, table, thr, gran, words, radius,
-                                           tile_off, cap, out_idx, out_val, st, sm, stream);
+                                           tile_off, cap, out_idx, out_val, st, sm, stream, sa);
 }
 
 }  // namespace hqmq
@@ -607,4 +775,32 @@ extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int
                                                             thr, gran, words, radius, tile_off,
                                                             cap, out_idx, out_val, st, sm_count,
                                                             stream);
+}
+
+// One-read chunk-mode Med3x, step B + speculative encode (after A + W).
+extern "C" int hqmq_launch_spec_encode(const void *x, int dtype, int B, int H, int T, int D,
+                                       const float *cb, uint32_t S, uint32_t b, const void *table,
+                                       uint32_t *words, uint16_t *radius, void *ws, int sm_count,
+                                       cudaStream_t stream) {
+    using namespace hqmq;
+    const SpecArgs sa = spec_args(reinterpret_cast<char *>(ws),
+                                  fused_layout(B, H, T, D, HQMQ_GRAN_CHUNK));
+    return launch_lut_dt<LIST_SPEC, true>(dtype, B, H, T, D, x, cb, S, b, table, nullptr,
+                                          HQMQ_GRAN_CHUNK, words, radius, nullptr, 0, nullptr,
+                                          nullptr, nullptr, sm_count, stream, sa);
+}
+
+// One-read chunk-mode Med3x, the list and the code fix-ups (after F + X + U + S).
+extern "C" int hqmq_launch_fix_pass(const void *x, int dtype, int B, int H, int T, int D,
+                                    const float *cb, uint32_t S, uint32_t b, const void *table,
+                                    const float *thr, uint32_t *words, uint16_t *radius,
+                                    const uint32_t *tile_off, uint64_t cap, uint32_t *out_idx,
+                                    uint16_t *out_val, void *ws, hqmq_status *st, int sm_count,
+                                    cudaStream_t stream) {
+    using namespace hqmq;
+    const SpecArgs sa = spec_args(reinterpret_cast<char *>(ws),
+                                  fused_layout(B, H, T, D, HQMQ_GRAN_CHUNK));
+    return launch_lut_dt<LIST_FIX, true>(dtype, B, H, T, D, x, cb, S, b, table, thr,
+                                         HQMQ_GRAN_CHUNK, words, radius, tile_off, cap, out_idx,
+                                         out_val, st, sm_count, stream, sa);
 }

@@ -1,6 +1,8 @@
-"""Med3x in two reads (hqmq_outlier_extract's window pipeline and the fused
-hqmq_encode_med3) against the oracle, including inputs built to defeat the
-sample window (so the exact fallback decides) and to overflow its buffers."""
+"""Med3x against the oracle: hqmq_outlier_extract's window pipeline (two reads
+of x) and the fused hqmq_encode_med3 (one read of x in chunk mode with search
+tables: speculative encode plus fix-up pass; two reads otherwise), including
+inputs built to defeat the sample window (so the exact fallback decides) and
+to overflow its buffers, and the status counts of the fused call."""
 import numpy as np
 import pytest
 import torch
@@ -149,3 +151,71 @@ def test_fused_equals_separate_calls_full_size_70b(oracle):
     x = W.as_numpy_bits(xd)
     rmed_o, thr_o = oracle.med3_threshold(x, w.C, 0)
     assert same_f32(to_host(thr), thr_o).all()
+
+
+def expected_status(oracle, x_np, cb, S, gran, cap):
+    """The oracle's status of Med3x + encode: outliers, list and radius
+    saturations, non-finite chunks, and the flags they raise."""
+    _, thr_o = oracle.med3_threshold(x_np, 3.0, gran)
+    _, _, _, n_o, st_x = oracle.extract(x_np, thr_o, gran=gran, cap=cap)
+    *_, st_e = oracle.encode(x_np, cb, S, thr=thr_o, gran=gran)
+    return {"n_outliers": n_o, "n_saturated": st_x["n_saturated"] + st_e["n_saturated"],
+            "n_nonfinite": st_e["n_nonfinite"], "flags": st_x["flags"] | st_e["flags"]}
+
+
+def status_mix_input(rng, T=512):
+    """fp32 (1, 2, T, 128): head 0 with a median chunk norm near 40000 (bulk
+    radii above 65504 saturate, outlier values above 65504 saturate in the
+    list) and a dense band of norms around 3x the median; head 1 N(0, 1)
+    with NaN and inf chunks and planted outliers."""
+    x = rng.standard_normal((1, 2, T, 128)).astype(np.float32)
+    c = x.reshape(1, 2, -1, 4)
+    n = c.shape[2]
+    u = c[0, 0] / np.linalg.norm(c[0, 0], axis=1, keepdims=True)
+    r = np.full(n, 40000.0) * (1 + 0.3 * rng.standard_normal(n))
+    band = rng.random(n) < 0.05
+    r[band] = np.median(r) * rng.uniform(2.95, 3.05, band.sum())
+    big = rng.random(n) < 0.01
+    r[big] = 1e6
+    c[0, 0] = u * np.abs(r)[:, None]
+    k = rng.choice(n, 12, replace=False)
+    c[0, 1, k[:4], 1] = np.nan
+    c[0, 1, k[4:8], 2] = np.inf
+    c[0, 1, k[8:], :] *= 50.0
+    return x
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_fused_status_counts_match_the_oracle(oracle, seed):
+    x = status_mix_input(np.random.default_rng(40 + seed))
+    B, H, T, D = x.shape
+    cb = oracle.make_codebook(seed + 3, 8, H)
+    g = check_fused(oracle, x, 8, 0, True, seed=seed + 3)
+    want = expected_status(oracle, x, cb, 8, 0, g["cap"])
+    got = g["status"]
+    assert not got["flags"] & hqmq.FLAG_MED3_FALLBACK
+    assert got["n_saturated"] > 0 and got["n_nonfinite"] == 4
+    for k in ("n_outliers", "n_saturated", "n_nonfinite"):
+        assert got[k] == want[k], (k, got, want)
+    assert got["flags"] & ~hqmq.FLAG_MED3_FALLBACK == want["flags"]
+
+
+def test_fused_status_counts_after_a_window_miss(oracle):
+    # the sampled quads made huge (see test_window_miss_takes_the_exact_fallback)
+    # plus non-finite and saturating chunks: the fallback head's status must
+    # come from the exact re-encode only
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((1, 2, 512, 128)).astype(np.float32)
+    c = x.reshape(1, 2, -1, 4)
+    pos = np.arange(c.shape[2])
+    sampled = (pos % 128) // 4 == (37 * (pos // 128)) % 32
+    c[:, :, sampled] *= 1000.0
+    c[0, 0, 5, 0] = np.nan
+    c[0, 1, 9, 3] = np.inf
+    c[0, 0, 700] = 3e4
+    cb = oracle.make_codebook(2, 8, 2)
+    g = check_fused(oracle, x, 8, 0, True, seed=2)
+    assert g["status"]["flags"] & hqmq.FLAG_MED3_FALLBACK
+    want = expected_status(oracle, x, cb, 8, 0, g["cap"])
+    for k in ("n_outliers", "n_saturated", "n_nonfinite"):
+        assert g["status"][k] == want[k], (k, g["status"], want)
