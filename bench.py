@@ -173,6 +173,10 @@ class Cache:
             self.out_idx = torch.empty((w.layers, 2, self.cap), dtype=torch.int32, device=device)
             self.out_val = torch.empty((w.layers, 2, self.cap * 4), dtype=torch.int16, device=device)
             self.slab_off = torch.empty((w.layers, 2, B * H + 1), dtype=torch.int32, device=device)
+            # list tile offsets (rows padded to 16 bytes: the library stores them as uint4)
+            self.n_tiles = hqmq.hqmq_list_tiles(B, H, T, D)
+            self.tile_off = torch.empty((w.layers, 2, (self.n_tiles + 4) // 4 * 4),
+                                        dtype=torch.int32, device=device)
             self.ws = torch.empty(hqmq.hqmq_encode_med3_workspace_size(B, H, T, D, self.gran),
                                   dtype=torch.uint8, device=device)
 
@@ -201,7 +205,7 @@ class Cache:
     def kernels_per_step(self):
         if self.w.med3:
             enc = KERNELS_MED3_ENCODE + (0 if self.table is not None else 1)
-            dec = 2                        # main pass + outlier pass
+            dec = 1                        # the list is applied in the main pass (tile offsets)
         else:
             enc, dec = 1, 1
         return self.w.n_calls * (enc + dec)
@@ -237,7 +241,7 @@ class Cache:
                                           self.radius[l, r], self.rmed[l, r], self.thr[l, r],
                                           self.out_idx[l, r], self.out_val[l, r],
                                           self.slab_off[l, r], self.cap, self.ws, self.status,
-                                          stream)
+                                          stream, tile_off=self.tile_off[l, r])
                 elif self.table is not None:
                     hqmq.hqmq_encode_lut(x, cb, w.S, tb, thr, self.gran, self.words[l, r],
                                          self.radius[l, r], self.status, stream)
@@ -248,7 +252,8 @@ class Cache:
                 if w.med3:
                     hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S,
                                      self.out_idx[l, r], self.out_val[l, r], self.slab_off[l, r],
-                                     self.cap, self.gran, self.y, self.status, stream)
+                                     self.cap, self.gran, self.y, self.status, stream,
+                                     tile_off=self.tile_off[l, r])
                 else:
                     hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S, None, None,
                                      None, 0, self.gran, self.y, self.status, stream)
@@ -440,6 +445,8 @@ def run_e2e(cache, args, dist, device):
     if w.med3:
         host_oi = torch.empty(cache.cap, dtype=torch.int32, pin_memory=True)
         host_ov = torch.empty(cache.cap * 4, dtype=torch.int16, pin_memory=True)
+        host_off = torch.empty(cache.slab_off.shape[-1] + cache.tile_off.shape[-1],
+                               dtype=torch.int32, pin_memory=True)
     xbuf = torch.empty(cache.shape, dtype=w.torch_dtype, device=device)
     h2d = d2h = 0
 
@@ -462,7 +469,10 @@ def run_e2e(cache, args, dist, device):
                 if w.med3:
                     host_oi.copy_(cache.out_idx[l, r], non_blocking=True)
                     host_ov.copy_(cache.out_val[l, r], non_blocking=True)
-                    d2h += cache.cap * 4 + cache.cap * 8
+                    ns, nt = cache.slab_off.shape[-1], cache.tile_off.shape[-1]
+                    host_off[:ns].copy_(cache.slab_off[l, r], non_blocking=True)
+                    host_off[ns:].copy_(cache.tile_off[l, r], non_blocking=True)
+                    d2h += cache.cap * 4 + cache.cap * 8 + (ns + nt) * 4
 
     steps = max(1, min(args.steps, 3))
     one_step()

@@ -121,8 +121,9 @@ HQMQ_API int hqmq_make_codebook(uint64_t seed, uint32_t S, uint32_t n_groups, ui
 
 /* Bytes of device workspace hqmq_outlier_extract (and hqmq_encode_med3) needs
  * for this shape: two 64 Ki-bin histograms per head, the keys of the median
- * window, the uncertain-threshold list and per-tile counts (about 10 MB for
- * a 1 x 8 x 131072 x 128 call). */
+ * window, the uncertain-threshold list, per-tile counts and offsets and one
+ * candidate bit per chunk (about 31 MB for a 1 x 8 x 131072 x 128 call in
+ * chunk mode). */
 HQMQ_API uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gran);
 
 /* Med3x (gist.science/nl, Technische Samenvatting, section 3; the pages
@@ -140,9 +141,14 @@ HQMQ_API uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gr
  *   element mode: d_out_idx[n] = element index, d_out_val[n] = fp16 bits;
  *   fp16 = round-to-nearest-even, finite values beyond +-65504 saturate.
  * d_slab_off[B*H+1]: entries of slab (b,h) are [slab_off[b*H+h], slab_off[b*H+h+1]).
- * Entries at positions >= cap are not written (d_slab_off still holds the
- * full offsets); the status then gets HQMQ_FLAG_OUTLIER_OVERFLOW and
- * n_outliers the required total, so the caller can retry with a larger cap.
+ * d_tile_off (NULL = not wanted): uint32[hqmq_list_tiles(B,H,T,D) + 1],
+ * 16-byte aligned: the list position of the first entry of each list tile
+ * (1024 consecutive chunks of a slab; a slab's last tile may be shorter),
+ * then the total.  hqmq_decode uses it to apply the list in its main pass.
+ * Entries at positions >= cap are not written (d_slab_off and d_tile_off
+ * still hold the full offsets); the status then gets
+ * HQMQ_FLAG_OUTLIER_OVERFLOW and n_outliers the required total, so the
+ * caller can retry with a larger cap.
  * Data flow (two reads of x): a 1/32 sample fixes per head a key window that
  * holds the median rank with overwhelming probability; one full read counts
  * the keys below the window, keeps the keys inside it and counts per
@@ -158,8 +164,13 @@ HQMQ_API uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gr
  * B*H*T*D must be < 2^32. */
 HQMQ_API int hqmq_outlier_extract(const void *d_x, int dtype, int B, int H, int T, int D, float C,
                          int gran, float *d_rmed, float *d_thr, uint32_t *d_out_idx,
-                         uint16_t *d_out_val, uint32_t *d_slab_off, uint64_t cap, void *d_ws,
-                         uint64_t ws_bytes, hqmq_status *d_status, void *stream);
+                         uint16_t *d_out_val, uint32_t *d_slab_off, uint32_t *d_tile_off,
+                         uint64_t cap, void *d_ws, uint64_t ws_bytes, hqmq_status *d_status,
+                         void *stream);
+
+/* Number of list tiles of a call (the length of d_tile_off minus one), or 0
+ * for a shape the library rejects. */
+HQMQ_API uint64_t hqmq_list_tiles(int B, int H, int T, int D);
 
 /* Encode (gist.science/nl, Technische Samenvatting, Methodologie and
  * section 1): per chunk j
@@ -187,12 +198,17 @@ HQMQ_API int hqmq_encode(const void *d_x, int dtype, int B, int H, int T, int D,
  * value); element mode gives round(fl32(fl32(r * c_i) + value)).  An index
  * >= 24 S decodes to 0 and sets HQMQ_FLAG_BAD_INDEX.
  * d_idx_words and d_radius as written by hqmq_encode; d_y: [B][H][T][D]
- * of out_dtype, 16-byte aligned.  With a list, a second kernel applies the
- * outliers after the main pass on the same stream. */
+ * of out_dtype, 16-byte aligned.  With a list and its d_tile_off (as written
+ * by hqmq_outlier_extract / hqmq_encode_med3), the main pass applies each
+ * tile's entries right after writing the tile; entries whose index lies
+ * outside their tile are ignored.  With a list and d_tile_off == NULL, a
+ * second kernel applies the outliers after the main pass on the same stream
+ * (entries outside the tensor are ignored). */
 HQMQ_API int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, const float *d_codebook,
                 uint32_t S, const uint32_t *d_out_idx, const uint16_t *d_out_val,
-                const uint32_t *d_slab_off, uint64_t cap, int gran, int B, int H, int T, int D,
-                void *d_y, int out_dtype, hqmq_status *d_status, void *stream);
+                const uint32_t *d_slab_off, const uint32_t *d_tile_off, uint64_t cap, int gran,
+                int B, int H, int T, int D, void *d_y, int out_dtype, hqmq_status *d_status,
+                void *stream);
 
 /* Exact table-driven search (same results as hqmq_encode; the argmax of
  * <x, c> over the 24 S codewords c = q_p q_s, ties to the lowest index:
@@ -232,19 +248,26 @@ HQMQ_API int hqmq_encode_lut(const void *d_x, int dtype, int B, int H, int T, in
                              const float *d_thr, int gran, uint32_t *d_idx_words,
                              uint16_t *d_radius, hqmq_status *d_status, void *stream);
 
-/* Med3x and encode in two reads of x: hqmq_outlier_extract's median and tile
- * counts (first read), then one pass that writes the ordered outlier list and
- * encodes the zeroed chunks with the search tables (second read).  Outputs
- * equal hqmq_outlier_extract followed by hqmq_encode_lut (or hqmq_encode when
- * d_table is NULL, which costs a third read).  Workspace as
+/* Med3x and encode in one call.  Outputs equal hqmq_outlier_extract followed
+ * by hqmq_encode_lut (or hqmq_encode when d_table is NULL), bit for bit, and
+ * the status counts equal theirs.
+ * Chunk mode with search tables reads x once: the encode pass runs before the
+ * exact threshold is known, encoding a chunk above the largest threshold the
+ * sample window allows as an outlier and every other chunk as a bulk chunk,
+ * and marks the chunks above the smallest such threshold; after the exact
+ * threshold a fix-up pass reads only the marked chunks, writes the ordered
+ * list and zeroes the codes of the marked chunks that are outliers.  A head
+ * whose window missed gets a full exact re-encode.  Element mode (whose
+ * encode depends on the threshold) reads x twice: once for the median, once
+ * for the list and the encode (a third read without d_table).  Workspace as
  * hqmq_outlier_workspace_size; other arguments as in those calls. */
 HQMQ_API uint64_t hqmq_encode_med3_workspace_size(int B, int H, int T, int D, int gran);
 HQMQ_API int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, float C,
                               int gran, const float *d_codebook, uint32_t S, const void *d_table,
                               uint32_t *d_idx_words, uint16_t *d_radius, float *d_rmed,
                               float *d_thr, uint32_t *d_out_idx, uint16_t *d_out_val,
-                              uint32_t *d_slab_off, uint64_t cap, void *d_ws, uint64_t ws_bytes,
-                              hqmq_status *d_status, void *stream);
+                              uint32_t *d_slab_off, uint32_t *d_tile_off, uint64_t cap,
+                              void *d_ws, uint64_t ws_bytes, hqmq_status *d_status, void *stream);
 
 /* Size of the fixed device scratch array of hqmq_outlier_extract_noalloc. */
 #define HQMQ_NOALLOC_SCRATCH_BYTES (1u << 20)
@@ -267,7 +290,8 @@ HQMQ_API int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, i
  * share the one array: calls whose execution overlaps on the GPU (different
  * streams without ordering between them) race and give wrong results.  Each
  * call clears what must start at zero.  Nothing is allocated or freed.
- * Arguments, results and errors are otherwise those of hqmq_outlier_extract. */
+ * Arguments, results and errors are otherwise those of hqmq_outlier_extract
+ * (it writes no tile offsets). */
 HQMQ_API int hqmq_outlier_extract_noalloc(const void *d_x, int dtype, int B, int H, int T, int D,
                                           float C, int gran, float *d_rmed, float *d_thr,
                                           uint32_t *d_out_idx, uint16_t *d_out_val,

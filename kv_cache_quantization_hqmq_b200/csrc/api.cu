@@ -15,7 +15,7 @@ extern "C" int hqmq_launch_encode(const void *x, int dtype, int B, int H, int T,
                                   int sm_count, cudaStream_t stream);
 extern "C" int hqmq_launch_decode(const uint32_t *words, const uint16_t *radius, const float *cb,
                                   uint32_t S, uint32_t b, const uint32_t *out_idx,
-                                  const uint16_t *out_val, const uint32_t *slab_off, uint64_t cap,
+                                  const uint16_t *out_val, const uint32_t *slab_off, const uint32_t *tile_off, uint64_t cap,
                                   int gran, int B, int H, int T, int D, void *y, int out_dtype,
                                   hqmq_status *st, int sm_count, cudaStream_t stream);
 extern "C" uint64_t hqmq_med3_workspace_bytes(int B, int H, int T, int D);
@@ -28,16 +28,18 @@ extern "C" int hqmq_launch_outlier_extract(const void *x, int dtype, int B, int 
 extern "C" uint64_t hqmq_window_workspace_bytes(int B, int H, int T, int D, int gran);
 extern "C" int hqmq_launch_med3_window(const void *x, int dtype, int B, int H, int T, int D,
                                        float C, int gran, float *rmed, float *thr,
-                                       uint32_t *slab_off, uint64_t cap, void *ws,
-                                       hqmq_status *st, int sm_count, cudaStream_t stream,
-                                       const uint32_t **tile_off, uint32_t *tiles_per_slab);
+                                       uint32_t *slab_off, uint32_t *tile_off_out, uint64_t cap,
+                                       void *ws, hqmq_status *st, int sm_count,
+                                       cudaStream_t stream, const uint32_t **tile_off,
+                                       uint32_t *tiles_per_slab);
+extern "C" uint64_t hqmq_list_tile_count(int B, int H, int T, int D);
 extern "C" int hqmq_launch_med3_front(const void *x, int dtype, int B, int H, int T, int D,
                                       float C, int gran, void *ws, int pass_b, int sm_count,
                                       cudaStream_t stream);
 extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, int T, int D,
                                        float C, int gran, float *rmed, float *thr,
-                                       uint32_t *slab_off, uint64_t cap, void *ws,
-                                       hqmq_status *st, cudaStream_t stream,
+                                       uint32_t *slab_off, uint32_t *tile_off_out, uint64_t cap,
+                                       void *ws, hqmq_status *st, cudaStream_t stream,
                                        const uint32_t **tile_off, uint32_t *tiles_per_slab);
 extern "C" int hqmq_launch_spec_encode(const void *x, int dtype, int B, int H, int T, int D,
                                        const float *cb, uint32_t S, uint32_t b, const void *table,
@@ -147,15 +149,16 @@ uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gran) {
 
 int hqmq_outlier_extract(const void *d_x, int dtype, int B, int H, int T, int D, float C,
                          int gran, float *d_rmed, float *d_thr, uint32_t *d_out_idx,
-                         uint16_t *d_out_val, uint32_t *d_slab_off, uint64_t cap, void *d_ws,
-                         uint64_t ws_bytes, hqmq_status *d_status, void *stream) {
+                         uint16_t *d_out_val, uint32_t *d_slab_off, uint32_t *d_tile_off,
+                         uint64_t cap, void *d_ws, uint64_t ws_bytes, hqmq_status *d_status,
+                         void *stream) {
     if (!shape_ok(B, H, T, D) || !dtype_ok(dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
     if (!(C > 0.0f) || !(C < 3.0e38f)) return HQMQ_ERR_ARG;
     if (!d_x || !d_rmed || !d_thr || !d_slab_off || !d_ws) return HQMQ_ERR_ARG;
     if (cap > 0 && (!d_out_idx || !d_out_val)) return HQMQ_ERR_ARG;
     if (!aligned(d_x, 16) || !aligned(d_rmed, 4) || !aligned(d_thr, 4) ||
-        !aligned(d_slab_off, 4) || !aligned(d_ws, 256) || !aligned(d_out_idx, 4) ||
-        !aligned(d_out_val, 4) || !aligned(d_status, 8))
+        !aligned(d_slab_off, 4) || !aligned(d_tile_off, 16) || !aligned(d_ws, 256) ||
+        !aligned(d_out_idx, 4) || !aligned(d_out_val, 4) || !aligned(d_status, 8))
         return HQMQ_ERR_ALIGN;
     if (ws_bytes < hqmq_window_workspace_bytes(B, H, T, D, gran)) return HQMQ_ERR_WORKSPACE;
     int sm = sm_count();
@@ -163,8 +166,8 @@ int hqmq_outlier_extract(const void *d_x, int dtype, int B, int H, int T, int D,
     const uint32_t *tile_off = nullptr;
     uint32_t tps = 0;
     int rc = hqmq_launch_med3_window(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_slab_off,
-                                     cap, d_ws, d_status, sm, (cudaStream_t)stream, &tile_off,
-                                     &tps);
+                                     d_tile_off, cap, d_ws, d_status, sm, (cudaStream_t)stream,
+                                     &tile_off, &tps);
     if (rc != HQMQ_OK) return rc;
     return hqmq_launch_list_pass(d_x, dtype, B, H, T, D, nullptr, 1, 5, nullptr, d_thr, gran,
                                  nullptr, nullptr, tile_off, cap, d_out_idx, d_out_val, d_status,
@@ -178,8 +181,9 @@ uint64_t hqmq_encode_med3_workspace_size(int B, int H, int T, int D, int gran) {
 int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, float C, int gran,
                      const float *d_codebook, uint32_t S, const void *d_table,
                      uint32_t *d_idx_words, uint16_t *d_radius, float *d_rmed, float *d_thr,
-                     uint32_t *d_out_idx, uint16_t *d_out_val, uint32_t *d_slab_off, uint64_t cap,
-                     void *d_ws, uint64_t ws_bytes, hqmq_status *d_status, void *stream) {
+                     uint32_t *d_out_idx, uint16_t *d_out_val, uint32_t *d_slab_off,
+                     uint32_t *d_tile_off, uint64_t cap, void *d_ws, uint64_t ws_bytes,
+                     hqmq_status *d_status, void *stream) {
     if (!shape_ok(B, H, T, D) || !dtype_ok(dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
     if (!(C > 0.0f) || !(C < 3.0e38f)) return HQMQ_ERR_ARG;
     if (S < 1 || S > S_MAX) return HQMQ_ERR_ARG;
@@ -190,7 +194,8 @@ int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, flo
     if (cap > 0 && (!d_out_idx || !d_out_val)) return HQMQ_ERR_ARG;
     if (!aligned(d_x, 16) || !aligned(d_codebook, 16) || !aligned(d_table, 16) ||
         !aligned(d_idx_words, 4) || !aligned(d_radius, 4) || !aligned(d_rmed, 4) ||
-        !aligned(d_thr, 4) || !aligned(d_slab_off, 4) || !aligned(d_ws, 256) ||
+        !aligned(d_thr, 4) || !aligned(d_slab_off, 4) || !aligned(d_tile_off, 16) ||
+        !aligned(d_ws, 256) ||
         !aligned(d_out_idx, 4) || !aligned(d_out_val, 4) || !aligned(d_status, 8))
         return HQMQ_ERR_ALIGN;
     if (ws_bytes < hqmq_window_workspace_bytes(B, H, T, D, gran)) return HQMQ_ERR_WORKSPACE;
@@ -210,7 +215,8 @@ int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, flo
                                          d_idx_words, d_radius, d_ws, sm, s);
         if (rc == HQMQ_OK)
             rc = hqmq_launch_med3_finish(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr,
-                                         d_slab_off, cap, d_ws, d_status, s, &tile_off, &tps);
+                                         d_slab_off, d_tile_off, cap, d_ws, d_status, s,
+                                         &tile_off, &tps);
         if (rc == HQMQ_OK)
             rc = hqmq_launch_fix_pass(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table, d_thr,
                                       d_idx_words, d_radius, tile_off, cap, d_out_idx, d_out_val,
@@ -218,7 +224,7 @@ int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, flo
         return rc;
     }
     int rc = hqmq_launch_med3_window(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_slab_off,
-                                     cap, d_ws, d_status, sm, s, &tile_off, &tps);
+                                     d_tile_off, cap, d_ws, d_status, sm, s, &tile_off, &tps);
     if (rc != HQMQ_OK) return rc;
     if (d_table)   // list and encode in the same (second) read of x
         return hqmq_launch_list_pass(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table, d_thr,
@@ -249,24 +255,30 @@ int hqmq_encode(const void *d_x, int dtype, int B, int H, int T, int D, const fl
 
 int hqmq_decode(const uint32_t *d_idx_words, const uint16_t *d_radius, const float *d_codebook,
                 uint32_t S, const uint32_t *d_out_idx, const uint16_t *d_out_val,
-                const uint32_t *d_slab_off, uint64_t cap, int gran, int B, int H, int T, int D,
-                void *d_y, int out_dtype, hqmq_status *d_status, void *stream) {
+                const uint32_t *d_slab_off, const uint32_t *d_tile_off, uint64_t cap, int gran,
+                int B, int H, int T, int D, void *d_y, int out_dtype, hqmq_status *d_status,
+                void *stream) {
     if (!shape_ok(B, H, T, D) || !dtype_ok(out_dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
     if (S < 1 || S > S_MAX) return HQMQ_ERR_ARG;
     if (!d_idx_words || !d_radius || !d_codebook || !d_y) return HQMQ_ERR_ARG;
     if (d_out_idx && (!d_out_val || !d_slab_off)) return HQMQ_ERR_ARG;
     if (!aligned(d_idx_words, 4) || !aligned(d_radius, 4) || !aligned(d_codebook, 16) ||
         !aligned(d_y, 16) || !aligned(d_out_idx, 4) || !aligned(d_out_val, 4) ||
-        !aligned(d_slab_off, 4) || !aligned(d_status, 8))
+        !aligned(d_slab_off, 4) || !aligned(d_tile_off, 4) || !aligned(d_status, 8))
         return HQMQ_ERR_ALIGN;
     int sm = sm_count();
     if (sm <= 0) return HQMQ_ERR_CUDA;
     return hqmq_launch_decode(d_idx_words, d_radius, d_codebook, S, hqmq_index_bits(S), d_out_idx,
-                              d_out_val, d_slab_off, cap, gran, B, H, T, D, d_y, out_dtype,
-                              d_status, sm, (cudaStream_t)stream);
+                              d_out_val, d_slab_off, d_out_idx ? d_tile_off : nullptr, cap, gran,
+                              B, H, T, D, d_y, out_dtype, d_status, sm, (cudaStream_t)stream);
 }
 
 uint64_t hqmq_search_table_bytes(uint32_t S) { return hqmq_lut_bytes_per_group(S); }
+
+uint64_t hqmq_list_tiles(int B, int H, int T, int D) {
+    if (!shape_ok(B, H, T, D)) return 0;
+    return hqmq_list_tile_count(B, H, T, D);
+}
 
 int hqmq_make_search_table(const float *d_codebook, uint32_t S, uint32_t n_groups,
                            void *d_table, void *stream) {

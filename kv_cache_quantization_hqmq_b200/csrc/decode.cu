@@ -6,16 +6,19 @@
 // inside their attention kernel ("Memory en Latentie"); here it is a
 // standalone streaming kernel that writes the dense bf16 (or fp32) tensor.
 //
-// Two launches on the caller's stream:
-//  * k_decode: each CTA owns one slab (b, h), builds that head's 24 S
-//    codeword table in shared memory once (S <= 170; larger S recomputes the
-//    codeword per chunk) and streams its chunks: per chunk pair one 4-byte
-//    radius load, the index bits, 8 products and one 16-byte store; no
-//    barriers after the table build;
-//  * k_decode_outliers (only with an outlier list): one thread per list
-//    entry overwrites the chunk (chunk mode) or adds the fp16 value to the
-//    recomputed fl32(r * c) of its element (element mode).
-#include "hqmq_device.cuh"
+// k_decode: each CTA owns one slab (b, h), builds that head's 24 S codeword
+// table in shared memory once (S <= 170; larger S recomputes the codeword
+// per chunk) and streams its chunks: per chunk pair one 4-byte radius load,
+// the index bits, 8 products and one 16-byte store; no barriers after the
+// table build.  Outlier list entries overwrite their chunk (chunk mode) or
+// add the fp16 value to the recomputed fl32(r * c) of their element (element
+// mode):
+//  * with the list's tile offsets (the list position of each 1024-chunk
+//    tile's first entry), inside k_decode: the warp that wrote a 256-chunk
+//    quarter writes the entries of that quarter after a __syncwarp();
+//  * without them, in a second launch, k_decode_outliers (one thread per
+//    entry).
+#include "med3_window.cuh"
 
 namespace hqmq {
 
@@ -33,15 +36,39 @@ __device__ __forceinline__ uint32_t get_index(const uint32_t *__restrict__ words
     return (uint32_t)(v >> o) & ((1u << b) - 1u);
 }
 
+// fl32(fl32(r c_e) + v) of element e of chunk j, r and c from the chunk's
+// code (the main pass's product), v the list's fp16 value; a bad index gives
+// r = 0.
+__device__ __forceinline__ float element_with_outlier(const uint32_t *__restrict__ words,
+                                                     const uint16_t *__restrict__ radius,
+                                                     const float4 *__restrict__ cb, uint32_t S,
+                                                     uint32_t b, uint64_t j, int e, uint32_t v16) {
+    const uint32_t ix = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
+    float r = f16_bits_to_f32(__ldg(radius + j));
+    float c = 0.0f;
+    if (ix < 24u * S) {
+        const float4 cw = codeword((int)(ix % 24u), __ldg(cb + ix / 24u));
+        c = e == 0 ? cw.x : e == 1 ? cw.y : e == 2 ? cw.z : cw.w;
+    } else {
+        r = 0.0f;
+    }
+    return __fadd_rn(__fmul_rn(r, c), f16_bits_to_f32(v16));
+}
+
 // Main pass: every chunk -> round(fl32(r * c_i)).  Thread t of a warp handles
 // the chunk pairs w*PAIRS*32 + u*32 + t (u < PAIRS): each load and each
 // 16-byte store instruction of the warp is contiguous, and PAIRS pairs of
 // loads are in flight per thread.
-template <int OUT_DT, bool TABLE>
+// LISTED: 0 = no list here, HQMQ_GRAN_CHUNK + 1 / HQMQ_GRAN_ELEMENT + 1 =
+// apply the list of that granularity through its tile offsets.
+template <int OUT_DT, bool TABLE, int LISTED>
 __global__ void __launch_bounds__(DEC_THREADS)
 k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius,
          const float4 *__restrict__ cb_all, uint32_t S, uint32_t b, int H,
-         uint32_t chunks_per_slab, void *__restrict__ y, DevStatus *st) {
+         uint32_t chunks_per_slab, void *__restrict__ y, DevStatus *st,
+         const uint32_t *__restrict__ tile_off, uint32_t tiles_per_slab,
+         const uint32_t *__restrict__ out_idx, const uint16_t *__restrict__ out_val,
+         uint32_t cap32) {
     extern __shared__ float4 s_tab[];              // [24 S] if TABLE
     const int slab = blockIdx.y;
     const int h = slab % H;
@@ -67,8 +94,18 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
             if (pr < pairs_per_slab) {
                 const uint64_t j = chunk0 + 2 * (uint64_t)pr;
                 rr[u] = __ldcs(reinterpret_cast<const uint32_t *>(radius) + (j >> 1));
-                idx[u][0] = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
-                idx[u][1] = get_index(words, j >> 5, (uint32_t)(j & 31u) + 1, b);
+                if (b <= 16) {                       // both indices from one 64-bit window
+                    const uint32_t *wg = words + (j >> 5) * b;
+                    const uint32_t bit = (uint32_t)(j & 31u) * b, o = bit & 31u;
+                    uint64_t v = __ldg(wg + (bit >> 5));
+                    if (o + 2 * b > 32u) v |= (uint64_t)__ldg(wg + (bit >> 5) + 1) << 32;
+                    const uint32_t mask = (1u << b) - 1u;
+                    idx[u][0] = (uint32_t)(v >> o) & mask;
+                    idx[u][1] = (uint32_t)(v >> (o + b)) & mask;
+                } else {
+                    idx[u][0] = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
+                    idx[u][1] = get_index(words, j >> 5, (uint32_t)(j & 31u) + 1, b);
+                }
             }
         }
 #pragma unroll
@@ -109,6 +146,48 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
                 float4 *yp = reinterpret_cast<float4 *>(y) + j;
                 __stcs(yp, make_float4(out[0], out[1], out[2], out[3]));
                 __stcs(yp + 1, make_float4(out[4], out[5], out[6], out[7]));
+            }
+        }
+        if (LISTED) {
+            // the list entries of this quarter [q0, q1) (chunk indices), from
+            // its tile's list range; ordered after the warp's stores above
+            __syncwarp();
+            const uint64_t q0 = chunk0 + 2 * (uint64_t)p0;
+            const uint64_t q1 = min(q0 + 2 * PAIRS * 32, chunk0 + chunks_per_slab);
+            const uint64_t gt = (uint64_t)slab * tiles_per_slab + (2 * p0) / TILE_CHUNKS;
+            const uint32_t a = __ldg(tile_off + gt);
+            uint32_t e = __ldg(tile_off + gt + 1);
+            if (e > cap32) e = cap32;
+            for (uint32_t k0 = a; k0 < e; k0 += 32) {
+                const uint32_t k = k0 + (uint32_t)lane;
+                if (k >= e) break;
+                const uint32_t qi = __ldg(out_idx + k);
+                if (LISTED == HQMQ_GRAN_CHUNK + 1) {
+                    if (qi < q0 || qi >= q1) continue;
+                    const uint32_t *vv = reinterpret_cast<const uint32_t *>(out_val + (uint64_t)k * 4);
+                    const uint32_t v01 = __ldg(vv), v23 = __ldg(vv + 1);
+                    const float f0 = f16_bits_to_f32(v01 & 0xFFFFu), f1 = f16_bits_to_f32(v01 >> 16);
+                    const float f2 = f16_bits_to_f32(v23 & 0xFFFFu), f3 = f16_bits_to_f32(v23 >> 16);
+                    if (OUT_DT == HQMQ_BF16) {
+                        __nv_bfloat162 a0 = __floats2bfloat162_rn(f0, f1);
+                        __nv_bfloat162 a1 = __floats2bfloat162_rn(f2, f3);
+                        uint2 o;
+                        o.x = *reinterpret_cast<uint32_t *>(&a0);
+                        o.y = *reinterpret_cast<uint32_t *>(&a1);
+                        reinterpret_cast<uint2 *>(y)[qi] = o;
+                    } else {
+                        reinterpret_cast<float4 *>(y)[qi] = make_float4(f0, f1, f2, f3);
+                    }
+                } else {
+                    const uint64_t jq = qi >> 2;
+                    if (jq < q0 || jq >= q1) continue;
+                    const float val = element_with_outlier(words, radius, cb, S, b, jq,
+                                                           (int)(qi & 3u), __ldg(out_val + k));
+                    if (OUT_DT == HQMQ_BF16)
+                        reinterpret_cast<__nv_bfloat16 *>(y)[qi] = __float2bfloat16_rn(val);
+                    else
+                        reinterpret_cast<float *>(y)[qi] = val;
+                }
             }
         }
     }
@@ -185,11 +264,12 @@ k_decode_outliers(const uint32_t *__restrict__ words, const uint16_t *__restrict
     }
 }
 
-template <int OUT_DT, bool TABLE>
+template <int OUT_DT, bool TABLE, int LISTED>
 static int launch_main(const uint32_t *words, const uint16_t *radius, const float *cb, uint32_t S,
                        uint32_t b, int B, int H, uint32_t cps, void *y, hqmq_status *st,
-                       int sm_count, cudaStream_t stream) {
-    auto kern = k_decode<OUT_DT, TABLE>;
+                       const uint32_t *tile_off, const uint32_t *out_idx, const uint16_t *out_val,
+                       uint64_t cap, int sm_count, cudaStream_t stream) {
+    auto kern = k_decode<OUT_DT, TABLE, LISTED>;
     size_t smem = TABLE ? (size_t)24 * S * sizeof(float4) : 0;
     if (smem > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -206,10 +286,30 @@ static int launch_main(const uint32_t *words, const uint16_t *radius, const floa
     const uint64_t fill = ((uint64_t)sm_count * occ + n_slabs - 1) / n_slabs;
     uint64_t gx = want < fill ? want : fill;
     if (gx < 1) gx = 1;
+    const uint32_t gps = cps / 32;
+    const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
+    const uint32_t cap32 = cap < 0xFFFFFFFFull ? (uint32_t)cap : 0xFFFFFFFFu;
     dim3 grid((unsigned)gx, (unsigned)n_slabs);
     kern<<<grid, DEC_THREADS, smem, stream>>>(words, radius, reinterpret_cast<const float4 *>(cb),
-                                              S, b, H, cps, y, reinterpret_cast<DevStatus *>(st));
+                                              S, b, H, cps, y, reinterpret_cast<DevStatus *>(st),
+                                              tile_off, tps, out_idx, out_val, cap32);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}
+
+template <int OUT_DT, bool TABLE>
+static int launch_main_l(int listed, const uint32_t *words, const uint16_t *radius,
+                         const float *cb, uint32_t S, uint32_t b, int B, int H, uint32_t cps,
+                         void *y, hqmq_status *st, const uint32_t *tile_off,
+                         const uint32_t *out_idx, const uint16_t *out_val, uint64_t cap, int sm,
+                         cudaStream_t stream) {
+    if (listed == HQMQ_GRAN_CHUNK + 1)
+        return launch_main<OUT_DT, TABLE, HQMQ_GRAN_CHUNK + 1>(
+            words, radius, cb, S, b, B, H, cps, y, st, tile_off, out_idx, out_val, cap, sm, stream);
+    if (listed == HQMQ_GRAN_ELEMENT + 1)
+        return launch_main<OUT_DT, TABLE, HQMQ_GRAN_ELEMENT + 1>(
+            words, radius, cb, S, b, B, H, cps, y, st, tile_off, out_idx, out_val, cap, sm, stream);
+    return launch_main<OUT_DT, TABLE, 0>(words, radius, cb, S, b, B, H, cps, y, st, nullptr,
+                                         nullptr, nullptr, 0, sm, stream);
 }
 
 template <int OUT_DT>
@@ -239,13 +339,17 @@ static int launch_out(int gran, const uint32_t *words, const uint16_t *radius, c
 template <int OUT_DT>
 static int launch_all(bool table, int gran, const uint32_t *words, const uint16_t *radius,
                       const float *cb, uint32_t S, uint32_t b, const uint32_t *out_idx,
-                      const uint16_t *out_val, const uint32_t *slab_off, uint64_t cap, int B,
-                      int H, uint32_t cps, void *y, hqmq_status *st, int sm,
+                      const uint16_t *out_val, const uint32_t *slab_off, const uint32_t *tile_off,
+                      uint64_t cap, int B, int H, uint32_t cps, void *y, hqmq_status *st, int sm,
                       cudaStream_t stream) {
-    int rc = table ? launch_main<OUT_DT, true>(words, radius, cb, S, b, B, H, cps, y, st, sm, stream)
-                   : launch_main<OUT_DT, false>(words, radius, cb, S, b, B, H, cps, y, st, sm,
-                                                stream);
-    if (rc != HQMQ_OK || out_idx == nullptr || cap == 0) return rc;
+    const bool has_list = out_idx != nullptr && cap > 0;
+    // with the list's tile offsets the main pass applies the list itself
+    const int listed = has_list && tile_off ? gran + 1 : 0;
+    int rc = table ? launch_main_l<OUT_DT, true>(listed, words, radius, cb, S, b, B, H, cps, y, st,
+                                                 tile_off, out_idx, out_val, cap, sm, stream)
+                   : launch_main_l<OUT_DT, false>(listed, words, radius, cb, S, b, B, H, cps, y,
+                                                  st, tile_off, out_idx, out_val, cap, sm, stream);
+    if (rc != HQMQ_OK || !has_list || listed) return rc;
     return launch_out<OUT_DT>(gran, words, radius, cb, S, b, B, H, cps, out_idx, out_val, slab_off,
                               cap, y, sm, stream);
 }
@@ -254,15 +358,16 @@ static int launch_all(bool table, int gran, const uint32_t *words, const uint16_
 
 extern "C" int hqmq_launch_decode(const uint32_t *words, const uint16_t *radius, const float *cb,
                                   uint32_t S, uint32_t b, const uint32_t *out_idx,
-                                  const uint16_t *out_val, const uint32_t *slab_off, uint64_t cap,
-                                  int gran, int B, int H, int T, int D, void *y, int out_dtype,
-                                  hqmq_status *st, int sm_count, cudaStream_t stream) {
+                                  const uint16_t *out_val, const uint32_t *slab_off,
+                                  const uint32_t *tile_off, uint64_t cap, int gran, int B, int H,
+                                  int T, int D, void *y, int out_dtype, hqmq_status *st,
+                                  int sm_count, cudaStream_t stream) {
     using namespace hqmq;
     const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
     const bool table = S <= 170;
     if (out_dtype == HQMQ_BF16)
         return launch_all<HQMQ_BF16>(table, gran, words, radius, cb, S, b, out_idx, out_val,
-                                     slab_off, cap, B, H, cps, y, st, sm_count, stream);
+                                     slab_off, tile_off, cap, B, H, cps, y, st, sm_count, stream);
     return launch_all<HQMQ_F32>(table, gran, words, radius, cb, S, b, out_idx, out_val, slab_off,
-                                cap, B, H, cps, y, st, sm_count, stream);
+                                tile_off, cap, B, H, cps, y, st, sm_count, stream);
 }

@@ -488,8 +488,8 @@ __device__ void exact_fallback(const void *x, int B, int H, int h, uint32_t cps,
     }
 }
 
-// Exclusive scan of the tile counts into tile offsets and slab offsets (one
-// CTA).  Per step, warp w owns SCAN_WARP consecutive tiles, read and written as
+// Exclusive scan of the tile counts into tile offsets (n_tiles + 1 entries,
+// the last one the total) and slab offsets (one CTA).  Per step, warp w owns SCAN_WARP consecutive tiles, read and written as
 // 128-tile pieces (lane l: tiles 4l..4l+3 of each piece, one 16-byte access;
 // all pieces in flight); each piece is scanned by the warp, the block scans
 // the 32 warp totals.
@@ -558,6 +558,7 @@ __device__ void scan_tiles(const uint32_t *tile_cnt, uint64_t n_tiles, uint32_t 
     for (uint32_t sl = t; sl < n_slabs; sl += WIN_THREADS)
         slab_off[sl] = tile_off[(uint64_t)sl * tiles_per_slab];
     if (t == 0) {
+        tile_off[n_tiles] = (uint32_t)carry;
         slab_off[n_slabs] = (uint32_t)carry;
         if (st) {
             atomicAdd(&st->n_outliers, carry);
@@ -656,17 +657,16 @@ static int run_front(const void *x, int B, int H, int T, int D, float C, char *w
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
-// F + X + U + S.
+// F + X + U + S; the tile offsets go to tile_off.
 template <int DT, int GRAN>
 static int run_finish(const void *x, int B, int H, int T, int D, float C, float *rmed, float *thr,
-                      uint32_t *slab_off, uint64_t cap, char *ws, hqmq_status *st_,
-                      cudaStream_t stream) {
+                      uint32_t *slab_off, uint32_t *tile_off, uint64_t cap, char *ws,
+                      hqmq_status *st_, cudaStream_t stream) {
     DevStatus *st = reinterpret_cast<DevStatus *>(st_);
     const FusedLayout L = fused_layout(B, H, T, D, GRAN);
     const SpecArgs a = spec_args(ws, L);
     Counters *ctr = reinterpret_cast<Counters *>(ws + L.counters);
     WinState *win = reinterpret_cast<WinState *>(ws + L.win);
-    uint32_t *tile_off = reinterpret_cast<uint32_t *>(ws + L.tile_off);
     const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
     k_finalize<DT, GRAN><<<H, WIN_THREADS, 0, stream>>>(
         x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, a.below, a.cand_n,
@@ -698,38 +698,45 @@ extern "C" int hqmq_launch_med3_front(const void *x, int dtype, int B, int H, in
                : run_front<HQMQ_F32, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, w, pb, sm_count, stream);
 }
 
-// Steps F + X + U + S; returns the tile offsets (inside ws) for the list pass.
+// Steps F + X + U + S.  The tile offsets go to tile_off_out (n_tiles + 1
+// entries) if given, else into ws; *tile_off returns where they are.
 extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, int T, int D,
                                        float C, int gran, float *rmed, float *thr,
-                                       uint32_t *slab_off, uint64_t cap, void *ws,
-                                       hqmq_status *st, cudaStream_t stream,
+                                       uint32_t *slab_off, uint32_t *tile_off_out, uint64_t cap,
+                                       void *ws, hqmq_status *st, cudaStream_t stream,
                                        const uint32_t **tile_off, uint32_t *tiles_per_slab) {
     using namespace hqmq;
     const FusedLayout L = fused_layout(B, H, T, D, gran);
     char *w = reinterpret_cast<char *>(ws);
-    *tile_off = reinterpret_cast<const uint32_t *>(w + L.tile_off);
+    uint32_t *to = tile_off_out ? tile_off_out : reinterpret_cast<uint32_t *>(w + L.tile_off);
+    *tile_off = to;
     *tiles_per_slab = L.tiles_per_slab;
     if (dtype == HQMQ_BF16)
         return gran == HQMQ_GRAN_CHUNK
                    ? run_finish<HQMQ_BF16, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off,
-                                                            cap, w, st, stream)
+                                                            to, cap, w, st, stream)
                    : run_finish<HQMQ_BF16, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr,
-                                                              slab_off, cap, w, st, stream);
+                                                              slab_off, to, cap, w, st, stream);
     return gran == HQMQ_GRAN_CHUNK
-               ? run_finish<HQMQ_F32, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off, cap,
-                                                       w, st, stream)
-               : run_finish<HQMQ_F32, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr, slab_off, cap,
-                                                         w, st, stream);
+               ? run_finish<HQMQ_F32, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off, to,
+                                                       cap, w, st, stream)
+               : run_finish<HQMQ_F32, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr, slab_off, to,
+                                                         cap, w, st, stream);
 }
 
 // All steps A..S (two-read path); returns the tile offsets for pass C.
 extern "C" int hqmq_launch_med3_window(const void *x, int dtype, int B, int H, int T, int D,
                                        float C, int gran, float *rmed, float *thr,
-                                       uint32_t *slab_off, uint64_t cap, void *ws,
-                                       hqmq_status *st, int sm_count, cudaStream_t stream,
-                                       const uint32_t **tile_off, uint32_t *tiles_per_slab) {
+                                       uint32_t *slab_off, uint32_t *tile_off_out, uint64_t cap,
+                                       void *ws, hqmq_status *st, int sm_count,
+                                       cudaStream_t stream, const uint32_t **tile_off,
+                                       uint32_t *tiles_per_slab) {
     const int rc = hqmq_launch_med3_front(x, dtype, B, H, T, D, C, gran, ws, 1, sm_count, stream);
     if (rc != HQMQ_OK) return rc;
-    return hqmq_launch_med3_finish(x, dtype, B, H, T, D, C, gran, rmed, thr, slab_off, cap, ws, st,
-                                   stream, tile_off, tiles_per_slab);
+    return hqmq_launch_med3_finish(x, dtype, B, H, T, D, C, gran, rmed, thr, slab_off,
+                                   tile_off_out, cap, ws, st, stream, tile_off, tiles_per_slab);
+}
+
+extern "C" uint64_t hqmq_list_tile_count(int B, int H, int T, int D) {
+    return hqmq::fused_layout(B, H, T, D, HQMQ_GRAN_CHUNK).n_tiles;
 }

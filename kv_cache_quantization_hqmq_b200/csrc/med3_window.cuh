@@ -73,7 +73,7 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     L.cand = off;        off = align256_(off + (uint64_t)H * L.cand_cap * 4);
     L.amb = off;         off = align256_(off + L.amb_cap * 8);
     L.tile_cnt = off;    off = align256_(off + L.n_tiles * 4);
-    L.tile_off = off;    off = align256_(off + L.n_tiles * 4);
+    L.tile_off = off;    off = align256_(off + (L.n_tiles + 1) * 4);
     L.cbits = off;       off = align256_(off + (uint64_t)B * H * gps * 4);
     L.total = off;
     return L;

@@ -45,15 +45,17 @@ _SIGS = {
     "hqmq_index_words": (_U64, [_I, _I, _I, _I, _U32]),
     "hqmq_make_codebook": (_I, [_U64, _U32, _U32, _U32, _P, _P]),
     "hqmq_outlier_workspace_size": (_U64, [_I, _I, _I, _I, _I]),
-    "hqmq_outlier_extract": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P, _U64, _P,
-                                  _U64, _P, _P]),
+    "hqmq_outlier_extract": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P, _P, _U64,
+                                  _P, _U64, _P, _P]),
+    "hqmq_list_tiles": (_U64, [_I, _I, _I, _I]),
     "hqmq_encode": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _I, _P, _P, _P, _P]),
-    "hqmq_decode": (_I, [_P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P, _I, _P, _P]),
+    "hqmq_decode": (_I, [_P, _P, _P, _U32, _P, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P, _I, _P,
+                         _P]),
     "hqmq_outlier_extract_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P,
                                           _U64, _P, _P]),
     "hqmq_encode_med3_workspace_size": (_U64, [_I, _I, _I, _I, _I]),
     "hqmq_encode_med3": (_I, [_P, _I, _I, _I, _I, _I, _F, _I, _P, _U32, _P, _P, _P, _P, _P, _P,
-                              _P, _P, _U64, _P, _U64, _P, _P]),
+                              _P, _P, _P, _U64, _P, _U64, _P, _P]),
     "hqmq_search_table_bytes": (_U64, [_U32]),
     "hqmq_make_search_table": (_I, [_P, _U32, _U32, _P, _P]),
     "hqmq_encode_lut": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _P, _I, _P, _P, _P, _P]),
@@ -134,12 +136,17 @@ def hqmq_make_codebook(seed, S, n_groups, group0, codebook, stream=None):
 
 
 def hqmq_outlier_extract(x, C, gran, rmed, thr, out_idx, out_val, slab_off, cap, ws,
-                         status=None, stream=None):
+                         status=None, stream=None, tile_off=None):
+    """tile_off: optional uint32 [hqmq_list_tiles(B, H, T, D) + 1] output."""
     B, H, T, D = _shape4(x)
     _check("hqmq_outlier_extract", _lib.hqmq_outlier_extract(
         _ptr(x), _dtype_code(x), B, H, T, D, float(C), gran, _ptr(rmed), _ptr(thr),
-        _ptr(out_idx), _ptr(out_val), _ptr(slab_off), int(cap), _ptr(ws),
+        _ptr(out_idx), _ptr(out_val), _ptr(slab_off), _ptr(tile_off), int(cap), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(status), _stream(stream)))
+
+
+def hqmq_list_tiles(B, H, T, D):
+    return int(_lib.hqmq_list_tiles(B, H, T, D))
 
 
 def hqmq_outlier_extract_noalloc(x, C, gran, rmed, thr, out_idx, out_val, slab_off, cap,
@@ -181,23 +188,25 @@ def hqmq_encode_lut(x, codebook, S, table, thr, gran, idx_words, radius, status=
 
 
 def hqmq_encode_med3(x, C, gran, codebook, S, table, idx_words, radius, rmed, thr, out_idx,
-                     out_val, slab_off, cap, ws, status=None, stream=None):
-    """Med3x + encode in two reads of x (table may be None: S-codeword loop)."""
+                     out_val, slab_off, cap, ws, status=None, stream=None, tile_off=None):
+    """Med3x + encode (table may be None: S-codeword loop); tile_off: optional
+    uint32 [hqmq_list_tiles(B, H, T, D) + 1] output."""
     B, H, T, D = _shape4(x)
     _check("hqmq_encode_med3", _lib.hqmq_encode_med3(
         _ptr(x), _dtype_code(x), B, H, T, D, float(C), gran, _ptr(codebook), S, _ptr(table),
         _ptr(idx_words), _ptr(radius), _ptr(rmed), _ptr(thr), _ptr(out_idx), _ptr(out_val),
-        _ptr(slab_off), int(cap), _ptr(ws), ws.numel() * ws.element_size(), _ptr(status),
-        _stream(stream)))
+        _ptr(slab_off), _ptr(tile_off), int(cap), _ptr(ws), ws.numel() * ws.element_size(),
+        _ptr(status), _stream(stream)))
 
 
 def hqmq_decode(idx_words, radius, codebook, S, out_idx, out_val, slab_off, cap, gran, y,
-                status=None, stream=None):
+                status=None, stream=None, tile_off=None):
+    """tile_off: the list's tile offsets (applied in the main pass), or None."""
     B, H, T, D = _shape4(y)
     _check("hqmq_decode", _lib.hqmq_decode(
         _ptr(idx_words), _ptr(radius), _ptr(codebook), S, _ptr(out_idx), _ptr(out_val),
-        _ptr(slab_off), int(cap), gran, B, H, T, D, _ptr(y), _dtype_code(y), _ptr(status),
-        _stream(stream)))
+        _ptr(slab_off), _ptr(tile_off), int(cap), gran, B, H, T, D, _ptr(y), _dtype_code(y),
+        _ptr(status), _stream(stream)))
 
 
 # ---------------------------------------------------------------- buffers
@@ -220,6 +229,14 @@ def alloc_codes(B, H, T, D, S, device="cuda"):
     words = torch.empty(nw, dtype=torch.int32, device=device)
     radius = torch.empty(B * H * T * D // 4, dtype=torch.int16, device=device)
     return words, radius
+
+
+def alloc_tile_off(B, H, T, D, device="cuda"):
+    """uint32 (as int32) [hqmq_list_tiles + 1]: a call's list tile offsets."""
+    n = hqmq_list_tiles(B, H, T, D)
+    if n == 0:
+        raise ValueError("bad shape")
+    return torch.empty(n + 1, dtype=torch.int32, device=device)
 
 
 def alloc_outliers(B, H, T, D, cap, gran=HQMQ_GRAN_CHUNK, device="cuda"):

@@ -63,10 +63,27 @@ def gpu_med3(x_dev, C=3.0, gran=0, cap=None):
     cap = n if cap is None else cap
     st = hqmq.new_status()
     rmed, thr, oi, ov, so, ws = hqmq.alloc_outliers(B, H, T, D, cap, gran)
-    hqmq.hqmq_outlier_extract(x_dev, C, gran, rmed, thr, oi, ov, so, cap, ws, st)
+    to = hqmq.alloc_tile_off(B, H, T, D)
+    hqmq.hqmq_outlier_extract(x_dev, C, gran, rmed, thr, oi, ov, so, cap, ws, st, tile_off=to)
     torch.cuda.synchronize()
-    return dict(rmed=rmed, thr=thr, out_idx=oi, out_val=ov, slab_off=so, cap=cap,
+    return dict(rmed=rmed, thr=thr, out_idx=oi, out_val=ov, slab_off=so, tile_off=to, cap=cap,
                 status=hqmq.read_status(st))
+
+
+LIST_TILE_CHUNKS = 1024
+
+
+def list_tile_off(idx, B, H, T, D, gran=0):
+    """The list's tile offsets from their definition: for every tile (1024
+    consecutive chunks of a slab, the slab's last tile possibly shorter) the
+    number of list entries before its first chunk, then the total."""
+    cps = T * D // 4
+    tps = -(-cps // LIST_TILE_CHUNKS)
+    starts = (np.arange(B * H)[:, None] * cps +
+              np.minimum(np.arange(tps)[None, :] * LIST_TILE_CHUNKS, cps)).reshape(-1)
+    chunk = np.asarray(idx, np.int64) // (4 if gran else 1)
+    off = np.searchsorted(chunk, starts, side="left")
+    return np.concatenate([off, [len(chunk)]]).astype(np.uint32)
 
 
 def gpu_search_table(cb_dev, S, n_groups):
@@ -90,14 +107,17 @@ def gpu_encode(x_dev, cb_dev, S, thr_dev=None, gran=0, encoder="sloop"):
     return words, radius, hqmq.read_status(st)
 
 
-def gpu_decode(words, radius, cb_dev, S, shape, out_dtype=torch.bfloat16, med=None, gran=0):
+def gpu_decode(words, radius, cb_dev, S, shape, out_dtype=torch.bfloat16, med=None, gran=0,
+               tiles=False):
+    """tiles: apply the list through med["tile_off"] (in the main pass)."""
     y = torch.empty(shape, dtype=out_dtype, device="cuda")
     st = hqmq.new_status()
     if med is None:
         hqmq.hqmq_decode(words, radius, cb_dev, S, None, None, None, 0, gran, y, st)
     else:
         hqmq.hqmq_decode(words, radius, cb_dev, S, med["out_idx"], med["out_val"],
-                         med["slab_off"], med["cap"], gran, y, st)
+                         med["slab_off"], med["cap"], gran, y, st,
+                         tile_off=med["tile_off"] if tiles else None)
     torch.cuda.synchronize()
     return y, hqmq.read_status(st)
 
@@ -145,4 +165,9 @@ def check_med3(oracle, x_np, g, C=3.0, gran=0):
     gv = to_host(g["out_val"]).view(np.uint16)[:k * vw].reshape(-1, vw) if gran == 0 else \
         to_host(g["out_val"]).view(np.uint16)[:k]
     assert same_f16_or_bf16_bits(gv, val_o, bf16=False).all()
+    if g.get("tile_off") is not None:
+        full = idx_o if k == n_o else oracle.extract(x_np, thr_o, gran=gran)[0]
+        B, H, T, D = x_np.shape
+        assert np.array_equal(to_host(g["tile_off"]).view(np.uint32),
+                              list_tile_off(full, B, H, T, D, gran))
     return thr_o, idx_o, val_o, so_o, n_o

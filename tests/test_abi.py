@@ -76,12 +76,12 @@ def test_bad_arguments_rejected_without_cuda(lib):
     # misaligned pointers -> HQMQ_ERR_ALIGN (2)
     assert lib.hqmq_encode(P((1 << 20) + 8), 0, 1, 1, 8, 128, good, 8, None, 0, good, good, st,
                            None) == 2
-    assert lib.hqmq_decode(good, P((1 << 20) + 2), good, 8, None, None, None, 0, 0, 1, 1, 8, 128,
-                           good, 0, st, None) == 2
+    assert lib.hqmq_decode(good, P((1 << 20) + 2), good, 8, None, None, None, None, 0, 0, 1, 1, 8,
+                           128, good, 0, st, None) == 2
     # outlier extract: C must be positive and finite; workspace must be large enough
     assert lib.hqmq_outlier_extract(good, 0, 1, 1, 8, 128, ctypes.c_float(0.0), 0, good, good,
-                                    good, good, good, 16, good, 1 << 20, st, None) == 1
+                                    good, good, good, None, 16, good, 1 << 20, st, None) == 1
     assert lib.hqmq_outlier_extract(good, 0, 1, 1, 8, 128, ctypes.c_float(float("inf")), 0, good,
-                                    good, good, good, good, 16, good, 1 << 20, st, None) == 1
+                                    good, good, good, good, None, 16, good, 1 << 20, st, None) == 1
     assert lib.hqmq_outlier_extract(good, 0, 1, 1, 8, 128, ctypes.c_float(3.0), 0, good, good,
-                                    good, good, good, 16, good, 16, st, None) == 4
+                                    good, good, good, None, 16, good, 16, st, None) == 4

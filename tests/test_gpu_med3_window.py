@@ -38,11 +38,12 @@ def fused(x_np, cb_np, S, gran, use_table, C=3.0, cap=None):
     ws = torch.empty(hqmq.hqmq_encode_med3_workspace_size(B, H, T, D, gran), dtype=torch.uint8,
                      device="cuda")
     st = hqmq.new_status()
+    to = hqmq.alloc_tile_off(B, H, T, D)
     hqmq.hqmq_encode_med3(xd, C, gran, cbd, S, table, words, radius, rmed, thr, oi, ov, so, cap,
-                          ws, st)
+                          ws, st, tile_off=to)
     torch.cuda.synchronize()
     return dict(words=words, radius=radius, rmed=rmed, thr=thr, out_idx=oi, out_val=ov,
-                slab_off=so, cap=cap, status=hqmq.read_status(st))
+                slab_off=so, tile_off=to, cap=cap, status=hqmq.read_status(st))
 
 
 def check_fused(oracle, x_np, S, gran, use_table, seed=1, cap=None):
@@ -121,8 +122,10 @@ def test_fused_capacity_overflow(oracle):
 
 
 def test_fused_equals_separate_calls_full_size_70b(oracle):
-    # one full 70B call: fused (two reads) vs hqmq_outlier_extract +
-    # hqmq_encode_lut (the same kernels' results by definition): bit-identical
+    # one full 70B call: fused (one read) vs hqmq_outlier_extract +
+    # hqmq_encode_lut (two reads): bit-identical codes, list, offsets and
+    # status; then the decode with the list applied inside the main pass
+    # equals the decode with the separate list kernel
     w = W.WORKLOADS["llama3_70b_128k"]
     B, H, T, D = w.call_shape
     xd = W.make_call_input(w, 11, 0, device="cuda")
@@ -133,16 +136,26 @@ def test_fused_equals_separate_calls_full_size_70b(oracle):
     words, radius = hqmq.alloc_codes(B, H, T, D, w.S)
     rmed, thr, oi, ov, so, ws = hqmq.alloc_outliers(B, H, T, D, cap)
     st = hqmq.new_status()
+    to = hqmq.alloc_tile_off(B, H, T, D)
     hqmq.hqmq_encode_med3(xd, w.C, 0, cb, w.S, table, words, radius, rmed, thr, oi, ov, so, cap,
-                          ws, st)
+                          ws, st, tile_off=to)
     words2, radius2 = hqmq.alloc_codes(B, H, T, D, w.S)
     rmed2, thr2, oi2, ov2, so2, ws2 = hqmq.alloc_outliers(B, H, T, D, cap)
     st2 = hqmq.new_status()
-    hqmq.hqmq_outlier_extract(xd, w.C, 0, rmed2, thr2, oi2, ov2, so2, cap, ws2, st2)
+    to2 = hqmq.alloc_tile_off(B, H, T, D)
+    hqmq.hqmq_outlier_extract(xd, w.C, 0, rmed2, thr2, oi2, ov2, so2, cap, ws2, st2, tile_off=to2)
     hqmq.hqmq_encode_lut(xd, cb, w.S, table, thr2, 0, words2, radius2, st2)
     torch.cuda.synchronize()
-    for a, b in ((words, words2), (radius, radius2), (thr, thr2), (so, so2)):
+    for a, b in ((words, words2), (radius, radius2), (thr, thr2), (so, so2), (to, to2)):
         assert torch.equal(a, b)
+    ys = []
+    for tiles in (False, True):
+        y = torch.empty(B, H, T, D, dtype=torch.bfloat16, device="cuda")
+        hqmq.hqmq_decode(words, radius, cb, w.S, oi, ov, so, cap, 0, y, hqmq.new_status(),
+                         tile_off=to if tiles else None)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0].view(torch.int16), ys[1].view(torch.int16))
     n = int(so[-1])
     assert torch.equal(oi[:n], oi2[:n]) and torch.equal(ov[:4 * n], ov2[:4 * n])
     assert hqmq.read_status(st) == hqmq.read_status(st2)

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 import torch
 
-from _parity import (DECODE_ABS_TOL, NEAR_TIE_REL, check_codes, check_med3, gpu_codebook,
+from _parity import (list_tile_off, DECODE_ABS_TOL, NEAR_TIE_REL, check_codes, check_med3, gpu_codebook,
                      gpu_decode, gpu_encode, gpu_med3, same_f16_or_bf16_bits, same_f32, to_host,
                      unpack_indices)
 
@@ -65,27 +65,31 @@ def full_call(oracle, x_np, S, cb_np, med3=False, C=3.0, gran=0, name="", check_
         k = oi_o.size
         med_o = dict(out_idx=dev(oi_o.view(np.int32)) if k else torch.zeros(1, dtype=torch.int32, device="cuda"),
                      out_val=dev(ov_o.reshape(-1).view(np.int16)) if k else torch.zeros(4, dtype=torch.int16, device="cuda"),
-                     slab_off=dev(so_o.view(np.int32)), cap=k)
+                     slab_off=dev(so_o.view(np.int32)), cap=k,
+                     tile_off=dev(list_tile_off(oi_o, B, H, T, D, gran).view(np.int32)))
     for out_dt, od in ((torch.bfloat16, 0), (torch.float32, 1)):
-        y, _ = gpu_decode(owd, orad_d, cbd, S, (B, H, T, D), out_dt, med_o, gran)
         yo, _ = oracle.decode(ow, orad, cb_np, S, B, H, T, D,
                               out_idx=oi_o if med3 else None, out_val=ov_o if med3 else None,
                               gran=gran, out_dtype=od)
-        if od == 0:
-            ok = same_f16_or_bf16_bits(to_host(y.view(torch.int16)), yo, bf16=True)
-        else:
-            ok = same_f32(to_host(y), yo)
-        assert ok.all(), "decode mismatch at %s" % np.argwhere(~ok)[:5]
+        # the list applied by a second kernel, and inside the main pass
+        for tiles in ((False, True) if med3 else (False,)):
+            y, _ = gpu_decode(owd, orad_d, cbd, S, (B, H, T, D), out_dt, med_o, gran, tiles)
+            if od == 0:
+                ok = same_f16_or_bf16_bits(to_host(y.view(torch.int16)), yo, bf16=True)
+            else:
+                ok = same_f32(to_host(y), yo)
+            assert ok.all(), "decode (tiles %d) mismatch at %s" % (tiles, np.argwhere(~ok)[:5])
     if check_e2e:
         # end to end: GPU encode + GPU decode vs oracle encode + decode
-        y, _ = gpu_decode(words, radius, cbd, S, (B, H, T, D), torch.float32,
-                          med if med3 else None, gran)
         yo, _ = oracle.decode(ow, orad, cb_np, S, B, H, T, D,
                               out_idx=oi_o if med3 else None, out_val=ov_o if med3 else None,
                               gran=gran, out_dtype=1)
-        diff = np.abs(to_host(y).reshape(-1, 4) - yo.reshape(-1, 4)).max(axis=1)
         exempt = gi != unpack_indices(ow, S, n_chunks)
-        assert np.all(diff[~exempt] <= DECODE_ABS_TOL)
+        for tiles in ((False, True) if med3 else (False,)):
+            y, _ = gpu_decode(words, radius, cbd, S, (B, H, T, D), torch.float32,
+                              med if med3 else None, gran, tiles)
+            diff = np.abs(to_host(y).reshape(-1, 4) - yo.reshape(-1, 4)).max(axis=1)
+            assert np.all(diff[~exempt] <= DECODE_ABS_TOL)
     return dict(words=words, radius=radius, status=st, med=med)
 
 
@@ -292,14 +296,16 @@ def _full_size_call(oracle, name, layer, role, n_sample=20000, gran=0, encoder="
     if med is not None:
         k = len(oi_o)
         med_o = dict(out_idx=dev(oi_o.view(np.int32)), out_val=dev(ov_o.reshape(-1).view(np.int16)),
-                     slab_off=dev(so_o.view(np.int32)), cap=k)
-    y, _ = gpu_decode(dev(wr.reshape(-1).view(np.int32)), dev(rad_r.view(np.int16)), cbd, w.S,
-                      (B, H, T, D), torch.bfloat16, med_o, gran)
+                     slab_off=dev(so_o.view(np.int32)), cap=k,
+                     tile_off=dev(list_tile_off(oi_o, B, H, T, D, gran).view(np.int32)))
     yo, _ = oracle.decode(wr.reshape(-1), rad_r, cb, w.S, B, H, T, D,
                           out_idx=oi_o if med is not None else None,
                           out_val=ov_o if med is not None else None, gran=gran, out_dtype=0)
-    ok = same_f16_or_bf16_bits(to_host(y.view(torch.int16)), yo, bf16=True)
-    assert ok.all(), np.argwhere(~ok.reshape(-1))[:5]
+    for tiles in ((False, True) if med is not None else (False,)):
+        y, _ = gpu_decode(dev(wr.reshape(-1).view(np.int32)), dev(rad_r.view(np.int16)), cbd,
+                          w.S, (B, H, T, D), torch.bfloat16, med_o, gran, tiles)
+        ok = same_f16_or_bf16_bits(to_host(y.view(torch.int16)), yo, bf16=True)
+        assert ok.all(), (tiles, np.argwhere(~ok.reshape(-1))[:5])
 
 
 @pytest.mark.parametrize("encoder", ENCODERS)
