@@ -8,8 +8,9 @@
 //
 // k_decode: each CTA owns one slab (b, h), builds that head's 24 S codeword
 // table in shared memory once (S <= 170; larger S recomputes the codeword
-// per chunk) and streams its chunks: per chunk pair one 4-byte radius load,
-// the index bits, 8 products and one 16-byte store; no barriers after the
+// per chunk) and streams its chunks in units of 8 packing groups: the unit's
+// index words staged in shared memory, one radius per lane and group, 4
+// products and one 8-byte (bf16) store per chunk; no block barriers after the
 // table build.  Outlier list entries overwrite their chunk (chunk mode) or
 // add the fp16 value to the recomputed fl32(r * c) of their element (element
 // mode):
@@ -23,7 +24,6 @@
 namespace hqmq {
 
 constexpr int DEC_THREADS = 256;
-constexpr int PAIRS = 4;             // chunk pairs per thread per step (8 chunks in flight)
 constexpr int OUT_THREADS = 256;
 
 __device__ __forceinline__ uint32_t get_index(const uint32_t *__restrict__ words, uint64_t grp,
@@ -55,106 +55,93 @@ __device__ __forceinline__ float element_with_outlier(const uint32_t *__restrict
     return __fadd_rn(__fmul_rn(r, c), f16_bits_to_f32(v16));
 }
 
-// Main pass: every chunk -> round(fl32(r * c_i)).  Thread t of a warp handles
-// the chunk pairs w*PAIRS*32 + u*32 + t (u < PAIRS): each load and each
-// 16-byte store instruction of the warp is contiguous, and PAIRS pairs of
-// loads are in flight per thread.
+// Main pass: every chunk -> round(fl32(r * c_i)).  A warp takes units of
+// DEC_UNIT packing groups (256 chunks) of one slab: it stages the unit's
+// index words in shared memory (coalesced loads), loads the unit's radii
+// (lane k: chunk k of each group, all in flight), then per group lane k
+// extracts its index from two staged words, multiplies and stores its chunk
+// (a warp store covers the group's 32 chunks).
 // LISTED: 0 = no list here, HQMQ_GRAN_CHUNK + 1 / HQMQ_GRAN_ELEMENT + 1 =
-// apply the list of that granularity through its tile offsets.
+// apply the list of that granularity through its tile offsets: after a unit's
+// stores and a __syncwarp(), the warp writes the entries of its tile that
+// fall inside the unit.
+constexpr int DEC_UNIT = 8;                      // packing groups per unit
 template <int OUT_DT, bool TABLE, int LISTED>
-__global__ void __launch_bounds__(DEC_THREADS)
+__global__ void __launch_bounds__(DEC_THREADS, 8)
 k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius,
          const float4 *__restrict__ cb_all, uint32_t S, uint32_t b, int H,
          uint32_t chunks_per_slab, void *__restrict__ y, DevStatus *st,
          const uint32_t *__restrict__ tile_off, uint32_t tiles_per_slab,
          const uint32_t *__restrict__ out_idx, const uint16_t *__restrict__ out_val,
          uint32_t cap32) {
-    extern __shared__ float4 s_tab[];              // [24 S] if TABLE
+    extern __shared__ float4 s_dyn[];
+    const uint32_t n_words = 24u * S;
+    float4 *s_tab = s_dyn;                         // [24 S] if TABLE
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t *s_w = reinterpret_cast<uint32_t *>(s_dyn + (TABLE ? n_words : 0)) +
+                    (uint32_t)warp * DEC_UNIT * b;  // this warp's staged words
     const int slab = blockIdx.y;
     const int h = slab % H;
     const float4 *cb = cb_all + (size_t)h * S;
-    const uint32_t n_words = 24u * S;
     if (TABLE) {
         for (uint32_t i = threadIdx.x; i < n_words; i += DEC_THREADS)
             s_tab[i] = codeword((int)(i % 24u), __ldg(cb + i / 24u));
         __syncthreads();
     }
-    const uint64_t chunk0 = (uint64_t)slab * chunks_per_slab;
-    const uint32_t pairs_per_slab = chunks_per_slab / 2;
-    const int lane = threadIdx.x & 31;
-    const uint32_t warp_g = blockIdx.x * (DEC_THREADS / 32) + (threadIdx.x >> 5);
+    const uint32_t gps = chunks_per_slab / 32;
+    const uint64_t gs0 = (uint64_t)slab * gps;     // the slab's first packing group
+    const uint32_t n_units = (gps + DEC_UNIT - 1) / DEC_UNIT;
+    const uint32_t lbit = (uint32_t)lane * b, lw = lbit >> 5, lo = lbit & 31u;
+    const bool two = lo + b > 32u;                 // index spans two words
+    const uint32_t mask = (1u << b) - 1u;
+    const uint32_t warp_g = blockIdx.x * (DEC_THREADS / 32) + (uint32_t)warp;
     const uint32_t n_warps = gridDim.x * (DEC_THREADS / 32);
     unsigned n_bad = 0;
-    for (uint32_t p0 = warp_g * PAIRS * 32; p0 < pairs_per_slab; p0 += n_warps * PAIRS * 32) {
-        uint32_t rr[PAIRS], idx[PAIRS][2];
+    for (uint32_t un = warp_g; un < n_units; un += n_warps) {
+        const uint32_t g0 = un * DEC_UNIT;
+        const uint32_t ng = min((uint32_t)DEC_UNIT, gps - g0);
+        const uint64_t gg0 = gs0 + g0;             // global packing group of the unit
+        uint32_t rr[DEC_UNIT];
 #pragma unroll
-        for (int u = 0; u < PAIRS; ++u) {              // all loads first
-            const uint32_t pr = p0 + u * 32 + lane;
-            rr[u] = 0; idx[u][0] = idx[u][1] = 0;
-            if (pr < pairs_per_slab) {
-                const uint64_t j = chunk0 + 2 * (uint64_t)pr;
-                rr[u] = __ldcs(reinterpret_cast<const uint32_t *>(radius) + (j >> 1));
-                if (b <= 16) {                       // both indices from one 64-bit window
-                    const uint32_t *wg = words + (j >> 5) * b;
-                    const uint32_t bit = (uint32_t)(j & 31u) * b, o = bit & 31u;
-                    uint64_t v = __ldg(wg + (bit >> 5));
-                    if (o + 2 * b > 32u) v |= (uint64_t)__ldg(wg + (bit >> 5) + 1) << 32;
-                    const uint32_t mask = (1u << b) - 1u;
-                    idx[u][0] = (uint32_t)(v >> o) & mask;
-                    idx[u][1] = (uint32_t)(v >> (o + b)) & mask;
-                } else {
-                    idx[u][0] = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
-                    idx[u][1] = get_index(words, j >> 5, (uint32_t)(j & 31u) + 1, b);
-                }
+        for (int u = 0; u < DEC_UNIT; ++u)         // radii: all in flight
+            rr[u] = (uint32_t)u < ng ? __ldcs(radius + (gg0 + u) * 32 + lane) : 0u;
+        __syncwarp();                              // (the previous unit's reads of s_w)
+        for (uint32_t i = lane; i < ng * b; i += 32) s_w[i] = __ldg(words + gg0 * b + i);
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < DEC_UNIT; ++u) {
+            if ((uint32_t)u >= ng) break;
+            const uint32_t *sw = s_w + u * b + lw;
+            const uint32_t ix = __funnelshift_r(sw[0], two ? sw[1] : 0u, lo) & mask;
+            float r = f16_bits_to_f32(rr[u]);
+            float4 cw;
+            if (ix < n_words) {
+                cw = TABLE ? s_tab[ix] : codeword((int)(ix % 24u), __ldg(cb + ix / 24u));
+            } else {
+                cw = make_float4(0.f, 0.f, 0.f, 0.f);
+                r = 0.0f;
+                ++n_bad;
             }
-        }
-#pragma unroll
-        for (int u = 0; u < PAIRS; ++u) {
-            const uint32_t pr = p0 + u * 32 + lane;
-            if (pr >= pairs_per_slab) break;
-            const uint64_t j = chunk0 + 2 * (uint64_t)pr;
-            float out[8];
-#pragma unroll
-            for (int v = 0; v < 2; ++v) {
-                float r = f16_bits_to_f32(v ? (rr[u] >> 16) : (rr[u] & 0xFFFFu));
-                const uint32_t ix = idx[u][v];
-                float4 cw;
-                if (ix < n_words) {
-                    cw = TABLE ? s_tab[ix] : codeword((int)(ix % 24u), __ldg(cb + ix / 24u));
-                } else {
-                    cw = make_float4(0.f, 0.f, 0.f, 0.f);
-                    r = 0.0f;
-                    ++n_bad;
-                }
-                out[4 * v + 0] = __fmul_rn(r, cw.x);
-                out[4 * v + 1] = __fmul_rn(r, cw.y);
-                out[4 * v + 2] = __fmul_rn(r, cw.z);
-                out[4 * v + 3] = __fmul_rn(r, cw.w);
-            }
+            const uint64_t j = (gg0 + u) * 32 + lane;
+            const float o0 = __fmul_rn(r, cw.x), o1 = __fmul_rn(r, cw.y);
+            const float o2 = __fmul_rn(r, cw.z), o3 = __fmul_rn(r, cw.w);
             if (OUT_DT == HQMQ_BF16) {
-                uint4 q;
-                __nv_bfloat162 a0 = __floats2bfloat162_rn(out[0], out[1]);
-                __nv_bfloat162 a1 = __floats2bfloat162_rn(out[2], out[3]);
-                __nv_bfloat162 a2 = __floats2bfloat162_rn(out[4], out[5]);
-                __nv_bfloat162 a3 = __floats2bfloat162_rn(out[6], out[7]);
+                __nv_bfloat162 a0 = __floats2bfloat162_rn(o0, o1);
+                __nv_bfloat162 a1 = __floats2bfloat162_rn(o2, o3);
+                uint2 q;
                 q.x = *reinterpret_cast<uint32_t *>(&a0);
                 q.y = *reinterpret_cast<uint32_t *>(&a1);
-                q.z = *reinterpret_cast<uint32_t *>(&a2);
-                q.w = *reinterpret_cast<uint32_t *>(&a3);
-                __stcs(reinterpret_cast<uint4 *>(y) + (j >> 1), q);
+                reinterpret_cast<uint2 *>(y)[j] = q;
             } else {
-                float4 *yp = reinterpret_cast<float4 *>(y) + j;
-                __stcs(yp, make_float4(out[0], out[1], out[2], out[3]));
-                __stcs(yp + 1, make_float4(out[4], out[5], out[6], out[7]));
+                reinterpret_cast<float4 *>(y)[j] = make_float4(o0, o1, o2, o3);
             }
         }
         if (LISTED) {
-            // the list entries of this quarter [q0, q1) (chunk indices), from
+            // the list entries of this unit [q0, q1) (chunk indices), from
             // its tile's list range; ordered after the warp's stores above
             __syncwarp();
-            const uint64_t q0 = chunk0 + 2 * (uint64_t)p0;
-            const uint64_t q1 = min(q0 + 2 * PAIRS * 32, chunk0 + chunks_per_slab);
-            const uint64_t gt = (uint64_t)slab * tiles_per_slab + (2 * p0) / TILE_CHUNKS;
+            const uint64_t q0 = gg0 * 32, q1 = (gg0 + ng) * 32;
+            const uint64_t gt = (uint64_t)slab * tiles_per_slab + g0 / TILE_GROUPS;
             const uint32_t a = __ldg(tile_off + gt);
             uint32_t e = __ldg(tile_off + gt + 1);
             if (e > cap32) e = cap32;
@@ -270,7 +257,8 @@ static int launch_main(const uint32_t *words, const uint16_t *radius, const floa
                        const uint32_t *tile_off, const uint32_t *out_idx, const uint16_t *out_val,
                        uint64_t cap, int sm_count, cudaStream_t stream) {
     auto kern = k_decode<OUT_DT, TABLE, LISTED>;
-    size_t smem = TABLE ? (size_t)24 * S * sizeof(float4) : 0;
+    const size_t smem = (TABLE ? (size_t)24 * S * sizeof(float4) : 0) +
+                        (size_t)(DEC_THREADS / 32) * DEC_UNIT * b * sizeof(uint32_t);
     if (smem > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
@@ -281,12 +269,12 @@ static int launch_main(const uint32_t *words, const uint16_t *radius, const floa
             cudaSuccess || occ < 1)
         occ = 1;
     const int n_slabs = B * H;
-    const uint64_t per_cta = (uint64_t)DEC_THREADS * PAIRS * 2;     // chunks per CTA step
-    const uint64_t want = (cps + per_cta - 1) / per_cta;
+    const uint32_t gps = cps / 32;
+    const uint64_t units = (gps + DEC_UNIT - 1) / DEC_UNIT;
+    const uint64_t want = (units + DEC_THREADS / 32 - 1) / (DEC_THREADS / 32);
     const uint64_t fill = ((uint64_t)sm_count * occ + n_slabs - 1) / n_slabs;
     uint64_t gx = want < fill ? want : fill;
     if (gx < 1) gx = 1;
-    const uint32_t gps = cps / 32;
     const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
     const uint32_t cap32 = cap < 0xFFFFFFFFull ? (uint32_t)cap : 0xFFFFFFFFu;
     dim3 grid((unsigned)gx, (unsigned)n_slabs);
