@@ -318,6 +318,26 @@ __device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b_rt, int la
 // r <= t_hi; a head whose window missed gets the full list + encode pass.
 // Work: warp tiles of TILE_GROUPS consecutive packing groups; a CTA owns a
 // contiguous range of tiles and walks it slab by slab (one head at a time).
+// Packs a warp tile's indices, staged in shared memory (s_idx[k], k = the
+// chunk's position in the tile), into the tile's ng * BB words: lane l
+// writes words l, l + 32, ... (coalesced), word w being the OR of the
+// pack_terms<BB>() indices that overlap it (see pack_group32).
+template <int BB>
+__device__ __forceinline__ void pack_tile(const uint16_t *s_idx, uint32_t ng, int lane,
+                                          uint32_t *__restrict__ dst) {
+    constexpr int NT = pack_terms<BB>();
+    static_assert(pack_plan_ok<BB>(), "packing plan out of range");
+    const uint32_t nw = ng * BB;
+    for (uint32_t w = (uint32_t)lane; w < nw; w += 32) {
+        const uint32_t k0 = (32u * w) / BB;
+        const uint32_t o = 32u * w - BB * k0;
+        uint32_t v = (uint32_t)s_idx[k0] >> o;
+#pragma unroll
+        for (int m = 1; m < NT; ++m) v |= (uint32_t)s_idx[k0 + m] << (uint32_t)(BB * m - o);
+        dst[w] = v;
+    }
+}
+
 constexpr int LIST_SPEC = 3;
 constexpr int LIST_FIX = 4;
 
@@ -355,6 +375,12 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
     unsigned n_nf = 0, n_sat = 0;
     // LIST_SPEC: this warp's stage of window keys (of head stage_h)
     uint32_t *stage = reinterpret_cast<uint32_t *>(s_tab + (size_t)(n_words + 1) * 8) + warp * STAGE;
+    // BB != 0: this warp's tile of indices, packed at the end of the tile
+    constexpr bool PACK_TILE = BB != 0;
+    uint16_t *s_idx = reinterpret_cast<uint16_t *>(
+                          reinterpret_cast<uint32_t *>(s_tab + (size_t)(n_words + 1) * 8) +
+                          (LIST == LIST_SPEC ? (ENC_THREADS / 32) * STAGE : 0)) +
+                      warp * TILE_CHUNKS;
     uint32_t n_stage = 0;
     int stage_h = -1;
     for (uint32_t seg = t_begin; seg < t_end;) {
@@ -605,7 +631,15 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                     if (!spec_cand) n_sat += sat;            // (LIST_FIX decides the others)
                 }
                 radius[j] = rh;
-                pack_group32<BB>(idx, b, lane, pc, words + (size_t)G * b);
+                if (PACK_TILE)
+                    s_idx[(g - g0) * 32 + lane] = (uint16_t)idx;
+                else
+                    pack_group32<BB>(idx, b, lane, pc, words + (size_t)G * b);
+            }
+            if (PACK_TILE && ENC) {
+                __syncwarp();
+                pack_tile<BB ? BB : 8>(s_idx, g1 - g0, lane, words + (size_t)(gbase + g0) * b);
+                __syncwarp();                                  // (s_idx is refilled next tile)
             }
             if (LIST == LIST_SPEC) {
                 t_def = __reduce_add_sync(FULL, t_def);
@@ -685,7 +719,8 @@ static int launch_lut_bb(int B, int H, int T, int D, const void *x, const float 
     const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
     const uint32_t n_tiles = (uint32_t)((uint64_t)B * H * tps);
     const size_t smem = (ENC ? enc_smem_bytes(S) : 0) +
-                        (LIST == LIST_SPEC ? (size_t)(ENC_THREADS / 32) * STAGE * 4 : 0);
+                        (LIST == LIST_SPEC ? (size_t)(ENC_THREADS / 32) * STAGE * 4 : 0) +
+                        (ENC && BB != 0 ? (size_t)(ENC_THREADS / 32) * TILE_CHUNKS * 2 : 0);
     auto kern = k_encode_lut<DT, LIST, ENC, BB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
