@@ -120,9 +120,9 @@ HQMQ_API int hqmq_make_codebook(uint64_t seed, uint32_t S, uint32_t n_groups, ui
                        float *d_codebook, void *stream);
 
 /* Bytes of device workspace hqmq_outlier_extract (and hqmq_encode_med3) needs
- * for this shape: two 64 Ki-bin histograms per head, the keys of the median
+ * for this shape: a 64 Ki-bin sample histogram per head, the keys of the median
  * window, the uncertain-threshold list, per-tile counts and offsets and one
- * candidate bit per chunk (about 31 MB for a 1 x 8 x 131072 x 128 call in
+ * candidate bit per chunk (about 29 MB for a 1 x 8 x 131072 x 128 call in
  * chunk mode). */
 HQMQ_API uint64_t hqmq_outlier_workspace_size(int B, int H, int T, int D, int gran);
 

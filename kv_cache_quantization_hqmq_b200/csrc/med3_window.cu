@@ -14,10 +14,12 @@
 //                      the median rank; the exact threshold then lies in
 //                      [t_lo, t_hi].
 //  B   k_pass_b        one full read: per head the count of keys below the
-//                      window and the keys inside it (list + fine histogram);
+//                      window and the keys inside it (staged per warp, appended
+//                      to the head's list);
 //                      per 1024-chunk tile the count of certain outliers
 //                      (r > t_hi) and a list of uncertain ones (t_lo < r <= t_hi).
-//  F   k_finalize      per head: the exact median from the window keys, or,
+//  F   k_finalize      per head: the exact median from the window keys (radix
+//                      select, 12-bit digits), or,
 //                      if the window missed the median (or a buffer
 //                      overflowed), the exact three-pass select over x and
 //                      exact tile counts (never taken on the bench workloads;
@@ -25,6 +27,10 @@
 //                      uncertain keys above the exact threshold; the last CTA
 //                      scans the tile counts into tile and slab offsets.
 //  C   (search.cu)     the second read writes the ordered list (and encodes).
+//                      In chunk mode with search tables the encode pass does
+//                      B's work in the same, single read of x, and a fix-up
+//                      pass after F writes the list (search.cu, LIST_SPEC and
+//                      LIST_FIX).
 //
 // A memset clears the histograms and counters first.  No CTA waits for
 // another: where a step needs the results of all CTAs of the previous one,
@@ -35,7 +41,7 @@ namespace hqmq {
 
 constexpr int WIN_THREADS = 1024;
 constexpr int PB_THREADS = 256;
-constexpr int FINAL_KEYS = 8192;   // per-key counters of one fine bin (bin width <= 2^13)
+constexpr int FINAL_BINS = 4096;   // radix digit of the exact median selection (12 bits)
 
 __device__ __forceinline__ float key_to_float(uint32_t k) {
     return k >= 0x7F800001u ? __int_as_float(0x7FC00000) : __uint_as_float(k);
@@ -166,16 +172,12 @@ __device__ void select_window(int h, uint64_t n_per_head, uint64_t n_samples, fl
         const uint64_t lo = (uint64_t)s_out[0] << 15;
         uint64_t hi = ((uint64_t)s_out[1] + 1) << 15;
         if (hi > 0x80000000ull) hi = 0x80000000ull;
-        const uint64_t span = hi - lo;
-        uint32_t sh = 0;
-        while (((span - 1) >> sh) >= (uint64_t)KEY_BINS) ++sh;
         w.lo_key = (uint32_t)lo;
         w.hi_key = (uint32_t)(hi - 1) + 1u;          // (hi <= 2^31)
-        w.shift = sh;
         w.miss = 0;
         w.t_lo = thr_of_key(C, (uint32_t)lo);
         w.t_hi = thr_of_key(C, (uint32_t)(hi - 1));
-        w.pad[0] = w.pad[1] = 0;
+        w.pad[0] = w.pad[1] = w.pad[2] = 0;
         win[h] = w;
         below[h] = 0;
         cand_n[h] = 0;
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(PB_THREADS)
 k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_slab, uint64_t n_tiles,
          const WinState *__restrict__ win, unsigned long long *__restrict__ below,
          unsigned long long *__restrict__ cand_n, uint32_t *__restrict__ cand, uint64_t cand_cap,
-         uint32_t *__restrict__ fine_hist, unsigned long long *__restrict__ amb_n,
+         unsigned long long *__restrict__ amb_n,
          uint2 *__restrict__ amb, uint64_t amb_cap, uint32_t *__restrict__ tile_cnt) {
     constexpr int NK = GRAN == HQMQ_GRAN_CHUNK ? 1 : 4;
     constexpr int U = 8;                              // groups in flight per lane
@@ -303,8 +305,6 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
                         }
                         if (in) {
                             stage[n_stage + __popc(m & lt)] = key;
-                            atomicAdd(fine_hist + (size_t)h * KEY_BINS + ((key - w.lo_key) >> w.shift),
-                                      1u);
                         }
                         n_stage += __popc(m);
                         __syncwarp();
@@ -342,63 +342,62 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
 // uncertain keys above it; the last CTA then scans the tile counts
 // ---------------------------------------------------------------------------
 struct __align__(16) FinalSmem {
-    uint32_t buf[FINAL_KEYS];          // per-key counters (median) or 2048 bins (fallback)
+    uint32_t buf[FINAL_BINS];          // digit counts (median) or 2048 bins (fallback)
     uint32_t wtot[32];
     uint32_t out[4];
     float thr;
     uint32_t miss, last;
 };
 
-// Exact median of head h from the window keys.  False if the window missed.
+// Exact median of head h from the window keys: the key of rank
+// k = N/2 - 1 - below among the head's staged keys, by a radix select on
+// d = key - lo_key in 12-bit digits from the top of the window's span (one
+// pass over the staged keys per digit).  False if the window missed.
 __device__ bool window_median(int h, uint64_t n_per_head, float C, const WinState &w,
                               const unsigned long long *below, const unsigned long long *cand_n,
-                              const uint32_t *cand, uint64_t cand_cap, const uint32_t *fine_hist,
-                              bool amb_overflow, float *rmed, float *thr, FinalSmem &sm) {
+                              const uint32_t *cand, uint64_t cand_cap, bool amb_overflow,
+                              float *rmed, float *thr, FinalSmem &sm) {
     const long long k = (long long)(n_per_head / 2 - 1) - (long long)below[h];
     const unsigned long long nc = cand_n[h];
-    if (amb_overflow || k < 0 || (unsigned long long)k >= nc || nc > cand_cap ||
-        (1u << w.shift) > (uint32_t)FINAL_KEYS)
+    if (amb_overflow || k < 0 || (unsigned long long)k >= nc || nc > cand_cap)
         return false;                                  // (block-uniform)
-    const uint32_t *fh = fine_hist + (size_t)h * KEY_BINS;
-    block_select2<KEY_BINS, false>(fh, (uint64_t)k, (uint64_t)k, sm.wtot, sm.out);
-    const uint32_t bin_lo = w.lo_key + (sm.out[0] << w.shift);
-    const uint32_t kk = sm.out[2];                     // rank inside the fine bin
-    const uint32_t width = 1u << w.shift;
-    __syncthreads();                                   // (everyone has read out[])
-    for (uint32_t i = threadIdx.x; i < (uint32_t)FINAL_KEYS; i += WIN_THREADS) sm.buf[i] = 0;
-    __syncthreads();
-    // count every candidate key of the bin by its exact value (bf16 inputs
-    // repeat values, so a bin may hold many equal keys); 16-byte loads, U in
-    // flight per thread
+    const uint32_t span = w.hi_key - w.lo_key;         // >= 2^15
+    const int bits = 32 - __clz(span - 1);
     const uint32_t *ch = cand + (uint64_t)h * cand_cap;
     const uint4 *ch4 = reinterpret_cast<const uint4 *>(ch);
     const uint64_t n4 = nc / 4;
-    constexpr int U = 8;
-    for (uint64_t i0 = threadIdx.x; i0 < n4; i0 += (uint64_t)U * WIN_THREADS) {
-        uint4 q[U];
+    uint32_t prefix = 0;                               // digits found so far (of d)
+    uint32_t rem = (uint32_t)k;
+    for (int sh = ((bits + 11) / 12 - 1) * 12; sh >= 0; sh -= 12) {
+        for (uint32_t i = threadIdx.x; i < FINAL_BINS; i += WIN_THREADS) sm.buf[i] = 0;
+        __syncthreads();
+        const int hs = sh + 12;                        // bits above this digit
+        const uint32_t want = hs >= 32 ? 0u : prefix >> hs;
+        auto add = [&](uint32_t key) {
+            const uint32_t d = key - w.lo_key;
+            if (d < span && (hs >= 32 || (d >> hs) == want))
+                atomicAdd(&sm.buf[(d >> sh) & (FINAL_BINS - 1)], 1u);
+        };
+        constexpr int U = 8;
+        for (uint64_t i0 = threadIdx.x; i0 < n4; i0 += (uint64_t)U * WIN_THREADS) {
+            uint4 q[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint64_t i = i0 + (uint64_t)u * WIN_THREADS;
-            q[u] = i < n4 ? ch4[i] : make_uint4(bin_lo - 1u, bin_lo - 1u, bin_lo - 1u, bin_lo - 1u);
-        }
+            for (int u = 0; u < U; ++u) {
+                const uint64_t i = i0 + (uint64_t)u * WIN_THREADS;
+                q[u] = i < n4 ? ch4[i] : make_uint4(w.hi_key, w.hi_key, w.hi_key, w.hi_key);
+            }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint32_t d0 = q[u].x - bin_lo, d1 = q[u].y - bin_lo;
-            const uint32_t d2 = q[u].z - bin_lo, d3 = q[u].w - bin_lo;
-            if (d0 < width) atomicAdd(&sm.buf[d0], 1u);
-            if (d1 < width) atomicAdd(&sm.buf[d1], 1u);
-            if (d2 < width) atomicAdd(&sm.buf[d2], 1u);
-            if (d3 < width) atomicAdd(&sm.buf[d3], 1u);
+            for (int u = 0; u < U; ++u) { add(q[u].x); add(q[u].y); add(q[u].z); add(q[u].w); }
         }
+        for (uint64_t i = 4 * n4 + threadIdx.x; i < nc; i += WIN_THREADS) add(ch[i]);
+        __syncthreads();
+        block_select2<FINAL_BINS, false>(sm.buf, rem, rem, sm.wtot, sm.out);
+        prefix |= sm.out[0] << sh;
+        rem = sm.out[2];
+        __syncthreads();                               // (everyone has read out[])
     }
-    for (uint64_t i = 4 * n4 + threadIdx.x; i < nc; i += WIN_THREADS) {
-        const uint32_t d = ch[i] - bin_lo;
-        if (d < width) atomicAdd(&sm.buf[d], 1u);
-    }
-    __syncthreads();
-    block_select2<FINAL_KEYS, false>(sm.buf, kk, kk, sm.wtot, sm.out);
     if (threadIdx.x == 0) {
-        const float m = key_to_float(bin_lo + sm.out[0]);
+        const float m = key_to_float(w.lo_key + prefix);
         const float t = __fmul_rn(C, m);
         rmed[h] = m;
         thr[h] = t;
@@ -573,7 +572,7 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
            uint64_t n_tiles, uint64_t n_per_head, float C, WinState *__restrict__ win,
            const unsigned long long *__restrict__ below,
            const unsigned long long *__restrict__ cand_n, const uint32_t *__restrict__ cand,
-           uint64_t cand_cap, const uint32_t *__restrict__ fine_hist,
+           uint64_t cand_cap,
            const unsigned long long *__restrict__ amb_n, const uint2 *__restrict__ amb,
            uint64_t amb_cap, float *__restrict__ rmed, float *__restrict__ thr,
            uint32_t *__restrict__ tile_cnt, uint32_t *__restrict__ tile_off,
@@ -584,7 +583,7 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
     const WinState w = win[h];
     const unsigned long long n_amb = *amb_n;
     const bool amb_overflow = n_amb > amb_cap;
-    const bool ok = window_median(h, n_per_head, C, w, below, cand_n, cand, cand_cap, fine_hist,
+    const bool ok = window_median(h, n_per_head, C, w, below, cand_n, cand, cand_cap,
                                   amb_overflow, rmed, thr, sm);
     if (!ok) {
         if (threadIdx.x == 0) win[h].miss = 1;
@@ -652,7 +651,7 @@ static int run_front(const void *x, int B, int H, int T, int D, float C, char *w
         if (bx > bmax) bx = bmax;
         k_pass_b<DT, GRAN><<<(unsigned)bx, PB_THREADS, 0, stream>>>(
             x, H, cps, L.tiles_per_slab, L.n_tiles, win, a.below, a.cand_n, a.cand, a.cand_cap,
-            a.fine_hist, a.amb_n, a.amb, a.amb_cap, a.tile_cnt);
+            a.amb_n, a.amb, a.amb_cap, a.tile_cnt);
     }
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
@@ -670,7 +669,7 @@ static int run_finish(const void *x, int B, int H, int T, int D, float C, float 
     const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
     k_finalize<DT, GRAN><<<H, WIN_THREADS, 0, stream>>>(
         x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, a.below, a.cand_n,
-        a.cand, a.cand_cap, a.fine_hist, a.amb_n, a.amb, a.amb_cap, rmed, thr, a.tile_cnt,
+        a.cand, a.cand_cap, a.amb_n, a.amb, a.amb_cap, rmed, thr, a.tile_cnt,
         tile_off, slab_off, (uint32_t)(B * H), cap, &ctr->fin_done, st);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }

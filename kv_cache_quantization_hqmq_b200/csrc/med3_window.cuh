@@ -1,4 +1,4 @@
-// med3_window.cuh -- shared layout of the two-read Med3x pipeline
+// med3_window.cuh -- shared layout of the windowed Med3x pipeline
 // (med3_window.cu: sample, window, full pass, selection, tile offsets;
 // search.cu: the encode pass that also writes the ordered outlier list).
 #pragma once
@@ -12,16 +12,15 @@ namespace hqmq {
 constexpr int TILE_GROUPS = 32;                  // packing groups per warp tile
 constexpr int TILE_CHUNKS = TILE_GROUPS * 32;    // 1024 chunks
 constexpr int SAMPLE_PERIOD = 128;               // sample chunks 4k..4k+3 of every 128
-constexpr int KEY_BINS = 65536;                  // sample and fine histograms
+constexpr int KEY_BINS = 65536;                  // sample histogram
 constexpr int WINDOW_SIGMAS = 8;                 // half-width of the rank window
 
 // Per-head state of the rank window.
 struct WinState {
     uint32_t lo_key, hi_key;   // candidate keys: lo_key <= key < hi_key
-    uint32_t shift;            // fine bin = (key - lo_key) >> shift
     uint32_t miss;             // 1: exact fallback decides this head
     float t_lo, t_hi;          // thr is known to lie in [t_lo, t_hi]
-    uint32_t pad[2];
+    uint32_t pad[3];
 };
 
 // Counters, cleared with the histograms at the start of every call.
@@ -33,7 +32,7 @@ struct Counters {
 };
 
 struct FusedLayout {
-    uint64_t sample_hist, fine_hist, counters, win, below, cand_n, cand, amb, tile_cnt, tile_off,
+    uint64_t sample_hist, counters, win, below, cand_n, cand, amb, tile_cnt, tile_off,
         cbits, head_stat, total;
     uint64_t zero_bytes;       // [0, zero_bytes) is cleared per call
     uint64_t cand_cap;         // keys per head
@@ -63,7 +62,6 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     L.amb_cap = n_keys / 25 + 4096;              // 4% of the keys may sit in thr's band
     uint64_t off = 0;
     L.sample_hist = off; off = align256_(off + (uint64_t)H * KEY_BINS * 4);
-    L.fine_hist = off;   off = align256_(off + (uint64_t)H * KEY_BINS * 4);
     L.counters = off;    off = align256_(off + sizeof(Counters) + (uint64_t)H * 4);
     L.head_stat = off;   off = align256_(off + (uint64_t)H * 16);   // per head: non-finite, saturated
     L.zero_bytes = off;
@@ -100,7 +98,7 @@ __device__ __forceinline__ void flush_stage(uint32_t *stage, uint32_t n, int lan
 struct SpecArgs {
     const WinState *win;
     unsigned long long *below, *cand_n, *amb_n;
-    uint32_t *cand, *fine_hist, *tile_cnt;
+    uint32_t *cand, *tile_cnt;
     uint2 *amb;
     uint64_t cand_cap, amb_cap;
     uint32_t *cbits;                 // per packing group: chunks with r > t_lo
@@ -114,7 +112,6 @@ inline SpecArgs spec_args(char *ws, const FusedLayout &L) {
     a.cand_n = reinterpret_cast<unsigned long long *>(ws + L.cand_n);
     a.amb_n = reinterpret_cast<unsigned long long *>(ws + L.counters);   // Counters::amb_n
     a.cand = reinterpret_cast<uint32_t *>(ws + L.cand);
-    a.fine_hist = reinterpret_cast<uint32_t *>(ws + L.fine_hist);
     a.tile_cnt = reinterpret_cast<uint32_t *>(ws + L.tile_cnt);
     a.amb = reinterpret_cast<uint2 *>(ws + L.amb);
     a.cand_cap = L.cand_cap;

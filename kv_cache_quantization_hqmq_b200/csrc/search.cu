@@ -313,9 +313,7 @@ __device__ __forceinline__ void pack_group32(uint32_t idx, uint32_t b_rt, int la
 // speculatively: a chunk with r > t_hi (above every possible threshold) as an
 // outlier (index 0, radius 0), every other chunk as a bulk chunk; records per
 // packing group the chunks with r > t_lo.
-// LIST_FIX (after the exact threshold): for each recorded chunk, decides
-// r > thr, writes the ordered list and zeroes the codes of the outliers with
-// r <= t_hi; a head whose window missed gets the full list + encode pass.
+// (k_list_fix, after the exact threshold, then writes the list.)
 // Work: warp tiles of TILE_GROUPS consecutive packing groups; a CTA owns a
 // contiguous range of tiles and walks it slab by slab (one head at a time).
 // Packs a warp tile's indices, staged in shared memory (s_idx[k], k = the
@@ -339,7 +337,6 @@ __device__ __forceinline__ void pack_tile(const uint16_t *s_idx, uint32_t ng, in
 }
 
 constexpr int LIST_SPEC = 3;
-constexpr int LIST_FIX = 4;
 
 // Clears the b-bit index of lane `lane` in its packing group's words.
 __device__ __forceinline__ void clear_index(uint32_t *gw, uint32_t b, int lane) {
@@ -390,8 +387,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
         const float4 *cb = cb_all + (size_t)h * S;
         const uint4 *tb = tables + (size_t)h * LUT_ENTRIES;
         WinState w{};
-        if (LIST == LIST_SPEC || LIST == LIST_FIX) w = sa.win[h];
-        const bool miss = LIST == LIST_FIX && w.miss != 0;    // (block-uniform)
+        if (LIST == LIST_SPEC) w = sa.win[h];
         if (LIST == LIST_SPEC && h != stage_h) {
             if (n_stage)
                 flush_stage(stage, n_stage, lane, sa.cand_n + stage_h,
@@ -399,7 +395,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
             n_stage = 0;
             stage_h = h;
         }
-        if (ENC && h != cur_head && (LIST != LIST_FIX || miss)) {   // (block-uniform)
+        if (ENC && h != cur_head) {                      // (block-uniform)
             __syncthreads();
             for (uint32_t i = threadIdx.x; i < (n_words + 1) * 8; i += ENC_THREADS) {
                 const uint32_t id = i >> 3;
@@ -416,67 +412,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
             const uint32_t g1 = min(g0 + TILE_GROUPS, groups_per_slab);
             const uint32_t gbase = slab * groups_per_slab;
             uint32_t lpos = (LIST && LIST != LIST_SPEC) ? __ldg(tile_off + t) : 0u;   // list position
-            if (LIST == LIST_FIX && !miss) {
-                // the recorded chunks (r > t_lo) of this tile, in order: lane i
-                // reads group i's bits; candidate k (in tile order) goes to lane
-                // k mod 32, which finds its group by a search over the
-                // inclusive counts and its chunk as the group's n-th set bit
-                const uint32_t ng = g1 - g0;
-                const uint32_t gw = (uint32_t)lane < ng ? __ldg(sa.cbits + gbase + g0 + lane) : 0u;
-                const uint32_t pcount = __popc(gw);
-                uint32_t incl = pcount;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t v = __shfl_up_sync(FULL, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                const uint32_t total = __shfl_sync(FULL, incl, 31);
-                for (uint32_t k0 = 0; k0 < total; k0 += 32) {        // (warp-uniform)
-                    const uint32_t k = k0 + (uint32_t)lane;
-                    const bool c = k < total;
-                    uint32_t gl = 0;                                // first group with incl > k
-#pragma unroll
-                    for (int step = 16; step >= 1; step >>= 1) {
-                        const uint32_t v = __shfl_sync(FULL, incl, (int)(gl + step - 1));
-                        if (v <= k) gl += step;
-                    }
-                    gl &= 31u;
-                    const uint32_t ex = __shfl_sync(FULL, incl - pcount, (int)gl);
-                    const uint32_t word = __shfl_sync(FULL, gw, (int)gl);
-                    const uint32_t bit = c ? __fns(word, 0u, (int)(k - ex + 1)) : 0u;
-                    const uint32_t G = gbase + g0 + gl;
-                    const uint32_t j = G * 32 + bit;
-                    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f, r = 0.f;
-                    if (c) {
-                        RawChunk<DT> v;
-                        v.load(x, j);
-                        x0 = v.e(0); x1 = v.e(1); x2 = v.e(2); x3 = v.e(3);
-                        r = chunk_norm(x0, x1, x2, x3);
-                    }
-                    const bool o = c && r > th;
-                    const uint32_t mo = __ballot_sync(FULL, o);
-                    if (o) {
-                        const uint32_t p = lpos + __popc(mo & lt);
-                        if (p < cap32) {
-                            int sv = 0;
-                            const uint32_t h01 = f32x2_to_f16x2_sat(x0, x1, sv);
-                            const uint32_t h23 = f32x2_to_f16x2_sat(x2, x3, sv);
-                            n_sat += sv;
-                            out_idx[p] = j;
-                            reinterpret_cast<uint2 *>(out_val)[p] = make_uint2(h01, h23);
-                        }
-                        if (!(r > w.t_hi)) {                // encoded as a bulk chunk: zero it
-                            radius[j] = 0;
-                            clear_index(words + (size_t)G * b, b, (int)bit);
-                        }
-                    } else if (c && !(r > w.t_hi) && r >= 65520.0f) {
-                        ++n_sat;                             // bulk radius saturated (uncounted)
-                    }
-                    lpos += __popc(mo);
-                }
-                continue;
-            }
-            uint32_t t_def = 0, t_below = 0;                  // LIST_SPEC
+            uint32_t t_def = 0, t_below = 0, t_cbits = 0;     // LIST_SPEC
             RawChunk<DT> nxt;
             nxt.load(x, (size_t)(gbase + g0) * 32 + lane);
             for (uint32_t g = g0; g < g1; ++g) {
@@ -486,7 +422,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 if (g + 1 < g1) nxt.load(x, (size_t)j + 32);
                 float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
                 float r = chunk_norm(x0, x1, x2, x3);
-                if (LIST == HQMQ_GRAN_CHUNK + 1 || LIST == LIST_FIX) {   // ordered chunk list
+                if (LIST == HQMQ_GRAN_CHUNK + 1) {           // ordered chunk list
                     const bool o = r > th;
                     const uint32_t m = __ballot_sync(FULL, o);
                     if (o) {
@@ -530,7 +466,9 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 }
                 bool spec_cand = false;                      // LIST_SPEC: r > t_lo
                 if (LIST == LIST_SPEC) {
-                    const uint32_t key = mag_key(r);
+                    // key: r's bits (r >= 0; a NaN's bits exceed every finite
+                    // key and +inf's, as in the median's order)
+                    const uint32_t key = __float_as_uint(r);
                     t_below += key < w.lo_key ? 1u : 0u;
                     const bool in = key >= w.lo_key && key < w.hi_key;
                     const uint32_t mi = __ballot_sync(FULL, in);
@@ -540,11 +478,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                                         sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap);
                             n_stage = 0;
                         }
-                        if (in) {
-                            stage[n_stage + __popc(mi & lt)] = key;
-                            atomicAdd(sa.fine_hist + (size_t)h * KEY_BINS +
-                                          ((key - w.lo_key) >> w.shift), 1u);
-                        }
+                        if (in) stage[n_stage + __popc(mi & lt)] = key;
                         n_stage += __popc(mi);
                         __syncwarp();
                     }
@@ -552,7 +486,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                     spec_cand = r > w.t_lo;
                     t_def += dfn ? 1u : 0u;
                     const uint32_t mc = __ballot_sync(FULL, spec_cand);
-                    if (lane == 0) sa.cbits[G] = mc;
+                    if (lane == (int)(g - g0)) t_cbits = mc;       // stored per tile
                     const bool unc = spec_cand && !dfn;
                     const uint32_t mu = __ballot_sync(FULL, unc);
                     if (mu) {
@@ -648,6 +582,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                     sa.tile_cnt[t] = t_def;
                     if (t_below) atomicAdd(sa.below + h, (unsigned long long)t_below);
                 }
+                if (lane < (int)(g1 - g0)) sa.cbits[gbase + g0 + lane] = t_cbits;
             }
         }
         if (LIST == LIST_SPEC) {                             // status counts per head
@@ -667,20 +602,160 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                         sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap);
         return;
     }
-    if (LIST == LIST_FIX && blockIdx.x == 0 && st) {
-        // the encode pass's status counts of the heads whose result stands
-        for (int hh = threadIdx.x; hh < H; hh += ENC_THREADS)
-            if (!sa.win[hh].miss) {
-                const unsigned long long nf = sa.head_stat[2 * hh], ns = sa.head_stat[2 * hh + 1];
-                status_add(st, HQMQ_FLAG_NONFINITE, &st->n_nonfinite, nf);
-                status_add(st, HQMQ_FLAG_SATURATED, &st->n_saturated, ns);
+    const unsigned nf = __reduce_add_sync(FULL, n_nf);
+    const unsigned ns = __reduce_add_sync(FULL, n_sat);
+    if (lane == 0 && st) {
+        if (nf) status_add(st, HQMQ_FLAG_NONFINITE, &st->n_nonfinite, nf);
+        if (ns) status_add(st, HQMQ_FLAG_SATURATED, &st->n_saturated, ns);
+    }
+}
+
+// The list pass of the one-read chunk-mode path (after the exact threshold):
+// per tile of a head whose window held, the chunks recorded by the encode
+// pass (r > t_lo) are read again, decided (r > thr) and written to the
+// ordered list; those with r <= t_hi were encoded as bulk chunks and get
+// index 0 and radius 0.  A head whose window missed is encoded again exactly
+// (S-codeword loop, list, radius, index), as hqmq_encode does.  Also adds the
+// encode pass's status counts of the heads whose result stands.
+constexpr int FIX_THREADS = 256;
+
+template <int DT>
+__global__ void __launch_bounds__(FIX_THREADS)
+k_list_fix(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32_t tiles_per_slab,
+           uint32_t n_tiles, const float4 *__restrict__ cb_all, uint32_t S, uint32_t b,
+           const float *__restrict__ thr, uint32_t *__restrict__ words,
+           uint16_t *__restrict__ radius, const uint32_t *__restrict__ tile_off, uint64_t cap,
+           uint32_t *__restrict__ out_idx, uint16_t *__restrict__ out_val, DevStatus *st,
+           SpecArgs sa) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    const uint32_t cap32 = cap < 0xFFFFFFFFull ? (uint32_t)cap : 0xFFFFFFFFu;
+    const PackConst pc = pack_const(b, lane);
+    const uint32_t warp_g = blockIdx.x * (FIX_THREADS / 32) + (threadIdx.x >> 5);
+    const uint32_t n_warps = gridDim.x * (FIX_THREADS / 32);
+    unsigned n_nf = 0, n_sat = 0;
+    for (uint32_t t = warp_g; t < n_tiles; t += n_warps) {
+        const uint32_t slab = t / tiles_per_slab;
+        const int h = (int)(slab % (uint32_t)H);
+        const WinState w = sa.win[h];
+        const bool miss = w.miss != 0;
+        const float th = __ldg(thr + h);
+        const uint32_t g0 = (t % tiles_per_slab) * TILE_GROUPS;
+        const uint32_t g1 = min(g0 + TILE_GROUPS, groups_per_slab);
+        const uint32_t gbase = slab * groups_per_slab;
+        uint32_t lpos = __ldg(tile_off + t);
+        if (!miss) {
+            // the recorded chunks (r > t_lo) of this tile, in order: lane i
+            // reads group i's bits; candidate k (in tile order) goes to lane
+            // k mod 32, which finds its group by a search over the
+            // inclusive counts and its chunk as the group's n-th set bit
+            const uint32_t ng = g1 - g0;
+            const uint32_t gw = (uint32_t)lane < ng ? __ldg(sa.cbits + gbase + g0 + lane) : 0u;
+            const uint32_t pcount = __popc(gw);
+            uint32_t incl = pcount;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t v = __shfl_up_sync(FULL, incl, o);
+                if (lane >= o) incl += v;
             }
+            const uint32_t total = __shfl_sync(FULL, incl, 31);
+            for (uint32_t k0 = 0; k0 < total; k0 += 32) {        // (warp-uniform)
+                const uint32_t k = k0 + (uint32_t)lane;
+                const bool c = k < total;
+                uint32_t gl = 0;                                // first group with incl > k
+#pragma unroll
+                for (int step = 16; step >= 1; step >>= 1) {
+                    const uint32_t v = __shfl_sync(FULL, incl, (int)(gl + step - 1));
+                    if (v <= k) gl += step;
+                }
+                gl &= 31u;
+                const uint32_t ex = __shfl_sync(FULL, incl - pcount, (int)gl);
+                const uint32_t word = __shfl_sync(FULL, gw, (int)gl);
+                const uint32_t bit = c ? __fns(word, 0u, (int)(k - ex + 1)) : 0u;
+                const uint32_t G = gbase + g0 + gl;
+                const uint32_t j = G * 32 + bit;
+                float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f, r = 0.f;
+                if (c) {
+                    RawChunk<DT> v;
+                    v.load(x, j);
+                    x0 = v.e(0); x1 = v.e(1); x2 = v.e(2); x3 = v.e(3);
+                    r = chunk_norm(x0, x1, x2, x3);
+                }
+                const bool o = c && r > th;
+                const uint32_t mo = __ballot_sync(FULL, o);
+                if (o) {
+                    const uint32_t p = lpos + __popc(mo & lt);
+                    if (p < cap32) {
+                        int sv = 0;
+                        const uint32_t h01 = f32x2_to_f16x2_sat(x0, x1, sv);
+                        const uint32_t h23 = f32x2_to_f16x2_sat(x2, x3, sv);
+                        n_sat += sv;
+                        out_idx[p] = j;
+                        reinterpret_cast<uint2 *>(out_val)[p] = make_uint2(h01, h23);
+                    }
+                    if (!(r > w.t_hi)) {                // encoded as a bulk chunk: zero it
+                        radius[j] = 0;
+                        clear_index(words + (size_t)G * b, b, (int)bit);
+                    }
+                } else if (c && !(r > w.t_hi) && r >= 65520.0f) {
+                    ++n_sat;                             // bulk radius saturated (uncounted)
+                }
+                lpos += __popc(mo);
+            }
+            continue;
+        }
+        // a head whose window missed: exact list and encode of the tile
+        const float4 *cb = cb_all + (size_t)h * S;
+        for (uint32_t g = g0; g < g1; ++g) {
+            const uint32_t G = gbase + g;
+            const uint32_t j = G * 32 + (uint32_t)lane;
+            RawChunk<DT> v;
+            v.load(x, j);
+            const float x0 = v.e(0), x1 = v.e(1), x2 = v.e(2), x3 = v.e(3);
+            float r = chunk_norm(x0, x1, x2, x3);
+            const bool o = r > th;
+            const uint32_t m = __ballot_sync(FULL, o);
+            if (o) {
+                const uint32_t p = lpos + __popc(m & lt);
+                if (p < cap32) {
+                    int sv = 0;
+                    const uint32_t h01 = f32x2_to_f16x2_sat(x0, x1, sv);
+                    const uint32_t h23 = f32x2_to_f16x2_sat(x2, x3, sv);
+                    n_sat += sv;
+                    out_idx[p] = j;
+                    reinterpret_cast<uint2 *>(out_val)[p] = make_uint2(h01, h23);
+                }
+                r = 0.0f;                                  // outlier chunk: radius 0, index 0
+            }
+            lpos += __popc(m);
+            const bool finite = r == r && r != __int_as_float(0x7F800000);
+            const uint32_t idx = (finite && r > 0.0f) ? sloop_index(x0, x1, x2, x3, cb, S) : 0u;
+            uint16_t rh;
+            if (!finite) {
+                rh = 0x7E00u;
+                ++n_nf;
+            } else {
+                int sat = 0;
+                rh = radius_to_f16(r, sat);
+                n_sat += sat;
+            }
+            radius[j] = rh;
+            pack_group32<0>(idx, b, lane, pc, words + (size_t)G * b);
+        }
     }
     const unsigned nf = __reduce_add_sync(FULL, n_nf);
     const unsigned ns = __reduce_add_sync(FULL, n_sat);
     if (lane == 0 && st) {
         if (nf) status_add(st, HQMQ_FLAG_NONFINITE, &st->n_nonfinite, nf);
         if (ns) status_add(st, HQMQ_FLAG_SATURATED, &st->n_saturated, ns);
+    }
+    if (blockIdx.x == 0 && st) {
+        // the encode pass's status counts of the heads whose result stands
+        for (int hh = threadIdx.x; hh < H; hh += FIX_THREADS)
+            if (!sa.win[hh].miss) {
+                status_add(st, HQMQ_FLAG_NONFINITE, &st->n_nonfinite, sa.head_stat[2 * hh]);
+                status_add(st, HQMQ_FLAG_SATURATED, &st->n_saturated, sa.head_stat[2 * hh + 1]);
+            }
     }
 }
 
@@ -833,9 +908,25 @@ extern "C" int hqmq_launch_fix_pass(const void *x, int dtype, int B, int H, int 
                                     uint16_t *out_val, void *ws, hqmq_status *st, int sm_count,
                                     cudaStream_t stream) {
     using namespace hqmq;
+    (void)table;
     const SpecArgs sa = spec_args(reinterpret_cast<char *>(ws),
                                   fused_layout(B, H, T, D, HQMQ_GRAN_CHUNK));
-    return launch_lut_dt<LIST_FIX, true>(dtype, B, H, T, D, x, cb, S, b, table, thr,
-                                         HQMQ_GRAN_CHUNK, words, radius, tile_off, cap, out_idx,
-                                         out_val, st, sm_count, stream, sa);
+    const uint32_t gps = (uint32_t)(((uint64_t)T * D / 4) / 32);
+    const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
+    const uint32_t n_tiles = (uint32_t)((uint64_t)B * H * tps);
+    uint64_t ctas = (uint64_t)sm_count * 8;
+    const uint64_t want = ((uint64_t)n_tiles + FIX_THREADS / 32 - 1) / (FIX_THREADS / 32);
+    if (ctas > want) ctas = want;
+    if (ctas < 1) ctas = 1;
+    const float4 *cb4 = reinterpret_cast<const float4 *>(cb);
+    DevStatus *dst = reinterpret_cast<DevStatus *>(st);
+    if (dtype == HQMQ_BF16)
+        k_list_fix<HQMQ_BF16><<<(unsigned)ctas, FIX_THREADS, 0, stream>>>(
+            x, H, gps, tps, n_tiles, cb4, S, b, thr, words, radius, tile_off, cap, out_idx,
+            out_val, dst, sa);
+    else
+        k_list_fix<HQMQ_F32><<<(unsigned)ctas, FIX_THREADS, 0, stream>>>(
+            x, H, gps, tps, n_tiles, cb4, S, b, thr, words, radius, tile_off, cap, out_idx,
+            out_val, dst, sa);
+    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
