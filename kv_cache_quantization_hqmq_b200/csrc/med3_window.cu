@@ -41,7 +41,7 @@ namespace hqmq {
 
 constexpr int WIN_THREADS = 1024;
 constexpr int PB_THREADS = 256;
-constexpr int FINAL_BINS = 4096;   // radix digit of the exact median selection (12 bits)
+
 
 __device__ __forceinline__ float key_to_float(uint32_t k) {
     return k >= 0x7F800001u ? __int_as_float(0x7FC00000) : __uint_as_float(k);
@@ -342,69 +342,72 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
 // uncertain keys above it; the last CTA then scans the tile counts
 // ---------------------------------------------------------------------------
 struct __align__(16) FinalSmem {
-    uint32_t buf[FINAL_BINS];          // digit counts (median) or 2048 bins (fallback)
+    uint32_t buf[MED_BINS];            // digit counts (median) or 2048 bins (fallback)
     uint32_t wtot[32];
     uint32_t out[4];
-    float thr;
-    uint32_t miss, last;
+    uint32_t last;
 };
 
-// Exact median of head h from the window keys: the key of rank
-// k = N/2 - 1 - below among the head's staged keys, by a radix select on
-// d = key - lo_key in 12-bit digits from the top of the window's span (one
-// pass over the staged keys per digit).  False if the window missed.
-__device__ bool window_median(int h, uint64_t n_per_head, float C, const WinState &w,
-                              const unsigned long long *below, const unsigned long long *cand_n,
-                              const uint32_t *cand, uint64_t cand_cap, bool amb_overflow,
-                              float *rmed, float *thr, FinalSmem &sm) {
+// Exact median of head h from its staged window keys: the key of rank
+// k = N/2 - 1 - below among them, by a radix select on d = key - lo_key in
+// 12-bit digits from the top of the window's span.  The top digit's counts
+// come from all MED_SLICES finalize CTAs of the head (each counts a slice of
+// the keys into the head's global histogram); the head's last CTA selects it
+// and runs the remaining digits alone (only keys inside the chosen bin
+// count).
+struct MedianPlan {
+    bool ok;                 // false: the window missed (the exact fallback decides)
+    uint32_t k;              // rank among the staged keys
+    uint64_t nc;             // staged keys
+    uint32_t span;           // hi_key - lo_key
+    int top;                 // shift of the top digit
+};
+
+__device__ MedianPlan median_plan(int h, uint64_t n_per_head, const WinState &w,
+                                  const unsigned long long *below,
+                                  const unsigned long long *cand_n, uint64_t cand_cap,
+                                  bool amb_overflow) {
+    MedianPlan p;
     const long long k = (long long)(n_per_head / 2 - 1) - (long long)below[h];
-    const unsigned long long nc = cand_n[h];
-    if (amb_overflow || k < 0 || (unsigned long long)k >= nc || nc > cand_cap)
-        return false;                                  // (block-uniform)
-    const uint32_t span = w.hi_key - w.lo_key;         // >= 2^15
-    const int bits = 32 - __clz(span - 1);
-    const uint32_t *ch = cand + (uint64_t)h * cand_cap;
-    const uint4 *ch4 = reinterpret_cast<const uint4 *>(ch);
-    const uint64_t n4 = nc / 4;
-    uint32_t prefix = 0;                               // digits found so far (of d)
-    uint32_t rem = (uint32_t)k;
-    for (int sh = ((bits + 11) / 12 - 1) * 12; sh >= 0; sh -= 12) {
-        for (uint32_t i = threadIdx.x; i < FINAL_BINS; i += WIN_THREADS) sm.buf[i] = 0;
-        __syncthreads();
-        const int hs = sh + 12;                        // bits above this digit
-        const uint32_t want = hs >= 32 ? 0u : prefix >> hs;
-        auto add = [&](uint32_t key) {
-            const uint32_t d = key - w.lo_key;
-            if (d < span && (hs >= 32 || (d >> hs) == want))
-                atomicAdd(&sm.buf[(d >> sh) & (FINAL_BINS - 1)], 1u);
-        };
-        constexpr int U = 8;
-        for (uint64_t i0 = threadIdx.x; i0 < n4; i0 += (uint64_t)U * WIN_THREADS) {
-            uint4 q[U];
+    p.nc = cand_n[h];
+    p.ok = !(amb_overflow || k < 0 || (unsigned long long)k >= p.nc || p.nc > cand_cap);
+    p.k = p.ok ? (uint32_t)k : 0u;
+    p.span = w.hi_key - w.lo_key;                      // >= 2^15
+    const int bits = 32 - __clz(p.span - 1);
+    p.top = ((bits + 11) / 12 - 1) * 12;
+    return p;
+}
+
+// Adds the digit at shift sh of every staged key d in [i_begin, i_end) whose
+// bits above the digit equal those of `prefix` to hist (shared, MED_BINS).
+__device__ void median_count(const uint32_t *ch, uint64_t i_begin, uint64_t i_end,
+                             const WinState &w, uint32_t span, int sh, uint32_t prefix,
+                             uint32_t *hist) {
+    const int hs = sh + 12;                            // bits above this digit
+    const uint32_t want = hs >= 32 ? 0u : prefix >> hs;
+    auto add = [&](uint32_t key) {
+        const uint32_t d = key - w.lo_key;
+        if (d < span && (hs >= 32 || (d >> hs) == want))
+            atomicAdd(&hist[(d >> sh) & (MED_BINS - 1)], 1u);
+    };
+    // 16-byte loads from the first multiple of 4 at or after i_begin
+    uint64_t a = (i_begin + 3) & ~(uint64_t)3;
+    if (a > i_end) a = i_end;
+    for (uint64_t i = i_begin + threadIdx.x; i < a; i += WIN_THREADS) add(ch[i]);
+    const uint64_t n4 = (i_end - a) / 4;
+    const uint4 *ch4 = reinterpret_cast<const uint4 *>(ch + a);
+    constexpr int U = 4;
+    for (uint64_t i0 = threadIdx.x; i0 < n4; i0 += (uint64_t)U * WIN_THREADS) {
+        uint4 q[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint64_t i = i0 + (uint64_t)u * WIN_THREADS;
-                q[u] = i < n4 ? ch4[i] : make_uint4(w.hi_key, w.hi_key, w.hi_key, w.hi_key);
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) { add(q[u].x); add(q[u].y); add(q[u].z); add(q[u].w); }
+        for (int u = 0; u < U; ++u) {
+            const uint64_t i = i0 + (uint64_t)u * WIN_THREADS;
+            q[u] = i < n4 ? ch4[i] : make_uint4(w.hi_key, w.hi_key, w.hi_key, w.hi_key);
         }
-        for (uint64_t i = 4 * n4 + threadIdx.x; i < nc; i += WIN_THREADS) add(ch[i]);
-        __syncthreads();
-        block_select2<FINAL_BINS, false>(sm.buf, rem, rem, sm.wtot, sm.out);
-        prefix |= sm.out[0] << sh;
-        rem = sm.out[2];
-        __syncthreads();                               // (everyone has read out[])
+#pragma unroll
+        for (int u = 0; u < U; ++u) { add(q[u].x); add(q[u].y); add(q[u].z); add(q[u].w); }
     }
-    if (threadIdx.x == 0) {
-        const float m = key_to_float(w.lo_key + prefix);
-        const float t = __fmul_rn(C, m);
-        rmed[h] = m;
-        thr[h] = t;
-        sm.thr = t;
-    }
-    __syncthreads();
-    return true;
+    for (uint64_t i = a + 4 * n4 + threadIdx.x; i < i_end; i += WIN_THREADS) add(ch[i]);
 }
 
 // Exact three-pass radix select over x for head h, then its exact tile
@@ -572,36 +575,70 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
            uint64_t n_tiles, uint64_t n_per_head, float C, WinState *__restrict__ win,
            const unsigned long long *__restrict__ below,
            const unsigned long long *__restrict__ cand_n, const uint32_t *__restrict__ cand,
-           uint64_t cand_cap,
-           const unsigned long long *__restrict__ amb_n, const uint2 *__restrict__ amb,
-           uint64_t amb_cap, float *__restrict__ rmed, float *__restrict__ thr,
-           uint32_t *__restrict__ tile_cnt, uint32_t *__restrict__ tile_off,
-           uint32_t *__restrict__ slab_off, uint32_t n_slabs, uint64_t cap,
+           uint64_t cand_cap, const unsigned long long *__restrict__ amb_n,
+           const uint2 *__restrict__ amb, uint64_t amb_cap, float *__restrict__ rmed,
+           float *__restrict__ thr, uint32_t *__restrict__ tile_cnt,
+           uint32_t *__restrict__ tile_off, uint32_t *__restrict__ slab_off, uint32_t n_slabs,
+           uint64_t cap, uint32_t *__restrict__ med_hist, uint32_t *__restrict__ median_done,
            uint32_t *__restrict__ fin_done, DevStatus *st) {
     __shared__ FinalSmem sm;
-    const int h = blockIdx.x;
+    const int h = blockIdx.y;
     const WinState w = win[h];
     const unsigned long long n_amb = *amb_n;
-    const bool amb_overflow = n_amb > amb_cap;
-    const bool ok = window_median(h, n_per_head, C, w, below, cand_n, cand, cand_cap,
-                                  amb_overflow, rmed, thr, sm);
-    if (!ok) {
+    const MedianPlan mp = median_plan(h, n_per_head, w, below, cand_n, cand_cap,
+                                      n_amb > amb_cap);
+    const uint32_t *ch = cand + (uint64_t)h * cand_cap;
+    uint32_t *gh = med_hist + (size_t)h * MED_BINS;
+    if (mp.ok) {                                       // (block-uniform) top digit, one slice
+        for (uint32_t i = threadIdx.x; i < MED_BINS; i += WIN_THREADS) sm.buf[i] = 0;
+        __syncthreads();
+        const uint64_t i0 = mp.nc * blockIdx.x / gridDim.x, i1 = mp.nc * (blockIdx.x + 1) / gridDim.x;
+        median_count(ch, i0, i1, w, mp.span, mp.top, 0u, sm.buf);
+        __syncthreads();
+        for (uint32_t i = threadIdx.x; i < MED_BINS; i += WIN_THREADS)
+            if (sm.buf[i]) atomicAdd(gh + i, sm.buf[i]);
+    }
+    // the head's last CTA (no CTA waits for another) finishes the head
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+        sm.last = atomicAdd(median_done + h, 1u) == gridDim.x - 1 ? 1u : 0u;
+    __syncthreads();
+    if (!sm.last) return;
+    __threadfence();
+    if (!mp.ok) {
         if (threadIdx.x == 0) win[h].miss = 1;
         exact_fallback<DT, GRAN>(x, B, H, h, cps, tiles_per_slab, n_per_head, C, rmed, thr,
                                  tile_cnt, st, sm);
     } else {
+        block_select2<MED_BINS, true>(gh, mp.k, mp.k, sm.wtot, sm.out);
+        uint32_t prefix = sm.out[0] << mp.top;
+        uint32_t rem = sm.out[2];
+        __syncthreads();                               // (everyone has read out[])
+        for (int sh = mp.top - 12; sh >= 0; sh -= 12) {
+            for (uint32_t i = threadIdx.x; i < MED_BINS; i += WIN_THREADS) sm.buf[i] = 0;
+            __syncthreads();
+            median_count(ch, 0, mp.nc, w, mp.span, sh, prefix, sm.buf);
+            __syncthreads();
+            block_select2<MED_BINS, false>(sm.buf, rem, rem, sm.wtot, sm.out);
+            prefix |= sm.out[0] << sh;
+            rem = sm.out[2];
+            __syncthreads();
+        }
+        const float m = key_to_float(w.lo_key + prefix);
+        const float th = __fmul_rn(C, m);
+        if (threadIdx.x == 0) { rmed[h] = m; thr[h] = th; }
         // uncertain keys of this head above its exact threshold
-        const float th = sm.thr;
         for (uint64_t i = threadIdx.x; i < n_amb; i += WIN_THREADS) {
             const uint2 e = amb[i];
             if ((int)((e.x / tiles_per_slab) % (uint32_t)H) != h) continue;
             if (__uint_as_float(e.y) > th) atomicAdd(tile_cnt + e.x, 1u);
         }
     }
-    // the last CTA to finish (no CTA waits for another) scans the tiles
+    // the last head to finish scans the tiles
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) sm.last = atomicAdd(fin_done, 1u) == gridDim.x - 1 ? 1u : 0u;
+    if (threadIdx.x == 0) sm.last = atomicAdd(fin_done, 1u) == gridDim.y - 1 ? 1u : 0u;
     __syncthreads();
     if (!sm.last) return;
     __threadfence();
@@ -667,10 +704,12 @@ static int run_finish(const void *x, int B, int H, int T, int D, float C, float 
     Counters *ctr = reinterpret_cast<Counters *>(ws + L.counters);
     WinState *win = reinterpret_cast<WinState *>(ws + L.win);
     const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
-    k_finalize<DT, GRAN><<<H, WIN_THREADS, 0, stream>>>(
+    uint32_t *median_done = reinterpret_cast<uint32_t *>(ws + L.counters + sizeof(Counters)) + H;
+    uint32_t *med_hist = reinterpret_cast<uint32_t *>(ws + L.med_hist);
+    k_finalize<DT, GRAN><<<dim3(MED_SLICES, H), WIN_THREADS, 0, stream>>>(
         x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, a.below, a.cand_n,
-        a.cand, a.cand_cap, a.amb_n, a.amb, a.amb_cap, rmed, thr, a.tile_cnt,
-        tile_off, slab_off, (uint32_t)(B * H), cap, &ctr->fin_done, st);
+        a.cand, a.cand_cap, a.amb_n, a.amb, a.amb_cap, rmed, thr, a.tile_cnt, tile_off, slab_off,
+        (uint32_t)(B * H), cap, med_hist, median_done, &ctr->fin_done, st);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 

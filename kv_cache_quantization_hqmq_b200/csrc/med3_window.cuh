@@ -28,11 +28,15 @@ struct Counters {
     unsigned long long amb_n;  // uncertain (tile, key) pairs appended
     uint32_t fin_done;         // CTAs of the finalize step that are done
     uint32_t pad;
-    // followed by uint32_t sample_done[H]: sample CTAs of head h that are done
+    // followed by uint32_t sample_done[H]: sample CTAs of head h that are done,
+    // then uint32_t median_done[H]: finalize CTAs of head h that are done
 };
 
+constexpr int MED_SLICES = 16;                   // finalize CTAs per head
+constexpr int MED_BINS = 4096;                   // radix digit of the median select (12 bits)
+
 struct FusedLayout {
-    uint64_t sample_hist, counters, win, below, cand_n, cand, amb, tile_cnt, tile_off,
+    uint64_t sample_hist, counters, med_hist, win, below, cand_n, cand, amb, tile_cnt, tile_off,
         cbits, head_stat, total;
     uint64_t zero_bytes;       // [0, zero_bytes) is cleared per call
     uint64_t cand_cap;         // keys per head
@@ -62,7 +66,8 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     L.amb_cap = n_keys / 25 + 4096;              // 4% of the keys may sit in thr's band
     uint64_t off = 0;
     L.sample_hist = off; off = align256_(off + (uint64_t)H * KEY_BINS * 4);
-    L.counters = off;    off = align256_(off + sizeof(Counters) + (uint64_t)H * 4);
+    L.counters = off;    off = align256_(off + sizeof(Counters) + (uint64_t)H * 8);
+    L.med_hist = off;    off = align256_(off + (uint64_t)H * MED_BINS * 4);
     L.head_stat = off;   off = align256_(off + (uint64_t)H * 16);   // per head: non-finite, saturated
     L.zero_bytes = off;
     L.win = off;         off = align256_(off + (uint64_t)H * sizeof(WinState));
