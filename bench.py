@@ -372,7 +372,7 @@ def run_hqmq(args):
             name = "k_encode_lut"
         elif one_read(w, cache.table is not None):
             name = ("hqmq_encode_med3 (one read of x: k_sample_window, k_encode_lut speculative "
-                    "encode, k_finalize, k_encode_lut fix-up)")
+                    "encode, k_finalize, k_list_fix)")
         else:
             name = "hqmq_encode_med3 (two reads of x: k_sample_window, k_pass_b, k_finalize, k_encode_lut)"
         roof = {"kernel": name, "bound": "hbm", "achieved": kern[enc_key]["hbm_gbs"],
