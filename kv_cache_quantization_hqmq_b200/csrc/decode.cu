@@ -9,11 +9,11 @@
 // k_decode: each CTA owns one slab (b, h), builds that head's 24 S codeword
 // table in shared memory once (S <= 170; larger S recomputes the codeword
 // per chunk) and streams its chunks in units of 8 packing groups: the unit's
-// index words staged in shared memory, one radius per lane and group, 4
-// products and one 8-byte (bf16) store per chunk; no block barriers after the
-// table build.  Outlier list entries overwrite their chunk (chunk mode) or
-// add the fp16 value to the recomputed fl32(r * c) of their element (element
-// mode):
+// index words staged in shared memory, one radius pair per lane and 64
+// chunks, 8 products and one 16-byte (bf16) store per chunk pair; no block
+// barriers after the table build.  Outlier list entries overwrite their
+// chunk (chunk mode) or add the fp16 value to the recomputed fl32(r * c) of
+// their element (element mode):
 //  * with the list's tile offsets (the list position of each 1024-chunk
 //    tile's first entry), inside k_decode: the warp that wrote a 256-chunk
 //    quarter writes the entries of that quarter after a __syncwarp();
@@ -57,10 +57,11 @@ __device__ __forceinline__ float element_with_outlier(const uint32_t *__restrict
 
 // Main pass: every chunk -> round(fl32(r * c_i)).  A warp takes units of
 // DEC_UNIT packing groups (256 chunks) of one slab: it stages the unit's
-// index words in shared memory (coalesced loads), loads the unit's radii
-// (lane k: chunk k of each group, all in flight), then per group lane k
-// extracts its index from two staged words, multiplies and stores its chunk
-// (a warp store covers the group's 32 chunks).
+// index words in shared memory (coalesced loads) and loads the unit's radii
+// (lane k: chunks 2k and 2k+1 of each 64-chunk half, one 4-byte load each,
+// all in flight); per half, lane k extracts its two indices from the staged
+// words, multiplies and stores its two chunks with one 16-byte (bf16) store
+// (a warp store covers the half's 64 chunks).
 // LISTED: 0 = no list here, HQMQ_GRAN_CHUNK + 1 / HQMQ_GRAN_ELEMENT + 1 =
 // apply the list of that granularity through its tile offsets: after a unit's
 // stores and a __syncwarp(), the warp writes the entries of its tile that
@@ -91,8 +92,6 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
     const uint32_t gps = chunks_per_slab / 32;
     const uint64_t gs0 = (uint64_t)slab * gps;     // the slab's first packing group
     const uint32_t n_units = (gps + DEC_UNIT - 1) / DEC_UNIT;
-    const uint32_t lbit = (uint32_t)lane * b, lw = lbit >> 5, lo = lbit & 31u;
-    const bool two = lo + b > 32u;                 // index spans two words
     const uint32_t mask = (1u << b) - 1u;
     const uint32_t warp_g = blockIdx.x * (DEC_THREADS / 32) + (uint32_t)warp;
     const uint32_t n_warps = gridDim.x * (DEC_THREADS / 32);
@@ -101,39 +100,69 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
         const uint32_t g0 = un * DEC_UNIT;
         const uint32_t ng = min((uint32_t)DEC_UNIT, gps - g0);
         const uint64_t gg0 = gs0 + g0;             // global packing group of the unit
-        uint32_t rr[DEC_UNIT];
+        // lane k: chunks 2k, 2k+1 of each 64-chunk half of the unit (u < 4):
+        // one 4-byte radius pair, one 16-byte (bf16) store per lane
+        uint32_t rr[DEC_UNIT / 2];
 #pragma unroll
-        for (int u = 0; u < DEC_UNIT; ++u)         // radii: all in flight
-            rr[u] = (uint32_t)u < ng ? __ldcs(radius + (gg0 + u) * 32 + lane) : 0u;
+        for (int u = 0; u < DEC_UNIT / 2; ++u)     // radius pairs: all in flight
+            rr[u] = (uint32_t)(2 * u) < ng
+                        ? __ldcs(reinterpret_cast<const uint32_t *>(radius + gg0 * 32) + u * 32 + lane)
+                        : 0u;
         __syncwarp();                              // (the previous unit's reads of s_w)
         for (uint32_t i = lane; i < ng * b; i += 32) s_w[i] = __ldg(words + gg0 * b + i);
         __syncwarp();
 #pragma unroll
-        for (int u = 0; u < DEC_UNIT; ++u) {
-            if ((uint32_t)u >= ng) break;
-            const uint32_t *sw = s_w + u * b + lw;
-            const uint32_t ix = __funnelshift_r(sw[0], two ? sw[1] : 0u, lo) & mask;
-            float r = f16_bits_to_f32(rr[u]);
-            float4 cw;
-            if (ix < n_words) {
-                cw = TABLE ? s_tab[ix] : codeword((int)(ix % 24u), __ldg(cb + ix / 24u));
+        for (int u = 0; u < DEC_UNIT / 2; ++u) {
+            if ((uint32_t)(2 * u) >= ng) break;
+            const uint32_t c = (uint32_t)u * 64 + 2u * lane;        // chunk within the unit
+            uint32_t ixs[2];
+            if (b <= 16) {                         // both indices from one 64-bit window
+                const uint32_t bit = c * b, o = bit & 31u;
+                const uint32_t *sw = s_w + (bit >> 5);
+                const uint64_t w64 = (uint64_t)sw[0] | ((uint64_t)(o + 2 * b > 32u ? sw[1] : 0u) << 32);
+                ixs[0] = (uint32_t)(w64 >> o) & mask;
+                ixs[1] = (uint32_t)(w64 >> (o + b)) & mask;
             } else {
-                cw = make_float4(0.f, 0.f, 0.f, 0.f);
-                r = 0.0f;
-                ++n_bad;
+#pragma unroll
+                for (int v = 0; v < 2; ++v) {
+                    const uint32_t bit = (c + v) * b, o = bit & 31u;
+                    const uint32_t *sw = s_w + (bit >> 5);
+                    ixs[v] = __funnelshift_r(sw[0], o + b > 32u ? sw[1] : 0u, o) & mask;
+                }
             }
-            const uint64_t j = (gg0 + u) * 32 + lane;
-            const float o0 = __fmul_rn(r, cw.x), o1 = __fmul_rn(r, cw.y);
-            const float o2 = __fmul_rn(r, cw.z), o3 = __fmul_rn(r, cw.w);
+            float out[8];
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+                float r = f16_bits_to_f32(v ? (rr[u] >> 16) : (rr[u] & 0xFFFFu));
+                float4 cw;
+                if (ixs[v] < n_words) {
+                    cw = TABLE ? s_tab[ixs[v]] : codeword((int)(ixs[v] % 24u), __ldg(cb + ixs[v] / 24u));
+                } else {
+                    cw = make_float4(0.f, 0.f, 0.f, 0.f);
+                    r = 0.0f;
+                    ++n_bad;
+                }
+                out[4 * v] = __fmul_rn(r, cw.x);
+                out[4 * v + 1] = __fmul_rn(r, cw.y);
+                out[4 * v + 2] = __fmul_rn(r, cw.z);
+                out[4 * v + 3] = __fmul_rn(r, cw.w);
+            }
+            const uint64_t j = gg0 * 32 + c;
             if (OUT_DT == HQMQ_BF16) {
-                __nv_bfloat162 a0 = __floats2bfloat162_rn(o0, o1);
-                __nv_bfloat162 a1 = __floats2bfloat162_rn(o2, o3);
-                uint2 q;
+                __nv_bfloat162 a0 = __floats2bfloat162_rn(out[0], out[1]);
+                __nv_bfloat162 a1 = __floats2bfloat162_rn(out[2], out[3]);
+                __nv_bfloat162 a2 = __floats2bfloat162_rn(out[4], out[5]);
+                __nv_bfloat162 a3 = __floats2bfloat162_rn(out[6], out[7]);
+                uint4 q;
                 q.x = *reinterpret_cast<uint32_t *>(&a0);
                 q.y = *reinterpret_cast<uint32_t *>(&a1);
-                reinterpret_cast<uint2 *>(y)[j] = q;
+                q.z = *reinterpret_cast<uint32_t *>(&a2);
+                q.w = *reinterpret_cast<uint32_t *>(&a3);
+                reinterpret_cast<uint4 *>(y)[j >> 1] = q;
             } else {
-                reinterpret_cast<float4 *>(y)[j] = make_float4(o0, o1, o2, o3);
+                float4 *yp = reinterpret_cast<float4 *>(y) + j;
+                yp[0] = make_float4(out[0], out[1], out[2], out[3]);
+                yp[1] = make_float4(out[4], out[5], out[6], out[7]);
             }
         }
         if (LISTED) {
