@@ -177,10 +177,16 @@ k_build_search_table(const float4 *__restrict__ cb_all, uint32_t S, uint4 *__res
 // encode with the table
 // ---------------------------------------------------------------------------
 
+// Cell index along one axis: floor((u(t) + 1) G / 2), as
+// v = t (A G/2 + B G/2 t^2) + G/2 (the G/2 scalings are exact).  |t| <= 1 up
+// to the rounding of t, so v >= -1e-6 truncates to 0; only the top needs a
+// clamp.  (Points within the cells' widening of a boundary may land on either
+// side: both cells list every codeword that can win there.)
 __device__ __forceinline__ int cell_coord(float t) {
-    const float u = t * __fmaf_rn(MAP_B, t * t, MAP_A);
-    int i = (int)((u + 1.0f) * (0.5f * LUT_G));
-    return i < 0 ? 0 : (i > LUT_G - 1 ? LUT_G - 1 : i);
+    constexpr float HG = 0.5f * LUT_G;
+    const float v = __fmaf_rn(t, __fmaf_rn(MAP_B * HG, t * t, MAP_A * HG), HG);
+    const int i = (int)v;
+    return i > LUT_G - 1 ? LUT_G - 1 : i;
 }
 
 // S-codeword loop for one chunk (used for OVERFLOW cells); same result rules
