@@ -301,6 +301,60 @@ def elapsed_ms(pairs):
     return [a.elapsed_time(b) for a, b in pairs]
 
 
+def kernel_stats(w, timers, peaks, n_out, table):
+    """Per-call time and algorithmic HBM rate of each timed call family."""
+    ab = algorithmic_bytes(w, n_out, table)
+    kern = {}
+    for name in ("med3_encode", "encode", "decode"):
+        if not timers[name]:
+            continue
+        t = statistics.mean(elapsed_ms(timers[name]))
+        gbs = ab[name] / (t * 1e-3) / 1e9
+        kern[name] = {"ms_per_call": round(t, 4), "calls_per_step": w.n_calls,
+                      "algorithmic_bytes_per_call": int(ab[name]),
+                      "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+                      "bf16_gbs": round(w.call_elems * w.elem_bytes / (t * 1e-3) / 1e9, 1)}
+    return kern
+
+
+# the other workloads of the metric (S = 8 and S = 32), measured after the
+# headline one: per call encode and decode rates
+SWEEP = ("llama3_8b", "qwen_outlier", "mha7b_s8", "mha7b_s32")
+
+
+def run_sweep(device, peaks, steps=3, warmup=3):
+    import torch
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    from kv_cache_quantization_hqmq_b200 import workloads as W
+    out = {}
+    for name in SWEEP:
+        w = W.WORKLOADS[name]
+        cache = Cache(w, 0, device)
+        cache.setup()
+        for _ in range(warmup):
+            cache.step()
+        torch.cuda.synchronize()
+        st = hqmq.read_status(cache.status)
+        timers = {"med3_encode": [], "encode": [], "decode": []}
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            cache.step(timers)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        n_out = st["n_outliers"] / max(1, warmup) / w.n_calls if w.med3 else 0.0
+        out[name] = {"S": w.S, "med3": ("chunk, C=%g" % w.C) if w.med3 else "off",
+                     "cache_gb": round(w.cache_bytes / 1e9, 2), "ms_per_step": round(ms, 3),
+                     "value_gbs": round(w.cache_bytes / (ms * 1e-3) / 1e9, 2),
+                     "kernels": kernel_stats(w, timers, peaks, n_out, cache.table is not None),
+                     "status_flags": st["flags"]}
+        del cache
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_hqmq(args):
     import torch
     rank, world, dist = dist_setup(args.gpus)
@@ -342,17 +396,7 @@ def run_hqmq(args):
     ms_step = ms_total / args.steps
 
     n_out = st["n_outliers"] / max(1, args.warmup) / w.n_calls if w.med3 else 0.0
-    ab = algorithmic_bytes(w, n_out, cache.table is not None)
-    kern = {}
-    for name in ("med3_encode", "encode", "decode"):
-        if not timers[name]:
-            continue
-        t = statistics.mean(elapsed_ms(timers[name]))
-        gbs = ab[name] / (t * 1e-3) / 1e9
-        kern[name] = {"ms_per_call": round(t, 4), "calls_per_step": w.n_calls,
-                      "algorithmic_bytes_per_call": int(ab[name]),
-                      "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
-                      "bf16_gbs": round(w.call_elems * w.elem_bytes / (t * 1e-3) / 1e9, 1)}
+    kern = kernel_stats(w, timers, peaks, n_out, cache.table is not None)
     B, H, T, D = w.call_shape
     n_chunks = B * H * T * D // 4
     enc_key = "med3_encode" if w.med3 else "encode"
@@ -415,6 +459,11 @@ def run_hqmq(args):
         "gpu_launches": cache.kernels_per_step() * args.steps,
         "clocks": clk,
     }
+    if world == 1 and not args.no_sweep:
+        # the metric's other workloads, after the headline's buffers are freed
+        del cache
+        torch.cuda.empty_cache()
+        line["per_config"] = run_sweep(device, peaks)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -587,6 +636,8 @@ def main():
     ap.add_argument("--impl", default="hqmq", choices=["hqmq", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-config encode/decode rates of the other workloads")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     args = ap.parse_args()
     if args.impl == "reference":
