@@ -298,6 +298,58 @@ HQMQ_API int hqmq_outlier_extract_noalloc(const void *d_x, int dtype, int B, int
                                           uint32_t *d_slab_off, uint64_t cap,
                                           hqmq_status *d_status, void *stream);
 
+/* One coded K or V cache for hqmq_attention_decode: HOST struct of DEVICE
+ * pointers, each as written by hqmq_encode / hqmq_encode_med3 for a
+ * [B][Hk][T][128] tensor (idx_words, radius 16-byte aligned; codebook fp32
+ * [Hk][S][4], 16-byte aligned).  out_idx == NULL: no outlier list; else
+ * out_val (8-byte aligned), tile_off (uint32 [hqmq_list_tiles(B,Hk,T,128) +
+ * 1]) and cap are the list, its tile offsets and the cap of that call, gran
+ * its granularity. */
+typedef struct {
+    const uint32_t *idx_words;
+    const uint16_t *radius;
+    const float *codebook;
+    const uint32_t *out_idx;
+    const uint16_t *out_val;
+    const uint32_t *tile_off;
+    uint64_t cap;
+    int gran;
+} hqmq_kv_codes;
+
+/* Bytes of device workspace hqmq_attention_decode needs for B x Hk KV heads
+ * (per-head counters plus room for 1024 partial results of 8 x 130 floats;
+ * about 4.3 MB). */
+HQMQ_API uint64_t hqmq_attention_workspace_size(int B, int Hk);
+
+/* Decode-phase attention read straight from the codes: the decoder runs
+ * inside the attention loop (gist.science/nl, Technische Samenvatting,
+ * "Memory en Latentie"), so the dense K and V are never written.
+ * For each batch b, query head h (GQA: KV head hk = h / G, G = Hq / Hk, so
+ * query heads hk*G .. hk*G + G - 1 share KV head hk):
+ *   K^, V^ = exactly what hqmq_decode writes as bf16 for the two caches
+ *            (codes, radius and outlier list);
+ *   s_t    = scale * <q[b][h], K^[b][hk][t]>, for t < len_b;
+ *   o[b][h] = sum_t softmax(s)_t V^[b][hk][t],
+ * with len_b = d_seq_len[b] clamped to [0, T] (NULL: len_b = T; len_b = 0
+ * gives o = 0).  Computation: per 16-token block the codes are decoded in
+ * registers straight into tensor-core operands; q K^T with bf16 products
+ * accumulated in fp32; softmax in base 2 with a running maximum; the
+ * weights enter P V as two bf16 terms (about 16 significant bits) with fp32
+ * accumulation; the token range of a KV head is split over CTAs whose
+ * partial (max, sum, P V) are merged by the last of them.  An index >= 24 S
+ * reads as the zero codeword (r * 0); unlike hqmq_decode, this call does not
+ * flag it.
+ * d_q: bf16 [B][Hq][128], 8-byte aligned.  d_o: [B][Hq][128] of out_dtype
+ * (HQMQ_BF16 or HQMQ_F32), 4-byte aligned.  d_seq_len: int32 [B] or NULL.
+ * D must be 128 and G <= 8; S in [1, 65535]; scale finite.  d_ws: at least
+ * hqmq_attention_workspace_size(B, Hk) bytes, 256-byte aligned, contents on
+ * entry ignored (the call clears what it needs). */
+HQMQ_API int hqmq_attention_decode(const uint16_t *d_q, const int32_t *d_seq_len,
+                                   const hqmq_kv_codes *k, const hqmq_kv_codes *v, uint32_t S,
+                                   int B, int Hq, int Hk, int T, int D, float scale, void *d_o,
+                                   int out_dtype, void *d_ws, uint64_t ws_bytes,
+                                   hqmq_status *d_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

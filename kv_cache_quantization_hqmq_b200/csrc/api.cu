@@ -58,6 +58,12 @@ extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int
                                      uint32_t *out_idx, uint16_t *out_val, hqmq_status *st,
                                      int sm_count, cudaStream_t stream);
 extern "C" uint64_t hqmq_lut_bytes_per_group(uint32_t S);
+extern "C" uint64_t hqmq_attn_workspace_bytes(int B, int Hk);
+extern "C" int hqmq_launch_attention(const uint16_t *q, const int *seq_len, const hqmq_kv_codes *k,
+                                     const hqmq_kv_codes *v, uint32_t S, uint32_t b, int B,
+                                     int Hk, int G, int T, float scale, void *o, int out_dtype,
+                                     void *ws, hqmq_status *st, int sm_count, int smem_optin,
+                                     cudaStream_t stream);
 extern "C" int hqmq_launch_build_search_table(const float *cb, uint32_t S, uint32_t n_groups,
                                               void *table, cudaStream_t stream);
 extern "C" int hqmq_launch_encode_lut(const void *x, int dtype, int B, int H, int T, int D,
@@ -101,6 +107,32 @@ int sm_count() {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
     if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
     return n;
+}
+
+// Opt-in shared memory per block of the current device, cached per device id.
+int smem_optin() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < 64) {
+        int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return -1;
+    if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// A coded cache of hqmq_attention_decode: pointers present and aligned.
+int kv_codes_check(const hqmq_kv_codes *c) {
+    if (!c || !c->idx_words || !c->radius || !c->codebook) return HQMQ_ERR_ARG;
+    if (c->out_idx && (!c->out_val || !c->tile_off || !gran_ok(c->gran))) return HQMQ_ERR_ARG;
+    if (!aligned(c->idx_words, 4) || !aligned(c->radius, 16) || !aligned(c->codebook, 16) ||
+        !aligned(c->out_idx, 4) || !aligned(c->out_val, 8) || !aligned(c->tile_off, 4))
+        return HQMQ_ERR_ALIGN;
+    return HQMQ_OK;
 }
 
 }  // namespace
@@ -304,6 +336,33 @@ int hqmq_encode_lut(const void *d_x, int dtype, int B, int H, int T, int D,
     return hqmq_launch_encode_lut(d_x, dtype, B, H, T, D, d_codebook, S, hqmq_index_bits(S),
                                   d_table, d_thr, gran, d_idx_words, d_radius, d_status, sm,
                                   (cudaStream_t)stream);
+}
+
+uint64_t hqmq_attention_workspace_size(int B, int Hk) {
+    if (B <= 0 || Hk <= 0 || (uint64_t)B * Hk > 65535) return 0;
+    return hqmq_attn_workspace_bytes(B, Hk);
+}
+
+int hqmq_attention_decode(const uint16_t *d_q, const int32_t *d_seq_len, const hqmq_kv_codes *k,
+                          const hqmq_kv_codes *v, uint32_t S, int B, int Hq, int Hk, int T, int D,
+                          float scale, void *d_o, int out_dtype, void *d_ws, uint64_t ws_bytes,
+                          hqmq_status *d_status, void *stream) {
+    if (D != 128 || !shape_ok(B, Hk, T, D) || !dtype_ok(out_dtype)) return HQMQ_ERR_ARG;
+    if (Hq <= 0 || Hq % Hk != 0 || Hq / Hk > 8) return HQMQ_ERR_ARG;
+    if (S < 1 || S > S_MAX || !(scale == scale) || scale - scale != 0.0f) return HQMQ_ERR_ARG;
+    if (!d_q || !d_o || !d_ws) return HQMQ_ERR_ARG;
+    int rc = kv_codes_check(k);
+    if (rc == HQMQ_OK) rc = kv_codes_check(v);
+    if (rc != HQMQ_OK) return rc;
+    if (!aligned(d_q, 8) || !aligned(d_o, 4) || !aligned(d_seq_len, 4) || !aligned(d_ws, 256) ||
+        !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    if (ws_bytes < hqmq_attn_workspace_bytes(B, Hk)) return HQMQ_ERR_WORKSPACE;
+    const int sm = sm_count(), optin = smem_optin();
+    if (sm <= 0 || optin <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_attention(d_q, d_seq_len, k, v, S, hqmq_index_bits(S), B, Hk, Hq / Hk, T,
+                                 scale, d_o, out_dtype, d_ws, d_status, sm, optin,
+                                 (cudaStream_t)stream);
 }
 
 }  // extern "C"

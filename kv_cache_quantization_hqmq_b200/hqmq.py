@@ -59,6 +59,9 @@ _SIGS = {
     "hqmq_search_table_bytes": (_U64, [_U32]),
     "hqmq_make_search_table": (_I, [_P, _U32, _U32, _P, _P]),
     "hqmq_encode_lut": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _P, _I, _P, _P, _P, _P]),
+    "hqmq_attention_workspace_size": (_U64, [_I, _I]),
+    "hqmq_attention_decode": (_I, [_P, _P, _P, _P, _U32, _I, _I, _I, _I, _I, _F, _P, _I, _P,
+                                   _U64, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -207,6 +210,48 @@ def hqmq_decode(idx_words, radius, codebook, S, out_idx, out_val, slab_off, cap,
         _ptr(idx_words), _ptr(radius), _ptr(codebook), S, _ptr(out_idx), _ptr(out_val),
         _ptr(slab_off), _ptr(tile_off), int(cap), gran, B, H, T, D, _ptr(y), _dtype_code(y),
         _ptr(status), _stream(stream)))
+
+
+class KVCodes(ctypes.Structure):
+    """hqmq_kv_codes: one coded K or V cache (device pointers)."""
+    _fields_ = [("idx_words", _P), ("radius", _P), ("codebook", _P), ("out_idx", _P),
+                ("out_val", _P), ("tile_off", _P), ("cap", _U64), ("gran", _I)]
+
+
+def kv_codes(idx_words, radius, codebook, out_idx=None, out_val=None, tile_off=None, cap=0,
+             gran=HQMQ_GRAN_CHUNK):
+    """The hqmq_kv_codes record of one coded cache (the tensors must outlive
+    the calls that use it)."""
+    c = KVCodes(_ptr(idx_words), _ptr(radius), _ptr(codebook), _ptr(out_idx), _ptr(out_val),
+                _ptr(tile_off), int(cap) if out_idx is not None else 0, int(gran))
+    c._keep = (idx_words, radius, codebook, out_idx, out_val, tile_off)
+    return c
+
+
+def hqmq_attention_workspace_size(B, Hk):
+    return int(_lib.hqmq_attention_workspace_size(B, Hk))
+
+
+def hqmq_attention_decode(q, k, v, S, Hk, T, o, ws, scale=None, seq_len=None, status=None,
+                          stream=None):
+    """o[b, h] = softmax(scale q[b, h] K^T) V over the first seq_len[b] tokens
+    of the coded caches k, v (KVCodes from kv_codes; [B, Hk, T, 128]).
+    q: bf16 [B, Hq, 128]; o: bf16 or fp32 [B, Hq, 128]; seq_len: int32 [B]
+    or None; scale defaults to 1/sqrt(128)."""
+    if q.dim() != 3 or q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bf16 [B, Hq, D] tensor")
+    B, Hq, D = (int(v_) for v_ in q.shape)
+    if scale is None:
+        scale = D ** -0.5
+    _check("hqmq_attention_decode", _lib.hqmq_attention_decode(
+        _ptr(q), _ptr(seq_len), ctypes.byref(k), ctypes.byref(v), S, B, Hq, Hk, T, D,
+        float(scale), _ptr(o), _dtype_code(o), _ptr(ws), ws.numel() * ws.element_size(),
+        _ptr(status), _stream(stream)))
+    return o
+
+
+def alloc_attention_ws(B, Hk, device="cuda"):
+    return torch.empty(hqmq_attention_workspace_size(B, Hk), dtype=torch.uint8, device=device)
 
 
 # ---------------------------------------------------------------- buffers

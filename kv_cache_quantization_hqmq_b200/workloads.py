@@ -47,6 +47,8 @@ class Workload:
     input_seed: int = 0
     codebook_seed: int = 1
     channel_seed: int = 2
+    q_heads: int = 0      # query heads per layer (GQA); 0 = heads (MHA)
+    query_seed: int = 3
     note: str = field(default="", compare=False)
 
     @property
@@ -81,6 +83,10 @@ class Workload:
         """Codebook groups: one per (layer, role, head)."""
         return self.layers * 2 * self.heads
 
+    @property
+    def n_q_heads(self):
+        return self.q_heads if self.q_heads > 0 else self.heads
+
     def n_outlier_channels(self):
         if self.channel_frac <= 0:
             return 0
@@ -101,9 +107,10 @@ WORKLOADS = {
     "tiny": Workload("tiny", 1, 1, 128, 1, 256, "f32", 8, False, "normal",
                      note="1 layer x 1 KV head x 128, 256 tokens, fp32 N(0,1), S=8, no Med3x"),
     "llama3_8b": Workload("llama3_8b", 32, 8, 128, 1, 8192, "bf16", 8, False, "normal",
+                          q_heads=32,
                           note="Llama-3-8B GQA cache, 8192 tokens, bf16 N(0,1), S=8"),
     "qwen_outlier": Workload("qwen_outlier", 28, 4, 128, 1, 32768, "bf16", 32, True, "student_t3",
-                             channel_frac=0.02, channel_scale=50.0,
+                             channel_frac=0.02, channel_scale=50.0, q_heads=28,
                              note="Qwen-class GQA cache, 32768 tokens, bf16 t(3), 2% channels x50, "
                                   "Med3x C=3, S=32"),
     "mha7b_s8": Workload("mha7b_s8", 32, 32, 128, 8, 4096, "bf16", 8, True, "lognormal_scale",
@@ -114,13 +121,14 @@ WORKLOADS = {
                                "scales, Med3x, S=32"),
     "llama3_70b_128k": Workload("llama3_70b_128k", 80, 8, 128, 1, 131072, "bf16", 32, True,
                                 "normal_channels", channel_frac=0.01, channel_scale=30.0,
+                                q_heads=64,
                                 note="Llama-3-70B GQA cache, 131072 tokens (42.95 GB K+V bf16), "
                                      "1% channels x30, Med3x C=3, S=32, layer by layer"),
     # one layer (K and V) of the Llama-3-70B 128k cache: the same calls and
     # kernels at 537 MB, small enough for a full ncu capture
     "llama3_70b_128k_1layer": Workload("llama3_70b_128k_1layer", 1, 8, 128, 1, 131072, "bf16", 32,
                                        True, "normal_channels", channel_frac=0.01,
-                                       channel_scale=30.0,
+                                       channel_scale=30.0, q_heads=64,
                                        note="one layer of the Llama-3-70B 128k cache (profiling)"),
 }
 
@@ -172,6 +180,18 @@ def make_call_input(w: Workload, layer: int, role: int, device="cpu",
             mult[0, h, 0, ch] = w.channel_scale
         x.mul_(mult.to(device))
     return x.to(w.torch_dtype).contiguous()
+
+
+def make_query(w: Workload, layer: int, device="cpu", batch: int | None = None,
+               step: int = 0) -> torch.Tensor:
+    """The bf16 [B, Hq, D] query of one decode step of one layer: N(0, 1)
+    (the pages give no query statistics; a trained model's queries are not
+    available here)."""
+    B = w.batch if batch is None else batch
+    g = _gen(device, _call_seed(w.query_seed, layer, 0) + 7919 * step)
+    q = torch.randn((B, w.n_q_heads, w.head_dim), generator=g, device=device,
+                    dtype=torch.float32)
+    return q.to(torch.bfloat16).contiguous()
 
 
 def as_numpy_bits(x: torch.Tensor):

@@ -317,3 +317,35 @@ def decode(words, radius, codebook, S, B, H, T, D, out_idx=None, out_val=None,
     lib().oracle_decode(_ptr(words), _ptr(radius), _ptr(cb), int(S), _ptr(oi), _ptr(ov), n_out,
                         gran, B, H, T, D, _ptr(y), out_dtype, ctypes.byref(st))
     return y, st.as_dict()
+
+
+def attention_decode(q_bits, k_hat, v_hat, scale, G, seq_len=None):
+    """Decode-phase attention over decoded caches, in fp64 (numpy).
+
+    The pages run their decoder inside the attention kernel
+    (gist.science/nl, Technische Samenvatting, "Memory en Latentie"); what
+    that kernel feeds is plain scaled dot-product attention of one new query
+    token per sequence over the decoded keys and values.  Written out:
+      q      = the bf16 query values, q_bits uint16 [B, Hq, D];
+      K, V   = k_hat / v_hat [B, Hk, T, D] (the decoded values, any float type);
+      len_b  = seq_len[b] clamped to [0, T] (None: T);
+      for query head h the KV head is h // G (G consecutive query heads share
+      one KV head);
+      s_t    = scale * <q[b, h], K[b, h // G, t]>, t < len_b;
+      o[b, h] = sum_t exp(s_t) V[b, h // G, t] / sum_t exp(s_t)   (0 if len_b = 0).
+    The maximum of s is subtracted before exp (the ratio is unchanged)."""
+    q = bf16_to_f32(np.asarray(q_bits, np.uint16)).astype(np.float64)
+    B, Hq, D = q.shape
+    T = k_hat.shape[2]
+    o = np.zeros((B, Hq, D), np.float64)
+    for b in range(B):
+        n = T if seq_len is None else min(max(int(seq_len[b]), 0), T)
+        if n == 0:
+            continue
+        for h in range(Hq):
+            K = np.asarray(k_hat[b, h // G, :n], np.float64)
+            V = np.asarray(v_hat[b, h // G, :n], np.float64)
+            s = scale * (K @ q[b, h])
+            w = np.exp(s - s.max())
+            o[b, h] = (w @ V) / w.sum()
+    return o
