@@ -319,6 +319,78 @@ def kernel_stats(w, timers, peaks, n_out, table):
 
 # the other workloads of the metric (S = 8 and S = 32), measured after the
 # headline one: per call encode and decode rates
+def run_attention(cache, peaks, iters=20, warmup=3):
+    """Decode-phase attention read straight from the codes of layer 0 (one
+    query token per sequence), timed with CUDA events; inputs (one layer's
+    codes) are larger than L2.  Context: torch SDPA over the same layer
+    decoded to dense bf16 (a library kernel)."""
+    import torch
+    import torch.nn.functional as F
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    from kv_cache_quantization_hqmq_b200 import workloads as W
+    w = cache.w
+    B, H, T, D = w.call_shape
+    Hq = w.n_q_heads
+    if D != 128 or Hq % H or Hq // H > 8:
+        return None
+    dev = cache.x.device
+    cbs, kv, dense, n_list = [], [], [], 0
+    for r in range(2):
+        cb = cache.codebook[r * H * w.S * 4:(r + 1) * H * w.S * 4]
+        y = torch.empty(cache.shape, dtype=torch.bfloat16, device=dev)
+        if w.med3:
+            kv.append(hqmq.kv_codes(cache.words[0, r], cache.radius[0, r], cb, cache.out_idx[0, r],
+                                    cache.out_val[0, r], cache.tile_off[0, r], cache.cap, cache.gran))
+            hqmq.hqmq_decode(cache.words[0, r], cache.radius[0, r], cb, w.S, cache.out_idx[0, r],
+                             cache.out_val[0, r], cache.slab_off[0, r], cache.cap, cache.gran, y,
+                             tile_off=cache.tile_off[0, r])
+            n_list += int(cache.slab_off[0, r][-1].item())
+        else:
+            kv.append(hqmq.kv_codes(cache.words[0, r], cache.radius[0, r], cb))
+            hqmq.hqmq_decode(cache.words[0, r], cache.radius[0, r], cb, w.S, None, None, None, 0,
+                             cache.gran, y)
+        cbs.append(cb)
+        dense.append(y)
+    q = W.make_query(w, 0, device=dev)
+    o = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    ws = hqmq.alloc_attention_ws(B, H, device=dev)
+    st = hqmq.new_status(dev)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    ms = timed(lambda: hqmq.hqmq_attention_decode(q, kv[0], kv[1], w.S, H, T, o, ws, status=st))
+    qd = q.view(B, Hq, 1, D)
+    ms_dense = timed(lambda: F.scaled_dot_product_attention(qd, dense[0], dense[1], enable_gqa=True))
+    ref = F.scaled_dot_product_attention(qd, dense[0], dense[1], enable_gqa=True).float().view(B, Hq, D)
+    b_idx = math.ceil(math.log2(24 * w.S))
+    code_bytes = 2 * B * H * T * (4 * b_idx + 2 * D // 4) + n_list * (4 + 8)
+    dense_bytes = 2 * B * H * T * D * 2
+    gbs = code_bytes / (ms * 1e-3) / 1e9
+    return {"op": "hqmq_attention_decode (k_attn)",
+            "workload": "layer 0 of %s: batch %d, %d query heads over %d KV heads, %d tokens, S=%d"
+                        % (w.name, B, Hq, H, T, w.S),
+            "ms_per_call": round(ms, 4), "algorithmic_bytes": code_bytes,
+            "gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+            "list_entries": n_list,
+            "dense_bf16_sdpa_ms": round(ms_dense, 4),
+            "dense_bf16_bytes": dense_bytes,
+            "dense_over_hqmq_time": round(ms_dense / ms, 3),
+            "max_abs_diff_vs_sdpa": float((o - ref).abs().max().item()),
+            "status_flags": hqmq.read_status(st)["flags"],
+            "note": "the SDPA line is context: a library kernel over the dense decoded caches"}
+
+
 SWEEP = ("llama3_8b", "qwen_outlier", "mha7b_s8", "mha7b_s32")
 
 
@@ -459,6 +531,8 @@ def run_hqmq(args):
         "gpu_launches": cache.kernels_per_step() * args.steps,
         "clocks": clk,
     }
+    if world == 1 and not args.no_attention:
+        line["attention"] = run_attention(cache, peaks)
     if world == 1 and not args.no_sweep:
         # the metric's other workloads, after the headline's buffers are freed
         del cache
@@ -638,6 +712,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the per-config encode/decode rates of the other workloads")
+    ap.add_argument("--no-attention", action="store_true",
+                    help="skip the decode-phase attention measurement on layer 0's codes")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     args = ap.parse_args()
     if args.impl == "reference":

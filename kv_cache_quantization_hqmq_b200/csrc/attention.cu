@@ -147,34 +147,37 @@ template <int BT> struct BlockRegs {
     uint32_t vw[4][Geo<BT>::VW];
 };
 
-// Tokens >= len read as zero.  kb0 / vb0: bit offset of the lane's K / V run
-// inside a token's b-word group; kneed / vneed: words it spans (BT = 0).
+// Per-lane base pointers of the block loads at token 0 of the slab: K
+// token n, V token 2 q (the other tokens of a block are fixed offsets).
+struct LanePtrs {
+    const uint32_t *kw, *vw;
+    const uint4 *kr;
+    const uint2 *vr;
+};
+
+// Loads of the block starting at token t0 (tokens >= len read as zero);
+// kneed / vneed: the words a run spans (BT = 0).
 template <int BT>
-__device__ __forceinline__ void load_block(const AttnArgs &a, uint64_t slab_g0, int t0, int len,
-                                           int lane, uint32_t kb0, uint32_t vb0, uint32_t kneed,
-                                           uint32_t vneed, BlockRegs<BT> &R) {
+__device__ __forceinline__ void load_block(const LanePtrs &P, uint32_t b, int t0, int len,
+                                           int lane, uint32_t kneed, uint32_t vneed,
+                                           BlockRegs<BT> &R) {
     const int n = lane >> 2, q = lane & 3;
-    const uint32_t b = BT ? (uint32_t)BT : a.b;
+    const uint32_t tb = (uint32_t)t0 * b;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        const int t = t0 + n + 8 * j;
-        const bool ok = t < len;
-        const uint64_t g = slab_g0 + (uint64_t)t;
-        R.kr[j] = ok ? __ldcs(reinterpret_cast<const uint4 *>(a.k.radius + g * 32) + q)
-                     : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t *w = a.k.words + g * b + (kb0 >> 5);
+        const bool ok = t0 + n + 8 * j < len;
+        R.kr[j] = ok ? __ldcs(P.kr + (size_t)(t0 + 8 * j) * 4) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t *w = P.kw + tb + 8 * j * b;
 #pragma unroll
         for (int i = 0; i < Geo<BT>::KW; ++i)
             R.kw[j][i] = (ok && (BT || (uint32_t)i < kneed)) ? __ldg(w + i) : 0u;
     }
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-        const int t = t0 + 2 * q + (s & 1) + 8 * (s >> 1);
-        const bool ok = t < len;
-        const uint64_t g = slab_g0 + (uint64_t)t;
-        R.vr[s] = ok ? __ldcs(reinterpret_cast<const uint2 *>(a.v.radius + g * 32) + n)
-                     : make_uint2(0u, 0u);
-        const uint32_t *w = a.v.words + g * b + (vb0 >> 5);
+        const int dt = (s & 1) + 8 * (s >> 1);
+        const bool ok = t0 + 2 * q + dt < len;
+        R.vr[s] = ok ? __ldcs(P.vr + (size_t)(t0 + dt) * 8) : make_uint2(0u, 0u);
+        const uint32_t *w = P.vw + tb + dt * b;
 #pragma unroll
         for (int i = 0; i < Geo<BT>::VW; ++i)
             R.vw[s][i] = (ok && (BT || (uint32_t)i < vneed)) ? __ldg(w + i) : 0u;
@@ -276,21 +279,28 @@ __device__ __forceinline__ bool map_block(const KVDev &X, const uint32_t *sidx, 
     return any;
 }
 
-// The 4 fp16 values of the chunk-mode entry of chunk `chunk` with map slot
-// `slot`: staged, or past the staged part of the tile [a, e) (found by a
-// binary search of the ascending list).
-template <int LC>
-__device__ __forceinline__ uint2 slot_entry(const KVDev &X, const uint2 *sval, uint32_t a,
-                                            uint32_t e, uint32_t slot, uint32_t chunk) {
-    if (slot != 255u) return sval[slot - 1];
-    uint32_t lo = a + LC, hi = e;
+// fp16 x 4 -> bf16 x 4 (RN-even), in place, for n staged entries.
+__device__ __forceinline__ uint2 f16x4_to_bf16x4(uint2 e) {
+    return make_uint2(pack_bf16(f16_bits_to_f32(e.x & 0xFFFFu), f16_bits_to_f32(e.x >> 16)),
+                      pack_bf16(f16_bits_to_f32(e.y & 0xFFFFu), f16_bits_to_f32(e.y >> 16)));
+}
+__device__ __forceinline__ void to_bf16x4(uint2 *sval, uint32_t n, int lane) {
+    for (uint32_t k = (uint32_t)lane; k < n; k += 32) sval[k] = f16x4_to_bf16x4(sval[k]);
+}
+
+// The bf16 values of the chunk-mode entry of chunk `chunk`, which lies in
+// the unstaged part [lo, e) of its tile: a binary search of the ascending
+// list.
+__device__ __noinline__ uint2 entry_past_stage(const KVDev &X, uint32_t lo, uint32_t e,
+                                               uint32_t chunk) {
+    uint32_t hi = e;
     while (lo < hi) {
         const uint32_t mid = (lo + hi) >> 1;
         if (__ldg(X.out_idx + mid) < chunk) lo = mid + 1;
         else hi = mid;
     }
     const uint32_t *vv = reinterpret_cast<const uint32_t *>(X.out_val + (uint64_t)lo * 4);
-    return make_uint2(__ldg(vv), __ldg(vv + 1));
+    return f16x4_to_bf16x4(make_uint2(__ldg(vv), __ldg(vv + 1)));
 }
 
 // Marks the entries of the tile [a, e) that fall in the block's units
@@ -474,12 +484,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
     uint32_t kt0 = 0, kt1 = 0, kt2 = 0, kt3 = 0, vt0 = 0, vt1 = 0, vt2 = 0, vt3 = 0;
     __syncthreads();                                           // tables ready
 
+    LanePtrs P;
+    P.kw = a.k.words + (slab_g0 + n) * b + (kb0 >> 5);
+    P.vw = a.v.words + (slab_g0 + 2 * q) * b + (vb0 >> 5);
+    P.kr = reinterpret_cast<const uint4 *>(a.k.radius + (slab_g0 + n) * 32) + q;
+    P.vr = reinterpret_cast<const uint2 *>(a.v.radius + (slab_g0 + 2 * q) * 32) + n;
     BlockRegs<BT> cur, nxt;
-    if (wb0 < wb1) load_block<BT>(a, slab_g0, wb0 * ATT_BLK, len, lane, kb0, vb0, kneed, vneed, cur);
+    if (wb0 < wb1) load_block<BT>(P, b, wb0 * ATT_BLK, len, lane, kneed, vneed, cur);
     for (int blk = wb0; blk < wb1; ++blk) {
         const int t0 = blk * ATT_BLK;
-        if (blk + 1 < wb1)
-            load_block<BT>(a, slab_g0, t0 + ATT_BLK, len, lane, kb0, vb0, kneed, vneed, nxt);
+        if (blk + 1 < wb1) load_block<BT>(P, b, t0 + ATT_BLK, len, lane, kneed, vneed, nxt);
         const int tau = t0 >> 5, par = tau & 1;
         if ((klist || vlist) && (blk == wb0 || (t0 & 31) == 0)) {
             // entering list tile tau: stage tile tau + 1, make sure tau is in
@@ -509,6 +523,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
             if (vlist) vt3 = toff(a.v, tau + 3);
             cp_wait1();
             __syncwarp();
+            if constexpr (LM == LM_CHUNK) {
+                // the staged fp16 values of tile tau -> the bf16 that hqmq_decode writes
+                if (klist) to_bf16x4(WL.val[par][0], min(kt1 - kt0, (uint32_t)LC), lane);
+                if (vlist) to_bf16x4(WL.val[par][1], min(vt1 - vt0, (uint32_t)LC), lane);
+                __syncwarp();
+            }
         }
         const uint32_t u0 = (uint32_t)((slab_g0 + (uint64_t)t0) * 32);   // the block's first chunk
         bool kany = false, vany = false;
@@ -552,10 +572,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
                         for (int ks = 0; ks < 8; ++ks) {
                             const uint32_t slot = ((ks < 4 ? m8.x : m8.y) >> (8 * (ks & 3))) & 0xFFu;
                             if (!slot) continue;
-                            const uint2 e = slot_entry<LC>(a.k, WL.val[par][0], kt0, kt1, slot,
-                                                           u0 + tl * 32 + 8 * q + ks);
-                            kf0[ks] = pack_bf16(f16_bits_to_f32(e.x & 0xFFFFu), f16_bits_to_f32(e.x >> 16));
-                            kf1[ks] = pack_bf16(f16_bits_to_f32(e.y & 0xFFFFu), f16_bits_to_f32(e.y >> 16));
+                            const uint2 e = slot != 255u ? WL.val[par][0][slot - 1]
+                                                         : entry_past_stage(a.k, kt0 + LC, kt1,
+                                                                            u0 + tl * 32 + 8 * q + ks);
+                            kf0[ks] = e.x;
+                            kf1[ks] = e.y;
                         }
                     }
                 } else if constexpr (LM == LM_ANY) {
@@ -656,12 +677,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
                         const uint32_t slot = (lv[s] >> (8 * i)) & 0xFFu;
                         if (!slot) continue;
                         const uint32_t tl = (uint32_t)(2 * q + (s & 1) + 8 * (s >> 1));
-                        const uint2 e = slot_entry<LC>(a.v, WL.val[par][1], vt0, vt1, slot,
-                                                       u0 + tl * 32 + 4 * n + i);
-                        v[s][0] = f16_bits_to_f32(e.x & 0xFFFFu);
-                        v[s][1] = f16_bits_to_f32(e.x >> 16);
-                        v[s][2] = f16_bits_to_f32(e.y & 0xFFFFu);
-                        v[s][3] = f16_bits_to_f32(e.y >> 16);
+                        const uint2 e = slot != 255u ? WL.val[par][1][slot - 1]
+                                                     : entry_past_stage(a.v, vt0 + LC, vt1,
+                                                                        u0 + tl * 32 + 4 * n + i);
+                        v[s][0] = bf16_lo(e.x);
+                        v[s][1] = bf16_hi(e.x);
+                        v[s][2] = bf16_lo(e.y);
+                        v[s][3] = bf16_hi(e.y);
                     }
                 }
             } else if constexpr (LM == LM_ANY) {
