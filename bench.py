@@ -391,6 +391,67 @@ def run_attention(cache, peaks, iters=20, warmup=3):
             "note": "the SDPA line is context: a library kernel over the dense decoded caches"}
 
 
+def run_qradius(cache, peaks, iters=20, warmup=3):
+    """The quantized-radius variant on layer 0's K call (needs Med3x, chunk
+    mode): hqmq_quantize_radius and hqmq_decode_qradius timed with CUDA
+    events, bits per element, and the relative RMS error of both decodes
+    against the input."""
+    import torch
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    w = cache.w
+    if not w.med3:
+        return None
+    B, H, T, D = cache.shape
+    dev = cache.x.device
+    cb = cache.codebook[0:H * w.S * 4]
+    rw = torch.empty(cache.n_words, dtype=torch.int32, device=dev)
+    y = torch.empty(cache.shape, dtype=torch.bfloat16, device=dev)
+    yq = torch.empty(cache.shape, dtype=torch.bfloat16, device=dev)
+    st = hqmq.new_status(dev)
+    args = (cache.words[0, 0], rw, cache.thr[0, 0], cb, w.S, cache.out_idx[0, 0],
+            cache.out_val[0, 0], cache.tile_off[0, 0], cache.cap, cache.gran)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    ms_q = timed(lambda: hqmq.hqmq_quantize_radius(cache.radius[0, 0], cache.thr[0, 0],
+                                                   cache.shape, w.S, rw))
+    ms_d = timed(lambda: hqmq.hqmq_decode_qradius(*args, yq, st))
+    hqmq.hqmq_decode(cache.words[0, 0], cache.radius[0, 0], cb, w.S, cache.out_idx[0, 0],
+                     cache.out_val[0, 0], cache.slab_off[0, 0], cache.cap, cache.gran, y,
+                     tile_off=cache.tile_off[0, 0])
+    x = cache.x[0, 0].float()
+    nx = x.norm()
+    err_f16 = float((y.float() - x).norm() / nx)
+    err_q = float((yq.float() - x).norm() / nx)
+    n_chunks = cache.n_chunks
+    b = math.ceil(math.log2(24 * w.S))
+    n_out = int(cache.slab_off[0, 0][-1].item())
+    q_bytes = n_chunks * (2 + b / 8)
+    d_bytes = n_chunks * (2 * b / 8 + 8) + 12 * n_out
+    return {"op": "hqmq_quantize_radius + hqmq_decode_qradius (layer 0, K)",
+            "levels": 24 * w.S, "code_bits_per_chunk": 2 * b,
+            "bits_per_element": round(2 * b / 4 + n_out * 96 / (B * H * T * D), 4),
+            "bits_per_element_fp16_radius": round((b + 16) / 4 + n_out * 96 / (B * H * T * D), 4),
+            "pages_bits_per_element": {"S8": 3.79, "S32": 5},
+            "quantize_ms": round(ms_q, 4),
+            "quantize_hbm_frac": round(q_bytes / (ms_q * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "decode_ms": round(ms_d, 4),
+            "decode_hbm_frac": round(d_bytes / (ms_d * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "rel_rms_error": {"fp16_radius": round(err_f16, 5), "quantized_radius": round(err_q, 5)},
+            "status_flags": hqmq.read_status(st)["flags"]}
+
+
 SWEEP = ("llama3_8b", "qwen_outlier", "mha7b_s8", "mha7b_s32")
 
 
@@ -533,6 +594,7 @@ def run_hqmq(args):
     }
     if world == 1 and not args.no_attention:
         line["attention"] = run_attention(cache, peaks)
+        line["quantized_radius"] = run_qradius(cache, peaks)
     if world == 1 and not args.no_sweep:
         # the metric's other workloads, after the headline's buffers are freed
         del cache

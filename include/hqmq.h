@@ -298,6 +298,38 @@ HQMQ_API int hqmq_outlier_extract_noalloc(const void *d_x, int dtype, int B, int
                                           uint32_t *d_slab_off, uint64_t cap,
                                           hqmq_status *d_status, void *stream);
 
+/* Quantized radius (our reading of the pages' bit budget: the abstract's 3.79
+ * bits per element at S = 8 is log2(24 S) / 2, i.e. about 2 log2(24 S) bits
+ * per chunk, a radius code with as many levels as there are codewords).
+ * With Med3x every bulk chunk has r <= thr_h (gist.science/nl, Technische
+ * Samenvatting, section 3), so the fp16 radius is quantized uniformly on
+ * [0, thr_h] into L = 24 S levels:
+ *   inv_h = fl32((L-1) / thr_h),  k = min(L-1, floor(fl32(fl32(r inv_h) + 0.5)))
+ * (k = 0 for a NaN radius and for every chunk of a head whose thr is not a
+ * positive finite value).  The codes are packed like the indices: b =
+ * ceil(log2(24 S)) bits per chunk, b uint32 words per 32 chunks, LSB first;
+ * index + radius code = 2b bits per chunk (4.0 bits per element at S = 8,
+ * 5.0 at S = 32), plus the outlier list.
+ * d_radius: fp16 bits [B*H*T*D/4] as written by the encode calls (2-byte
+ * aligned); d_thr: fp32 [H], the top of each head's radius range: the Med3x
+ * thr in chunk mode (hqmq_outlier_extract / hqmq_encode_med3), 2 thr in
+ * element mode (a chunk whose 4 elements are all <= thr has r <= 2 thr);
+ * d_rcode_words: uint32[hqmq_index_words(B,H,T,D,S)], fully overwritten. */
+HQMQ_API int hqmq_quantize_radius(const uint16_t *d_radius, const float *d_thr, int B, int H,
+                                  int T, int D, uint32_t S, uint32_t *d_rcode_words,
+                                  void *stream);
+
+/* hqmq_decode with each chunk's radius taken from its code:
+ * r = fl32(k fl32(thr_h / (L-1))) (codes >= L read as L-1; d_thr the same
+ * ranges as given to hqmq_quantize_radius).  Everything else
+ * as hqmq_decode; a list needs its d_tile_off (applied in the main pass). */
+HQMQ_API int hqmq_decode_qradius(const uint32_t *d_idx_words, const uint32_t *d_rcode_words,
+                                 const float *d_thr, const float *d_codebook, uint32_t S,
+                                 const uint32_t *d_out_idx, const uint16_t *d_out_val,
+                                 const uint32_t *d_tile_off, uint64_t cap, int gran, int B, int H,
+                                 int T, int D, void *d_y, int out_dtype, hqmq_status *d_status,
+                                 void *stream);
+
 /* One coded K or V cache for hqmq_attention_decode: HOST struct of DEVICE
  * pointers, each as written by hqmq_encode / hqmq_encode_med3 for a
  * [B][Hk][T][128] tensor (idx_words, radius 16-byte aligned; codebook fp32

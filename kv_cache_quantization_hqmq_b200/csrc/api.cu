@@ -59,6 +59,15 @@ extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int
                                      int sm_count, cudaStream_t stream);
 extern "C" uint64_t hqmq_lut_bytes_per_group(uint32_t S);
 extern "C" uint64_t hqmq_attn_workspace_bytes(int B, int Hk);
+extern "C" int hqmq_launch_quantize_radius(const uint16_t *radius, const float *thr, int B, int H,
+                                           int T, int D, uint32_t S, uint32_t b, uint32_t *rwords,
+                                           int sm_count, cudaStream_t stream);
+extern "C" int hqmq_launch_decode_qr(const uint32_t *words, const uint32_t *rwords, const float *thr,
+                                     const float *cb, uint32_t S, uint32_t b,
+                                     const uint32_t *out_idx, const uint16_t *out_val,
+                                     const uint32_t *tile_off, uint64_t cap, int gran, int B, int H,
+                                     int T, int D, void *y, int out_dtype, hqmq_status *st,
+                                     int sm_count, cudaStream_t stream);
 extern "C" int hqmq_launch_attention(const uint16_t *q, const int *seq_len, const hqmq_kv_codes *k,
                                      const hqmq_kv_codes *v, uint32_t S, uint32_t b, int B,
                                      int Hk, int G, int T, float scale, void *o, int out_dtype,
@@ -363,6 +372,39 @@ int hqmq_attention_decode(const uint16_t *d_q, const int32_t *d_seq_len, const h
     return hqmq_launch_attention(d_q, d_seq_len, k, v, S, hqmq_index_bits(S), B, Hk, Hq / Hk, T,
                                  scale, d_o, out_dtype, d_ws, d_status, sm, optin,
                                  (cudaStream_t)stream);
+}
+
+int hqmq_quantize_radius(const uint16_t *d_radius, const float *d_thr, int B, int H, int T, int D,
+                         uint32_t S, uint32_t *d_rcode_words, void *stream) {
+    if (!shape_ok(B, H, T, D) || S < 1 || S > S_MAX) return HQMQ_ERR_ARG;
+    if (!d_radius || !d_thr || !d_rcode_words) return HQMQ_ERR_ARG;
+    if (!aligned(d_radius, 2) || !aligned(d_thr, 4) || !aligned(d_rcode_words, 4))
+        return HQMQ_ERR_ALIGN;
+    const int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_quantize_radius(d_radius, d_thr, B, H, T, D, S, hqmq_index_bits(S),
+                                       d_rcode_words, sm, (cudaStream_t)stream);
+}
+
+int hqmq_decode_qradius(const uint32_t *d_idx_words, const uint32_t *d_rcode_words,
+                        const float *d_thr, const float *d_codebook, uint32_t S,
+                        const uint32_t *d_out_idx, const uint16_t *d_out_val,
+                        const uint32_t *d_tile_off, uint64_t cap, int gran, int B, int H, int T,
+                        int D, void *d_y, int out_dtype, hqmq_status *d_status, void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(out_dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
+    if (S < 1 || S > S_MAX) return HQMQ_ERR_ARG;
+    if (!d_idx_words || !d_rcode_words || !d_thr || !d_codebook || !d_y) return HQMQ_ERR_ARG;
+    if (d_out_idx && (!d_out_val || !d_tile_off)) return HQMQ_ERR_ARG;
+    if (!aligned(d_idx_words, 4) || !aligned(d_rcode_words, 4) || !aligned(d_thr, 4) ||
+        !aligned(d_codebook, 16) || !aligned(d_y, 16) || !aligned(d_out_idx, 4) ||
+        !aligned(d_out_val, 4) || !aligned(d_tile_off, 4) || !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    const int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_decode_qr(d_idx_words, d_rcode_words, d_thr, d_codebook, S,
+                                 hqmq_index_bits(S), d_out_idx, d_out_val,
+                                 d_out_idx ? d_tile_off : nullptr, cap, gran, B, H, T, D, d_y,
+                                 out_dtype, d_status, sm, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -36,15 +36,30 @@ __device__ __forceinline__ uint32_t get_index(const uint32_t *__restrict__ words
     return (uint32_t)(v >> o) & ((1u << b) - 1u);
 }
 
+// Quantized-radius mode: the step delta = fl32(thr / (L - 1)) of a head
+// (0 unless thr is a positive finite value), and the radius fl32(k delta) of
+// level k (codes >= L read as L - 1).
+__device__ __forceinline__ float qr_delta(float thr, uint32_t L) {
+    if (!(thr > 0.0f) || isinf(thr) || L < 2u) return 0.0f;
+    return __fdiv_rn(thr, (float)(L - 1u));
+}
+__device__ __forceinline__ float qr_radius(uint32_t k, uint32_t L, float delta) {
+    return __fmul_rn((float)(k < L ? k : L - 1u), delta);
+}
+
 // fl32(fl32(r c_e) + v) of element e of chunk j, r and c from the chunk's
 // code (the main pass's product), v the list's fp16 value; a bad index gives
-// r = 0.
+// r = 0.  RQ: r from the chunk's radius code (rwords, delta).
+template <int RQ>
 __device__ __forceinline__ float element_with_outlier(const uint32_t *__restrict__ words,
                                                      const uint16_t *__restrict__ radius,
+                                                     const uint32_t *__restrict__ rwords,
+                                                     float delta,
                                                      const float4 *__restrict__ cb, uint32_t S,
                                                      uint32_t b, uint64_t j, int e, uint32_t v16) {
     const uint32_t ix = get_index(words, j >> 5, (uint32_t)(j & 31u), b);
-    float r = f16_bits_to_f32(__ldg(radius + j));
+    float r = RQ ? qr_radius(get_index(rwords, j >> 5, (uint32_t)(j & 31u), b), 24u * S, delta)
+                 : f16_bits_to_f32(__ldg(radius + j));
     float c = 0.0f;
     if (ix < 24u * S) {
         const float4 cw = codeword((int)(ix % 24u), __ldg(cb + ix / 24u));
@@ -67,23 +82,27 @@ __device__ __forceinline__ float element_with_outlier(const uint32_t *__restrict
 // stores and a __syncwarp(), the warp writes the entries of its tile that
 // fall inside the unit.
 constexpr int DEC_UNIT = 8;                      // packing groups per unit
-template <int OUT_DT, bool TABLE, int LISTED>
+// RQ: quantized-radius mode, the radius of a chunk is fl32(k delta_h) with k
+// its b-bit radius code (rwords, laid out like the index words).
+template <int OUT_DT, bool TABLE, int LISTED, int RQ>
 __global__ void __launch_bounds__(DEC_THREADS, 8)
 k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius,
          const float4 *__restrict__ cb_all, uint32_t S, uint32_t b, int H,
          uint32_t chunks_per_slab, void *__restrict__ y, DevStatus *st,
          const uint32_t *__restrict__ tile_off, uint32_t tiles_per_slab,
          const uint32_t *__restrict__ out_idx, const uint16_t *__restrict__ out_val,
-         uint32_t cap32) {
+         uint32_t cap32, const uint32_t *__restrict__ rwords, const float *__restrict__ thr) {
     extern __shared__ float4 s_dyn[];
     const uint32_t n_words = 24u * S;
     float4 *s_tab = s_dyn;                         // [24 S] if TABLE
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t *s_w = reinterpret_cast<uint32_t *>(s_dyn + (TABLE ? n_words : 0)) +
                     (uint32_t)warp * DEC_UNIT * b;  // this warp's staged words
+    uint32_t *s_rw = s_w + (DEC_THREADS / 32) * DEC_UNIT * b;   // its staged radius codes (RQ)
     const int slab = blockIdx.y;
     const int h = slab % H;
     const float4 *cb = cb_all + (size_t)h * S;
+    const float delta = RQ ? qr_delta(__ldg(thr + h), n_words) : 0.0f;
     if (TABLE) {
         for (uint32_t i = threadIdx.x; i < n_words; i += DEC_THREADS)
             s_tab[i] = codeword((int)(i % 24u), __ldg(cb + i / 24u));
@@ -105,35 +124,49 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
         uint32_t rr[DEC_UNIT / 2];
 #pragma unroll
         for (int u = 0; u < DEC_UNIT / 2; ++u)     // radius pairs: all in flight
-            rr[u] = (uint32_t)(2 * u) < ng
+            rr[u] = (!RQ && (uint32_t)(2 * u) < ng)
                         ? __ldcs(reinterpret_cast<const uint32_t *>(radius + gg0 * 32) + u * 32 + lane)
                         : 0u;
         __syncwarp();                              // (the previous unit's reads of s_w)
-        for (uint32_t i = lane; i < ng * b; i += 32) s_w[i] = __ldg(words + gg0 * b + i);
+        for (uint32_t i = lane; i < ng * b; i += 32) {
+            s_w[i] = __ldg(words + gg0 * b + i);
+            if (RQ) s_rw[i] = __ldcs(rwords + gg0 * b + i);
+        }
         __syncwarp();
 #pragma unroll
         for (int u = 0; u < DEC_UNIT / 2; ++u) {
             if ((uint32_t)(2 * u) >= ng) break;
             const uint32_t c = (uint32_t)u * 64 + 2u * lane;        // chunk within the unit
-            uint32_t ixs[2];
+            uint32_t ixs[2], rks[2] = {0u, 0u};
             if (b <= 16) {                         // both indices from one 64-bit window
                 const uint32_t bit = c * b, o = bit & 31u;
                 const uint32_t *sw = s_w + (bit >> 5);
                 const uint64_t w64 = (uint64_t)sw[0] | ((uint64_t)(o + 2 * b > 32u ? sw[1] : 0u) << 32);
                 ixs[0] = (uint32_t)(w64 >> o) & mask;
                 ixs[1] = (uint32_t)(w64 >> (o + b)) & mask;
+                if (RQ) {
+                    const uint32_t *sr = s_rw + (bit >> 5);
+                    const uint64_t r64 = (uint64_t)sr[0] | ((uint64_t)(o + 2 * b > 32u ? sr[1] : 0u) << 32);
+                    rks[0] = (uint32_t)(r64 >> o) & mask;
+                    rks[1] = (uint32_t)(r64 >> (o + b)) & mask;
+                }
             } else {
 #pragma unroll
                 for (int v = 0; v < 2; ++v) {
                     const uint32_t bit = (c + v) * b, o = bit & 31u;
                     const uint32_t *sw = s_w + (bit >> 5);
                     ixs[v] = __funnelshift_r(sw[0], o + b > 32u ? sw[1] : 0u, o) & mask;
+                    if (RQ) {
+                        const uint32_t *sr = s_rw + (bit >> 5);
+                        rks[v] = __funnelshift_r(sr[0], o + b > 32u ? sr[1] : 0u, o) & mask;
+                    }
                 }
             }
             float out[8];
 #pragma unroll
             for (int v = 0; v < 2; ++v) {
-                float r = f16_bits_to_f32(v ? (rr[u] >> 16) : (rr[u] & 0xFFFFu));
+                float r = RQ ? qr_radius(rks[v], n_words, delta)
+                             : f16_bits_to_f32(v ? (rr[u] >> 16) : (rr[u] & 0xFFFFu));
                 float4 cw;
                 if (ixs[v] < n_words) {
                     cw = TABLE ? s_tab[ixs[v]] : codeword((int)(ixs[v] % 24u), __ldg(cb + ixs[v] / 24u));
@@ -197,8 +230,9 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
                 } else {
                     const uint64_t jq = qi >> 2;
                     if (jq < q0 || jq >= q1) continue;
-                    const float val = element_with_outlier(words, radius, cb, S, b, jq,
-                                                           (int)(qi & 3u), __ldg(out_val + k));
+                    const float val = element_with_outlier<RQ>(words, radius, rwords, delta, cb, S,
+                                                               b, jq, (int)(qi & 3u),
+                                                               __ldg(out_val + k));
                     if (OUT_DT == HQMQ_BF16)
                         reinterpret_cast<__nv_bfloat16 *>(y)[qi] = __float2bfloat16_rn(val);
                     else
@@ -280,14 +314,15 @@ k_decode_outliers(const uint32_t *__restrict__ words, const uint16_t *__restrict
     }
 }
 
-template <int OUT_DT, bool TABLE, int LISTED>
+template <int OUT_DT, bool TABLE, int LISTED, int RQ = 0>
 static int launch_main(const uint32_t *words, const uint16_t *radius, const float *cb, uint32_t S,
                        uint32_t b, int B, int H, uint32_t cps, void *y, hqmq_status *st,
                        const uint32_t *tile_off, const uint32_t *out_idx, const uint16_t *out_val,
-                       uint64_t cap, int sm_count, cudaStream_t stream) {
-    auto kern = k_decode<OUT_DT, TABLE, LISTED>;
+                       uint64_t cap, int sm_count, cudaStream_t stream,
+                       const uint32_t *rwords = nullptr, const float *thr = nullptr) {
+    auto kern = k_decode<OUT_DT, TABLE, LISTED, RQ>;
     const size_t smem = (TABLE ? (size_t)24 * S * sizeof(float4) : 0) +
-                        (size_t)(DEC_THREADS / 32) * DEC_UNIT * b * sizeof(uint32_t);
+                        (size_t)(RQ ? 2 : 1) * (DEC_THREADS / 32) * DEC_UNIT * b * sizeof(uint32_t);
     if (smem > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
@@ -309,7 +344,7 @@ static int launch_main(const uint32_t *words, const uint16_t *radius, const floa
     dim3 grid((unsigned)gx, (unsigned)n_slabs);
     kern<<<grid, DEC_THREADS, smem, stream>>>(words, radius, reinterpret_cast<const float4 *>(cb),
                                               S, b, H, cps, y, reinterpret_cast<DevStatus *>(st),
-                                              tile_off, tps, out_idx, out_val, cap32);
+                                              tile_off, tps, out_idx, out_val, cap32, rwords, thr);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
@@ -387,4 +422,44 @@ extern "C" int hqmq_launch_decode(const uint32_t *words, const uint16_t *radius,
                                      slab_off, tile_off, cap, B, H, cps, y, st, sm_count, stream);
     return launch_all<HQMQ_F32>(table, gran, words, radius, cb, S, b, out_idx, out_val, slab_off,
                                 tile_off, cap, B, H, cps, y, st, sm_count, stream);
+}
+
+// Quantized-radius decode: as hqmq_launch_decode, the radius of chunk j being
+// fl32(k_j delta_h) (k_j its radius code, delta_h = fl32(thr_h / (24 S - 1))).
+// A list needs its tile offsets (applied in the main pass).
+extern "C" int hqmq_launch_decode_qr(const uint32_t *words, const uint32_t *rwords, const float *thr,
+                                     const float *cb, uint32_t S, uint32_t b,
+                                     const uint32_t *out_idx, const uint16_t *out_val,
+                                     const uint32_t *tile_off, uint64_t cap, int gran, int B, int H,
+                                     int T, int D, void *y, int out_dtype, hqmq_status *st,
+                                     int sm_count, cudaStream_t stream) {
+    using namespace hqmq;
+    const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
+    const bool table = S <= 170;
+    const bool listed = out_idx != nullptr && cap > 0 && tile_off != nullptr;
+    const int L = listed ? gran + 1 : 0;
+#define HQMQ_QR_LAUNCH(DT, TB, LS)                                                              \
+    return launch_main<DT, TB, LS, 1>(words, nullptr, cb, S, b, B, H, cps, y, st,               \
+                                      LS ? tile_off : nullptr, LS ? out_idx : nullptr,           \
+                                      LS ? out_val : nullptr, LS ? cap : 0, sm_count, stream,    \
+                                      rwords, thr)
+    if (out_dtype == HQMQ_BF16) {
+        if (table) {
+            if (L == HQMQ_GRAN_CHUNK + 1) HQMQ_QR_LAUNCH(HQMQ_BF16, true, HQMQ_GRAN_CHUNK + 1);
+            if (L == HQMQ_GRAN_ELEMENT + 1) HQMQ_QR_LAUNCH(HQMQ_BF16, true, HQMQ_GRAN_ELEMENT + 1);
+            HQMQ_QR_LAUNCH(HQMQ_BF16, true, 0);
+        }
+        if (L == HQMQ_GRAN_CHUNK + 1) HQMQ_QR_LAUNCH(HQMQ_BF16, false, HQMQ_GRAN_CHUNK + 1);
+        if (L == HQMQ_GRAN_ELEMENT + 1) HQMQ_QR_LAUNCH(HQMQ_BF16, false, HQMQ_GRAN_ELEMENT + 1);
+        HQMQ_QR_LAUNCH(HQMQ_BF16, false, 0);
+    }
+    if (table) {
+        if (L == HQMQ_GRAN_CHUNK + 1) HQMQ_QR_LAUNCH(HQMQ_F32, true, HQMQ_GRAN_CHUNK + 1);
+        if (L == HQMQ_GRAN_ELEMENT + 1) HQMQ_QR_LAUNCH(HQMQ_F32, true, HQMQ_GRAN_ELEMENT + 1);
+        HQMQ_QR_LAUNCH(HQMQ_F32, true, 0);
+    }
+    if (L == HQMQ_GRAN_CHUNK + 1) HQMQ_QR_LAUNCH(HQMQ_F32, false, HQMQ_GRAN_CHUNK + 1);
+    if (L == HQMQ_GRAN_ELEMENT + 1) HQMQ_QR_LAUNCH(HQMQ_F32, false, HQMQ_GRAN_ELEMENT + 1);
+    HQMQ_QR_LAUNCH(HQMQ_F32, false, 0);
+#undef HQMQ_QR_LAUNCH
 }

@@ -59,6 +59,9 @@ _SIGS = {
     "hqmq_search_table_bytes": (_U64, [_U32]),
     "hqmq_make_search_table": (_I, [_P, _U32, _U32, _P, _P]),
     "hqmq_encode_lut": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _P, _I, _P, _P, _P, _P]),
+    "hqmq_quantize_radius": (_I, [_P, _P, _I, _I, _I, _I, _U32, _P, _P]),
+    "hqmq_decode_qradius": (_I, [_P, _P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P,
+                                 _I, _P, _P]),
     "hqmq_attention_workspace_size": (_U64, [_I, _I]),
     "hqmq_attention_decode": (_I, [_P, _P, _P, _P, _U32, _I, _I, _I, _I, _I, _F, _P, _I, _P,
                                    _U64, _P, _P]),
@@ -209,6 +212,25 @@ def hqmq_decode(idx_words, radius, codebook, S, out_idx, out_val, slab_off, cap,
     _check("hqmq_decode", _lib.hqmq_decode(
         _ptr(idx_words), _ptr(radius), _ptr(codebook), S, _ptr(out_idx), _ptr(out_val),
         _ptr(slab_off), _ptr(tile_off), int(cap), gran, B, H, T, D, _ptr(y), _dtype_code(y),
+        _ptr(status), _stream(stream)))
+
+
+def hqmq_quantize_radius(radius, thr, shape, S, rcode_words, stream=None):
+    """Radius codes (b bits per chunk, uniform on [0, thr_h], 24 S levels) of a
+    call's fp16 radii; shape = (B, H, T, D)."""
+    B, H, T, D = shape
+    _check("hqmq_quantize_radius", _lib.hqmq_quantize_radius(
+        _ptr(radius), _ptr(thr), B, H, T, D, S, _ptr(rcode_words), _stream(stream)))
+    return rcode_words
+
+
+def hqmq_decode_qradius(idx_words, rcode_words, thr, codebook, S, out_idx, out_val, tile_off,
+                        cap, gran, y, status=None, stream=None):
+    """hqmq_decode with the radii taken from their codes; a list needs tile_off."""
+    B, H, T, D = _shape4(y)
+    _check("hqmq_decode_qradius", _lib.hqmq_decode_qradius(
+        _ptr(idx_words), _ptr(rcode_words), _ptr(thr), _ptr(codebook), S, _ptr(out_idx),
+        _ptr(out_val), _ptr(tile_off), int(cap), gran, B, H, T, D, _ptr(y), _dtype_code(y),
         _ptr(status), _stream(stream)))
 
 

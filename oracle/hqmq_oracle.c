@@ -655,3 +655,99 @@ void oracle_score_chunks(const void *x, int dtype, int B, int H, int T, int D,
         out[q] = oracle_score(c, codebook + (size_t)h * S * 4, S, idx[q]);
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Quantized radius (our reading of the pages' bit budget [ABS], [NL 3]:     */
+/* about 2 log2(24 S) bits per chunk, i.e. a radius code of as many levels  */
+/* as there are codewords).  With Med3x every bulk chunk has r <= thr, so   */
+/* the fp16 radius is quantized uniformly on [0, thr_h] into L = 24 S       */
+/* levels, code k stored in b = ceil(log2(24 S)) bits, packed like the      */
+/* indices.  Outliers are in the list; their codes are zero, so k = 0.      */
+/* ------------------------------------------------------------------------ */
+
+/* Step and inverse step of head h: delta = fl32(thr / (L-1)),
+ * inv = fl32((L-1) / thr); both 0 when thr is not a positive finite value. */
+static void qr_steps(float thr, uint32_t L, float *delta, float *inv)
+{
+    float lm1 = (float)(L - 1u);
+    if (!(thr > 0.0f) || isinf(thr) || L < 2u) { *delta = 0.0f; *inv = 0.0f; return; }
+    *delta = thr / lm1;
+    *inv = lm1 / thr;
+}
+
+/* Level of one radius: k = min(L-1, floor(fl32(fl32(r * inv) + 0.5))),
+ * every step one fp32 operation; a NaN radius gives 0. */
+uint32_t oracle_radius_level(uint16_t radius_f16, float thr, uint32_t L)
+{
+    float delta, inv;
+    qr_steps(thr, L, &delta, &inv);
+    float r = oracle_f16_to_f32(radius_f16);
+    float q = r * inv;
+    if (isnan(q)) return 0u;
+    float t = q + 0.5f;
+    float k = floorf(t);
+    if (k >= (float)(L - 1u)) return L - 1u;
+    if (k < 0.0f) return 0u;
+    return (uint32_t)k;
+}
+
+/* Radius codes of a whole call: rcode_words laid out like the index words. */
+void oracle_quantize_radius(const uint16_t *radius, const float *thr, int B, int H, int T, int D,
+                            uint32_t S, uint32_t *rcode_words)
+{
+    size_t n_chunks = (size_t)B * H * T * D / 4;
+    uint32_t b = oracle_index_bits(S), L = 24u * S;
+    memset(rcode_words, 0, (n_chunks / 32) * b * sizeof(uint32_t));
+    for (size_t j = 0; j < n_chunks; ++j) {
+        int h = head_of_chunk(j, H, T, D);
+        put_index(rcode_words, b, j, oracle_radius_level(radius[j], thr[h], L));
+    }
+}
+
+/* Decoded radius of level k: fl32(k * delta). */
+float oracle_radius_of_level(uint32_t k, float thr, uint32_t L)
+{
+    float delta, inv;
+    qr_steps(thr, L, &delta, &inv);
+    return (float)k * delta;
+}
+
+/* oracle_decode with the radius of chunk j taken from its code:
+ * r = fl32(k * delta_h).  Everything else (codeword, outliers, rounding,
+ * bad-index rule) as in oracle_decode. */
+void oracle_decode_qradius(const uint32_t *words, const uint32_t *rcode_words, const float *thr,
+                           const float *codebook, uint32_t S, const uint32_t *out_idx,
+                           const uint16_t *out_val, int64_t n_out, int gran, int B, int H, int T,
+                           int D, void *y, int out_dtype, oracle_status *st)
+{
+    size_t n_chunks = (size_t)B * H * T * D / 4;
+    uint32_t b = oracle_index_bits(S), L = 24u * S;
+    float *acc = (float *)malloc(n_chunks * 4 * sizeof(float));
+    uint64_t n_bad = 0;
+    for (size_t j = 0; j < n_chunks; ++j) {
+        int h = head_of_chunk(j, H, T, D);
+        uint32_t idx = oracle_get_index(words, b, j);
+        uint32_t k = oracle_get_index(rcode_words, b, j);
+        float r = oracle_radius_of_level(k < L ? k : L - 1u, thr[h], L);
+        float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (idx >= 24u * S) { ++n_bad; r = 0.0f; }
+        else oracle_codeword_f32((int)(idx % 24u), codebook + ((size_t)h * S + idx / 24u) * 4, c);
+        for (int e = 0; e < 4; ++e) acc[4 * j + e] = r * c[e];
+    }
+    if (out_idx && n_out > 0) {
+        if (gran == OR_GRAN_CHUNK) {
+            for (int64_t q = 0; q < n_out; ++q) {
+                size_t j = out_idx[q];
+                for (int i = 0; i < 4; ++i) acc[4 * j + i] = oracle_f16_to_f32(out_val[4 * q + i]);
+            }
+        } else {
+            for (int64_t q = 0; q < n_out; ++q) {
+                size_t e = out_idx[q];
+                acc[e] = acc[e] + oracle_f16_to_f32(out_val[q]);
+            }
+        }
+    }
+    for (size_t e = 0; e < n_chunks * 4; ++e) store_elem(y, out_dtype, e, acc[e]);
+    if (st && n_bad) { st->flags |= OR_FLAG_BAD_INDEX; }
+    free(acc);
+}

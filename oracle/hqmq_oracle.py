@@ -88,6 +88,11 @@ _SIGS = {
     "oracle_chunk_norm_array": (None, [_P, _P, _I64]),
     "oracle_get_index_array": (None, [_P, _U32, _P, _I64, _P]),
     "oracle_score_chunks": (None, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _I, _P, _P, _I64, _P]),
+    "oracle_radius_level": (_U32, [ctypes.c_uint16, _F, _U32]),
+    "oracle_radius_of_level": (_F, [_U32, _F, _U32]),
+    "oracle_quantize_radius": (None, [_P, _P, _I, _I, _I, _I, _U32, _P]),
+    "oracle_decode_qradius": (None, [_P, _P, _P, _P, _U32, _P, _P, _I64, _I, _I, _I, _I, _I, _P,
+                                     _I, _P]),
 }
 
 
@@ -316,6 +321,46 @@ def decode(words, radius, codebook, S, B, H, T, D, out_idx=None, out_val=None,
     st = Status()
     lib().oracle_decode(_ptr(words), _ptr(radius), _ptr(cb), int(S), _ptr(oi), _ptr(ov), n_out,
                         gran, B, H, T, D, _ptr(y), out_dtype, ctypes.byref(st))
+    return y, st.as_dict()
+
+
+def radius_level(radius_f16, thr, S):
+    """Level k of one fp16 radius (bits) for threshold thr: the quantized-radius
+    reading (uniform on [0, thr], L = 24 S levels); see hqmq_oracle.c."""
+    return int(lib().oracle_radius_level(int(radius_f16), float(thr), 24 * int(S)))
+
+
+def radius_of_level(k, thr, S):
+    return float(lib().oracle_radius_of_level(int(k), float(thr), 24 * int(S)))
+
+
+def quantize_radius(radius, thr, B, H, T, D, S):
+    """Radius codes of a whole call (uint32 words laid out like the index words)."""
+    radius = _c(radius, np.uint16)
+    thr = _c(thr, np.float32)
+    words = np.zeros(index_words(B, H, T, D, S), np.uint32)
+    lib().oracle_quantize_radius(_ptr(radius), _ptr(thr), B, H, T, D, int(S), _ptr(words))
+    return words
+
+
+def decode_qradius(words, rcode_words, thr, codebook, S, B, H, T, D, out_idx=None, out_val=None,
+                   gran=CHUNK, out_dtype=BF16):
+    """decode() with each chunk's radius taken from its radius code."""
+    words = _c(words, np.uint32)
+    rw = _c(rcode_words, np.uint32)
+    thr = _c(thr, np.float32)
+    cb = _c(codebook, np.float32)
+    n_out = 0
+    oi = ov = None
+    if out_idx is not None and len(out_idx) > 0:
+        oi = _c(out_idx, np.uint32)
+        ov = _c(out_val, np.uint16)
+        n_out = oi.size
+    y = np.zeros((B, H, T, D), np.uint16 if out_dtype == BF16 else np.float32)
+    st = Status()
+    lib().oracle_decode_qradius(_ptr(words), _ptr(rw), _ptr(thr), _ptr(cb), int(S), _ptr(oi),
+                                _ptr(ov), n_out, gran, B, H, T, D, _ptr(y), out_dtype,
+                                ctypes.byref(st))
     return y, st.as_dict()
 
 

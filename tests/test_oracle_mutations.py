@@ -44,11 +44,17 @@ MUTATIONS = [
     ("decode_drops_radius", "for (int i = 0; i < 4; ++i) acc[4 * j + i] = r * c[i];",
      "for (int i = 0; i < 4; ++i) acc[4 * j + i] = c[i];",
      ["test_decode_is_radius_times_codeword"]),
+    ("qradius_rounds_down", "float t = q + 0.5f;", "float t = q;",
+     ["test_level_is_the_nearest_grid_point"], "tests/test_oracle_qradius.py"),
+    ("qradius_levels_pow2", "uint32_t b = oracle_index_bits(S), L = 24u * S;\n    float *acc",
+     "uint32_t b = oracle_index_bits(S), L = 1u << oracle_index_bits(S);\n    float *acc",
+     ["test_decode_on_the_grid_equals_the_fp16_radius_decode"], "tests/test_oracle_qradius.py"),
 ]
+MUTATIONS = [m if len(m) == 5 else m + (PINS,) for m in MUTATIONS]
 
 
-@pytest.mark.parametrize("mid,old,new,pins", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_planted_mistake_is_caught(tmp_path, mid, old, new, pins):
+@pytest.mark.parametrize("mid,old,new,pins,pin_file", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(tmp_path, mid, old, new, pins, pin_file):
     src = open(SRC).read()
     assert src.count(old) == 1, mid
     mutant = tmp_path / ("mut_%s.c" % mid)
@@ -59,7 +65,7 @@ def test_planted_mistake_is_caught(tmp_path, mid, old, new, pins):
     subprocess.check_call(["gcc", *hqmq_oracle.CFLAGS, "-o", str(so), str(mutant), "-lm"])
     env = dict(os.environ, HQMQ_ORACLE_LIB=str(so))
     sel = " or ".join(pins)
-    r = subprocess.run([sys.executable, "-m", "pytest", PINS, "-q", "-x", "-k", sel, "-p", "no:cacheprovider"],
+    r = subprocess.run([sys.executable, "-m", "pytest", pin_file, "-q", "-x", "-k", sel, "-p", "no:cacheprovider"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert "passed" in r.stdout or "failed" in r.stdout, r.stdout + r.stderr
     assert r.returncode != 0, "mutation %s was not caught:\n%s" % (mid, r.stdout[-2000:])
