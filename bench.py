@@ -29,6 +29,8 @@ import subprocess
 import sys
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -452,6 +454,121 @@ def run_qradius(cache, peaks, iters=20, warmup=3):
             "status_flags": hqmq.read_status(st)["flags"]}
 
 
+def run_streaming(cache, iters=20, warmup=3):
+    """One decode step of the whole model: for every (layer, role), the Med3x
+    list of one new token per sequence under the prefill's threshold
+    (hqmq_outlier_extract_given_thr) and its encode with that threshold, by
+    the search table (hqmq_encode_lut) or the codeword loop (hqmq_encode),
+    timed as plain launches and as one CUDA graph of the whole step.  The new
+    tokens are drawn like the cache (same distribution, other seeds)."""
+    import torch
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    from kv_cache_quantization_hqmq_b200 import workloads as W
+    w = cache.w
+    if not w.med3:
+        return None
+    B, H, T, D = cache.shape
+    dev = cache.x.device
+    L2 = (w.layers, 2)
+    wn = w.with_(input_seed=w.input_seed + 4242)
+    x1 = torch.empty(L2 + (B, H, 1, D), dtype=w.torch_dtype, device=dev)
+    for l in range(w.layers):
+        for r in range(2):
+            x1[l, r].copy_(W.make_call_input(wn, l, r, device=dev, tokens=1))
+    n_words = hqmq.hqmq_index_words(B, H, 1, D, w.S)
+    n_chunks = B * H * D // 4
+    words = torch.empty(L2 + (n_words,), dtype=torch.int32, device=dev)
+    radius = torch.empty(L2 + (n_chunks,), dtype=torch.int16, device=dev)
+    oi = torch.empty(L2 + (n_chunks,), dtype=torch.int32, device=dev)
+    ov = torch.empty(L2 + (4 * n_chunks,), dtype=torch.int16, device=dev)
+    so = torch.empty(L2 + (B * H + 1,), dtype=torch.int32, device=dev)
+    to = torch.empty(L2 + (hqmq.hqmq_list_tiles(B, H, 1, D) + 1,), dtype=torch.int32, device=dev)
+    ws = torch.empty(L2 + (hqmq.hqmq_outlier_extract_given_thr_workspace_size(B, H, 1, D),),
+                     dtype=torch.uint8, device=dev)
+
+    def step(lut):
+        for l in range(w.layers):
+            for r in range(2):
+                g0 = (l * 2 + r) * H
+                cb = cache.codebook[g0 * w.S * 4:(g0 + H) * w.S * 4]
+                hqmq.hqmq_outlier_extract_given_thr(x1[l, r], cache.thr[l, r], cache.gran, oi[l, r],
+                                                    ov[l, r], so[l, r], n_chunks, ws[l, r],
+                                                    tile_off=to[l, r])
+                if lut:
+                    tb = cache.table[g0 * cache.table_bytes:(g0 + H) * cache.table_bytes]
+                    hqmq.hqmq_encode_lut(x1[l, r], cb, w.S, tb, cache.thr[l, r], cache.gran,
+                                         words[l, r], radius[l, r])
+                else:
+                    hqmq.hqmq_encode(x1[l, r], cb, w.S, cache.thr[l, r], cache.gran, words[l, r],
+                                     radius[l, r])
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    out = {"op": "decode-step append: hqmq_outlier_extract_given_thr + encode per (layer, role)",
+           "new_tokens_per_step": B, "calls_per_step": w.layers * 2,
+           "launches_per_step": 4 * w.layers * 2,
+           "threshold": "per (layer, role, head) from the timed step (the prefill)"}
+    for name, lut in (("search_table", True), ("codeword_loop", False)):
+        if lut and cache.table is None:
+            continue
+        ms_plain = timed(lambda: step(lut))
+        graph = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            step(lut)
+        torch.cuda.current_stream().wait_stream(s)
+        with torch.cuda.graph(graph):
+            step(lut)
+        ms_graph = timed(graph.replay)
+        out[name] = {"us_per_step_plain": round(ms_plain * 1e3, 1),
+                     "us_per_step_graph": round(ms_graph * 1e3, 1)}
+        del graph
+    out["outliers_last_step"] = int(so[:, :, -1].sum().item())
+    return out
+
+
+def run_covering(device, n_chunks=1 << 20):
+    """The covering rate of the codebook measured with the GPU encode: mean and
+    largest angle between a chunk and its decoded codeword over S = 1 .. 64 for
+    Haar-random chunks (fp32), and the fitted slope of log mean angle against
+    log 24 S (the pages' Proposition 3.1: -1/3)."""
+    import torch
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    x = torch.randn((1, 1, n_chunks // 32, 128), generator=g, device=device)
+    xu = torch.nn.functional.normalize(x.view(-1, 4), dim=1)
+    out, Ss = {}, (1, 2, 4, 8, 16, 32, 64)
+    means = []
+    for S in Ss:
+        cb = torch.empty(S * 4, dtype=torch.float32, device=device)
+        hqmq.hqmq_make_codebook(11, S, 1, 0, cb)
+        words, radius = hqmq.alloc_codes(1, 1, n_chunks // 32, 128, S, device=device)
+        hqmq.hqmq_encode(x, cb, S, None, 0, words, radius)
+        y = torch.empty_like(x)
+        hqmq.hqmq_decode(words, radius, cb, S, None, None, None, 0, 0, y)
+        yu = torch.nn.functional.normalize(y.view(-1, 4), dim=1)
+        ang = torch.rad2deg(torch.arccos((xu * yu).sum(1).clamp(-1, 1)))
+        means.append(float(ang.mean()))
+        out["S%d" % S] = {"mean_deg": round(means[-1], 3), "max_deg": round(float(ang.max()), 3)}
+    slope = float(np.polyfit(np.log(24.0 * np.array(Ss)), np.log(means), 1)[0])
+    out["slope_log_mean_angle_vs_log_24S"] = round(slope, 4)
+    out["chunks_per_S"] = n_chunks
+    return out
+
+
 SWEEP = ("llama3_8b", "qwen_outlier", "mha7b_s8", "mha7b_s32")
 
 
@@ -595,6 +712,8 @@ def run_hqmq(args):
     if world == 1 and not args.no_attention:
         line["attention"] = run_attention(cache, peaks)
         line["quantized_radius"] = run_qradius(cache, peaks)
+        line["streaming_append"] = run_streaming(cache)
+        line["covering"] = run_covering(device)
     if world == 1 and not args.no_sweep:
         # the metric's other workloads, after the headline's buffers are freed
         del cache

@@ -298,6 +298,27 @@ HQMQ_API int hqmq_outlier_extract_noalloc(const void *d_x, int dtype, int B, int
                                           uint32_t *d_slab_off, uint64_t cap,
                                           hqmq_status *d_status, void *stream);
 
+/* Outlier list of a call under a GIVEN per-head threshold, without a median
+ * of its own: the streaming form of Med3x for decode-phase tokens, whose
+ * batches (often one token per sequence) are too small for a median of
+ * their own (the pages take the median of the current batch, gist.science/
+ * nl, Technische Samenvatting, section 3; a previous batch's threshold,
+ * e.g. the prefill's d_thr from hqmq_outlier_extract, is our reading for a
+ * batch that has none).  Outlier rule, list order and format, d_slab_off,
+ * the optional d_tile_off (list tile offsets and total, as
+ * hqmq_outlier_extract writes them), cap and status as in
+ * hqmq_outlier_extract.  The new tokens are then encoded with the same
+ * d_thr (hqmq_encode / hqmq_encode_lut).  d_thr: fp32 [H] (4-byte
+ * aligned); d_ws: hqmq_outlier_extract_given_thr_workspace_size bytes,
+ * 256-byte aligned, contents on entry ignored. */
+HQMQ_API uint64_t hqmq_outlier_extract_given_thr_workspace_size(int B, int H, int T, int D);
+HQMQ_API int hqmq_outlier_extract_given_thr(const void *d_x, int dtype, int B, int H, int T, int D,
+                                            const float *d_thr, int gran, uint32_t *d_out_idx,
+                                            uint16_t *d_out_val, uint32_t *d_slab_off,
+                                            uint32_t *d_tile_off, uint64_t cap, void *d_ws,
+                                            uint64_t ws_bytes, hqmq_status *d_status,
+                                            void *stream);
+
 /* Quantized radius (our reading of the pages' bit budget: the abstract's 3.79
  * bits per element at S = 8 is log2(24 S) / 2, i.e. about 2 log2(24 S) bits
  * per chunk, a radius code with as many levels as there are codewords).

@@ -59,6 +59,12 @@ extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int
                                      int sm_count, cudaStream_t stream);
 extern "C" uint64_t hqmq_lut_bytes_per_group(uint32_t S);
 extern "C" uint64_t hqmq_attn_workspace_bytes(int B, int Hk);
+extern "C" uint64_t hqmq_thr_extract_workspace_bytes(int B, int H, int T, int D);
+extern "C" int hqmq_launch_outlier_extract_thr(const void *x, int dtype, int B, int H, int T, int D,
+                                               const float *thr, int gran, uint32_t *out_idx,
+                                               uint16_t *out_val, uint32_t *slab_off,
+                                               uint32_t *tile_off, uint64_t cap, void *ws,
+                                               hqmq_status *st, cudaStream_t stream);
 extern "C" int hqmq_launch_quantize_radius(const uint16_t *radius, const float *thr, int B, int H,
                                            int T, int D, uint32_t S, uint32_t b, uint32_t *rwords,
                                            int sm_count, cudaStream_t stream);
@@ -405,6 +411,29 @@ int hqmq_decode_qradius(const uint32_t *d_idx_words, const uint32_t *d_rcode_wor
                                  hqmq_index_bits(S), d_out_idx, d_out_val,
                                  d_out_idx ? d_tile_off : nullptr, cap, gran, B, H, T, D, d_y,
                                  out_dtype, d_status, sm, (cudaStream_t)stream);
+}
+
+uint64_t hqmq_outlier_extract_given_thr_workspace_size(int B, int H, int T, int D) {
+    if (!shape_ok(B, H, T, D)) return 0;
+    return hqmq_thr_extract_workspace_bytes(B, H, T, D);
+}
+
+int hqmq_outlier_extract_given_thr(const void *d_x, int dtype, int B, int H, int T, int D,
+                                   const float *d_thr, int gran, uint32_t *d_out_idx,
+                                   uint16_t *d_out_val, uint32_t *d_slab_off,
+                                   uint32_t *d_tile_off, uint64_t cap, void *d_ws,
+                                   uint64_t ws_bytes, hqmq_status *d_status, void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
+    if (!d_x || !d_thr || !d_slab_off || !d_ws || (cap > 0 && (!d_out_idx || !d_out_val)))
+        return HQMQ_ERR_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_thr, 4) || !aligned(d_out_idx, 4) ||
+        !aligned(d_out_val, 4) || !aligned(d_slab_off, 4) || !aligned(d_tile_off, 4) ||
+        !aligned(d_ws, 256) || !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    if (ws_bytes < hqmq_thr_extract_workspace_bytes(B, H, T, D)) return HQMQ_ERR_WORKSPACE;
+    return hqmq_launch_outlier_extract_thr(d_x, dtype, B, H, T, D, d_thr, gran, d_out_idx,
+                                           d_out_val, d_slab_off, d_tile_off, cap, d_ws, d_status,
+                                           (cudaStream_t)stream);
 }
 
 }  // extern "C"

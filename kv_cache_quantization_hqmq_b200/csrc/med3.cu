@@ -25,6 +25,7 @@ constexpr int HIST_BINS = 2048;
 constexpr int MED_THREADS = 256;
 constexpr int MED_UNROLL = 4;        // chunks in flight per thread
 constexpr int TILE = 4096;           // chunks per extraction tile
+constexpr int LIST_TILE = 1024;      // chunks per list tile (the tile offsets callers get)
 constexpr int EXT_THREADS = 256;
 constexpr int EXT_ROWS = 8;          // rows of EXT_THREADS chunks loaded at once (count)
 constexpr int WR_ROWS = 4;           // the same for the ordered write
@@ -155,7 +156,7 @@ __device__ __forceinline__ uint32_t outlier_mask(float x0, float x1, float x2, f
            (fabsf(x3) > th ? 8u : 0u);
 }
 
-template <int DT, int GRAN>
+template <int DT, int GRAN, int TL = TILE>
 __global__ void __launch_bounds__(EXT_THREADS)
 k_extract_count(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
                 uint32_t tiles_per_slab, const float *__restrict__ thr,
@@ -163,8 +164,8 @@ k_extract_count(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
     __shared__ uint32_t s_red[EXT_THREADS / 32];
     const int slab = blockIdx.y;
     const float th = thr[slab % H];
-    const uint32_t c0 = blockIdx.x * TILE;
-    const uint32_t c1 = min(c0 + TILE, chunks_per_slab);
+    const uint32_t c0 = blockIdx.x * TL;
+    const uint32_t c1 = min(c0 + TL, chunks_per_slab);
     const uint64_t base = (uint64_t)slab * chunks_per_slab;
     uint32_t cnt = 0;
     for (uint32_t cb = c0 + threadIdx.x; cb < c1; cb += EXT_ROWS * EXT_THREADS) {
@@ -195,7 +196,8 @@ k_extract_count(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
 __global__ void __launch_bounds__(1024)
 k_extract_scan(const uint32_t *__restrict__ tile_count, uint64_t n_tiles,
                uint32_t tiles_per_slab, uint32_t n_slabs, uint64_t cap,
-               uint32_t *__restrict__ tile_off, uint32_t *__restrict__ slab_off, DevStatus *st) {
+               uint32_t *__restrict__ tile_off, uint32_t *__restrict__ slab_off, DevStatus *st,
+               bool write_total = false) {
     __shared__ uint32_t s_warp[32];
     __shared__ unsigned long long s_carry;
     if (threadIdx.x == 0) s_carry = 0;
@@ -235,6 +237,7 @@ k_extract_scan(const uint32_t *__restrict__ tile_count, uint64_t n_tiles,
     if (threadIdx.x == 0) {
         unsigned long long total = s_carry;
         slab_off[n_slabs] = (uint32_t)total;
+        if (write_total) tile_off[n_tiles] = (uint32_t)total;
         if (st) {
             atomicAdd(&st->n_outliers, total);
             if (total > cap) atomicOr(&st->flags, HQMQ_FLAG_OUTLIER_OVERFLOW);
@@ -242,7 +245,7 @@ k_extract_scan(const uint32_t *__restrict__ tile_count, uint64_t n_tiles,
     }
 }
 
-template <int DT, int GRAN>
+template <int DT, int GRAN, int TL = TILE>
 __global__ void __launch_bounds__(EXT_THREADS)
 k_extract_write(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
                 uint32_t tiles_per_slab, const float *__restrict__ thr,
@@ -252,8 +255,8 @@ k_extract_write(const void *__restrict__ x, int H, uint32_t chunks_per_slab,
     __shared__ uint32_t s_tot[WR_ROWS][NW];
     const int slab = blockIdx.y;
     const float th = thr[slab % H];
-    const uint32_t c0 = blockIdx.x * TILE;
-    const uint32_t c1 = min(c0 + TILE, chunks_per_slab);
+    const uint32_t c0 = blockIdx.x * TL;
+    const uint32_t c1 = min(c0 + TL, chunks_per_slab);
     const uint64_t base = (uint64_t)slab * chunks_per_slab;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     uint64_t pos = tile_off[(uint64_t)slab * tiles_per_slab + blockIdx.x];
@@ -400,7 +403,65 @@ static int run(const void *x, int B, int H, int T, int D, float C, float *rmed, 
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
+// The list of a call under a given per-head threshold (no median): count
+// per 1024-chunk list tile, scan, ordered write.  tile_off_out (NULL: kept
+// in the workspace) receives the list tile offsets and the total.
+inline uint64_t thr_ws_bytes(int B, int H, int T, int D, uint64_t *n_tiles_out) {
+    const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
+    const uint64_t n_tiles = (uint64_t)B * H * ((cps + LIST_TILE - 1) / LIST_TILE);
+    if (n_tiles_out) *n_tiles_out = n_tiles;
+    return align256(n_tiles * 4) + align256((n_tiles + 1) * 4);
+}
+
+template <int DT, int GRAN>
+static int run_thr(const void *x, int B, int H, int T, int D, const float *thr, uint32_t *out_idx,
+                   uint16_t *out_val, uint32_t *slab_off, uint32_t *tile_off_out, uint64_t cap,
+                   char *ws, hqmq_status *st_, cudaStream_t stream) {
+    DevStatus *st = reinterpret_cast<DevStatus *>(st_);
+    uint64_t n_tiles = 0;
+    thr_ws_bytes(B, H, T, D, &n_tiles);
+    const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
+    const uint32_t tps = (cps + LIST_TILE - 1) / LIST_TILE;
+    uint32_t *tile_count = reinterpret_cast<uint32_t *>(ws);
+    uint32_t *tile_off = tile_off_out ? tile_off_out
+                                      : reinterpret_cast<uint32_t *>(ws + align256(n_tiles * 4));
+    const int n_slabs = B * H;
+    dim3 tgrid(tps, (unsigned)n_slabs);
+    k_extract_count<DT, GRAN, LIST_TILE><<<tgrid, EXT_THREADS, 0, stream>>>(x, H, cps, tps, thr,
+                                                                              tile_count);
+    k_extract_scan<<<1, 1024, 0, stream>>>(tile_count, n_tiles, tps, (uint32_t)n_slabs, cap,
+                                           tile_off, slab_off, st, true);
+    k_extract_write<DT, GRAN, LIST_TILE><<<tgrid, EXT_THREADS, 0, stream>>>(
+        x, H, cps, tps, thr, tile_off, cap, out_idx, out_val, st);
+    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}
+
 }  // namespace hqmq
+
+extern "C" uint64_t hqmq_thr_extract_workspace_bytes(int B, int H, int T, int D) {
+    return hqmq::thr_ws_bytes(B, H, T, D, nullptr);
+}
+
+extern "C" int hqmq_launch_outlier_extract_thr(const void *x, int dtype, int B, int H, int T, int D,
+                                               const float *thr, int gran, uint32_t *out_idx,
+                                               uint16_t *out_val, uint32_t *slab_off,
+                                               uint32_t *tile_off, uint64_t cap, void *ws,
+                                               hqmq_status *st, cudaStream_t stream) {
+    using namespace hqmq;
+    char *w = reinterpret_cast<char *>(ws);
+    if (dtype == HQMQ_BF16) {
+        if (gran == HQMQ_GRAN_CHUNK)
+            return run_thr<HQMQ_BF16, HQMQ_GRAN_CHUNK>(x, B, H, T, D, thr, out_idx, out_val,
+                                                       slab_off, tile_off, cap, w, st, stream);
+        return run_thr<HQMQ_BF16, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, thr, out_idx, out_val, slab_off,
+                                                     tile_off, cap, w, st, stream);
+    }
+    if (gran == HQMQ_GRAN_CHUNK)
+        return run_thr<HQMQ_F32, HQMQ_GRAN_CHUNK>(x, B, H, T, D, thr, out_idx, out_val, slab_off,
+                                                  tile_off, cap, w, st, stream);
+    return run_thr<HQMQ_F32, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, thr, out_idx, out_val, slab_off,
+                                                tile_off, cap, w, st, stream);
+}
 
 extern "C" uint64_t hqmq_med3_workspace_bytes(int B, int H, int T, int D) {
     return hqmq::ws_layout(B, H, T, D).total;

@@ -60,6 +60,9 @@ _SIGS = {
     "hqmq_make_search_table": (_I, [_P, _U32, _U32, _P, _P]),
     "hqmq_encode_lut": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _P, _I, _P, _P, _P, _P]),
     "hqmq_quantize_radius": (_I, [_P, _P, _I, _I, _I, _I, _U32, _P, _P]),
+    "hqmq_outlier_extract_given_thr_workspace_size": (_U64, [_I, _I, _I, _I]),
+    "hqmq_outlier_extract_given_thr": (_I, [_P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _U64,
+                                            _P, _U64, _P, _P]),
     "hqmq_decode_qradius": (_I, [_P, _P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P,
                                  _I, _P, _P]),
     "hqmq_attention_workspace_size": (_U64, [_I, _I]),
@@ -212,6 +215,21 @@ def hqmq_decode(idx_words, radius, codebook, S, out_idx, out_val, slab_off, cap,
     _check("hqmq_decode", _lib.hqmq_decode(
         _ptr(idx_words), _ptr(radius), _ptr(codebook), S, _ptr(out_idx), _ptr(out_val),
         _ptr(slab_off), _ptr(tile_off), int(cap), gran, B, H, T, D, _ptr(y), _dtype_code(y),
+        _ptr(status), _stream(stream)))
+
+
+def hqmq_outlier_extract_given_thr_workspace_size(B, H, T, D):
+    return int(_lib.hqmq_outlier_extract_given_thr_workspace_size(B, H, T, D))
+
+
+def hqmq_outlier_extract_given_thr(x, thr, gran, out_idx, out_val, slab_off, cap, ws,
+                                   status=None, stream=None, tile_off=None):
+    """Med3x list of x under a given threshold thr [H] (no median of its own):
+    the streaming form for decode-phase tokens."""
+    B, H, T, D = _shape4(x)
+    _check("hqmq_outlier_extract_given_thr", _lib.hqmq_outlier_extract_given_thr(
+        _ptr(x), _dtype_code(x), B, H, T, D, _ptr(thr), gran, _ptr(out_idx), _ptr(out_val),
+        _ptr(slab_off), _ptr(tile_off), int(cap), _ptr(ws), ws.numel() * ws.element_size(),
         _ptr(status), _stream(stream)))
 
 
