@@ -911,6 +911,9 @@ extern "C" int hqmq_launch_attention(const uint16_t *q, const int *seq_len, cons
         return launch_attn<8, 8, 8, LM_ANY, 192>(a, sm_count, stream);
     }
     if (b == 10 && attn_smem(S, 8, 4, LM_ANY, 192) <= opt) {
+        // without lists there is no list scratch: 8 V-table copies fit too
+        if (lm == LM_NONE && attn_smem(S, 8, 8, LM_NONE, 192) <= opt)
+            return launch_attn<8, 8, 10, LM_NONE, 192>(a, sm_count, stream);
         if (lm == LM_NONE) return launch_attn<8, 4, 10, LM_NONE, 192>(a, sm_count, stream);
         if (lm == LM_CHUNK) return launch_attn<8, 4, 10, LM_CHUNK, 192>(a, sm_count, stream);
         return launch_attn<8, 4, 10, LM_ANY, 192>(a, sm_count, stream);
