@@ -535,6 +535,29 @@ def run_streaming(cache, iters=20, warmup=3):
         out[name] = {"us_per_step_plain": round(ms_plain * 1e3, 1),
                      "us_per_step_graph": round(ms_graph * 1e3, 1)}
         del graph
+    # all calls of the step in one launch (hqmq_append_batch), same outputs
+    cbs = cache.codebook.view(w.layers * 2, H * w.S * 4)
+    thr_all = cache.thr.view(w.layers * 2, H)
+    oi_b = oi.view(-1)
+    ov_b = ov.view(-1)
+    xb = x1.view((w.layers * 2,) + x1.shape[2:])
+
+    def batched():
+        hqmq.hqmq_append_batch(xb, thr_all, cache.gran, cbs, w.S, words.view(-1), radius.view(-1),
+                               oi_b, ov_b, so.view(-1), n_chunks, tile_off=to.view(-1))
+    ms_plain = timed(batched)
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        batched()
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(graph):
+        batched()
+    ms_graph = timed(graph.replay)
+    out["batched_one_launch"] = {"us_per_step_plain": round(ms_plain * 1e3, 1),
+                                 "us_per_step_graph": round(ms_graph * 1e3, 1)}
+    del graph
     out["outliers_last_step"] = int(so[:, :, -1].sum().item())
     return out
 

@@ -319,6 +319,26 @@ HQMQ_API int hqmq_outlier_extract_given_thr(const void *d_x, int dtype, int B, i
                                             uint64_t ws_bytes, hqmq_status *d_status,
                                             void *stream);
 
+/* n_calls small calls at once (e.g. one decode step's new tokens of every
+ * (layer, role)), one launch: for each call c the outputs equal
+ * hqmq_outlier_extract_given_thr(x_c, thr_c) followed by
+ * hqmq_encode(x_c, codebook_c, S, thr_c, gran), bit for bit (list, slab and
+ * tile offsets, index words, radii, status counts).  Every array is the
+ * calls' arrays back to back:
+ *   d_x [n_calls][B][H][T][D] (bf16 or fp32, 16-byte aligned), d_thr
+ *   [n_calls][H], d_codebook [n_calls][H][S][4] (16-byte aligned; H*S*16
+ *   <= 160 KB), d_idx_words [n_calls][hqmq_index_words(B,H,T,D,S)],
+ *   d_radius [n_calls][B*H*T*D/4], d_out_idx [n_calls][cap], d_out_val
+ *   [n_calls][cap*4] (chunk) or [n_calls][cap] (element), 8-byte aligned,
+ *   d_slab_off [n_calls][B*H+1], d_tile_off (NULL or) [n_calls]
+ *   [hqmq_list_tiles(B,H,T,D)+1]; cap < 2^32 entries per call.
+ * One CTA per call: meant for small calls, where per-launch costs dominate. */
+HQMQ_API int hqmq_append_batch(const void *d_x, int dtype, int n_calls, int B, int H, int T, int D,
+                               const float *d_thr, int gran, const float *d_codebook, uint32_t S,
+                               uint32_t *d_idx_words, uint16_t *d_radius, uint32_t *d_out_idx,
+                               uint16_t *d_out_val, uint32_t *d_slab_off, uint32_t *d_tile_off,
+                               uint64_t cap, hqmq_status *d_status, void *stream);
+
 /* Quantized radius (our reading of the pages' bit budget: the abstract's 3.79
  * bits per element at S = 8 is log2(24 S) / 2, i.e. about 2 log2(24 S) bits
  * per chunk, a radius code with as many levels as there are codewords).

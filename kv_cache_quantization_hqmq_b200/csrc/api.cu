@@ -60,6 +60,11 @@ extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int
 extern "C" uint64_t hqmq_lut_bytes_per_group(uint32_t S);
 extern "C" uint64_t hqmq_attn_workspace_bytes(int B, int Hk);
 extern "C" uint64_t hqmq_thr_extract_workspace_bytes(int B, int H, int T, int D);
+extern "C" int hqmq_launch_append(const void *x, int dtype, int n_calls, int B, int H, int T, int D,
+                                  const float *thr, int gran, const float *cb, uint32_t S,
+                                  uint32_t b, uint32_t *words, uint16_t *radius, uint32_t *out_idx,
+                                  uint16_t *out_val, uint32_t *slab_off, uint32_t *tile_off,
+                                  uint32_t cap, hqmq_status *st, cudaStream_t stream);
 extern "C" int hqmq_launch_outlier_extract_thr(const void *x, int dtype, int B, int H, int T, int D,
                                                const float *thr, int gran, uint32_t *out_idx,
                                                uint16_t *out_val, uint32_t *slab_off,
@@ -434,6 +439,29 @@ int hqmq_outlier_extract_given_thr(const void *d_x, int dtype, int B, int H, int
     return hqmq_launch_outlier_extract_thr(d_x, dtype, B, H, T, D, d_thr, gran, d_out_idx,
                                            d_out_val, d_slab_off, d_tile_off, cap, d_ws, d_status,
                                            (cudaStream_t)stream);
+}
+
+int hqmq_append_batch(const void *d_x, int dtype, int n_calls, int B, int H, int T, int D,
+                      const float *d_thr, int gran, const float *d_codebook, uint32_t S,
+                      uint32_t *d_idx_words, uint16_t *d_radius, uint32_t *d_out_idx,
+                      uint16_t *d_out_val, uint32_t *d_slab_off, uint32_t *d_tile_off,
+                      uint64_t cap, hqmq_status *d_status, void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(dtype) || !gran_ok(gran)) return HQMQ_ERR_ARG;
+    if (n_calls < 1 || n_calls > (1 << 30) || S < 1 || S > S_MAX) return HQMQ_ERR_ARG;
+    if ((uint64_t)H * S * 16 > 160 * 1024) return HQMQ_ERR_ARG;   // codebooks of a call in smem
+    if (cap >= (1ull << 32)) return HQMQ_ERR_ARG;
+    if (!d_x || !d_thr || !d_codebook || !d_idx_words || !d_radius || !d_slab_off)
+        return HQMQ_ERR_ARG;
+    if (cap > 0 && (!d_out_idx || !d_out_val)) return HQMQ_ERR_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_thr, 4) || !aligned(d_codebook, 16) ||
+        !aligned(d_idx_words, 4) || !aligned(d_radius, 2) || !aligned(d_out_idx, 4) ||
+        !aligned(d_out_val, 8) || !aligned(d_slab_off, 4) || !aligned(d_tile_off, 4) ||
+        !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    return hqmq_launch_append(d_x, dtype, n_calls, B, H, T, D, d_thr, gran, d_codebook, S,
+                              hqmq_index_bits(S), d_idx_words, d_radius, d_out_idx, d_out_val,
+                              d_slab_off, d_tile_off, (uint32_t)cap, d_status,
+                              (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -60,6 +60,8 @@ _SIGS = {
     "hqmq_make_search_table": (_I, [_P, _U32, _U32, _P, _P]),
     "hqmq_encode_lut": (_I, [_P, _I, _I, _I, _I, _I, _P, _U32, _P, _P, _I, _P, _P, _P, _P]),
     "hqmq_quantize_radius": (_I, [_P, _P, _I, _I, _I, _I, _U32, _P, _P]),
+    "hqmq_append_batch": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _U32, _P, _P, _P, _P, _P,
+                               _P, _U64, _P, _P]),
     "hqmq_outlier_extract_given_thr_workspace_size": (_U64, [_I, _I, _I, _I]),
     "hqmq_outlier_extract_given_thr": (_I, [_P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _U64,
                                             _P, _U64, _P, _P]),
@@ -231,6 +233,19 @@ def hqmq_outlier_extract_given_thr(x, thr, gran, out_idx, out_val, slab_off, cap
         _ptr(x), _dtype_code(x), B, H, T, D, _ptr(thr), gran, _ptr(out_idx), _ptr(out_val),
         _ptr(slab_off), _ptr(tile_off), int(cap), _ptr(ws), ws.numel() * ws.element_size(),
         _ptr(status), _stream(stream)))
+
+
+def hqmq_append_batch(x, thr, gran, codebook, S, idx_words, radius, out_idx, out_val, slab_off,
+                      cap, tile_off=None, status=None, stream=None):
+    """n_calls small calls in one launch; x: [n_calls, B, H, T, D]; every other
+    array holds the calls' arrays back to back (see include/hqmq.h)."""
+    if x.dim() != 5 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous [n_calls, B, H, T, D] tensor")
+    C, B, H, T, D = (int(v) for v in x.shape)
+    _check("hqmq_append_batch", _lib.hqmq_append_batch(
+        _ptr(x), _dtype_code(x), C, B, H, T, D, _ptr(thr), gran, _ptr(codebook), S,
+        _ptr(idx_words), _ptr(radius), _ptr(out_idx), _ptr(out_val), _ptr(slab_off),
+        _ptr(tile_off), int(cap), _ptr(status), _stream(stream)))
 
 
 def hqmq_quantize_radius(radius, thr, shape, S, rcode_words, stream=None):
