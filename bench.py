@@ -272,7 +272,10 @@ def one_read(w, table):
 
 
 def algorithmic_bytes(w, n_outliers_per_call, table=True):
-    """Bytes the method must move per call (Measurement)."""
+    """Bytes the method must move per call: x read once (twice when Med3x needs
+    a second read), the codes (b/8 + 2 bytes per chunk) written, 12 bytes per
+    outlier written (encode); codes and outliers read and bf16 y written
+    (decode)."""
     B, H, T, D = w.call_shape
     n_chunks = B * H * T * D // 4
     x_bytes = B * H * T * D * w.elem_bytes
@@ -291,7 +294,7 @@ def algorithmic_bytes(w, n_outliers_per_call, table=True):
 
 
 def alu_ops_per_chunk(S):
-    """Lane operations of the S-codeword search per chunk (see DESIGN.md):
+    """Lane operations of the S-codeword search per chunk:
     per secondary codeword one quaternion product (16 FMA), the 2T score
     (3 max + 3 add + 1 add + 1 max) and the argmax update (1 compare +
     2 select) = 27; per chunk ~60 more (load, norm, closed-form p, radius,

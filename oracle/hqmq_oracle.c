@@ -20,12 +20,13 @@
  *           sections 1 and 3 (same content as NL 1 / NL 3)
  *   [FR]    signal-ia-rouge.vercel.app article, section "La mecanique"
  *
- * Readings where the pages are silent (every one is listed in the design doc):
+ * Readings where the pages are silent:
  *   quaternion order (w,i,j,k) = 4 consecutive elements; Hamilton product with
  *   ij = k; the 2T enumeration p in [0,24); global index s*24+p with ties to
  *   the lowest index; codebook RNG = Philox4x32-10 + Box-Muller in fp64;
  *   fp32 chunk norm in a fixed fma order; fp16 radius; lower median; strict
- *   r > C*r_med; LSB-first bit packing in groups of 32 chunks.
+ *   r > C*r_med; LSB-first bit packing in groups of 32 chunks; the optional
+ *   quantized radius uniform on [0, thr] in 24 S levels.
  *
  * Precision: the argmax and the outlier test are integer-valued decisions, so
  * they are taken in fp32, the precision of the GPU kernels.  The codebook is
