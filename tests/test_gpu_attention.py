@@ -225,3 +225,36 @@ def test_attention_other_codebook_sizes(oracle, S):
     fewer table copies)."""
     w = WORKLOADS["qwen_outlier"].with_(S=S, heads=2, q_heads=6)
     run_case(oracle, w, B=2, T=96, seq_len=[96, 40])
+
+
+def test_attention_list_truncated_at_cap(oracle):
+    """A list whose writer ran out of room: only the entries below cap exist
+    (the tile offsets still count all of them); the chunks past cap keep
+    their zeroed codes, exactly as hqmq_decode reads them."""
+    w = WORKLOADS["qwen_outlier"].with_(heads=2, q_heads=6)
+    B, T, D, H = 1, 256, 128, 2
+    G = w.n_q_heads // H
+    kc = oracle_cache(oracle, w, 0, 0, B, T)
+    vc = oracle_cache(oracle, w, 0, 1, B, T)
+    kd, keep_k = device_codes(kc, B, H, T, D)
+    vd, keep_v = device_codes(vc, B, H, T, D)
+    cap_k, cap_v = len(kc["idx"]) // 2, len(vc["idx"]) // 3
+    kd.cap, vd.cap = cap_k, cap_v                     # the tile offsets keep the full counts
+    q = make_query(w, 0, batch=B)
+    o = torch.empty(B, w.n_q_heads, D, dtype=torch.float32, device="cuda")
+    hqmq.hqmq_attention_decode(q.cuda(), kd, vd, w.S, H, T, o, hqmq.alloc_attention_ws(B, H))
+    torch.cuda.synchronize()
+
+    def trunc_decode(c, cap):
+        y, _ = oracle.decode(c["words"], c["radius"], c["cb"], w.S, B, H, T, D, c["idx"][:cap],
+                             c["val"][:cap], 0, oracle.BF16)
+        return oracle.bf16_to_f32(y).reshape(B, H, T, D)
+
+    kt, vt = trunc_decode(kc, cap_k), trunc_decode(vc, cap_v)
+    qb = as_numpy_bits(q)
+    ref = oracle.attention_decode(qb, kt, vt, D ** -0.5, G)
+    tol = 2 * bound(qb, kt, vt, ref, D ** -0.5, G, None, T)[:, :, None]
+    err = np.abs(o.cpu().numpy() - ref)
+    assert (err <= tol).all(), (err / tol).max()
+    full = oracle.attention_decode(qb, kc["y"], vc["y"], D ** -0.5, G)
+    assert np.abs(full - ref).max() > 10 * tol.max()    # the truncation does change the result
