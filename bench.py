@@ -444,7 +444,27 @@ def run_qradius(cache, peaks, iters=20, warmup=3):
     n_out = int(cache.slab_off[0, 0][-1].item())
     q_bytes = n_chunks * (2 + b / 8)
     d_bytes = n_chunks * (2 * b / 8 + 8) + 12 * n_out
+    # decode-phase attention over both caches in the quantized format
+    att = None
+    Hq = w.n_q_heads
+    if D == 128 and Hq % H == 0 and Hq // H <= 8:
+        from kv_cache_quantization_hqmq_b200 import workloads as W
+        rwv = torch.empty(cache.n_words, dtype=torch.int32, device=dev)
+        hqmq.hqmq_quantize_radius(cache.radius[0, 1], cache.thr[0, 1], cache.shape, w.S, rwv)
+        kvs = [hqmq.kv_codes(cache.words[0, r], None, cache.codebook[r * H * w.S * 4:(r + 1) * H * w.S * 4],
+                             cache.out_idx[0, r], cache.out_val[0, r], cache.tile_off[0, r], cache.cap,
+                             cache.gran, rcode_words=(rw if r == 0 else rwv), thr=cache.thr[0, r])
+               for r in range(2)]
+        q = W.make_query(w, 0, device=dev)
+        o = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+        aws = hqmq.alloc_attention_ws(B, H, device=dev)
+        ms_a = timed(lambda: hqmq.hqmq_attention_decode(q, kvs[0], kvs[1], w.S, H, T, o, aws))
+        n_list = n_out + int(cache.slab_off[0, 1][-1].item())
+        a_bytes = 2 * B * H * T * (8 * b) + n_list * 12
+        att = {"ms_per_call": round(ms_a, 4), "algorithmic_bytes": a_bytes,
+               "hbm_frac": round(a_bytes / (ms_a * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
     return {"op": "hqmq_quantize_radius + hqmq_decode_qradius (layer 0, K)",
+            "attention_from_quantized_codes": att,
             "levels": 24 * w.S, "code_bits_per_chunk": 2 * b,
             "bits_per_element": round(2 * b / 4 + n_out * 96 / (B * H * T * D), 4),
             "bits_per_element_fp16_radius": round((b + 16) / 4 + n_out * 96 / (B * H * T * D), 4),

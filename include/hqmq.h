@@ -377,7 +377,9 @@ HQMQ_API int hqmq_decode_qradius(const uint32_t *d_idx_words, const uint32_t *d_
  * [Hk][S][4], 16-byte aligned).  out_idx == NULL: no outlier list; else
  * out_val (8-byte aligned), tile_off (uint32 [hqmq_list_tiles(B,Hk,T,128) +
  * 1]) and cap are the list, its tile offsets and the cap of that call, gran
- * its granularity. */
+ * its granularity.  Quantized radius: rcode_words (as hqmq_quantize_radius
+ * writes them) and thr (fp32 [Hk], their range) replace radius, which may then
+ * be NULL; K and V must then both be given this way. */
 typedef struct {
     const uint32_t *idx_words;
     const uint16_t *radius;
@@ -387,6 +389,8 @@ typedef struct {
     const uint32_t *tile_off;
     uint64_t cap;
     int gran;
+    const uint32_t *rcode_words;
+    const float *thr;
 } hqmq_kv_codes;
 
 /* Bytes of device workspace hqmq_attention_decode needs for B x Hk KV heads
@@ -399,7 +403,8 @@ HQMQ_API uint64_t hqmq_attention_workspace_size(int B, int Hk);
  * "Memory en Latentie"), so the dense K and V are never written.
  * For each batch b, query head h (GQA: KV head hk = h / G, G = Hq / Hk, so
  * query heads hk*G .. hk*G + G - 1 share KV head hk):
- *   K^, V^ = exactly what hqmq_decode writes as bf16 for the two caches
+ *   K^, V^ = exactly what hqmq_decode (or, with radius codes,
+ *            hqmq_decode_qradius) writes as bf16 for the two caches
  *            (codes, radius and outlier list);
  *   s_t    = scale * <q[b][h], K^[b][hk][t]>, for t < len_b;
  *   o[b][h] = sum_t softmax(s)_t V^[b][hk][t],

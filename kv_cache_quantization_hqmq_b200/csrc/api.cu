@@ -147,7 +147,9 @@ int smem_optin() {
 
 // A coded cache of hqmq_attention_decode: pointers present and aligned.
 int kv_codes_check(const hqmq_kv_codes *c) {
-    if (!c || !c->idx_words || !c->radius || !c->codebook) return HQMQ_ERR_ARG;
+    if (!c || !c->idx_words || !c->codebook) return HQMQ_ERR_ARG;
+    if (c->rcode_words ? !c->thr : !c->radius) return HQMQ_ERR_ARG;
+    if (!aligned(c->rcode_words, 4) || !aligned(c->thr, 4)) return HQMQ_ERR_ALIGN;
     if (c->out_idx && (!c->out_val || !c->tile_off || !gran_ok(c->gran))) return HQMQ_ERR_ARG;
     if (!aligned(c->idx_words, 4) || !aligned(c->radius, 16) || !aligned(c->codebook, 16) ||
         !aligned(c->out_idx, 4) || !aligned(c->out_val, 8) || !aligned(c->tile_off, 4))
@@ -374,6 +376,7 @@ int hqmq_attention_decode(const uint16_t *d_q, const int32_t *d_seq_len, const h
     int rc = kv_codes_check(k);
     if (rc == HQMQ_OK) rc = kv_codes_check(v);
     if (rc != HQMQ_OK) return rc;
+    if ((k->rcode_words == nullptr) != (v->rcode_words == nullptr)) return HQMQ_ERR_ARG;
     if (!aligned(d_q, 8) || !aligned(d_o, 4) || !aligned(d_seq_len, 4) || !aligned(d_ws, 256) ||
         !aligned(d_status, 8))
         return HQMQ_ERR_ALIGN;

@@ -79,6 +79,8 @@ struct KVDev {
     const uint32_t *tile_off;   // list position of each 1024-chunk tile's first entry
     uint32_t cap32;
     int gran;
+    const uint32_t *rwords;     // quantized radius: b-bit codes laid out like the indices
+    const float *thr;           // [Hk]: the range of the codes
 };
 
 struct AttnArgs {
@@ -145,6 +147,8 @@ template <int BT> struct BlockRegs {
     uint32_t kw[2][Geo<BT>::KW];
     uint2 vr[4];
     uint32_t vw[4][Geo<BT>::VW];
+    uint32_t krw[2][Geo<BT>::KW];             // RQ: radius-code words (same geometry)
+    uint32_t vrw[4][Geo<BT>::VW];
 };
 
 // Per-lane base pointers of the block loads at token 0 of the slab: K
@@ -153,11 +157,12 @@ struct LanePtrs {
     const uint32_t *kw, *vw;
     const uint4 *kr;
     const uint2 *vr;
+    const uint32_t *krw, *vrw;                // RQ: radius-code words
 };
 
 // Loads of the block starting at token t0 (tokens >= len read as zero);
 // kneed / vneed: the words a run spans (BT = 0).
-template <int BT>
+template <int BT, int RQ>
 __device__ __forceinline__ void load_block(const LanePtrs &P, uint32_t b, int t0, int len,
                                            int lane, uint32_t kneed, uint32_t vneed,
                                            BlockRegs<BT> &R) {
@@ -166,21 +171,33 @@ __device__ __forceinline__ void load_block(const LanePtrs &P, uint32_t b, int t0
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         const bool ok = t0 + n + 8 * j < len;
-        R.kr[j] = ok ? __ldcs(P.kr + (size_t)(t0 + 8 * j) * 4) : make_uint4(0u, 0u, 0u, 0u);
+        if (!RQ) R.kr[j] = ok ? __ldcs(P.kr + (size_t)(t0 + 8 * j) * 4) : make_uint4(0u, 0u, 0u, 0u);
         const uint32_t *w = P.kw + tb + 8 * j * b;
 #pragma unroll
         for (int i = 0; i < Geo<BT>::KW; ++i)
             R.kw[j][i] = (ok && (BT || (uint32_t)i < kneed)) ? __ldg(w + i) : 0u;
+        if (RQ) {
+            const uint32_t *rw = P.krw + tb + 8 * j * b;
+#pragma unroll
+            for (int i = 0; i < Geo<BT>::KW; ++i)
+                R.krw[j][i] = (ok && (BT || (uint32_t)i < kneed)) ? __ldcs(rw + i) : 0u;
+        }
     }
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
         const int dt = (s & 1) + 8 * (s >> 1);
         const bool ok = t0 + 2 * q + dt < len;
-        R.vr[s] = ok ? __ldcs(P.vr + (size_t)(t0 + dt) * 8) : make_uint2(0u, 0u);
+        if (!RQ) R.vr[s] = ok ? __ldcs(P.vr + (size_t)(t0 + dt) * 8) : make_uint2(0u, 0u);
         const uint32_t *w = P.vw + tb + dt * b;
 #pragma unroll
         for (int i = 0; i < Geo<BT>::VW; ++i)
             R.vw[s][i] = (ok && (BT || (uint32_t)i < vneed)) ? __ldg(w + i) : 0u;
+        if (RQ) {
+            const uint32_t *rw = P.vrw + tb + dt * b;
+#pragma unroll
+            for (int i = 0; i < Geo<BT>::VW; ++i)
+                R.vrw[s][i] = (ok && (BT || (uint32_t)i < vneed)) ? __ldcs(rw + i) : 0u;
+        }
     }
 }
 
@@ -414,7 +431,7 @@ __device__ __forceinline__ void scale_cw(float r, const float4 &cw, float (&v)[4
 // or any lists (bitmaps; element mode).
 constexpr int LM_NONE = 0, LM_CHUNK = 1, LM_ANY = 2;
 
-template <int RK, int RV, int BT, int LM, int LC>
+template <int RK, int RV, int BT, int LM, int LC, int RQ>
 __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
     extern __shared__ float4 s_dyn[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -487,13 +504,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
     LanePtrs P;
     P.kw = a.k.words + (slab_g0 + n) * b + (kb0 >> 5);
     P.vw = a.v.words + (slab_g0 + 2 * q) * b + (vb0 >> 5);
-    P.kr = reinterpret_cast<const uint4 *>(a.k.radius + (slab_g0 + n) * 32) + q;
-    P.vr = reinterpret_cast<const uint2 *>(a.v.radius + (slab_g0 + 2 * q) * 32) + n;
+    P.kr = RQ ? nullptr : reinterpret_cast<const uint4 *>(a.k.radius + (slab_g0 + n) * 32) + q;
+    P.vr = RQ ? nullptr : reinterpret_cast<const uint2 *>(a.v.radius + (slab_g0 + 2 * q) * 32) + n;
+    P.krw = RQ ? a.k.rwords + (slab_g0 + n) * b + (kb0 >> 5) : nullptr;
+    P.vrw = RQ ? a.v.rwords + (slab_g0 + 2 * q) * b + (vb0 >> 5) : nullptr;
+    const float dk = RQ ? qr_delta(__ldg(a.k.thr + hk), nw) : 0.0f;   // radius steps (RQ)
+    const float dv = RQ ? qr_delta(__ldg(a.v.thr + hk), nw) : 0.0f;
     BlockRegs<BT> cur, nxt;
-    if (wb0 < wb1) load_block<BT>(P, b, wb0 * ATT_BLK, len, lane, kneed, vneed, cur);
+    if (wb0 < wb1) load_block<BT, RQ>(P, b, wb0 * ATT_BLK, len, lane, kneed, vneed, cur);
     for (int blk = wb0; blk < wb1; ++blk) {
         const int t0 = blk * ATT_BLK;
-        if (blk + 1 < wb1) load_block<BT>(P, b, t0 + ATT_BLK, len, lane, kneed, vneed, nxt);
+        if (blk + 1 < wb1) load_block<BT, RQ>(P, b, t0 + ATT_BLK, len, lane, kneed, vneed, nxt);
         const int tau = t0 >> 5, par = tau & 1;
         if ((klist || vlist) && (blk == wb0 || (t0 & 31) == 0)) {
             // entering list tile tau: stage tile tau + 1, make sure tau is in
@@ -550,14 +571,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
         for (int j = 0; j < 2; ++j) {
             sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
             sd[j][0] = sd[j][1] = sd[j][2] = sd[j][3] = 0.f;
-            Run<BT, Geo<BT>::KW> rk;
+            Run<BT, Geo<BT>::KW> rk, rkr;
             rk.init(cur.kw[j], kbo);
+            if (RQ) rkr.init(cur.krw[j], kbo);
             const uint32_t rr[4] = {cur.kr[j].x, cur.kr[j].y, cur.kr[j].z, cur.kr[j].w};
+            // radius of K chunk 8 q + ks: fp16, or from its code (RQ)
+            auto krad = [&](int ks) -> float {
+                return RQ ? qr_radius(rkr.get(ks, b, mask), nw, dk)
+                          : f16_bits_to_f32((rr[ks >> 1] >> (16 * (ks & 1))) & 0xFFFFu);
+            };
             uint32_t kf0[8], kf1[8];
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t id = min(rk.get(ks, b, mask), nw);
-                const float r = f16_bits_to_f32((rr[ks >> 1] >> (16 * (ks & 1))) & 0xFFFFu);
+                const float r = krad(ks);
                 float v[4];
                 scale_cw(r, cw_lookup<RK>(s_tk, cbk, id, nw, lane), v);
                 kf0[ks] = pack_bf16(v[0], v[1]);
@@ -588,7 +615,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
                             float v[4] = {0.f, 0.f, 0.f, 0.f};
                             if (ke) {
                                 const uint32_t id = min(rk.get(ks, b, mask), nw);
-                                const float r = f16_bits_to_f32((rr[ks >> 1] >> (16 * (ks & 1))) & 0xFFFFu);
+                                const float r = krad(ks);
                                 scale_cw(r, cw_lookup<RK>(s_tk, cbk, id, nw, lane), v);
                             }
                             patch_values<LC>(a.k, LK, WL.bm(0), WL.pre(0), WL.val[par][0], kt0,
@@ -645,11 +672,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
 
         // ---- O^T += V^T P^T: V^ decoded straight into A fragments; tile
         //      2 i + h, slot n + 8 v holds element 2 h + v of chunk 4 n + i ----
-        Run<BT, Geo<BT>::VW> rv[4];
+        Run<BT, Geo<BT>::VW> rv[4], rvr[4];
         uint32_t lv[4] = {0u, 0u, 0u, 0u}, lvor = 0;
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             rv[s].init(cur.vw[s], vbo);
+            if (RQ) rvr[s].init(cur.vrw[s], vbo);
             if (vany) {
                 const uint32_t tl = (uint32_t)(2 * q + (s & 1) + 8 * (s >> 1));
                 if constexpr (LM == LM_CHUNK)
@@ -667,7 +695,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
             for (int s = 0; s < 4; ++s) {
                 const uint32_t id = min(rv[s].get(i, b, mask), nw);
                 const uint32_t rw = i < 2 ? cur.vr[s].x : cur.vr[s].y;
-                const float r = f16_bits_to_f32((rw >> (16 * (i & 1))) & 0xFFFFu);
+                const float r = RQ ? qr_radius(rvr[s].get(i, b, mask), nw, dv)
+                                   : f16_bits_to_f32((rw >> (16 * (i & 1))) & 0xFFFFu);
                 scale_cw(r, cw_lookup<RV>(s_tv, cbv, id, nw, lane), v[s]);
             }
             if constexpr (LM == LM_CHUNK) {
@@ -816,6 +845,8 @@ inline KVDev kv_dev(const hqmq_kv_codes *c) {
     d.tile_off = c->out_idx && c->cap > 0 ? c->tile_off : nullptr;
     d.cap32 = c->cap < 0xFFFFFFFFull ? (uint32_t)c->cap : 0xFFFFFFFFu;
     d.gran = c->gran;
+    d.rwords = c->rcode_words;
+    d.thr = c->thr;
     return d;
 }
 
@@ -843,9 +874,9 @@ inline int attn_plan(int n_heads, int T, int slots) {
     return best;
 }
 
-template <int RK, int RV, int BT, int LM, int LC>
-static int launch_attn(AttnArgs &a, int sm_count, cudaStream_t stream) {
-    auto kern = k_attn<RK, RV, BT, LM, LC>;
+template <int RK, int RV, int BT, int LM, int LC, int RQ>
+static int launch_attn1(AttnArgs &a, int sm_count, cudaStream_t stream) {
+    auto kern = k_attn<RK, RV, BT, LM, LC, RQ>;
     const size_t smem = attn_smem(a.S, RK, RV, LM, LC);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
@@ -861,6 +892,12 @@ static int launch_attn(AttnArgs &a, int sm_count, cudaStream_t stream) {
         return HQMQ_ERR_CUDA;
     kern<<<(unsigned)(n_heads * a.cph), ATT_THREADS, smem, stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}
+
+template <int RK, int RV, int BT, int LM, int LC>
+static int launch_attn(AttnArgs &a, int sm_count, cudaStream_t stream) {
+    if (a.k.rwords) return launch_attn1<RK, RV, BT, LM, LC, 1>(a, sm_count, stream);
+    return launch_attn1<RK, RV, BT, LM, LC, 0>(a, sm_count, stream);
 }
 
 }  // namespace hqmq

@@ -36,17 +36,6 @@ __device__ __forceinline__ uint32_t get_index(const uint32_t *__restrict__ words
     return (uint32_t)(v >> o) & ((1u << b) - 1u);
 }
 
-// Quantized-radius mode: the step delta = fl32(thr / (L - 1)) of a head
-// (0 unless thr is a positive finite value), and the radius fl32(k delta) of
-// level k (codes >= L read as L - 1).
-__device__ __forceinline__ float qr_delta(float thr, uint32_t L) {
-    if (!(thr > 0.0f) || isinf(thr) || L < 2u) return 0.0f;
-    return __fdiv_rn(thr, (float)(L - 1u));
-}
-__device__ __forceinline__ float qr_radius(uint32_t k, uint32_t L, float delta) {
-    return __fmul_rn((float)(k < L ? k : L - 1u), delta);
-}
-
 // fl32(fl32(r c_e) + v) of element e of chunk j, r and c from the chunk's
 // code (the main pass's product), v the list's fp16 value; a bad index gives
 // r = 0.  RQ: r from the chunk's radius code (rwords, delta).

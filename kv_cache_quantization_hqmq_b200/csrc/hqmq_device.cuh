@@ -176,6 +176,17 @@ __device__ __forceinline__ float4 codeword(int p, float4 q) {
     return c;
 }
 
+// Quantized-radius mode: the step delta = fl32(thr / (L - 1)) of a head
+// (0 unless thr is a positive finite value), and the radius fl32(k delta) of
+// level k (codes >= L read as L - 1).
+__device__ __forceinline__ float qr_delta(float thr, uint32_t L) {
+    if (!(thr > 0.0f) || isinf(thr) || L < 2u) return 0.0f;
+    return __fdiv_rn(thr, (float)(L - 1u));
+}
+__device__ __forceinline__ float qr_radius(uint32_t k, uint32_t L, float delta) {
+    return __fmul_rn((float)(k < L ? k : L - 1u), delta);
+}
+
 __device__ __forceinline__ void status_add(DevStatus *st, unsigned flag,
                                            unsigned long long *ctr, unsigned long long n) {
     if (st && n) {

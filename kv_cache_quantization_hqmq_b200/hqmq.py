@@ -270,16 +270,19 @@ def hqmq_decode_qradius(idx_words, rcode_words, thr, codebook, S, out_idx, out_v
 class KVCodes(ctypes.Structure):
     """hqmq_kv_codes: one coded K or V cache (device pointers)."""
     _fields_ = [("idx_words", _P), ("radius", _P), ("codebook", _P), ("out_idx", _P),
-                ("out_val", _P), ("tile_off", _P), ("cap", _U64), ("gran", _I)]
+                ("out_val", _P), ("tile_off", _P), ("cap", _U64), ("gran", _I),
+                ("rcode_words", _P), ("thr", _P)]
 
 
 def kv_codes(idx_words, radius, codebook, out_idx=None, out_val=None, tile_off=None, cap=0,
-             gran=HQMQ_GRAN_CHUNK):
+             gran=HQMQ_GRAN_CHUNK, rcode_words=None, thr=None):
     """The hqmq_kv_codes record of one coded cache (the tensors must outlive
-    the calls that use it)."""
+    the calls that use it).  rcode_words + thr: the quantized-radius format
+    (radius may then be None)."""
     c = KVCodes(_ptr(idx_words), _ptr(radius), _ptr(codebook), _ptr(out_idx), _ptr(out_val),
-                _ptr(tile_off), int(cap) if out_idx is not None else 0, int(gran))
-    c._keep = (idx_words, radius, codebook, out_idx, out_val, tile_off)
+                _ptr(tile_off), int(cap) if out_idx is not None else 0, int(gran),
+                _ptr(rcode_words), _ptr(thr))
+    c._keep = (idx_words, radius, codebook, out_idx, out_val, tile_off, rcode_words, thr)
     return c
 
 

@@ -43,8 +43,10 @@ if not torch.cuda.is_available():
 U = 2.0 ** -24
 
 
-def oracle_cache(oracle, w, layer, role, B, T, gran=0, med3=None):
-    """Oracle-written codes (and list) of one cache, and its bf16 decode as fp32."""
+def oracle_cache(oracle, w, layer, role, B, T, gran=0, med3=None, rq=False):
+    """Oracle-written codes (and list) of one cache, and its bf16 decode as fp32
+    (rq: with the radius quantized on [0, range], range = thr in chunk mode and
+    2 thr in element mode)."""
     S = w.S
     H, D = w.heads, w.head_dim
     x = as_numpy_bits(make_call_input(w, layer, role, tokens=T, batch=B))
@@ -54,8 +56,15 @@ def oracle_cache(oracle, w, layer, role, B, T, gran=0, med3=None):
         _, thr = oracle.med3_threshold(x, w.C, gran)
         idx, val, _, _, _ = oracle.extract(x, thr, gran)
     words, radius, _, _, _ = oracle.encode(x, cb, S, thr, gran)
-    y, _ = oracle.decode(words, radius, cb, S, B, H, T, D, idx, val, gran, oracle.BF16)
-    return dict(words=words, radius=radius, cb=cb, idx=idx, val=val, gran=gran,
+    rw = rng_ = None
+    if rq:
+        rng_ = (thr * (2 if gran else 1)).astype(np.float32)
+        rw = oracle.quantize_radius(radius, rng_, B, H, T, D, S)
+        y, _ = oracle.decode_qradius(words, rw, rng_, cb, S, B, H, T, D, idx, val, gran,
+                                     oracle.BF16)
+    else:
+        y, _ = oracle.decode(words, radius, cb, S, B, H, T, D, idx, val, gran, oracle.BF16)
+    return dict(words=words, radius=radius, cb=cb, idx=idx, val=val, gran=gran, rw=rw, rrange=rng_,
                 y=oracle.bf16_to_f32(y).reshape(B, H, T, D))
 
 
@@ -68,9 +77,17 @@ def device_codes(c, B, H, T, D, reps=1):
     rd = torch.from_numpy(np.ascontiguousarray(np.tile(radius, (1, reps))).view(np.int16).reshape(-1))
     assert wd.numel() == B * H * T * reps * D // 128 * b
     dev = dict(words=wd.cuda(), radius=rd.cuda(), cb=torch.from_numpy(c["cb"].reshape(-1)).cuda())
+    qr = {}
+    if c.get("rw") is not None:
+        rw = c["rw"].reshape(B * H, -1)
+        dev["rw"] = torch.from_numpy(np.ascontiguousarray(np.tile(rw, (1, reps))).view(np.int32)
+                                     .reshape(-1)).cuda()
+        dev["rrange"] = torch.from_numpy(c["rrange"]).cuda()
+        dev["radius"] = None
+        qr = dict(rcode_words=dev["rw"], thr=dev["rrange"])
     idx, val = c["idx"], c["val"]
     if idx is None or len(idx) == 0:
-        return hqmq.kv_codes(dev["words"], dev["radius"], dev["cb"]), dev
+        return hqmq.kv_codes(dev["words"], dev["radius"], dev["cb"], **qr), dev
     el = 4 if c["gran"] else 1                       # list units per chunk
     cps = T * D // 4 * el                            # units per slab, one period
     slab, off = np.asarray(idx, np.int64) // cps, np.asarray(idx, np.int64) % cps
@@ -84,7 +101,7 @@ def device_codes(c, B, H, T, D, reps=1):
                val=torch.from_numpy(np.ascontiguousarray(vt).view(np.int16).reshape(-1)).cuda(),
                to=torch.from_numpy(to.view(np.int32)).cuda())
     return hqmq.kv_codes(dev["words"], dev["radius"], dev["cb"], dev["idx"], dev["val"],
-                         dev["to"], len(tiled), c["gran"]), dev
+                         dev["to"], len(tiled), c["gran"], **qr), dev
 
 
 def bound(q_bits, k, v, o_ref, scale, G, seq_len, T):
@@ -113,11 +130,11 @@ def hqmq_bf16(bits):
 
 
 def run_case(oracle, w, B, T, seq_len=None, gran=0, out_dtype=torch.float32, layer=0, reps=1,
-             med3=None):
+             med3=None, rq=False):
     H, D, Hq = w.heads, w.head_dim, w.n_q_heads
     G = Hq // H
-    kc = oracle_cache(oracle, w, layer, 0, B, T, gran, med3)
-    vc = oracle_cache(oracle, w, layer, 1, B, T, gran, med3)
+    kc = oracle_cache(oracle, w, layer, 0, B, T, gran, med3, rq)
+    vc = oracle_cache(oracle, w, layer, 1, B, T, gran, med3, rq)
     kd, keep_k = device_codes(kc, B, H, T, D, reps)
     vd, keep_v = device_codes(vc, B, H, T, D, reps)
     q = make_query(w, layer, batch=B)
@@ -258,3 +275,17 @@ def test_attention_list_truncated_at_cap(oracle):
     assert (err <= tol).all(), (err / tol).max()
     full = oracle.attention_decode(qb, kc["y"], vc["y"], D ** -0.5, G)
     assert np.abs(full - ref).max() > 10 * tol.max()    # the truncation does change the result
+
+
+def test_attention_quantized_radius_gqa7_list(oracle):
+    """K and V with radius codes (5 bits per element with the index at S = 32)."""
+    run_case(oracle, WORKLOADS["qwen_outlier"], B=2, T=600, seq_len=[600, 257], rq=True)
+
+
+def test_attention_quantized_radius_element_mode(oracle):
+    w = WORKLOADS["llama3_70b_128k"].with_(heads=2, q_heads=16)
+    run_case(oracle, w, B=1, T=512, gran=1, rq=True)
+
+
+def test_attention_quantized_radius_full_size_70b_128k(oracle):
+    run_case(oracle, WORKLOADS["llama3_70b_128k"], B=1, T=1024, reps=128, rq=True)
