@@ -289,3 +289,12 @@ def test_attention_quantized_radius_element_mode(oracle):
 
 def test_attention_quantized_radius_full_size_70b_128k(oracle):
     run_case(oracle, WORKLOADS["llama3_70b_128k"], B=1, T=1024, reps=128, rq=True)
+
+
+def test_attention_many_sequences(oracle):
+    """160 (b, hk) heads: one CTA per head writes the output directly (no CTA
+    partials); ragged lengths."""
+    w = WORKLOADS["llama3_8b"].with_(heads=4, q_heads=16)
+    B = 40
+    lens = [(7 * i) % 97 + 1 for i in range(B)]
+    run_case(oracle, w, B=B, T=96, seq_len=lens)
