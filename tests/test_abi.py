@@ -85,3 +85,56 @@ def test_bad_arguments_rejected_without_cuda(lib):
                                     good, good, good, good, None, 16, good, 1 << 20, st, None) == 1
     assert lib.hqmq_outlier_extract(good, 0, 1, 1, 8, 128, ctypes.c_float(3.0), 0, good, good,
                                     good, good, good, None, 16, good, 16, st, None) == 4
+
+
+def test_next_row_queries_and_argument_checks(lib):
+    """The attention, quantized-radius, given-threshold and batched-append
+    entry points: size queries, and synchronous rejection of bad arguments
+    (no CUDA call is made)."""
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    # workspace sizes
+    assert hqmq.hqmq_attention_workspace_size(1, 8) > 1024 * 8 * 130 * 4
+    assert hqmq.hqmq_attention_workspace_size(0, 8) == 0
+    assert hqmq.hqmq_outlier_extract_given_thr_workspace_size(1, 8, 1, 128) > 0
+    assert hqmq.hqmq_outlier_extract_given_thr_workspace_size(1, 8, 1, 6) == 0
+    # attention: D must be 128, G <= 8, Hq a multiple of Hk, a finite scale
+    codes = hqmq.KVCodes(good, good, good, None, None, None, 0, 0, None, None)
+    ref = ctypes.byref(codes)
+    F = ctypes.c_float
+    ws = 1 << 30
+    assert lib.hqmq_attention_decode(good, None, ref, ref, 8, 1, 8, 8, 64, 64, F(0.1), good, 1,
+                                     good, ws, None, None) == 1          # D = 64
+    assert lib.hqmq_attention_decode(good, None, ref, ref, 8, 1, 72, 8, 64, 128, F(0.1), good, 1,
+                                     good, ws, None, None) == 1          # G = 9
+    assert lib.hqmq_attention_decode(good, None, ref, ref, 8, 1, 12, 8, 64, 128, F(0.1), good, 1,
+                                     good, ws, None, None) == 1          # Hq % Hk != 0
+    assert lib.hqmq_attention_decode(good, None, ref, ref, 8, 1, 8, 8, 64, 128, F(float("nan")),
+                                     good, 1, good, ws, None, None) == 1  # scale NaN
+    assert lib.hqmq_attention_decode(good, None, ref, ref, 8, 1, 8, 8, 64, 128, F(0.1), good, 1,
+                                     good, 16, None, None) == 4          # workspace too small
+    qr = hqmq.KVCodes(good, None, good, None, None, None, 0, 0, good, good)
+    assert lib.hqmq_attention_decode(good, None, ref, ctypes.byref(qr), 8, 1, 8, 8, 64, 128,
+                                     F(0.1), good, 1, good, ws, None, None) == 1  # mixed formats
+    noradius = hqmq.KVCodes(good, None, good, None, None, None, 0, 0, None, None)
+    assert lib.hqmq_attention_decode(good, None, ctypes.byref(noradius), ctypes.byref(noradius),
+                                     8, 1, 8, 8, 64, 128, F(0.1), good, 1, good, ws, None,
+                                     None) == 1                         # no radius of any form
+    # quantized radius
+    assert lib.hqmq_quantize_radius(good, good, 1, 1, 32, 128, 0, good, None) == 1
+    assert lib.hqmq_quantize_radius(None, good, 1, 1, 32, 128, 8, good, None) == 1
+    assert lib.hqmq_decode_qradius(good, good, good, good, 8, good, good, None, 16, 0, 1, 1, 32,
+                                   128, good, 0, None, None) == 1       # a list needs tile_off
+    # given-threshold list: workspace too small, misaligned threshold
+    assert lib.hqmq_outlier_extract_given_thr(good, 0, 1, 8, 1, 128, good, 0, good, good, good,
+                                              None, 64, good, 16, None, None) == 4
+    assert lib.hqmq_outlier_extract_given_thr(good, 0, 1, 8, 1, 128, P((1 << 20) + 2), 0, good,
+                                              good, good, None, 64, good, 1 << 20, None, None) == 2
+    # batched append: codebooks of a call must fit in shared memory; cap < 2^32
+    assert lib.hqmq_append_batch(good, 0, 4, 1, 64, 1, 128, good, 0, good, 1000, good, good, good,
+                                 good, good, None, 64, None, None) == 1
+    assert lib.hqmq_append_batch(good, 0, 4, 1, 8, 1, 128, good, 0, good, 32, good, good, good,
+                                 good, good, None, 1 << 33, None, None) == 1
+    assert lib.hqmq_append_batch(good, 0, 0, 1, 8, 1, 128, good, 0, good, 32, good, good, good,
+                                 good, good, None, 64, None, None) == 1
