@@ -265,6 +265,12 @@ class Cache:
                     timers["decode"].append((t1, t2))
 
 
+# DRAM bytes (read + write) of one one-read hqmq_encode_med3 call, from one ncu
+# capture of its four kernels (k_sample_window, k_encode_lut, k_finalize,
+# k_list_fix) on a call of this shape; valid while those kernels are unchanged.
+MED3_CALL_TRAFFIC = {((1, 8, 131072, 128), 32): 461744128 + 68536064}
+
+
 def one_read(w, table):
     """True when hqmq_encode_med3 reads x once: with search tables, since the
     bench runs Med3x in chunk mode."""
@@ -717,7 +723,12 @@ def run_hqmq(args):
             name = "hqmq_encode_med3 (two reads of x: k_sample_window, k_pass_b, k_finalize, k_encode_lut)"
         roof = {"kernel": name, "bound": "hbm", "achieved": kern[enc_key]["hbm_gbs"],
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kern[enc_key]["hbm_frac"],
-                "traffic": None, "peak_source": peaks["source"]}
+                "traffic": MED3_CALL_TRAFFIC.get((w.call_shape, w.S)) if w.med3 and one_read(
+                    w, cache.table is not None) else None,
+                "peak_source": peaks["source"]}
+        if roof["traffic"] is not None:
+            roof["traffic_source"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4 "
+                                      "kernels of one call of this shape (profiles/)")
 
     cache_bytes = w.cache_bytes
     value = world * cache_bytes / (ms_step * 1e-3) / 1e9
