@@ -8,6 +8,23 @@ raises.
 Entry points keep the C names.  Tensors are passed where the C ABI takes
 device pointers; shapes and dtypes are read from them; `stream` defaults to
 torch's current stream.  Non-zero return codes raise HQMQError.
+
+A serving flow, per (layer, role) cache x [B, H, T, 128] (bf16):
+
+    hqmq_make_codebook(seed, S, n_groups, 0, cb)          # once per model
+    hqmq_make_search_table(cb_call, S, H, table)          # once per model (S <= 48)
+    hqmq_encode_med3(x, 3.0, HQMQ_GRAN_CHUNK, cb_call, S, table, words, radius, rmed,
+                     thr, out_idx, out_val, slab_off, cap, ws, tile_off=tile_off)
+    # optional 2b bits per chunk: hqmq_quantize_radius(radius, thr, x.shape, S, rwords)
+    # decode step, every (layer, role) at once, against the prefill's thr:
+    hqmq_append_batch(x_new, thr_all, HQMQ_GRAN_CHUNK, cb_all, S, words_new, radius_new,
+                      oi_new, ov_new, so_new, cap_new, tile_off=to_new)
+    # attention of the new queries straight from the codes:
+    k = kv_codes(words_k, radius_k, cb_k, out_idx_k, out_val_k, tile_off_k, cap, 0)
+    v = kv_codes(words_v, radius_v, cb_v, out_idx_v, out_val_v, tile_off_v, cap, 0)
+    hqmq_attention_decode(q, k, v, S, H, T, o, alloc_attention_ws(B, H), seq_len=lens)
+    # or the dense cache: hqmq_decode(words, radius, cb_call, S, out_idx, out_val,
+    #                                  slab_off, cap, 0, y, tile_off=tile_off)
 """
 from __future__ import annotations
 
