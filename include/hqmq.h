@@ -415,8 +415,8 @@ HQMQ_API uint64_t hqmq_attention_workspace_size(int B, int Hk);
  * weights enter P V as two bf16 terms (about 16 significant bits) with fp32
  * accumulation; the token range of a KV head is split over CTAs whose
  * partial (max, sum, P V) are merged by the last of them.  An index >= 24 S
- * reads as the zero codeword (r * 0); unlike hqmq_decode, this call does not
- * flag it.
+ * reads as the zero codeword (r * 0); unlike hqmq_decode, this call records
+ * nothing in d_status (which may be NULL).
  * d_q: bf16 [B][Hq][128], 8-byte aligned.  d_o: [B][Hq][128] of out_dtype
  * (HQMQ_BF16 or HQMQ_F32), 4-byte aligned.  d_seq_len: int32 [B] or NULL.
  * D must be 128 and G <= 8; S in [1, 65535]; scale finite.  d_ws: at least

@@ -96,7 +96,7 @@ struct AttnArgs {
     int out_dtype;
     float *part;                // [B*Hk][cph][ATT_G][ATT_PART] when cph > 1
     uint32_t *done;             // [B*Hk] arrival counters, zero on entry
-    DevStatus *st;
+    DevStatus *st;              // (nothing is recorded)
 };
 
 constexpr int ATT_G = 8;                      // query rows per KV head (GQA group) handled
