@@ -19,7 +19,14 @@
  *     Uitbijterextractie"; gist.science/pt, Resumo Tecnico, section 3);
  *   - decode rebuilds r * (q_p q_s) and restores the outliers (the fused
  *     decoder of gist.science/nl, Technische Samenvatting, "Memory en
- *     Latentie", reads the same stored pair).
+ *     Latentie", reads the same stored pair);
+ *   - decode-phase attention straight from the codes (that same section:
+ *     the decoder runs inside attention), hqmq_attention_decode;
+ *   - an optional b-bit radius code matching the pages' bit budget
+ *     (hqmq_quantize_radius, hqmq_decode_qradius);
+ *   - Med3x under a given threshold for decode-step tokens, and all of a
+ *     step's small calls in one launch (hqmq_outlier_extract_given_thr,
+ *     hqmq_append_batch).
  *
  * Conventions fixed by this library where the pages are silent:
  *   - one call = one (layer, role) tensor x[B][H][T][D], row-major, D % 4 == 0
