@@ -44,6 +44,39 @@ MUTATIONS = [
     ("decode_drops_radius", "for (int i = 0; i < 4; ++i) acc[4 * j + i] = r * c[i];",
      "for (int i = 0; i < 4; ++i) acc[4 * j + i] = c[i];",
      ["test_decode_is_radius_times_codeword"]),
+    # the near-tie arbiter (score of a given codeword, best / second) and the
+    # sampled encode used by the full-size parity checks
+    ("score_wrong_head", "out[q] = oracle_score(c, codebook + (size_t)h * S * 4, S, idx[q]);",
+     "out[q] = oracle_score(c, codebook, S, idx[q]);",
+     ["test_score_chunks_matches_independent_fp64_scores"]),
+    ("score_secondary_zero", "oracle_codeword_f32((int)(idx % 24u), qs_head + (size_t)(idx / 24u) * 4, c);",
+     "oracle_codeword_f32((int)(idx % 24u), qs_head, c);",
+     ["test_score_chunks_matches_independent_fp64_scores"]),
+    ("score_returns_best", "    return dot4_f32(u, c);\n}",
+     "    float bb = -INFINITY;\n"
+     "    for (uint32_t i2 = 0; i2 < 24u * S; ++i2) {\n"
+     "        float c2[4];\n"
+     "        oracle_codeword_f32((int)(i2 % 24u), qs_head + (size_t)(i2 / 24u) * 4, c2);\n"
+     "        float v2 = dot4_f32(u, c2);\n"
+     "        if (v2 > bb) bb = v2;\n"
+     "    }\n"
+     "    (void)c;\n"
+     "    return bb;\n}",
+     ["test_score_chunks_matches_independent_fp64_scores"]),
+    ("score_skips_zeroing", "load_chunk(x, dtype, j, thr ? thr + h : NULL, gran, c);\n        out[q]",
+     "load_chunk(x, dtype, j, NULL, gran, c);\n        out[q]",
+     ["test_score_chunks_matches_independent_fp64_scores"]),
+    ("second_not_tracked", "else if (sc > second) second = sc;", ";",
+     ["test_best_and_second_are_the_top_two_scores"]),
+    ("chunks_head0", "if (h != cur_h) { build_table(codebook + (size_t)h * S * 4, S, table); cur_h = h; }",
+     "if (h != cur_h) { build_table(codebook, S, table); cur_h = h; }",
+     ["test_encode_chunks_equals_the_whole_call_encode"]),
+    ("chunks_skip_zeroing",
+     "load_chunk(x, dtype, j, thr ? thr + h : NULL, gran, c);\n        float r, bs, sc;\n"
+     "        uint32_t idx = search_chunk(c, table, S",
+     "load_chunk(x, dtype, j, NULL, gran, c);\n        float r, bs, sc;\n"
+     "        uint32_t idx = search_chunk(c, table, S",
+     ["test_encode_chunks_equals_the_whole_call_encode"]),
     ("qradius_rounds_down", "float t = q + 0.5f;", "float t = q;",
      ["test_level_is_the_nearest_grid_point"], "tests/test_oracle_qradius.py"),
     ("qradius_levels_pow2", "uint32_t b = oracle_index_bits(S), L = 24u * S;\n    float *acc",

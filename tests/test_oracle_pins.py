@@ -515,3 +515,142 @@ def test_pages_figures():
     assert round(gb) == fig["cache_70b_128k_gb"]["value"]
     assert fig["med3_C"]["value"] == 3
     assert fig["min_angle_deg"]["value"] == 60
+
+
+# ---------------------------------------------------------------- the near-tie arbiter
+# Every GPU index that differs from the oracle's is excused or failed by the
+# oracle's own scores (score_chunks: the fp32 score of a given codeword; best /
+# second of encode and encode_chunks).  These pins tie those functions to an
+# independent fp64 model: codewords built from complex 2x2 matrices in the
+# enumeration order the pages' set is given in (8 axis units p = 2a + sign,
+# then the 16 half units p = 8 + m), scored against x / |x| in fp64.
+def _units_enumerated():
+    out = []
+    for p in range(24):
+        if p < 8:
+            v = np.zeros(4)
+            v[p // 2] = -1.0 if p % 2 else 1.0
+        else:
+            v = np.array([-0.5 if ((p - 8) >> c) & 1 else 0.5 for c in range(4)])
+        out.append(v)
+    return np.array(out)
+
+
+def _fp64_scores(chunk, cb_head):
+    """fp64 <x/|x|, q_p q_s> for every global index s*24 + p."""
+    units = _units_enumerated()
+    W = np.array([qmul_ref(units[p], cb_head[s].astype(np.float64))
+                  for s in range(cb_head.shape[0]) for p in range(24)])
+    x = chunk.astype(np.float64)
+    n = np.linalg.norm(x)
+    return W @ (x / n) if n > 0 else np.zeros(W.shape[0])
+
+
+def _zeroed(chunk, thr_h, gran):
+    """The chunk as the search sees it after Med3x zeroing (pages, section 3):
+    chunk mode zeroes a chunk whose fp32 norm exceeds thr, element mode zeroes
+    each element with |x| > thr."""
+    c = chunk.astype(np.float32).copy()
+    if thr_h is None:
+        return c
+    if gran == 0:
+        r = np.sqrt(np.sum(c.astype(np.float64) ** 2))
+        return np.zeros(4, np.float32) if r > thr_h else c
+    c[np.abs(c) > thr_h] = 0.0
+    return c
+
+
+def _arbiter_case(oracle):
+    # three heads with distinct codebooks, two batches, a few planted large
+    # chunks so that Med3x zeroes something in both granularities
+    rng = np.random.default_rng(21)
+    B, H, T, D, S = 2, 3, 8, 128, 8
+    x = rng.standard_normal((B, H, T, D)).astype(np.float32)
+    xc = x.reshape(-1, 4)
+    big = rng.choice(xc.shape[0], 24, replace=False)
+    xc[big] *= 9.0
+    xc[big[:6], 1] = 40.0                  # one large element in some chunks
+    cb = oracle.make_codebook(4, S, H)
+    return x, cb, S
+
+
+# (fp32 score vs fp64: |u| = |c| = 1 up to rounding; u_i is a rounded quotient
+# of a rounded norm, c_i a sum of 4 exact terms rounded 3 times, the dot product
+# 4 rounded products and 3 rounded sums: well under 24 units of 2^-24)
+SCORE_ABS_TOL = 24 * 2.0 ** -24
+
+
+@pytest.mark.parametrize("gran,use_thr", [(0, False), (0, True), (1, True)])
+def test_score_chunks_matches_independent_fp64_scores(oracle, gran, use_thr):
+    x, cb, S = _arbiter_case(oracle)
+    B, H, T, D = x.shape
+    thr = oracle.med3_threshold(x, 3.0, gran)[1] if use_thr else None
+    rng = np.random.default_rng(22)
+    chunks = np.sort(rng.choice(B * H * T * D // 4, 60, replace=False)).astype(np.int64)
+    per_slab = T * D // 4
+    n_words = 24 * S
+    all_idx = np.tile(np.arange(n_words, dtype=np.uint32), chunks.size)
+    rep = np.repeat(chunks, n_words)
+    sc = oracle.score_chunks(x, cb, S, rep, all_idx, thr=thr, gran=gran).reshape(-1, n_words)
+    xc = x.reshape(-1, 4)
+    for q, j in enumerate(chunks):
+        h = (j // per_slab) % H
+        c = _zeroed(xc[j], None if thr is None else thr[h], gran)
+        ref = _fp64_scores(c, cb[h])
+        if not np.any(c):
+            assert np.all(sc[q] == 0.0)          # a zero chunk has no search
+            continue
+        assert np.abs(sc[q].astype(np.float64) - ref).max() <= SCORE_ABS_TOL, (j, h)
+
+
+@pytest.mark.parametrize("gran,use_thr", [(0, False), (0, True), (1, True)])
+def test_best_and_second_are_the_top_two_scores(oracle, gran, use_thr):
+    x, cb, S = _arbiter_case(oracle)
+    B, H, T, D = x.shape
+    thr = oracle.med3_threshold(x, 3.0, gran)[1] if use_thr else None
+    words, radius, best, second, _ = oracle.encode(x, cb, S, thr=thr, gran=gran)
+    n = B * H * T * D // 4
+    idx = oracle.get_index(words, S, np.arange(n))
+    per_slab = T * D // 4
+    n_words = 24 * S
+    xc = x.reshape(-1, 4)
+    chunks = np.arange(0, n, 7, dtype=np.int64)
+    sc = oracle.score_chunks(x, cb, S, np.repeat(chunks, n_words),
+                             np.tile(np.arange(n_words, dtype=np.uint32), chunks.size),
+                             thr=thr, gran=gran).reshape(-1, n_words)
+    at_pick = oracle.score_chunks(x, cb, S, chunks, idx[chunks], thr=thr, gran=gran)
+    for q, j in enumerate(chunks):
+        h = (j // per_slab) % H
+        c = _zeroed(xc[j], None if thr is None else thr[h], gran)
+        if not np.any(c):
+            assert idx[j] == 0 and best[j] == 0.0 and second[j] == 0.0
+            continue
+        # the score of the oracle's own pick is its best, bit for bit
+        assert at_pick[q].view(np.uint32) == best[j].view(np.uint32)
+        # best and second are the two largest of the 24 S scores (second may
+        # equal best on an exact tie), and the pick is the lowest index of best
+        srt = np.sort(sc[q])[::-1]
+        assert best[j] == srt[0] and second[j] == srt[1], j
+        assert idx[j] == int(np.nonzero(sc[q] == srt[0])[0][0])
+        # and against the independent fp64 scores
+        ref = np.sort(_fp64_scores(c, cb[h]))[::-1]
+        assert abs(float(best[j]) - ref[0]) <= SCORE_ABS_TOL
+        assert abs(float(second[j]) - ref[1]) <= SCORE_ABS_TOL
+
+
+@pytest.mark.parametrize("gran,use_thr", [(0, False), (0, True), (1, True)])
+def test_encode_chunks_equals_the_whole_call_encode(oracle, gran, use_thr):
+    # the sampled form used at full size must give what the whole-call encode
+    # gives on the same chunks (head selection, zeroing, radius, scores)
+    x, cb, S = _arbiter_case(oracle)
+    B, H, T, D = x.shape
+    thr = oracle.med3_threshold(x, 3.0, gran)[1] if use_thr else None
+    words, radius, best, second, _ = oracle.encode(x, cb, S, thr=thr, gran=gran)
+    n = B * H * T * D // 4
+    rng = np.random.default_rng(23)
+    chunks = rng.permutation(n)[:300].astype(np.int64)      # any order, all heads
+    i2, r2, b2, s2 = oracle.encode_chunks(x, cb, S, chunks, thr=thr, gran=gran)
+    assert np.array_equal(i2, oracle.get_index(words, S, chunks))
+    assert np.array_equal(r2, radius[chunks])
+    assert np.array_equal(b2.view(np.uint32), best[chunks].view(np.uint32))
+    assert np.array_equal(s2.view(np.uint32), second[chunks].view(np.uint32))
