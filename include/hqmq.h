@@ -290,10 +290,16 @@ HQMQ_API int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, i
  * median, two for the list), whose scratch is 8 KB per head plus 8 bytes per
  * 4096 chunks, in one file-scope device array of HQMQ_NOALLOC_SCRATCH_BYTES
  * (1 MiB) that every GPU which loads libhqmq holds until the process exits.
- * Shapes that need more are rejected with HQMQ_ERR_WORKSPACE (a
- * 1 x 8 x 131072 x 128 call needs about 130 KB).  The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress, with that device current) and caches it;
- * make that first call before any stream capture.  All calls on a device
+ * Shapes that need more are rejected with HQMQ_ERR_WORKSPACE.  The need is
+ * 8192 H + ceil256(8 H) + 2 ceil256(4 B H ceil(T D / 16384)) bytes
+ * (ceil256: rounded up to a multiple of 256), so at most 127 heads per call
+ * fit, and a 1 x 8 x 131072 x 128 call needs about 130 KB.  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it for the life of the process;
+ * make that first call before any stream capture.  The cached address
+ * belongs to the device's primary context: after cudaDeviceReset, or with
+ * another driver context current, it is stale, so neither is supported once
+ * this entry point has been called.  All calls on a device
  * share the one array: calls whose execution overlaps on the GPU (different
  * streams without ordering between them) race and give wrong results.  Each
  * call clears what must start at zero.  Nothing is allocated or freed.

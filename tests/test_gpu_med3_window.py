@@ -232,3 +232,56 @@ def test_fused_status_counts_after_a_window_miss(oracle):
     want = expected_status(oracle, x, cb, 8, 0, g["cap"])
     for k in ("n_outliers", "n_saturated", "n_nonfinite"):
         assert g["status"][k] == want[k], (k, g["status"], want)
+
+
+# ------------------------------------------------------------------ full sizes
+# The fused call the bench times (chunk mode, search tables, tile offsets), at
+# the full call shape of each Med3x workload, against the oracle directly:
+# r_med and thr, the whole ordered list, slab and tile offsets and the status
+# bit-exact; indices and radii on a sample that includes every listed
+# chunk's neighbourhood of the threshold.
+FULL_SIZE_FUSED = [("llama3_70b_128k", 40, 1), ("mha7b_s8", 5, 1), ("mha7b_s32", 3, 0),
+                   ("qwen_outlier", 27, 1)]
+
+
+def threshold_band_chunks(x_np, thr, H, T, D, k, rng):
+    """Up to k chunks whose norm lies within 5% of their head's threshold
+    (the chunks whose outlier decision is the closest), chosen at random."""
+    xc = x_np.reshape(-1, 4)
+    if x_np.dtype == np.uint16:
+        xc = (xc.astype(np.uint32) << 16).view(np.float32)
+    r = np.sqrt(np.sum(xc.astype(np.float64) ** 2, axis=1))
+    head = (np.arange(r.size) // (T * D // 4)) % H
+    t = thr.astype(np.float64)[head]
+    band = np.nonzero(np.abs(r - t) <= 0.05 * t)[0]
+    return rng.choice(band, min(k, band.size), replace=False) if band.size else band
+
+
+@pytest.mark.parametrize("name,layer,role", FULL_SIZE_FUSED,
+                         ids=["%s-L%d-r%d" % f for f in FULL_SIZE_FUSED])
+def test_fused_full_size_against_the_oracle(oracle, name, layer, role):
+    w = W.WORKLOADS[name]
+    B, H, T, D = w.call_shape
+    n_chunks = B * H * T * D // 4
+    x = W.as_numpy_bits(W.make_call_input(w, layer, role, device="cuda"))
+    cb = oracle.make_codebook(w.codebook_seed, w.S, H, W.group0(layer, role, H))
+    g = fused(x, cb, w.S, 0, True, cap=n_chunks // 5)
+    thr_o, idx_o, val_o, so_o, n_o = check_med3(oracle, x, g, w.C, 0)
+    # status: the list's count and saturations (bulk chunks have r <= thr, far
+    # below the fp16 limit, and the inputs are finite), no fallback
+    _, _, _, _, st_x = oracle.extract(x, thr_o, gran=0, cap=g["cap"])
+    assert g["status"] == {"flags": st_x["flags"], "n_outliers": n_o,
+                           "n_saturated": st_x["n_saturated"], "n_nonfinite": 0}, g["status"]
+    rng = np.random.default_rng(layer * 2 + role + 17)
+    chunks = np.concatenate([rng.choice(n_chunks, 12000, replace=False),
+                             threshold_band_chunks(x, thr_o, H, T, D, 3000, rng),
+                             idx_o[rng.choice(idx_o.size, min(1000, idx_o.size), replace=False)],
+                             np.array([0, n_chunks - 1])]).astype(np.int64)
+    chunks = np.unique(chunks)
+    gi = unpack_indices(to_host(g["words"]), w.S, n_chunks)
+    n, mm, near = check_codes(oracle, x, cb, w.S, gi, to_host(g["radius"]), thr=thr_o, gran=0,
+                              chunks=chunks)
+    assert n >= 10000
+    print("[fused full size] %s L%d role %d: %d outliers (%.3f%%), %d sampled chunks, "
+          "%d near-tie index differences, %d near-tie pairs"
+          % (name, layer, role, n_o, 100.0 * n_o / n_chunks, n, mm, near))
