@@ -41,6 +41,11 @@ extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, i
                                        uint32_t *slab_off, uint32_t *tile_off_out, uint64_t cap,
                                        void *ws, hqmq_status *st, cudaStream_t stream,
                                        const uint32_t **tile_off, uint32_t *tiles_per_slab);
+extern "C" int hqmq_spec_encode_supported(uint32_t b);
+extern "C" int hqmq_launch_spec_encode_units(const void *x, int dtype, int B, int H, int T, int D,
+                                             const float *cb, uint32_t S, uint32_t b,
+                                             const void *table, uint32_t *words, uint16_t *radius,
+                                             void *ws, int sm_count, cudaStream_t stream);
 extern "C" int hqmq_launch_spec_encode(const void *x, int dtype, int B, int H, int T, int D,
                                        const float *cb, uint32_t S, uint32_t b, const void *table,
                                        uint32_t *words, uint16_t *radius, void *ws, int sm_count,
@@ -265,8 +270,11 @@ int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, flo
         // be outliers
         int rc = hqmq_launch_med3_front(d_x, dtype, B, H, T, D, C, gran, d_ws, 0, sm, s);
         if (rc == HQMQ_OK)
-            rc = hqmq_launch_spec_encode(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table,
-                                         d_idx_words, d_radius, d_ws, sm, s);
+            rc = hqmq_spec_encode_supported(b)
+                     ? hqmq_launch_spec_encode_units(d_x, dtype, B, H, T, D, d_codebook, S, b,
+                                                     d_table, d_idx_words, d_radius, d_ws, sm, s)
+                     : hqmq_launch_spec_encode(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table,
+                                               d_idx_words, d_radius, d_ws, sm, s);
         if (rc == HQMQ_OK)
             rc = hqmq_launch_med3_finish(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr,
                                          d_slab_off, d_tile_off, cap, d_ws, d_status, s,

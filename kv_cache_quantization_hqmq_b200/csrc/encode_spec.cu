@@ -1,0 +1,321 @@
+// encode_spec.cu -- the one-read Med3x encode pass (chunk mode, search tables).
+//
+// Med3x needs the exact median of a head's chunk norms before any chunk can
+// be called an outlier (gist.science/nl, Technische Samenvatting, section 3),
+// but the encode of a chunk does not depend on the median unless the chunk
+// is an outlier.  This pass therefore reads x once and, per chunk:
+//  * does the window bookkeeping of the median (keys below the sampled rank
+//    window counted per head, keys inside it staged for the exact selection,
+//    per 1024-chunk tile the count of chunks above every possible threshold
+//    t_hi, and (tile, key) pairs of chunks inside the threshold's band
+//    (t_lo, t_hi]);
+//  * records per packing group which chunks lie above t_lo (the only ones
+//    that can be outliers), for the fix-up pass after the exact threshold;
+//  * encodes speculatively: a chunk above t_hi as an outlier (index 0,
+//    radius 0), every other chunk as a bulk chunk: fp16 radius and the index
+//    of the nearest of the 24 S codewords q_p q_s (section 1), found through
+//    the per-face search table (search.cuh).
+//
+// Data flow (B200): one CTA of 32 warps per SM, each CTA a contiguous range
+// of work units (8 packing groups, 256 chunks) walked head by head; inside a
+// head's range every warp takes a contiguous share of the units.  Each warp
+// streams its chunks through a private cp.async ring in shared memory
+// (7 groups = 1.75 KB ahead per warp, ~56 KB in flight per SM), so that HBM
+// latency is hidden without registers; the head's codeword table sits in
+// shared memory in R copies (lane l reads copy l mod R: the 8 lanes of a
+// 16-byte phase hit distinct bank groups for R = 8).  Indices of a unit are
+// staged in shared memory and packed into the unit's b-bit words with
+// coalesced stores.
+//
+// The outputs equal those of k_encode_lut's speculative mode (search.cu) bit
+// for bit; the per-tile counts are added atomically because a tile's four
+// units may belong to different warps.
+#include "search.cuh"
+
+namespace hqmq {
+
+constexpr int SPEC_THREADS = 1024;
+constexpr int SPEC_WARPS = SPEC_THREADS / 32;
+constexpr int UNIT_G = 8;                          // packing groups per work unit
+constexpr int RING_BYTES = 2048;                   // input ring per warp
+constexpr int SPEC_STAGE = 128;                    // window keys staged per warp
+constexpr int WARP_SMEM = RING_BYTES + SPEC_STAGE * 4 + UNIT_G * 32 * 2 + UNIT_G * 4;
+static_assert(WARP_SMEM % 16 == 0, "per-warp shared regions stay 16-byte aligned");
+static_assert(TILE_GROUPS % UNIT_G == 0, "a unit lies inside one list tile");
+constexpr size_t SPEC_SMEM_MAX = 227 * 1024;
+
+template <int CB>
+__device__ __forceinline__ void cp_async_chunk(uint32_t dst, const void *src) {
+    if constexpr (CB == 8)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(src) : "memory");
+    else
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// <x, c> in fp32 (the order of the table encode)
+__device__ __forceinline__ float score4(float x0, float x1, float x2, float x3, float4 c) {
+    return __fmaf_rn(x3, c.w, __fmaf_rn(x2, c.z, __fmaf_rn(x1, c.y, __fmul_rn(x0, c.x))));
+}
+
+template <int DT, int BB, int R>
+__global__ void __launch_bounds__(SPEC_THREADS, 1)
+k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uint32_t tps,
+              uint32_t n_units, const float4 *__restrict__ cb_all, uint32_t S,
+              const uint4 *__restrict__ tables, uint32_t *__restrict__ words,
+              uint16_t *__restrict__ radius, SpecArgs sa) {
+    constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;       // bytes per chunk
+    constexpr int NS = RING_BYTES / (32 * CB);         // ring slots (packing groups)
+    static_assert(NS >= 2, "ring");
+    extern __shared__ __align__(16) unsigned char s_raw[];
+    float4 *s_tab = reinterpret_cast<float4 *>(s_raw); // [24 S + 1][R]
+    const uint32_t n_words = 24u * S;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    const uint32_t lr = (uint32_t)(lane & (R - 1));
+    unsigned char *wsm = s_raw + (size_t)(n_words + 1) * R * sizeof(float4) +
+                         (size_t)warp * WARP_SMEM;
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(wsm) + (uint32_t)lane * CB;
+    const unsigned char *ring_p = wsm + lane * CB;     // this lane's chunk in slot 0
+    uint32_t *stage = reinterpret_cast<uint32_t *>(wsm + RING_BYTES);
+    uint16_t *s_idx = reinterpret_cast<uint16_t *>(wsm + RING_BYTES + SPEC_STAGE * 4);
+    uint32_t *s_cb = reinterpret_cast<uint32_t *>(wsm + RING_BYTES + SPEC_STAGE * 4 + UNIT_G * 64);
+    const unsigned char *xl = reinterpret_cast<const unsigned char *>(x) + (size_t)lane * CB;
+
+    const uint32_t u_begin = (uint32_t)((uint64_t)n_units * blockIdx.x / gridDim.x);
+    const uint32_t u_end = (uint32_t)((uint64_t)n_units * (blockIdx.x + 1) / gridDim.x);
+    int cur_h = -1;
+    for (uint32_t seg = u_begin; seg < u_end;) {
+        const uint32_t slab = seg / ups;
+        const uint32_t seg_end = min(u_end, (slab + 1) * ups);
+        const int h = (int)(slab % (uint32_t)H);
+        if (h != cur_h) {                                // (block-uniform)
+            __syncthreads();
+            const float4 *cbh = cb_all + (size_t)h * S;
+            for (uint32_t i = threadIdx.x; i < (n_words + 1) * R; i += SPEC_THREADS) {
+                const uint32_t id = i / R;
+                s_tab[i] = id < n_words ? codeword((int)(id % 24u), __ldg(cbh + id / 24u))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            __syncthreads();
+            cur_h = h;
+        }
+        // this warp's share of the head's units: [ua, ub)
+        const uint32_t nseg = seg_end - seg;
+        const uint32_t ua = seg + (uint32_t)((uint64_t)nseg * warp / SPEC_WARPS);
+        const uint32_t ub = seg + (uint32_t)((uint64_t)nseg * (warp + 1) / SPEC_WARPS);
+        seg = seg_end;
+        if (ua >= ub) continue;                          // (warp-uniform)
+        const WinState w = sa.win[h];
+        const uint32_t span = w.hi_key - w.lo_key;
+        const uint4 *tb = tables + (size_t)h * LUT_ENTRIES;
+        const float4 *cb = cb_all + (size_t)h * S;
+        const uint32_t u_slab = slab * ups;              // the slab's first unit
+        const uint64_t g_slab = (uint64_t)slab * gps;    // the slab's first packing group
+        const uint64_t Gb = g_slab + (uint64_t)(ua - u_slab) * UNIT_G;
+        const uint64_t Ge = g_slab + min((uint64_t)(ub - u_slab) * UNIT_G, (uint64_t)gps);
+        // ring prologue: groups Gb .. Gb + NS - 2, one commit group each
+#pragma unroll
+        for (int i = 0; i < NS - 1; ++i) {
+            const uint64_t G = Gb + (uint64_t)i;
+            if (G < Ge) cp_async_chunk<CB>(ring_s + (uint32_t)(G % NS) * 32u * CB, xl + G * 32u * CB);
+            cp_async_commit();
+        }
+        uint32_t n_stage = 0, n_below = 0;
+        unsigned n_nf = 0, n_sat = 0;
+        for (uint32_t u = ua; u < ub; ++u) {
+            const uint32_t g0 = (u - u_slab) * UNIT_G;
+            const uint32_t ng = min((uint32_t)UNIT_G, gps - g0);
+            const uint64_t Gu = g_slab + g0;
+            const uint32_t tile = slab * tps + g0 / TILE_GROUPS;
+            uint32_t n_def = 0;
+            for (uint32_t k = 0; k < ng; ++k) {
+                const uint64_t G = Gu + k;
+                const uint32_t j = (uint32_t)(G * 32u) + (uint32_t)lane;   // chunk index
+                // group G's copy was the (NS-1)-th latest commit: wait for it
+                cp_async_wait<NS - 2>();
+                RawChunk<DT> cur;
+                cur.v = *reinterpret_cast<const decltype(cur.v) *>(
+                    ring_p + (uint32_t)(G % NS) * 32u * CB);
+                {   // refill the slot read in the previous step (this lane's bytes only)
+                    const uint64_t Gn = G + (NS - 1);
+                    if (Gn < Ge)
+                        cp_async_chunk<CB>(ring_s + (uint32_t)(Gn % NS) * 32u * CB,
+                                           xl + Gn * 32u * CB);
+                    cp_async_commit();
+                }
+                const float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
+                float r = chunk_norm(x0, x1, x2, x3);
+                // median window: key = r's bits (r >= 0; a NaN's bits exceed
+                // every finite key and +inf's, as in the median's order)
+                const uint32_t key = __float_as_uint(r);
+                n_below += key < w.lo_key ? 1u : 0u;
+                const bool in = key - w.lo_key < span;   // lo_key <= key < hi_key
+                const uint32_t mi = __ballot_sync(FULL, in);
+                if (mi) {
+                    if (n_stage + 32 > SPEC_STAGE) {
+                        flush_stage(stage, n_stage, lane, sa.cand_n + h,
+                                    sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap);
+                        n_stage = 0;
+                    }
+                    if (in) stage[n_stage + __popc(mi & lt)] = key;
+                    n_stage += __popc(mi);
+                    __syncwarp();
+                }
+                // threshold band: above t_hi always an outlier, above t_lo possibly
+                const bool dfn = r > w.t_hi;             // (NaN: false)
+                const bool cnd = r > w.t_lo;
+                n_def += dfn ? 1u : 0u;
+                const uint32_t mc = __ballot_sync(FULL, cnd);
+                if (lane == 0) s_cb[k] = mc;
+                const uint32_t mu = __ballot_sync(FULL, cnd && !dfn);
+                if (mu) {
+                    unsigned long long base = 0;
+                    if (lane == 0) base = atomicAdd(sa.amb_n, (unsigned long long)__popc(mu));
+                    base = __shfl_sync(FULL, base, 0);
+                    if ((mu >> lane) & 1u) {
+                        const unsigned long long pos = base + __popc(mu & lt);
+                        if (pos < sa.amb_cap) sa.amb[pos] = make_uint2(tile, key);
+                    }
+                }
+                if (dfn) r = 0.0f;                       // certain outlier: radius 0, index 0
+                const bool finite = r == r && r != __int_as_float(0x7F800000);
+                const bool search = finite && r > 0.0f;
+                // lanes without a search read the default record (one candidate)
+                uint4 rec = make_uint4(1u << 12, 0u, 0u, 0u);
+                if (search) {
+                    const float a0 = fabsf(x0), a1 = fabsf(x1), a2 = fabsf(x2), a3 = fabsf(x3);
+                    const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+                    const bool e0 = a0 == m, e01 = e0 || a1 == m, e012 = e01 || a2 == m;
+                    const int a = e0 ? 0 : e01 ? 1 : e012 ? 2 : 3;
+                    const float xa = e0 ? x0 : e01 ? x1 : e012 ? x2 : x3;
+                    const float c1 = e0 ? x1 : x0;
+                    const float c2 = e01 ? x2 : x1;
+                    const float c3 = e012 ? x3 : x2;
+                    float inv;
+                    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(m));   // cells are widened
+                    const int cell = (cell_coord(c1 * inv) * LUT_G + cell_coord(c2 * inv)) * LUT_G +
+                                     cell_coord(c3 * inv);
+                    const int face = 2 * a + (xa < 0.0f ? 1 : 0);
+                    rec = __ldg(tb + face * LUT_CELLS + cell);
+                }
+                const uint32_t cnt = (rec.x >> 12) & 0xFu;          // 0: overflowing cell
+                const uint32_t kmax = __reduce_max_sync(FULL, cnt);
+                // slots hold increasing ids; a strictly higher score replaces
+                // the best, so equal scores keep the lowest index
+                uint32_t bid = rec.x & LUT_ID_MASK;
+                float best = score4(x0, x1, x2, x3, s_tab[bid * R + lr]);
+#pragma unroll
+                for (int q = 1; q < LUT_SLOTS; ++q) {
+                    if ((uint32_t)q >= kmax) break;                 // (warp-uniform)
+                    const uint32_t wd = q < 2 ? rec.x : q < 4 ? rec.y : q < 6 ? rec.z : rec.w;
+                    const uint32_t id = (q & 1) ? (wd >> 16) : (wd & LUT_ID_MASK);
+                    const float sc = score4(x0, x1, x2, x3, s_tab[id * R + lr]);
+                    if (sc > best) { best = sc; bid = id; }
+                }
+                uint32_t idx = 0;
+                if (search) idx = cnt != 0 ? bid : sloop_index(x0, x1, x2, x3, cb, S);
+                uint16_t rh;
+                if (!finite) {
+                    rh = 0x7E00u;
+                    ++n_nf;
+                } else {
+                    int sat = 0;
+                    rh = radius_to_f16(r, sat);
+                    if (!cnd) n_sat += sat;              // (the fix-up pass decides the others)
+                }
+                radius[j] = rh;
+                s_idx[k * 32 + lane] = (uint16_t)idx;
+            }
+            __syncwarp();
+            pack_tile<BB>(s_idx, ng, lane, words + Gu * BB);
+            if ((uint32_t)lane < ng) sa.cbits[Gu + lane] = s_cb[lane];
+            n_def = __reduce_add_sync(FULL, n_def);
+            if (lane == 0 && n_def) atomicAdd(sa.tile_cnt + tile, n_def);
+            __syncwarp();                                // (s_idx, s_cb are refilled next unit)
+        }
+        n_below = __reduce_add_sync(FULL, n_below);
+        if (lane == 0 && n_below) atomicAdd(sa.below + h, (unsigned long long)n_below);
+        if (n_stage)
+            flush_stage(stage, n_stage, lane, sa.cand_n + h, sa.cand + (uint64_t)h * sa.cand_cap,
+                        sa.cand_cap);
+        const unsigned nf = __reduce_add_sync(FULL, n_nf);
+        const unsigned ns = __reduce_add_sync(FULL, n_sat);
+        if (lane == 0 && (nf | ns)) {
+            atomicAdd(sa.head_stat + 2 * h, (unsigned long long)nf);
+            atomicAdd(sa.head_stat + 2 * h + 1, (unsigned long long)ns);
+        }
+    }
+}
+
+template <int DT, int BB, int R>
+static int launch_spec(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
+                       const void *table, uint32_t *words, uint16_t *radius, const SpecArgs &sa,
+                       int sm_count, cudaStream_t stream) {
+    const uint32_t gps = (uint32_t)(((uint64_t)T * D / 4) / 32);
+    const uint32_t ups = (gps + UNIT_G - 1) / UNIT_G;
+    const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
+    const uint64_t n_units = (uint64_t)B * H * ups;
+    const size_t smem = ((size_t)24 * S + 1) * R * sizeof(float4) + (size_t)SPEC_WARPS * WARP_SMEM;
+    if (smem > SPEC_SMEM_MAX) return HQMQ_ERR_ARG;
+    auto kern = k_encode_spec<DT, BB, R>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return HQMQ_ERR_CUDA;
+    uint64_t ctas = (uint64_t)sm_count;                  // one CTA per SM
+    if (ctas > n_units) ctas = n_units;
+    if (ctas < 1) ctas = 1;
+    kern<<<(unsigned)ctas, SPEC_THREADS, smem, stream>>>(
+        x, H, gps, ups, tps, (uint32_t)n_units, reinterpret_cast<const float4 *>(cb), S,
+        reinterpret_cast<const uint4 *>(table), words, radius, sa);
+    return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
+}
+
+template <int DT, int BB>
+static int launch_spec_r(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
+                         const void *table, uint32_t *words, uint16_t *radius, const SpecArgs &sa,
+                         int sm_count, cudaStream_t stream) {
+    // 8 table copies when they fit next to the warps' regions, else 4
+    const size_t smem8 = ((size_t)24 * S + 1) * 8 * sizeof(float4) + (size_t)SPEC_WARPS * WARP_SMEM;
+    if (smem8 <= SPEC_SMEM_MAX)
+        return launch_spec<DT, BB, 8>(B, H, T, D, x, cb, S, table, words, radius, sa, sm_count,
+                                      stream);
+    return launch_spec<DT, BB, 4>(B, H, T, D, x, cb, S, table, words, radius, sa, sm_count, stream);
+}
+
+}  // namespace hqmq
+
+// True when the one-read speculative pass has a kernel here for this index
+// width (b = 8: S = 8..10; b = 10: S = 22..42).
+extern "C" int hqmq_spec_encode_supported(uint32_t b) { return b == 8 || b == 10; }
+
+extern "C" int hqmq_launch_spec_encode_units(const void *x, int dtype, int B, int H, int T, int D,
+                                             const float *cb, uint32_t S, uint32_t b,
+                                             const void *table, uint32_t *words, uint16_t *radius,
+                                             void *ws, int sm_count, cudaStream_t stream) {
+    using namespace hqmq;
+    const SpecArgs sa = spec_args(reinterpret_cast<char *>(ws),
+                                  fused_layout(B, H, T, D, HQMQ_GRAN_CHUNK));
+    if (dtype == HQMQ_BF16) {
+        if (b == 8)
+            return launch_spec_r<HQMQ_BF16, 8>(B, H, T, D, x, cb, S, table, words, radius, sa,
+                                               sm_count, stream);
+        if (b == 10)
+            return launch_spec_r<HQMQ_BF16, 10>(B, H, T, D, x, cb, S, table, words, radius, sa,
+                                                sm_count, stream);
+    } else {
+        if (b == 8)
+            return launch_spec_r<HQMQ_F32, 8>(B, H, T, D, x, cb, S, table, words, radius, sa,
+                                              sm_count, stream);
+        if (b == 10)
+            return launch_spec_r<HQMQ_F32, 10>(B, H, T, D, x, cb, S, table, words, radius, sa,
+                                               sm_count, stream);
+    }
+    return HQMQ_ERR_ARG;
+}

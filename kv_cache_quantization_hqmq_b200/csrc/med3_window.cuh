@@ -69,13 +69,13 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     L.counters = off;    off = align256_(off + sizeof(Counters) + (uint64_t)H * 8);
     L.med_hist = off;    off = align256_(off + (uint64_t)H * MED_BINS * 4);
     L.head_stat = off;   off = align256_(off + (uint64_t)H * 16);   // per head: non-finite, saturated
+    L.tile_cnt = off;    off = align256_(off + L.n_tiles * 4);      // (a tile may be counted by several warps)
     L.zero_bytes = off;
     L.win = off;         off = align256_(off + (uint64_t)H * sizeof(WinState));
     L.below = off;       off = align256_(off + (uint64_t)H * 8);
     L.cand_n = off;      off = align256_(off + (uint64_t)H * 8);
     L.cand = off;        off = align256_(off + (uint64_t)H * L.cand_cap * 4);
     L.amb = off;         off = align256_(off + L.amb_cap * 8);
-    L.tile_cnt = off;    off = align256_(off + L.n_tiles * 4);
     L.tile_off = off;    off = align256_(off + (L.n_tiles + 1) * 4);
     L.cbits = off;       off = align256_(off + (uint64_t)B * H * gps * 4);
     L.total = off;
