@@ -43,6 +43,9 @@ constexpr int WARP_SMEM = RING_BYTES + SPEC_STAGE * 4 + UNIT_G * 32 * 2 + UNIT_G
 static_assert(WARP_SMEM % 16 == 0, "per-warp shared regions stay 16-byte aligned");
 static_assert(TILE_GROUPS % UNIT_G == 0, "a unit lies inside one list tile");
 constexpr size_t SPEC_SMEM_MAX = 227 * 1024;
+// Steps of a unit unrolled per loop trip: 2 measured fastest on B200 (4 and 8
+// run slower: the body no longer stays in the instruction cache).
+constexpr int kSpecUnroll = 2;
 
 template <int CB>
 __device__ __forceinline__ void cp_async_chunk(uint32_t dst, const void *src) {
@@ -64,6 +67,34 @@ __device__ __forceinline__ float score4(float x0, float x1, float x2, float x3, 
     return __fmaf_rn(x3, c.w, __fmaf_rn(x2, c.z, __fmaf_rn(x1, c.y, __fmul_rn(x0, c.x))));
 }
 
+// Shared-memory accesses of the hot loop, by 32-bit shared address.
+template <int CB> struct RingWord;
+template <> struct RingWord<8> { using T = uint2; };
+template <> struct RingWord<16> { using T = float4; };
+__device__ __forceinline__ uint2 lds_u2(uint32_t a) {       // (ordered after cp.async waits)
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 lds_f4_ring(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 lds_cw(uint32_t a) {     // codeword table (read-only here)
+    float4 v;
+    asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts_u16(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"((unsigned short)v) : "memory");
+}
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
 template <int DT, int BB, int R>
 __global__ void __launch_bounds__(SPEC_THREADS, 1)
 k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uint32_t tps,
@@ -72,20 +103,23 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
               uint16_t *__restrict__ radius, SpecArgs sa) {
     constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;       // bytes per chunk
     constexpr int NS = RING_BYTES / (32 * CB);         // ring slots (packing groups)
-    static_assert(NS >= 2, "ring");
+    static_assert(NS >= 2 && UNIT_G % NS == 0, "a unit's groups fill whole ring rounds");
     extern __shared__ __align__(16) unsigned char s_raw[];
     float4 *s_tab = reinterpret_cast<float4 *>(s_raw); // [24 S + 1][R]
     const uint32_t n_words = 24u * S;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = (1u << lane) - 1u;
-    const uint32_t lr = (uint32_t)(lane & (R - 1));
     unsigned char *wsm = s_raw + (size_t)(n_words + 1) * R * sizeof(float4) +
                          (size_t)warp * WARP_SMEM;
-    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(wsm) + (uint32_t)lane * CB;
-    const unsigned char *ring_p = wsm + lane * CB;     // this lane's chunk in slot 0
     uint32_t *stage = reinterpret_cast<uint32_t *>(wsm + RING_BYTES);
     uint16_t *s_idx = reinterpret_cast<uint16_t *>(wsm + RING_BYTES + SPEC_STAGE * 4);
     uint32_t *s_cb = reinterpret_cast<uint32_t *>(wsm + RING_BYTES + SPEC_STAGE * 4 + UNIT_G * 64);
+    // 32-bit shared addresses of this lane's ring chunk (slot 0), table copy,
+    // index stage entry (group 0) and the warp's candidate-bit words
+    const uint32_t a_ring = (uint32_t)__cvta_generic_to_shared(wsm) + (uint32_t)lane * CB;
+    const uint32_t a_tab = (uint32_t)__cvta_generic_to_shared(s_tab) + (uint32_t)(lane & (R - 1)) * 16u;
+    const uint32_t a_idx = (uint32_t)__cvta_generic_to_shared(s_idx) + (uint32_t)lane * 2u;
+    const uint32_t a_cb = (uint32_t)__cvta_generic_to_shared(s_cb);
     const unsigned char *xl = reinterpret_cast<const unsigned char *>(x) + (size_t)lane * CB;
 
     const uint32_t u_begin = (uint32_t)((uint64_t)n_units * blockIdx.x / gridDim.x);
@@ -116,40 +150,38 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
         const uint32_t span = w.hi_key - w.lo_key;
         const uint4 *tb = tables + (size_t)h * LUT_ENTRIES;
         const float4 *cb = cb_all + (size_t)h * S;
-        const uint32_t u_slab = slab * ups;              // the slab's first unit
-        const uint64_t g_slab = (uint64_t)slab * gps;    // the slab's first packing group
-        const uint64_t Gb = g_slab + (uint64_t)(ua - u_slab) * UNIT_G;
-        const uint64_t Ge = g_slab + min((uint64_t)(ub - u_slab) * UNIT_G, (uint64_t)gps);
-        // ring prologue: groups Gb .. Gb + NS - 2, one commit group each
+        // packing groups of the call (fewer than 2^27: 32-bit indices)
+        const uint32_t u_slab = slab * ups;
+        const uint32_t g_slab = slab * gps;
+        const uint32_t Gb = g_slab + (ua - u_slab) * UNIT_G;
+        const uint32_t Ge = g_slab + min((ub - u_slab) * UNIT_G, gps);
+        // ring: group Gb + i sits in slot i mod NS (a unit's groups fill whole
+        // rounds of the ring); prologue: groups Gb .. Gb + NS - 2
 #pragma unroll
         for (int i = 0; i < NS - 1; ++i) {
-            const uint64_t G = Gb + (uint64_t)i;
-            if (G < Ge) cp_async_chunk<CB>(ring_s + (uint32_t)(G % NS) * 32u * CB, xl + G * 32u * CB);
+            if (Gb + i < Ge)
+                cp_async_chunk<CB>(a_ring + (uint32_t)i * 32u * CB, xl + (size_t)(Gb + i) * (32u * CB));
             cp_async_commit();
         }
-        uint32_t n_stage = 0, n_below = 0;
-        unsigned n_nf = 0, n_sat = 0;
+        uint32_t n_stage = 0, n_below = 0, n_nf = 0, n_sat = 0;
         for (uint32_t u = ua; u < ub; ++u) {
             const uint32_t g0 = (u - u_slab) * UNIT_G;
             const uint32_t ng = min((uint32_t)UNIT_G, gps - g0);
-            const uint64_t Gu = g_slab + g0;
+            const uint32_t Gu = g_slab + g0;
             const uint32_t tile = slab * tps + g0 / TILE_GROUPS;
-            uint32_t n_def = 0;
-            for (uint32_t k = 0; k < ng; ++k) {
-                const uint64_t G = Gu + k;
-                const uint32_t j = (uint32_t)(G * 32u) + (uint32_t)lane;   // chunk index
+            uint32_t n_def = 0, fbm = 0;
+            auto step = [&](const uint32_t k) {
+                const uint32_t G = Gu + k;
                 // group G's copy was the (NS-1)-th latest commit: wait for it
                 cp_async_wait<NS - 2>();
                 RawChunk<DT> cur;
-                cur.v = *reinterpret_cast<const decltype(cur.v) *>(
-                    ring_p + (uint32_t)(G % NS) * 32u * CB);
-                {   // refill the slot read in the previous step (this lane's bytes only)
-                    const uint64_t Gn = G + (NS - 1);
-                    if (Gn < Ge)
-                        cp_async_chunk<CB>(ring_s + (uint32_t)(Gn % NS) * 32u * CB,
-                                           xl + Gn * 32u * CB);
-                    cp_async_commit();
-                }
+                if constexpr (CB == 8) cur.v = lds_u2(a_ring + (k % NS) * 32u * CB);
+                else cur.v = lds_f4_ring(a_ring + (k % NS) * 32u * CB);
+                // refill the slot read in the previous step (this lane's bytes only)
+                if (G + (NS - 1) < Ge)
+                    cp_async_chunk<CB>(a_ring + ((k + NS - 1) % NS) * 32u * CB,
+                                       xl + (size_t)(G + (NS - 1)) * (32u * CB));
+                cp_async_commit();
                 const float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
                 float r = chunk_norm(x0, x1, x2, x3);
                 // median window: key = r's bits (r >= 0; a NaN's bits exceed
@@ -173,7 +205,7 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
                 const bool cnd = r > w.t_lo;
                 n_def += dfn ? 1u : 0u;
                 const uint32_t mc = __ballot_sync(FULL, cnd);
-                if (lane == 0) s_cb[k] = mc;
+                if (lane == 0) sts_u32(a_cb + k * 4u, mc);
                 const uint32_t mu = __ballot_sync(FULL, cnd && !dfn);
                 if (mu) {
                     unsigned long long base = 0;
@@ -185,56 +217,83 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
                     }
                 }
                 if (dfn) r = 0.0f;                       // certain outlier: radius 0, index 0
-                const bool finite = r == r && r != __int_as_float(0x7F800000);
-                const bool search = finite && r > 0.0f;
-                // lanes without a search read the default record (one candidate)
-                uint4 rec = make_uint4(1u << 12, 0u, 0u, 0u);
-                if (search) {
-                    const float a0 = fabsf(x0), a1 = fabsf(x1), a2 = fabsf(x2), a3 = fabsf(x3);
-                    const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-                    const bool e0 = a0 == m, e01 = e0 || a1 == m, e012 = e01 || a2 == m;
-                    const int a = e0 ? 0 : e01 ? 1 : e012 ? 2 : 3;
-                    const float xa = e0 ? x0 : e01 ? x1 : e012 ? x2 : x3;
-                    const float c1 = e0 ? x1 : x0;
-                    const float c2 = e01 ? x2 : x1;
-                    const float c3 = e012 ? x3 : x2;
-                    float inv;
-                    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(m));   // cells are widened
-                    const int cell = (cell_coord(c1 * inv) * LUT_G + cell_coord(c2 * inv)) * LUT_G +
-                                     cell_coord(c3 * inv);
-                    const int face = 2 * a + (xa < 0.0f ? 1 : 0);
-                    rec = __ldg(tb + face * LUT_CELLS + cell);
-                }
+                // search every lane (branch-free); a lane whose chunk is zero,
+                // non-finite or a certain outlier reads some in-range record and
+                // keeps index 0.  r in (0, FLT_MAX] <=> its bits in [1, 0x7F7FFFFF].
+                const bool srch = __float_as_uint(r) - 1u < 0x7F7FFFFFu;
+                const float a0 = fabsf(x0), a1 = fabsf(x1), a2 = fabsf(x2), a3 = fabsf(x3);
+                const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+                const bool e0 = a0 == m, e01 = e0 || a1 == m, e012 = e01 || a2 == m;
+                const uint32_t a = e0 ? 0u : e01 ? 1u : e012 ? 2u : 3u;
+                const float xa = e0 ? x0 : e01 ? x1 : e012 ? x2 : x3;
+                const float c1 = e0 ? x1 : x0;
+                const float c2 = e01 ? x2 : x1;
+                const float c3 = e012 ? x3 : x2;
+                float inv;
+                asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(m));   // cells are widened
+                const uint32_t cell = (uint32_t)((cell_coord(c1 * inv) * LUT_G + cell_coord(c2 * inv)) *
+                                                     LUT_G + cell_coord(c3 * inv)) & (LUT_CELLS - 1u);
+                const uint32_t face = 2u * a + (xa < 0.0f ? 1u : 0u);
+                const uint4 rec = __ldg(tb + (face * LUT_CELLS + cell));
                 const uint32_t cnt = (rec.x >> 12) & 0xFu;          // 0: overflowing cell
                 const uint32_t kmax = __reduce_max_sync(FULL, cnt);
-                // slots hold increasing ids; a strictly higher score replaces
-                // the best, so equal scores keep the lowest index
-                uint32_t bid = rec.x & LUT_ID_MASK;
-                float best = score4(x0, x1, x2, x3, s_tab[bid * R + lr]);
-#pragma unroll
-                for (int q = 1; q < LUT_SLOTS; ++q) {
-                    if ((uint32_t)q >= kmax) break;                 // (warp-uniform)
-                    const uint32_t wd = q < 2 ? rec.x : q < 4 ? rec.y : q < 6 ? rec.z : rec.w;
-                    const uint32_t id = (q & 1) ? (wd >> 16) : (wd & LUT_ID_MASK);
-                    const float sc = score4(x0, x1, x2, x3, s_tab[id * R + lr]);
-                    if (sc > best) { best = sc; bid = id; }
+                // the slots hold increasing ids (padded with the zero codeword
+                // 24 S); scored from the last to the first, a candidate that
+                // scores at least the best so far replaces it, so among equal
+                // scores the lowest index wins.  Only the warp's longest list
+                // is walked (straight-line code entered at slot kmax - 1).
+                float best = __int_as_float(0xFF800000);
+                uint32_t bid = 0;
+#define HQMQ_CAND(EXPR)                                                              \
+    {                                                                                \
+        const uint32_t id_ = (EXPR);                                                 \
+        const float sc_ = score4(x0, x1, x2, x3, lds_cw(a_tab + id_ * (16u * R)));   \
+        if (sc_ >= best) { best = sc_; bid = id_; }                                  \
+    }
+                switch (kmax) {
+                    default:
+                    case 8: HQMQ_CAND(rec.w >> 16)
+                    case 7: HQMQ_CAND(rec.w & 0xFFFFu)
+                    case 6: HQMQ_CAND(rec.z >> 16)
+                    case 5: HQMQ_CAND(rec.z & 0xFFFFu)
+                    case 4: HQMQ_CAND(rec.y >> 16)
+                    case 3: HQMQ_CAND(rec.y & 0xFFFFu)
+                    case 2: HQMQ_CAND(rec.x >> 16)
+                    case 1:
+                    case 0: HQMQ_CAND(rec.x & LUT_ID_MASK)
                 }
-                uint32_t idx = 0;
-                if (search) idx = cnt != 0 ? bid : sloop_index(x0, x1, x2, x3, cb, S);
-                uint16_t rh;
-                if (!finite) {
-                    rh = 0x7E00u;
-                    ++n_nf;
-                } else {
-                    int sat = 0;
-                    rh = radius_to_f16(r, sat);
-                    if (!cnd) n_sat += sat;              // (the fix-up pass decides the others)
+#undef HQMQ_CAND
+                const uint32_t idx = srch ? bid : 0u;
+                fbm |= (srch && cnt == 0u ? 1u : 0u) << k;   // overflowing cell: S-codeword loop later
+                // fp16 radius: RN-even, saturating at 65504 from 65520 up;
+                // NaN or inf -> 0x7E00 (counted)
+                const bool fin = r <= 3.40282347e38f;
+                const bool sat = fin && r >= 65520.0f;
+                uint16_t rh = __half_as_ushort(__float2half_rn(r));
+                rh = sat ? (uint16_t)0x7BFFu : rh;
+                rh = fin ? rh : (uint16_t)0x7E00u;
+                n_nf += fin ? 0u : 1u;
+                n_sat += (sat && !cnd) ? 1u : 0u;        // (the fix-up pass decides the others)
+                radius[G * 32u + (uint32_t)lane] = rh;
+                sts_u16(a_idx + k * 64u, idx);
+            };
+            if (ng == UNIT_G) {
+#pragma unroll kSpecUnroll
+                for (uint32_t k = 0; k < UNIT_G; ++k) step(k);
+            } else {
+                for (uint32_t k = 0; k < ng; ++k) step(k);
+            }
+            if (__any_sync(FULL, fbm != 0u)) {          // (rare) overflowing cells
+                for (uint32_t k = 0; k < ng; ++k) {
+                    if (!((fbm >> k) & 1u)) continue;
+                    RawChunk<DT> v;
+                    v.load(x, (size_t)(Gu + k) * 32u + (uint32_t)lane);
+                    s_idx[k * 32 + lane] =
+                        (uint16_t)sloop_index(v.e(0), v.e(1), v.e(2), v.e(3), cb, S);
                 }
-                radius[j] = rh;
-                s_idx[k * 32 + lane] = (uint16_t)idx;
             }
             __syncwarp();
-            pack_tile<BB>(s_idx, ng, lane, words + Gu * BB);
+            pack_tile<BB>(s_idx, ng, lane, words + (size_t)Gu * BB);
             if ((uint32_t)lane < ng) sa.cbits[Gu + lane] = s_cb[lane];
             n_def = __reduce_add_sync(FULL, n_def);
             if (lane == 0 && n_def) atomicAdd(sa.tile_cnt + tile, n_def);
