@@ -55,7 +55,8 @@ extern "C" int hqmq_launch_fix_pass(const void *x, int dtype, int B, int H, int 
                                     const float *thr, uint32_t *words, uint16_t *radius,
                                     const uint32_t *tile_off, uint64_t cap, uint32_t *out_idx,
                                     uint16_t *out_val, void *ws, hqmq_status *st, int sm_count,
-                                    cudaStream_t stream);
+                                    cudaStream_t stream,
+                                    int use_cvals);
 extern "C" int hqmq_launch_list_pass(const void *x, int dtype, int B, int H, int T, int D,
                                      const float *cb, uint32_t S, uint32_t b, const void *table,
                                      const float *thr, int gran, uint32_t *words,
@@ -282,7 +283,7 @@ int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, flo
         if (rc == HQMQ_OK)
             rc = hqmq_launch_fix_pass(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table, d_thr,
                                       d_idx_words, d_radius, tile_off, cap, d_out_idx, d_out_val,
-                                      d_ws, d_status, sm, s);
+                                      d_ws, d_status, sm, s, hqmq_spec_encode_supported(b));
         return rc;
     }
     int rc = hqmq_launch_med3_window(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr, d_slab_off,

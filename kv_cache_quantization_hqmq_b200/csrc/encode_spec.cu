@@ -148,6 +148,7 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
         if (ua >= ub) continue;                          // (warp-uniform)
         const WinState w = sa.win[h];
         const uint32_t span = w.hi_key - w.lo_key;
+        const int top = median_top_shift(span);
         const uint4 *tb = tables + (size_t)h * LUT_ENTRIES;
         const float4 *cb = cb_all + (size_t)h * S;
         // packing groups of the call (fewer than 2^27: 32-bit indices)
@@ -169,7 +170,8 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
             const uint32_t ng = min((uint32_t)UNIT_G, gps - g0);
             const uint32_t Gu = g_slab + g0;
             const uint32_t tile = slab * tps + g0 / TILE_GROUPS;
-            uint32_t n_def = 0, fbm = 0;
+            uint32_t n_def = 0, fbm = 0, n_cv = 0;
+            unsigned char *cv_u = sa.cvals + (size_t)u * (CVAL_SLOTS * CB);
             auto step = [&](const uint32_t k) {
                 const uint32_t G = Gu + k;
                 // group G's copy was the (NS-1)-th latest commit: wait for it
@@ -193,7 +195,8 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
                 if (mi) {
                     if (n_stage + 32 > SPEC_STAGE) {
                         flush_stage(stage, n_stage, lane, sa.cand_n + h,
-                                    sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap);
+                                    sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap,
+                                    sa.med_hist + (size_t)h * MED_BINS, w.lo_key, top);
                         n_stage = 0;
                     }
                     if (in) stage[n_stage + __popc(mi & lt)] = key;
@@ -206,6 +209,12 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
                 n_def += dfn ? 1u : 0u;
                 const uint32_t mc = __ballot_sync(FULL, cnd);
                 if (lane == 0) sts_u32(a_cb + k * 4u, mc);
+                {   // the raw value of a possible outlier, for the fix-up pass
+                    const uint32_t pos = n_cv + __popc(mc & lt);
+                    if (cnd && pos < (uint32_t)CVAL_SLOTS)
+                        *reinterpret_cast<decltype(cur.v) *>(cv_u + pos * CB) = cur.v;
+                    n_cv += __popc(mc);
+                }
                 const uint32_t mu = __ballot_sync(FULL, cnd && !dfn);
                 if (mu) {
                     unsigned long long base = 0;
@@ -303,7 +312,7 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
         if (lane == 0 && n_below) atomicAdd(sa.below + h, (unsigned long long)n_below);
         if (n_stage)
             flush_stage(stage, n_stage, lane, sa.cand_n + h, sa.cand + (uint64_t)h * sa.cand_cap,
-                        sa.cand_cap);
+                        sa.cand_cap, sa.med_hist + (size_t)h * MED_BINS, w.lo_key, top);
         const unsigned nf = __reduce_add_sync(FULL, n_nf);
         const unsigned ns = __reduce_add_sync(FULL, n_sat);
         if (lane == 0 && (nf | ns)) {

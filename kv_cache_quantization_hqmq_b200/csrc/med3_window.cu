@@ -251,7 +251,8 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
          const WinState *__restrict__ win, unsigned long long *__restrict__ below,
          unsigned long long *__restrict__ cand_n, uint32_t *__restrict__ cand, uint64_t cand_cap,
          unsigned long long *__restrict__ amb_n,
-         uint2 *__restrict__ amb, uint64_t amb_cap, uint32_t *__restrict__ tile_cnt) {
+         uint2 *__restrict__ amb, uint64_t amb_cap, uint32_t *__restrict__ tile_cnt,
+         uint32_t *__restrict__ med_hist) {
     constexpr int NK = GRAN == HQMQ_GRAN_CHUNK ? 1 : 4;
     constexpr int U = 8;                              // groups in flight per lane
     const int lane = threadIdx.x & 31;
@@ -269,9 +270,13 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
         const int h = (int)(slab % (uint64_t)H);
         const WinState w = win[h];
         if (h != stage_h) {                                   // warp-uniform
-            if (n_stage)
+            if (n_stage) {
+                const WinState ws = win[stage_h];
                 flush_stage(stage, n_stage, lane, cand_n + stage_h,
-                            cand + (uint64_t)stage_h * cand_cap, cand_cap);
+                            cand + (uint64_t)stage_h * cand_cap, cand_cap,
+                            med_hist + (size_t)stage_h * MED_BINS, ws.lo_key,
+                            median_top_shift(ws.hi_key - ws.lo_key));
+            }
             n_stage = 0;
             stage_h = h;
         }
@@ -300,7 +305,9 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
                     if (m) {
                         if (n_stage + 32 > STAGE) {
                             flush_stage(stage, n_stage, lane, cand_n + h,
-                                        cand + (uint64_t)h * cand_cap, cand_cap);
+                                        cand + (uint64_t)h * cand_cap, cand_cap,
+                                        med_hist + (size_t)h * MED_BINS, w.lo_key,
+                                        median_top_shift(w.hi_key - w.lo_key));
                             n_stage = 0;
                         }
                         if (in) {
@@ -332,9 +339,12 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
             if (n_below) atomicAdd(below + h, n_below);
         }
     }
-    if (n_stage)
+    if (n_stage) {
+        const WinState ws = win[stage_h];
         flush_stage(stage, n_stage, lane, cand_n + stage_h, cand + (uint64_t)stage_h * cand_cap,
-                    cand_cap);
+                    cand_cap, med_hist + (size_t)stage_h * MED_BINS, ws.lo_key,
+                    median_top_shift(ws.hi_key - ws.lo_key));
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -373,8 +383,7 @@ __device__ MedianPlan median_plan(int h, uint64_t n_per_head, const WinState &w,
     p.ok = !(amb_overflow || k < 0 || (unsigned long long)k >= p.nc || p.nc > cand_cap);
     p.k = p.ok ? (uint32_t)k : 0u;
     p.span = w.hi_key - w.lo_key;                      // >= 2^15
-    const int bits = 32 - __clz(p.span - 1);
-    p.top = ((bits + 11) / 12 - 1) * 12;
+    p.top = median_top_shift(p.span);
     return p;
 }
 
@@ -579,8 +588,8 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
            const uint2 *__restrict__ amb, uint64_t amb_cap, float *__restrict__ rmed,
            float *__restrict__ thr, uint32_t *__restrict__ tile_cnt,
            uint32_t *__restrict__ tile_off, uint32_t *__restrict__ slab_off, uint32_t n_slabs,
-           uint64_t cap, uint32_t *__restrict__ med_hist, uint32_t *__restrict__ median_done,
-           uint32_t *__restrict__ fin_done, DevStatus *st) {
+           uint64_t cap, const uint32_t *__restrict__ med_hist, uint32_t *__restrict__ fin_done,
+           DevStatus *st) {
     __shared__ FinalSmem sm;
     const int h = blockIdx.y;
     const WinState w = win[h];
@@ -588,24 +597,9 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
     const MedianPlan mp = median_plan(h, n_per_head, w, below, cand_n, cand_cap,
                                       n_amb > amb_cap);
     const uint32_t *ch = cand + (uint64_t)h * cand_cap;
-    uint32_t *gh = med_hist + (size_t)h * MED_BINS;
-    if (mp.ok) {                                       // (block-uniform) top digit, one slice
-        for (uint32_t i = threadIdx.x; i < MED_BINS; i += WIN_THREADS) sm.buf[i] = 0;
-        __syncthreads();
-        const uint64_t i0 = mp.nc * blockIdx.x / gridDim.x, i1 = mp.nc * (blockIdx.x + 1) / gridDim.x;
-        median_count(ch, i0, i1, w, mp.span, mp.top, 0u, sm.buf);
-        __syncthreads();
-        for (uint32_t i = threadIdx.x; i < MED_BINS; i += WIN_THREADS)
-            if (sm.buf[i]) atomicAdd(gh + i, sm.buf[i]);
-    }
-    // the head's last CTA (no CTA waits for another) finishes the head
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0)
-        sm.last = atomicAdd(median_done + h, 1u) == gridDim.x - 1 ? 1u : 0u;
-    __syncthreads();
-    if (!sm.last) return;
-    __threadfence();
+    // the top digit's counts of the staged keys were added when they were
+    // staged (flush_stage): the histogram is complete here
+    const uint32_t *gh = med_hist + (size_t)h * MED_BINS;
     if (!mp.ok) {
         if (threadIdx.x == 0) win[h].miss = 1;
         exact_fallback<DT, GRAN>(x, B, H, h, cps, tiles_per_slab, n_per_head, C, rmed, thr,
@@ -688,7 +682,7 @@ static int run_front(const void *x, int B, int H, int T, int D, float C, char *w
         if (bx > bmax) bx = bmax;
         k_pass_b<DT, GRAN><<<(unsigned)bx, PB_THREADS, 0, stream>>>(
             x, H, cps, L.tiles_per_slab, L.n_tiles, win, a.below, a.cand_n, a.cand, a.cand_cap,
-            a.amb_n, a.amb, a.amb_cap, a.tile_cnt);
+            a.amb_n, a.amb, a.amb_cap, a.tile_cnt, a.med_hist);
     }
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
@@ -704,12 +698,11 @@ static int run_finish(const void *x, int B, int H, int T, int D, float C, float 
     Counters *ctr = reinterpret_cast<Counters *>(ws + L.counters);
     WinState *win = reinterpret_cast<WinState *>(ws + L.win);
     const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
-    uint32_t *median_done = reinterpret_cast<uint32_t *>(ws + L.counters + sizeof(Counters)) + H;
     uint32_t *med_hist = reinterpret_cast<uint32_t *>(ws + L.med_hist);
-    k_finalize<DT, GRAN><<<dim3(MED_SLICES, H), WIN_THREADS, 0, stream>>>(
+    k_finalize<DT, GRAN><<<dim3(1, H), WIN_THREADS, 0, stream>>>(
         x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, a.below, a.cand_n,
         a.cand, a.cand_cap, a.amb_n, a.amb, a.amb_cap, rmed, thr, a.tile_cnt, tile_off, slab_off,
-        (uint32_t)(B * H), cap, med_hist, median_done, &ctr->fin_done, st);
+        (uint32_t)(B * H), cap, med_hist, &ctr->fin_done, st);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 

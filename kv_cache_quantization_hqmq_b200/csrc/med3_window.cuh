@@ -29,15 +29,14 @@ struct Counters {
     uint32_t fin_done;         // CTAs of the finalize step that are done
     uint32_t pad;
     // followed by uint32_t sample_done[H]: sample CTAs of head h that are done,
-    // then uint32_t median_done[H]: finalize CTAs of head h that are done
 };
 
-constexpr int MED_SLICES = 16;                   // finalize CTAs per head
 constexpr int MED_BINS = 4096;                   // radix digit of the median select (12 bits)
+constexpr int CVAL_SLOTS = 32;                   // possible outliers kept per 256-chunk unit
 
 struct FusedLayout {
     uint64_t sample_hist, counters, med_hist, win, below, cand_n, cand, amb, tile_cnt, tile_off,
-        cbits, head_stat, total;
+        cbits, head_stat, cvals, total;
     uint64_t zero_bytes;       // [0, zero_bytes) is cleared per call
     uint64_t cand_cap;         // keys per head
     uint64_t amb_cap;          // (tile, key) pairs per call
@@ -78,21 +77,39 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     L.amb = off;         off = align256_(off + L.amb_cap * 8);
     L.tile_off = off;    off = align256_(off + (L.n_tiles + 1) * 4);
     L.cbits = off;       off = align256_(off + (uint64_t)B * H * gps * 4);
+    // raw values of the possible outliers (r > t_lo), CVAL_SLOTS per 8-group
+    // unit (chunk mode; 16 bytes per chunk covers fp32 input)
+    L.cvals = off;       off = align256_(off + (uint64_t)B * H * ((gps + 7) / 8) * CVAL_SLOTS * 16);
     L.total = off;
     return L;
 }
 
 constexpr int STAGE = 256;          // window keys staged per warp before one global append
 
-// Appends the warp's staged window keys to the head's buffer (one atomic).
+// Shift of the top radix digit of the median select: keys are taken as
+// d = key - lo_key < span, cut into 12-bit digits from the top of the span.
+__host__ __device__ __forceinline__ int median_top_shift(uint32_t span) {
+    int bits = 0;
+    for (uint32_t v = span - 1u; v; v >>= 1) ++bits;
+    return ((bits + 11) / 12 - 1) * 12;
+}
+
+// Appends the warp's staged window keys to the head's buffer (one atomic) and
+// counts each appended key's top digit (median_top_shift) into the head's
+// digit histogram, so that the select starts from a complete histogram.
 __device__ __forceinline__ void flush_stage(uint32_t *stage, uint32_t n, int lane,
                                             unsigned long long *cand_n_h, uint32_t *cand_h,
-                                            uint64_t cand_cap) {
+                                            uint64_t cand_cap, uint32_t *hist_h, uint32_t lo_key,
+                                            int top) {
     unsigned long long base = 0;
     if (lane == 0) base = atomicAdd(cand_n_h, (unsigned long long)n);
     base = __shfl_sync(FULL, base, 0);
     for (uint32_t i = lane; i < n; i += 32)
-        if (base + i < cand_cap) cand_h[base + i] = stage[i];
+        if (base + i < cand_cap) {
+            const uint32_t key = stage[i];
+            cand_h[base + i] = key;
+            atomicAdd(hist_h + (((key - lo_key) >> top) & (MED_BINS - 1)), 1u);
+        }
     __syncwarp();
 }
 
@@ -108,6 +125,8 @@ struct SpecArgs {
     uint64_t cand_cap, amb_cap;
     uint32_t *cbits;                 // per packing group: chunks with r > t_lo
     unsigned long long *head_stat;   // per head: [non-finite, saturated] of the encode pass
+    uint32_t *med_hist;              // per head: top-digit counts of the staged keys
+    unsigned char *cvals;            // per unit: raw values of its first CVAL_SLOTS possible outliers
 };
 
 inline SpecArgs spec_args(char *ws, const FusedLayout &L) {
@@ -123,6 +142,8 @@ inline SpecArgs spec_args(char *ws, const FusedLayout &L) {
     a.amb_cap = L.amb_cap;
     a.cbits = reinterpret_cast<uint32_t *>(ws + L.cbits);
     a.head_stat = reinterpret_cast<unsigned long long *>(ws + L.head_stat);
+    a.med_hist = reinterpret_cast<uint32_t *>(ws + L.med_hist);
+    a.cvals = reinterpret_cast<unsigned char *>(ws + L.cvals);
     return a;
 }
 

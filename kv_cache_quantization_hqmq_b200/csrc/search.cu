@@ -198,9 +198,13 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
         WinState w{};
         if (LIST == LIST_SPEC) w = sa.win[h];
         if (LIST == LIST_SPEC && h != stage_h) {
-            if (n_stage)
+            if (n_stage) {
+                const WinState ws = sa.win[stage_h];
                 flush_stage(stage, n_stage, lane, sa.cand_n + stage_h,
-                            sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap);
+                            sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap,
+                            sa.med_hist + (size_t)stage_h * MED_BINS, ws.lo_key,
+                            median_top_shift(ws.hi_key - ws.lo_key));
+            }
             n_stage = 0;
             stage_h = h;
         }
@@ -284,7 +288,9 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                     if (mi) {
                         if (n_stage + 32 > STAGE) {
                             flush_stage(stage, n_stage, lane, sa.cand_n + h,
-                                        sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap);
+                                        sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap,
+                                        sa.med_hist + (size_t)h * MED_BINS, w.lo_key,
+                                        median_top_shift(w.hi_key - w.lo_key));
                             n_stage = 0;
                         }
                         if (in) stage[n_stage + __popc(mi & lt)] = key;
@@ -406,9 +412,13 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
         seg = seg_end;
     }
     if (LIST == LIST_SPEC) {
-        if (n_stage)
+        if (n_stage) {
+            const WinState ws = sa.win[stage_h];
             flush_stage(stage, n_stage, lane, sa.cand_n + stage_h,
-                        sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap);
+                        sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap,
+                        sa.med_hist + (size_t)stage_h * MED_BINS, ws.lo_key,
+                        median_top_shift(ws.hi_key - ws.lo_key));
+        }
         return;
     }
     const unsigned nf = __reduce_add_sync(FULL, n_nf);
@@ -435,7 +445,12 @@ k_list_fix(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32_t
            const float *__restrict__ thr, uint32_t *__restrict__ words,
            uint16_t *__restrict__ radius, const uint32_t *__restrict__ tile_off, uint64_t cap,
            uint32_t *__restrict__ out_idx, uint16_t *__restrict__ out_val, DevStatus *st,
-           SpecArgs sa) {
+           SpecArgs sa, int use_cvals) {
+    // use_cvals: the encode pass kept the raw values of the first CVAL_SLOTS
+    // possible outliers of each 8-group unit, in chunk order (sa.cvals);
+    // chunks of a unit with more of them are read from x
+    constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;
+    const uint32_t units_per_slab = (groups_per_slab + 7) / 8;
     const int lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
     const uint32_t cap32 = cap < 0xFFFFFFFFull ? (uint32_t)cap : 0xFFFFFFFFu;
@@ -480,13 +495,23 @@ k_list_fix(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32_t
                 gl &= 31u;
                 const uint32_t ex = __shfl_sync(FULL, incl - pcount, (int)gl);
                 const uint32_t word = __shfl_sync(FULL, gw, (int)gl);
+                // the candidate's unit (8 groups) and its rank there
+                const uint32_t ug = gl & ~7u;
+                const uint32_t u_before = __shfl_sync(FULL, incl - pcount, (int)ug);
+                const uint32_t u_total = __shfl_sync(FULL, incl, (int)(ug + 7)) - u_before;
                 const uint32_t bit = c ? __fns(word, 0u, (int)(k - ex + 1)) : 0u;
                 const uint32_t G = gbase + g0 + gl;
                 const uint32_t j = G * 32 + bit;
                 float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f, r = 0.f;
                 if (c) {
                     RawChunk<DT> v;
-                    v.load(x, j);
+                    if (use_cvals && u_total <= (uint32_t)CVAL_SLOTS) {
+                        const uint32_t u = slab * units_per_slab + (g0 + gl) / 8;
+                        v.v = *reinterpret_cast<const decltype(v.v) *>(
+                            sa.cvals + ((size_t)u * CVAL_SLOTS + (k - u_before)) * CB);
+                    } else {
+                        v.load(x, j);
+                    }
                     x0 = v.e(0); x1 = v.e(1); x2 = v.e(2); x3 = v.e(3);
                     r = chunk_norm(x0, x1, x2, x3);
                 }
@@ -714,7 +739,7 @@ extern "C" int hqmq_launch_fix_pass(const void *x, int dtype, int B, int H, int 
                                     const float *thr, uint32_t *words, uint16_t *radius,
                                     const uint32_t *tile_off, uint64_t cap, uint32_t *out_idx,
                                     uint16_t *out_val, void *ws, hqmq_status *st, int sm_count,
-                                    cudaStream_t stream) {
+                                    cudaStream_t stream, int use_cvals) {
     using namespace hqmq;
     (void)table;
     const SpecArgs sa = spec_args(reinterpret_cast<char *>(ws),
@@ -731,10 +756,10 @@ extern "C" int hqmq_launch_fix_pass(const void *x, int dtype, int B, int H, int 
     if (dtype == HQMQ_BF16)
         k_list_fix<HQMQ_BF16><<<(unsigned)ctas, FIX_THREADS, 0, stream>>>(
             x, H, gps, tps, n_tiles, cb4, S, b, thr, words, radius, tile_off, cap, out_idx,
-            out_val, dst, sa);
+            out_val, dst, sa, use_cvals);
     else
         k_list_fix<HQMQ_F32><<<(unsigned)ctas, FIX_THREADS, 0, stream>>>(
             x, H, gps, tps, n_tiles, cb4, S, b, thr, words, radius, tile_off, cap, out_idx,
-            out_val, dst, sa);
+            out_val, dst, sa, use_cvals);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
