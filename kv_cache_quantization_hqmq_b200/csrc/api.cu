@@ -39,8 +39,9 @@ extern "C" int hqmq_launch_med3_front(const void *x, int dtype, int B, int H, in
 extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, int T, int D,
                                        float C, int gran, float *rmed, float *thr,
                                        uint32_t *slab_off, uint32_t *tile_off_out, uint64_t cap,
-                                       void *ws, hqmq_status *st, cudaStream_t stream,
-                                       const uint32_t **tile_off, uint32_t *tiles_per_slab);
+                                       void *ws, hqmq_status *st, int sm_count,
+                                       cudaStream_t stream, const uint32_t **tile_off,
+                                       uint32_t *tiles_per_slab);
 extern "C" int hqmq_spec_encode_supported(uint32_t b);
 extern "C" int hqmq_launch_spec_encode_units(const void *x, int dtype, int B, int H, int T, int D,
                                              const float *cb, uint32_t S, uint32_t b,
@@ -278,7 +279,7 @@ int hqmq_encode_med3(const void *d_x, int dtype, int B, int H, int T, int D, flo
                                                d_idx_words, d_radius, d_ws, sm, s);
         if (rc == HQMQ_OK)
             rc = hqmq_launch_med3_finish(d_x, dtype, B, H, T, D, C, gran, d_rmed, d_thr,
-                                         d_slab_off, d_tile_off, cap, d_ws, d_status, s,
+                                         d_slab_off, d_tile_off, cap, d_ws, d_status, sm, s,
                                          &tile_off, &tps);
         if (rc == HQMQ_OK)
             rc = hqmq_launch_fix_pass(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table, d_thr,

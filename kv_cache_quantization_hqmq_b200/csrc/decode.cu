@@ -113,7 +113,7 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
         uint32_t rr[DEC_UNIT / 2];
 #pragma unroll
         for (int u = 0; u < DEC_UNIT / 2; ++u)     // radius pairs: all in flight
-            rr[u] = (!RQ && (uint32_t)(2 * u) < ng)
+            rr[u] = (!RQ && (uint32_t)(u * 64 + 2 * lane) < ng * 32u)
                         ? __ldcs(reinterpret_cast<const uint32_t *>(radius + gg0 * 32) + u * 32 + lane)
                         : 0u;
         __syncwarp();                              // (the previous unit's reads of s_w)
@@ -126,6 +126,9 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
         for (int u = 0; u < DEC_UNIT / 2; ++u) {
             if ((uint32_t)(2 * u) >= ng) break;
             const uint32_t c = (uint32_t)u * 64 + 2u * lane;        // chunk within the unit
+            // (a unit with an odd number of groups ends inside its last half:
+            // lanes past it neither load nor store)
+            const bool live = c < ng * 32u;
             uint32_t ixs[2], rks[2] = {0u, 0u};
             if (b <= 16) {                         // both indices from one 64-bit window
                 const uint32_t bit = c * b, o = bit & 31u;
@@ -162,7 +165,7 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
                 } else {
                     cw = make_float4(0.f, 0.f, 0.f, 0.f);
                     r = 0.0f;
-                    ++n_bad;
+                    n_bad += live ? 1u : 0u;
                 }
                 out[4 * v] = __fmul_rn(r, cw.x);
                 out[4 * v + 1] = __fmul_rn(r, cw.y);
@@ -170,7 +173,8 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
                 out[4 * v + 3] = __fmul_rn(r, cw.w);
             }
             const uint64_t j = gg0 * 32 + c;
-            if (OUT_DT == HQMQ_BF16) {
+            if (!live) {
+            } else if (OUT_DT == HQMQ_BF16) {
                 __nv_bfloat162 a0 = __floats2bfloat162_rn(out[0], out[1]);
                 __nv_bfloat162 a1 = __floats2bfloat162_rn(out[2], out[3]);
                 __nv_bfloat162 a2 = __floats2bfloat162_rn(out[4], out[5]);

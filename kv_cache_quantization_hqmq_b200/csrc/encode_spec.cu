@@ -196,7 +196,7 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
                     if (n_stage + 32 > SPEC_STAGE) {
                         flush_stage(stage, n_stage, lane, sa.cand_n + h,
                                     sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap,
-                                    sa.med_hist + (size_t)h * MED_BINS, w.lo_key, top);
+                                    sa.med_hist + (size_t)h * MED_BINS * 2, w.lo_key, top);
                         n_stage = 0;
                     }
                     if (in) stage[n_stage + __popc(mi & lt)] = key;
@@ -312,7 +312,7 @@ k_encode_spec(const void *__restrict__ x, int H, uint32_t gps, uint32_t ups, uin
         if (lane == 0 && n_below) atomicAdd(sa.below + h, (unsigned long long)n_below);
         if (n_stage)
             flush_stage(stage, n_stage, lane, sa.cand_n + h, sa.cand + (uint64_t)h * sa.cand_cap,
-                        sa.cand_cap, sa.med_hist + (size_t)h * MED_BINS, w.lo_key, top);
+                        sa.cand_cap, sa.med_hist + (size_t)h * MED_BINS * 2, w.lo_key, top);
         const unsigned nf = __reduce_add_sync(FULL, n_nf);
         const unsigned ns = __reduce_add_sync(FULL, n_sat);
         if (lane == 0 && (nf | ns)) {

@@ -274,7 +274,7 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
                 const WinState ws = win[stage_h];
                 flush_stage(stage, n_stage, lane, cand_n + stage_h,
                             cand + (uint64_t)stage_h * cand_cap, cand_cap,
-                            med_hist + (size_t)stage_h * MED_BINS, ws.lo_key,
+                            med_hist + (size_t)stage_h * MED_BINS * 2, ws.lo_key,
                             median_top_shift(ws.hi_key - ws.lo_key));
             }
             n_stage = 0;
@@ -306,7 +306,7 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
                         if (n_stage + 32 > STAGE) {
                             flush_stage(stage, n_stage, lane, cand_n + h,
                                         cand + (uint64_t)h * cand_cap, cand_cap,
-                                        med_hist + (size_t)h * MED_BINS, w.lo_key,
+                                        med_hist + (size_t)h * MED_BINS * 2, w.lo_key,
                                         median_top_shift(w.hi_key - w.lo_key));
                             n_stage = 0;
                         }
@@ -342,7 +342,7 @@ k_pass_b(const void *__restrict__ x, int H, uint32_t cps, uint32_t tiles_per_sla
     if (n_stage) {
         const WinState ws = win[stage_h];
         flush_stage(stage, n_stage, lane, cand_n + stage_h, cand + (uint64_t)stage_h * cand_cap,
-                    cand_cap, med_hist + (size_t)stage_h * MED_BINS, ws.lo_key,
+                    cand_cap, med_hist + (size_t)stage_h * MED_BINS * 2, ws.lo_key,
                     median_top_shift(ws.hi_key - ws.lo_key));
     }
 }
@@ -588,8 +588,8 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
            const uint2 *__restrict__ amb, uint64_t amb_cap, float *__restrict__ rmed,
            float *__restrict__ thr, uint32_t *__restrict__ tile_cnt,
            uint32_t *__restrict__ tile_off, uint32_t *__restrict__ slab_off, uint32_t n_slabs,
-           uint64_t cap, const uint32_t *__restrict__ med_hist, uint32_t *__restrict__ fin_done,
-           DevStatus *st) {
+           uint64_t cap, uint32_t *__restrict__ med_hist, uint32_t *__restrict__ median_done,
+           uint32_t *__restrict__ fin_done, DevStatus *st) {
     __shared__ FinalSmem sm;
     const int h = blockIdx.y;
     const WinState w = win[h];
@@ -597,19 +597,50 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
     const MedianPlan mp = median_plan(h, n_per_head, w, below, cand_n, cand_cap,
                                       n_amb > amb_cap);
     const uint32_t *ch = cand + (uint64_t)h * cand_cap;
-    // the top digit's counts of the staged keys were added when they were
-    // staged (flush_stage): the histogram is complete here
-    const uint32_t *gh = med_hist + (size_t)h * MED_BINS;
+    // per head two digit histograms: the top digit's counts of the staged keys
+    // were added when they were staged (flush_stage), so the top digit is
+    // known here; the MED_SLICES CTAs of the head count the next digit of
+    // the keys inside that top bin, each over a slice of the keys
+    uint32_t *gh = med_hist + (size_t)h * MED_BINS * 2;
+    uint32_t *gh2 = gh + MED_BINS;
+    uint32_t prefix = 0, rem = 0;
+    if (mp.ok) {                                       // (block-uniform)
+        block_select2<MED_BINS, true>(gh, mp.k, mp.k, sm.wtot, sm.out);
+        prefix = sm.out[0] << mp.top;
+        rem = sm.out[2];
+        __syncthreads();                               // (everyone has read out[])
+        if (mp.top > 0) {
+            for (uint32_t i = threadIdx.x; i < MED_BINS; i += WIN_THREADS) sm.buf[i] = 0;
+            __syncthreads();
+            const uint64_t i0 = mp.nc * blockIdx.x / gridDim.x;
+            const uint64_t i1 = mp.nc * (blockIdx.x + 1) / gridDim.x;
+            median_count(ch, i0, i1, w, mp.span, mp.top - 12, prefix, sm.buf);
+            __syncthreads();
+            for (uint32_t i = threadIdx.x; i < MED_BINS; i += WIN_THREADS)
+                if (sm.buf[i]) atomicAdd(gh2 + i, sm.buf[i]);
+        }
+    }
+    // the head's last CTA (no CTA waits for another) finishes the head
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+        sm.last = atomicAdd(median_done + h, 1u) == gridDim.x - 1 ? 1u : 0u;
+    __syncthreads();
+    if (!sm.last) return;
+    __threadfence();
     if (!mp.ok) {
         if (threadIdx.x == 0) win[h].miss = 1;
         exact_fallback<DT, GRAN>(x, B, H, h, cps, tiles_per_slab, n_per_head, C, rmed, thr,
                                  tile_cnt, st, sm);
     } else {
-        block_select2<MED_BINS, true>(gh, mp.k, mp.k, sm.wtot, sm.out);
-        uint32_t prefix = sm.out[0] << mp.top;
-        uint32_t rem = sm.out[2];
-        __syncthreads();                               // (everyone has read out[])
-        for (int sh = mp.top - 12; sh >= 0; sh -= 12) {
+        if (mp.top > 0) {
+            block_select2<MED_BINS, true>(gh2, rem, rem, sm.wtot, sm.out);
+            prefix |= sm.out[0] << (mp.top - 12);
+            rem = sm.out[2];
+            __syncthreads();
+        }
+        // further digits (spans above 2^24 only): this CTA over all keys
+        for (int sh = mp.top - 24; sh >= 0; sh -= 12) {
             for (uint32_t i = threadIdx.x; i < MED_BINS; i += WIN_THREADS) sm.buf[i] = 0;
             __syncthreads();
             median_count(ch, 0, mp.nc, w, mp.span, sh, prefix, sm.buf);
@@ -691,18 +722,26 @@ static int run_front(const void *x, int B, int H, int T, int D, float C, char *w
 template <int DT, int GRAN>
 static int run_finish(const void *x, int B, int H, int T, int D, float C, float *rmed, float *thr,
                       uint32_t *slab_off, uint32_t *tile_off, uint64_t cap, char *ws,
-                      hqmq_status *st_, cudaStream_t stream) {
+                      hqmq_status *st_, int sm_count, cudaStream_t stream) {
     DevStatus *st = reinterpret_cast<DevStatus *>(st_);
     const FusedLayout L = fused_layout(B, H, T, D, GRAN);
     const SpecArgs a = spec_args(ws, L);
     Counters *ctr = reinterpret_cast<Counters *>(ws + L.counters);
     WinState *win = reinterpret_cast<WinState *>(ws + L.win);
     const uint32_t cps = (uint32_t)((uint64_t)T * D / 4);
+    uint32_t *median_done = reinterpret_cast<uint32_t *>(ws + L.counters + sizeof(Counters)) + H;
     uint32_t *med_hist = reinterpret_cast<uint32_t *>(ws + L.med_hist);
-    k_finalize<DT, GRAN><<<dim3(1, H), WIN_THREADS, 0, stream>>>(
+    // slices per head: one per 2^18 keys of the head (the window holds a few
+    // percent of them), at most MED_SLICES and about one wave of CTAs in all
+    uint64_t slices = L.n_per_head >> 18;
+    const uint64_t wave = (uint64_t)sm_count / (uint64_t)(H > 0 ? H : 1);
+    if (slices > wave) slices = wave;
+    if (slices > (uint64_t)MED_SLICES) slices = MED_SLICES;
+    if (slices < 1) slices = 1;
+    k_finalize<DT, GRAN><<<dim3((unsigned)slices, H), WIN_THREADS, 0, stream>>>(
         x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, a.below, a.cand_n,
         a.cand, a.cand_cap, a.amb_n, a.amb, a.amb_cap, rmed, thr, a.tile_cnt, tile_off, slab_off,
-        (uint32_t)(B * H), cap, med_hist, &ctr->fin_done, st);
+        (uint32_t)(B * H), cap, med_hist, median_done, &ctr->fin_done, st);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
@@ -734,7 +773,7 @@ extern "C" int hqmq_launch_med3_front(const void *x, int dtype, int B, int H, in
 extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, int T, int D,
                                        float C, int gran, float *rmed, float *thr,
                                        uint32_t *slab_off, uint32_t *tile_off_out, uint64_t cap,
-                                       void *ws, hqmq_status *st, cudaStream_t stream,
+                                       void *ws, hqmq_status *st, int sm_count, cudaStream_t stream,
                                        const uint32_t **tile_off, uint32_t *tiles_per_slab) {
     using namespace hqmq;
     const FusedLayout L = fused_layout(B, H, T, D, gran);
@@ -745,14 +784,14 @@ extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, i
     if (dtype == HQMQ_BF16)
         return gran == HQMQ_GRAN_CHUNK
                    ? run_finish<HQMQ_BF16, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off,
-                                                            to, cap, w, st, stream)
+                                                            to, cap, w, st, sm_count, stream)
                    : run_finish<HQMQ_BF16, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr,
-                                                              slab_off, to, cap, w, st, stream);
+                                                              slab_off, to, cap, w, st, sm_count, stream);
     return gran == HQMQ_GRAN_CHUNK
                ? run_finish<HQMQ_F32, HQMQ_GRAN_CHUNK>(x, B, H, T, D, C, rmed, thr, slab_off, to,
-                                                       cap, w, st, stream)
+                                                       cap, w, st, sm_count, stream)
                : run_finish<HQMQ_F32, HQMQ_GRAN_ELEMENT>(x, B, H, T, D, C, rmed, thr, slab_off, to,
-                                                         cap, w, st, stream);
+                                                         cap, w, st, sm_count, stream);
 }
 
 // All steps A..S (two-read path); returns the tile offsets for pass C.
@@ -765,7 +804,8 @@ extern "C" int hqmq_launch_med3_window(const void *x, int dtype, int B, int H, i
     const int rc = hqmq_launch_med3_front(x, dtype, B, H, T, D, C, gran, ws, 1, sm_count, stream);
     if (rc != HQMQ_OK) return rc;
     return hqmq_launch_med3_finish(x, dtype, B, H, T, D, C, gran, rmed, thr, slab_off,
-                                   tile_off_out, cap, ws, st, stream, tile_off, tiles_per_slab);
+                                   tile_off_out, cap, ws, st, sm_count, stream, tile_off,
+                                   tiles_per_slab);
 }
 
 extern "C" uint64_t hqmq_list_tile_count(int B, int H, int T, int D) {

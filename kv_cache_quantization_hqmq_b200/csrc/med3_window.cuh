@@ -29,10 +29,12 @@ struct Counters {
     uint32_t fin_done;         // CTAs of the finalize step that are done
     uint32_t pad;
     // followed by uint32_t sample_done[H]: sample CTAs of head h that are done,
+    // then uint32_t median_done[H]: finalize CTAs of head h that are done
 };
 
 constexpr int MED_BINS = 4096;                   // radix digit of the median select (12 bits)
 constexpr int CVAL_SLOTS = 32;                   // possible outliers kept per 256-chunk unit
+constexpr int MED_SLICES = 16;                   // finalize CTAs per head
 
 struct FusedLayout {
     uint64_t sample_hist, counters, med_hist, win, below, cand_n, cand, amb, tile_cnt, tile_off,
@@ -66,7 +68,7 @@ inline FusedLayout fused_layout(int B, int H, int T, int D, int gran) {
     uint64_t off = 0;
     L.sample_hist = off; off = align256_(off + (uint64_t)H * KEY_BINS * 4);
     L.counters = off;    off = align256_(off + sizeof(Counters) + (uint64_t)H * 8);
-    L.med_hist = off;    off = align256_(off + (uint64_t)H * MED_BINS * 4);
+    L.med_hist = off;    off = align256_(off + (uint64_t)H * MED_BINS * 4 * 2);   // top digit, then next
     L.head_stat = off;   off = align256_(off + (uint64_t)H * 16);   // per head: non-finite, saturated
     L.tile_cnt = off;    off = align256_(off + L.n_tiles * 4);      // (a tile may be counted by several warps)
     L.zero_bytes = off;

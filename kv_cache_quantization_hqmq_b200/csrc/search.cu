@@ -202,7 +202,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                 const WinState ws = sa.win[stage_h];
                 flush_stage(stage, n_stage, lane, sa.cand_n + stage_h,
                             sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap,
-                            sa.med_hist + (size_t)stage_h * MED_BINS, ws.lo_key,
+                            sa.med_hist + (size_t)stage_h * MED_BINS * 2, ws.lo_key,
                             median_top_shift(ws.hi_key - ws.lo_key));
             }
             n_stage = 0;
@@ -289,7 +289,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
                         if (n_stage + 32 > STAGE) {
                             flush_stage(stage, n_stage, lane, sa.cand_n + h,
                                         sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap,
-                                        sa.med_hist + (size_t)h * MED_BINS, w.lo_key,
+                                        sa.med_hist + (size_t)h * MED_BINS * 2, w.lo_key,
                                         median_top_shift(w.hi_key - w.lo_key));
                             n_stage = 0;
                         }
@@ -416,7 +416,7 @@ k_encode_lut(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32
             const WinState ws = sa.win[stage_h];
             flush_stage(stage, n_stage, lane, sa.cand_n + stage_h,
                         sa.cand + (uint64_t)stage_h * sa.cand_cap, sa.cand_cap,
-                        sa.med_hist + (size_t)stage_h * MED_BINS, ws.lo_key,
+                        sa.med_hist + (size_t)stage_h * MED_BINS * 2, ws.lo_key,
                         median_top_shift(ws.hi_key - ws.lo_key));
         }
         return;

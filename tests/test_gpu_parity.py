@@ -231,6 +231,47 @@ def test_outlier_capacity_overflow(oracle):
     assert g["status"]["n_outliers"] > 100
 
 
+@pytest.mark.parametrize("shape", [(2, 3, 1, 128), (1, 2, 3, 128), (2, 1, 9, 128), (3, 2, 32, 4)])
+def test_decode_odd_group_counts(oracle, shape):
+    # slabs with an odd number of 32-chunk packing groups (one-token decode
+    # steps, D = 4): the last pair of groups of a slab is half empty; nothing
+    # may be written past the slab (the next slab, or past the tensor)
+    B, H, T, D = shape
+    rng = np.random.default_rng(sum(shape))
+    x = rng.standard_normal(shape).astype(np.float32)
+    x.reshape(-1, 4)[::7] *= 6.0
+    S = 8
+    cb = oracle.make_codebook(2, S, H)
+    cbd = dev(cb.reshape(-1))
+    _, thr_o = oracle.med3_threshold(x, 3.0, 0)
+    oi_o, ov_o, so_o, n_o, _ = oracle.extract(x, thr_o)
+    assert n_o > 0
+    ow, orad, _, _, _ = oracle.encode(x, cb, S, thr=thr_o)
+    n = B * H * T * D
+    for listed in ("none", "kernel", "tiles"):
+        yo, _ = oracle.decode(ow, orad, cb, S, B, H, T, D,
+                              out_idx=None if listed == "none" else oi_o,
+                              out_val=None if listed == "none" else ov_o, out_dtype=0)
+        guard = torch.full((n + 8192,), 0x5A5A, dtype=torch.int16, device="cuda")
+        y = guard[:n].view(torch.bfloat16).view(B, H, T, D)
+        st = hqmq.new_status()
+        if listed == "none":
+            hqmq.hqmq_decode(dev(ow.view(np.int32)), dev(orad.view(np.int16)), cbd, S, None, None,
+                             None, 0, 0, y, st)
+        else:
+            to = dev(list_tile_off(oi_o, B, H, T, D, 0).view(np.int32))
+            hqmq.hqmq_decode(dev(ow.view(np.int32)), dev(orad.view(np.int16)), cbd, S,
+                             dev(oi_o.view(np.int32)), dev(ov_o.reshape(-1).view(np.int16)),
+                             dev(so_o.view(np.int32)), n_o, 0, y, st,
+                             tile_off=to if listed == "tiles" else None)
+        torch.cuda.synchronize()
+        g = to_host(guard)
+        assert np.all(g[n:] == 0x5A5A), "decode wrote past the tensor (%s)" % listed
+        ok = same_f16_or_bf16_bits(g[:n].view(np.uint16), yo.reshape(-1), bf16=True)
+        assert ok.all(), (listed, np.argwhere(~ok.reshape(-1))[:5])
+        assert hqmq.read_status(st)["flags"] == 0
+
+
 def test_decode_bad_index_flag(oracle):
     words = torch.full((8,), -1, dtype=torch.int32, device="cuda")
     radius = torch.full((32,), 0x3C00, dtype=torch.int16, device="cuda")
