@@ -216,59 +216,98 @@ class Cache:
         """One pass over the cache.  timers: dict name -> list of (start, end)
         CUDA events recorded around the launches of that kernel family."""
         import torch
+        w = self.w
+        stream = torch.cuda.current_stream()
+        for l in range(w.layers):
+            for r in range(2):
+                x = self.x[l, r] if x_override is None else x_override(l, r)
+                self.call(l, r, x, stream, timers)
+
+    def call(self, l, r, x, stream, timers=None):
+        """One (layer, role) call on `stream`: Med3x + encode, then decode."""
+        import torch
         from kv_cache_quantization_hqmq_b200 import hqmq
         w = self.w
         H = w.heads
-        stream = torch.cuda.current_stream()
 
         def ev():
             e = torch.cuda.Event(enable_timing=True)
             e.record(stream)
             return e
 
-        for l in range(w.layers):
-            for r in range(2):
-                x = self.x[l, r] if x_override is None else x_override(l, r)
-                g0 = (l * 2 + r) * H
-                cb = self.codebook[g0 * w.S * 4:(g0 + H) * w.S * 4]
-                thr = None
-                tb = None
-                if self.table is not None:
-                    tb = self.table[g0 * self.table_bytes:(g0 + H) * self.table_bytes]
-                t0 = ev() if timers is not None else None
-                if w.med3:
-                    # Med3x and encode in one fused call (one read of x in chunk mode
-                    # with search tables, two otherwise)
-                    hqmq.hqmq_encode_med3(x, w.C, self.gran, cb, w.S, tb, self.words[l, r],
-                                          self.radius[l, r], self.rmed[l, r], self.thr[l, r],
-                                          self.out_idx[l, r], self.out_val[l, r],
-                                          self.slab_off[l, r], self.cap, self.ws, self.status,
-                                          stream, tile_off=self.tile_off[l, r])
-                elif self.table is not None:
-                    hqmq.hqmq_encode_lut(x, cb, w.S, tb, thr, self.gran, self.words[l, r],
-                                         self.radius[l, r], self.status, stream)
-                else:
-                    hqmq.hqmq_encode(x, cb, w.S, thr, self.gran, self.words[l, r],
-                                     self.radius[l, r], self.status, stream)
-                t1 = ev() if timers is not None else None
-                if w.med3:
-                    hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S,
-                                     self.out_idx[l, r], self.out_val[l, r], self.slab_off[l, r],
-                                     self.cap, self.gran, self.y, self.status, stream,
-                                     tile_off=self.tile_off[l, r])
-                else:
-                    hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S, None, None,
-                                     None, 0, self.gran, self.y, self.status, stream)
-                if timers is not None:
-                    t2 = ev()
-                    timers["med3_encode" if w.med3 else "encode"].append((t0, t1))
-                    timers["decode"].append((t1, t2))
+        g0 = (l * 2 + r) * H
+        cb = self.codebook[g0 * w.S * 4:(g0 + H) * w.S * 4]
+        tb = None
+        if self.table is not None:
+            tb = self.table[g0 * self.table_bytes:(g0 + H) * self.table_bytes]
+        t0 = ev() if timers is not None else None
+        if w.med3:
+            # Med3x and encode in one fused call (one read of x in chunk mode
+            # with search tables, two otherwise)
+            hqmq.hqmq_encode_med3(x, w.C, self.gran, cb, w.S, tb, self.words[l, r],
+                                  self.radius[l, r], self.rmed[l, r], self.thr[l, r],
+                                  self.out_idx[l, r], self.out_val[l, r],
+                                  self.slab_off[l, r], self.cap, self.ws, self.status,
+                                  stream, tile_off=self.tile_off[l, r])
+        elif self.table is not None:
+            hqmq.hqmq_encode_lut(x, cb, w.S, tb, None, self.gran, self.words[l, r],
+                                 self.radius[l, r], self.status, stream)
+        else:
+            hqmq.hqmq_encode(x, cb, w.S, None, self.gran, self.words[l, r],
+                             self.radius[l, r], self.status, stream)
+        t1 = ev() if timers is not None else None
+        if w.med3:
+            hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S,
+                             self.out_idx[l, r], self.out_val[l, r], self.slab_off[l, r],
+                             self.cap, self.gran, self.y, self.status, stream,
+                             tile_off=self.tile_off[l, r])
+        else:
+            hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S, None, None,
+                             None, 0, self.gran, self.y, self.status, stream)
+        if timers is not None:
+            t2 = ev()
+            timers["med3_encode" if w.med3 else "encode"].append((t0, t1))
+            timers["decode"].append((t1, t2))
 
 
-# DRAM bytes (read + write) of one one-read hqmq_encode_med3 call, from one ncu
-# capture of its four kernels (k_sample_window, k_encode_lut, k_finalize,
-# k_list_fix) on a call of this shape; valid while those kernels are unchanged.
-MED3_CALL_TRAFFIC = {((1, 8, 131072, 128), 32): 461744128 + 68536064}
+# DRAM bytes (read + write) of one hqmq_encode_med3 call of the 70B 128k call
+# shape, from an ncu capture of its kernels, kept with the SHA-256 of the
+# kernel sources it was taken on (profiles/traffic_encode_med3_call_llama3_70b_128k.md);
+# a capture taken on other sources is reported as stale, not used.
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "traffic_encode_med3_call_llama3_70b_128k.md")
+TRAFFIC_SHAPE = ((1, 8, 131072, 128), 32)
+
+
+def kernel_sources_sha256():
+    """SHA-256 over the CUDA sources of the library (file name and contents,
+    in name order)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kv_cache_quantization_hqmq_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def captured_traffic():
+    """(bytes per call, note) from the traffic profile, or (None, why)."""
+    try:
+        text = open(TRAFFIC_PROFILE).read()
+    except OSError:
+        return None, "no traffic capture"
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith(("traffic_bytes_per_call", "kernel_sources_sha256")):
+            k, v = line.strip().strip("`").split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if "traffic_bytes_per_call" not in vals:
+        return None, "no traffic figure in the capture summary"
+    if vals.get("kernel_sources_sha256") != kernel_sources_sha256():
+        return None, "stale: the kernel sources changed since the ncu capture"
+    return int(vals["traffic_bytes_per_call"]), "ncu dram__bytes_read.sum + dram__bytes_write.sum of the call's kernels (profiles/)"
 
 
 def one_read(w, table):
@@ -289,11 +328,14 @@ def algorithmic_bytes(w, n_outliers_per_call, table=True):
     code_bytes = n_chunks * (b / 8.0 + 2.0)
     out_bytes = n_outliers_per_call * 12.0 if w.med3 else 0.0
     return {
-        # chunk mode with tables: x is read once (the encode runs before the
-        # median is known and only possible outliers are revisited); element
-        # mode zeroes elements before encoding, so x is read once for the
-        # median and once more for the list and the encode
-        "med3_encode": (1 if one_read(w, table) else 2) * x_bytes + code_bytes + out_bytes,
+        # the scope's definition: with Med3x, x is read twice (the exact
+        # median precedes classification), then the codes and the list
+        "med3_encode": 2 * x_bytes + code_bytes + out_bytes,
+        # what this implementation must move: in chunk mode with tables x is
+        # read once (the encode runs before the median is known and only
+        # possible outliers are revisited); element mode zeroes elements
+        # before encoding and reads x twice
+        "med3_encode_one_read": (1 if one_read(w, table) else 2) * x_bytes + code_bytes + out_bytes,
         "encode": x_bytes + code_bytes,
         "decode": code_bytes + out_bytes + B * H * T * D * 2,
     }
@@ -325,6 +367,10 @@ def kernel_stats(w, timers, peaks, n_out, table):
                       "algorithmic_bytes_per_call": int(ab[name]),
                       "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
                       "bf16_gbs": round(w.call_elems * w.elem_bytes / (t * 1e-3) / 1e9, 1)}
+        if name == "med3_encode":
+            g1 = ab["med3_encode_one_read"] / (t * 1e-3) / 1e9
+            kern[name]["one_read_bytes_per_call"] = int(ab["med3_encode_one_read"])
+            kern[name]["one_read_hbm_frac"] = round(g1 / peaks["hbm_gbs"], 4)
     return kern
 
 
@@ -719,18 +765,19 @@ def run_hqmq(args):
         if not w.med3:
             name = "k_encode_lut"
         elif one_read(w, cache.table is not None):
-            name = ("hqmq_encode_med3 (one read of x: k_sample_window, k_encode_lut speculative "
+            name = ("hqmq_encode_med3 (one read of x: k_sample_window, k_encode_spec speculative "
                     "encode, k_finalize, k_list_fix)")
         else:
             name = "hqmq_encode_med3 (two reads of x: k_sample_window, k_pass_b, k_finalize, k_encode_lut)"
         roof = {"kernel": name, "bound": "hbm", "achieved": kern[enc_key]["hbm_gbs"],
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kern[enc_key]["hbm_frac"],
-                "traffic": MED3_CALL_TRAFFIC.get((w.call_shape, w.S)) if w.med3 and one_read(
-                    w, cache.table is not None) else None,
-                "peak_source": peaks["source"]}
-        if roof["traffic"] is not None:
-            roof["traffic_source"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4 "
-                                      "kernels of one call of this shape (profiles/)")
+                "traffic": None, "peak_source": peaks["source"]}
+        if w.med3:
+            roof["algorithmic_bytes"] = ("x read twice (the exact median precedes classification) + "
+                                         "codes + 12 B per outlier, per call")
+            roof["frac_one_read"] = kern[enc_key]["one_read_hbm_frac"]
+            if (w.call_shape, w.S) == TRAFFIC_SHAPE and one_read(w, cache.table is not None):
+                roof["traffic"], roof["traffic_source"] = captured_traffic()
 
     cache_bytes = w.cache_bytes
     value = world * cache_bytes / (ms_step * 1e-3) / 1e9
@@ -757,6 +804,10 @@ def run_hqmq(args):
                    "value_is": "bf16 KV bytes through Med3x+encode+decode per second"},
         "kernels": kern,
         "encoder": "search table (exact)" if cache.table is not None else "S-codeword loop",
+        "search_tables": None if cache.table is None else {
+            "bytes_per_group": cache.table_bytes, "groups": w.n_groups,
+            "bytes_per_call": cache.table_bytes * H, "total_bytes": cache.table_bytes * w.n_groups,
+            "vs_cache_bytes": round(cache.table_bytes * w.n_groups / cache_bytes, 4)},
         "setup_ms": round(setup_ms, 3),
         "roofline": roof,
         "bits_per_element": {"ours_codes": bits, "ours_outliers": round(out_bits, 4),
@@ -790,9 +841,13 @@ def run_hqmq(args):
 def run_e2e(cache, args, dist, device):
     """Same step through the C ABI with the input in pinned host memory: every
     call's input is copied H2D, and the compressed cache (index words, radii,
-    outlier list) D2H, inside the timed region."""
+    the outlier list with its offsets) D2H, inside the timed region.
+    Three streams: input copies (two device input buffers, so the copy of
+    call i + 1 runs while call i is coded), the coding calls, and output
+    copies.  The outlier lists are copied at their exact size: after the
+    step's calls one D2H read of every call's list count, then one copy per
+    call."""
     import torch
-    from kv_cache_quantization_hqmq_b200 import hqmq
     w = cache.w
     call_bytes = w.call_elems * w.elem_bytes
     try:
@@ -807,58 +862,85 @@ def run_e2e(cache, args, dist, device):
         hx.copy_(cache.x[i // 2 % w.layers, i % 2])
     host_words = torch.empty(cache.n_words, dtype=torch.int32, pin_memory=True)
     host_rad = torch.empty(cache.n_chunks, dtype=torch.int16, pin_memory=True)
-    host_oi = host_ov = None
     if w.med3:
         host_oi = torch.empty(cache.cap, dtype=torch.int32, pin_memory=True)
         host_ov = torch.empty(cache.cap * 4, dtype=torch.int16, pin_memory=True)
-        host_off = torch.empty(cache.slab_off.shape[-1] + cache.tile_off.shape[-1],
-                               dtype=torch.int32, pin_memory=True)
-    xbuf = torch.empty(cache.shape, dtype=w.torch_dtype, device=device)
-    h2d = d2h = 0
-
-    def x_of(l, r):
-        nonlocal h2d
-        xbuf.copy_(host_x[(l * 2 + r) % n_host], non_blocking=True)
-        h2d += call_bytes
-        return xbuf
+        ns, nt = cache.slab_off.shape[-1], cache.tile_off.shape[-1]
+        host_off = torch.empty(ns + nt, dtype=torch.int32, pin_memory=True)
+        host_counts = torch.empty(w.n_calls, dtype=torch.int32, pin_memory=True)
+    xbuf = [torch.empty(cache.shape, dtype=w.torch_dtype, device=device) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    s_run = torch.cuda.current_stream()
+    moved = {"h2d": 0, "d2h": 0}
 
     def one_step():
-        nonlocal d2h
-        cache.step(x_override=x_of)
-        # compressed cache back to the host (per call, last call's buffers
-        # stand for all: same sizes)
-        for l in range(w.layers):
-            for r in range(2):
+        done = [None, None]              # per input buffer: its last call finished
+        for i in range(w.n_calls):
+            l, r = i // 2, i % 2
+            k = i % 2
+            if done[k] is not None:
+                s_in.wait_event(done[k])
+            with torch.cuda.stream(s_in):
+                xbuf[k].copy_(host_x[i % n_host], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+            moved["h2d"] += call_bytes
+            s_run.wait_event(ready)
+            cache.call(l, r, xbuf[k], s_run)
+            fin = torch.cuda.Event()
+            fin.record(s_run)
+            done[k] = fin
+            # the call's codes back to the host (one output buffer reused: the
+            # copies are ordered on their stream)
+            s_out.wait_event(fin)
+            with torch.cuda.stream(s_out):
                 host_words.copy_(cache.words[l, r], non_blocking=True)
                 host_rad.copy_(cache.radius[l, r], non_blocking=True)
-                d2h += cache.n_words * 4 + cache.n_chunks * 2
                 if w.med3:
-                    host_oi.copy_(cache.out_idx[l, r], non_blocking=True)
-                    host_ov.copy_(cache.out_val[l, r], non_blocking=True)
-                    ns, nt = cache.slab_off.shape[-1], cache.tile_off.shape[-1]
                     host_off[:ns].copy_(cache.slab_off[l, r], non_blocking=True)
                     host_off[ns:].copy_(cache.tile_off[l, r], non_blocking=True)
-                    d2h += cache.cap * 4 + cache.cap * 8 + (ns + nt) * 4
+            moved["d2h"] += cache.n_words * 4 + cache.n_chunks * 2
+            if w.med3:
+                moved["d2h"] += (ns + nt) * 4
+        if w.med3:
+            # exact outlier lists: every call's count, then that many entries
+            with torch.cuda.stream(s_out):
+                s_out.wait_stream(s_run)
+                host_counts.copy_(cache.slab_off[:, :, -1].reshape(-1), non_blocking=True)
+            s_out.synchronize()
+            moved["d2h"] += w.n_calls * 4
+            for i, n in enumerate(host_counts.tolist()):
+                n = max(0, min(int(n), cache.cap))
+                l, r = i // 2, i % 2
+                with torch.cuda.stream(s_out):
+                    host_oi[:n].copy_(cache.out_idx[l, r, :n], non_blocking=True)
+                    host_ov[:4 * n].copy_(cache.out_val[l, r, :4 * n], non_blocking=True)
+                moved["d2h"] += n * 12
+        s_run.wait_stream(s_out)
+        s_run.wait_stream(s_in)
 
     steps = max(1, min(args.steps, 3))
     one_step()
     torch.cuda.synchronize()
-    h2d = d2h = 0
+    moved["h2d"] = moved["d2h"] = 0
     barrier(dist)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
+    t0.record(s_run)
+    s_in.wait_stream(s_run)
     for _ in range(steps):
         one_step()
-    t1.record()
+    t1.record(s_run)
     torch.cuda.synchronize()
     barrier(dist)
     ms = max_over_ranks(t0.elapsed_time(t1), dist, device) / steps
     world = 1 if dist is None else dist.get_world_size()
     return {"value": round(world * w.cache_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 2), "steps": steps,
-            "h2d_bytes_per_step": h2d // steps, "d2h_bytes_per_step": d2h // steps,
-            "host_inputs": "%d distinct pinned call inputs reused round-robin" % n_host}
+            "h2d_bytes_per_step": moved["h2d"] // steps, "d2h_bytes_per_step": moved["d2h"] // steps,
+            "host_inputs": "%d distinct pinned call inputs reused round-robin" % n_host,
+            "streams": "input copies, coding calls and output copies on three streams "
+                       "(two device input buffers); outlier lists copied at their exact size"}
 
 
 # ---------------------------------------------------------------- CPU oracle

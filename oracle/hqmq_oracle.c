@@ -752,3 +752,145 @@ void oracle_decode_qradius(const uint32_t *words, const uint32_t *rcode_words, c
     if (st && n_bad) { st->flags |= OR_FLAG_BAD_INDEX; }
     free(acc);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Joint (index, radius level) code: the pages' bit budget [ABS], [FR]      */
+/* "La mecanique" (3.79 bits per element at S = 8: log2(192^2) bits per    */
+/* chunk of 4 elements) reached by coding each chunk's pair as one digit   */
+/* D = idx * L + k in base L^2 (L = 24 S) and n consecutive chunks of a     */
+/* slab as one number V = sum_c D_c (L^2)^c (least significant chunk       */
+/* first), n the largest count with L^(2n) < 2^64; V takes w = bit length  */
+/* of L^(2n) - 1 bits.  Each slab's blocks (its last one padded with zero   */
+/* digits) are packed LSB-first into its own run of 32-bit words.           */
+/* ------------------------------------------------------------------------ */
+
+uint32_t oracle_joint_block_chunks(uint32_t S)
+{
+    uint64_t m = (uint64_t)(24u * S) * (uint64_t)(24u * S);   /* L^2 */
+    uint64_t p = 1;
+    uint32_t n = 0;
+    while (p <= UINT64_MAX / m) { p *= m; ++n; }                /* p = L^(2n) fits */
+    return n;
+}
+
+uint32_t oracle_joint_block_bits(uint32_t S)
+{
+    uint64_t m = (uint64_t)(24u * S) * (uint64_t)(24u * S);
+    uint32_t n = oracle_joint_block_chunks(S);
+    uint64_t top = 1;
+    for (uint32_t i = 0; i < n; ++i) top *= m;                  /* L^(2n) */
+    top -= 1u;                                                  /* largest V */
+    uint32_t w = 0;
+    while (w < 64 && (top >> w) != 0) ++w;
+    return w;
+}
+
+/* words of one slab's run */
+uint64_t oracle_joint_slab_words(int T, int D, uint32_t S)
+{
+    uint64_t cps = (uint64_t)T * D / 4;
+    uint32_t n = oracle_joint_block_chunks(S), w = oracle_joint_block_bits(S);
+    uint64_t nb = (cps + n - 1) / n;
+    return (nb * w + 31) / 32;
+}
+
+/* bit i of a word run */
+static void put_bits(uint32_t *run, uint64_t bit0, uint32_t w, uint64_t v)
+{
+    for (uint32_t i = 0; i < w; ++i)
+        if ((v >> i) & 1u) run[(bit0 + i) / 32] |= 1u << ((bit0 + i) % 32);
+}
+
+static uint64_t get_bits(const uint32_t *run, uint64_t bit0, uint32_t w)
+{
+    uint64_t v = 0;
+    for (uint32_t i = 0; i < w; ++i)
+        v |= (uint64_t)((run[(bit0 + i) / 32] >> ((bit0 + i) % 32)) & 1u) << i;
+    return v;
+}
+
+/* Joint code of a call from its index words and radius-code words (both
+ * laid out as b-bit fields in groups of 32 chunks).  joint: B*H runs of
+ * oracle_joint_slab_words(T, D, S) words, zeroed here.  Returns the number
+ * of chunks whose index or level is not below L (stored as digit 0). */
+uint64_t oracle_pack_joint(const uint32_t *words, const uint32_t *rcode_words, int B, int H, int T,
+                           int D, uint32_t S, uint32_t *joint)
+{
+    uint32_t b = oracle_index_bits(S), L = 24u * S;
+    uint64_t m = (uint64_t)L * L;
+    uint32_t n = oracle_joint_block_chunks(S), w = oracle_joint_block_bits(S);
+    uint64_t cps = (uint64_t)T * D / 4, wps = oracle_joint_slab_words(T, D, S);
+    uint64_t nb = (cps + n - 1) / n, bad = 0;
+    memset(joint, 0, (size_t)B * H * wps * sizeof(uint32_t));
+    for (uint64_t s = 0; s < (uint64_t)B * H; ++s) {
+        for (uint64_t q = 0; q < nb; ++q) {
+            uint64_t v = 0, p = 1;
+            for (uint32_t c = 0; c < n; ++c) {
+                uint64_t j = q * n + c;
+                uint64_t d = 0;
+                if (j < cps) {
+                    uint32_t idx = oracle_get_index(words, b, s * cps + j);
+                    uint32_t k = oracle_get_index(rcode_words, b, s * cps + j);
+                    if (idx < L && k < L) d = (uint64_t)idx * L + k;
+                    else ++bad;
+                }
+                v += d * p;
+                p *= m;                        /* (the last product may wrap: unused) */
+            }
+            put_bits(joint + s * wps, q * w, w, v);
+        }
+    }
+    return bad;
+}
+
+/* The (index, level) pair of every chunk of a call from its joint code. */
+void oracle_unpack_joint(const uint32_t *joint, int B, int H, int T, int D, uint32_t S,
+                         uint32_t *idx, uint32_t *k)
+{
+    uint32_t L = 24u * S;
+    uint64_t m = (uint64_t)L * L;
+    uint32_t n = oracle_joint_block_chunks(S), w = oracle_joint_block_bits(S);
+    uint64_t cps = (uint64_t)T * D / 4, wps = oracle_joint_slab_words(T, D, S);
+    uint64_t nb = (cps + n - 1) / n;
+    for (uint64_t s = 0; s < (uint64_t)B * H; ++s) {
+        for (uint64_t q = 0; q < nb; ++q) {
+            uint64_t v = get_bits(joint + s * wps, q * w, w);
+            for (uint32_t c = 0; c < n; ++c) {
+                uint64_t j = q * n + c;
+                uint64_t d = v % m;
+                v /= m;
+                if (j < cps) {
+                    idx[s * cps + j] = (uint32_t)(d / L);
+                    k[s * cps + j] = (uint32_t)(d % L);
+                }
+            }
+        }
+    }
+}
+
+/* The pages' outlier flag [NL 3] ("met een 1-bit vlag"): bit c of word g is
+ * set when chunk 32 g + c is in the (chunk-mode) outlier list.  flags:
+ * n_chunks / 32 words, zeroed here. */
+void oracle_list_flags(const uint32_t *out_idx, int64_t n_out, uint64_t n_chunks, uint32_t *flags)
+{
+    memset(flags, 0, (size_t)(n_chunks / 32) * sizeof(uint32_t));
+    for (int64_t q = 0; q < n_out; ++q) {
+        uint64_t j = out_idx[q];
+        if (j < n_chunks) flags[j / 32] |= 1u << (j % 32);
+    }
+}
+
+/* The chunk-mode outlier list (chunk indices, in order) read back from the
+ * flags: the values stay in the list's order, so entry q of the list is the
+ * q-th set flag.  Returns the number of set flags (written up to cap). */
+int64_t oracle_list_from_flags(const uint32_t *flags, uint64_t n_chunks, uint32_t *out_idx,
+                               int64_t cap)
+{
+    int64_t n = 0;
+    for (uint64_t j = 0; j < n_chunks; ++j)
+        if ((flags[j / 32] >> (j % 32)) & 1u) {
+            if (n < cap) out_idx[n] = (uint32_t)j;
+            ++n;
+        }
+    return n;
+}

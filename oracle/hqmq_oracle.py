@@ -93,6 +93,13 @@ _SIGS = {
     "oracle_quantize_radius": (None, [_P, _P, _I, _I, _I, _I, _U32, _P]),
     "oracle_decode_qradius": (None, [_P, _P, _P, _P, _U32, _P, _P, _I64, _I, _I, _I, _I, _I, _P,
                                      _I, _P]),
+    "oracle_joint_block_chunks": (_U32, [_U32]),
+    "oracle_joint_block_bits": (_U32, [_U32]),
+    "oracle_joint_slab_words": (_U64, [_I, _I, _U32]),
+    "oracle_pack_joint": (_U64, [_P, _P, _I, _I, _I, _I, _U32, _P]),
+    "oracle_unpack_joint": (None, [_P, _I, _I, _I, _I, _U32, _P, _P]),
+    "oracle_list_flags": (None, [_P, _I64, _U64, _P]),
+    "oracle_list_from_flags": (_I64, [_P, _U64, _P, _I64]),
 }
 
 
@@ -394,3 +401,54 @@ def attention_decode(q_bits, k_hat, v_hat, scale, G, seq_len=None):
             w = np.exp(s - s.max())
             o[b, h] = (w @ V) / w.sum()
     return o
+
+
+def joint_block_chunks(S):
+    """Chunks per block of the joint (index, radius level) code."""
+    return int(lib().oracle_joint_block_chunks(int(S)))
+
+
+def joint_block_bits(S):
+    """Bits per block of the joint code."""
+    return int(lib().oracle_joint_block_bits(int(S)))
+
+
+def joint_words(B, H, T, D, S):
+    return B * H * int(lib().oracle_joint_slab_words(T, D, int(S)))
+
+
+def pack_joint(words, rcode_words, B, H, T, D, S):
+    """Joint code of a call from its index and radius-code words: (uint32
+    words of the B*H slab runs, number of chunks stored as digit 0 because
+    their index or level was out of range)."""
+    words = _c(words, np.uint32)
+    rw = _c(rcode_words, np.uint32)
+    out = np.zeros(joint_words(B, H, T, D, S), np.uint32)
+    bad = lib().oracle_pack_joint(_ptr(words), _ptr(rw), B, H, T, D, int(S), _ptr(out))
+    return out, int(bad)
+
+
+def unpack_joint(joint, B, H, T, D, S):
+    """(index, level) of every chunk of a call from its joint code."""
+    joint = _c(joint, np.uint32)
+    n = B * H * T * D // 4
+    idx = np.zeros(n, np.uint32)
+    k = np.zeros(n, np.uint32)
+    lib().oracle_unpack_joint(_ptr(joint), B, H, T, D, int(S), _ptr(idx), _ptr(k))
+    return idx, k
+
+
+def list_flags(out_idx, n_chunks):
+    """Per packing group of 32 chunks, the flag word of its listed outliers."""
+    oi = _c(out_idx, np.uint32)
+    flags = np.zeros(n_chunks // 32, np.uint32)
+    lib().oracle_list_flags(_ptr(oi), oi.size, int(n_chunks), _ptr(flags))
+    return flags
+
+
+def list_from_flags(flags, n_chunks, cap=None):
+    flags = _c(flags, np.uint32)
+    cap = int(n_chunks) if cap is None else int(cap)
+    out = np.zeros(max(cap, 1), np.uint32)
+    n = lib().oracle_list_from_flags(_ptr(flags), int(n_chunks), _ptr(out), cap)
+    return out[:min(n, cap)], int(n)

@@ -77,6 +77,15 @@ MUTATIONS = [
      "load_chunk(x, dtype, j, NULL, gran, c);\n        float r, bs, sc;\n"
      "        uint32_t idx = search_chunk(c, table, S",
      ["test_encode_chunks_equals_the_whole_call_encode"]),
+    # the joint (index, radius level) code and the outlier flags
+    ("joint_most_significant_first", "                v += d * p;\n", "                v = v * m + d;\n",
+     ["test_pack_equals_the_big_integer_definition"], "tests/test_oracle_joint.py"),
+    ("joint_base_L", "uint64_t m = (uint64_t)(24u * S) * (uint64_t)(24u * S);   /* L^2 */",
+     "uint64_t m = (uint64_t)(24u * S);   /* L^2 */",
+     ["test_block_size_is_the_largest_that_fits_64_bits"], "tests/test_oracle_joint.py"),
+    ("flags_msb_first", "if (j < n_chunks) flags[j / 32] |= 1u << (j % 32);",
+     "if (j < n_chunks) flags[j / 32] |= 1u << (31 - j % 32);",
+     ["test_flags_are_the_list_as_a_bitmap"], "tests/test_oracle_joint.py"),
     ("qradius_rounds_down", "float t = q + 0.5f;", "float t = q;",
      ["test_level_is_the_nearest_grid_point"], "tests/test_oracle_qradius.py"),
     ("qradius_levels_pow2", "uint32_t b = oracle_index_bits(S), L = 24u * S;\n    float *acc",
