@@ -515,7 +515,33 @@ def run_qradius(cache, peaks, iters=20, warmup=3):
         a_bytes = 2 * B * H * T * (8 * b) + n_list * 12
         att = {"ms_per_call": round(ms_a, 4), "algorithmic_bytes": a_bytes,
                "hbm_frac": round(a_bytes / (ms_a * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    # the joint (index, level) block code and the 1-bit outlier flags
+    joint = hqmq.alloc_joint(B, H, T, D, w.S, device=dev)
+    flags = torch.empty(n_chunks // 32, dtype=torch.int32, device=dev)
+    yj = torch.empty(cache.shape, dtype=torch.bfloat16, device=dev)
+    ms_p = timed(lambda: hqmq.hqmq_pack_joint(cache.words[0, 0], rw, w.S, cache.shape, joint))
+    ms_f = timed(lambda: hqmq.hqmq_list_flags(cache.out_idx[0, 0], cache.slab_off[0, 0], cache.cap,
+                                              cache.shape, flags))
+    ms_j = timed(lambda: hqmq.hqmq_decode_joint(joint, cache.thr[0, 0], cb, w.S, flags,
+                                                cache.out_val[0, 0], cache.tile_off[0, 0],
+                                                cache.cap, yj))
+    hqmq.hqmq_decode_qradius(*args, yq, st)
+    torch.cuda.synchronize()
+    nblk, wbits = hqmq.hqmq_joint_block(w.S)
+    n_el = B * H * T * D
+    tiles = hqmq.hqmq_list_tiles(B, H, T, D)
+    jb = {"codes": joint.numel() * 32 / n_el, "flags": n_chunks / n_el,
+          "tile_offsets": (tiles + 1) * 32 / n_el, "values": n_out * 64 / n_el}
+    jd_bytes = joint.numel() * 4 + n_chunks // 8 + n_out * 8 + n_el * 2
+    joint_obj = {
+        "chunks_per_block": nblk, "bits_per_block": wbits,
+        "bits_per_element": {k: round(v, 4) for k, v in jb.items()},
+        "bits_per_element_total": round(sum(jb.values()), 4),
+        "pack_ms": round(ms_p, 4), "flags_ms": round(ms_f, 4), "decode_ms": round(ms_j, 4),
+        "decode_hbm_frac": round(jd_bytes / (ms_j * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "decode_equals_qradius_decode": bool(torch.equal(yj.view(torch.int16), yq.view(torch.int16)))}
     return {"op": "hqmq_quantize_radius + hqmq_decode_qradius (layer 0, K)",
+            "joint_code_with_flags": joint_obj,
             "attention_from_quantized_codes": att,
             "levels": 24 * w.S, "code_bits_per_chunk": 2 * b,
             "bits_per_element": round(2 * b / 4 + n_out * 96 / (B * H * T * D), 4),

@@ -23,7 +23,9 @@
  *   - decode-phase attention straight from the codes (that same section:
  *     the decoder runs inside attention), hqmq_attention_decode;
  *   - an optional b-bit radius code matching the pages' bit budget
- *     (hqmq_quantize_radius, hqmq_decode_qradius);
+ *     (hqmq_quantize_radius, hqmq_decode_qradius), the joint (index, level)
+ *     block code and the 1-bit outlier flags (hqmq_pack_joint,
+ *     hqmq_list_flags, hqmq_decode_joint);
  *   - Med3x under a given threshold for decode-step tokens, and all of a
  *     step's small calls in one launch (hqmq_outlier_extract_given_thr,
  *     hqmq_append_batch).
@@ -383,6 +385,48 @@ HQMQ_API int hqmq_decode_qradius(const uint32_t *d_idx_words, const uint32_t *d_
                                  const uint32_t *d_tile_off, uint64_t cap, int gran, int B, int H,
                                  int T, int D, void *d_y, int out_dtype, hqmq_status *d_status,
                                  void *stream);
+
+/* Joint (index, radius level) code: the pages' bit budget (signal-ia-rouge,
+ * "La mecanique": 3.79 bits per element at S = 8, about 5 at S = 32, i.e. two
+ * digits of L = 24 S values per chunk of four elements).  Each chunk's pair
+ * is one digit D = idx * L + k in base L^2 (k its radius level, as written by
+ * hqmq_quantize_radius); n consecutive chunks of a slab form one block value
+ * V = sum_c D_c (L^2)^c (least significant chunk first), n the largest count
+ * with L^(2n) < 2^64, stored in w = bit length of L^(2n) - 1 bits.  Every
+ * slab's blocks (its last one padded with zero digits) are packed LSB-first
+ * into its own run of uint32 words.  S = 8: n = 4, w = 61 (3.8125 bits per
+ * element); S = 32: n = 3, w = 58 (4.833).  Valid for S in [1, 2730]
+ * (L^2 < 2^32); other S give 0 / HQMQ_ERR_ARG.  No counterpart format is
+ * given on the pages: the block code is this library's. */
+HQMQ_API void hqmq_joint_block(uint32_t S, uint32_t *chunks_per_block, uint32_t *bits_per_block);
+/* uint32 words of a call's joint code (B*H runs); 0 for a bad shape or S. */
+HQMQ_API uint64_t hqmq_joint_words(int B, int H, int T, int D, uint32_t S);
+/* Joint code of a call from its index words and radius-code words (both
+ * uint32[hqmq_index_words(B,H,T,D,S)], 4-byte aligned).  d_joint:
+ * uint32[hqmq_joint_words(...)], fully overwritten.  A chunk whose index or
+ * level is not below L is stored as digit 0 and raises HQMQ_FLAG_BAD_INDEX
+ * in d_status (optional). */
+HQMQ_API int hqmq_pack_joint(const uint32_t *d_idx_words, const uint32_t *d_rcode_words,
+                             uint32_t S, int B, int H, int T, int D, uint32_t *d_joint,
+                             hqmq_status *d_status, void *stream);
+/* The pages' 1-bit outlier flag (gist.science/nl, Technische Samenvatting,
+ * section 3): d_flags uint32[B*H*T*D/128], bit c of word g set when chunk
+ * 32 g + c is in the chunk-mode outlier list (d_out_idx, its first
+ * min(d_slab_off[B*H], cap) entries).  With the list's values (d_out_val, in
+ * list order) and tile offsets, the flags replace the list's 32-bit indices:
+ * a flagged chunk's values are the q-th of its 1024-chunk list tile, q its
+ * rank among the tile's flags.  d_flags is fully overwritten. */
+HQMQ_API int hqmq_list_flags(const uint32_t *d_out_idx, const uint32_t *d_slab_off, uint64_t cap,
+                             int B, int H, int T, int D, uint32_t *d_flags, void *stream);
+/* Decode from the joint code: r = fl32(k fl32(thr_h / (L-1))) times the
+ * codeword of idx, rounded to out_dtype, exactly as hqmq_decode_qradius;
+ * then, if d_flags is given, every flagged chunk becomes its fp16 values
+ * (d_out_val in list order, d_tile_off the list's tile offsets, entries at
+ * or past cap skipped).  d_y 8-byte (bf16) or 16-byte (fp32) aligned. */
+HQMQ_API int hqmq_decode_joint(const uint32_t *d_joint, const float *d_thr,
+                               const float *d_codebook, uint32_t S, const uint32_t *d_flags,
+                               const uint16_t *d_out_val, const uint32_t *d_tile_off, uint64_t cap,
+                               int B, int H, int T, int D, void *d_y, int out_dtype, void *stream);
 
 /* One coded K or V cache for hqmq_attention_decode: HOST struct of DEVICE
  * pointers, each as written by hqmq_encode / hqmq_encode_med3 for a

@@ -80,6 +80,19 @@ extern "C" int hqmq_launch_outlier_extract_thr(const void *x, int dtype, int B, 
 extern "C" int hqmq_launch_quantize_radius(const uint16_t *radius, const float *thr, int B, int H,
                                            int T, int D, uint32_t S, uint32_t b, uint32_t *rwords,
                                            int sm_count, cudaStream_t stream);
+extern "C" uint64_t hqmq_launch_joint_words(int B, int H, int T, int D, uint32_t S);
+extern "C" void hqmq_launch_joint_block(uint32_t S, uint32_t *n, uint32_t *w);
+extern "C" int hqmq_launch_pack_joint(const uint32_t *iw, const uint32_t *kw, uint32_t S, int B,
+                                      int H, int T, int D, uint32_t *joint, hqmq_status *st,
+                                      int sm_count, cudaStream_t stream);
+extern "C" int hqmq_launch_list_flags(const uint32_t *out_idx, const uint32_t *total,
+                                      uint64_t cap, uint64_t n_chunks, uint32_t *flags,
+                                      int sm_count, cudaStream_t stream);
+extern "C" int hqmq_launch_decode_joint(const uint32_t *joint, const float *thr, const float *cb,
+                                        uint32_t S, const uint32_t *flags, const uint16_t *out_val,
+                                        const uint32_t *tile_off, uint64_t cap, int B, int H,
+                                        int T, int D, void *y, int out_dtype, int sm_count,
+                                        cudaStream_t stream);
 extern "C" int hqmq_launch_decode_qr(const uint32_t *words, const uint32_t *rwords, const float *thr,
                                      const float *cb, uint32_t S, uint32_t b,
                                      const uint32_t *out_idx, const uint16_t *out_val,
@@ -102,6 +115,7 @@ extern "C" int hqmq_launch_encode_lut(const void *x, int dtype, int B, int H, in
 namespace {
 
 constexpr uint32_t S_MAX = 65535;
+constexpr uint32_t JOINT_MAX_S = 2730;        // joint code: L^2 = (24 S)^2 < 2^32
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -429,6 +443,63 @@ int hqmq_decode_qradius(const uint32_t *d_idx_words, const uint32_t *d_rcode_wor
                                  hqmq_index_bits(S), d_out_idx, d_out_val,
                                  d_out_idx ? d_tile_off : nullptr, cap, gran, B, H, T, D, d_y,
                                  out_dtype, d_status, sm, (cudaStream_t)stream);
+}
+
+static bool joint_S_ok(uint32_t S) { return S >= 1 && S <= JOINT_MAX_S; }
+
+void hqmq_joint_block(uint32_t S, uint32_t *chunks_per_block, uint32_t *bits_per_block) {
+    uint32_t n = 0, w = 0;
+    if (joint_S_ok(S)) hqmq_launch_joint_block(S, &n, &w);
+    if (chunks_per_block) *chunks_per_block = n;
+    if (bits_per_block) *bits_per_block = w;
+}
+
+uint64_t hqmq_joint_words(int B, int H, int T, int D, uint32_t S) {
+    if (!shape_ok(B, H, T, D) || !joint_S_ok(S)) return 0;
+    return hqmq_launch_joint_words(B, H, T, D, S);
+}
+
+int hqmq_pack_joint(const uint32_t *d_idx_words, const uint32_t *d_rcode_words, uint32_t S, int B,
+                    int H, int T, int D, uint32_t *d_joint, hqmq_status *d_status, void *stream) {
+    if (!shape_ok(B, H, T, D) || !joint_S_ok(S)) return HQMQ_ERR_ARG;
+    if (!d_idx_words || !d_rcode_words || !d_joint) return HQMQ_ERR_ARG;
+    if (!aligned(d_idx_words, 4) || !aligned(d_rcode_words, 4) || !aligned(d_joint, 4) ||
+        !aligned(d_status, 8))
+        return HQMQ_ERR_ALIGN;
+    const int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_pack_joint(d_idx_words, d_rcode_words, S, B, H, T, D, d_joint, d_status,
+                                  sm, (cudaStream_t)stream);
+}
+
+int hqmq_list_flags(const uint32_t *d_out_idx, const uint32_t *d_slab_off, uint64_t cap, int B,
+                    int H, int T, int D, uint32_t *d_flags, void *stream) {
+    if (!shape_ok(B, H, T, D)) return HQMQ_ERR_ARG;
+    if (!d_slab_off || !d_flags || (cap > 0 && !d_out_idx)) return HQMQ_ERR_ARG;
+    if (!aligned(d_out_idx, 4) || !aligned(d_slab_off, 4) || !aligned(d_flags, 4))
+        return HQMQ_ERR_ALIGN;
+    const int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    const uint64_t n_chunks = (uint64_t)B * H * T * D / 4;
+    return hqmq_launch_list_flags(d_out_idx, d_slab_off + (size_t)B * H, cap, n_chunks, d_flags,
+                                  sm, (cudaStream_t)stream);
+}
+
+int hqmq_decode_joint(const uint32_t *d_joint, const float *d_thr, const float *d_codebook,
+                      uint32_t S, const uint32_t *d_flags, const uint16_t *d_out_val,
+                      const uint32_t *d_tile_off, uint64_t cap, int B, int H, int T, int D,
+                      void *d_y, int out_dtype, void *stream) {
+    if (!shape_ok(B, H, T, D) || !dtype_ok(out_dtype) || !joint_S_ok(S)) return HQMQ_ERR_ARG;
+    if (!d_joint || !d_thr || !d_codebook || !d_y) return HQMQ_ERR_ARG;
+    if (d_flags && (!d_tile_off || (cap > 0 && !d_out_val))) return HQMQ_ERR_ARG;
+    if (!aligned(d_joint, 4) || !aligned(d_thr, 4) || !aligned(d_codebook, 16) ||
+        !aligned(d_y, out_dtype == HQMQ_BF16 ? 8 : 16) || !aligned(d_flags, 4) ||
+        !aligned(d_out_val, 4) || !aligned(d_tile_off, 4))
+        return HQMQ_ERR_ALIGN;
+    const int sm = sm_count();
+    if (sm <= 0) return HQMQ_ERR_CUDA;
+    return hqmq_launch_decode_joint(d_joint, d_thr, d_codebook, S, d_flags, d_out_val, d_tile_off,
+                                    cap, B, H, T, D, d_y, out_dtype, sm, (cudaStream_t)stream);
 }
 
 uint64_t hqmq_outlier_extract_given_thr_workspace_size(int B, int H, int T, int D) {

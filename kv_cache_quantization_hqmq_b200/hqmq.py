@@ -84,6 +84,11 @@ _SIGS = {
                                             _P, _U64, _P, _P]),
     "hqmq_decode_qradius": (_I, [_P, _P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _I, _P,
                                  _I, _P, _P]),
+    "hqmq_joint_block": (None, [_U32, _P, _P]),
+    "hqmq_joint_words": (_U64, [_I, _I, _I, _I, _U32]),
+    "hqmq_pack_joint": (_I, [_P, _P, _U32, _I, _I, _I, _I, _P, _P, _P]),
+    "hqmq_list_flags": (_I, [_P, _P, _U64, _I, _I, _I, _I, _P, _P]),
+    "hqmq_decode_joint": (_I, [_P, _P, _P, _U32, _P, _P, _P, _U64, _I, _I, _I, _I, _P, _I, _P]),
     "hqmq_attention_workspace_size": (_U64, [_I, _I]),
     "hqmq_attention_decode": (_I, [_P, _P, _P, _P, _U32, _I, _I, _I, _I, _I, _F, _P, _I, _P,
                                    _U64, _P, _P]),
@@ -282,6 +287,51 @@ def hqmq_decode_qradius(idx_words, rcode_words, thr, codebook, S, out_idx, out_v
         _ptr(idx_words), _ptr(rcode_words), _ptr(thr), _ptr(codebook), S, _ptr(out_idx),
         _ptr(out_val), _ptr(tile_off), int(cap), gran, B, H, T, D, _ptr(y), _dtype_code(y),
         _ptr(status), _stream(stream)))
+
+
+def hqmq_joint_block(S):
+    """(chunks per block, bits per block) of the joint (index, level) code."""
+    n, w = ctypes.c_uint32(0), ctypes.c_uint32(0)
+    _lib.hqmq_joint_block(S, ctypes.byref(n), ctypes.byref(w))
+    return n.value, w.value
+
+
+def hqmq_joint_words(B, H, T, D, S):
+    return int(_lib.hqmq_joint_words(B, H, T, D, S))
+
+
+def alloc_joint(B, H, T, D, S, device="cuda"):
+    n = hqmq_joint_words(B, H, T, D, S)
+    if n == 0:
+        raise ValueError("bad shape/S for the joint code")
+    return torch.empty(n, dtype=torch.int32, device=device)
+
+
+def hqmq_pack_joint(idx_words, rcode_words, S, shape, joint, status=None, stream=None):
+    """The joint code of a call (shape = (B, H, T, D)) from its index and
+    radius-code words."""
+    B, H, T, D = shape
+    _check("hqmq_pack_joint", _lib.hqmq_pack_joint(
+        _ptr(idx_words), _ptr(rcode_words), S, B, H, T, D, _ptr(joint), _ptr(status),
+        _stream(stream)))
+    return joint
+
+
+def hqmq_list_flags(out_idx, slab_off, cap, shape, flags, stream=None):
+    """The 1-bit outlier flags (uint32 [B*H*T*D/128]) of a chunk-mode list."""
+    B, H, T, D = shape
+    _check("hqmq_list_flags", _lib.hqmq_list_flags(
+        _ptr(out_idx), _ptr(slab_off), int(cap), B, H, T, D, _ptr(flags), _stream(stream)))
+    return flags
+
+
+def hqmq_decode_joint(joint, thr, codebook, S, flags, out_val, tile_off, cap, y, stream=None):
+    """Decode from the joint code; flags (with the list's values and tile
+    offsets) restore the chunk-mode outliers, or None."""
+    B, H, T, D = _shape4(y)
+    _check("hqmq_decode_joint", _lib.hqmq_decode_joint(
+        _ptr(joint), _ptr(thr), _ptr(codebook), S, _ptr(flags), _ptr(out_val), _ptr(tile_off),
+        int(cap), B, H, T, D, _ptr(y), _dtype_code(y), _stream(stream)))
 
 
 class KVCodes(ctypes.Structure):

@@ -138,3 +138,26 @@ def test_next_row_queries_and_argument_checks(lib):
                                  good, good, None, 1 << 33, None, None) == 1
     assert lib.hqmq_append_batch(good, 0, 0, 1, 8, 1, 128, good, 0, good, 32, good, good, good,
                                  good, good, None, 64, None, None) == 1
+
+
+def test_joint_code_queries_and_argument_errors(lib):
+    from kv_cache_quantization_hqmq_b200 import hqmq
+    assert hqmq.hqmq_joint_block(8) == (4, 61) and hqmq.hqmq_joint_block(32) == (3, 58)
+    assert hqmq.hqmq_joint_block(0) == (0, 0) and hqmq.hqmq_joint_block(2731) == (0, 0)
+    # 70B call at S = 32: 8 slabs, each ceil(4194304 / 3) blocks of 58 bits
+    nb = -(-4194304 // 3)
+    assert hqmq.hqmq_joint_words(1, 8, 131072, 128, 32) == 8 * ((nb * 58 + 31) // 32)
+    assert hqmq.hqmq_joint_words(1, 8, 131072, 128, 2731) == 0
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    # rejected before any CUDA call: bad S, missing pointers, misalignment
+    assert lib.hqmq_pack_joint(good, good, 0, 1, 1, 32, 128, good, None, None) == hqmq.HQMQ_ERR_ARG
+    assert lib.hqmq_pack_joint(None, good, 8, 1, 1, 32, 128, good, None, None) == hqmq.HQMQ_ERR_ARG
+    assert lib.hqmq_pack_joint(odd, good, 8, 1, 1, 32, 128, good, None, None) == hqmq.HQMQ_ERR_ALIGN
+    assert lib.hqmq_list_flags(good, None, 16, 1, 1, 32, 128, good, None) == hqmq.HQMQ_ERR_ARG
+    assert lib.hqmq_list_flags(odd, good, 16, 1, 1, 32, 128, good, None) == hqmq.HQMQ_ERR_ALIGN
+    y4 = ctypes.c_void_p((1 << 20) + 4)       # 4-byte aligned: not enough for bf16 chunks
+    assert lib.hqmq_decode_joint(good, good, good, 8, None, None, None, 0, 1, 1, 32, 128, y4, 0,
+                                 None) == hqmq.HQMQ_ERR_ALIGN
+    assert lib.hqmq_decode_joint(good, good, good, 8, good, None, None, 16, 1, 1, 32, 128, good, 0,
+                                 None) == hqmq.HQMQ_ERR_ARG      # flags without tile offsets
