@@ -300,9 +300,10 @@ def captured_traffic():
         return None, "no traffic capture"
     vals = {}
     for line in text.splitlines():
-        if ":" in line and line.strip().startswith(("traffic_bytes_per_call", "kernel_sources_sha256")):
-            k, v = line.strip().strip("`").split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
+        line = line.strip().lstrip("-* ").replace("`", "")
+        if ":" in line and line.startswith(("traffic_bytes_per_call", "kernel_sources_sha256")):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
     if "traffic_bytes_per_call" not in vals:
         return None, "no traffic figure in the capture summary"
     if vals.get("kernel_sources_sha256") != kernel_sources_sha256():
