@@ -43,6 +43,11 @@ extern "C" int hqmq_launch_med3_finish(const void *x, int dtype, int B, int H, i
                                        cudaStream_t stream, const uint32_t **tile_off,
                                        uint32_t *tiles_per_slab);
 extern "C" int hqmq_spec_encode_supported(uint32_t b);
+extern "C" int hqmq_launch_table_encode_units(const void *x, int dtype, int B, int H, int T, int D,
+                                              const float *cb, uint32_t S, uint32_t b,
+                                              const void *table, uint32_t *words,
+                                              uint16_t *radius, hqmq_status *st, int sm_count,
+                                              cudaStream_t stream);
 extern "C" int hqmq_launch_spec_encode_units(const void *x, int dtype, int B, int H, int T, int D,
                                              const float *cb, uint32_t S, uint32_t b,
                                              const void *table, uint32_t *words, uint16_t *radius,
@@ -379,9 +384,13 @@ int hqmq_encode_lut(const void *d_x, int dtype, int B, int H, int T, int D,
         return HQMQ_ERR_ALIGN;
     int sm = sm_count();
     if (sm <= 0) return HQMQ_ERR_CUDA;
-    return hqmq_launch_encode_lut(d_x, dtype, B, H, T, D, d_codebook, S, hqmq_index_bits(S),
-                                  d_table, d_thr, gran, d_idx_words, d_radius, d_status, sm,
-                                  (cudaStream_t)stream);
+    const uint32_t b = hqmq_index_bits(S);
+    if (!d_thr && hqmq_spec_encode_supported(b))
+        return hqmq_launch_table_encode_units(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table,
+                                              d_idx_words, d_radius, d_status, sm,
+                                              (cudaStream_t)stream);
+    return hqmq_launch_encode_lut(d_x, dtype, B, H, T, D, d_codebook, S, b, d_table, d_thr, gran,
+                                  d_idx_words, d_radius, d_status, sm, (cudaStream_t)stream);
 }
 
 uint64_t hqmq_attention_workspace_size(int B, int Hk) {

@@ -99,12 +99,14 @@ __device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
-template <int DT, int BB, int R>
+// SPEC = false: the plain table encode (no Med3x): no window bookkeeping, no
+// candidate bits or values, status counts straight to st.
+template <int DT, int BB, int R, bool SPEC>
 __global__ void __launch_bounds__(SPEC_THREADS, 1)
 k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t ups, uint32_t tps,
               uint32_t n_units, uint32_t round_units, const float4 *__restrict__ cb_all, uint32_t S,
               const uint4 *__restrict__ tables, uint32_t *__restrict__ words,
-              uint16_t *__restrict__ radius, SpecArgs sa) {
+              uint16_t *__restrict__ radius, SpecArgs sa, DevStatus *st) {
     constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;       // bytes per chunk
     constexpr int NS = RING_BYTES / (32 * CB);         // ring slots (packing groups)
     static_assert(NS >= 2 && UNIT_G % NS == 0, "a unit's groups fill whole ring rounds");
@@ -157,9 +159,10 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
             const uint32_t ub = seg + (uint32_t)((uint64_t)nseg * (warp + 1) / SPEC_WARPS);
             seg = seg_end;
             if (ua >= ub) continue;                          // (warp-uniform)
-            const WinState w = sa.win[h];
+            WinState w{};
+            if constexpr (SPEC) w = sa.win[h];
             const uint32_t span = w.hi_key - w.lo_key;
-            const int top = median_top_shift(span);
+            const int top = SPEC ? median_top_shift(span) : 0;
             const uint4 *tb = tables + (size_t)h * LUT_ENTRIES;
             const float4 *cb = cb_all + (size_t)h * S;
             // packing groups of the call (fewer than 2^27: 32-bit indices)
@@ -200,6 +203,8 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
                     // median window: key = r's bits (r >= 0; a NaN's bits exceed
                     // every finite key and +inf's, as in the median's order)
                     const uint32_t key = __float_as_uint(r);
+                    bool cnd = false;
+                    if constexpr (SPEC) {
                     n_below += key < w.lo_key ? 1u : 0u;
                     const bool in = key - w.lo_key < span;   // lo_key <= key < hi_key
                     const uint32_t mi = __ballot_sync(FULL, in);
@@ -216,7 +221,7 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
                     }
                     // threshold band: above t_hi always an outlier, above t_lo possibly
                     const bool dfn = r > w.t_hi;             // (NaN: false)
-                    const bool cnd = r > w.t_lo;
+                    cnd = r > w.t_lo;
                     n_def += dfn ? 1u : 0u;
                     const uint32_t mc = __ballot_sync(FULL, cnd);
                     if (lane == 0) sts_u32(a_cb + k * 4u, mc);
@@ -237,6 +242,7 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
                         }
                     }
                     if (dfn) r = 0.0f;                       // certain outlier: radius 0, index 0
+                    }
                     // search every lane (branch-free); a lane whose chunk is zero,
                     // non-finite or a certain outlier reads some in-range record and
                     // keeps index 0.  r in (0, FLT_MAX] <=> its bits in [1, 0x7F7FFFFF].
@@ -314,37 +320,46 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
                 }
                 __syncwarp();
                 pack_tile<BB>(s_idx, ng, lane, words + (size_t)Gu * BB);
-                if ((uint32_t)lane < ng) sa.cbits[Gu + lane] = s_cb[lane];
-                n_def = __reduce_add_sync(FULL, n_def);
-                if (lane == 0 && n_def) atomicAdd(sa.tile_cnt + tile, n_def);
+                if constexpr (SPEC) {
+                    if ((uint32_t)lane < ng) sa.cbits[Gu + lane] = s_cb[lane];
+                    n_def = __reduce_add_sync(FULL, n_def);
+                    if (lane == 0 && n_def) atomicAdd(sa.tile_cnt + tile, n_def);
+                }
                 __syncwarp();                                // (s_idx, s_cb are refilled next unit)
             }
+            if constexpr (SPEC) {
             n_below = __reduce_add_sync(FULL, n_below);
             if (lane == 0 && n_below) atomicAdd(sa.below + h, (unsigned long long)n_below);
             if (n_stage)
                 flush_stage(stage, n_stage, lane, sa.cand_n + h, sa.cand + (uint64_t)h * sa.cand_cap,
                             sa.cand_cap, sa.med_hist + (size_t)h * MED_BINS * 2, w.lo_key, top);
+            }
             const unsigned nf = __reduce_add_sync(FULL, n_nf);
             const unsigned ns = __reduce_add_sync(FULL, n_sat);
             if (lane == 0 && (nf | ns)) {
-                atomicAdd(sa.head_stat + 2 * h, (unsigned long long)nf);
-                atomicAdd(sa.head_stat + 2 * h + 1, (unsigned long long)ns);
+                if constexpr (SPEC) {
+                    atomicAdd(sa.head_stat + 2 * h, (unsigned long long)nf);
+                    atomicAdd(sa.head_stat + 2 * h + 1, (unsigned long long)ns);
+                } else if (st) {
+                    if (nf) status_add(st, HQMQ_FLAG_NONFINITE, &st->n_nonfinite, nf);
+                    if (ns) status_add(st, HQMQ_FLAG_SATURATED, &st->n_saturated, ns);
+                }
             }
         }
     }
 }
 
-template <int DT, int BB, int R>
+template <int DT, int BB, int R, bool SPEC>
 static int launch_spec(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
                        const void *table, uint32_t *words, uint16_t *radius, const SpecArgs &sa,
-                       int sm_count, cudaStream_t stream) {
+                       DevStatus *st, int sm_count, cudaStream_t stream) {
     const uint32_t gps = (uint32_t)(((uint64_t)T * D / 4) / 32);
     const uint32_t ups = (gps + UNIT_G - 1) / UNIT_G;
     const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
     const uint64_t n_units = (uint64_t)B * H * ups;
     const size_t smem = ((size_t)24 * S + 1) * R * sizeof(float4) + (size_t)SPEC_WARPS * WARP_SMEM;
     if (smem > SPEC_SMEM_MAX) return HQMQ_ERR_ARG;
-    auto kern = k_encode_spec<DT, BB, R>;
+    auto kern = k_encode_spec<DT, BB, R, SPEC>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return HQMQ_ERR_CUDA;
@@ -359,28 +374,53 @@ static int launch_spec(int B, int H, int T, int D, const void *x, const float *c
     kern<<<(unsigned)ctas, SPEC_THREADS, smem, stream>>>(
         x, B, H, gps, ups, tps, (uint32_t)n_units, (uint32_t)round_units,
         reinterpret_cast<const float4 *>(cb), S,
-        reinterpret_cast<const uint4 *>(table), words, radius, sa);
+        reinterpret_cast<const uint4 *>(table), words, radius, sa, st);
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 
-template <int DT, int BB>
+template <int DT, int BB, bool SPEC>
 static int launch_spec_r(int B, int H, int T, int D, const void *x, const float *cb, uint32_t S,
                          const void *table, uint32_t *words, uint16_t *radius, const SpecArgs &sa,
-                         int sm_count, cudaStream_t stream) {
+                         DevStatus *st, int sm_count, cudaStream_t stream) {
     // 8 table copies when they fit next to the warps' regions, else 4
     const size_t smem8 = ((size_t)24 * S + 1) * 8 * sizeof(float4) + (size_t)SPEC_WARPS * WARP_SMEM;
     if (smem8 <= SPEC_SMEM_MAX)
-        return launch_spec<DT, BB, 8>(B, H, T, D, x, cb, S, table, words, radius, sa, sm_count,
-                                      stream);
-    return launch_spec<DT, BB, 4>(B, H, T, D, x, cb, S, table, words, radius, sa, sm_count, stream);
+        return launch_spec<DT, BB, 8, SPEC>(B, H, T, D, x, cb, S, table, words, radius, sa, st,
+                                            sm_count, stream);
+    return launch_spec<DT, BB, 4, SPEC>(B, H, T, D, x, cb, S, table, words, radius, sa, st,
+                                        sm_count, stream);
+}
+
+template <bool SPEC>
+static int launch_spec_dt(int dtype, uint32_t b, int B, int H, int T, int D, const void *x,
+                          const float *cb, uint32_t S, const void *table, uint32_t *words,
+                          uint16_t *radius, const SpecArgs &sa, DevStatus *st, int sm_count,
+                          cudaStream_t stream) {
+    if (dtype == HQMQ_BF16) {
+        if (b == 8)
+            return launch_spec_r<HQMQ_BF16, 8, SPEC>(B, H, T, D, x, cb, S, table, words, radius,
+                                                     sa, st, sm_count, stream);
+        if (b == 10)
+            return launch_spec_r<HQMQ_BF16, 10, SPEC>(B, H, T, D, x, cb, S, table, words, radius,
+                                                      sa, st, sm_count, stream);
+    } else {
+        if (b == 8)
+            return launch_spec_r<HQMQ_F32, 8, SPEC>(B, H, T, D, x, cb, S, table, words, radius,
+                                                    sa, st, sm_count, stream);
+        if (b == 10)
+            return launch_spec_r<HQMQ_F32, 10, SPEC>(B, H, T, D, x, cb, S, table, words, radius,
+                                                     sa, st, sm_count, stream);
+    }
+    return HQMQ_ERR_ARG;
 }
 
 }  // namespace hqmq
 
-// True when the one-read speculative pass has a kernel here for this index
-// width (b = 8: S = 8..10; b = 10: S = 22..42).
+// True when the unit kernels of this file cover this index width (b = 8:
+// S = 8..10; b = 10: S = 22..42).
 extern "C" int hqmq_spec_encode_supported(uint32_t b) { return b == 8 || b == 10; }
 
+// The one-read Med3x encode pass (speculative, chunk mode).
 extern "C" int hqmq_launch_spec_encode_units(const void *x, int dtype, int B, int H, int T, int D,
                                              const float *cb, uint32_t S, uint32_t b,
                                              const void *table, uint32_t *words, uint16_t *radius,
@@ -388,20 +428,17 @@ extern "C" int hqmq_launch_spec_encode_units(const void *x, int dtype, int B, in
     using namespace hqmq;
     const SpecArgs sa = spec_args(reinterpret_cast<char *>(ws),
                                   fused_layout(B, H, T, D, HQMQ_GRAN_CHUNK));
-    if (dtype == HQMQ_BF16) {
-        if (b == 8)
-            return launch_spec_r<HQMQ_BF16, 8>(B, H, T, D, x, cb, S, table, words, radius, sa,
-                                               sm_count, stream);
-        if (b == 10)
-            return launch_spec_r<HQMQ_BF16, 10>(B, H, T, D, x, cb, S, table, words, radius, sa,
-                                                sm_count, stream);
-    } else {
-        if (b == 8)
-            return launch_spec_r<HQMQ_F32, 8>(B, H, T, D, x, cb, S, table, words, radius, sa,
-                                              sm_count, stream);
-        if (b == 10)
-            return launch_spec_r<HQMQ_F32, 10>(B, H, T, D, x, cb, S, table, words, radius, sa,
-                                               sm_count, stream);
-    }
-    return HQMQ_ERR_ARG;
+    return launch_spec_dt<true>(dtype, b, B, H, T, D, x, cb, S, table, words, radius, sa, nullptr,
+                                sm_count, stream);
+}
+
+// The plain table encode (no Med3x threshold) with the same data flow.
+extern "C" int hqmq_launch_table_encode_units(const void *x, int dtype, int B, int H, int T, int D,
+                                              const float *cb, uint32_t S, uint32_t b,
+                                              const void *table, uint32_t *words,
+                                              uint16_t *radius, hqmq_status *st, int sm_count,
+                                              cudaStream_t stream) {
+    using namespace hqmq;
+    return launch_spec_dt<false>(dtype, b, B, H, T, D, x, cb, S, table, words, radius, SpecArgs{},
+                                 reinterpret_cast<DevStatus *>(st), sm_count, stream);
 }
