@@ -22,11 +22,20 @@
 // into contiguous unit ranges over the CTAs, so that at any time the GPU
 // works on at most 8 heads, whose search tables stay in L2.  Inside a slab's
 // share of a range every warp takes a contiguous share of the units.  Each warp
-// streams its chunks through a private cp.async ring in shared memory
-// (7 groups = 1.75 KB ahead per warp, ~56 KB in flight per SM), so that HBM
-// latency is hidden without registers; the head's codeword table sits in
-// shared memory in R copies (lane l reads copy l mod R: the 8 lanes of a
-// 16-byte phase hit distinct bank groups for R = 8).  Indices of a unit are
+// streams its chunks through a private cp.async ring in shared memory (4
+// packing groups, 3 ahead; 16-byte copies that bypass L1).  The head's
+// codeword table sits in shared memory in R copies (lane l reads copy
+// l mod R; R = 8 makes the 8 lanes of a 16-byte phase hit distinct bank
+// groups), R chosen so that the CTA's shared memory stays within 144 KB and
+// the SM keeps 92 KB of L1, through which the random table records go: at
+// S = 32 that is R = 4, and the larger L1 is worth more than conflict-free
+// codeword loads.
+//
+// A chunk step is software-pipelined: the next chunk's face, cell and record
+// load are issued before the current chunk's candidates are scored.  The
+// Med3x bookkeeping per chunk is only the count below the window and the
+// candidate bit; chunks inside the window or above t_lo (a few per cent) are
+// queued per warp and handled a queue at a time.  Indices of a unit are
 // staged in shared memory and packed into the unit's b-bit words with
 // coalesced stores.
 //
@@ -40,12 +49,23 @@ namespace hqmq {
 constexpr int SPEC_THREADS = 1024;
 constexpr int SPEC_WARPS = SPEC_THREADS / 32;
 constexpr int UNIT_G = 8;                          // packing groups per work unit
-constexpr int RING_BYTES = 2048;                   // input ring per warp
+constexpr int RING_SLOTS = 4;                      // input ring per warp: packing groups
 constexpr int SPEC_STAGE = 128;                    // window keys staged per warp
-constexpr int WARP_SMEM = RING_BYTES + SPEC_STAGE * 4 + UNIT_G * 32 * 2 + UNIT_G * 4;
-static_assert(WARP_SMEM % 16 == 0, "per-warp shared regions stay 16-byte aligned");
+constexpr int EVQ = 64;                            // event queue entries per warp
+// per-warp shared bytes: input ring, window-key stage, index stage, candidate
+// bits, event queue (keys, then raw chunks of CB bytes)
+__host__ __device__ constexpr int warp_smem(int CB) {
+    return RING_SLOTS * 32 * CB + SPEC_STAGE * 4 + UNIT_G * 32 * 2 + UNIT_G * 4 + EVQ * (4 + CB);
+}
+static_assert(warp_smem(8) % 16 == 0 && warp_smem(16) % 16 == 0,
+              "per-warp shared regions stay 16-byte aligned");
 static_assert(TILE_GROUPS % UNIT_G == 0, "a unit lies inside one list tile");
 constexpr size_t SPEC_SMEM_MAX = 227 * 1024;
+// Shared memory of a CTA up to which more table copies are taken: the rest of
+// the SM's 256 KB is L1 (the carve-out rounds shared memory up: 144 KB -> 164
+// KB, L1 92 KB), which the table records go through; measured on B200, the
+// kernel runs faster with that L1 than with conflict-free codeword loads.
+constexpr size_t SPEC_SMEM_L1 = 144 * 1024;
 constexpr int SPEC_ROUND_HEADS = 8;               // heads per round of the walk
 // Steps of a unit unrolled per loop trip: 2 measured fastest on B200 (4 and 8
 // run slower: the body no longer stays in the instruction cache).
@@ -99,6 +119,52 @@ __device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
+// Cell of the gnomonic point (t1, t2, t3) on the 32^3 grid, without
+// float-to-int conversions: each coordinate's grid position v in [0, 32) is
+// floored by adding 2^23 with rounding toward zero, which leaves floor(v) in
+// the low bits of the sum; the three sums are combined with integer
+// multiply-adds and the exponent bits subtracted once.  The map's constants
+// are scaled by (1 - 2^-20) and offset by 2^-17 so that t = 1 stays below 32
+// and t = -1 above 0; the shift of a boundary is below 3.2e-6 in t, inside
+// the 1e-5 by which every cell of the table is widened.  A non-finite t gives
+// some in-range cell (the mask).
+__device__ __forceinline__ uint32_t cell_of(float c1, float c2, float c3, float inv) {
+    constexpr float SC = 1.0f - 1.0f / 1048576.0f;
+    constexpr float HG = 0.5f * LUT_G;
+    constexpr float PA = MAP_A * HG * SC, PB = MAP_B * HG * SC, P0 = HG * SC + 1.0f / 131072.0f;
+    constexpr float MAGIC = 8388608.0f;                    // 2^23
+    constexpr uint32_t EXP = 0x4B000000u;                  // bits of 2^23
+    // t1 and t2 as one pair through the packed f32x2 operations (each lane of
+    // a pair is the IEEE operation on its own: the same values as scalar code)
+    uint32_t b1, b2;
+    asm("{.reg .b64 t, u, p, q;\n\t"
+        "mov.b64 t, {%2, %3};\n\t"
+        "mov.b64 u, {%4, %4};\n\t"
+        "mul.rn.f32x2 t, t, u;\n\t"                       // (t1, t2)
+        "mul.rn.f32x2 u, t, t;\n\t"                       // squares
+        "mov.b64 p, {%5, %5};\n\t"
+        "mov.b64 q, {%6, %6};\n\t"
+        "fma.rn.f32x2 u, p, u, q;\n\t"                    // PB t^2 + PA
+        "mov.b64 p, {%7, %7};\n\t"
+        "fma.rn.f32x2 t, t, u, p;\n\t"                    // t (PB t^2 + PA) + P0
+        "mov.b64 p, {%8, %8};\n\t"
+        "add.rz.f32x2 t, t, p;\n\t"
+        "mov.b64 {%0, %1}, t;}"
+        : "=r"(b1), "=r"(b2)
+        : "f"(c1), "f"(c2), "f"(inv), "f"(PB), "f"(PA), "f"(P0), "f"(MAGIC));
+    const float t3 = c3 * inv;
+    const uint32_t b3 = __float_as_uint(__fadd_rz(__fmaf_rn(t3, __fmaf_rn(PB, t3 * t3, PA), P0), MAGIC));
+    const uint32_t c = (b1 * (uint32_t)LUT_G + b2) * (uint32_t)LUT_G + b3;
+    return (c - EXP * (uint32_t)(LUT_G * LUT_G + LUT_G + 1)) & (uint32_t)(LUT_CELLS - 1);
+}
+
+// What a chunk step carries from its front half to its back half.
+template <int DT> struct StepState {
+    RawChunk<DT> v;         // the chunk as read
+    float r;                // its norm (0 for a certain outlier)
+    uint4 rec;              // its cell's record (in flight until used)
+};
+
 // SPEC = false: the plain table encode (no Med3x): no window bookkeeping, no
 // candidate bits or values, status counts straight to st.
 template <int DT, int BB, int R, bool SPEC>
@@ -108,7 +174,8 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
               const uint4 *__restrict__ tables, uint32_t *__restrict__ words,
               uint16_t *__restrict__ radius, SpecArgs sa, DevStatus *st) {
     constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;       // bytes per chunk
-    constexpr int NS = RING_BYTES / (32 * CB);         // ring slots (packing groups)
+    constexpr int NS = RING_SLOTS;                     // ring slots (packing groups)
+    constexpr int RING_BYTES = NS * 32 * CB;
     static_assert(NS >= 2 && UNIT_G % NS == 0, "a unit's groups fill whole ring rounds");
     extern __shared__ __align__(16) unsigned char s_raw[];
     float4 *s_tab = reinterpret_cast<float4 *>(s_raw); // [24 S + 1][R]
@@ -116,10 +183,15 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = (1u << lane) - 1u;
     unsigned char *wsm = s_raw + (size_t)(n_words + 1) * R * sizeof(float4) +
-                         (size_t)warp * WARP_SMEM;
+                         (size_t)warp * warp_smem(CB);
     uint32_t *stage = reinterpret_cast<uint32_t *>(wsm + RING_BYTES);
     uint16_t *s_idx = reinterpret_cast<uint16_t *>(wsm + RING_BYTES + SPEC_STAGE * 4);
     uint32_t *s_cb = reinterpret_cast<uint32_t *>(wsm + RING_BYTES + SPEC_STAGE * 4 + UNIT_G * 64);
+    // event queue: chunks of the current unit inside the median window or above
+    // t_lo, in chunk order (their keys and raw values)
+    uint32_t *q_key = s_cb + UNIT_G;
+    using Raw = typename RingWord<CB>::T;
+    Raw *q_raw = reinterpret_cast<Raw *>(q_key + EVQ);
     // 32-bit shared addresses of this lane's ring chunk (slot 0), table copy,
     // index stage entry (group 0) and the warp's candidate-bit words
     const uint32_t a_ring = (uint32_t)__cvta_generic_to_shared(wsm) + (uint32_t)lane * CB;
@@ -127,6 +199,19 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
     const uint32_t a_idx = (uint32_t)__cvta_generic_to_shared(s_idx) + (uint32_t)lane * 2u;
     const uint32_t a_cb = (uint32_t)__cvta_generic_to_shared(s_cb);
     const unsigned char *xl = reinterpret_cast<const unsigned char *>(x) + (size_t)lane * CB;
+    // Copies packing group G into ring slot `slot`: 16-byte copies that bypass
+    // L1 (bf16: lanes 0..15 copy two chunks each), so that x does not take L1
+    // space from the table records.
+    const uint32_t a_ring0 = (uint32_t)__cvta_generic_to_shared(wsm);
+    auto ring_copy = [&](uint32_t slot, uint32_t G) {
+        if constexpr (CB == 8) {
+            if (lane < 16)
+                cp_async_chunk<16>(a_ring0 + slot * 256u + (uint32_t)lane * 16u,
+                                   reinterpret_cast<const unsigned char *>(x) + (size_t)G * 256u + lane * 16u);
+        } else {
+            cp_async_chunk<16>(a_ring + slot * 32u * CB, xl + (size_t)G * (32u * CB));
+        }
+    };
 
     int cur_h = -1;
     // rounds of round_units units (a few heads' worth), each split into
@@ -175,7 +260,7 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
     #pragma unroll
             for (int i = 0; i < NS - 1; ++i) {
                 if (Gb + i < Ge)
-                    cp_async_chunk<CB>(a_ring + (uint32_t)i * 32u * CB, xl + (size_t)(Gb + i) * (32u * CB));
+                    ring_copy(i, Gb + i);
                 cp_async_commit();
             }
             uint32_t n_stage = 0, n_below = 0, n_nf = 0, n_sat = 0;
@@ -184,69 +269,92 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
                 const uint32_t ng = min((uint32_t)UNIT_G, gps - g0);
                 const uint32_t Gu = g_slab + g0;
                 const uint32_t tile = slab * tps + g0 / TILE_GROUPS;
-                uint32_t n_def = 0, fbm = 0, n_cv = 0;
+                uint32_t n_def = 0, fbm = 0, n_cv = 0, n_q = 0;
                 unsigned char *cv_u = sa.cvals + (size_t)(slab * ups + (u - u_slab)) * (CVAL_SLOTS * CB);
-                auto step = [&](const uint32_t k) {
+                // The queued events of this unit, in chunk order: window keys to the
+                // stage (flushed to the head's key list when full), the raw values
+                // of the unit's first CVAL_SLOTS candidates (r > t_lo), the count of
+                // certain outliers (r > t_hi) for the unit's list tile, and the
+                // (tile, key) pairs of the band t_lo < r <= t_hi.  Warp-collective.
+                auto events = [&]() {
+                    __syncwarp();                            // (the lanes' queue writes)
+                    for (uint32_t e0 = 0; e0 < n_q; e0 += 32) {
+                        const uint32_t e = e0 + (uint32_t)lane;
+                        const bool valid = e < n_q;
+                        const uint32_t key = valid ? q_key[e] : 0u;
+                        const float r = __uint_as_float(key);
+                        const bool in = valid && key - w.lo_key < span;
+                        const bool cnd = valid && r > w.t_lo;
+                        const bool dfn = valid && r > w.t_hi;
+                        const uint32_t mi = __ballot_sync(FULL, in);
+                        if (mi) {
+                            if (n_stage > (uint32_t)SPEC_STAGE - 32u) {
+                                flush_stage(stage, n_stage, lane, sa.cand_n + h,
+                                            sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap,
+                                            sa.med_hist + (size_t)h * MED_BINS * 2, w.lo_key, top);
+                                n_stage = 0;
+                            }
+                            if (in) stage[n_stage + __popc(mi & lt)] = key;
+                            n_stage += __popc(mi);
+                        }
+                        const uint32_t mc = __ballot_sync(FULL, cnd);
+                        const uint32_t pos = n_cv + __popc(mc & lt);
+                        if (cnd && pos < (uint32_t)CVAL_SLOTS)
+                            *reinterpret_cast<Raw *>(cv_u + pos * CB) = q_raw[e];
+                        n_cv += __popc(mc);
+                        n_def += dfn ? 1u : 0u;
+                        if (cnd && !dfn) {                   // (rare) inside the band
+                            const unsigned long long p = atomicAdd(sa.amb_n, 1ull);
+                            if (p < sa.amb_cap) sa.amb[p] = make_uint2(tile, key);
+                        }
+                    }
+                    __syncwarp();                            // (the queue is refilled next)
+                    n_q = 0;
+                };
+                // One chunk step is split in two: front(k) reads the chunk, does the
+                // Med3x bookkeeping, finds its face and cell and issues the load of
+                // the cell's record; back(k) scores the candidates and stores the
+                // codes.  front(k + 1) runs before back(k), so that the record's L2
+                // latency overlaps the scoring of the previous step.
+                auto front = [&](const uint32_t k) -> StepState<DT> {
                     const uint32_t G = Gu + k;
                     // group G's copy was the (NS-1)-th latest commit: wait for it
                     cp_async_wait<NS - 2>();
+                    if constexpr (CB == 8) __syncwarp();     // (lanes read chunks another lane copied)
                     RawChunk<DT> cur;
                     if constexpr (CB == 8) cur.v = lds_u2(a_ring + (k % NS) * 32u * CB);
                     else cur.v = lds_f4_ring(a_ring + (k % NS) * 32u * CB);
                     // refill the slot read in the previous step (this lane's bytes only)
                     if (G + (NS - 1) < Ge)
-                        cp_async_chunk<CB>(a_ring + ((k + NS - 1) % NS) * 32u * CB,
-                                           xl + (size_t)(G + (NS - 1)) * (32u * CB));
+                        ring_copy((k + NS - 1) % NS, G + (NS - 1));
                     cp_async_commit();
                     const float x0 = cur.e(0), x1 = cur.e(1), x2 = cur.e(2), x3 = cur.e(3);
                     float r = chunk_norm(x0, x1, x2, x3);
                     // median window: key = r's bits (r >= 0; a NaN's bits exceed
                     // every finite key and +inf's, as in the median's order)
                     const uint32_t key = __float_as_uint(r);
-                    bool cnd = false;
                     if constexpr (SPEC) {
+                    // Per chunk only what every chunk needs: the count below the
+                    // window and the candidate bit.  Chunks inside the window or
+                    // above t_lo (a few per cent) go to the event queue, handled
+                    // a queue at a time by events().
                     n_below += key < w.lo_key ? 1u : 0u;
                     const bool in = key - w.lo_key < span;   // lo_key <= key < hi_key
-                    const uint32_t mi = __ballot_sync(FULL, in);
-                    if (mi) {
-                        if (n_stage + 32 > SPEC_STAGE) {
-                            flush_stage(stage, n_stage, lane, sa.cand_n + h,
-                                        sa.cand + (uint64_t)h * sa.cand_cap, sa.cand_cap,
-                                        sa.med_hist + (size_t)h * MED_BINS * 2, w.lo_key, top);
-                            n_stage = 0;
-                        }
-                        if (in) stage[n_stage + __popc(mi & lt)] = key;
-                        n_stage += __popc(mi);
-                        __syncwarp();
-                    }
-                    // threshold band: above t_hi always an outlier, above t_lo possibly
-                    const bool dfn = r > w.t_hi;             // (NaN: false)
-                    cnd = r > w.t_lo;
-                    n_def += dfn ? 1u : 0u;
+                    const bool cnd = r > w.t_lo;             // (NaN: false)
                     const uint32_t mc = __ballot_sync(FULL, cnd);
                     if (lane == 0) sts_u32(a_cb + k * 4u, mc);
-                    {   // the raw value of a possible outlier, for the fix-up pass
-                        const uint32_t pos = n_cv + __popc(mc & lt);
-                        if (cnd && pos < (uint32_t)CVAL_SLOTS)
-                            *reinterpret_cast<decltype(cur.v) *>(cv_u + pos * CB) = cur.v;
-                        n_cv += __popc(mc);
+                    const uint32_t me = __ballot_sync(FULL, in || cnd);
+                    if (n_q > (uint32_t)(EVQ - 32)) events();   // (warp-uniform) make room
+                    if (in || cnd) {
+                        const uint32_t q = n_q + __popc(me & lt);
+                        q_key[q] = key;
+                        q_raw[q] = cur.v;
                     }
-                    const uint32_t mu = __ballot_sync(FULL, cnd && !dfn);
-                    if (mu) {
-                        unsigned long long base = 0;
-                        if (lane == 0) base = atomicAdd(sa.amb_n, (unsigned long long)__popc(mu));
-                        base = __shfl_sync(FULL, base, 0);
-                        if ((mu >> lane) & 1u) {
-                            const unsigned long long pos = base + __popc(mu & lt);
-                            if (pos < sa.amb_cap) sa.amb[pos] = make_uint2(tile, key);
-                        }
-                    }
-                    if (dfn) r = 0.0f;                       // certain outlier: radius 0, index 0
+                    n_q += __popc(me);
                     }
                     // search every lane (branch-free); a lane whose chunk is zero,
                     // non-finite or a certain outlier reads some in-range record and
                     // keeps index 0.  r in (0, FLT_MAX] <=> its bits in [1, 0x7F7FFFFF].
-                    const bool srch = __float_as_uint(r) - 1u < 0x7F7FFFFFu;
                     const float a0 = fabsf(x0), a1 = fabsf(x1), a2 = fabsf(x2), a3 = fabsf(x3);
                     const float m = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
                     const bool e0 = a0 == m, e01 = e0 || a1 == m, e012 = e01 || a2 == m;
@@ -257,10 +365,22 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
                     const float c3 = e012 ? x3 : x2;
                     float inv;
                     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(m));   // cells are widened
-                    const uint32_t cell = (uint32_t)((cell_coord(c1 * inv) * LUT_G + cell_coord(c2 * inv)) *
-                                                         LUT_G + cell_coord(c3 * inv)) & (LUT_CELLS - 1u);
+                    const uint32_t cell = cell_of(c1, c2, c3, inv);
                     const uint32_t face = 2u * a + (xa < 0.0f ? 1u : 0u);
-                    const uint4 rec = __ldg(tb + (face * LUT_CELLS + cell));
+                    StepState<DT> o;
+                    o.v = cur;
+                    o.r = r;
+                    o.rec = __ldg(tb + (face * LUT_CELLS + cell));
+                    return o;
+                };
+                auto back = [&](const uint32_t k, const StepState<DT> &c) {
+                    const uint32_t G = Gu + k;
+                    const float x0 = c.v.e(0), x1 = c.v.e(1), x2 = c.v.e(2), x3 = c.v.e(3);
+                    // a certain outlier (r > t_hi) is encoded as index 0, radius 0
+                    const bool cnd = SPEC && c.r > w.t_lo;
+                    const float r = SPEC && c.r > w.t_hi ? 0.0f : c.r;
+                    const uint4 rec = c.rec;
+                    const bool srch = __float_as_uint(r) - 1u < 0x7F7FFFFFu;
                     const uint32_t cnt = (rec.x >> 12) & 0xFu;          // 0: overflowing cell
                     const uint32_t kmax = __reduce_max_sync(FULL, cnt);
                     // the slots hold increasing ids (padded with the zero codeword
@@ -304,10 +424,16 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
                     sts_u16(a_idx + k * 64u, idx);
                 };
                 if (ng == UNIT_G) {
+                    StepState<DT> cs = front(0);
     #pragma unroll kSpecUnroll
-                    for (uint32_t k = 0; k < UNIT_G; ++k) step(k);
+                    for (uint32_t k = 0; k < UNIT_G - 1; ++k) {
+                        const StepState<DT> ns = front(k + 1);
+                        back(k, cs);
+                        cs = ns;
+                    }
+                    back(UNIT_G - 1, cs);
                 } else {
-                    for (uint32_t k = 0; k < ng; ++k) step(k);
+                    for (uint32_t k = 0; k < ng; ++k) back(k, front(k));
                 }
                 if (__any_sync(FULL, fbm != 0u)) {          // (rare) overflowing cells
                     for (uint32_t k = 0; k < ng; ++k) {
@@ -321,6 +447,7 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
                 __syncwarp();
                 pack_tile<BB>(s_idx, ng, lane, words + (size_t)Gu * BB);
                 if constexpr (SPEC) {
+                    if (n_q) events();
                     if ((uint32_t)lane < ng) sa.cbits[Gu + lane] = s_cb[lane];
                     n_def = __reduce_add_sync(FULL, n_def);
                     if (lane == 0 && n_def) atomicAdd(sa.tile_cnt + tile, n_def);
@@ -357,7 +484,8 @@ static int launch_spec(int B, int H, int T, int D, const void *x, const float *c
     const uint32_t ups = (gps + UNIT_G - 1) / UNIT_G;
     const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
     const uint64_t n_units = (uint64_t)B * H * ups;
-    const size_t smem = ((size_t)24 * S + 1) * R * sizeof(float4) + (size_t)SPEC_WARPS * WARP_SMEM;
+    constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;
+    const size_t smem = ((size_t)24 * S + 1) * R * sizeof(float4) + (size_t)SPEC_WARPS * warp_smem(CB);
     if (smem > SPEC_SMEM_MAX) return HQMQ_ERR_ARG;
     auto kern = k_encode_spec<DT, BB, R, SPEC>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -383,11 +511,18 @@ static int launch_spec_r(int B, int H, int T, int D, const void *x, const float 
                          const void *table, uint32_t *words, uint16_t *radius, const SpecArgs &sa,
                          DevStatus *st, int sm_count, cudaStream_t stream) {
     // 8 table copies when they fit next to the warps' regions, else 4
-    const size_t smem8 = ((size_t)24 * S + 1) * 8 * sizeof(float4) + (size_t)SPEC_WARPS * WARP_SMEM;
-    if (smem8 <= SPEC_SMEM_MAX)
+    // as many table copies (8, 4 or 2) as keep the CTA's shared memory within
+    // SPEC_SMEM_L1, so that the SM keeps that much L1 for the table records
+    constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;
+    const size_t warps = (size_t)SPEC_WARPS * warp_smem(CB);
+    const size_t copy = ((size_t)24 * S + 1) * sizeof(float4);
+    if (8 * copy + warps <= SPEC_SMEM_L1)
         return launch_spec<DT, BB, 8, SPEC>(B, H, T, D, x, cb, S, table, words, radius, sa, st,
                                             sm_count, stream);
-    return launch_spec<DT, BB, 4, SPEC>(B, H, T, D, x, cb, S, table, words, radius, sa, st,
+    if (4 * copy + warps <= SPEC_SMEM_L1)
+        return launch_spec<DT, BB, 4, SPEC>(B, H, T, D, x, cb, S, table, words, radius, sa, st,
+                                            sm_count, stream);
+    return launch_spec<DT, BB, 2, SPEC>(B, H, T, D, x, cb, S, table, words, radius, sa, st,
                                         sm_count, stream);
 }
 

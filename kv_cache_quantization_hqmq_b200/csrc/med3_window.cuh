@@ -103,6 +103,7 @@ __device__ __forceinline__ void flush_stage(uint32_t *stage, uint32_t n, int lan
                                             unsigned long long *cand_n_h, uint32_t *cand_h,
                                             uint64_t cand_cap, uint32_t *hist_h, uint32_t lo_key,
                                             int top) {
+    __syncwarp();                                  // the lanes' stage writes
     unsigned long long base = 0;
     if (lane == 0) base = atomicAdd(cand_n_h, (unsigned long long)n);
     base = __shfl_sync(FULL, base, 0);
