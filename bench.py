@@ -226,21 +226,35 @@ class Cache:
     def call(self, l, r, x, stream, timers=None):
         """One (layer, role) call on `stream`: Med3x + encode, then decode."""
         import torch
-        from kv_cache_quantization_hqmq_b200 import hqmq
-        w = self.w
-        H = w.heads
 
         def ev():
             e = torch.cuda.Event(enable_timing=True)
             e.record(stream)
             return e
 
-        g0 = (l * 2 + r) * H
-        cb = self.codebook[g0 * w.S * 4:(g0 + H) * w.S * 4]
+        t0 = ev() if timers is not None else None
+        self.encode_call(l, r, x, stream)
+        t1 = ev() if timers is not None else None
+        self.decode_call(l, r, stream)
+        if timers is not None:
+            t2 = ev()
+            timers["med3_encode" if self.w.med3 else "encode"].append((t0, t1))
+            timers["decode"].append((t1, t2))
+
+    def _groups(self, l, r):
+        w = self.w
+        g0 = (l * 2 + r) * w.heads
+        cb = self.codebook[g0 * w.S * 4:(g0 + w.heads) * w.S * 4]
         tb = None
         if self.table is not None:
-            tb = self.table[g0 * self.table_bytes:(g0 + H) * self.table_bytes]
-        t0 = ev() if timers is not None else None
+            tb = self.table[g0 * self.table_bytes:(g0 + w.heads) * self.table_bytes]
+        return cb, tb
+
+    def encode_call(self, l, r, x, stream):
+        """Med3x + encode of one (layer, role) call."""
+        from kv_cache_quantization_hqmq_b200 import hqmq
+        w = self.w
+        cb, tb = self._groups(l, r)
         if w.med3:
             # Med3x and encode in one fused call (one read of x in chunk mode
             # with search tables, two otherwise)
@@ -255,7 +269,12 @@ class Cache:
         else:
             hqmq.hqmq_encode(x, cb, w.S, None, self.gran, self.words[l, r],
                              self.radius[l, r], self.status, stream)
-        t1 = ev() if timers is not None else None
+
+    def decode_call(self, l, r, stream):
+        """Decode of one (layer, role) call into the reusable output buffer."""
+        from kv_cache_quantization_hqmq_b200 import hqmq
+        w = self.w
+        cb, _ = self._groups(l, r)
         if w.med3:
             hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S,
                              self.out_idx[l, r], self.out_val[l, r], self.slab_off[l, r],
@@ -264,10 +283,46 @@ class Cache:
         else:
             hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S, None, None,
                              None, 0, self.gran, self.y, self.status, stream)
-        if timers is not None:
-            t2 = ev()
-            timers["med3_encode" if w.med3 else "encode"].append((t0, t1))
-            timers["decode"].append((t1, t2))
+
+    def graph_times(self, reps):
+        """Device time of one step, of the step's encode calls and of its
+        decode calls, each captured in one CUDA graph and replayed `reps`
+        times: (ms per step, {family: ms per call}).  Small calls issued one
+        by one from Python are bound by the host's launch rate; a graph
+        replay measures the kernels."""
+        import torch
+        w = self.w
+
+        def encodes():
+            s = torch.cuda.current_stream()
+            for l in range(w.layers):
+                for r in range(2):
+                    self.encode_call(l, r, self.x[l, r], s)
+
+        def decodes():
+            s = torch.cuda.current_stream()
+            for l in range(w.layers):
+                for r in range(2):
+                    self.decode_call(l, r, s)
+
+        out = {}
+        for key, fn in (("step", self.step), ("enc", encodes), ("dec", decodes)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            g.replay()
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            out[key] = a.elapsed_time(b) / reps
+            del g
+        fam = "med3_encode" if w.med3 else "encode"
+        return out["step"], {fam: out["enc"] / w.n_calls, "decode": out["dec"] / w.n_calls}
 
 
 # DRAM bytes (read + write) of one hqmq_encode_med3 call of the 70B 128k call
@@ -355,14 +410,20 @@ def elapsed_ms(pairs):
     return [a.elapsed_time(b) for a, b in pairs]
 
 
-def kernel_stats(w, timers, peaks, n_out, table):
-    """Per-call time and algorithmic HBM rate of each timed call family."""
+def kernel_stats(w, timers, peaks, n_out, table, per_call_ms=None):
+    """Per-call time and algorithmic HBM rate of each timed call family, from
+    the event pairs in `timers` or from `per_call_ms` {family: ms}."""
     ab = algorithmic_bytes(w, n_out, table)
     kern = {}
     for name in ("med3_encode", "encode", "decode"):
-        if not timers[name]:
+        if per_call_ms is not None:
+            if name not in per_call_ms:
+                continue
+            t = per_call_ms[name]
+        elif not timers[name]:
             continue
-        t = statistics.mean(elapsed_ms(timers[name]))
+        else:
+            t = statistics.mean(elapsed_ms(timers[name]))
         gbs = ab[name] / (t * 1e-3) / 1e9
         kern[name] = {"ms_per_call": round(t, 4), "calls_per_step": w.n_calls,
                       "algorithmic_bytes_per_call": int(ab[name]),
@@ -728,20 +789,27 @@ def run_sweep(device, peaks, steps=3, warmup=3, near_ties=None):
             cache.step()
         torch.cuda.synchronize()
         st = hqmq.read_status(cache.status)
-        timers = {"med3_encode": [], "encode": [], "decode": []}
+        # launches from Python (as the headline step) and the same work as
+        # CUDA graphs (the device time of the kernels)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
         for _ in range(steps):
-            cache.step(timers)
+            cache.step()
         b.record()
         torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / steps
+        ms_plain = a.elapsed_time(b) / steps
+        ms, per_call = cache.graph_times(steps)
         n_out = st["n_outliers"] / max(1, warmup) / w.n_calls if w.med3 else 0.0
         out[name] = {"S": w.S, "med3": ("chunk, C=%g" % w.C) if w.med3 else "off",
                      "cache_gb": round(w.cache_bytes / 1e9, 2), "ms_per_step": round(ms, 3),
                      "value_gbs": round(w.cache_bytes / (ms * 1e-3) / 1e9, 2),
-                     "kernels": kernel_stats(w, timers, peaks, n_out, cache.table is not None),
+                     "timing": "one CUDA graph per step (and per call family for the "
+                               "kernels); ms_per_step_python_launches: the same step "
+                               "launched call by call from Python",
+                     "ms_per_step_python_launches": round(ms_plain, 3),
+                     "kernels": kernel_stats(w, None, peaks, n_out, cache.table is not None,
+                                             per_call_ms=per_call),
                      "status_flags": st["flags"]}
         if near_ties is not None:
             near_ties[name] = oracle_parity_sample(cache, w.layers // 2, 1)
@@ -864,6 +932,11 @@ def run_hqmq(args):
         "gpu_launches": cache.kernels_per_step() * args.steps,
         "clocks": clk,
     }
+    if world == 1:
+        # the same step as one CUDA graph (outside the timed region): equal to
+        # ms_per_step when the Python launches keep ahead of the device
+        ms_graph, _ = cache.graph_times(args.steps)
+        line["ms_per_step_cuda_graph"] = round(ms_graph, 3)
     if world == 1 and not args.no_cpu_baseline:
         line["near_ties"] = {w.name: oracle_parity_sample(cache, w.layers // 2, 1)}
     if world == 1 and not args.no_attention:

@@ -285,3 +285,28 @@ def test_fused_full_size_against_the_oracle(oracle, name, layer, role):
     print("[fused full size] %s L%d role %d: %d outliers (%.3f%%), %d sampled chunks, "
           "%d near-tie index differences, %d near-tie pairs"
           % (name, layer, role, n_o, 100.0 * n_o / n_chunks, n, mm, near))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_fused_every_chunk_inside_the_window(oracle, dtype):
+    # Chunk norms within 0.1% of 1 (all in one bin of the sample's histogram,
+    # so every chunk is a window key and goes through the encode pass's event
+    # queue, which then fills up inside a unit), a contiguous run of 100
+    # outliers (more than one unit's candidate-value slots), 2% scattered
+    # outliers and 1% of chunks around the threshold 3 r_med (its band).
+    rng = np.random.default_rng(11)
+    B, H, T, D = 1, 2, 256, 128
+    n = B * H * T * D // 4
+    u = rng.standard_normal((n, 4))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    r = 1.0 + 1e-3 * rng.random(n)
+    pick = rng.random(n)
+    r = np.where(pick < 0.02, 50.0, r)
+    r = np.where((pick >= 0.02) & (pick < 0.03), 3.0015 * (1 + 2e-4 * rng.standard_normal(n)), r)
+    r[5000:5100] = 20.0
+    x = (u * r[:, None]).astype(np.float32).reshape(B, H, T, D)
+    if dtype == "bf16":
+        x = W.as_numpy_bits(torch.from_numpy(x).to(torch.bfloat16))
+    g = check_fused(oracle, x, 32, 0, True)
+    assert not g["status"]["flags"] & hqmq.FLAG_MED3_FALLBACK
+    assert g["status"]["n_outliers"] > 0.02 * n
