@@ -6,8 +6,8 @@
 // iff r > fl32(C r_med).  The results are exactly those of the three-pass radix
 // select of med3.cu; only the data flow differs:
 //
-//  A+W k_sample_window reads a 1/32 sample (4 consecutive chunks of every 128,
-//                      the quad's slot rotating through all 32 slots) into a
+//  A+W k_sample_window reads a 1/32 sample (the first 128 chunks of every
+//                      4096, read by a warp as one contiguous block) into a
 //                      per-head histogram of the top 16 key bits; the last
 //                      CTA of each head then picks a key window [lo, hi) that
 //                      holds the sample ranks within +-8 standard deviations of
@@ -204,12 +204,14 @@ k_sample_window(const void *__restrict__ x, int H, uint32_t cps, uint32_t ctas_p
     const uint32_t n_quads = (cps + SAMPLE_PERIOD - 1) / SAMPLE_PERIOD;
     for (uint32_t q = blockIdx.x * blockDim.x + threadIdx.x; q < n_quads;
          q += gridDim.x * blockDim.x) {
-        // quad slot (37 q) mod 32 of the q-th 128-chunk period: over 32
-        // periods every slot is sampled once, whatever the chunks' position
-        // inside a head vector
-        const uint32_t slot = (37u * q) & 31u;
-        uint64_t j0 = base + (uint64_t)q * SAMPLE_PERIOD + 4u * slot;
-        if (j0 + 4 > base + cps) j0 = base + (uint64_t)q * SAMPLE_PERIOD;   // short last period
+        // quads 32 m .. 32 m + 31 read the first 128 chunks (1 KB of bf16) of
+        // the m-th run of 32 x 128 chunks: a warp reads one contiguous block
+        // (the same sample size as one quad per 128 chunks, without the DRAM
+        // fetch granularity reading 4 x the sampled bytes), and the block
+        // holds whole head vectors, every position inside them; a quad past
+        // the slab's last full run reads the start of its own 128 chunks
+        uint64_t j0 = base + (uint64_t)(q >> 5) * (32u * SAMPLE_PERIOD) + 4u * (q & 31u);
+        if (j0 + 4 > base + cps) j0 = base + (uint64_t)q * SAMPLE_PERIOD;
         RawChunk<DT> v[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) v[c].load(x, j0 + c);

@@ -11,7 +11,7 @@ namespace hqmq {
 
 constexpr int TILE_GROUPS = 32;                  // packing groups per warp tile
 constexpr int TILE_CHUNKS = TILE_GROUPS * 32;    // 1024 chunks
-constexpr int SAMPLE_PERIOD = 128;               // sample chunks 4k..4k+3 of every 128
+constexpr int SAMPLE_PERIOD = 128;               // one sampled quad (4 chunks) per 128 chunks
 constexpr int KEY_BINS = 65536;                  // sample histogram
 constexpr int WINDOW_SIGMAS = 8;                 // half-width of the rank window
 

@@ -26,6 +26,20 @@ def x_dev(x):
     return dev(x.view(np.int16)).view(torch.bfloat16) if x.dtype == np.uint16 else dev(x)
 
 
+def sampled_chunks(cps):
+    """Mask of the chunks of a slab of cps chunks that the Med3x sample reads:
+    quad q (one per 128 chunks) is chunks 4 (q mod 32) .. + 3 of the first
+    128 of the (q div 32)-th run of 4096 chunks, or the first 4 of its own 128
+    chunks when that lies past the slab."""
+    mask = np.zeros(cps, dtype=bool)
+    for q in range((cps + 127) // 128):
+        j0 = (q // 32) * 4096 + 4 * (q % 32)
+        if j0 + 4 > cps:
+            j0 = q * 128
+        mask[j0:j0 + 4] = True
+    return mask
+
+
 def fused(x_np, cb_np, S, gran, use_table, C=3.0, cap=None):
     B, H, T, D = x_np.shape
     xd = x_dev(x_np)
@@ -86,15 +100,12 @@ def test_fused_fp32_input(oracle):
 
 
 def test_window_miss_takes_the_exact_fallback(oracle):
-    # the sample reads, in the q-th period of 128 chunks of a slab, the quad of
-    # chunks in slot (37 q) mod 32: make exactly those huge, so that the
-    # sampled median is far above the true one
+    # make exactly the chunks the sample reads huge, so that the sampled
+    # median is far above the true one
     rng = np.random.default_rng(4)
     x = rng.standard_normal((1, 2, 512, 128)).astype(np.float32)
     c = x.reshape(1, 2, -1, 4)
-    pos = np.arange(c.shape[2])
-    sampled = (pos % 128) // 4 == (37 * (pos // 128)) % 32
-    c[:, :, sampled] *= 1000.0
+    c[:, :, sampled_chunks(c.shape[2])] *= 1000.0
     x = W.as_numpy_bits(torch.from_numpy(x).to(torch.bfloat16))
     g = check_fused(oracle, x, 8, 0, True)
     assert g["status"]["flags"] & hqmq.FLAG_MED3_FALLBACK
@@ -220,9 +231,7 @@ def test_fused_status_counts_after_a_window_miss(oracle):
     rng = np.random.default_rng(9)
     x = rng.standard_normal((1, 2, 512, 128)).astype(np.float32)
     c = x.reshape(1, 2, -1, 4)
-    pos = np.arange(c.shape[2])
-    sampled = (pos % 128) // 4 == (37 * (pos // 128)) % 32
-    c[:, :, sampled] *= 1000.0
+    c[:, :, sampled_chunks(c.shape[2])] *= 1000.0
     c[0, 0, 5, 0] = np.nan
     c[0, 1, 9, 3] = np.inf
     c[0, 0, 700] = 3e4
