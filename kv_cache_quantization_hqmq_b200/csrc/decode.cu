@@ -82,6 +82,7 @@ k_decode(const uint32_t *__restrict__ words, const uint16_t *__restrict__ radius
          const uint32_t *__restrict__ out_idx, const uint16_t *__restrict__ out_val,
          uint32_t cap32, const uint32_t *__restrict__ rwords, const float *__restrict__ thr) {
     extern __shared__ float4 s_dyn[];
+    pdl_wait();                                    // (launched with launch_pdl)
     const uint32_t n_words = 24u * S;
     float4 *s_tab = s_dyn;                         // [24 S] if TABLE
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -335,9 +336,11 @@ static int launch_main(const uint32_t *words, const uint16_t *radius, const floa
     const uint32_t tps = (gps + TILE_GROUPS - 1) / TILE_GROUPS;
     const uint32_t cap32 = cap < 0xFFFFFFFFull ? (uint32_t)cap : 0xFFFFFFFFu;
     dim3 grid((unsigned)gx, (unsigned)n_slabs);
-    kern<<<grid, DEC_THREADS, smem, stream>>>(words, radius, reinterpret_cast<const float4 *>(cb),
-                                              S, b, H, cps, y, reinterpret_cast<DevStatus *>(st),
-                                              tile_off, tps, out_idx, out_val, cap32, rwords, thr);
+    if (launch_pdl(kern, grid, dim3(DEC_THREADS), smem, stream, words, radius,
+                   reinterpret_cast<const float4 *>(cb), S, b, H, cps, y,
+                   reinterpret_cast<DevStatus *>(st), tile_off, tps, out_idx, out_val, cap32,
+                   rwords, thr) != cudaSuccess)
+        return HQMQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 

@@ -174,6 +174,8 @@ k_encode_spec(const void *__restrict__ x, int B, int H, uint32_t gps, uint32_t u
               const uint4 *__restrict__ tables, uint32_t *__restrict__ words,
               uint16_t *__restrict__ radius, SpecArgs sa, DevStatus *st) {
     constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;       // bytes per chunk
+    pdl_wait();                                        // (launched with launch_pdl)
+    pdl_trigger();
     constexpr int NS = RING_SLOTS;                     // ring slots (packing groups)
     constexpr int RING_BYTES = NS * 32 * CB;
     static_assert(NS >= 2 && UNIT_G % NS == 0, "a unit's groups fill whole ring rounds");
@@ -499,10 +501,11 @@ static int launch_spec(int B, int H, int T, int D, const void *x, const float *c
     uint64_t round_units = (uint64_t)SPEC_ROUND_HEADS * B * ups;
     if (round_units < ctas * SPEC_WARPS) round_units = ctas * SPEC_WARPS;
     if (round_units > n_units) round_units = n_units;
-    kern<<<(unsigned)ctas, SPEC_THREADS, smem, stream>>>(
-        x, B, H, gps, ups, tps, (uint32_t)n_units, (uint32_t)round_units,
-        reinterpret_cast<const float4 *>(cb), S,
-        reinterpret_cast<const uint4 *>(table), words, radius, sa, st);
+    if (launch_pdl(kern, dim3((unsigned)ctas), dim3(SPEC_THREADS), smem, stream, x, B, H, gps, ups,
+                   tps, (uint32_t)n_units, (uint32_t)round_units,
+                   reinterpret_cast<const float4 *>(cb), S, reinterpret_cast<const uint4 *>(table),
+                   words, radius, sa, st) != cudaSuccess)
+        return HQMQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 

@@ -195,4 +195,30 @@ __device__ __forceinline__ void status_add(DevStatus *st, unsigned flag,
     }
 }
 
+// Programmatic dependent launch (sm_90 and later): a kernel launched with
+// launch_pdl may be scheduled while the previous kernel on its stream is
+// still running; it executes pdl_wait() before its first access to global
+// memory, which returns once that kernel has completed and its writes are
+// visible, so any predecessor is safe.  pdl_trigger() lets the next such
+// kernel be scheduled before this one ends.  Only the launch latency and the
+// CTAs' start overlap the predecessor.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 }  // namespace hqmq

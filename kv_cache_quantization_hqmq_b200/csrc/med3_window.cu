@@ -195,6 +195,7 @@ k_sample_window(const void *__restrict__ x, int H, uint32_t cps, uint32_t ctas_p
     // per non-empty bin
     extern __shared__ uint32_t s_pair[];                       // [KEY_BINS / 2]
     __shared__ uint32_t s_warp[32], s_out[4], s_last;
+    pdl_trigger();                                 // (the encode pass may be scheduled)
     for (int i = threadIdx.x; i < KEY_BINS / 2; i += blockDim.x) s_pair[i] = 0;
     __syncthreads();
     const int slab = blockIdx.y;
@@ -593,6 +594,8 @@ k_finalize(const void *__restrict__ x, int B, int H, uint32_t cps, uint32_t tile
            uint64_t cap, uint32_t *__restrict__ med_hist, uint32_t *__restrict__ median_done,
            uint32_t *__restrict__ fin_done, DevStatus *st) {
     __shared__ FinalSmem sm;
+    pdl_wait();                                    // (launched with launch_pdl)
+    pdl_trigger();
     const int h = blockIdx.y;
     const WinState w = win[h];
     const unsigned long long n_amb = *amb_n;
@@ -740,10 +743,12 @@ static int run_finish(const void *x, int B, int H, int T, int D, float C, float 
     if (slices > wave) slices = wave;
     if (slices > (uint64_t)MED_SLICES) slices = MED_SLICES;
     if (slices < 1) slices = 1;
-    k_finalize<DT, GRAN><<<dim3((unsigned)slices, H), WIN_THREADS, 0, stream>>>(
-        x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, a.below, a.cand_n,
-        a.cand, a.cand_cap, a.amb_n, a.amb, a.amb_cap, rmed, thr, a.tile_cnt, tile_off, slab_off,
-        (uint32_t)(B * H), cap, med_hist, median_done, &ctr->fin_done, st);
+    if (launch_pdl(k_finalize<DT, GRAN>, dim3((unsigned)slices, H), dim3(WIN_THREADS), 0, stream,
+                   x, B, H, cps, L.tiles_per_slab, L.n_tiles, L.n_per_head, C, win, a.below,
+                   a.cand_n, a.cand, a.cand_cap, a.amb_n, a.amb, a.amb_cap, rmed, thr,
+                   a.tile_cnt, tile_off, slab_off, (uint32_t)(B * H), cap, med_hist, median_done,
+                   &ctr->fin_done, st) != cudaSuccess)
+        return HQMQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
 

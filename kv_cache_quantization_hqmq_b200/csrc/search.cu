@@ -450,6 +450,8 @@ k_list_fix(const void *__restrict__ x, int H, uint32_t groups_per_slab, uint32_t
     // possible outliers of each 8-group unit, in chunk order (sa.cvals);
     // chunks of a unit with more of them are read from x
     constexpr int CB = DT == HQMQ_BF16 ? 8 : 16;
+    pdl_wait();                                    // (launched with launch_pdl)
+    pdl_trigger();
     const uint32_t units_per_slab = (groups_per_slab + 7) / 8;
     const int lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
@@ -753,13 +755,14 @@ extern "C" int hqmq_launch_fix_pass(const void *x, int dtype, int B, int H, int 
     if (ctas < 1) ctas = 1;
     const float4 *cb4 = reinterpret_cast<const float4 *>(cb);
     DevStatus *dst = reinterpret_cast<DevStatus *>(st);
-    if (dtype == HQMQ_BF16)
-        k_list_fix<HQMQ_BF16><<<(unsigned)ctas, FIX_THREADS, 0, stream>>>(
-            x, H, gps, tps, n_tiles, cb4, S, b, thr, words, radius, tile_off, cap, out_idx,
-            out_val, dst, sa, use_cvals);
-    else
-        k_list_fix<HQMQ_F32><<<(unsigned)ctas, FIX_THREADS, 0, stream>>>(
-            x, H, gps, tps, n_tiles, cb4, S, b, thr, words, radius, tile_off, cap, out_idx,
-            out_val, dst, sa, use_cvals);
+    const cudaError_t e =
+        dtype == HQMQ_BF16
+            ? launch_pdl(k_list_fix<HQMQ_BF16>, dim3((unsigned)ctas), dim3(FIX_THREADS), 0, stream,
+                         x, H, gps, tps, n_tiles, cb4, S, b, thr, words, radius, tile_off, cap,
+                         out_idx, out_val, dst, sa, use_cvals)
+            : launch_pdl(k_list_fix<HQMQ_F32>, dim3((unsigned)ctas), dim3(FIX_THREADS), 0, stream,
+                         x, H, gps, tps, n_tiles, cb4, S, b, thr, words, radius, tile_off, cap,
+                         out_idx, out_val, dst, sa, use_cvals);
+    if (e != cudaSuccess) return HQMQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HQMQ_OK : HQMQ_ERR_CUDA;
 }
