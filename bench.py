@@ -284,6 +284,16 @@ class Cache:
             hqmq.hqmq_decode(self.words[l, r], self.radius[l, r], cb, w.S, None, None,
                              None, 0, self.gran, self.y, self.status, stream)
 
+    def capture(self, fn):
+        """fn's launches captured in one CUDA graph (replayed once)."""
+        import torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
     def graph_times(self, reps):
         """Device time of one step, of the step's encode calls and of its
         decode calls, each captured in one CUDA graph and replayed `reps`
@@ -307,11 +317,7 @@ class Cache:
 
         out = {}
         for key, fn in (("step", self.step), ("enc", encodes), ("dec", decodes)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                fn()
-            g.replay()
-            torch.cuda.synchronize()
+            g = self.capture(fn)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record()
@@ -840,7 +846,9 @@ def run_hqmq(args):
     torch.cuda.synchronize()
     st = hqmq.read_status(cache.status)
 
-    timers = {"med3_encode": [], "encode": [], "decode": []}
+    # each step is one CUDA graph of the step's launches (captured after the
+    # warm-up), so that the host's launch rate does not enter the device time
+    step_graph = cache.capture(cache.step)
     clocks = ClockSampler(torch.cuda.current_device())
     barrier(dist)
     torch.cuda.synchronize()
@@ -849,7 +857,7 @@ def run_hqmq(args):
     end = torch.cuda.Event(enable_timing=True)
     start.record()
     for _ in range(args.steps):
-        cache.step(timers)
+        step_graph.replay()
     end.record()
     torch.cuda.synchronize()
     barrier(dist)
@@ -857,9 +865,23 @@ def run_hqmq(args):
     ms_total = start.elapsed_time(end)
     ms_total = max_over_ranks(ms_total, dist, device)
     ms_step = ms_total / args.steps
+    del step_graph
+
+    # outside the timed region: the same step launched call by call from
+    # Python, and the per-call times of the encode and decode calls (each
+    # family of the step in one graph)
+    a_ev = torch.cuda.Event(enable_timing=True)
+    b_ev = torch.cuda.Event(enable_timing=True)
+    a_ev.record()
+    for _ in range(args.steps):
+        cache.step()
+    b_ev.record()
+    torch.cuda.synchronize()
+    ms_plain = a_ev.elapsed_time(b_ev) / args.steps
+    _, per_call = cache.graph_times(args.steps)
 
     n_out = st["n_outliers"] / max(1, args.warmup) / w.n_calls if w.med3 else 0.0
-    kern = kernel_stats(w, timers, peaks, n_out, cache.table is not None)
+    kern = kernel_stats(w, None, peaks, n_out, cache.table is not None, per_call_ms=per_call)
     B, H, T, D = w.call_shape
     n_chunks = B * H * T * D // 4
     enc_key = "med3_encode" if w.med3 else "encode"
@@ -932,11 +954,11 @@ def run_hqmq(args):
         "gpu_launches": cache.kernels_per_step() * args.steps,
         "clocks": clk,
     }
-    if world == 1:
-        # the same step as one CUDA graph (outside the timed region): equal to
-        # ms_per_step when the Python launches keep ahead of the device
-        ms_graph, _ = cache.graph_times(args.steps)
-        line["ms_per_step_cuda_graph"] = round(ms_graph, 3)
+    line["timing"] = ("each timed step is one CUDA graph replay of the step's launches; "
+                      "ms_per_step_python_launches: the same step launched call by call from "
+                      "Python; per-call kernel times from graphs of the step's encode calls and "
+                      "of its decode calls")
+    line["ms_per_step_python_launches"] = round(ms_plain, 3)
     if world == 1 and not args.no_cpu_baseline:
         line["near_ties"] = {w.name: oracle_parity_sample(cache, w.layers // 2, 1)}
     if world == 1 and not args.no_attention:
@@ -1185,7 +1207,6 @@ def run_reference(args):
     cpu = None
     per_step = max(3.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
         cpu = cpu_baseline(w, per_step)
         if i >= args.warmup:
             times.append(cpu["value"])
@@ -1193,7 +1214,11 @@ def run_reference(args):
     cpu["value"] = round(value, 6)
     line = {"metric": METRIC, "value": round(value, 6), "unit": "GB/s",
             "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "warmup": args.warmup,
+            # a whole step's bf16 cache bytes at the sample's rate
+            "ms_per_step": round(w.cache_bytes / (value * 1e9) * 1e3, 1),
+            "ms_per_step_is": "extrapolated: the step's cache bytes at the rate of the timed sample",
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "S": w.S,
                        "med3": ("chunk, C=%g" % w.C) if w.med3 else "off"},
