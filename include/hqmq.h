@@ -434,7 +434,9 @@ HQMQ_API int hqmq_decode_joint(const uint32_t *d_joint, const float *d_thr,
  * [Hk][S][4], 16-byte aligned).  out_idx == NULL: no outlier list; else
  * out_val (8-byte aligned), tile_off (uint32 [hqmq_list_tiles(B,Hk,T,128) +
  * 1]) and cap are the list, its tile offsets and the cap of that call, gran
- * its granularity.  Quantized radius: rcode_words (as hqmq_quantize_radius
+ * its granularity.  In chunk mode a listed chunk's code must have radius 0
+ * (radius code 0), as every encoder of this library writes an outlier; the
+ * list values then stand for the whole chunk.  Quantized radius: rcode_words (as hqmq_quantize_radius
  * writes them) and thr (fp32 [Hk], their range) replace radius, which may then
  * be NULL; K and V must then both be given this way. */
 typedef struct {

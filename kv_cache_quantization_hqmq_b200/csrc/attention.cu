@@ -440,6 +440,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
     const uint32_t tabk = RK > 0 ? (nw + 1) * RK : 0u, tabv = RV > 0 ? (nw + 1) * RV : 0u;
     float4 *s_tk = s_dyn, *s_tv = s_dyn + tabk;
     WarpList<LC> &WL = reinterpret_cast<WarpList<LC> *>(s_dyn + tabk + tabv)[warp];
+    // chunk-mode lists: the CTA's query rows in shared memory, bf16 [ATT_G][ATT_D]
+    // (rows >= G zero), for the K list's score corrections
+    uint16_t *s_q = reinterpret_cast<uint16_t *>(
+        reinterpret_cast<WarpList<LC> *>(s_dyn + tabk + tabv) + ATT_WARPS);
     const int head = blockIdx.x / a.cph, cta = blockIdx.x % a.cph;
     const int bb = head / a.Hk, hk = head % a.Hk;
     const float4 *cbk = a.k.cb + (size_t)hk * a.S, *cbv = a.v.cb + (size_t)hk * a.S;
@@ -499,6 +503,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     uint32_t kt0 = 0, kt1 = 0, kt2 = 0, kt3 = 0, vt0 = 0, vt1 = 0, vt2 = 0, vt3 = 0;
+    if constexpr (LM == LM_CHUNK) {
+        if (threadIdx.x < ATT_G * ATT_D / 8) {                 // 16 bytes per thread
+            const int row = threadIdx.x / (ATT_D / 8), c8 = threadIdx.x % (ATT_D / 8);
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (row < a.G)
+                v = __ldg(reinterpret_cast<const uint4 *>(
+                              a.q + (((size_t)bb * a.Hk + hk) * a.G + row) * ATT_D) + c8);
+            reinterpret_cast<uint4 *>(s_q)[threadIdx.x] = v;
+        }
+    }
     __syncthreads();                                           // tables ready
 
     LanePtrs P;
@@ -553,9 +567,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
         }
         const uint32_t u0 = (uint32_t)((slab_g0 + (uint64_t)t0) * 32);   // the block's first chunk
         bool kany = false, vany = false;
+        uint32_t kbs = 0, kbe = 0;                             // LM_CHUNK: the block's K entries
         ListView LK{false, 0u}, LV{false, 0u};
         if constexpr (LM == LM_CHUNK) {
-            if (klist) kany = map_block<LC>(a.k, WL.idx[par][0], kt0, kt1, u0, WL.map(0), lane);
+            if (klist && kt1 > kt0) {
+                // the block's K entries: tile positions [kbs, kbe) (the list is
+                // in ascending chunk order; the tile holds two blocks)
+                uint32_t lo = 0, in = 0;
+                for (uint32_t k = (uint32_t)lane; k < kt1 - kt0; k += 32) {
+                    const uint32_t ix = k < (uint32_t)LC ? WL.idx[par][0][k] : __ldg(a.k.out_idx + kt0 + k);
+                    lo += ix < u0 ? 1u : 0u;
+                    in += ix - u0 < 512u ? 1u : 0u;
+                }
+                kbs = __reduce_add_sync(FULL, lo);
+                kbe = kbs + __reduce_add_sync(FULL, in);
+            }
             if (vlist) vany = map_block<LC>(a.v, WL.idx[par][1], vt0, vt1, u0, WL.map(1), lane);
         } else if constexpr (LM == LM_ANY) {
             if (klist) LK = block_bits<LC>(a.k, WL.idx[par][0], kt0, kt1, ke ? 4 * u0 : u0, WL.bm(0), WL.pre(0), lane);
@@ -591,22 +617,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
                 kf1[ks] = pack_bf16(v[2], v[3]);
             }
             if (kany) {
+                // (chunk-mode K lists are applied as score corrections below)
                 const uint32_t tl = (uint32_t)(n + 8 * j);
-                if constexpr (LM == LM_CHUNK) {
-                    const uint2 m8 = *reinterpret_cast<const uint2 *>(WL.map(0) + tl * 32 + 8 * q);
-                    if (m8.x | m8.y) {
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t slot = ((ks < 4 ? m8.x : m8.y) >> (8 * (ks & 3))) & 0xFFu;
-                            if (!slot) continue;
-                            const uint2 e = slot != 255u ? WL.val[par][0][slot - 1]
-                                                         : entry_past_stage(a.k, kt0 + LC, kt1,
-                                                                            u0 + tl * 32 + 8 * q + ks);
-                            kf0[ks] = e.x;
-                            kf1[ks] = e.y;
-                        }
-                    }
-                } else if constexpr (LM == LM_ANY) {
+                if constexpr (LM == LM_ANY) {
                     const uint32_t lb = ke ? WL.bm(0)[tl * 4 + q] : (WL.bm(0)[tl] >> (8 * q)) & 0xFFu;
                     if (lb) {
 #pragma unroll
@@ -630,6 +643,38 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) k_attn(const AttnArgs a) {
             for (int ks = 0; ks < 8; ks += 2) {
                 mma_bf16(sc[j], aq[ks][0], 0u, aq[ks][1], 0u, kf0[ks], kf1[ks]);
                 mma_bf16(sd[j], aq[ks + 1][0], 0u, aq[ks + 1][1], 0u, kf0[ks + 1], kf1[ks + 1]);
+            }
+        }
+
+        // ---- chunk-mode K list: a listed chunk's code has radius 0, so its
+        //      decoded K^ is zero above; its values enter the scores as extra
+        //      k-steps: A = the query rows at the entries' chunks, B = each
+        //      entry's 4 values in the column of its token (4 entries per step)
+        if constexpr (LM == LM_CHUNK) {
+            for (uint32_t e0 = kbs; e0 < kbe; e0 += 4) {           // (warp-uniform)
+                const uint32_t e = e0 + (uint32_t)q;
+                uint32_t tok = 0xFFu, c = 0u;
+                uint2 v = make_uint2(0u, 0u);
+                if (e < kbe) {
+                    uint32_t ix;
+                    if (e < (uint32_t)LC) {
+                        ix = WL.idx[par][0][e];
+                        v = WL.val[par][0][e];                      // (already bf16)
+                    } else {
+                        ix = __ldg(a.k.out_idx + kt0 + e);
+                        const uint32_t *vv = reinterpret_cast<const uint32_t *>(
+                            a.k.out_val + (uint64_t)(kt0 + e) * 4);
+                        v = f16x4_to_bf16x4(make_uint2(__ldg(vv), __ldg(vv + 1)));
+                    }
+                    tok = (ix - u0) >> 5;
+                    c = (ix - u0) & 31u;
+                }
+                const uint2 qa = *reinterpret_cast<const uint2 *>(s_q + n * ATT_D + 4 * c);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const bool hit = tok == (uint32_t)(n + 8 * j);
+                    mma_bf16(sc[j], qa.x, 0u, qa.y, 0u, hit ? v.x : 0u, hit ? v.y : 0u);
+                }
             }
         }
 
@@ -830,7 +875,8 @@ inline uint64_t attn_align256(uint64_t v) { return (v + 255) & ~(uint64_t)255; }
 // Dynamic shared memory of k_attn<RK, RV, *, LM, LC> for S codewords per head.
 inline size_t attn_smem(uint32_t S, int RK, int RV, int LM, int LC) {
     const size_t tab = (size_t)(24u * S + 1u) * (RK + RV) * sizeof(float4);
-    const size_t list = LM == LM_NONE ? 0 : (size_t)ATT_WARPS * (48 * LC + 1024);
+    const size_t list = LM == LM_NONE ? 0 : (size_t)ATT_WARPS * (48 * LC + 1024) +
+                                            (LM == LM_CHUNK ? (size_t)ATT_G * ATT_D * 2 : 0);
     const size_t merge = (size_t)(2 * ATT_WARPS * ATT_G + ATT_WARPS * ATT_G * ATT_D) * sizeof(float);
     return tab + list > merge ? tab + list : merge;
 }
@@ -944,7 +990,8 @@ extern "C" int hqmq_launch_attention(const uint16_t *q, const int *seq_len, cons
     // (conflict-free lookups), 8 or 4 V-table copies, 192 staged entries
     if (b == 8 && attn_smem(S, 8, 8, LM_ANY, 192) <= opt) {
         if (lm == LM_NONE) return launch_attn<8, 8, 8, LM_NONE, 192>(a, sm_count, stream);
-        if (lm == LM_CHUNK) return launch_attn<8, 8, 8, LM_CHUNK, 192>(a, sm_count, stream);
+        if (lm == LM_CHUNK && attn_smem(S, 8, 8, LM_CHUNK, 192) <= opt)
+            return launch_attn<8, 8, 8, LM_CHUNK, 192>(a, sm_count, stream);
         return launch_attn<8, 8, 8, LM_ANY, 192>(a, sm_count, stream);
     }
     if (b == 10 && attn_smem(S, 8, 4, LM_ANY, 192) <= opt) {
@@ -952,7 +999,8 @@ extern "C" int hqmq_launch_attention(const uint16_t *q, const int *seq_len, cons
         if (lm == LM_NONE && attn_smem(S, 8, 8, LM_NONE, 192) <= opt)
             return launch_attn<8, 8, 10, LM_NONE, 192>(a, sm_count, stream);
         if (lm == LM_NONE) return launch_attn<8, 4, 10, LM_NONE, 192>(a, sm_count, stream);
-        if (lm == LM_CHUNK) return launch_attn<8, 4, 10, LM_CHUNK, 192>(a, sm_count, stream);
+        if (lm == LM_CHUNK && attn_smem(S, 8, 4, LM_CHUNK, 192) <= opt)
+            return launch_attn<8, 4, 10, LM_CHUNK, 192>(a, sm_count, stream);
         return launch_attn<8, 4, 10, LM_ANY, 192>(a, sm_count, stream);
     }
     // any other S: the most table copies that fit, 64 staged entries
