@@ -27,10 +27,14 @@
 //     terms P_hi + P_lo (about 16 significant bits).
 // The codeword table of each head lives in shared memory in R copies, lane
 // l reading copy l % R (R = 8: the 8 lanes of a 16-byte phase never share a
-// bank group).  Outlier list entries of a block are marked in a per-warp
-// bitmap and patched into the decoded chunk before it enters the mma.  The
-// warps' (max, sum, P V) partials are merged in shared memory; with several
-// CTAs per (b, hk), the last one to finish merges the CTA partials.
+// bank group).  Outlier lists: a chunk-mode K entry (its code has radius 0,
+// so its decoded chunk is zero) enters the scores through extra mma k-steps,
+// the CTA's query rows at the entry's chunk against the entry's values in
+// its token's column; V entries, and both in element mode, are marked per
+// block (slot map or bitmap) and patched into the decoded chunk before it
+// enters the mma.  The warps' (max, sum, P V) partials are merged in shared
+// memory; with several CTAs per (b, hk), the last one to finish merges the
+// CTA partials.
 #include <cuda_bf16.h>
 
 #include "med3_window.cuh"
