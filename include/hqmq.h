@@ -49,8 +49,12 @@
  * are device pointers unless stated; nothing is allocated, freed or kept
  * between calls.  Every compute entry point only enqueues work on `stream`
  * (a cudaStream_t passed as void*; NULL = the legacy default stream) and
- * returns without synchronising.  Argument errors are returned synchronously
- * and nothing is enqueued.  Data-dependent conditions (outlier capacity
+ * returns without synchronising.  Some kernels are launched with
+ * programmatic dependent launch: such a kernel may be scheduled while the
+ * previous kernel on the stream is still running, but waits for it to
+ * complete before it touches memory, so stream order holds for any
+ * predecessor; the calls can also be captured in CUDA graphs.  Argument
+ * errors are returned synchronously and nothing is enqueued.  Data-dependent conditions (outlier capacity
  * overflow, fp16 saturation, non-finite input, corrupt indices) never trap:
  * they are recorded in the device-resident hqmq_status (if non-NULL), whose
  * counters the calls add to; the caller zeroes it.
