@@ -1206,6 +1206,8 @@ def run_reference(args):
     times = []
     cpu = None
     per_step = max(3.0, 60.0 / max(1, args.steps + args.warmup))
+    if args.ref_seconds is not None:
+        per_step = args.ref_seconds
     for i in range(args.warmup + args.steps):
         cpu = cpu_baseline(w, per_step)
         if i >= args.warmup:
@@ -1242,6 +1244,9 @@ def main():
     ap.add_argument("--no-attention", action="store_true",
                     help="skip the decode-phase attention measurement on layer 0's codes")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="oracle seconds per step of --impl reference (default: about "
+                         "60 s over all steps)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
