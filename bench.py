@@ -86,28 +86,84 @@ def barrier(dist):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """SM clock and throttle-reason samples during the timed region, taken
+    every 10 ms through NVML from a thread (nvidia-smi as a fallback), on the
+    GPU that CUDA device `gpu_index` is (found by its PCI address: the CUDA
+    index and the NVML index differ when CUDA_VISIBLE_DEVICES is set)."""
 
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
-        self.gpu = gpu_index
+        import torch
+        self.gpu = str(gpu_index)
         self.proc = None
+        self.thread = None
+        self.nv = None
         self.path = "/tmp/hqmq_clocks_%d.csv" % os.getpid()
+        try:
+            pr = torch.cuda.get_device_properties(gpu_index)
+            self.gpu = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+        except Exception:
+            pass
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(self.gpu)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(int(gpu_index))
+            self.nv = pynvml
+        except Exception:
+            self.nv = None
+
+    def _loop(self):
+        nv, h = self.nv, self.h
+        bits = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+        while not self.halt.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, [n for n, b in zip(self.NAMES, bits) if r & b]))
+            except Exception:
+                pass
+            self.halt.wait(0.01)
 
     def start(self):
+        if self.nv is not None:
+            import threading
+            self.samples = []
+            self.halt = threading.Event()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+            return
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                ["nvidia-smi", "-i", self.gpu, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.halt.set()
+            self.thread.join(timeout=5)
+            self.thread = None
+            if not self.samples:
+                return None
+            try:
+                mx = float(self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            except Exception:
+                mx = 0.0
+            reasons = sorted({n for _, rs in self.samples for n in rs})
+            return {"sm_mhz": statistics.median(float(c) for c, _ in self.samples),
+                    "sm_max_mhz": mx, "reasons": reasons, "samples": len(self.samples),
+                    "source": "nvml, every 10 ms", "device": self.gpu}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -117,7 +173,6 @@ class ClockSampler:
             self.proc.kill()
         self.f.close()
         sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
@@ -127,14 +182,14 @@ class ClockSampler:
                 mx = max(mx, float(parts[2]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            for n, v in zip(self.NAMES, parts[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         os.unlink(self.path)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi", "device": self.gpu}
 
 
 # ---------------------------------------------------------------- the path
