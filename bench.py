@@ -267,34 +267,20 @@ class Cache:
             enc, dec = 1, 1
         return self.w.n_calls * (enc + dec)
 
-    def step(self, timers=None, x_override=None):
-        """One pass over the cache.  timers: dict name -> list of (start, end)
-        CUDA events recorded around the launches of that kernel family."""
+    def step(self):
+        """One pass over the cache: every (layer, role) call, on the current
+        stream."""
         import torch
         w = self.w
         stream = torch.cuda.current_stream()
         for l in range(w.layers):
             for r in range(2):
-                x = self.x[l, r] if x_override is None else x_override(l, r)
-                self.call(l, r, x, stream, timers)
+                self.call(l, r, self.x[l, r], stream)
 
-    def call(self, l, r, x, stream, timers=None):
+    def call(self, l, r, x, stream):
         """One (layer, role) call on `stream`: Med3x + encode, then decode."""
-        import torch
-
-        def ev():
-            e = torch.cuda.Event(enable_timing=True)
-            e.record(stream)
-            return e
-
-        t0 = ev() if timers is not None else None
         self.encode_call(l, r, x, stream)
-        t1 = ev() if timers is not None else None
         self.decode_call(l, r, stream)
-        if timers is not None:
-            t2 = ev()
-            timers["med3_encode" if self.w.med3 else "encode"].append((t0, t1))
-            timers["decode"].append((t1, t2))
 
     def _groups(self, l, r):
         w = self.w
@@ -467,24 +453,15 @@ def alu_ops_per_chunk(S):
     return 27 * S + 60
 
 
-def elapsed_ms(pairs):
-    return [a.elapsed_time(b) for a, b in pairs]
-
-
-def kernel_stats(w, timers, peaks, n_out, table, per_call_ms=None):
-    """Per-call time and algorithmic HBM rate of each timed call family, from
-    the event pairs in `timers` or from `per_call_ms` {family: ms}."""
+def kernel_stats(w, per_call_ms, peaks, n_out, table):
+    """Per-call time and algorithmic HBM rate of each call family timed in
+    `per_call_ms` {family: ms per call}."""
     ab = algorithmic_bytes(w, n_out, table)
     kern = {}
     for name in ("med3_encode", "encode", "decode"):
-        if per_call_ms is not None:
-            if name not in per_call_ms:
-                continue
-            t = per_call_ms[name]
-        elif not timers[name]:
+        if name not in per_call_ms:
             continue
-        else:
-            t = statistics.mean(elapsed_ms(timers[name]))
+        t = per_call_ms[name]
         gbs = ab[name] / (t * 1e-3) / 1e9
         kern[name] = {"ms_per_call": round(t, 4), "calls_per_step": w.n_calls,
                       "algorithmic_bytes_per_call": int(ab[name]),
@@ -869,8 +846,7 @@ def run_sweep(device, peaks, steps=3, warmup=3, near_ties=None):
                                "kernels); ms_per_step_python_launches: the same step "
                                "launched call by call from Python",
                      "ms_per_step_python_launches": round(ms_plain, 3),
-                     "kernels": kernel_stats(w, None, peaks, n_out, cache.table is not None,
-                                             per_call_ms=per_call),
+                     "kernels": kernel_stats(w, per_call, peaks, n_out, cache.table is not None),
                      "status_flags": st["flags"]}
         if near_ties is not None:
             near_ties[name] = oracle_parity_sample(cache, w.layers // 2, 1)
@@ -936,7 +912,7 @@ def run_hqmq(args):
     _, per_call = cache.graph_times(args.steps)
 
     n_out = st["n_outliers"] / max(1, args.warmup) / w.n_calls if w.med3 else 0.0
-    kern = kernel_stats(w, None, peaks, n_out, cache.table is not None, per_call_ms=per_call)
+    kern = kernel_stats(w, per_call, peaks, n_out, cache.table is not None)
     B, H, T, D = w.call_shape
     n_chunks = B * H * T * D // 4
     enc_key = "med3_encode" if w.med3 else "encode"

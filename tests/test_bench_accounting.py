@@ -32,8 +32,7 @@ def test_70b_call_bytes_by_hand():
 def test_hbm_fraction_from_a_call_time():
     w = W.WORKLOADS["llama3_70b_128k"]
     peaks = {"hbm_gbs": 6553.9}
-    kern = bench.kernel_stats(w, None, peaks, 901_499, True,
-                              per_call_ms={"med3_encode": 0.334, "decode": 0.0868})
+    kern = bench.kernel_stats(w, {"med3_encode": 0.334, "decode": 0.0868}, peaks, 901_499, True)
     ab = bench.algorithmic_bytes(w, 901_499, True)
     e = kern["med3_encode"]
     assert e["hbm_gbs"] == pytest.approx(ab["med3_encode"] / 0.334e-3 / 1e9, rel=1e-3)
